@@ -1,0 +1,344 @@
+"""Benchmark of the record-and-replay discrete adjoint on B200.
+
+One step = the whole hot path on the 2^20-trajectory stellar-orbit ensemble (test particles in an
+NFW halo + Miyamoto-Nagai disk, d = 6, 5 parameters per trajectory, fp64, Tsit5, rtol 1e-8,
+atol 1e-10, t in [0, 20]): the record pass (adaptive solve + record of accepted steps + record
+finalisation), the caller's loss cotangent dL/dy1 = 2 (x(20) - x*) (velocities 0), and the replay
+gradient dL/dtheta [N, 5], dL/dy0 [N, 6].  `value` = trajectories whose gradient is delivered per
+second.  Inputs are resident in HBM before the timed region; the record (~9 GB) is far larger than
+the 126 MB L2, so no L2 flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun each rank solves its own 2^20 ensemble (weak scaling, no collective on the path).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "replay-gradient trajectories/s and forward-solve traj/s at 2^20; % FP64 peak"
+UNIT = "traj/s"
+
+# Algorithmic FP64 flops per accepted step of the replay adjoint on the stellar field (add, sub,
+# mul, fma = 2, div, sqrt, log1p each counted as one operation), and per attempted step of the
+# forward solve: counted from the definitions of the Tsit5 replay step, its reverse sweep and the
+# field's f and vector-Jacobian product (tests/test_flop_counts.py re-derives these numbers).
+FLOPS_ADJOINT_STEP = {"nfw_mn": 1386}
+FLOPS_FORWARD_ATTEMPT = {"nfw_mn": 593}
+# FP64 peak: 148 SMs x 64 FP64 FMA lanes/SM/clk x 2 flop x clock (1965 MHz max) = 37.2 TFLOP/s,
+# the datasheet FP64 figure of B200; the same formula at the measured SM clock is reported too.
+SMS, FP64_LANES = 148, 64
+
+
+def fp64_peak_tflops(mhz):
+    return SMS * FP64_LANES * 2 * mhz * 1e6 / 1e12
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_reference(args):
+    """The CPU oracle as it stands, on the host cores, on a bounded sample of the same workload."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    from differentiable_adaptive_ode_b200 import workloads as W
+    from oracle import oracle as orc
+    nthreads = orc.host_threads()
+    n_sample = args.ref_sample
+    w = W.nfw_mn(N=n_sample)
+    lam = None
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        r = orc.solve(w.field, w.method, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol,
+                      keep_record=True, nthreads=nthreads)
+        lam = W.loss_cotangent(w, r["y1"], w.target)
+        orc.replay_grad(w.field, w.method, w.theta, w.y0, r["H"], r["S"], lam, nthreads=nthreads)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    t = statistics.median(times)
+    v = n_sample / t
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": "nfw_mn stellar orbits, N=2^20 (sampled), d=6, m=5, fp64, "
+                                   "Tsit5 rtol=1e-8 atol=1e-10, t=[0,20]",
+                       "global_batch": 1 << 20, "sample": n_sample},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                             "sample": "%d trajectories of the 2^20 ensemble per step: record "
+                                       "solve + replay gradient" % n_sample},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline_sample(seconds_target=15.0):
+    """Oracle throughput (record + replay gradient) on a bounded sample, all host threads."""
+    from differentiable_adaptive_ode_b200 import workloads as W
+    from oracle import oracle as orc
+    nthreads = orc.host_threads()
+    n = 256
+    while True:
+        w = W.nfw_mn(N=n)
+        t0 = time.perf_counter()
+        r = orc.solve(w.field, w.method, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol,
+                      keep_record=True, nthreads=nthreads)
+        lam = W.loss_cotangent(w, r["y1"], w.target)
+        orc.replay_grad(w.field, w.method, w.theta, w.y0, r["H"], r["S"], lam, nthreads=nthreads)
+        dt = time.perf_counter() - t0
+        if dt > seconds_target / 4 or n >= 1 << 16:
+            return {"value": n / dt, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                    "sample": "%d trajectories of the 2^20 stellar ensemble (record solve + "
+                              "replay gradient), %.1f s" % (n, dt)}
+        n *= 2
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--N", type=int, default=1 << 20)
+    ap.add_argument("--ref-sample", type=int, default=1024)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    args.warmup = max(3, args.warmup)
+
+    import torch
+    from differentiable_adaptive_ode_b200 import gradsolve as G
+    from differentiable_adaptive_ode_b200 import workloads as W
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+
+    N = args.N
+    w = W.nfw_mn(N=N, seed=4 + 1000 * rank)
+    dt = torch.float64
+    th = torch.as_tensor(w.theta, dtype=dt, device=dev)
+    y0 = torch.as_tensor(w.y0, dtype=dt, device=dev)
+    target = torch.as_tensor(w.target, dtype=dt, device=dev)
+    mask = torch.as_tensor(w.loss_mask, dtype=dt, device=dev)
+    y1 = torch.empty((N, 6), dtype=dt, device=dev)
+    lam = torch.empty((N, 6), dtype=dt, device=dev)
+    gt = torch.empty((N, 5), dtype=dt, device=dev)
+    gy = torch.empty((N, 6), dtype=dt, device=dev)
+    sys_ = G.system("nfw_mn", "tsit5", "f64")
+    rec = G.Record()
+
+    def step():
+        G.gs_solve_record(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, rec=rec)
+        torch.mul(torch.sub(y1, target), mask, out=lam).mul_(2.0)     # caller's loss cotangent
+        G.gs_replay_grad(rec, th, lam, gt, gy)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if ws > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    # ---- timed: whole steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    adj_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    barrier()
+    with ClockSampler(dev.index) as clk:
+        start = torch.cuda.Event(enable_timing=True)
+        stop = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            G.gs_solve_record(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, rec=rec)
+            torch.mul(torch.sub(y1, target), mask, out=lam).mul_(2.0)
+            adj_ev[i][0].record(stream)
+            G.gs_replay_grad(rec, th, lam, gt, gy)
+            adj_ev[i][1].record(stream)
+            ev[i][1].record(stream)
+        stop.record(stream)
+        barrier()
+    total_ms = start.elapsed_time(stop)
+    if ws > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    value = ws * N * args.steps / (total_ms / 1e3)
+    adj_ms = statistics.median(a.elapsed_time(b) for a, b in adj_ev)
+    info = rec.info()
+    total_steps = int(info.total_steps)
+
+    # ---- breakdown (not part of `value`): forward-only solve, record alone, replay alone
+    def timeit(fn, reps=max(3, args.steps // 2)):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    S = torch.empty(N, dtype=torch.int32, device=dev)
+    rj = torch.empty(N, dtype=torch.int32, device=dev)
+    stt = torch.empty(N, dtype=torch.int32, device=dev)
+    fwd_ms = timeit(lambda: G.gs_solve_forward(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, S,
+                                               rj, stt))
+    attempts = int(S.sum().item() + rj.sum().item())
+    rec_ms = timeit(lambda: G.gs_solve_record(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1,
+                                              rec=rec))
+    grad_ms = timeit(lambda: G.gs_replay_grad(rec, th, lam, gt, gy))
+
+    # ---- end to end through the public API with host buffers (pinned), copies inside the region
+    h_th = torch.as_tensor(w.theta, dtype=dt).pin_memory()
+    h_y0 = torch.as_tensor(w.y0, dtype=dt).pin_memory()
+    h_gt = torch.empty((N, 5), dtype=dt).pin_memory()
+    h_gy = torch.empty((N, 6), dtype=dt).pin_memory()
+    e2e_steps = max(3, args.steps // 2)
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        th.copy_(h_th, non_blocking=True)
+        y0.copy_(h_y0, non_blocking=True)
+        step()
+        h_gt.copy_(gt, non_blocking=True)
+        h_gy.copy_(gy, non_blocking=True)
+    b.record(stream)
+    barrier()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    if ws > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = (h_th.numel() + h_y0.numel()) * 8
+    d2h = (h_gt.numel() + h_gy.numel()) * 8
+
+    clocks = clk.summary()
+    peak_max = fp64_peak_tflops(1965.0)
+    flops_adj = total_steps * FLOPS_ADJOINT_STEP["nfw_mn"]
+    achieved = flops_adj / (adj_ms / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "nfw_mn stellar orbits: NFW halo + Miyamoto-Nagai disk, N=2^20 "
+                               "per GPU, d=6, m=5 per trajectory, fp64, Tsit5 rtol=1e-8 atol=1e-10, "
+                               "t=[0,20]; step = record + loss cotangent + replay gradient",
+                   "global_batch": ws * N, "parallelism": "independent trajectories, %d rank(s)" % ws,
+                   "l2": "inputs larger than L2 (record %.1f GB)" % (info.pool_bytes / 1e9),
+                   "accepted_steps": total_steps, "attempts_forward": attempts},
+        "roofline": {"kernel": "k_adjoint<NfwMiyamotoNagai, double, Tsit5>", "bound": "alu",
+                     "achieved": achieved, "peak": peak_max, "unit": "TFLOP/s",
+                     "frac": achieved / peak_max, "traffic": None,
+                     "peak_source": "derived: 148 SM x 64 FP64 FMA/clk x 2 x 1965 MHz",
+                     "flops_per_step": FLOPS_ADJOINT_STEP["nfw_mn"],
+                     "frac_at_measured_clock": (achieved / fp64_peak_tflops(clocks["sm_mhz"])
+                                                if clocks.get("sm_mhz") else None),
+                     "kernel_ms": adj_ms},
+        "breakdown_ms": {"forward_only": fwd_ms, "record": rec_ms, "replay_grad": grad_ms,
+                         "step": ms_step},
+        "forward_traj_per_s": ws * N / (fwd_ms / 1e3),
+        "replay_grad_traj_per_s": ws * N / (grad_ms / 1e3),
+        "record_traj_per_s": ws * N / (rec_ms / 1e3),
+        "forward_fp64_frac": (attempts * FLOPS_FORWARD_ATTEMPT["nfw_mn"] / (fwd_ms / 1e3) / 1e12)
+        / peak_max,
+        "e2e": {"value": ws * N / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * 11,
+        "clocks": clocks,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_sample()
+    else:
+        line["cpu_baseline"] = None
+    rec.close()
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

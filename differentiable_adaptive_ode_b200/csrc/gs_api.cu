@@ -1,0 +1,733 @@
+// gs_api.cu -- the C ABI declared in include/gradsolve_b200.h: argument checks, record lifecycle,
+// kernel launches.  Every entry point returns a status; nothing here aborts.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <atomic>
+#include <mutex>
+#include <new>
+#include <string>
+#include <unordered_map>
+
+#include "gradsolve_b200.h"
+#include "gs_kernels.cuh"
+
+namespace {
+
+thread_local std::string g_err;
+
+gs_status fail(gs_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+gs_status fail(gs_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+#define GS_CUDA(call)                                                                    \
+  do {                                                                                   \
+    cudaError_t e_ = (call);                                                             \
+    if (e_ != cudaSuccess)                                                               \
+      return fail(GS_ERR_CUDA, "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_),   \
+                  __FILE__, __LINE__);                                                   \
+  } while (0)
+
+struct FieldInfo {
+  int d, m;
+  bool tsit5, ros;
+};
+
+bool field_info(int field, FieldInfo* fi) {
+  switch (field) {
+    case GS_LOTKA_VOLTERRA: *fi = {2, 4, true, false}; return true;
+    case GS_LORENZ63: *fi = {3, 3, true, false}; return true;
+    case GS_MLP_4_32_32_4: *fi = {4, 1348, false, false}; return true;  // not built yet
+    case GS_ROBERTSON: *fi = {3, 3, false, true}; return true;
+    case GS_NFW_MN: *fi = {6, 5, true, false}; return true;
+    case GS_LINEAR: *fi = {3, 9, true, true}; return true;
+    default: return false;
+  }
+}
+
+gs_status check_system(const gs_system* sys) {
+  if (!sys) return fail(GS_ERR_INVALID_ARG, "gs_system pointer is NULL");
+  FieldInfo fi;
+  if (!field_info(sys->field, &fi)) return fail(GS_ERR_INVALID_ARG, "unknown field %d", sys->field);
+  if (sys->dtype != GS_F64 && sys->dtype != GS_F32)
+    return fail(GS_ERR_INVALID_ARG, "unknown dtype %d", sys->dtype);
+  if (sys->method != GS_TSIT5 && sys->method != GS_ROS34PW2)
+    return fail(GS_ERR_INVALID_ARG, "unknown method %d", sys->method);
+  if (sys->d != fi.d || sys->m != fi.m)
+    return fail(GS_ERR_INVALID_ARG, "field %d has d=%d m=%d, got d=%d m=%d", sys->field, fi.d,
+                fi.m, sys->d, sys->m);
+  if ((sys->method == GS_TSIT5 && !fi.tsit5) || (sys->method == GS_ROS34PW2 && !fi.ros))
+    return fail(GS_ERR_UNSUPPORTED, "field %d is not built for method %d", sys->field, sys->method);
+  if (sys->theta_shared != 0 && sys->theta_shared != 1)
+    return fail(GS_ERR_INVALID_ARG, "theta_shared must be 0 or 1");
+  return GS_OK;
+}
+
+// Per-device library state, created on first use and kept until exit: the SM count, a ring of
+// work-queue counters (each call takes its own slot, zeroes it on its stream and hands it to its
+// kernel, so calls on different streams never share a counter), and cached occupancy figures.
+struct DeviceCtx {
+  std::once_flag once;
+  cudaError_t init_err = cudaSuccess;
+  int sms = 148;
+  int* ring = nullptr;
+  std::atomic<unsigned> next{0};
+  std::mutex occ_mu;
+  std::unordered_map<const void*, int> occ;
+};
+constexpr int MAX_DEVICES = 64;
+constexpr unsigned RING = 4096;
+DeviceCtx g_dev[MAX_DEVICES];
+
+DeviceCtx* device_ctx(cudaError_t* err) {
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return nullptr;
+  if (dev < 0 || dev >= MAX_DEVICES) {
+    *err = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  DeviceCtx& c = g_dev[dev];
+  std::call_once(c.once, [&]() {
+    c.init_err = cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (c.init_err == cudaSuccess) c.init_err = cudaMalloc(&c.ring, RING * sizeof(int));
+  });
+  *err = c.init_err;
+  return c.init_err == cudaSuccess ? &c : nullptr;
+}
+
+// A zeroed work counter for one launch on stream s.
+cudaError_t take_counter(cudaStream_t s, int** out) {
+  cudaError_t e;
+  DeviceCtx* c = device_ctx(&e);
+  if (!c) return e;
+  int* p = c->ring + (c->next.fetch_add(1) % RING);
+  *out = p;
+  return cudaMemsetAsync(p, 0, sizeof(int), s);
+}
+
+constexpr int BLOCK = 128;
+
+template <class K>
+int persistent_grid(K kernel, size_t smem, long long N) {
+  cudaError_t e;
+  DeviceCtx* c = device_ctx(&e);
+  const int sms = c ? c->sms : 148;
+  int nb = 0;
+  const void* key = reinterpret_cast<const void*>(kernel);
+  if (c) {
+    std::lock_guard<std::mutex> lk(c->occ_mu);
+    auto it = c->occ.find(key);
+    if (it != c->occ.end()) nb = it->second;
+  }
+  if (nb == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, BLOCK, smem) != cudaSuccess ||
+        nb < 1)
+      nb = 1;
+    if (c) {
+      std::lock_guard<std::mutex> lk(c->occ_mu);
+      c->occ[key] = nb;
+    }
+  }
+  const long long g = (long long)sms * nb;
+  const long long need = (N + BLOCK - 1) / BLOCK;
+  return (int)std::max(1LL, std::min(g, need));
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------------------------------------
+// Record object.
+// ------------------------------------------------------------------------------------------------
+struct gs_record {
+  gs_system sys{};
+  int64_t N = 0;
+  int device = 0;
+  int C = 0, E = 0;
+  size_t rsz = 0;
+  double t0 = 0, t1 = 0;
+  // step pool
+  void* pool = nullptr;
+  int64_t pool_chunks = 0;
+  int* chunk_traj = nullptr;
+  int* chunk_seq = nullptr;
+  int* chunk_table = nullptr;
+  int64_t chunk_arrays_cap = 0;
+  // per trajectory
+  int64_t n_cap = 0;
+  int* nsteps = nullptr;
+  int* status = nullptr;
+  long long* offsets = nullptr;
+  long long* choff = nullptr;
+  long long* tiles = nullptr;  // scan scratch (tile totals) + grand totals
+  int* counters = nullptr;     // [0] queue [1] chunk count [2] overflow [3] max S [4] max status
+  int* host = nullptr;         // pinned mirror of counters, then offsets[N] at host+8
+  // scratch of the replay calls (grown on demand; calls on one record are stream-ordered)
+  void* red_scratch = nullptr;   // per-trajectory theta-bar [N][m] for a shared theta
+  void* red_partials = nullptr;  // block partials of the reduction
+  size_t red_bytes = 0, part_bytes = 0;
+  void* y1_scratch = nullptr;    // y_S of gs_replay_forward when the caller passes no y1
+  size_t y1_bytes = 0;
+  // summary
+  int64_t nchunks = 0, total_steps = 0;
+  int max_steps = 0;
+};
+
+namespace {
+
+void free_ptr(void* p) {
+  if (p) cudaFree(p);
+}
+
+gs_status ensure_traj_arrays(gs_record* r, int64_t N) {
+  if (r->n_cap >= N && r->counters) return GS_OK;
+  free_ptr(r->nsteps); free_ptr(r->status); free_ptr(r->offsets); free_ptr(r->choff);
+  free_ptr(r->tiles);
+  r->nsteps = r->status = nullptr;
+  r->offsets = r->choff = r->tiles = nullptr;
+  const int64_t n = std::max<int64_t>(N, 1);
+  const int64_t ntiles = (n + gs::SCAN_BLOCK - 1) / gs::SCAN_BLOCK;
+  GS_CUDA(cudaMalloc(&r->nsteps, n * sizeof(int)));
+  GS_CUDA(cudaMalloc(&r->status, n * sizeof(int)));
+  GS_CUDA(cudaMalloc(&r->offsets, (n + 1) * sizeof(long long)));
+  GS_CUDA(cudaMalloc(&r->choff, (n + 1) * sizeof(long long)));
+  GS_CUDA(cudaMalloc(&r->tiles, (ntiles + 2) * sizeof(long long)));
+  if (!r->counters) GS_CUDA(cudaMalloc(&r->counters, 16 * sizeof(int)));
+  if (!r->host) GS_CUDA(cudaMallocHost(&r->host, 16 * sizeof(int)));
+  r->n_cap = n;
+  return GS_OK;
+}
+
+gs_status ensure_pool(gs_record* r, int64_t chunks) {
+  if (chunks > 0x7fffffffLL)
+    return fail(GS_ERR_CAPACITY, "record needs %lld chunks, more than 2^31-1", (long long)chunks);
+  if (r->pool_chunks >= chunks && r->chunk_arrays_cap >= chunks) return GS_OK;
+  free_ptr(r->pool); free_ptr(r->chunk_traj); free_ptr(r->chunk_seq); free_ptr(r->chunk_table);
+  r->pool = nullptr;
+  r->chunk_traj = r->chunk_seq = r->chunk_table = nullptr;
+  r->pool_chunks = r->chunk_arrays_cap = 0;
+  const int64_t c = std::max<int64_t>(chunks, 1);
+  GS_CUDA(cudaMalloc(&r->pool, (size_t)c * r->C * r->E * r->rsz));
+  GS_CUDA(cudaMalloc(&r->chunk_traj, c * sizeof(int)));
+  GS_CUDA(cudaMalloc(&r->chunk_seq, c * sizeof(int)));
+  GS_CUDA(cudaMalloc(&r->chunk_table, c * sizeof(int)));
+  r->pool_chunks = r->chunk_arrays_cap = c;
+  return GS_OK;
+}
+
+// exclusive scan of nsteps (MODE 0) or chunk counts (MODE 1) into out[0..N]
+template <int MODE>
+gs_status scan_counts(const int* S, int N, int C, long long* out, long long* tiles,
+                      cudaStream_t st) {
+  const int ntiles = (N + gs::SCAN_BLOCK - 1) / gs::SCAN_BLOCK;
+  gs::k_scan_tiles<MODE><<<ntiles, gs::SCAN_BLOCK, 0, st>>>(S, N, C, out, tiles);
+  gs::k_scan_totals<<<1, gs::SCAN_BLOCK, 0, st>>>(tiles, ntiles, tiles + ntiles);
+  gs::k_scan_add<<<(N + 255) / 256, 256, 0, st>>>(out, N, tiles, tiles + ntiles);
+  GS_CUDA(cudaGetLastError());
+  return GS_OK;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Typed launchers.
+// ------------------------------------------------------------------------------------------------
+struct SolveCall {
+  int64_t N;
+  const void* theta;
+  int theta_shared;
+  const void* y0;
+  double t0, t1, rtol, atol;
+  long long max_attempts;
+  void* y1;
+  int* nsteps;
+  int* nrejected;
+  int* status;
+  int* queue;
+  gs_record* rec;  // non-null: record pass
+  cudaStream_t stream;
+};
+
+template <class F, class R, int METHOD>
+gs_status launch_solve(const SolveCall& c) {
+  gs::SolveParams<R> p{};
+  p.N = (int)c.N;
+  p.theta = static_cast<const R*>(c.theta);
+  p.theta_stride = c.theta_shared ? 0 : F::M;
+  p.y0 = static_cast<const R*>(c.y0);
+  p.t0 = R(c.t0); p.t1 = R(c.t1); p.rtol = R(c.rtol); p.atol = R(c.atol);
+  p.max_attempts = c.max_attempts;
+  p.y1 = static_cast<R*>(c.y1);
+  p.nsteps = c.nsteps;
+  p.nrejected = c.nrejected;
+  p.status = c.status;
+  p.queue = c.queue;
+  if (c.rec) {
+    using L = gs::RecLayout<F, R>;
+    p.pool = static_cast<R*>(c.rec->pool);
+    p.chunk_traj = c.rec->chunk_traj;
+    p.chunk_seq = c.rec->chunk_seq;
+    p.pool_chunks = (int)c.rec->pool_chunks;
+    p.chunk_count = c.rec->counters + 1;
+    p.overflow = c.rec->counters + 2;
+    const size_t smem = (size_t)(BLOCK / 32) * 32 * L::STAGE_STRIDE * sizeof(R);
+    auto kern = gs::k_solve<F, R, METHOD, true>;
+    GS_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    const int grid = persistent_grid(kern, smem, c.N);
+    kern<<<grid, BLOCK, smem, c.stream>>>(p);
+  } else {
+    auto kern = gs::k_solve<F, R, METHOD, false>;
+    const int grid = persistent_grid(kern, 0, c.N);
+    kern<<<grid, BLOCK, 0, c.stream>>>(p);
+  }
+  GS_CUDA(cudaGetLastError());
+  return GS_OK;
+}
+
+struct AdjCall {
+  const gs_record* rec;
+  const void* theta;
+  const void* dL_dy1;
+  void* dL_dy0;
+  void* dL_dtheta_traj;  // [N][M] (may be scratch)
+  int* queue;
+  cudaStream_t stream;
+};
+
+template <class F, class R, int METHOD>
+gs_status launch_adjoint(const AdjCall& c) {
+  gs::AdjointParams<R> p{};
+  const gs_record* r = c.rec;
+  p.N = (int)r->N;
+  p.theta = static_cast<const R*>(c.theta);
+  p.theta_stride = r->sys.theta_shared ? 0 : F::M;
+  p.dL_dy1 = static_cast<const R*>(c.dL_dy1);
+  p.dL_dy0 = static_cast<R*>(c.dL_dy0);
+  p.dL_dtheta = static_cast<R*>(c.dL_dtheta_traj);
+  p.nsteps = r->nsteps;
+  p.choff = r->choff;
+  p.chunk_table = r->chunk_table;
+  p.pool = static_cast<const R*>(r->pool);
+  p.queue = c.queue;
+  auto kern = gs::k_adjoint<F, R, METHOD>;
+  const int grid = persistent_grid(kern, 0, r->N);
+  kern<<<grid, BLOCK, 0, c.stream>>>(p);
+  GS_CUDA(cudaGetLastError());
+  return GS_OK;
+}
+
+template <class F, class R>
+void layout_of(int* C, int* E) {
+  *C = gs::RecLayout<F, R>::C;
+  *E = gs::RecLayout<F, R>::E;
+}
+
+// Dispatch over (field, method, dtype) for the combinations that are built.
+template <class Fn>
+gs_status dispatch(const gs_system& s, Fn&& fn) {
+  const bool f64 = s.dtype == GS_F64;
+  using namespace gs;
+  if (s.method == GS_TSIT5) {
+    switch (s.field) {
+      case GS_LOTKA_VOLTERRA:
+        return f64 ? fn.template operator()<FLotkaVolterra, double, M_TSIT5>()
+                   : fn.template operator()<FLotkaVolterra, float, M_TSIT5>();
+      case GS_LORENZ63:
+        return f64 ? fn.template operator()<FLorenz63, double, M_TSIT5>()
+                   : fn.template operator()<FLorenz63, float, M_TSIT5>();
+      case GS_NFW_MN:
+        return f64 ? fn.template operator()<FNfwMiyamotoNagai, double, M_TSIT5>()
+                   : fn.template operator()<FNfwMiyamotoNagai, float, M_TSIT5>();
+      case GS_LINEAR:
+        return f64 ? fn.template operator()<FLinear3, double, M_TSIT5>()
+                   : fn.template operator()<FLinear3, float, M_TSIT5>();
+      default: break;
+    }
+  } else {
+    switch (s.field) {
+      case GS_ROBERTSON:
+        return f64 ? fn.template operator()<FRobertson, double, M_ROS>()
+                   : fn.template operator()<FRobertson, float, M_ROS>();
+      case GS_LINEAR:
+        return f64 ? fn.template operator()<FLinear3, double, M_ROS>()
+                   : fn.template operator()<FLinear3, float, M_ROS>();
+      default: break;
+    }
+  }
+  return fail(GS_ERR_UNSUPPORTED, "field %d / method %d is not built", s.field, s.method);
+}
+
+gs_status check_common(const gs_system* sys, int64_t N, const void* theta, const void* y0,
+                       double t0, double t1, double rtol, double atol, const void* y1) {
+  gs_status st = check_system(sys);
+  if (st != GS_OK) return st;
+  if (N < 0 || N > 0x7fffffffLL) return fail(GS_ERR_INVALID_ARG, "N=%lld out of range", (long long)N);
+  if (N > 0 && (!theta || !y0 || !y1))
+    return fail(GS_ERR_INVALID_ARG, "theta, y0 and y1 must be non-NULL");
+  if (!(rtol > 0) || !(atol > 0)) return fail(GS_ERR_INVALID_ARG, "rtol and atol must be > 0");
+  if (!std::isfinite(t0) || !std::isfinite(t1))
+    return fail(GS_ERR_INVALID_ARG, "t0 and t1 must be finite");
+  return GS_OK;
+}
+
+long long attempts_of(const gs_options* opt) {
+  return (opt && opt->max_attempts > 0) ? (long long)opt->max_attempts : 100000LL;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gs_last_error(void) { return g_err.c_str(); }
+
+const char* gs_version(void) { return "gradsolve_b200 0.1 (sm_100a)"; }
+
+gs_status gs_solve_forward(const gs_system* sys, const gs_options* opt, int64_t N,
+                           const void* theta, const void* y0, double t0, double t1, double rtol,
+                           double atol, void* y1, int32_t* nsteps, int32_t* nrejected,
+                           int32_t* status, void* stream) {
+  gs_status st = check_common(sys, N, theta, y0, t0, t1, rtol, atol, y1);
+  if (st != GS_OK) return st;
+  if (N == 0) return GS_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* queue = nullptr;
+  GS_CUDA(take_counter(s, &queue));
+  SolveCall c{N, theta, sys->theta_shared, y0, t0, t1, rtol, atol, attempts_of(opt), y1,
+              nsteps, nrejected, status, queue, nullptr, s};
+  return dispatch(*sys, [&]<class F, class R, int METHOD>() { return launch_solve<F, R, METHOD>(c); });
+}
+
+gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N,
+                          const void* theta, const void* y0, double t0, double t1, double rtol,
+                          double atol, gs_record** rec, void* y1, int32_t* status, void* stream) {
+  gs_status st = check_common(sys, N, theta, y0, t0, t1, rtol, atol, y1);
+  if (st != GS_OK) return st;
+  if (!rec) return fail(GS_ERR_INVALID_ARG, "rec must be non-NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  gs_record* r = *rec;
+  bool fresh = false;
+  if (!r) {
+    r = new (std::nothrow) gs_record();
+    if (!r) return fail(GS_ERR_CAPACITY, "out of host memory");
+    fresh = true;
+  }
+  auto bail = [&](gs_status e) {
+    if (fresh) gs_record_destroy(r);
+    return e;
+  };
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return bail(fail(GS_ERR_CUDA, "cudaGetDevice failed"));
+  if (!fresh && r->device != dev)
+    return bail(fail(GS_ERR_INVALID_ARG, "record belongs to device %d, current is %d", r->device, dev));
+  r->device = dev;
+  // layout of this system
+  int C = 0, E = 0;
+  st = dispatch(*sys, [&]<class F, class R, int METHOD>() {
+    layout_of<F, R>(&C, &E);
+    return GS_OK;
+  });
+  if (st != GS_OK) return bail(st);
+  const size_t rsz = sys->dtype == GS_F64 ? 8 : 4;
+  if (!fresh && (r->C != C || r->E != E || r->rsz != rsz)) {
+    // a different layout: drop the old pool
+    free_ptr(r->pool); free_ptr(r->chunk_traj); free_ptr(r->chunk_seq); free_ptr(r->chunk_table);
+    r->pool = nullptr; r->chunk_traj = r->chunk_seq = r->chunk_table = nullptr;
+    r->pool_chunks = r->chunk_arrays_cap = 0;
+  }
+  r->sys = *sys;
+  r->N = N;
+  r->C = C;
+  r->E = E;
+  r->rsz = rsz;
+  r->t0 = t0;
+  r->t1 = t1;
+  if ((st = ensure_traj_arrays(r, N)) != GS_OK) return bail(st);
+  int64_t want_chunks = r->pool_chunks;
+  if (want_chunks == 0) {
+    const int64_t steps = (opt && opt->record_capacity_steps > 0) ? opt->record_capacity_steps
+                                                                   : std::max<int64_t>(N, 1) * 64;
+    want_chunks = (steps + C - 1) / C + std::max<int64_t>(N, 1);
+  }
+  if ((st = ensure_pool(r, want_chunks)) != GS_OK) return bail(st);
+  if (N == 0) {
+    r->nchunks = r->total_steps = 0;
+    r->max_steps = 0;
+    return GS_OK;
+  }
+  int32_t* status_out = status ? status : r->status;
+  for (int pass = 0; pass < 2; ++pass) {
+    if (cudaMemsetAsync(r->counters, 0, 16 * sizeof(int), s) != cudaSuccess)
+      return bail(fail(GS_ERR_CUDA, "cudaMemsetAsync failed"));
+    SolveCall c{N, theta, sys->theta_shared, y0, t0, t1, rtol, atol, attempts_of(opt), y1,
+                r->nsteps, nullptr, status_out, r->counters, r, s};
+    st = dispatch(*sys, [&]<class F, class R, int METHOD>() { return launch_solve<F, R, METHOD>(c); });
+    if (st != GS_OK) return bail(st);
+    if (status_out != r->status &&
+        cudaMemcpyAsync(r->status, status_out, N * sizeof(int), cudaMemcpyDeviceToDevice, s) !=
+            cudaSuccess)
+      return bail(fail(GS_ERR_CUDA, "status copy failed"));
+    const int nb = (int)((N + 255) / 256);
+    gs::k_max_int<<<nb, 256, 0, s>>>(r->nsteps, (int)N, r->counters + 3);
+    gs::k_max_int<<<nb, 256, 0, s>>>(r->status, (int)N, r->counters + 4);
+    if ((st = scan_counts<0>(r->nsteps, (int)N, C, r->offsets, r->tiles, s)) != GS_OK) return bail(st);
+    if (cudaMemcpyAsync(r->host, r->counters, 8 * sizeof(int), cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(r->host + 8, r->offsets + N, sizeof(long long), cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess)
+      return bail(fail(GS_ERR_CUDA, "readback failed"));
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess)
+      return bail(fail(GS_ERR_CUDA, "record solve failed: %s", cudaGetErrorString(e)));
+    const int used = r->host[1];
+    const int overflow = r->host[2];
+    if (!overflow) {
+      r->nchunks = used;
+      r->max_steps = r->host[3];
+      long long tot;
+      std::memcpy(&tot, r->host + 8, sizeof(tot));
+      r->total_steps = tot;
+      break;
+    }
+    if (pass == 1) return bail(fail(GS_ERR_CAPACITY, "record pool overflow after resize"));
+    if ((st = ensure_pool(r, (int64_t)used + (used >> 4) + 1024)) != GS_OK) return bail(st);
+  }
+  // chunk offsets and table
+  if ((st = scan_counts<1>(r->nsteps, (int)N, C, r->choff, r->tiles, s)) != GS_OK) return bail(st);
+  if (r->nchunks > 0)
+    gs::k_chunk_table<<<(int)((r->nchunks + 255) / 256), 256, 0, s>>>(
+        r->chunk_traj, r->chunk_seq, (int)r->nchunks, r->choff, r->chunk_table);
+  if (cudaGetLastError() != cudaSuccess) return bail(fail(GS_ERR_CUDA, "chunk table launch failed"));
+  *rec = r;
+  if (r->host[4] != 0) {
+    fail(GS_ERR_TRAJ_FAILED, "some trajectories did not reach t1 (max status %d)", r->host[4]);
+    return GS_ERR_TRAJ_FAILED;
+  }
+  return GS_OK;
+}
+
+gs_status gs_replay_grad(const gs_record* rec, const void* theta, const void* dL_dy1,
+                         void* dL_dtheta, void* dL_dy0, void* stream) {
+  if (!rec) return fail(GS_ERR_INVALID_ARG, "record is NULL");
+  if (rec->N == 0) return GS_OK;
+  if (!theta || !dL_dy1) return fail(GS_ERR_INVALID_ARG, "theta and dL_dy1 must be non-NULL");
+  if (!dL_dtheta && !dL_dy0) return fail(GS_ERR_INVALID_ARG, "no output requested");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int M = rec->sys.m;
+  const int64_t N = rec->N;
+  const bool shared = rec->sys.theta_shared && dL_dtheta;
+  const int per_block = 4096;
+  const int nred = (int)((N + per_block - 1) / per_block);
+  gs_record* r = const_cast<gs_record*>(rec);
+  if (shared) {
+    const size_t need = (size_t)N * M * rec->rsz, needp = (size_t)nred * M * rec->rsz;
+    if (r->red_bytes < need) {
+      free_ptr(r->red_scratch);
+      r->red_scratch = nullptr;
+      r->red_bytes = 0;
+      GS_CUDA(cudaMalloc(&r->red_scratch, need));
+      r->red_bytes = need;
+    }
+    if (r->part_bytes < needp) {
+      free_ptr(r->red_partials);
+      r->red_partials = nullptr;
+      r->part_bytes = 0;
+      GS_CUDA(cudaMalloc(&r->red_partials, needp));
+      r->part_bytes = needp;
+    }
+  }
+  void* scratch = r->red_scratch;
+  void* partials = r->red_partials;
+  int* queue = nullptr;
+  GS_CUDA(take_counter(s, &queue));
+  AdjCall c{rec, theta, dL_dy1, dL_dy0, shared ? scratch : dL_dtheta, queue, s};
+  return dispatch(rec->sys, [&]<class F, class R, int METHOD>() {
+    gs_status rs = launch_adjoint<F, R, METHOD>(c);
+    if (rs != GS_OK || !shared) return rs;
+    gs::k_reduce_theta<R><<<nred, gs::RED_BLOCK, 0, s>>>(static_cast<const R*>(scratch), (int)N, M,
+                                                        per_block, static_cast<R*>(partials));
+    gs::k_reduce_partials<R><<<1, 256, 0, s>>>(static_cast<const R*>(partials), nred, M,
+                                               static_cast<R*>(dL_dtheta));
+    GS_CUDA(cudaGetLastError());
+    return GS_OK;
+  });
+}
+
+gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, void* y1,
+                            void* stream) {
+  if (!rec) return fail(GS_ERR_INVALID_ARG, "record is NULL");
+  if (rec->N == 0) return GS_OK;
+  if (!theta || !y0) return fail(GS_ERR_INVALID_ARG, "theta and y0 must be non-NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* y1buf = y1;
+  if (!y1buf) {
+    const size_t need = (size_t)rec->N * rec->sys.d * rec->rsz;
+    if (rec->y1_bytes < need) {
+      free_ptr(rec->y1_scratch);
+      rec->y1_scratch = nullptr;
+      rec->y1_bytes = 0;
+      GS_CUDA(cudaMalloc(&rec->y1_scratch, need));
+      rec->y1_bytes = need;
+    }
+    y1buf = rec->y1_scratch;
+  }
+  int* queue = nullptr;
+  GS_CUDA(take_counter(s, &queue));
+  gs_status st = dispatch(rec->sys, [&]<class F, class R, int METHOD>() {
+    gs::ReplayParams<R> p{};
+    p.N = (int)rec->N;
+    p.theta = static_cast<const R*>(theta);
+    p.theta_stride = rec->sys.theta_shared ? 0 : F::M;
+    p.y0 = static_cast<const R*>(y0);
+    p.y1 = static_cast<R*>(y1buf);
+    p.nsteps = rec->nsteps;
+    p.choff = rec->choff;
+    p.chunk_table = rec->chunk_table;
+    p.pool = static_cast<R*>(rec->pool);
+    p.queue = queue;
+    auto kern = gs::k_replay_forward<F, R, METHOD>;
+    const int grid = persistent_grid(kern, 0, rec->N);
+    kern<<<grid, BLOCK, 0, s>>>(p);
+    GS_CUDA(cudaGetLastError());
+    return GS_OK;
+  });
+  return st;
+}
+
+gs_status gs_record_info(const gs_record* rec, gs_record_info_t* out) {
+  if (!rec || !out) return fail(GS_ERR_INVALID_ARG, "NULL argument");
+  out->N = rec->N;
+  out->total_steps = rec->total_steps;
+  out->max_steps = rec->max_steps;
+  out->chunk_steps = rec->C;
+  out->entry_reals = rec->E;
+  out->dtype = rec->sys.dtype;
+  out->nchunks = rec->nchunks;
+  out->pool_bytes = (int64_t)rec->pool_chunks * rec->C * rec->E * (int64_t)rec->rsz;
+  out->nsteps = rec->nsteps;
+  out->status = rec->status;
+  out->offsets = reinterpret_cast<const int64_t*>(rec->offsets);
+  out->chunk_offsets = reinterpret_cast<const int64_t*>(rec->choff);
+  out->chunk_table = rec->chunk_table;
+  out->pool = rec->pool;
+  return GS_OK;
+}
+
+gs_status gs_record_export(const gs_record* rec, void* T, void* H, void* Y, int64_t* offsets,
+                           void* stream) {
+  if (!rec) return fail(GS_ERR_INVALID_ARG, "record is NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (offsets && rec->N >= 0)
+    GS_CUDA(cudaMemcpyAsync(offsets, rec->offsets, (rec->N + 1) * sizeof(long long),
+                            cudaMemcpyDeviceToDevice, s));
+  if (rec->total_steps == 0) return GS_OK;
+  const int nb = (int)((rec->total_steps + 255) / 256);
+  if (rec->sys.dtype == GS_F64)
+    gs::k_export<double><<<nb, 256, 0, s>>>(static_cast<const double*>(rec->pool), rec->chunk_table,
+                                            rec->choff, rec->offsets, (int)rec->N, rec->sys.d,
+                                            rec->C, rec->total_steps, static_cast<double*>(T),
+                                            static_cast<double*>(H), static_cast<double*>(Y));
+  else
+    gs::k_export<float><<<nb, 256, 0, s>>>(static_cast<const float*>(rec->pool), rec->chunk_table,
+                                           rec->choff, rec->offsets, (int)rec->N, rec->sys.d,
+                                           rec->C, rec->total_steps, static_cast<float*>(T),
+                                           static_cast<float*>(H), static_cast<float*>(Y));
+  GS_CUDA(cudaGetLastError());
+  return GS_OK;
+}
+
+gs_status gs_record_import(const gs_system* sys, int64_t N, const int32_t* nsteps, const void* T,
+                           const void* H, const void* Y, gs_record** rec, void* stream) {
+  gs_status st = check_system(sys);
+  if (st != GS_OK) return st;
+  if (!rec) return fail(GS_ERR_INVALID_ARG, "rec must be non-NULL");
+  if (N < 0 || N > 0x7fffffffLL) return fail(GS_ERR_INVALID_ARG, "N out of range");
+  if (N > 0 && (!nsteps || !H || !Y)) return fail(GS_ERR_INVALID_ARG, "nsteps, H, Y required");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  gs_record* r = new (std::nothrow) gs_record();
+  if (!r) return fail(GS_ERR_CAPACITY, "out of host memory");
+  auto bail = [&](gs_status e) {
+    gs_record_destroy(r);
+    return e;
+  };
+  int C = 0, E = 0;
+  st = dispatch(*sys, [&]<class F, class R, int METHOD>() {
+    layout_of<F, R>(&C, &E);
+    return GS_OK;
+  });
+  if (st != GS_OK) return bail(st);
+  cudaGetDevice(&r->device);
+  r->sys = *sys;
+  r->N = N;
+  r->C = C;
+  r->E = E;
+  r->rsz = sys->dtype == GS_F64 ? 8 : 4;
+  if ((st = ensure_traj_arrays(r, N)) != GS_OK) return bail(st);
+  if (N > 0) {
+    if (cudaMemcpyAsync(r->nsteps, nsteps, N * sizeof(int), cudaMemcpyDeviceToDevice, s) !=
+            cudaSuccess ||
+        cudaMemsetAsync(r->status, 0, N * sizeof(int), s) != cudaSuccess ||
+        cudaMemsetAsync(r->counters, 0, 16 * sizeof(int), s) != cudaSuccess)
+      return bail(fail(GS_ERR_CUDA, "import copies failed"));
+    if ((st = scan_counts<0>(r->nsteps, (int)N, C, r->offsets, r->tiles, s)) != GS_OK) return bail(st);
+    gs::k_max_int<<<(int)((N + 255) / 256), 256, 0, s>>>(r->nsteps, (int)N, r->counters + 3);
+    if ((st = scan_counts<1>(r->nsteps, (int)N, C, r->choff, r->tiles, s)) != GS_OK) return bail(st);
+    long long tot[2] = {0, 0};
+    if (cudaMemcpyAsync(&tot[0], r->offsets + N, sizeof(long long), cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(&tot[1], r->choff + N, sizeof(long long), cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(r->host, r->counters, 8 * sizeof(int), cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return bail(fail(GS_ERR_CUDA, "import readback failed"));
+    r->total_steps = tot[0];
+    r->nchunks = tot[1];
+    r->max_steps = r->host[3];
+    if ((st = ensure_pool(r, std::max<int64_t>(r->nchunks, 1))) != GS_OK) return bail(st);
+    if (r->nchunks > 0) {
+      gs::k_iota<<<(int)((r->nchunks + 255) / 256), 256, 0, s>>>(r->chunk_table, (int)r->nchunks);
+      const int nb = (int)((r->total_steps + 255) / 256);
+      if (sys->dtype == GS_F64)
+        gs::k_import<double><<<nb, 256, 0, s>>>(static_cast<double*>(r->pool), r->choff, r->offsets,
+                                                (int)N, sys->d, C, r->total_steps,
+                                                static_cast<const double*>(T),
+                                                static_cast<const double*>(H),
+                                                static_cast<const double*>(Y));
+      else
+        gs::k_import<float><<<nb, 256, 0, s>>>(static_cast<float*>(r->pool), r->choff, r->offsets,
+                                               (int)N, sys->d, C, r->total_steps,
+                                               static_cast<const float*>(T),
+                                               static_cast<const float*>(H),
+                                               static_cast<const float*>(Y));
+      if (cudaGetLastError() != cudaSuccess) return bail(fail(GS_ERR_CUDA, "import launch failed"));
+    }
+  }
+  *rec = r;
+  return GS_OK;
+}
+
+void gs_record_destroy(gs_record* r) {
+  if (!r) return;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(r->device);
+  cudaDeviceSynchronize();
+  free_ptr(r->pool); free_ptr(r->chunk_traj); free_ptr(r->chunk_seq); free_ptr(r->chunk_table);
+  free_ptr(r->nsteps); free_ptr(r->status); free_ptr(r->offsets); free_ptr(r->choff);
+  free_ptr(r->tiles); free_ptr(r->counters);
+  free_ptr(r->red_scratch); free_ptr(r->red_partials); free_ptr(r->y1_scratch);
+  if (r->host) cudaFreeHost(r->host);
+  cudaSetDevice(prev);
+  delete r;
+}
+
+}  // extern "C"

@@ -1,0 +1,245 @@
+// gs_fields.cuh -- right-hand sides f(y; theta) and their hand-written vector-Jacobian products
+// for the device kernels.  Every field is autonomous.
+//
+// Interface of a field F (R = double or float):
+//   F::D, F::M                       state size, parameter count
+//   F::Theta<R>                      per-lane parameters (registers) plus hoisted invariants
+//   F::load(Theta&, const R* src)    read M parameters, precompute what depends only on theta
+//   F::f(y, th, dy)                  dy = f(y; theta)
+//   F::vjp(y, th, kb, yb, thb)       yb = (df/dy)^T kb (overwritten), thb += (df/dtheta)^T kb
+// Stiff fields also provide
+//   F::jac(y, th, J)                 J = df/dy, row-major D x D
+//   F::jac_vjp(y, th, Jb, yb, thb)   yb += sum_rc Jb_rc dJ_rc/dy,  thb += sum_rc Jb_rc dJ_rc/dtheta
+//
+// The reverse sweep that calls vjp() is the discrete adjoint of "gradsolve: fast exact gradients
+// for ODE ensembles on GPUs" §3 (the gradient of the fixed-mesh replay) and §3.2 (the Rosenbrock
+// stage also differentiates J, i.e. second derivatives of f).
+#pragma once
+// Fields are host-callable too (and compile as plain C++) so that their arithmetic can be
+// tallied on the host with a counting scalar.
+#ifdef __CUDACC__
+#include <cuda_runtime.h>
+#define GS_HD __host__ __device__ __forceinline__
+#else
+#define GS_HD inline
+#endif
+
+namespace gs {
+
+// ----------------------------------------------------------------------------------------------
+// Lotka-Volterra, theta = (alpha, beta, gamma, delta): x' = alpha x - beta x y, y' = delta x y - gamma y
+// ----------------------------------------------------------------------------------------------
+struct FLotkaVolterra {
+  static constexpr int D = 2, M = 4;
+  template <class R> struct Theta { R a, b, g, d; };
+  template <class R> GS_HD static void load(Theta<R>& t, const R* s) {
+    t.a = s[0]; t.b = s[1]; t.g = s[2]; t.d = s[3];
+  }
+  template <class R> GS_HD static void f(const R* y, const Theta<R>& t, R* dy) {
+    const R xy = y[0] * y[1];
+    dy[0] = t.a * y[0] - t.b * xy;
+    dy[1] = t.d * xy - t.g * y[1];
+  }
+  template <class R>
+  GS_HD static void vjp(const R* y, const Theta<R>& t, const R* kb, R* yb, R* thb) {
+    yb[0] = (t.a - t.b * y[1]) * kb[0] + t.d * y[1] * kb[1];
+    yb[1] = -(t.b * y[0]) * kb[0] + (t.d * y[0] - t.g) * kb[1];
+    const R xy = y[0] * y[1];
+    thb[0] += y[0] * kb[0];
+    thb[1] -= xy * kb[0];
+    thb[2] -= y[1] * kb[1];
+    thb[3] += xy * kb[1];
+  }
+};
+
+// ----------------------------------------------------------------------------------------------
+// Lorenz-63, theta = (sigma, rho, beta)
+// ----------------------------------------------------------------------------------------------
+struct FLorenz63 {
+  static constexpr int D = 3, M = 3;
+  template <class R> struct Theta { R s, r, b; };
+  template <class R> GS_HD static void load(Theta<R>& t, const R* s) {
+    t.s = s[0]; t.r = s[1]; t.b = s[2];
+  }
+  template <class R> GS_HD static void f(const R* y, const Theta<R>& t, R* dy) {
+    dy[0] = t.s * (y[1] - y[0]);
+    dy[1] = y[0] * (t.r - y[2]) - y[1];
+    dy[2] = y[0] * y[1] - t.b * y[2];
+  }
+  template <class R>
+  GS_HD static void vjp(const R* y, const Theta<R>& t, const R* kb, R* yb, R* thb) {
+    yb[0] = -t.s * kb[0] + (t.r - y[2]) * kb[1] + y[1] * kb[2];
+    yb[1] = t.s * kb[0] - kb[1] + y[0] * kb[2];
+    yb[2] = -y[0] * kb[1] - t.b * kb[2];
+    thb[0] += (y[1] - y[0]) * kb[0];
+    thb[1] += y[0] * kb[1];
+    thb[2] -= y[2] * kb[2];
+  }
+};
+
+// ----------------------------------------------------------------------------------------------
+// Robertson kinetics (stiff), theta = (k1, k2, k3)
+//   y1' = -k1 y1 + k3 y2 y3,  y2' = k1 y1 - k2 y2^2 - k3 y2 y3,  y3' = k2 y2^2
+// ----------------------------------------------------------------------------------------------
+struct FRobertson {
+  static constexpr int D = 3, M = 3;
+  template <class R> struct Theta { R k1, k2, k3; };
+  template <class R> GS_HD static void load(Theta<R>& t, const R* s) {
+    t.k1 = s[0]; t.k2 = s[1]; t.k3 = s[2];
+  }
+  template <class R> GS_HD static void f(const R* y, const Theta<R>& t, R* dy) {
+    const R a = t.k1 * y[0], b = t.k2 * y[1] * y[1], c = t.k3 * y[1] * y[2];
+    dy[0] = -a + c;
+    dy[1] = a - b - c;
+    dy[2] = b;
+  }
+  template <class R> GS_HD static void jac(const R* y, const Theta<R>& t, R* J) {
+    J[0] = -t.k1; J[1] = t.k3 * y[2];                        J[2] = t.k3 * y[1];
+    J[3] = t.k1;  J[4] = -R(2) * t.k2 * y[1] - t.k3 * y[2];  J[5] = -t.k3 * y[1];
+    J[6] = R(0);  J[7] = R(2) * t.k2 * y[1];                 J[8] = R(0);
+  }
+  template <class R>
+  GS_HD static void vjp(const R* y, const Theta<R>& t, const R* kb, R* yb, R* thb) {
+    // yb = J^T kb
+    const R d01 = kb[1] - kb[0];     // k1 y1 leaves y1 and enters y2
+    const R d12 = kb[2] - kb[1];     // k2 y2^2 leaves y2 and enters y3
+    const R d10 = kb[0] - kb[1];     // k3 y2 y3 leaves y2 and enters y1
+    yb[0] = t.k1 * d01;
+    yb[1] = R(2) * t.k2 * y[1] * d12 + t.k3 * y[2] * d10;
+    yb[2] = t.k3 * y[1] * d10;
+    thb[0] += y[0] * d01;
+    thb[1] += y[1] * y[1] * d12;
+    thb[2] += y[1] * y[2] * d10;
+  }
+  // J depends on y only through y2, y3 and linearly: the second derivatives are constants.
+  template <class R>
+  GS_HD static void jac_vjp(const R* y, const Theta<R>& t, const R* Jb, R* yb, R* thb) {
+    // dJ12/dy3 = k3, dJ13/dy2 = k3, dJ22/dy2 = -2 k2, dJ22/dy3 = -k3, dJ23/dy2 = -k3, dJ32/dy2 = 2 k2
+    yb[1] += t.k3 * (Jb[2] - Jb[5]) + R(2) * t.k2 * (Jb[7] - Jb[4]);
+    yb[2] += t.k3 * (Jb[1] - Jb[4]);
+    // dJ/dk1: J11 = -k1, J21 = k1;  dJ/dk2: J22 = -2 k2 y2, J32 = 2 k2 y2;
+    // dJ/dk3: J12 = k3 y3, J13 = k3 y2, J22 = -k3 y3, J23 = -k3 y2
+    thb[0] += Jb[3] - Jb[0];
+    thb[1] += R(2) * y[1] * (Jb[7] - Jb[4]);
+    thb[2] += y[2] * (Jb[1] - Jb[4]) + y[1] * (Jb[2] - Jb[5]);
+  }
+};
+
+// ----------------------------------------------------------------------------------------------
+// Linear test field y' = A y, theta = A (row-major 3x3); J = A.
+// ----------------------------------------------------------------------------------------------
+struct FLinear3 {
+  static constexpr int D = 3, M = 9;
+  template <class R> struct Theta { R A[9]; };
+  template <class R> GS_HD static void load(Theta<R>& t, const R* s) {
+#pragma unroll
+    for (int i = 0; i < 9; ++i) t.A[i] = s[i];
+  }
+  template <class R> GS_HD static void f(const R* y, const Theta<R>& t, R* dy) {
+#pragma unroll
+    for (int r = 0; r < 3; ++r) dy[r] = t.A[3 * r] * y[0] + t.A[3 * r + 1] * y[1] + t.A[3 * r + 2] * y[2];
+  }
+  template <class R> GS_HD static void jac(const R*, const Theta<R>& t, R* J) {
+#pragma unroll
+    for (int i = 0; i < 9; ++i) J[i] = t.A[i];
+  }
+  template <class R>
+  GS_HD static void vjp(const R* y, const Theta<R>& t, const R* kb, R* yb, R* thb) {
+#pragma unroll
+    for (int c = 0; c < 3; ++c) yb[c] = t.A[c] * kb[0] + t.A[3 + c] * kb[1] + t.A[6 + c] * kb[2];
+#pragma unroll
+    for (int r = 0; r < 3; ++r)
+#pragma unroll
+      for (int c = 0; c < 3; ++c) thb[3 * r + c] += kb[r] * y[c];
+  }
+  template <class R>
+  GS_HD static void jac_vjp(const R*, const Theta<R>&, const R* Jb, R*, R* thb) {
+#pragma unroll
+    for (int i = 0; i < 9; ++i) thb[i] += Jb[i];
+  }
+};
+
+// ----------------------------------------------------------------------------------------------
+// Test particle in an NFW halo plus a Miyamoto-Nagai disk, G = 1.
+// State (x, y, z, vx, vy, vz); theta = (M_h, r_s, M_d, a, b).
+//   Phi = -M_h ln(1 + r/r_s)/r - M_d/D,  D^2 = R^2 + (a + B)^2,  B = sqrt(z^2 + b^2)
+//   x' = v,  v' = acc = -gN x - gM w,  w = (x, y, z q),  q = (a + B)/B,
+//   gN = M_h (L/r^3 - 1/(r^2 (r_s + r))),  L = ln(1 + r/r_s),  gM = M_d / D^3.
+// VJP (u = cotangent of v'):
+//   d acc/dx = -[gN I + (gN'/r) x x^T] - [gM diag(1, 1, q - a z^2/B^3) - 3 gM/D^2 w w^T]
+//   gN'/r = M_h [3/(r^4 (r_s + r)) - 3 L / r^5 + 1/(r^3 (r_s + r)^2)]
+//   d acc/dM_h = -(gN/M_h) x,     d acc/dr_s = M_h/(r r_s (r_s + r)^2) x,
+//   d acc/dM_d = -w/D^3,
+//   d acc/da = 3 gM (a+B)/D^2 w - gM (0, 0, z/B),
+//   d acc/db = 3 gM (a+B) b/(B D^2) w + gM (0, 0, a b z/B^3).
+// Per-lane invariants of theta (1/r_s, b^2) are hoisted into Theta.
+// ----------------------------------------------------------------------------------------------
+struct FNfwMiyamotoNagai {
+  static constexpr int D = 6, M = 5;
+  template <class R> struct Theta { R Mh, rs, Md, a, b, irs, b2; };
+  template <class R> GS_HD static void load(Theta<R>& t, const R* s) {
+    t.Mh = s[0]; t.rs = s[1]; t.Md = s[2]; t.a = s[3]; t.b = s[4];
+    t.irs = R(1) / t.rs;
+    t.b2 = t.b * t.b;
+  }
+  template <class R> GS_HD static void f(const R* y, const Theta<R>& t, R* dy) {
+    const R x = y[0], yy = y[1], z = y[2];
+    const R R2 = x * x + yy * yy;
+    const R r2 = R2 + z * z;
+    const R r = sqrt(r2);
+    const R L = log1p(r * t.irs);
+    const R ir2 = R(1) / r2;
+    const R gN = t.Mh * ir2 * (L / r - R(1) / (t.rs + r));
+    const R B = sqrt(z * z + t.b2);
+    const R apB = t.a + B;
+    const R D2 = R2 + apB * apB;
+    const R gM = t.Md / (D2 * sqrt(D2));
+    const R g = gN + gM;
+    dy[0] = y[3];
+    dy[1] = y[4];
+    dy[2] = y[5];
+    dy[3] = -g * x;
+    dy[4] = -g * yy;
+    dy[5] = -(gN + gM * apB / B) * z;
+  }
+  template <class R>
+  GS_HD static void vjp(const R* y, const Theta<R>& t, const R* kb, R* yb, R* thb) {
+    const R x = y[0], yy = y[1], z = y[2];
+    const R ux = kb[3], uy = kb[4], uz = kb[5];
+    const R R2 = x * x + yy * yy;
+    const R r2 = R2 + z * z;
+    const R r = sqrt(r2);
+    const R ir = R(1) / r;
+    const R L = log1p(r * t.irs);
+    const R ir2 = ir * ir;
+    const R isr = R(1) / (t.rs + r);
+    const R Lir = L * ir;
+    const R gN = t.Mh * ir2 * (Lir - isr);
+    const R gNp_r = t.Mh * ir2 * ir2 * (R(3) * isr - R(3) * Lir + r * isr * isr);   // gN'/r
+    const R B = sqrt(z * z + t.b2);
+    const R iB = R(1) / B;
+    const R apB = t.a + B;
+    const R q = apB * iB;
+    const R D2 = R2 + apB * apB;
+    const R iD2 = R(1) / D2;
+    const R gM = t.Md * iD2 * sqrt(iD2);
+    const R wz = z * q;
+    const R xu = x * ux + yy * uy + z * uz;
+    const R wu = x * ux + yy * uy + wz * uz;
+    const R c3 = R(3) * gM * iD2 * wu;
+    const R hz = q - t.a * z * z * iB * iB * iB;
+    yb[0] = -(gN * ux + gNp_r * xu * x) - (gM * ux - c3 * x);
+    yb[1] = -(gN * uy + gNp_r * xu * yy) - (gM * uy - c3 * yy);
+    yb[2] = -(gN * uz + gNp_r * xu * z) - (gM * hz * uz - c3 * wz);
+    yb[3] = kb[0];
+    yb[4] = kb[1];
+    yb[5] = kb[2];
+    thb[0] -= ir2 * (Lir - isr) * xu;
+    thb[1] += t.Mh * ir * t.irs * isr * isr * xu;
+    thb[2] -= iD2 * sqrt(iD2) * wu;
+    thb[3] += apB * c3 - gM * z * iB * uz;
+    thb[4] += t.b * iB * (apB * c3 + gM * t.a * z * iB * iB * uz);
+  }
+};
+
+}  // namespace gs

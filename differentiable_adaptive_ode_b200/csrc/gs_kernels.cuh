@@ -1,0 +1,622 @@
+// gs_kernels.cuh -- the ensemble kernels.
+//
+//  k_solve<F,R,Method,REC>   one trajectory per lane, state in registers; persistent grid whose
+//                            warps refill retired lanes from a global work counter (one ballot +
+//                            one atomicAdd per warp per refill).  REC = true also keeps the record:
+//                            each accepted step (t_n, h_n, y_n) is staged in shared memory and a
+//                            full chunk of C steps is written by the whole warp as one contiguous,
+//                            coalesced block of the record pool.
+//  k_adjoint<F,R,Method>     the replay-adjoint: each lane walks its trajectory's record from the
+//                            last accepted step back to the first, recomputes the stages from the
+//                            recorded y_n, and pulls lambda and theta-bar back through each step.
+//  k_scan_*, k_chunk_table   record finalisation: prefix offsets and the per-trajectory chunk table.
+//  k_reduce_theta            deterministic ensemble sum of theta-bar for a shared theta.
+//
+// Source of the method: "gradsolve: fast exact gradients for ODE ensembles on GPUs" -- §2.1
+// (adaptive loop, RMS test, reject-and-retry), §2.4 (one thread per trajectory with its state
+// in registers), §3 (record of accepted steps; replay with the mesh as data; exact reverse-mode
+// derivative of the replay), §3.3 (the adjoint keeps one accepted state per step and recomputes
+// the stages from it).
+#pragma once
+#include <cstdint>
+
+#include "gs_methods.cuh"
+
+namespace gs {
+
+constexpr unsigned FULL = 0xffffffffu;
+
+// Record chunk: C accepted steps of one trajectory, entry = (t, h, y[0..D-1]) contiguous.
+template <class F, class R>
+struct RecLayout {
+  static constexpr int E = 2 + F::D;                                     // reals per step
+  static constexpr int C = (E * int(sizeof(R)) >= 48) ? 4 : 8;           // steps per chunk
+  static constexpr int STAGE_STRIDE = C * E + 1;                         // per-lane smem stride
+};
+
+template <class R>
+struct SolveParams {
+  int N;
+  const R* theta;
+  int theta_stride;  // 0 when theta is shared by the ensemble
+  const R* y0;
+  R t0, t1, rtol, atol;
+  long long max_attempts;
+  R* y1;
+  int* nsteps;
+  int* nrejected;
+  int* status;
+  int* queue;        // work counter
+  // record (REC only)
+  R* pool;
+  int* chunk_traj;
+  int* chunk_seq;
+  int pool_chunks;   // capacity in chunks
+  int* chunk_count;  // bump allocator
+  int* overflow;     // set to 1 when the pool ran out
+};
+
+template <class R> __device__ __forceinline__ R pw(R x, R e);
+template <> __device__ __forceinline__ double pw<double>(double x, double e) { return pow(x, e); }
+template <> __device__ __forceinline__ float pw<float>(float x, float e) { return powf(x, e); }
+template <class R> __device__ __forceinline__ R eps_of();
+template <> __device__ __forceinline__ double eps_of<double>() { return 2.220446049250313e-16; }
+template <> __device__ __forceinline__ float eps_of<float>() { return 1.1920929e-07f; }
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Warp-aggregated draw from the work counter: every lane with `need` receives the next id.
+__device__ __forceinline__ int warp_take(bool need, int* counter) {
+  const unsigned m = __ballot_sync(FULL, need);
+  if (m == 0) return -1;
+  const int leader = __ffs(m) - 1;
+  const int lane = threadIdx.x & 31;
+  int base = 0;
+  if (lane == leader) base = atomicAdd(counter, __popc(m));
+  base = __shfl_sync(FULL, base, leader);
+  return need ? base + __popc(m & lanemask_lt()) : -1;
+}
+
+// Hairer-Norsett-Wanner starting step (Solving ODEs I, §II.4), RMS norm with sc = atol + rtol|y0|.
+template <class F, class R>
+__device__ R initial_step(const R (&y0)[F::D], const R (&f0)[F::D],
+                          const typename F::template Theta<R>& th, R t0, R t1, R rtol, R atol,
+                          int p) {
+  constexpr int D = F::D;
+  R s0 = R(0), s1 = R(0);
+#pragma unroll
+  for (int i = 0; i < D; ++i) {
+    const R sc = atol + rtol * fabs(y0[i]);
+    const R a = y0[i] / sc, b = f0[i] / sc;
+    s0 += a * a;
+    s1 += b * b;
+  }
+  const R d0 = sqrt(s0 / R(D)), d1 = sqrt(s1 / R(D));
+  const R h0 = (d0 < R(1e-5) || d1 < R(1e-5)) ? R(1e-6) : R(0.01) * d0 / d1;
+  R y1[D], f1[D];
+#pragma unroll
+  for (int i = 0; i < D; ++i) y1[i] = y0[i] + h0 * f0[i];
+  F::f(y1, th, f1);
+  R s2 = R(0);
+#pragma unroll
+  for (int i = 0; i < D; ++i) {
+    const R sc = atol + rtol * fabs(y0[i]);
+    const R q = (f1[i] - f0[i]) / sc;
+    s2 += q * q;
+  }
+  const R d2 = sqrt(s2 / R(D)) / h0;
+  const R dm = d1 > d2 ? d1 : d2;   // same selection as max(d1, d2) with d1 first
+  const R h1 = (dm <= R(1e-15)) ? fmax(R(1e-6), h0 * R(1e-3)) : pw<R>(R(0.01) / dm, R(1) / R(p));
+  R h = R(100) * h0;
+  h = h1 < h ? h1 : h;
+  h = (t1 - t0) < h ? (t1 - t0) : h;
+  return h;
+}
+
+template <int METHOD> struct MethodTag {};
+constexpr int M_TSIT5 = 0, M_ROS = 1;
+
+template <class F, class R, int METHOD, bool REC>
+__global__ void __launch_bounds__(128) k_solve(SolveParams<R> p) {
+  using L = RecLayout<F, R>;
+  constexpr int D = F::D;
+  constexpr int order = METHOD == M_TSIT5 ? Tsit5::order : Ros34pw2::order;
+  constexpr int qerr = METHOD == M_TSIT5 ? Tsit5::err_order : Ros34pw2::err_order;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  R* stage = nullptr;
+  const int lane = threadIdx.x & 31;
+  if (REC) {
+    const int warp = threadIdx.x >> 5;
+    stage = reinterpret_cast<R*>(smem_raw) + (size_t)warp * 32 * L::STAGE_STRIDE;
+  }
+  R* mystage = REC ? stage + lane * L::STAGE_STRIDE : nullptr;
+
+  const R expo = R(-1.0 / double(qerr));
+  const R eps = eps_of<R>();
+  const R span = fabs(p.t1 - p.t0);
+
+  int k = -1;           // current trajectory, -1 when the lane needs work
+  bool alive = true;    // false once the work counter is exhausted for this lane
+  R t = R(0), h = R(0);
+  R y[D], k1[D];
+  typename F::template Theta<R> th;
+  int S = 0, Rj = 0, ns = 0, seq = 0;
+  long long att = 0;
+  bool last_rej = false;
+
+#pragma unroll
+  for (int c = 0; c < D; ++c) { y[c] = R(0); k1[c] = R(0); }
+
+  for (;;) {
+    // ---- refill retired lanes
+    const bool need = alive && k < 0;
+    if (__any_sync(FULL, need)) {
+      const int id = warp_take(need, p.queue);
+      if (need) {
+        if (id < p.N) {
+          k = id;
+          F::load(th, p.theta + (size_t)p.theta_stride * k);
+#pragma unroll
+          for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
+          t = p.t0;
+          S = 0; Rj = 0; att = 0; last_rej = false; ns = 0; seq = 0;
+        } else {
+          alive = false;
+        }
+      }
+      // start-up of the newly taken trajectories: f(y0), finiteness, starting step
+      if (need && k >= 0) {
+        int st = -1;
+        if (!(p.t1 > p.t0)) {
+          st = 0;
+        } else {
+          F::f(y, th, k1);
+          bool finite = true;
+#pragma unroll
+          for (int c = 0; c < D; ++c) finite = finite && isfinite(y[c]) && isfinite(k1[c]);
+          if (!finite) st = 3;
+          else h = initial_step<F, R>(y, k1, th, p.t0, p.t1, p.rtol, p.atol, order);
+        }
+        if (st >= 0) {
+#pragma unroll
+          for (int c = 0; c < D; ++c) p.y1[(size_t)k * D + c] = y[c];
+          if (p.nsteps) p.nsteps[k] = 0;
+          if (p.nrejected) p.nrejected[k] = 0;
+          if (p.status) p.status[k] = st;
+          k = -1;
+        }
+      }
+    }
+    if (!__any_sync(FULL, k >= 0 || alive)) break;
+
+    // ---- one attempted step per active lane
+    bool finishing = false;
+    int fin_traj = -1;
+    if (k >= 0) {
+      int st = -1;
+      if (att >= p.max_attempts) {
+        st = 1;
+      } else if (!(h >= R(16) * eps * fmax(fabs(t), span))) {
+        st = 2;
+      } else {
+        bool clipped = false;
+        if (t + h > p.t1) { h = p.t1 - t; clipped = true; }
+        ++att;
+        R ynew[D];
+        R err;
+        if constexpr (METHOD == M_TSIT5) {
+          R k7[D];
+          err = tsit5_trial<F, R>(y, h, th, k1, ynew, k7, p.rtol, p.atol);
+          if (err <= R(1)) {
+#pragma unroll
+            for (int c = 0; c < D; ++c) k1[c] = k7[c];
+          }
+        } else {
+          err = ros_trial<F, R>(y, h, th, ynew, p.rtol, p.atol);
+        }
+        if (err <= R(1)) {
+          if (REC) {
+            R* e = mystage + ns * L::E;
+            e[0] = t;
+            e[1] = h;
+#pragma unroll
+            for (int c = 0; c < D; ++c) e[2 + c] = y[c];
+            ++ns;
+          }
+          ++S;
+          const R facmax = last_rej ? R(1) : R(10);
+          R fac = (err == R(0)) ? facmax : R(0.9) * pw<R>(err, expo);
+          fac = fmin(facmax, fmax(R(0.2), fac));
+          t = (clipped || t + h >= p.t1) ? p.t1 : t + h;
+#pragma unroll
+          for (int c = 0; c < D; ++c) y[c] = ynew[c];
+          h = h * fac;
+          last_rej = false;
+          if (t == p.t1) st = 0;
+        } else {
+          ++Rj;
+          R fac = isfinite(err) ? R(0.9) * pw<R>(err, expo) : R(0.2);
+          fac = fmin(R(10), fmax(R(0.2), fac));
+          h = h * fac;
+          last_rej = true;
+        }
+      }
+      if (st >= 0) {
+#pragma unroll
+        for (int c = 0; c < D; ++c) p.y1[(size_t)k * D + c] = y[c];
+        if (p.nsteps) p.nsteps[k] = S;
+        if (p.nrejected) p.nrejected[k] = Rj;
+        if (p.status) p.status[k] = st;
+        finishing = true;
+        fin_traj = k;
+        k = -1;
+      }
+    }
+
+    // ---- record: flush full (or final partial) chunks, one warp-wide coalesced copy each
+    if (REC) {
+      const bool want = (ns == L::C) || (finishing && ns > 0);
+      const int owner = finishing ? fin_traj : k;
+      unsigned fm = __ballot_sync(FULL, want);
+      if (fm) {
+        const int leader = __ffs(fm) - 1;
+        int base = 0;
+        if (lane == leader) base = atomicAdd(p.chunk_count, __popc(fm));
+        base = __shfl_sync(FULL, base, leader);
+        const int mychunk = base + __popc(fm & lanemask_lt());
+        if (want) {
+          if (mychunk < p.pool_chunks) {
+            p.chunk_traj[mychunk] = owner;
+            p.chunk_seq[mychunk] = seq;
+          } else {
+            *p.overflow = 1;
+          }
+        }
+        __syncwarp();
+        while (fm) {
+          const int src = __ffs(fm) - 1;
+          fm &= fm - 1;
+          const int ch = __shfl_sync(FULL, mychunk, src);
+          const int cnt = __shfl_sync(FULL, ns, src);
+          if (ch < p.pool_chunks) {
+            R* dst = p.pool + (size_t)ch * (L::C * L::E);
+            const R* s = stage + src * L::STAGE_STRIDE;
+            for (int i = lane; i < cnt * L::E; i += 32) dst[i] = s[i];
+          }
+        }
+        __syncwarp();
+        if (want) { ++seq; ns = 0; }
+      }
+    }
+  }
+}
+
+template <class R>
+struct AdjointParams {
+  int N;
+  const R* theta;
+  int theta_stride;
+  const R* dL_dy1;
+  R* dL_dy0;        // nullable
+  R* dL_dtheta;     // [N][M] per trajectory (or scratch for the shared reduction); nullable
+  const int* nsteps;
+  const long long* choff;   // chunk offsets [N+1]
+  const int* chunk_table;
+  const R* pool;
+  int* queue;
+};
+
+template <class F, class R, int METHOD>
+__global__ void __launch_bounds__(128) k_adjoint(AdjointParams<R> p) {
+  using L = RecLayout<F, R>;
+  constexpr int D = F::D, M = F::M;
+  int k = -1;
+  bool alive = true;
+  int n = 0;
+  long long cbase = 0;
+  R lam[D], thb[M];
+  typename F::template Theta<R> th;
+#pragma unroll
+  for (int c = 0; c < D; ++c) lam[c] = R(0);
+#pragma unroll
+  for (int j = 0; j < M; ++j) thb[j] = R(0);
+
+  for (;;) {
+    const bool need = alive && k < 0;
+    if (__any_sync(FULL, need)) {
+      const int id = warp_take(need, p.queue);
+      if (need) {
+        if (id < p.N) {
+          k = id;
+          F::load(th, p.theta + (size_t)p.theta_stride * k);
+#pragma unroll
+          for (int c = 0; c < D; ++c) lam[c] = p.dL_dy1[(size_t)k * D + c];
+#pragma unroll
+          for (int j = 0; j < M; ++j) thb[j] = R(0);
+          n = p.nsteps[k] - 1;
+          cbase = p.choff[k];
+        } else {
+          alive = false;
+        }
+      }
+    }
+    if (!__any_sync(FULL, k >= 0 || alive)) break;
+    if (k >= 0) {
+      if (n >= 0) {
+        const int ch = __ldg(p.chunk_table + cbase + n / L::C);
+        const R* e = p.pool + ((size_t)ch * L::C + (n % L::C)) * L::E;
+        const R h = __ldg(e + 1);
+        R y[D];
+#pragma unroll
+        for (int c = 0; c < D; ++c) y[c] = __ldg(e + 2 + c);
+        if constexpr (METHOD == M_TSIT5) tsit5_adjoint_step<F, R>(y, h, th, lam, thb);
+        else ros_adjoint_step<F, R>(y, h, th, lam, thb);
+        --n;
+      }
+      if (n < 0) {
+        if (p.dL_dy0)
+#pragma unroll
+          for (int c = 0; c < D; ++c) p.dL_dy0[(size_t)k * D + c] = lam[c];
+        if (p.dL_dtheta)
+#pragma unroll
+          for (int j = 0; j < M; ++j) p.dL_dtheta[(size_t)k * M + j] = thb[j];
+        k = -1;
+      }
+    }
+  }
+}
+
+// Forward replay over the recorded mesh at (possibly new) parameters: y_{n+1} = Phi(y_n, h_n),
+// rewriting the stored y_n of every step so that a following k_adjoint differentiates the replay
+// at these parameters; writes y_S to y1.  t_n and h_n are left as recorded.
+template <class R>
+struct ReplayParams {
+  int N;
+  const R* theta;
+  int theta_stride;
+  const R* y0;
+  R* y1;
+  const int* nsteps;
+  const long long* choff;
+  const int* chunk_table;
+  R* pool;
+  int* queue;
+};
+
+template <class F, class R, int METHOD>
+__global__ void __launch_bounds__(128) k_replay_forward(ReplayParams<R> p) {
+  using L = RecLayout<F, R>;
+  constexpr int D = F::D;
+  int k = -1, n = 0, S = 0;
+  bool alive = true;
+  long long cbase = 0;
+  R y[D];
+  typename F::template Theta<R> th;
+#pragma unroll
+  for (int c = 0; c < D; ++c) y[c] = R(0);
+  for (;;) {
+    const bool need = alive && k < 0;
+    if (__any_sync(FULL, need)) {
+      const int id = warp_take(need, p.queue);
+      if (need) {
+        if (id < p.N) {
+          k = id;
+          F::load(th, p.theta + (size_t)p.theta_stride * k);
+#pragma unroll
+          for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
+          n = 0;
+          S = p.nsteps[k];
+          cbase = p.choff[k];
+        } else {
+          alive = false;
+        }
+      }
+    }
+    if (!__any_sync(FULL, k >= 0 || alive)) break;
+    if (k >= 0) {
+      if (n < S) {
+        const int ch = p.chunk_table[cbase + n / L::C];
+        R* e = p.pool + ((size_t)ch * L::C + (n % L::C)) * L::E;
+        const R h = e[1];
+#pragma unroll
+        for (int c = 0; c < D; ++c) e[2 + c] = y[c];
+        R ynew[D];
+        if constexpr (METHOD == M_TSIT5) tsit5_replay_step<F, R>(y, h, th, ynew);
+        else ros_replay_step<F, R>(y, h, th, ynew);
+#pragma unroll
+        for (int c = 0; c < D; ++c) y[c] = ynew[c];
+        ++n;
+      }
+      if (n >= S) {
+#pragma unroll
+        for (int c = 0; c < D; ++c) p.y1[(size_t)k * D + c] = y[c];
+        k = -1;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Record finalisation.
+// ---------------------------------------------------------------------------------------------
+// Block-wide exclusive scan of per-trajectory counts (steps, or chunks = ceil(steps / C)).
+// Pass 1: each block scans its tile and writes the tile total; pass 2: one block scans the tile
+// totals; pass 3: add the tile base.  Deterministic; int64 outputs.
+constexpr int SCAN_BLOCK = 1024;
+
+template <int MODE>  // 0: steps, 1: chunks of C
+__device__ __forceinline__ long long scan_value(const int* S, int i, int N, int C) {
+  if (i >= N) return 0;
+  const int s = S[i];
+  return MODE == 0 ? (long long)s : (long long)((s + C - 1) / C);
+}
+
+__device__ __forceinline__ long long block_exclusive_scan(long long v, long long* total) {
+  __shared__ long long warp_sums[SCAN_BLOCK / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(FULL, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    long long w = (lane < SCAN_BLOCK / 32) ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(FULL, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sums[lane] = w;
+  }
+  __syncthreads();
+  const long long before = (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
+  *total = warp_sums[SCAN_BLOCK / 32 - 1];
+  __syncthreads();
+  return before;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(SCAN_BLOCK) k_scan_tiles(const int* S, int N, int C,
+                                                           long long* out, long long* tile_tot) {
+  const int i = blockIdx.x * SCAN_BLOCK + threadIdx.x;
+  long long tot;
+  const long long ex = block_exclusive_scan(scan_value<MODE>(S, i, N, C), &tot);
+  if (i < N) out[i] = ex;
+  if (threadIdx.x == 0) tile_tot[blockIdx.x] = tot;
+}
+
+__global__ void __launch_bounds__(SCAN_BLOCK) k_scan_totals(long long* tile_tot, int ntiles,
+                                                            long long* grand) {
+  long long carry = 0;
+  for (int b0 = 0; b0 < ntiles; b0 += SCAN_BLOCK) {
+    const int i = b0 + threadIdx.x;
+    long long tot;
+    const long long v = i < ntiles ? tile_tot[i] : 0;
+    const long long ex = block_exclusive_scan(v, &tot);
+    if (i < ntiles) tile_tot[i] = carry + ex;
+    carry += tot;
+  }
+  if (threadIdx.x == 0) *grand = carry;
+}
+
+__global__ void k_scan_add(long long* out, int N, const long long* tile_base,
+                           const long long* grand) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < N) out[i] += tile_base[i / SCAN_BLOCK];
+  if (i == 0) out[N] = *grand;
+}
+
+// chunk_table[choff[traj] + seq] = chunk
+__global__ void k_chunk_table(const int* chunk_traj, const int* chunk_seq, int nchunks,
+                              const long long* choff, int* table) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c < nchunks) table[choff[chunk_traj[c]] + chunk_seq[c]] = c;
+}
+
+// max over S (int), via warp reduce + atomicMax
+__global__ void k_max_int(const int* S, int N, int* out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  int v = i < N ? S[i] : 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(FULL, v, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(out, v);
+}
+
+// Export: write the record as contiguous ragged arrays T[tot], H[tot], Y[tot][D] in
+// trajectory-major order (offsets = prefix sums of S).  One thread per trajectory-step.
+template <class R>
+__global__ void k_export(const R* pool, const int* table, const long long* choff,
+                         const long long* offsets, int N, int D, int C, long long total, R* T,
+                         R* H, R* Y) {
+  const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (g >= total) return;
+  // binary search the trajectory owning step g
+  int lo = 0, hi = N - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (offsets[mid] <= g) lo = mid; else hi = mid - 1;
+  }
+  const int k = lo;
+  const long long n = g - offsets[k];
+  const int E = 2 + D;
+  const int ch = table[choff[k] + n / C];
+  const R* e = pool + ((size_t)ch * C + (n % C)) * E;
+  if (T) T[g] = e[0];
+  if (H) H[g] = e[1];
+  if (Y) for (int c = 0; c < D; ++c) Y[g * D + c] = e[2 + c];
+}
+
+// Import: inverse of export into a pool whose chunks are laid out trajectory by trajectory
+// (chunk id = choff[k] + n / C, so chunk_table is the identity).
+template <class R>
+__global__ void k_import(R* pool, const long long* choff, const long long* offsets, int N, int D,
+                         int C, long long total, const R* T, const R* H, const R* Y) {
+  const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (g >= total) return;
+  int lo = 0, hi = N - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (offsets[mid] <= g) lo = mid; else hi = mid - 1;
+  }
+  const int k = lo;
+  const long long n = g - offsets[k];
+  const int E = 2 + D;
+  const long long ch = choff[k] + n / C;
+  R* e = pool + ((size_t)ch * C + (n % C)) * E;
+  e[0] = T ? T[g] : R(0);
+  e[1] = H[g];
+  for (int c = 0; c < D; ++c) e[2 + c] = Y[g * D + c];
+}
+
+__global__ void k_iota(int* a, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) a[i] = i;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Shared-theta reduction: out[j] = sum_k part[k][j] in a fixed order.  Each block reduces a fixed
+// contiguous slice of trajectories (warp shuffles, then shared memory), writes its partial; a
+// second launch with one block sums the partials in block order.  Bitwise reproducible.
+// ---------------------------------------------------------------------------------------------
+constexpr int RED_BLOCK = 256;
+
+template <class R>
+__global__ void __launch_bounds__(RED_BLOCK) k_reduce_theta(const R* part, int N, int M,
+                                                            int per_block, R* partials) {
+  __shared__ R warp_acc[RED_BLOCK / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int k0 = blockIdx.x * per_block;
+  const int k1 = min(N, k0 + per_block);
+  for (int j = 0; j < M; ++j) {
+    R acc = R(0);
+    for (int k = k0 + threadIdx.x; k < k1; k += RED_BLOCK) acc += part[(size_t)k * M + j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
+    if (lane == 0) warp_acc[warp] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      R s = R(0);
+      for (int w = 0; w < RED_BLOCK / 32; ++w) s += warp_acc[w];
+      partials[(size_t)blockIdx.x * M + j] = s;
+    }
+    __syncthreads();
+  }
+}
+
+template <class R>
+__global__ void k_reduce_partials(const R* partials, int nblocks, int M, R* out) {
+  for (int j = threadIdx.x; j < M; j += blockDim.x) {
+    R s = R(0);
+    for (int b = 0; b < nblocks; ++b) s += partials[(size_t)b * M + j];
+    out[j] = s;
+  }
+}
+
+}  // namespace gs

@@ -1,0 +1,472 @@
+// gs_methods.cuh -- the one-step maps on the device: Tsit5 trial step (record / forward),
+// Tsit5 replay-adjoint step, ROS34PW2 trial step and its replay-adjoint step.
+//
+// Method structure: "gradsolve: fast exact gradients for ODE ensembles on GPUs" §2.1 (embedded
+// explicit pair with first-same-as-last reuse; RMS error test), §3 (replay map Phi with the
+// recorded step size as data; its reverse-mode derivative), §3.2 (Rosenbrock stage solves with
+// I - gamma h J; the backward pass needs one solve with the transpose and differentiates J).
+// Coefficients (not printed on the pages): Tsitouras (2011) for Tsit5, Rang & Angermann (2005)
+// for ROS34PW2 -- the published decimals, rounded to the working precision at compile time.
+#pragma once
+#include "gs_fields.cuh"
+
+namespace gs {
+
+struct Tsit5 {
+  static constexpr int order = 5, err_order = 5;
+  // a_ij, i = 2..7, j < i; row 7 equals b (b_7 = 0).
+  static constexpr double a21 = 0.161;
+  static constexpr double a31 = -0.008480655492356989, a32 = 0.335480655492357;
+  static constexpr double a41 = 2.897153057105493, a42 = -6.359448489975075,
+                          a43 = 4.3622954328695815;
+  static constexpr double a51 = 5.325864828439257, a52 = -11.748883564062828,
+                          a53 = 7.4955393428898365, a54 = -0.09249506636175525;
+  static constexpr double a61 = 5.86145544294642, a62 = -12.92096931784711,
+                          a63 = 8.159367898576159, a64 = -0.071584973281401,
+                          a65 = -0.028269050394068383;
+  static constexpr double b1 = 0.09646076681806523, b2 = 0.01, b3 = 0.4798896504144996,
+                          b4 = 1.379008574103742, b5 = -3.290069515436081,
+                          b6 = 2.324710524099774;
+  // error weights b - b_hat
+  static constexpr double e1 = -0.00178001105222577714, e2 = -0.0008164344596567469,
+                          e3 = 0.007880878010261995, e4 = -0.1447110071732629,
+                          e5 = 0.5823571654525552, e6 = -0.45808210592918697,
+                          e7 = 0.015151515151515152;
+};
+
+// A[i][j] of the explicit stages as a device-evaluable table (i = 0..5 stage index, j < i).
+template <class R> __device__ __forceinline__ R ta(int i, int j) {
+  // Resolved at compile time inside fully unrolled loops.
+  constexpr double A[6][5] = {
+      {0, 0, 0, 0, 0},
+      {Tsit5::a21, 0, 0, 0, 0},
+      {Tsit5::a31, Tsit5::a32, 0, 0, 0},
+      {Tsit5::a41, Tsit5::a42, Tsit5::a43, 0, 0},
+      {Tsit5::a51, Tsit5::a52, Tsit5::a53, Tsit5::a54, 0},
+      {Tsit5::a61, Tsit5::a62, Tsit5::a63, Tsit5::a64, Tsit5::a65}};
+  return R(A[i][j]);
+}
+template <class R> __device__ __forceinline__ R tb(int i) {
+  constexpr double B[6] = {Tsit5::b1, Tsit5::b2, Tsit5::b3, Tsit5::b4, Tsit5::b5, Tsit5::b6};
+  return R(B[i]);
+}
+template <class R> __device__ __forceinline__ R te(int i) {
+  constexpr double E[7] = {Tsit5::e1, Tsit5::e2, Tsit5::e3, Tsit5::e4,
+                           Tsit5::e5, Tsit5::e6, Tsit5::e7};
+  return R(E[i]);
+}
+
+// One Tsit5 trial from y with step h; k1 = f(y) is carried (first-same-as-last).  Produces the
+// step result ynew, its slope k7 = f(ynew) (the next k1) and the scaled RMS error
+//   err = sqrt(mean_i (e_i / (atol + rtol max(|y_i|, |ynew_i|)))^2),  e = h sum_j (b_j - bh_j) k_j.
+template <class F, class R>
+__device__ __forceinline__ R tsit5_trial(const R (&y)[F::D], R h, const typename F::template Theta<R>& th,
+                                         const R (&k1)[F::D], R (&ynew)[F::D], R (&k7)[F::D],
+                                         R rtol, R atol) {
+  constexpr int D = F::D;
+  R k[6][D];
+#pragma unroll
+  for (int c = 0; c < D; ++c) k[0][c] = k1[c];
+#pragma unroll
+  for (int i = 1; i < 6; ++i) {
+    R Y[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+      R s = ta<R>(i, 0) * k[0][c];
+#pragma unroll
+      for (int j = 1; j < i; ++j) s += ta<R>(i, j) * k[j][c];
+      Y[c] = y[c] + h * s;
+    }
+    F::f(Y, th, k[i]);
+  }
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    R s = tb<R>(0) * k[0][c];
+#pragma unroll
+    for (int j = 1; j < 6; ++j) s += tb<R>(j) * k[j][c];
+    ynew[c] = y[c] + h * s;
+  }
+  F::f(ynew, th, k7);
+  R acc = R(0);
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    R s = te<R>(0) * k[0][c];
+#pragma unroll
+    for (int j = 1; j < 6; ++j) s += te<R>(j) * k[j][c];
+    s += te<R>(6) * k7[c];
+    const R e = h * s;
+    const R sc = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
+    const R q = e / sc;
+    acc += q * q;
+  }
+  return sqrt(acc / R(D));
+}
+
+// The Tsit5 replay map Phi(y, h) = y + h sum_{i<=6} b_i k_i with k_1 = f(y) (no error estimate).
+template <class F, class R>
+__device__ __forceinline__ void tsit5_replay_step(const R (&y)[F::D], R h,
+                                                  const typename F::template Theta<R>& th,
+                                                  R (&ynew)[F::D]) {
+  constexpr int D = F::D;
+  R k[6][D];
+  F::f(y, th, k[0]);
+#pragma unroll
+  for (int i = 1; i < 6; ++i) {
+    R Y[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+      R s = ta<R>(i, 0) * k[0][c];
+#pragma unroll
+      for (int j = 1; j < i; ++j) s += ta<R>(i, j) * k[j][c];
+      Y[c] = y[c] + h * s;
+    }
+    F::f(Y, th, k[i]);
+  }
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    R s = tb<R>(0) * k[0][c];
+#pragma unroll
+    for (int j = 1; j < 6; ++j) s += tb<R>(j) * k[j][c];
+    ynew[c] = y[c] + h * s;
+  }
+}
+
+// Reverse-mode step of the Tsit5 replay map y_{n+1} = y_n + h sum_{i<=6} b_i k_i with h fixed:
+// recompute the stages from the recorded y_n, then sweep them backwards.
+//   kb_i = h (b_i lam + sum_{j>i} a_ji Yb_j),  Yb_i = J_y(Y_i)^T kb_i,  thb += J_th(Y_i)^T kb_i,
+//   lam <- lam + sum_i Yb_i.
+template <class F, class R>
+__device__ __forceinline__ void tsit5_adjoint_step(const R (&y)[F::D], R h,
+                                                   const typename F::template Theta<R>& th,
+                                                   R (&lam)[F::D], R (&thb)[F::M]) {
+  constexpr int D = F::D;
+  R Y[6][D];
+  {
+    R k[5][D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) Y[0][c] = y[c];
+    F::f(Y[0], th, k[0]);
+#pragma unroll
+    for (int i = 1; i < 6; ++i) {
+#pragma unroll
+      for (int c = 0; c < D; ++c) {
+        R s = ta<R>(i, 0) * k[0][c];
+#pragma unroll
+        for (int j = 1; j < i; ++j) s += ta<R>(i, j) * k[j][c];
+        Y[i][c] = y[c] + h * s;
+      }
+      if (i < 5) F::f(Y[i], th, k[i]);
+    }
+  }
+  R G[5][D];
+#pragma unroll
+  for (int i = 0; i < 5; ++i)
+#pragma unroll
+    for (int c = 0; c < D; ++c) G[i][c] = R(0);
+  R lnew[D];
+#pragma unroll
+  for (int c = 0; c < D; ++c) lnew[c] = lam[c];
+#pragma unroll
+  for (int i = 5; i >= 0; --i) {
+    R kb[D], Yb[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+      const R g = (i < 5) ? G[i][c] : R(0);
+      kb[c] = h * (tb<R>(i) * lam[c] + g);
+    }
+    F::vjp(Y[i], th, kb, Yb, thb);
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+      lnew[c] += Yb[c];
+#pragma unroll
+      for (int j = 0; j < i; ++j) G[j][c] += ta<R>(i, j) * Yb[c];
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < D; ++c) lam[c] = lnew[c];
+}
+
+// ------------------------------------------------------------------------------------------------
+// ROS34PW2: (I - gamma h J) k_i = h f(y + sum_{j<i} alpha_ij k_j) + h J sum_{j<i} gamma_ij k_j,
+// y_{n+1} = y + sum b_i k_i, e = sum (b_i - bh_i) k_i, J = f_y(y_n) exact.
+// ------------------------------------------------------------------------------------------------
+struct Ros34pw2 {
+  static constexpr int order = 3, err_order = 3;
+  static constexpr double gamma = 0.435866521508459;
+};
+template <class R> __device__ __forceinline__ R ral(int i, int j) {
+  constexpr double A[4][3] = {{0, 0, 0},
+                              {0.87173304301691801, 0, 0},
+                              {0.84457060015369423, -0.11299064236484185, 0},
+                              {0, 0, 1.0}};
+  return R(A[i][j]);
+}
+template <class R> __device__ __forceinline__ R rga(int i, int j) {
+  constexpr double G[4][3] = {{0, 0, 0},
+                              {-0.87173304301691801, 0, 0},
+                              {-0.90338057013044082, 0.054180672388095326, 0},
+                              {0.24212380706095346, -1.2232505839045147, 0.54526025533510214}};
+  return R(G[i][j]);
+}
+template <class R> __device__ __forceinline__ R rb(int i) {
+  constexpr double B[4] = {0.24212380706095346, -1.2232505839045147, 1.5452602553351020,
+                           0.435866521508459};
+  return R(B[i]);
+}
+// b_i - bhat_i
+template <class R> __device__ __forceinline__ R rbe(int i) {
+  constexpr double B[4] = {0.24212380706095346, -1.2232505839045147, 1.5452602553351020,
+                           0.435866521508459};
+  constexpr double BH[4] = {0.37810903145819369, -0.096042292212423178, 0.5, 0.2179332607542295};
+  return R(B[i]) - R(BH[i]);
+}
+
+// In-register LU of a D x D matrix with partial pivoting (largest |entry|, ties to the lowest
+// row).  The permutation is kept as a row map p[] so that solves index without data movement.
+template <class R, int D>
+struct SmallLU {
+  R lu[D][D];
+  int p[D];
+  __device__ __forceinline__ void factor(const R (&A)[D][D]) {
+#pragma unroll
+    for (int r = 0; r < D; ++r) {
+      p[r] = r;
+#pragma unroll
+      for (int c = 0; c < D; ++c) lu[r][c] = A[r][c];
+    }
+#pragma unroll
+    for (int col = 0; col < D; ++col) {
+      // choose the pivot among rows col..D-1 and swap it into place (register-resident selects)
+#pragma unroll
+      for (int r = col + 1; r < D; ++r) {
+        if (fabs(lu[r][col]) > fabs(lu[col][col])) {
+#pragma unroll
+          for (int c = 0; c < D; ++c) { R tmp = lu[r][c]; lu[r][c] = lu[col][c]; lu[col][c] = tmp; }
+          int t = p[r]; p[r] = p[col]; p[col] = t;
+        }
+      }
+      const R inv = R(1) / lu[col][col];
+#pragma unroll
+      for (int r = col + 1; r < D; ++r) {
+        const R l = lu[r][col] * inv;
+        lu[r][col] = l;
+#pragma unroll
+        for (int c = col + 1; c < D; ++c) lu[r][c] -= l * lu[col][c];
+      }
+    }
+  }
+  // x = A^{-1} b   (P A = L U)
+  __device__ __forceinline__ void solve(const R (&bb)[D], R (&x)[D]) const {
+#pragma unroll
+    for (int r = 0; r < D; ++r) {
+      R v = R(0);
+#pragma unroll
+      for (int s = 0; s < D; ++s) v = (p[r] == s) ? bb[s] : v;
+      x[r] = v;
+    }
+#pragma unroll
+    for (int r = 1; r < D; ++r)
+#pragma unroll
+      for (int c = 0; c < r; ++c) x[r] -= lu[r][c] * x[c];
+#pragma unroll
+    for (int r = D - 1; r >= 0; --r) {
+#pragma unroll
+      for (int c = r + 1; c < D; ++c) x[r] -= lu[r][c] * x[c];
+      x[r] = x[r] / lu[r][r];
+    }
+  }
+  // x = A^{-T} b:  A^T = U^T L^T P, so solve U^T z = b, L^T w = z, x = P^T w.
+  __device__ __forceinline__ void solve_t(const R (&bb)[D], R (&x)[D]) const {
+    R z[D];
+#pragma unroll
+    for (int r = 0; r < D; ++r) {
+      R v = bb[r];
+#pragma unroll
+      for (int c = 0; c < r; ++c) v -= lu[c][r] * z[c];
+      z[r] = v / lu[r][r];
+    }
+#pragma unroll
+    for (int r = D - 1; r >= 0; --r)
+#pragma unroll
+      for (int c = r + 1; c < D; ++c) z[r] -= lu[c][r] * z[c];
+#pragma unroll
+    for (int s = 0; s < D; ++s) {
+      R v = R(0);
+#pragma unroll
+      for (int r = 0; r < D; ++r) v = (p[r] == s) ? z[r] : v;
+      x[s] = v;
+    }
+  }
+};
+
+template <class F, class R>
+__device__ __forceinline__ void ros_stages(const R (&y)[F::D], R h,
+                                           const typename F::template Theta<R>& th,
+                                           const R (&J)[F::D * F::D], const SmallLU<R, F::D>& lu,
+                                           R (&k)[4][F::D]) {
+  constexpr int D = F::D;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    R Y[D], G[D], fy[D], r[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+      R u = R(0), g = R(0);
+#pragma unroll
+      for (int j = 0; j < i; ++j) {
+        u += ral<R>(i, j) * k[j][c];
+        g += rga<R>(i, j) * k[j][c];
+      }
+      Y[c] = y[c] + u;
+      G[c] = g;
+    }
+    F::f(Y, th, fy);
+#pragma unroll
+    for (int rr = 0; rr < D; ++rr) {
+      R jg = R(0);
+#pragma unroll
+      for (int c = 0; c < D; ++c) jg += J[rr * D + c] * G[c];
+      r[rr] = h * fy[rr] + h * jg;
+    }
+    lu.solve(r, k[i]);
+  }
+}
+
+template <class F, class R>
+__device__ __forceinline__ void ros_matrix(const R (&y)[F::D], R h,
+                                           const typename F::template Theta<R>& th,
+                                           R (&J)[F::D * F::D], SmallLU<R, F::D>& lu) {
+  constexpr int D = F::D;
+  F::jac(y, th, J);
+  const R gh = R(Ros34pw2::gamma) * h;
+  R Mx[D][D];
+#pragma unroll
+  for (int r = 0; r < D; ++r)
+#pragma unroll
+    for (int c = 0; c < D; ++c) Mx[r][c] = (r == c ? R(1) : R(0)) - gh * J[r * D + c];
+  lu.factor(Mx);
+}
+
+template <class F, class R>
+__device__ __forceinline__ R ros_trial(const R (&y)[F::D], R h,
+                                       const typename F::template Theta<R>& th,
+                                       R (&ynew)[F::D], R rtol, R atol) {
+  constexpr int D = F::D;
+  R J[D * D];
+  SmallLU<R, D> lu;
+  ros_matrix<F, R>(y, h, th, J, lu);
+  R k[4][D];
+  ros_stages<F, R>(y, h, th, J, lu, k);
+  R acc = R(0);
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    R s = rb<R>(0) * k[0][c];
+    R e = rbe<R>(0) * k[0][c];
+#pragma unroll
+    for (int i = 1; i < 4; ++i) {
+      s += rb<R>(i) * k[i][c];
+      e += rbe<R>(i) * k[i][c];
+    }
+    ynew[c] = y[c] + s;
+    const R sc = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
+    const R q = e / sc;
+    acc += q * q;
+  }
+  return sqrt(acc / R(D));
+}
+
+// The ROS34PW2 replay map (no error estimate).
+template <class F, class R>
+__device__ __forceinline__ void ros_replay_step(const R (&y)[F::D], R h,
+                                                const typename F::template Theta<R>& th,
+                                                R (&ynew)[F::D]) {
+  constexpr int D = F::D;
+  R J[D * D];
+  SmallLU<R, D> lu;
+  ros_matrix<F, R>(y, h, th, J, lu);
+  R k[4][D];
+  ros_stages<F, R>(y, h, th, J, lu, k);
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    R s = rb<R>(0) * k[0][c];
+#pragma unroll
+    for (int i = 1; i < 4; ++i) s += rb<R>(i) * k[i][c];
+    ynew[c] = y[c] + s;
+  }
+}
+
+// Reverse-mode step of the ROS34PW2 replay map with h fixed.  With M = I - gamma h J,
+// r_i = h f(Y_i) + h J G_i, M k_i = r_i, the backward pass for stage i = 4..1 is
+//   mu_i = M^{-T} kb_i                          (one transpose solve, same LU)
+//   Jb  += gamma h mu_i k_i^T + h mu_i G_i^T     (M depends on J; r_i depends on J)
+//   fb_i = h mu_i -> Yb_i = J_y(Y_i)^T fb_i, thb += J_th(Y_i)^T fb_i
+//   kb_j += alpha_ij Yb_i + gamma_ij h J^T mu_i   for j < i
+//   yb  += Yb_i
+// and finally yb += Jb : dJ/dy, thb += Jb : dJ/dtheta; lam <- yb (with yb starting at lam).
+template <class F, class R>
+__device__ __forceinline__ void ros_adjoint_step(const R (&y)[F::D], R h,
+                                                 const typename F::template Theta<R>& th,
+                                                 R (&lam)[F::D], R (&thb)[F::M]) {
+  constexpr int D = F::D;
+  R J[D * D];
+  SmallLU<R, D> lu;
+  ros_matrix<F, R>(y, h, th, J, lu);
+  R k[4][D];
+  ros_stages<F, R>(y, h, th, J, lu, k);
+  R kb[4][D], Jb[D * D], yb[D];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int c = 0; c < D; ++c) kb[i][c] = rb<R>(i) * lam[c];
+#pragma unroll
+  for (int i = 0; i < D * D; ++i) Jb[i] = R(0);
+#pragma unroll
+  for (int c = 0; c < D; ++c) yb[c] = lam[c];
+  const R gh = R(Ros34pw2::gamma) * h;
+#pragma unroll
+  for (int i = 3; i >= 0; --i) {
+    R mu[D];
+    lu.solve_t(kb[i], mu);
+    R Y[D], G[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+      R u = R(0), g = R(0);
+#pragma unroll
+      for (int j = 0; j < i; ++j) {
+        u += ral<R>(i, j) * k[j][c];
+        g += rga<R>(i, j) * k[j][c];
+      }
+      Y[c] = y[c] + u;
+      G[c] = g;
+    }
+#pragma unroll
+    for (int r = 0; r < D; ++r)
+#pragma unroll
+      for (int c = 0; c < D; ++c) Jb[r * D + c] += mu[r] * (gh * k[i][c] + h * G[c]);
+    R fb[D], Yb[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) fb[c] = h * mu[c];
+    F::vjp(Y, th, fb, Yb, thb);
+    if (i > 0) {
+      R Jtmu[D];
+#pragma unroll
+      for (int c = 0; c < D; ++c) {
+        R s = R(0);
+#pragma unroll
+        for (int r = 0; r < D; ++r) s += J[r * D + c] * mu[r];
+        Jtmu[c] = h * s;
+      }
+#pragma unroll
+      for (int j = 0; j < i; ++j)
+#pragma unroll
+        for (int c = 0; c < D; ++c)
+          kb[j][c] += ral<R>(i, j) * Yb[c] + rga<R>(i, j) * Jtmu[c];
+    }
+#pragma unroll
+    for (int c = 0; c < D; ++c) yb[c] += Yb[c];
+  }
+  F::jac_vjp(y, th, Jb, yb, thb);
+#pragma unroll
+  for (int c = 0; c < D; ++c) lam[c] = yb[c];
+}
+
+}  // namespace gs

@@ -1,0 +1,170 @@
+/* gradsolve_b200.h -- C ABI of the B200 record-and-replay discrete-adjoint library.
+ *
+ * What it computes ("gradsolve: fast exact gradients for ODE ensembles on GPUs"):
+ *   An ensemble of N independent trajectories dy/dt = f(y; theta_k), y(t0) = y0_k, is solved with
+ *   an adaptive embedded pair (§2.1: trial steps, RMS error test
+ *   RMS(e / (atol + rtol max(|y|, |y_new|))) <= 1, reject and retry from the same (t, y)).
+ *   The record pass keeps each trajectory's accepted steps (§3, Fig. 2: the mesh h = R(theta0);
+ *   rejected trials leave no trace), and the replay gradient is the exact reverse-mode derivative of
+ *   the fixed-step replay over that mesh with the mesh held fixed as data (§3: d Psi(theta;
+ *   sg[R(theta0)]) / d theta, Eq. 4), with respect to theta, y0 or both.  The loss is a scalar
+ *   L = sum_k l(y_k(t1; theta)) (§2.2), so the caller passes dL/dy1 and receives the pull-back.
+ *   Non-stiff problems use the Tsit5 5(4) pair with first-same-as-last reuse (§2.1, §3.1); stiff
+ *   problems a linearly implicit Rosenbrock-Wanner step, here ROS34PW2, whose stages solve with
+ *   I - gamma h J and whose backward pass uses one transpose solve per stage and differentiates J
+ *   (§3.2).  One GPU thread integrates one trajectory with its state in registers (§2.4, §4.1).
+ *
+ * Conventions (all entry points):
+ *   - Real arrays are double (GS_F64) or float (GS_F32) per gs_system.dtype, row-major:
+ *     y0, y1, dL_dy1, dL_dy0: [N][d];  theta, dL_dtheta: [N][m], or [m] when theta_shared.
+ *   - Array pointers are DEVICE pointers owned by the caller, unless stated otherwise.  The record
+ *     (gs_record) is owned by the library and freed by gs_record_destroy.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued on it; calls
+ *     return when the work is enqueued, except where a host synchronisation is stated.
+ *   - Errors: every entry point returns a gs_status and never aborts or exits; gs_last_error()
+ *     returns a message for the calling thread's most recent failure.
+ *   - Per-trajectory status codes (status arrays): 0 ok; 1 max_attempts reached; 2 step size
+ *     underflow (h < 16 eps max(|t|, |t1 - t0|) or h not finite); 3 y0 or f(y0) not finite.  A
+ *     failed trajectory's record ends at its last accepted step and y1 holds its state there.
+ *   - Sizes: N <= 2^31 - 1; the record holds at most 2^31 - 1 chunks.
+ */
+#ifndef GRADSOLVE_B200_H
+#define GRADSOLVE_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GS_OK = 0,
+  GS_ERR_INVALID_ARG = 1,  /* bad pointer, size, enum or inconsistent d/m */
+  GS_ERR_CUDA = 2,         /* a CUDA call failed; see gs_last_error() */
+  GS_ERR_CAPACITY = 3,     /* a size limit of the library was exceeded */
+  GS_ERR_UNSUPPORTED = 4,  /* field/method/dtype combination not built */
+  GS_ERR_TRAJ_FAILED = 5   /* gs_solve_record only: some trajectory status != 0 */
+} gs_status;
+
+typedef enum { GS_F64 = 0, GS_F32 = 1 } gs_dtype;
+typedef enum { GS_TSIT5 = 0, GS_ROS34PW2 = 1 } gs_method;
+
+/* Built-in fields (all autonomous).  d = state size, m = parameters per trajectory.
+ *   GS_LOTKA_VOLTERRA  d=2 m=4     theta = (alpha, beta, gamma, delta)
+ *   GS_LORENZ63        d=3 m=3     theta = (sigma, rho, beta)            ([GS] §4.3)
+ *   GS_MLP_4_32_32_4   d=4 m=1348  tanh MLP 4->32->32->4, theta = (W1,b1,W2,b2,W3,b3), shared
+ *   GS_ROBERTSON       d=3 m=3     theta = (k1, k2, k3), stiff          ([GS] §4.2, §4.5)
+ *   GS_NFW_MN          d=6 m=5     test particle in NFW halo + Miyamoto-Nagai disk,
+ *                                  theta = (M_h, r_s, M_d, a, b), G = 1
+ *   GS_LINEAR          d=3 m=9     y' = A y, theta = A row-major         ([GS] §4.6-4.7) */
+typedef enum {
+  GS_LOTKA_VOLTERRA = 0,
+  GS_LORENZ63 = 1,
+  GS_MLP_4_32_32_4 = 2,
+  GS_ROBERTSON = 3,
+  GS_NFW_MN = 4,
+  GS_LINEAR = 5
+} gs_field;
+
+typedef struct {
+  int32_t field;        /* gs_field */
+  int32_t method;       /* gs_method: GS_TSIT5 for non-stiff fields, GS_ROS34PW2 for stiff ones */
+  int32_t dtype;        /* gs_dtype */
+  int32_t d, m;         /* must equal the field's sizes (checked) */
+  int32_t theta_shared; /* 1: theta is [m] shared by all trajectories; 0: [N][m] */
+} gs_system;
+
+typedef struct {
+  int64_t max_attempts;          /* per trajectory; <= 0 means the default 100000 */
+  int64_t record_capacity_steps; /* initial record pool size in steps; 0 = automatic */
+} gs_options;
+
+typedef struct gs_record gs_record; /* opaque, library-owned, device resident */
+
+typedef struct {
+  int64_t N;
+  int64_t total_steps;      /* sum of accepted steps over the ensemble */
+  int32_t max_steps;        /* longest record */
+  int32_t chunk_steps;      /* C: steps per pool chunk */
+  int32_t entry_reals;      /* E = 2 + d: reals per recorded step (t_n, h_n, y_n[0..d-1]) */
+  int32_t dtype;
+  int64_t nchunks;          /* chunks in use */
+  int64_t pool_bytes;       /* device bytes of the step pool */
+  /* device pointers owned by the record */
+  const int32_t* nsteps;        /* [N] accepted steps S_k */
+  const int32_t* status;        /* [N] per-trajectory status */
+  const int64_t* offsets;       /* [N+1] exclusive prefix sum of S_k (ragged-array offsets) */
+  const int64_t* chunk_offsets; /* [N+1] exclusive prefix sum of ceil(S_k / C) */
+  const int32_t* chunk_table;   /* [nchunks]: chunk id of trajectory k's j-th chunk at
+                                   chunk_offsets[k] + j */
+  const void* pool;             /* chunk c holds steps of one trajectory at
+                                   pool + (c*C + slot)*E reals, entry = (t, h, y[0..d-1]) */
+} gs_record_info_t;
+
+/* Forward-only solve ([GS] §4.1: one thread per trajectory, final state only).
+ * In:  theta, y0 (device), t0 < t1 (t1 <= t0 returns y1 = y0 with 0 steps), rtol, atol > 0.
+ * Out: y1 [N][d]; nsteps, nrejected, status [N] (int32, each nullable).
+ * Asynchronous: no host synchronisation; per-trajectory failures appear only in `status`. */
+gs_status gs_solve_forward(const gs_system* sys, const gs_options* opt, int64_t N,
+                           const void* theta, const void* y0, double t0, double t1, double rtol,
+                           double atol, void* y1, int32_t* nsteps, int32_t* nrejected,
+                           int32_t* status, void* stream);
+
+/* Record pass ([GS] §3, Fig. 2): the same adaptive solve, keeping each accepted step
+ * (t_n, h_n, y_n) = (start time, step size used, state at the start of the step), n < S_k.
+ * *rec: if NULL on entry a new record is created; otherwise its storage is reused (grown when
+ * needed) and its contents replaced.  y1 [N][d] (device, required), status [N] (nullable).
+ * Synchronises the stream once to size the record; if the pool was too small the solve is run
+ * again with exactly the needed size.  Returns GS_ERR_TRAJ_FAILED (with the record complete)
+ * when some trajectory status != 0. */
+gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N,
+                          const void* theta, const void* y0, double t0, double t1, double rtol,
+                          double atol, gs_record** rec, void* y1, int32_t* status, void* stream);
+
+/* Replay gradient ([GS] §3): the exact reverse-mode derivative of the replay over the recorded
+ * mesh with the mesh held fixed as data.  The backward sweep recomputes each step's stages from
+ * the state stored for that step ([GS] §3.3: one accepted state kept per step): the states of the
+ * record pass, or of the latest gs_replay_forward.  With the stored states made at theta0 and
+ * `theta` = theta0 the result is d Psi(theta0; sg[R(theta0)]) / d theta.  For a gradient at another
+ * theta on the same mesh (d Psi(theta; sg[R(theta0)]) / d theta), call gs_replay_forward(theta)
+ * first.
+ * In:  theta (as for the solve), dL_dy1 [N][d].  Out (each nullable, at least one non-NULL):
+ * dL_dy0 [N][d]; dL_dtheta [N][m], or [m] = sum over the ensemble when theta is shared (summed in
+ * a fixed order: bitwise reproducible).  Asynchronous. */
+gs_status gs_replay_grad(const gs_record* rec, const void* theta, const void* dL_dy1,
+                         void* dL_dtheta, void* dL_dy0, void* stream);
+
+/* Forward replay ([GS] §3, Eq. 4): y_{n+1} = Phi(y_n, h_n; theta) over the recorded mesh from y0,
+ * storing each y_n in the record (t_n and h_n are kept) and y_S in y1 [N][d] (device, nullable).
+ * Asynchronous. */
+gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, void* y1,
+                            void* stream);
+
+/* Sizes and device pointers of a record (no synchronisation). */
+gs_status gs_record_info(const gs_record* rec, gs_record_info_t* out);
+
+/* Copy the record out as contiguous ragged arrays in trajectory order: T[total], H[total],
+ * Y[total][d] (device, each nullable) and offsets [N+1] (device int64, nullable). */
+gs_status gs_record_export(const gs_record* rec, void* T, void* H, void* Y, int64_t* offsets,
+                           void* stream);
+
+/* Build a record from contiguous ragged arrays (device): nsteps [N] int32, T [total] (nullable,
+ * zeros when NULL), H [total], Y [total][d] with total = sum nsteps.  Lets one mesh be replayed
+ * by another producer's record or reused across many gradients ([GS] §4.8).  Synchronises once. */
+gs_status gs_record_import(const gs_system* sys, int64_t N, const int32_t* nsteps, const void* T,
+                           const void* H, const void* Y, gs_record** rec, void* stream);
+
+/* Free a record (NULL is ignored).  Synchronises the record's device. */
+void gs_record_destroy(gs_record* rec);
+
+/* Message of the calling thread's last failure ("" if none). */
+const char* gs_last_error(void);
+
+/* Library version string. */
+const char* gs_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GRADSOLVE_B200_H */

@@ -1,0 +1,56 @@
+// Host program that tallies the arithmetic of the device fields' f and vector-Jacobian product
+// (add/sub, mul, div, sqrt, log1p per call) by instantiating them with a counting scalar.
+// Compiled as plain C++ (g++) and run by tests/test_flop_counts.py; prints one JSON object per field.
+#include <cmath>
+#include <cstdio>
+
+#include "gs_fields.cuh"
+
+struct Tally { long add = 0, mul = 0, div = 0, sqrt = 0, log1p = 0; };
+static Tally T;
+struct Cnt {
+  double v;
+  Cnt() : v(0) {}
+  Cnt(double x) : v(x) {}
+  Cnt& operator+=(Cnt o) { T.add++; v += o.v; return *this; }
+  Cnt& operator-=(Cnt o) { T.add++; v -= o.v; return *this; }
+};
+inline Cnt operator+(Cnt a, Cnt b) { T.add++; return Cnt(a.v + b.v); }
+inline Cnt operator-(Cnt a, Cnt b) { T.add++; return Cnt(a.v - b.v); }
+inline Cnt operator-(Cnt a) { return Cnt(-a.v); }
+inline Cnt operator*(Cnt a, Cnt b) { T.mul++; return Cnt(a.v * b.v); }
+inline Cnt operator/(Cnt a, Cnt b) { T.div++; return Cnt(a.v / b.v); }
+inline Cnt sqrt(Cnt a) { T.sqrt++; return Cnt(std::sqrt(a.v)); }
+inline Cnt log1p(Cnt a) { T.log1p++; return Cnt(std::log1p(a.v)); }
+
+template <class F>
+void run(const char* name, const double* theta, const double* y) {
+  Cnt th_src[F::M], yy[F::D], dy[F::D], kb[F::D], yb[F::D], thb[F::M];
+  for (int j = 0; j < F::M; ++j) { th_src[j] = Cnt(theta[j]); thb[j] = Cnt(0); }
+  for (int c = 0; c < F::D; ++c) { yy[c] = Cnt(y[c]); kb[c] = Cnt(0.1 * (c + 1)); }
+  typename F::template Theta<Cnt> th;
+  F::load(th, th_src);
+  T = Tally();
+  F::f(yy, th, dy);
+  Tally tf = T;
+  T = Tally();
+  F::vjp(yy, th, kb, yb, thb);
+  Tally tv = T;
+  std::printf("{\"field\": \"%s\", \"D\": %d, \"M\": %d, "
+              "\"f\": {\"add\": %ld, \"mul\": %ld, \"div\": %ld, \"sqrt\": %ld, \"log1p\": %ld}, "
+              "\"vjp\": {\"add\": %ld, \"mul\": %ld, \"div\": %ld, \"sqrt\": %ld, \"log1p\": %ld}}\n",
+              name, F::D, F::M, tf.add, tf.mul, tf.div, tf.sqrt, tf.log1p, tv.add, tv.mul, tv.div,
+              tv.sqrt, tv.log1p);
+}
+
+int main() {
+  const double nfw_th[5] = {1, 1, 0.1, 0.3, 0.03}, nfw_y[6] = {0.7, 0.2, 0.1, 0.1, 0.5, 0.05};
+  const double lor_th[3] = {10, 28, 8.0 / 3}, lor_y[3] = {1, 1, 1};
+  const double lv_th[4] = {1.5, 1, 3, 1}, lv_y[2] = {1, 1};
+  const double rob_th[3] = {0.04, 3e7, 1e4}, rob_y[3] = {0.9, 1e-5, 0.1};
+  run<gs::FNfwMiyamotoNagai>("nfw_mn", nfw_th, nfw_y);
+  run<gs::FLorenz63>("lorenz63", lor_th, lor_y);
+  run<gs::FLotkaVolterra>("lotka_volterra", lv_th, lv_y);
+  run<gs::FRobertson>("robertson", rob_th, rob_y);
+  return 0;
+}

@@ -1,0 +1,49 @@
+"""The per-step operation counts that bench.py divides by kernel time are re-derived here.
+
+Per accepted step of the Tsit5 replay adjoint (recompute stages k1..k6 from y_n, reverse sweep):
+  stage states Y_2..Y_6: sum_{i=2..6} (2i - 1) = 35 ops per component;
+  kb_i = h (b_i lam + G_i): 2 + 5 * 3 = 17;  lam += Yb_i: 6;  G_j += a_ij Yb_i: 30
+  => 88 d + 6 c_f + 6 c_v.
+Per attempted step of the forward solve (k1 carried):
+  stages 35, y_new 13, error 14, scale 2, quotient 1, square-accumulate 2 per component,
+  plus mean, sqrt, pow, safety factor, h update (5) => 67 d + 6 c_f + 5.
+c_f and c_v are the op counts (add/sub, mul, div, sqrt, log1p; an FMA counts as two) of the
+field's f and vector-Jacobian product as written in csrc/gs_fields.cuh, tallied by compiling that
+header with a counting scalar (tests/flop_counter.cpp)."""
+import json
+import os
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def counts(tmp_path_factory):
+    exe = str(tmp_path_factory.mktemp("fc") / "flop_counter")
+    subprocess.run(["g++", "-std=c++17", "-O1", "-Wno-unknown-pragmas",
+                    "-I" + os.path.join(ROOT, "differentiable_adaptive_ode_b200", "csrc"),
+                    "-o", exe, os.path.join(ROOT, "tests", "flop_counter.cpp")], check=True)
+    out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout
+    return {r["field"]: r for r in map(json.loads, out.splitlines())}
+
+
+def ops(t):
+    return t["add"] + t["mul"] + t["div"] + t["sqrt"] + t["log1p"]
+
+
+def test_bench_constants_match_counts(counts):
+    import bench
+    c = counts["nfw_mn"]
+    D = c["D"]
+    adj = 88 * D + 6 * ops(c["f"]) + 6 * ops(c["vjp"])
+    fwd = 67 * D + 6 * ops(c["f"]) + 5
+    assert bench.FLOPS_ADJOINT_STEP["nfw_mn"] == adj
+    assert bench.FLOPS_FORWARD_ATTEMPT["nfw_mn"] == fwd
+
+
+def test_field_counts_are_plausible(counts):
+    # Lorenz f: sigma (y - x), x (rho - z) - y, x y - beta z -> 4 add/sub + 4 mul
+    assert ops(counts["lorenz63"]["f"]) == 8
+    assert counts["nfw_mn"]["f"]["log1p"] == 1 and counts["nfw_mn"]["f"]["sqrt"] == 3

@@ -1,0 +1,201 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle on the same seeded
+inputs.
+
+Bars: final states within relative 1e-9 (fp64) / 1e-4 (fp32) on trajectories whose accepted-step
+counts agree, counts identical on >= 99.9 % of trajectories, replay gradients on a shared recorded
+mesh within relative 1e-8 (fp64) / 1e-3 (fp32), per trajectory (per ensemble for a shared theta).
+Relative errors use max(||reference||_inf, atol) (states) or max(||reference||_inf, 1e-300)
+(gradients) as the denominator.  The method: "gradsolve: fast exact gradients for ODE ensembles
+on GPUs" §2.1 (solve), §3 (record, replay, gradient with the mesh held fixed).
+"""
+import numpy as np
+import pytest
+
+import gpu_util as U
+from differentiable_adaptive_ode_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+STATE_TOL = {np.float64: 1e-9, np.float32: 1e-4}
+GRAD_TOL = {np.float64: 1e-8, np.float32: 1e-3}
+COUNT_FRAC = 0.999
+
+# small ensembles: several 128-lane blocks plus a ragged tail
+SMALL = [("lotka_volterra", 300), ("lorenz63", 300), ("robertson", 200), ("nfw_mn", 300),
+         ("nfw_mn_f32", 300)]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from differentiable_adaptive_ode_b200 import gradsolve
+    gradsolve.lib()
+
+
+def _oracle_solve(orc, w, keep_record=False):
+    return orc.solve(w.field, w.method, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol, dtype=w.dtype,
+                     theta_shared=w.theta_shared, keep_record=keep_record, nthreads=8)
+
+
+def _check_states(w, gpu, ref):
+    same = gpu["S"] == ref["S"]
+    dS = np.abs(gpu["S"].astype(int) - ref["S"].astype(int))
+    err_all = U.rel_rows(gpu["y1"], ref["y1"], w.atol)
+    print("%s: identical counts %.4f, max |dS| %d, max rel state err %.3g (identical) %.3g (all)"
+          % (w.name, same.mean(), dS.max(), err_all[same].max() if same.any() else -1,
+             err_all.max()))
+    if w.dtype == np.float64:
+        assert same.mean() >= COUNT_FRAC, (w.name, np.flatnonzero(~same)[:10])
+    else:
+        # fp32: the accept test compares an error estimate formed by cancellation; rounding
+        # differences between the two sides move it by ~1e-3 relative, so a decision near
+        # err = 1 can flip.  Counts are held to |dS| <= 3 and states on every trajectory to the
+        # fp32 state bar times 10 (trajectories on different meshes differ by ~rtol).
+        assert np.mean(dS <= 3) >= COUNT_FRAC, (w.name, dS.max())
+        assert err_all.max() <= 10 * STATE_TOL[w.dtype], (w.name, err_all.max())
+    err = err_all[same]
+    assert err.max() <= STATE_TOL[w.dtype], (w.name, err.max(), np.argmax(err))
+
+
+@pytest.mark.parametrize("name,N", SMALL)
+def test_forward_parity(orc, name, N):
+    w = U.small(name, N)
+    gpu = U.forward(w)
+    ref = _oracle_solve(orc, w)
+    assert np.all(gpu["status"] == 0) and np.all(ref["status"] == 0)
+    _check_states(w, gpu, ref)
+    same = gpu["S"] == ref["S"]
+    assert np.array_equal(gpu["rejected"][same], ref["rejected"][same]) or w.dtype == np.float32
+
+
+@pytest.mark.parametrize("name,N", SMALL)
+def test_record_parity_and_replay(orc, name, N):
+    w = U.small(name, N)
+    rec, out = U.record(w)
+    ex = U.export_padded(w, rec)
+    ref = _oracle_solve(orc, w, keep_record=True)
+    assert np.all(out["status"] == 0)
+    gpu = dict(S=ex["S"], y1=out["y1"])
+    _check_states(w, gpu, ref)
+    # the record agrees with the oracle's record step by step where the counts agree
+    same = np.flatnonzero(ex["S"] == ref["S"])
+    for k in same[:50]:
+        S = ex["S"][k]
+        hr = U.rel_rows(ex["H"][k, :S, None], ref["H"][k, :S, None], 1e-300)
+        assert hr.max() <= 1e4 * STATE_TOL[w.dtype], (k, hr.max())
+        assert np.array_equal(ex["T"][k, 0], ref["T"][k, 0])
+    # the forward-only kernel and the record kernel take identical steps
+    fw = U.forward(w)
+    assert np.array_equal(fw["S"], ex["S"]) and np.array_equal(fw["y1"], out["y1"])
+    # replaying the GPU mesh in the oracle reproduces the GPU's final state
+    yrep = orc.replay(w.field, w.method, w.theta, w.y0, ex["H"], ex["S"], dtype=w.dtype,
+                      theta_shared=w.theta_shared)
+    err = U.rel_rows(out["y1"], yrep, w.atol)
+    assert err.max() <= STATE_TOL[w.dtype], err.max()
+    # recorded states are the states at the start of each step: y_0 is the initial state
+    assert np.array_equal(ex["Y"][:, 0, :].astype(w.dtype), w.y0.astype(w.dtype))
+
+
+@pytest.mark.parametrize("name,N", SMALL)
+def test_gradient_parity_on_shared_mesh(orc, name, N):
+    w = U.small(name, N)
+    rec, out = U.record(w)
+    ex = U.export_padded(w, rec)
+    lam = np.random.default_rng(1).normal(size=(w.N, w.d))
+    gy, gt = U.replay_grad(w, rec, lam)
+    ry, rt = orc.replay_grad(w.field, w.method, w.theta, w.y0, ex["H"], ex["S"], lam,
+                             dtype=w.dtype, theta_shared=w.theta_shared, nthreads=8)
+    tol = GRAD_TOL[w.dtype]
+    assert U.rel_rows(gy, ry, 1e-300).max() <= tol
+    assert U.rel_rows(gt, rt, 1e-300).max() <= tol
+
+
+@pytest.mark.parametrize("name,N", [("lorenz63", 200), ("robertson", 100), ("nfw_mn", 200)])
+def test_gradient_on_imported_oracle_record(orc, name, N):
+    w = U.small(name, N)
+    ref = _oracle_solve(orc, w, keep_record=True)
+    rec = U.import_record(w, ref["S"], ref["T"], ref["H"], ref["Y"])
+    lam = np.random.default_rng(2).normal(size=(w.N, w.d))
+    gy, gt = U.replay_grad(w, rec, lam)
+    ry, rt = orc.replay_grad(w.field, w.method, w.theta, w.y0, ref["H"], ref["S"], lam,
+                             nthreads=8)
+    assert U.rel_rows(gy, ry, 1e-300).max() <= 1e-8
+    assert U.rel_rows(gt, rt, 1e-300).max() <= 1e-8
+
+
+@pytest.mark.parametrize("method", ["tsit5", "ros34pw2"])
+def test_linear_field_both_methods(orc, method):
+    rng = np.random.default_rng(9)
+    N = 160
+    A = rng.normal(size=(N, 3, 3)) * 0.5 - 1.5 * np.eye(3)[None]
+    y0 = rng.normal(size=(N, 3))
+    w = W.Workload("linear3", "linear3", method, np.float64, N, 3, 9, False, A.reshape(N, 9), y0,
+                   0.0, 3.0, 1e-7, 1e-9, 0)
+    rec, out = U.record(w)
+    ex = U.export_padded(w, rec)
+    ref = _oracle_solve(orc, w)
+    _check_states(w, dict(S=ex["S"], y1=out["y1"]), ref)
+    lam = rng.normal(size=(N, 3))
+    gy, gt = U.replay_grad(w, rec, lam)
+    ry, rt = orc.replay_grad("linear3", method, w.theta, w.y0, ex["H"], ex["S"], lam)
+    assert U.rel_rows(gy, ry, 1e-300).max() <= 1e-8
+    assert U.rel_rows(gt, rt, 1e-300).max() <= 1e-8
+
+
+@pytest.mark.parametrize("name", ["nfw_mn", "lotka_volterra"])
+def test_shared_theta_reduction(orc, name):
+    w = U.small(name, 700)
+    w.theta_shared = True
+    w.theta = w.theta[0].copy()
+    rec, out = U.record(w)
+    ex = U.export_padded(w, rec)
+    lam = np.random.default_rng(3).normal(size=(w.N, w.d))
+    gy, gt = U.replay_grad(w, rec, lam)
+    ry, rt = orc.replay_grad(w.field, w.method, w.theta, w.y0, ex["H"], ex["S"], lam,
+                             theta_shared=True, nthreads=8)
+    assert gt.shape == (w.m,)
+    assert np.max(np.abs(gt - rt.sum(0))) <= 1e-8 * np.max(np.abs(rt.sum(0)))
+    assert U.rel_rows(gy, ry, 1e-300).max() <= 1e-8
+    # deterministic: a second call is bitwise identical
+    gy2, gt2 = U.replay_grad(w, rec, lam)
+    assert np.array_equal(gt, gt2) and np.array_equal(gy, gy2)
+
+
+def test_gradient_at_other_theta_on_fixed_mesh(orc):
+    # one record made at theta0 serves a gradient at theta on the same mesh ([GS] §3: the
+    # derivative of Psi(theta; sg[R(theta0)])): forward replay at theta, then the backward sweep
+    import torch
+    w = U.small("lorenz63", 200)
+    rec, out = U.record(w)
+    ex = U.export_padded(w, rec)
+    th2 = w.theta * 1.01
+    y1 = torch.empty((w.N, w.d), dtype=torch.float64, device="cuda")
+    from differentiable_adaptive_ode_b200 import gradsolve as G
+    G.gs_replay_forward(rec, U.dev(th2, torch.float64), U.dev(w.y0, torch.float64), y1)
+    yrep = orc.replay(w.field, w.method, th2, w.y0, ex["H"], ex["S"])
+    assert U.rel_rows(y1.cpu().numpy(), yrep, w.atol).max() <= 1e-9
+    lam = np.random.default_rng(4).normal(size=(w.N, w.d))
+    gy, gt = U.replay_grad(w, rec, lam, theta=th2)
+    ry, rt = orc.replay_grad(w.field, w.method, th2, w.y0, ex["H"], ex["S"], lam, nthreads=8)
+    assert U.rel_rows(gt, rt, 1e-300).max() <= 1e-8
+    assert U.rel_rows(gy, ry, 1e-300).max() <= 1e-8
+    # replaying at theta0 restores the record's own states: the gradient at theta0 again
+    G.gs_replay_forward(rec, U.dev(w.theta, torch.float64), U.dev(w.y0, torch.float64), y1)
+    assert U.rel_rows(y1.cpu().numpy(), out["y1"], w.atol).max() <= 1e-13
+    gy0, gt0 = U.replay_grad(w, rec, lam)
+    ry0, rt0 = orc.replay_grad(w.field, w.method, w.theta, w.y0, ex["H"], ex["S"], lam)
+    assert U.rel_rows(gt0, rt0, 1e-300).max() <= 1e-8
+
+
+def test_loss_gradient_end_to_end(orc):
+    # L = sum |y1 - target|^2 on the Lorenz benchmark ensemble: the whole chain
+    w = U.small("lorenz63", 256)
+    rec, out = U.record(w)
+    ex = U.export_padded(w, rec)
+    lam = W.loss_cotangent(w, out["y1"], w.target)
+    gy, gt = U.replay_grad(w, rec, lam)
+    ry, rt = orc.replay_grad(w.field, w.method, w.theta, w.y0, ex["H"], ex["S"], lam, nthreads=8)
+    assert U.rel_rows(gt, rt, 1e-300).max() <= 1e-8
+    assert U.rel_rows(gy, ry, 1e-300).max() <= 1e-8
