@@ -31,8 +31,8 @@ UNIT = "traj/s"
 # mul, fma = 2, div, sqrt, log1p each counted as one operation), and per attempted step of the
 # forward solve: counted from the definitions of the Tsit5 replay step, its reverse sweep and the
 # field's f and vector-Jacobian product (tests/test_flop_counts.py re-derives these numbers).
-FLOPS_ADJOINT_STEP = {"nfw_mn": 1386}
-FLOPS_FORWARD_ATTEMPT = {"nfw_mn": 593}
+FLOPS_ADJOINT_STEP = {"nfw_mn": 1416}
+FLOPS_FORWARD_ATTEMPT = {"nfw_mn": 611}
 # FP64 peak: 148 SMs x 64 FP64 FMA lanes/SM/clk x 2 flop x clock (1965 MHz max) = 37.2 TFLOP/s,
 # the datasheet FP64 figure of B200; the same formula at the measured SM clock is reported too.
 SMS, FP64_LANES = 148, 64

@@ -15,6 +15,7 @@
 
 #include "gradsolve_b200.h"
 #include "gs_kernels.cuh"
+#include "gs_mlp.cuh"
 
 namespace {
 
@@ -48,7 +49,7 @@ bool field_info(int field, FieldInfo* fi) {
   switch (field) {
     case GS_LOTKA_VOLTERRA: *fi = {2, 4, true, false}; return true;
     case GS_LORENZ63: *fi = {3, 3, true, false}; return true;
-    case GS_MLP_4_32_32_4: *fi = {4, 1348, false, false}; return true;  // not built yet
+    case GS_MLP_4_32_32_4: *fi = {4, 1348, true, false}; return true;
     case GS_ROBERTSON: *fi = {3, 3, false, true}; return true;
     case GS_NFW_MN: *fi = {6, 5, true, false}; return true;
     case GS_LINEAR: *fi = {3, 9, true, true}; return true;
@@ -71,6 +72,8 @@ gs_status check_system(const gs_system* sys) {
     return fail(GS_ERR_UNSUPPORTED, "field %d is not built for method %d", sys->field, sys->method);
   if (sys->theta_shared != 0 && sys->theta_shared != 1)
     return fail(GS_ERR_INVALID_ARG, "theta_shared must be 0 or 1");
+  if (sys->field == GS_MLP_4_32_32_4 && !sys->theta_shared)
+    return fail(GS_ERR_UNSUPPORTED, "the MLP field takes one weight vector shared by the ensemble");
   return GS_OK;
 }
 
@@ -173,6 +176,13 @@ struct gs_record {
   long long* tiles = nullptr;  // scan scratch (tile totals) + grand totals
   int* counters = nullptr;     // [0] queue [1] chunk count [2] overflow [3] max S [4] max status
   int* host = nullptr;         // pinned mirror of counters, then offsets[N] at host+8
+  // visiting order of the replay kernels (longest records first) and its counting-sort scratch
+  int* perm = nullptr;
+  int64_t perm_cap = 0;
+  int* bins = nullptr;          // [nb] counts, then [nb] cursors
+  long long* binoff = nullptr;  // [nb + 1]
+  long long* btiles = nullptr;
+  int64_t bins_cap = 0;
   // scratch of the replay calls (grown on demand; calls on one record are stream-ordered)
   void* red_scratch = nullptr;   // per-trajectory theta-bar [N][m] for a shared theta
   void* red_partials = nullptr;  // block partials of the reduction
@@ -238,6 +248,38 @@ gs_status scan_counts(const int* S, int N, int C, long long* out, long long* til
   return GS_OK;
 }
 
+// perm = trajectories by decreasing S (needs r->nsteps, r->max_steps).
+gs_status build_perm(gs_record* r, cudaStream_t s) {
+  const int64_t N = r->N;
+  if (N <= 0) return GS_OK;
+  if (r->perm_cap < N) {
+    free_ptr(r->perm);
+    r->perm = nullptr;
+    r->perm_cap = 0;
+    GS_CUDA(cudaMalloc(&r->perm, N * sizeof(int)));
+    r->perm_cap = N;
+  }
+  const int64_t nb = (int64_t)r->max_steps + 1;
+  if (r->bins_cap < nb) {
+    free_ptr(r->bins); free_ptr(r->binoff); free_ptr(r->btiles);
+    r->bins = nullptr; r->binoff = r->btiles = nullptr;
+    r->bins_cap = 0;
+    GS_CUDA(cudaMalloc(&r->bins, 2 * nb * sizeof(int)));
+    GS_CUDA(cudaMalloc(&r->binoff, (nb + 1) * sizeof(long long)));
+    GS_CUDA(cudaMalloc(&r->btiles, (nb / gs::SCAN_BLOCK + 3) * sizeof(long long)));
+    r->bins_cap = nb;
+  }
+  GS_CUDA(cudaMemsetAsync(r->bins, 0, 2 * nb * sizeof(int), s));
+  const int grid = (int)((N + 255) / 256);
+  gs::k_bin_count<<<grid, 256, 0, s>>>(r->nsteps, (int)N, r->max_steps, r->bins);
+  gs_status st = scan_counts<0>(r->bins, (int)nb, 1, r->binoff, r->btiles, s);
+  if (st != GS_OK) return st;
+  gs::k_bin_scatter<<<grid, 256, 0, s>>>(r->nsteps, (int)N, r->max_steps, r->binoff,
+                                         r->bins + nb, r->perm);
+  GS_CUDA(cudaGetLastError());
+  return GS_OK;
+}
+
 // ------------------------------------------------------------------------------------------------
 // Typed launchers.
 // ------------------------------------------------------------------------------------------------
@@ -271,26 +313,44 @@ gs_status launch_solve(const SolveCall& c) {
   p.nrejected = c.nrejected;
   p.status = c.status;
   p.queue = c.queue;
-  if (c.rec) {
-    using L = gs::RecLayout<F, R>;
-    p.pool = static_cast<R*>(c.rec->pool);
-    p.chunk_traj = c.rec->chunk_traj;
-    p.chunk_seq = c.rec->chunk_seq;
-    p.pool_chunks = (int)c.rec->pool_chunks;
-    p.chunk_count = c.rec->counters + 1;
-    p.overflow = c.rec->counters + 2;
-    const size_t smem = (size_t)(BLOCK / 32) * 32 * L::STAGE_STRIDE * sizeof(R);
-    auto kern = gs::k_solve<F, R, METHOD, true>;
-    GS_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    const int grid = persistent_grid(kern, smem, c.N);
-    kern<<<grid, BLOCK, smem, c.stream>>>(p);
+  if constexpr (std::is_same_v<F, gs::FMlpWarp>) {
+    if (c.rec) {
+      p.pool = static_cast<R*>(c.rec->pool);
+      p.chunk_traj = c.rec->chunk_traj;
+      p.chunk_seq = c.rec->chunk_seq;
+      p.pool_chunks = (int)c.rec->pool_chunks;
+      p.chunk_count = c.rec->counters + 1;
+      p.overflow = c.rec->counters + 2;
+      auto kern = gs::k_solve_mlp<R, true>;
+      kern<<<persistent_grid(kern, 0, c.N * 32), BLOCK, 0, c.stream>>>(p);
+    } else {
+      auto kern = gs::k_solve_mlp<R, false>;
+      kern<<<persistent_grid(kern, 0, c.N * 32), BLOCK, 0, c.stream>>>(p);
+    }
+    GS_CUDA(cudaGetLastError());
+    return GS_OK;
   } else {
-    auto kern = gs::k_solve<F, R, METHOD, false>;
-    const int grid = persistent_grid(kern, 0, c.N);
-    kern<<<grid, BLOCK, 0, c.stream>>>(p);
+    if (c.rec) {
+      using L = gs::RecLayout<F, R>;
+      p.pool = static_cast<R*>(c.rec->pool);
+      p.chunk_traj = c.rec->chunk_traj;
+      p.chunk_seq = c.rec->chunk_seq;
+      p.pool_chunks = (int)c.rec->pool_chunks;
+      p.chunk_count = c.rec->counters + 1;
+      p.overflow = c.rec->counters + 2;
+      const size_t smem = (size_t)(BLOCK / 32) * 32 * L::STAGE_STRIDE * sizeof(R);
+      auto kern = gs::k_solve<F, R, METHOD, true>;
+      GS_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+      const int grid = persistent_grid(kern, smem, c.N);
+      kern<<<grid, BLOCK, smem, c.stream>>>(p);
+    } else {
+      auto kern = gs::k_solve<F, R, METHOD, false>;
+      const int grid = persistent_grid(kern, 0, c.N);
+      kern<<<grid, BLOCK, 0, c.stream>>>(p);
+    }
+    GS_CUDA(cudaGetLastError());
+    return GS_OK;
   }
-  GS_CUDA(cudaGetLastError());
-  return GS_OK;
 }
 
 struct AdjCall {
@@ -305,6 +365,9 @@ struct AdjCall {
 
 template <class F, class R, int METHOD>
 gs_status launch_adjoint(const AdjCall& c) {
+  if constexpr (std::is_same_v<F, gs::FMlpWarp>) {
+    return fail(GS_ERR_UNSUPPORTED, "the MLP field has its own adjoint launcher");
+  } else {
   gs::AdjointParams<R> p{};
   const gs_record* r = c.rec;
   p.N = (int)r->N;
@@ -318,11 +381,13 @@ gs_status launch_adjoint(const AdjCall& c) {
   p.chunk_table = r->chunk_table;
   p.pool = static_cast<const R*>(r->pool);
   p.queue = c.queue;
+  p.perm = r->perm;
   auto kern = gs::k_adjoint<F, R, METHOD>;
   const int grid = persistent_grid(kern, 0, r->N);
   kern<<<grid, BLOCK, 0, c.stream>>>(p);
   GS_CUDA(cudaGetLastError());
   return GS_OK;
+  }
 }
 
 template <class F, class R>
@@ -350,6 +415,9 @@ gs_status dispatch(const gs_system& s, Fn&& fn) {
       case GS_LINEAR:
         return f64 ? fn.template operator()<FLinear3, double, M_TSIT5>()
                    : fn.template operator()<FLinear3, float, M_TSIT5>();
+      case GS_MLP_4_32_32_4:
+        return f64 ? fn.template operator()<FMlpWarp, double, M_TSIT5>()
+                   : fn.template operator()<FMlpWarp, float, M_TSIT5>();
       default: break;
     }
   } else {
@@ -384,6 +452,49 @@ long long attempts_of(const gs_options* opt) {
 }
 
 }  // namespace
+
+// Replay adjoint of the MLP field: one warp per trajectory, per-warp weight-cotangent partials,
+// then a fixed-order sum over warps.
+static gs_status replay_grad_mlp(const gs_record* rec, const void* theta, const void* dL_dy1,
+                          void* dL_dtheta, void* dL_dy0, cudaStream_t s) {
+  gs_record* r = const_cast<gs_record*>(rec);
+  auto run = [&](auto zero) -> gs_status {
+    using R = decltype(zero);
+    auto kern = gs::k_adjoint_mlp<R>;
+    const int grid = persistent_grid(kern, 0, rec->N * 32);
+    const int nwarps = grid * (BLOCK / 32);
+    R* partials = nullptr;
+    if (dL_dtheta) {
+      const size_t need = (size_t)nwarps * gs::MLP_M * sizeof(R);
+      if (r->part_bytes < need) {
+        free_ptr(r->red_partials);
+        r->red_partials = nullptr;
+        r->part_bytes = 0;
+        GS_CUDA(cudaMalloc(&r->red_partials, need));
+        r->part_bytes = need;
+      }
+      partials = static_cast<R*>(r->red_partials);
+    }
+    gs::MlpAdjParams<R> p{};
+    p.N = (int)rec->N;
+    p.theta = static_cast<const R*>(theta);
+    p.dL_dy1 = static_cast<const R*>(dL_dy1);
+    p.dL_dy0 = static_cast<R*>(dL_dy0);
+    p.partials = partials;
+    p.nsteps = rec->nsteps;
+    p.choff = rec->choff;
+    p.chunk_table = rec->chunk_table;
+    p.pool = static_cast<const R*>(rec->pool);
+    p.perm = rec->perm;
+    kern<<<grid, BLOCK, 0, s>>>(p);
+    if (partials)
+      gs::k_reduce_partials<R><<<(gs::MLP_M + 255) / 256, 256, 0, s>>>(partials, nwarps, gs::MLP_M,
+                                                                    static_cast<R*>(dL_dtheta));
+    GS_CUDA(cudaGetLastError());
+    return GS_OK;
+  };
+  return rec->sys.dtype == GS_F64 ? run(0.0) : run(0.0f);
+}
 
 extern "C" {
 
@@ -506,6 +617,7 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
     gs::k_chunk_table<<<(int)((r->nchunks + 255) / 256), 256, 0, s>>>(
         r->chunk_traj, r->chunk_seq, (int)r->nchunks, r->choff, r->chunk_table);
   if (cudaGetLastError() != cudaSuccess) return bail(fail(GS_ERR_CUDA, "chunk table launch failed"));
+  if ((st = build_perm(r, s)) != GS_OK) return bail(st);
   *rec = r;
   if (r->host[4] != 0) {
     fail(GS_ERR_TRAJ_FAILED, "some trajectories did not reach t1 (max status %d)", r->host[4]);
@@ -523,6 +635,7 @@ gs_status gs_replay_grad(const gs_record* rec, const void* theta, const void* dL
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int M = rec->sys.m;
   const int64_t N = rec->N;
+  if (rec->sys.field == GS_MLP_4_32_32_4) return replay_grad_mlp(rec, theta, dL_dy1, dL_dtheta, dL_dy0, s);
   const bool shared = rec->sys.theta_shared && dL_dtheta;
   const int per_block = 4096;
   const int nred = (int)((N + per_block - 1) / per_block);
@@ -583,6 +696,22 @@ gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, v
   GS_CUDA(take_counter(s, &queue));
   gs_status st = dispatch(rec->sys, [&]<class F, class R, int METHOD>() {
     gs::ReplayParams<R> p{};
+    if constexpr (std::is_same_v<F, gs::FMlpWarp>) {
+      p.N = (int)rec->N;
+      p.theta = static_cast<const R*>(theta);
+      p.y0 = static_cast<const R*>(y0);
+      p.y1 = static_cast<R*>(y1buf);
+      p.nsteps = rec->nsteps;
+      p.choff = rec->choff;
+      p.chunk_table = rec->chunk_table;
+      p.pool = static_cast<R*>(rec->pool);
+      p.queue = queue;
+      p.perm = rec->perm;
+      auto kern = gs::k_replay_forward_mlp<R>;
+      kern<<<persistent_grid(kern, 0, rec->N * 32), BLOCK, 0, s>>>(p);
+      GS_CUDA(cudaGetLastError());
+      return GS_OK;
+    } else {
     p.N = (int)rec->N;
     p.theta = static_cast<const R*>(theta);
     p.theta_stride = rec->sys.theta_shared ? 0 : F::M;
@@ -593,11 +722,13 @@ gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, v
     p.chunk_table = rec->chunk_table;
     p.pool = static_cast<R*>(rec->pool);
     p.queue = queue;
+    p.perm = rec->perm;
     auto kern = gs::k_replay_forward<F, R, METHOD>;
     const int grid = persistent_grid(kern, 0, rec->N);
     kern<<<grid, BLOCK, 0, s>>>(p);
     GS_CUDA(cudaGetLastError());
     return GS_OK;
+    }
   });
   return st;
 }
@@ -710,6 +841,7 @@ gs_status gs_record_import(const gs_system* sys, int64_t N, const int32_t* nstep
                                                static_cast<const float*>(Y));
       if (cudaGetLastError() != cudaSuccess) return bail(fail(GS_ERR_CUDA, "import launch failed"));
     }
+    if ((st = build_perm(r, s)) != GS_OK) return bail(st);
   }
   *rec = r;
   return GS_OK;
@@ -725,6 +857,7 @@ void gs_record_destroy(gs_record* r) {
   free_ptr(r->nsteps); free_ptr(r->status); free_ptr(r->offsets); free_ptr(r->choff);
   free_ptr(r->tiles); free_ptr(r->counters);
   free_ptr(r->red_scratch); free_ptr(r->red_partials); free_ptr(r->y1_scratch);
+  free_ptr(r->perm); free_ptr(r->bins); free_ptr(r->binoff); free_ptr(r->btiles);
   if (r->host) cudaFreeHost(r->host);
   cudaSetDevice(prev);
   delete r;

@@ -21,7 +21,10 @@
 #include <cuda_runtime.h>
 #define GS_HD __host__ __device__ __forceinline__
 #else
+#include <cmath>
 #define GS_HD inline
+inline double rsqrt(double x) { return 1.0 / std::sqrt(x); }
+inline float rsqrt(float x) { return 1.0f / std::sqrt(x); }
 #endif
 
 namespace gs {
@@ -182,63 +185,61 @@ struct FNfwMiyamotoNagai {
     t.irs = R(1) / t.rs;
     t.b2 = t.b * t.b;
   }
-  template <class R> GS_HD static void f(const R* y, const Theta<R>& t, R* dy) {
+  // Quantities of f shared with the VJP; one division, three reciprocal square roots, one log1p.
+  template <class R> struct Inter { R R2, r, ir, L, isr, gN, iB, apB, iD, gM; };
+  template <class R> GS_HD static void inter(const R* y, const Theta<R>& t, Inter<R>& I) {
     const R x = y[0], yy = y[1], z = y[2];
-    const R R2 = x * x + yy * yy;
-    const R r2 = R2 + z * z;
-    const R r = sqrt(r2);
-    const R L = log1p(r * t.irs);
-    const R ir2 = R(1) / r2;
-    const R gN = t.Mh * ir2 * (L / r - R(1) / (t.rs + r));
-    const R B = sqrt(z * z + t.b2);
-    const R apB = t.a + B;
-    const R D2 = R2 + apB * apB;
-    const R gM = t.Md / (D2 * sqrt(D2));
-    const R g = gN + gM;
+    I.R2 = x * x + yy * yy;
+    const R r2 = I.R2 + z * z;
+    I.ir = rsqrt(r2);
+    I.r = r2 * I.ir;
+    I.L = log1p(I.r * t.irs);
+    I.isr = R(1) / (t.rs + I.r);
+    I.gN = t.Mh * (I.ir * I.ir) * (I.L * I.ir - I.isr);
+    const R B2 = z * z + t.b2;
+    I.iB = rsqrt(B2);
+    I.apB = t.a + B2 * I.iB;
+    I.iD = rsqrt(I.R2 + I.apB * I.apB);
+    I.gM = t.Md * (I.iD * I.iD * I.iD);
+  }
+  template <class R> GS_HD static void f(const R* y, const Theta<R>& t, R* dy) {
+    Inter<R> I;
+    inter(y, t, I);
+    const R g = I.gN + I.gM;
     dy[0] = y[3];
     dy[1] = y[4];
     dy[2] = y[5];
-    dy[3] = -g * x;
-    dy[4] = -g * yy;
-    dy[5] = -(gN + gM * apB / B) * z;
+    dy[3] = -g * y[0];
+    dy[4] = -g * y[1];
+    dy[5] = -(I.gN + I.gM * I.apB * I.iB) * y[2];
   }
   template <class R>
   GS_HD static void vjp(const R* y, const Theta<R>& t, const R* kb, R* yb, R* thb) {
+    Inter<R> I;
+    inter(y, t, I);
     const R x = y[0], yy = y[1], z = y[2];
     const R ux = kb[3], uy = kb[4], uz = kb[5];
-    const R R2 = x * x + yy * yy;
-    const R r2 = R2 + z * z;
-    const R r = sqrt(r2);
-    const R ir = R(1) / r;
-    const R L = log1p(r * t.irs);
-    const R ir2 = ir * ir;
-    const R isr = R(1) / (t.rs + r);
-    const R Lir = L * ir;
-    const R gN = t.Mh * ir2 * (Lir - isr);
-    const R gNp_r = t.Mh * ir2 * ir2 * (R(3) * isr - R(3) * Lir + r * isr * isr);   // gN'/r
-    const R B = sqrt(z * z + t.b2);
-    const R iB = R(1) / B;
-    const R apB = t.a + B;
-    const R q = apB * iB;
-    const R D2 = R2 + apB * apB;
-    const R iD2 = R(1) / D2;
-    const R gM = t.Md * iD2 * sqrt(iD2);
+    const R ir2 = I.ir * I.ir;
+    const R Lir = I.L * I.ir;
+    const R gNp_r = t.Mh * ir2 * ir2 * (R(3) * I.isr - R(3) * Lir + I.r * I.isr * I.isr);  // gN'/r
+    const R q = I.apB * I.iB;
+    const R iD2 = I.iD * I.iD;
     const R wz = z * q;
     const R xu = x * ux + yy * uy + z * uz;
     const R wu = x * ux + yy * uy + wz * uz;
-    const R c3 = R(3) * gM * iD2 * wu;
-    const R hz = q - t.a * z * z * iB * iB * iB;
-    yb[0] = -(gN * ux + gNp_r * xu * x) - (gM * ux - c3 * x);
-    yb[1] = -(gN * uy + gNp_r * xu * yy) - (gM * uy - c3 * yy);
-    yb[2] = -(gN * uz + gNp_r * xu * z) - (gM * hz * uz - c3 * wz);
+    const R c3 = R(3) * I.gM * iD2 * wu;
+    const R hz = q - t.a * z * z * I.iB * I.iB * I.iB;
+    yb[0] = -(I.gN * ux + gNp_r * xu * x) - (I.gM * ux - c3 * x);
+    yb[1] = -(I.gN * uy + gNp_r * xu * yy) - (I.gM * uy - c3 * yy);
+    yb[2] = -(I.gN * uz + gNp_r * xu * z) - (I.gM * hz * uz - c3 * wz);
     yb[3] = kb[0];
     yb[4] = kb[1];
     yb[5] = kb[2];
-    thb[0] -= ir2 * (Lir - isr) * xu;
-    thb[1] += t.Mh * ir * t.irs * isr * isr * xu;
-    thb[2] -= iD2 * sqrt(iD2) * wu;
-    thb[3] += apB * c3 - gM * z * iB * uz;
-    thb[4] += t.b * iB * (apB * c3 + gM * t.a * z * iB * iB * uz);
+    thb[0] -= ir2 * (Lir - I.isr) * xu;
+    thb[1] += t.Mh * I.ir * t.irs * I.isr * I.isr * xu;
+    thb[2] -= iD2 * I.iD * wu;
+    thb[3] += I.apB * c3 - I.gM * z * I.iB * uz;
+    thb[4] += t.b * I.iB * (I.apB * c3 + I.gM * t.a * z * I.iB * I.iB * uz);
   }
 };
 

@@ -117,8 +117,13 @@ __device__ R initial_step(const R (&y0)[F::D], const R (&f0)[F::D],
   return h;
 }
 
-template <int METHOD> struct MethodTag {};
 constexpr int M_TSIT5 = 0, M_ROS = 1;
+
+// Minimum resident 128-thread blocks per SM asked of the compiler (register cap 65536 / (128 b)).
+// Measured on B200 for the stellar field in double precision: the replay adjoint runs 13 % faster
+// at 3 blocks (168 registers, a few spilled) than unconstrained (2 blocks, 236 registers).
+template <class F, class R> struct Tune { static constexpr int adj_blocks = 1; };
+template <> struct Tune<FNfwMiyamotoNagai, double> { static constexpr int adj_blocks = 3; };
 
 template <class F, class R, int METHOD, bool REC>
 __global__ void __launch_bounds__(128) k_solve(SolveParams<R> p) {
@@ -308,10 +313,11 @@ struct AdjointParams {
   const int* chunk_table;
   const R* pool;
   int* queue;
+  const int* perm;          // visiting order (longest records first); nullable = identity
 };
 
 template <class F, class R, int METHOD>
-__global__ void __launch_bounds__(128) k_adjoint(AdjointParams<R> p) {
+__global__ void __launch_bounds__(128, Tune<F, R>::adj_blocks) k_adjoint(AdjointParams<R> p) {
   using L = RecLayout<F, R>;
   constexpr int D = F::D, M = F::M;
   int k = -1;
@@ -331,7 +337,7 @@ __global__ void __launch_bounds__(128) k_adjoint(AdjointParams<R> p) {
       const int id = warp_take(need, p.queue);
       if (need) {
         if (id < p.N) {
-          k = id;
+          k = p.perm ? p.perm[id] : id;
           F::load(th, p.theta + (size_t)p.theta_stride * k);
 #pragma unroll
           for (int c = 0; c < D; ++c) lam[c] = p.dL_dy1[(size_t)k * D + c];
@@ -385,6 +391,7 @@ struct ReplayParams {
   const int* chunk_table;
   R* pool;
   int* queue;
+  const int* perm;
 };
 
 template <class F, class R, int METHOD>
@@ -404,7 +411,7 @@ __global__ void __launch_bounds__(128) k_replay_forward(ReplayParams<R> p) {
       const int id = warp_take(need, p.queue);
       if (need) {
         if (id < p.N) {
-          k = id;
+          k = p.perm ? p.perm[id] : id;
           F::load(th, p.theta + (size_t)p.theta_stride * k);
 #pragma unroll
           for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
@@ -575,6 +582,22 @@ __global__ void k_import(R* pool, const long long* choff, const long long* offse
   for (int c = 0; c < D; ++c) e[2 + c] = Y[g * D + c];
 }
 
+// Visiting order for the replay kernels: trajectories sorted by decreasing record length
+// (counting sort on S; bin b holds S = smax - b), so that the work queue hands out the longest
+// records first and the tail of the launch is made of the shortest ones.
+__global__ void k_bin_count(const int* S, int N, int smax, int* bins) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < N) atomicAdd(&bins[smax - S[i]], 1);
+}
+__global__ void k_bin_scatter(const int* S, int N, int smax, const long long* binoff, int* cursor,
+                              int* perm) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < N) {
+    const int b = smax - S[i];
+    perm[binoff[b] + atomicAdd(&cursor[b], 1)] = i;
+  }
+}
+
 __global__ void k_iota(int* a, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) a[i] = i;
@@ -612,7 +635,7 @@ __global__ void __launch_bounds__(RED_BLOCK) k_reduce_theta(const R* part, int N
 
 template <class R>
 __global__ void k_reduce_partials(const R* partials, int nblocks, int M, R* out) {
-  for (int j = threadIdx.x; j < M; j += blockDim.x) {
+  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < M; j += gridDim.x * blockDim.x) {
     R s = R(0);
     for (int b = 0; b < nblocks; ++b) s += partials[(size_t)b * M + j];
     out[j] = s;

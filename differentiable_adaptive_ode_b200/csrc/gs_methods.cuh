@@ -134,7 +134,7 @@ __device__ __forceinline__ void tsit5_replay_step(const R (&y)[F::D], R h,
 // Reverse-mode step of the Tsit5 replay map y_{n+1} = y_n + h sum_{i<=6} b_i k_i with h fixed:
 // recompute the stages from the recorded y_n, then sweep them backwards.
 //   kb_i = h (b_i lam + sum_{j>i} a_ji Yb_j),  Yb_i = J_y(Y_i)^T kb_i,  thb += J_th(Y_i)^T kb_i,
-//   lam <- lam + sum_i Yb_i.
+//   lam <- lam + sum_i Yb_i.   (b_7 = 0, so the seventh stage never enters the replay map.)
 template <class F, class R>
 __device__ __forceinline__ void tsit5_adjoint_step(const R (&y)[F::D], R h,
                                                    const typename F::template Theta<R>& th,
@@ -158,29 +158,25 @@ __device__ __forceinline__ void tsit5_adjoint_step(const R (&y)[F::D], R h,
       if (i < 5) F::f(Y[i], th, k[i]);
     }
   }
-  R G[5][D];
-#pragma unroll
-  for (int i = 0; i < 5; ++i)
-#pragma unroll
-    for (int c = 0; c < D; ++c) G[i][c] = R(0);
+  // Reverse sweep.  Yb_j is kept for the stages j > i still to be visited, so that at every
+  // point only six stage vectors are live (the Y_i not yet consumed plus the Yb_j already made).
+  R Yb[6][D];
   R lnew[D];
 #pragma unroll
   for (int c = 0; c < D; ++c) lnew[c] = lam[c];
 #pragma unroll
   for (int i = 5; i >= 0; --i) {
-    R kb[D], Yb[D];
+    R kb[D];
 #pragma unroll
     for (int c = 0; c < D; ++c) {
-      const R g = (i < 5) ? G[i][c] : R(0);
+      R g = R(0);
+#pragma unroll
+      for (int j = i + 1; j < 6; ++j) g += ta<R>(j, i) * Yb[j][c];
       kb[c] = h * (tb<R>(i) * lam[c] + g);
     }
-    F::vjp(Y[i], th, kb, Yb, thb);
+    F::vjp(Y[i], th, kb, Yb[i], thb);
 #pragma unroll
-    for (int c = 0; c < D; ++c) {
-      lnew[c] += Yb[c];
-#pragma unroll
-      for (int j = 0; j < i; ++j) G[j][c] += ta<R>(i, j) * Yb[c];
-    }
+    for (int c = 0; c < D; ++c) lnew[c] += Yb[i][c];
   }
 #pragma unroll
   for (int c = 0; c < D; ++c) lam[c] = lnew[c];

@@ -22,6 +22,7 @@ inline Cnt operator*(Cnt a, Cnt b) { T.mul++; return Cnt(a.v * b.v); }
 inline Cnt operator/(Cnt a, Cnt b) { T.div++; return Cnt(a.v / b.v); }
 inline Cnt sqrt(Cnt a) { T.sqrt++; return Cnt(std::sqrt(a.v)); }
 inline Cnt log1p(Cnt a) { T.log1p++; return Cnt(std::log1p(a.v)); }
+inline Cnt rsqrt(Cnt a) { T.sqrt++; return Cnt(1.0 / std::sqrt(a.v)); }
 
 template <class F>
 void run(const char* name, const double* theta, const double* y) {

@@ -7,7 +7,7 @@ Per accepted step of the Tsit5 replay adjoint (recompute stages k1..k6 from y_n,
 Per attempted step of the forward solve (k1 carried):
   stages 35, y_new 13, error 14, scale 2, quotient 1, square-accumulate 2 per component,
   plus mean, sqrt, pow, safety factor, h update (5) => 67 d + 6 c_f + 5.
-c_f and c_v are the op counts (add/sub, mul, div, sqrt, log1p; an FMA counts as two) of the
+c_f and c_v are the op counts (add/sub, mul, div, sqrt or rsqrt, log1p; an FMA counts as two) of the
 field's f and vector-Jacobian product as written in csrc/gs_fields.cuh, tallied by compiling that
 header with a counting scalar (tests/flop_counter.cpp)."""
 import json
@@ -47,3 +47,4 @@ def test_field_counts_are_plausible(counts):
     # Lorenz f: sigma (y - x), x (rho - z) - y, x y - beta z -> 4 add/sub + 4 mul
     assert ops(counts["lorenz63"]["f"]) == 8
     assert counts["nfw_mn"]["f"]["log1p"] == 1 and counts["nfw_mn"]["f"]["sqrt"] == 3
+    assert counts["nfw_mn"]["f"]["div"] == 1
