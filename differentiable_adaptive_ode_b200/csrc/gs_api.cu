@@ -864,3 +864,115 @@ void gs_record_destroy(gs_record* r) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// gs_replay_grad_noalloc: the replay gradient with its scratch in a fixed device array, for
+// callers that cannot allocate device memory when they ask for a gradient.
+// Layout of the array: [0, 256) work counter; then theta-bar per trajectory [N][m]; then the
+// block partials [nred][m] of the shared-theta sum.
+// ------------------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GS_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+struct NoallocDevice {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+  unsigned char* ptr = nullptr;  // device address of g_noalloc_scratch on this device
+  int sms = 0;
+};
+NoallocDevice g_noalloc[MAX_DEVICES];
+
+// Once per device, with that device current: the device address of the array (host code may
+// not use the array's name as an address) and the SM count.
+gs_status noalloc_setup(NoallocDevice** out) {
+  int dev = 0;
+  GS_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= MAX_DEVICES) return fail(GS_ERR_CUDA, "device %d out of range", dev);
+  NoallocDevice& d = g_noalloc[dev];
+  std::call_once(d.once, [&]() {
+    d.err = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.ptr), g_noalloc_scratch);
+    if (d.err == cudaSuccess) d.err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  });
+  if (d.err != cudaSuccess)
+    return fail(GS_ERR_CUDA, "no-alloc scratch set-up failed on device %d: %s", dev,
+                cudaGetErrorString(d.err));
+  *out = &d;
+  return GS_OK;
+}
+
+template <class F, class R, int METHOD>
+gs_status noalloc_adjoint(const gs_record* r, const void* theta, const void* dL_dy1,
+                          void* dL_dtheta, void* dL_dy0, unsigned char* scratch, int sms,
+                          cudaStream_t s) {
+  if constexpr (std::is_same_v<F, gs::FMlpWarp>) {
+    return fail(GS_ERR_UNSUPPORTED, "gs_replay_grad_noalloc does not take the MLP field");
+  } else {
+    const bool shared = r->sys.theta_shared && dL_dtheta;
+    const int M = F::M;
+    const int64_t N = r->N;
+    const int per_block = 4096;
+    const int nred = (int)((N + per_block - 1) / per_block);
+    R* traj = reinterpret_cast<R*>(scratch + 256);
+    R* partials = traj + (size_t)N * M;
+    gs::AdjointParams<R> p{};
+    p.N = (int)N;
+    p.theta = static_cast<const R*>(theta);
+    p.theta_stride = r->sys.theta_shared ? 0 : M;
+    p.dL_dy1 = static_cast<const R*>(dL_dy1);
+    p.dL_dy0 = static_cast<R*>(dL_dy0);
+    p.dL_dtheta = shared ? traj : static_cast<R*>(dL_dtheta);
+    p.nsteps = r->nsteps;
+    p.choff = r->choff;
+    p.chunk_table = r->chunk_table;
+    p.pool = static_cast<const R*>(r->pool);
+    p.queue = reinterpret_cast<int*>(scratch);
+    p.perm = r->perm;
+    auto kern = gs::k_adjoint<F, R, METHOD>;
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, BLOCK, 0) != cudaSuccess || nb < 1)
+      nb = 1;
+    const long long grid =
+        std::max(1LL, std::min((long long)sms * nb, (long long)((N + BLOCK - 1) / BLOCK)));
+    GS_CUDA(cudaMemsetAsync(scratch, 0, sizeof(int), s));  // the counter starts at zero
+    kern<<<(int)grid, BLOCK, 0, s>>>(p);
+    if (shared) {
+      gs::k_reduce_theta<R><<<nred, gs::RED_BLOCK, 0, s>>>(traj, (int)N, M, per_block, partials);
+      gs::k_reduce_partials<R><<<1, 256, 0, s>>>(partials, nred, M, static_cast<R*>(dL_dtheta));
+    }
+    GS_CUDA(cudaGetLastError());
+    return GS_OK;
+  }
+}
+
+}  // namespace
+
+extern "C" gs_status gs_replay_grad_noalloc(const gs_record* rec, const void* theta,
+                                            const void* dL_dy1, void* dL_dtheta, void* dL_dy0,
+                                            void* stream) {
+  if (!rec) return fail(GS_ERR_INVALID_ARG, "record is NULL");
+  if (rec->N == 0) return GS_OK;
+  if (!theta || !dL_dy1) return fail(GS_ERR_INVALID_ARG, "theta and dL_dy1 must be non-NULL");
+  if (!dL_dtheta && !dL_dy0) return fail(GS_ERR_INVALID_ARG, "no output requested");
+  if (rec->sys.field == GS_MLP_4_32_32_4)
+    return fail(GS_ERR_UNSUPPORTED, "gs_replay_grad_noalloc does not take the MLP field");
+  const bool shared = rec->sys.theta_shared && dL_dtheta;
+  const size_t nred = (size_t)((rec->N + 4095) / 4096);
+  const size_t need = 256 + (shared ? ((size_t)rec->N + nred) * rec->sys.m * rec->rsz : 0);
+  if (need > GS_NOALLOC_SCRATCH_BYTES)
+    return fail(GS_ERR_CAPACITY,
+                "gs_replay_grad_noalloc needs %zu bytes of scratch for N=%lld, m=%d; its fixed "
+                "array holds %u bytes (use gs_replay_grad)",
+                need, (long long)rec->N, rec->sys.m, GS_NOALLOC_SCRATCH_BYTES);
+  NoallocDevice* d = nullptr;
+  gs_status st = noalloc_setup(&d);
+  if (st != GS_OK) return st;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != rec->device)
+    return fail(GS_ERR_INVALID_ARG, "record belongs to device %d, current is %d", rec->device, dev);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return dispatch(rec->sys, [&]<class F, class R, int METHOD>() {
+    return noalloc_adjoint<F, R, METHOD>(rec, theta, dL_dy1, dL_dtheta, dL_dy0, d->ptr, d->sms, s);
+  });
+}

@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "GS_OK", 1: "GS_ERR_INVALID_ARG", 2: "GS_ERR_CUDA", 3: "GS_ER
 
 # every entry point declared in include/gradsolve_b200.h
 EXPORTS = ("gs_solve_forward", "gs_solve_record", "gs_replay_grad", "gs_replay_forward",
-           "gs_record_info",
+           "gs_replay_grad_noalloc", "gs_record_info",
            "gs_record_export", "gs_record_import", "gs_record_destroy", "gs_last_error",
            "gs_version")
 
@@ -74,6 +74,7 @@ def lib():
                                       P(vp), vp, vp, vp]
         L.gs_replay_grad.argtypes = [vp, vp, vp, vp, vp, vp]
         L.gs_replay_forward.argtypes = [vp, vp, vp, vp, vp]
+        L.gs_replay_grad_noalloc.argtypes = [vp, vp, vp, vp, vp, vp]
         L.gs_record_info.argtypes = [vp, P(GsRecordInfo)]
         L.gs_record_export.argtypes = [vp, vp, vp, vp, vp, vp]
         L.gs_record_import.argtypes = [P(GsSystem), i64, vp, vp, vp, vp, P(vp), vp]
@@ -82,7 +83,7 @@ def lib():
         L.gs_last_error.restype = C.c_char_p
         L.gs_version.restype = C.c_char_p
         for name in ("gs_solve_forward", "gs_solve_record", "gs_replay_grad", "gs_replay_forward",
-                     "gs_record_info",
+                     "gs_replay_grad_noalloc", "gs_record_info",
                      "gs_record_export", "gs_record_import"):
             getattr(L, name).restype = C.c_int
         _lib = L
@@ -173,6 +174,14 @@ def gs_replay_grad(rec, theta, dL_dy1, dL_dtheta=None, dL_dy0=None, stream=None)
     """Replay gradient over the recorded mesh: fills dL_dtheta ([N, m] or [m]) and/or dL_dy0."""
     _check(lib().gs_replay_grad(rec.handle, _ptr(theta), _ptr(dL_dy1), _ptr(dL_dtheta),
                                 _ptr(dL_dy0), _stream(stream)))
+
+
+def gs_replay_grad_noalloc(rec, theta, dL_dy1, dL_dtheta=None, dL_dy0=None, stream=None):
+    """gs_replay_grad without any device allocation: for callers that may not allocate when they
+    ask for a gradient (e.g. inside CUDA-graph capture); its scratch is a fixed 8 MiB array in the
+    library, shared by all calls, so calls must not overlap on the GPU."""
+    _check(lib().gs_replay_grad_noalloc(rec.handle, _ptr(theta), _ptr(dL_dy1), _ptr(dL_dtheta),
+                                        _ptr(dL_dy0), _stream(stream)))
 
 
 def gs_replay_forward(rec, theta, y0, y1=None, stream=None):

@@ -140,6 +140,27 @@ gs_status gs_replay_grad(const gs_record* rec, const void* theta, const void* dL
 gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, void* y1,
                             void* stream);
 
+/* Replay gradient that allocates no device memory.  The paper has no counterpart: this entry
+ * point exists for callers that must not allocate at the moment they ask for a gradient -- code
+ * that runs while a stream is being captured into a CUDA graph (allocation is not a capturable
+ * operation), code living under an allocator that forbids driver allocations, or a time-critical
+ * loop in which cudaMalloc/cudaFree would synchronise the device.  gs_replay_grad, by contrast,
+ * may allocate on its first use (work counters, and for a shared theta its per-trajectory
+ * scratch).
+ * Same arguments and result as gs_replay_grad, for every field except GS_MLP_4_32_32_4
+ * (GS_ERR_UNSUPPORTED).  Its scratch -- a work counter and, when theta is shared, the
+ * per-trajectory theta-bar [N][m] plus the block partials of the ensemble sum -- lives in one
+ * fixed array of GS_NOALLOC_SCRATCH_BYTES (8 MiB) inside the library, held by every GPU that
+ * loads the library until the process exits.  A record whose shared-theta scratch would not fit
+ * (about N*m <= 1.04e6 in double, 2.09e6 in float) is rejected with GS_ERR_CAPACITY.
+ * The first call on a device looks up that array's device address (a one-time set-up per
+ * device); make that first call before any stream capture begins.  All calls share the one
+ * array and the counter is cleared at the start of each call: calls that overlap on the GPU (on
+ * different streams, or from different threads) race and must not be issued.  Asynchronous. */
+#define GS_NOALLOC_SCRATCH_BYTES (8u << 20)
+gs_status gs_replay_grad_noalloc(const gs_record* rec, const void* theta, const void* dL_dy1,
+                                 void* dL_dtheta, void* dL_dy0, void* stream);
+
 /* Sizes and device pointers of a record (no synchronisation). */
 gs_status gs_record_info(const gs_record* rec, gs_record_info_t* out);
 
