@@ -189,6 +189,9 @@ struct gs_record {
   size_t red_bytes = 0, part_bytes = 0;
   void* y1_scratch = nullptr;    // y_S of gs_replay_forward when the caller passes no y1
   size_t y1_bytes = 0;
+  // device time of the solve kernel of the last record pass
+  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+  double solve_ms = 0;
   // summary
   int64_t nchunks = 0, total_steps = 0;
   int max_steps = 0;
@@ -353,6 +356,12 @@ gs_status launch_solve(const SolveCall& c) {
   }
 }
 
+// Dynamic shared memory of the adjoint kernel (none at present).
+template <class F, class R>
+constexpr size_t adjoint_smem() {
+  return 0;
+}
+
 struct AdjCall {
   const gs_record* rec;
   const void* theta;
@@ -383,8 +392,11 @@ gs_status launch_adjoint(const AdjCall& c) {
   p.queue = c.queue;
   p.perm = r->perm;
   auto kern = gs::k_adjoint<F, R, METHOD>;
-  const int grid = persistent_grid(kern, 0, r->N);
-  kern<<<grid, BLOCK, 0, c.stream>>>(p);
+  const size_t smem = adjoint_smem<F, R>();
+  if (smem > 48 * 1024)
+    GS_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const int grid = persistent_grid(kern, smem, r->N);
+  kern<<<grid, BLOCK, smem, c.stream>>>(p);
   GS_CUDA(cudaGetLastError());
   return GS_OK;
   }
@@ -575,13 +587,18 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
     return GS_OK;
   }
   int32_t* status_out = status ? status : r->status;
+  if (!r->ev0 && (cudaEventCreate(&r->ev0) != cudaSuccess || cudaEventCreate(&r->ev1) != cudaSuccess))
+    return bail(fail(GS_ERR_CUDA, "cudaEventCreate failed"));
+  r->solve_ms = 0;
   for (int pass = 0; pass < 2; ++pass) {
     if (cudaMemsetAsync(r->counters, 0, 16 * sizeof(int), s) != cudaSuccess)
       return bail(fail(GS_ERR_CUDA, "cudaMemsetAsync failed"));
     SolveCall c{N, theta, sys->theta_shared, y0, t0, t1, rtol, atol, attempts_of(opt), y1,
                 r->nsteps, nullptr, status_out, r->counters, r, s};
+    cudaEventRecord(r->ev0, s);
     st = dispatch(*sys, [&]<class F, class R, int METHOD>() { return launch_solve<F, R, METHOD>(c); });
     if (st != GS_OK) return bail(st);
+    cudaEventRecord(r->ev1, s);
     if (status_out != r->status &&
         cudaMemcpyAsync(r->status, status_out, N * sizeof(int), cudaMemcpyDeviceToDevice, s) !=
             cudaSuccess)
@@ -598,6 +615,8 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
     cudaError_t e = cudaStreamSynchronize(s);
     if (e != cudaSuccess)
       return bail(fail(GS_ERR_CUDA, "record solve failed: %s", cudaGetErrorString(e)));
+    float pass_ms = 0;
+    if (cudaEventElapsedTime(&pass_ms, r->ev0, r->ev1) == cudaSuccess) r->solve_ms += pass_ms;
     const int used = r->host[1];
     const int overflow = r->host[2];
     if (!overflow) {
@@ -749,6 +768,7 @@ gs_status gs_record_info(const gs_record* rec, gs_record_info_t* out) {
   out->chunk_offsets = reinterpret_cast<const int64_t*>(rec->choff);
   out->chunk_table = rec->chunk_table;
   out->pool = rec->pool;
+  out->solve_ms = rec->solve_ms;
   return GS_OK;
 }
 
@@ -859,6 +879,8 @@ void gs_record_destroy(gs_record* r) {
   free_ptr(r->red_scratch); free_ptr(r->red_partials); free_ptr(r->y1_scratch);
   free_ptr(r->perm); free_ptr(r->bins); free_ptr(r->binoff); free_ptr(r->btiles);
   if (r->host) cudaFreeHost(r->host);
+  if (r->ev0) cudaEventDestroy(r->ev0);
+  if (r->ev1) cudaEventDestroy(r->ev1);
   cudaSetDevice(prev);
   delete r;
 }
@@ -929,13 +951,14 @@ gs_status noalloc_adjoint(const gs_record* r, const void* theta, const void* dL_
     p.queue = reinterpret_cast<int*>(scratch);
     p.perm = r->perm;
     auto kern = gs::k_adjoint<F, R, METHOD>;
+    const size_t smem = adjoint_smem<F, R>();
     int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, BLOCK, 0) != cudaSuccess || nb < 1)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, BLOCK, smem) != cudaSuccess || nb < 1)
       nb = 1;
     const long long grid =
         std::max(1LL, std::min((long long)sms * nb, (long long)((N + BLOCK - 1) / BLOCK)));
     GS_CUDA(cudaMemsetAsync(scratch, 0, sizeof(int), s));  // the counter starts at zero
-    kern<<<(int)grid, BLOCK, 0, s>>>(p);
+    kern<<<(int)grid, BLOCK, smem, s>>>(p);
     if (shared) {
       gs::k_reduce_theta<R><<<nred, gs::RED_BLOCK, 0, s>>>(traj, (int)N, M, per_block, partials);
       gs::k_reduce_partials<R><<<1, 256, 0, s>>>(partials, nred, M, static_cast<R*>(dL_dtheta));

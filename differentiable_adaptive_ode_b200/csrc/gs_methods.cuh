@@ -56,6 +56,108 @@ template <class R> __device__ __forceinline__ R te(int i) {
   return R(E[i]);
 }
 
+// The same tables in constant memory, 1-based stage indices, zero-padded, for the rolled stage
+// loop below (the loop index selects the coefficients, so one copy of f serves every stage):
+//   fwd[i][m] = a_{i+1+m, i}  (stage i's slope into the stage states still open, m = 0..5)
+//   rev[i][m] = a_{i, i-1-m}  (stage i's cotangent into the earlier stages, m = 0..4)
+//   b[i] = b_i,  e[i] = b_i - bh_i.
+struct Tsit5Rolled {
+  double fwd[8][6], rev[8][5], b[8], e[8];
+};
+constexpr double tsit5_a1(int i, int j) {
+  // a_ij, 1-based, i = 2..7 (row 7 = b), j < i; 0 elsewhere
+  constexpr double A[8][8] = {
+      {0, 0, 0, 0, 0, 0, 0, 0},
+      {0, 0, 0, 0, 0, 0, 0, 0},
+      {0, Tsit5::a21, 0, 0, 0, 0, 0, 0},
+      {0, Tsit5::a31, Tsit5::a32, 0, 0, 0, 0, 0},
+      {0, Tsit5::a41, Tsit5::a42, Tsit5::a43, 0, 0, 0, 0},
+      {0, Tsit5::a51, Tsit5::a52, Tsit5::a53, Tsit5::a54, 0, 0, 0},
+      {0, Tsit5::a61, Tsit5::a62, Tsit5::a63, Tsit5::a64, Tsit5::a65, 0, 0},
+      {0, Tsit5::b1, Tsit5::b2, Tsit5::b3, Tsit5::b4, Tsit5::b5, Tsit5::b6, 0}};
+  return (i >= 0 && i < 8 && j >= 0 && j < 8) ? A[i][j] : 0.0;
+}
+constexpr Tsit5Rolled make_tsit5_rolled() {
+  Tsit5Rolled t{};
+  const double B[8] = {0, Tsit5::b1, Tsit5::b2, Tsit5::b3, Tsit5::b4, Tsit5::b5, Tsit5::b6, 0};
+  const double E[8] = {0, Tsit5::e1, Tsit5::e2, Tsit5::e3, Tsit5::e4, Tsit5::e5, Tsit5::e6, Tsit5::e7};
+  for (int i = 0; i < 8; ++i) {
+    t.b[i] = B[i];
+    t.e[i] = E[i];
+    for (int m = 0; m < 6; ++m) t.fwd[i][m] = (i >= 1 && i + 1 + m <= 7) ? tsit5_a1(i + 1 + m, i) : 0.0;
+    for (int m = 0; m < 5; ++m) t.rev[i][m] = (i - 1 - m >= 1) ? tsit5_a1(i, i - 1 - m) : 0.0;
+  }
+  return t;
+}
+static __constant__ Tsit5Rolled c_tsit5_d = make_tsit5_rolled();
+struct Tsit5RolledF {
+  float fwd[8][6], rev[8][5], b[8], e[8];
+};
+constexpr Tsit5RolledF make_tsit5_rolled_f() {
+  Tsit5RolledF t{};
+  const Tsit5Rolled d = make_tsit5_rolled();
+  for (int i = 0; i < 8; ++i) {
+    t.b[i] = float(d.b[i]);
+    t.e[i] = float(d.e[i]);
+    for (int m = 0; m < 6; ++m) t.fwd[i][m] = float(d.fwd[i][m]);
+    for (int m = 0; m < 5; ++m) t.rev[i][m] = float(d.rev[i][m]);
+  }
+  return t;
+}
+static __constant__ Tsit5RolledF c_tsit5_f = make_tsit5_rolled_f();
+template <class R> __device__ __forceinline__ const auto& tsit5_tab();
+template <> __device__ __forceinline__ const auto& tsit5_tab<double>() { return c_tsit5_d; }
+template <> __device__ __forceinline__ const auto& tsit5_tab<float>() { return c_tsit5_f; }
+
+// Tsit5 trial with the stage loop rolled: the open stage states are kept as running sums
+// acc[m] = partial Y_{i+m} (all slopes k_l, l < i, already added), so the loop body holds a
+// single copy of f.  Same result as tsit5_trial up to the order of the roundings; the products
+// are fused explicitly so that every kernel using it rounds identically.
+template <class F, class R>
+__device__ __forceinline__ R tsit5_trial_rolled(const R (&y)[F::D], R h,
+                                                const typename F::template Theta<R>& th,
+                                                const R (&k1)[F::D], R (&ynew)[F::D],
+                                                R (&k7)[F::D], R rtol, R atol) {
+  constexpr int D = F::D;
+  const auto& T = tsit5_tab<R>();
+  R acc[6][D], er[D];
+#pragma unroll
+  for (int m = 0; m < 6; ++m) {
+    const R hc = h * T.fwd[1][m];
+#pragma unroll
+    for (int c = 0; c < D; ++c) acc[m][c] = fma(hc, k1[c], y[c]);
+  }
+#pragma unroll
+  for (int c = 0; c < D; ++c) er[c] = T.e[1] * k1[c];
+#pragma unroll 1
+  for (int i = 2; i <= 7; ++i) {
+    R kk[D];
+    F::f(acc[0], th, kk);
+    const R ei = T.e[i];
+#pragma unroll
+    for (int c = 0; c < D; ++c) er[c] = fma(ei, kk[c], er[c]);
+    if (i == 7) {
+#pragma unroll
+      for (int c = 0; c < D; ++c) { ynew[c] = acc[0][c]; k7[c] = kk[c]; }
+    }
+#pragma unroll
+    for (int m = 0; m < 5; ++m) {
+      const R hc = h * T.fwd[i][m];
+#pragma unroll
+      for (int c = 0; c < D; ++c) acc[m][c] = fma(hc, kk[c], acc[m + 1][c]);
+    }
+  }
+  R s2 = R(0);
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    const R e = h * er[c];
+    const R sc = fma(rtol, fmax(fabs(y[c]), fabs(ynew[c])), atol);
+    const R q = e / sc;
+    s2 = fma(q, q, s2);
+  }
+  return sqrt(s2 / R(D));
+}
+
 // One Tsit5 trial from y with step h; k1 = f(y) is carried (first-same-as-last).  Produces the
 // step result ynew, its slope k7 = f(ynew) (the next k1) and the scaled RMS error
 //   err = sqrt(mean_i (e_i / (atol + rtol max(|y_i|, |ynew_i|)))^2),  e = h sum_j (b_j - bh_j) k_j.

@@ -99,6 +99,8 @@ typedef struct {
                                    chunk_offsets[k] + j */
   const void* pool;             /* chunk c holds steps of one trajectory at
                                    pool + (c*C + slot)*E reals, entry = (t, h, y[0..d-1]) */
+  double solve_ms;              /* device time of the solve kernel(s) of the last
+                                   gs_solve_record (CUDA events around the launch), 0 if none */
 } gs_record_info_t;
 
 /* Forward-only solve ([GS] §4.1: one thread per trajectory, final state only).

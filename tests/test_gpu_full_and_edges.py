@@ -1,0 +1,186 @@
+"""GPU parity at the benchmark sizes (sampled trajectories the oracle computes one by one) and the
+edge cases: empty and single-trajectory ensembles, a zero-length interval, non-finite parameters,
+the attempt cap, record reuse, the pool-overflow re-run, and zero-length padding steps in an
+imported record ([GS] = "gradsolve: fast exact gradients for ODE ensembles on GPUs", §3: a step of
+size zero leaves the state and its derivative unchanged)."""
+import numpy as np
+import pytest
+
+import gpu_util as U
+from differentiable_adaptive_ode_b200 import gradsolve as G
+from differentiable_adaptive_ode_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    G.lib()
+
+
+def _sample(N, n=24, seed=0):
+    rng = np.random.default_rng(seed)
+    return np.unique(np.concatenate([[0, N - 1], rng.choice(N, size=n, replace=False)]))
+
+
+def _target(orc, w):
+    """Loss targets: drawn (Lorenz, stellar) or solved at nominal parameters by the oracle."""
+    if w.target is not None:
+        return w.target
+    if w.target_kind == "nominal_solve":
+        r = orc.solve(w.field, w.method, w.nominal_theta[None, :], w.y0[:1], w.t0, w.t1, w.rtol,
+                      w.atol)
+        return np.repeat(r["y1"], w.N, axis=0)
+    r = orc.solve(w.field, w.method, w.nominal_theta, w.y0, w.t0, w.t1, 1e-10, 1e-12,
+                  theta_shared=True, nthreads=8)
+    return r["y1"]
+
+
+@pytest.mark.parametrize("name", ["lotka_volterra", "lorenz63", "robertson", "nfw_mn"])
+def test_full_size_sampled_parity(orc, name):
+    w = W.by_name(name)
+    rec, out = U.record(w)
+    info = rec.info()
+    idx = _sample(w.N)
+    sub = W.subset(w, idx)
+    ref = orc.solve(sub.field, sub.method, sub.theta, sub.y0, sub.t0, sub.t1, sub.rtol, sub.atol,
+                    nthreads=8)
+    assert np.all(out["status"] == 0)
+    # counts and final states of the sampled trajectories
+    import torch
+    off = torch.empty(w.N + 1, dtype=torch.int64, device="cuda")
+    tot = int(info.total_steps)
+    H = torch.empty(tot, dtype=torch.float64, device="cuda")
+    G.gs_record_export(rec, None, H, None, off)
+    torch.cuda.synchronize()
+    off = off.cpu().numpy()
+    S = np.diff(off)
+    assert np.array_equal(S[idx], ref["S"])
+    rel = U.rel_rows(out["y1"][idx], ref["y1"], w.atol)
+    assert rel.max() <= 1e-9, rel.max()
+    # gradient of the loss on the GPU mesh for the sampled trajectories
+    tgt = _target(orc, w)
+    lam = W.loss_cotangent(w, out["y1"], tgt)
+    gy, gt = U.replay_grad(w, rec, lam)
+    Hn = H.cpu().numpy()
+    Hs = np.zeros((len(idx), S[idx].max()))
+    for r_, k in enumerate(idx):
+        Hs[r_, :S[k]] = Hn[off[k]:off[k + 1]]
+    ry, rt = orc.replay_grad(sub.field, sub.method, sub.theta, sub.y0, Hs, S[idx], lam[idx],
+                             nthreads=8)
+    assert U.rel_rows(gy[idx], ry, 1e-300).max() <= 1e-8
+    assert U.rel_rows(gt[idx], rt, 1e-300).max() <= 1e-8
+
+
+def test_full_size_mlp_sampled_shared_gradient(orc):
+    # the ensemble weight gradient is linear in dL/dy1: zero the cotangent outside a sample and
+    # the GPU returns the sample's weight gradient, which the oracle computes directly
+    import torch
+    w = W.mlp()
+    rec, out = U.record(w)
+    idx = _sample(w.N, n=16)
+    sub = W.subset(w, idx)
+    ref = orc.solve("mlp", "tsit5", w.theta, sub.y0, 0.0, 1.0, w.rtol, w.atol, dtype=np.float32,
+                    theta_shared=True, nthreads=8)
+    assert np.all(out["status"] == 0)
+    info = rec.info()
+    off = torch.empty(w.N + 1, dtype=torch.int64, device="cuda")
+    H = torch.empty(int(info.total_steps), dtype=torch.float32, device="cuda")
+    G.gs_record_export(rec, None, H, None, off)
+    torch.cuda.synchronize()
+    off = off.cpu().numpy()
+    S = np.diff(off)
+    # fp32: accept decisions near err = 1 sit on the rounding floor (the oracle against itself
+    # under a one-ulp change of y0 keeps ~85 % of the counts on this ensemble)
+    assert np.all(np.abs(S[idx].astype(int) - ref["S"]) <= 1)
+    assert np.mean(S[idx] == ref["S"]) >= 0.5
+    tgt = _target(orc, w).astype(np.float32)
+    lam = np.zeros((w.N, 4))
+    lam[idx] = W.loss_cotangent(w, out["y1"], tgt)[idx]
+    gy, gt = U.replay_grad(w, rec, lam)
+    Hn = H.cpu().numpy().astype(np.float64)
+    Hs = np.zeros((len(idx), S[idx].max()))
+    for r_, k in enumerate(idx):
+        Hs[r_, :S[k]] = Hn[off[k]:off[k + 1]]
+    ry, rt = orc.replay_grad("mlp", "tsit5", w.theta, sub.y0, Hs, S[idx], lam[idx],
+                             theta_shared=True, nthreads=8)
+    want = rt.sum(0)
+    assert np.linalg.norm(gt - want) <= 1e-3 * np.linalg.norm(want)
+    others = np.setdiff1d(np.arange(w.N), idx)
+    assert np.all(gy[others] == 0)
+
+
+def test_empty_and_single_and_zero_interval():
+    import torch
+    w = W.lorenz63(N=1)
+    rec, out = U.record(w)
+    assert rec.info().N == 1 and out["status"][0] == 0
+    # N = 0: nothing to do, success
+    sys_ = U.gsys(w)
+    z = torch.empty((0, 3), dtype=torch.float64, device="cuda")
+    G.gs_solve_forward(sys_, 0, z, z, 0.0, 1.0, 1e-6, 1e-9, z)
+    # t1 == t0: zero steps, y1 = y0, gradient = identity in y0 and zero in theta
+    w0 = W.lorenz63(N=5)
+    w0.t1 = 0.0
+    rec0, out0 = U.record(w0)
+    assert rec0.info().total_steps == 0
+    assert np.array_equal(out0["y1"], w0.y0)
+    lam = np.random.default_rng(0).normal(size=(5, 3))
+    gy, gt = U.replay_grad(w0, rec0, lam)
+    assert np.array_equal(gy, lam) and np.all(gt == 0)
+
+
+def test_status_codes_and_failed_record():
+    w = W.lorenz63(N=8)
+    w.theta = w.theta.copy()
+    w.theta[3, 0] = np.nan
+    fw = U.forward(w)
+    assert fw["status"][3] == 3 and np.all(np.delete(fw["status"], 3) == 0)
+    with pytest.raises(G.GradsolveError) as e:
+        U.record(w)
+    assert e.value.code == G.GS_ERR_TRAJ_FAILED
+    rec, out = U.record(w, allow_failed=True)
+    assert out["status"][3] == 3
+    w2 = W.lorenz63(N=8)
+    fw2 = U.forward(w2, max_attempts=5)
+    assert np.all(fw2["status"] == 1) and np.all(fw2["S"] + fw2["rejected"] == 5)
+
+
+def test_record_reuse_and_overflow_rerun(orc):
+    w = W.nfw_mn(N=700)
+    # a pool far too small: the solve runs again with the exact size; results unchanged
+    rec, out = U.record(w, capacity=50)
+    ex = U.export_padded(w, rec)
+    ref = orc.solve(w.field, w.method, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol, nthreads=8)
+    assert np.array_equal(ex["S"], ref["S"])
+    # reuse the record for another ensemble of a different size
+    w2 = W.lorenz63(N=900)
+    rec2, out2 = U.record(w2, rec=rec)
+    ex2 = U.export_padded(w2, rec2)
+    ref2 = orc.solve(w2.field, w2.method, w2.theta, w2.y0, w2.t0, w2.t1, w2.rtol, w2.atol,
+                     nthreads=8)
+    assert np.array_equal(ex2["S"], ref2["S"])
+    assert U.rel_rows(out2["y1"], ref2["y1"], w2.atol).max() <= 1e-9
+
+
+def test_zero_steps_in_imported_record_change_nothing(orc):
+    w = W.lorenz63(N=50)
+    ref = orc.solve(w.field, w.method, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol, keep_record=True)
+    lam = np.random.default_rng(1).normal(size=(w.N, 3))
+    rec = U.import_record(w, ref["S"], ref["T"], ref["H"], ref["Y"])
+    gy, gt = U.replay_grad(w, rec, lam)
+    # append three h = 0 steps (state repeated) to every record
+    S2 = ref["S"] + 3
+    Smax = S2.max()
+    T2 = np.zeros((w.N, Smax)); H2 = np.zeros((w.N, Smax)); Y2 = np.zeros((w.N, Smax, 3))
+    for k in range(w.N):
+        s = ref["S"][k]
+        T2[k, :s], H2[k, :s], Y2[k, :s] = ref["T"][k, :s], ref["H"][k, :s], ref["Y"][k, :s]
+        T2[k, s:s + 3] = w.t1
+        Y2[k, s:s + 3] = ref["y1"][k]
+    rec2 = U.import_record(w, S2, T2, H2, Y2)
+    gy2, gt2 = U.replay_grad(w, rec2, lam)
+    assert np.array_equal(gy, gy2) and np.array_equal(gt, gt2)

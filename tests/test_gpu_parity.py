@@ -101,8 +101,10 @@ def test_record_parity_and_replay(orc, name, N):
     same = np.flatnonzero(ex["S"] == ref["S"]) if w.dtype == np.float64 else []
     for k in same[:50]:
         S = ex["S"][k]
-        hr = U.rel_rows(ex["H"][k, :S, None], ref["H"][k, :S, None], 1e-300)
-        assert hr.max() <= 1e4 * STATE_TOL[w.dtype], (k, hr.max())
+        # step sizes relative to the trajectory's largest step (the last, clipped step can be
+        # tiny, and its size is a difference of nearly equal times)
+        dh = np.max(np.abs(ex["H"][k, :S] - ref["H"][k, :S])) / np.max(np.abs(ref["H"][k, :S]))
+        assert dh <= 1e-6, (k, dh)
         assert np.array_equal(ex["T"][k, 0], ref["T"][k, 0])
     # the forward-only kernel and the record kernel take identical steps
     fw = U.forward(w)
