@@ -36,6 +36,11 @@ FLOPS_FORWARD_ATTEMPT = {"nfw_mn": 611}
 # FP64 peak: 148 SMs x 64 FP64 FMA lanes/SM/clk x 2 flop x clock (1965 MHz max) = 37.2 TFLOP/s,
 # the datasheet FP64 figure of B200; the same formula at the measured SM clock is reported too.
 SMS, FP64_LANES = 148, 64
+# DRAM bytes (read + write) per accepted step, from one ncu capture of each kernel on the
+# 2^18-trajectory case of this workload; both kernels move a fixed number of bytes per accepted
+# step, so a launch's traffic is this times its accepted steps.  Record kernel: 64 B of record
+# per step written plus inputs; adjoint: the 64 B entry read per step plus chunk table and inputs.
+TRAFFIC_PER_STEP = {"record": 65.85, "adjoint": 72.16}
 # library kernels per step: record = k_solve + 2 k_max_int + 3 prefix scans of 3 kernels each
 # (step offsets, chunk offsets, length bins) + k_chunk_table + k_bin_count + k_bin_scatter (15);
 # replay gradient = k_adjoint (1).
@@ -305,10 +310,11 @@ def main():
     peak_max = fp64_peak_tflops(1965.0)
     at_clock = fp64_peak_tflops(clocks["sm_mhz"]) if clocks.get("sm_mhz") else None
 
-    def roof(name, flops, ms, per_unit, unit_name):
+    def roof(name, flops, ms, per_unit, unit_name, traffic):
         achieved = flops / (ms / 1e3) / 1e12
         return {"kernel": name, "bound": "alu", "achieved": achieved, "peak": peak_max,
-                "unit": "TFLOP/s", "frac": achieved / peak_max, "traffic": None,
+                "unit": "TFLOP/s", "frac": achieved / peak_max, "traffic": traffic,
+                "traffic_source": "ncu dram bytes per accepted step on the 2^18 case x steps",
                 "peak_source": "derived: 148 SM x 64 FP64 FMA/clk x 2 x 1965 MHz (FP64 pipe)",
                 "flops_per_unit": per_unit, "unit_counted": unit_name, "kernel_ms": ms,
                 "frac_at_measured_clock": achieved / at_clock if at_clock else None}
@@ -316,10 +322,12 @@ def main():
     rec_ms = statistics.median(solve_ms)
     roof_rec = roof("k_solve<NfwMiyamotoNagai, double, Tsit5, record>",
                     attempts * FLOPS_FORWARD_ATTEMPT["nfw_mn"], rec_ms,
-                    FLOPS_FORWARD_ATTEMPT["nfw_mn"], "attempted step")
+                    FLOPS_FORWARD_ATTEMPT["nfw_mn"], "attempted step",
+                    TRAFFIC_PER_STEP["record"] * total_steps)
     roof_adj = roof("k_adjoint<NfwMiyamotoNagai, double, Tsit5>",
                     total_steps * FLOPS_ADJOINT_STEP["nfw_mn"], adj_ms,
-                    FLOPS_ADJOINT_STEP["nfw_mn"], "accepted step")
+                    FLOPS_ADJOINT_STEP["nfw_mn"], "accepted step",
+                    TRAFFIC_PER_STEP["adjoint"] * total_steps)
     dominant, other = (roof_rec, roof_adj) if rec_ms >= adj_ms else (roof_adj, roof_rec)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,

@@ -335,7 +335,8 @@ __global__ void __launch_bounds__(128, Tune<F, R>::adj_blocks) k_adjoint(Adjoint
   constexpr int D = F::D, M = F::M;
   int k = -1;
   bool alive = true;
-  int n = 0;
+  int n = 0, first_n = -1, cur_ch = 0, next_ch = -1;
+  bool pf_pending = false;
   long long cbase = 0;
   R lam[D], thb[M];
   typename F::template Theta<R> th;
@@ -357,6 +358,7 @@ __global__ void __launch_bounds__(128, Tune<F, R>::adj_blocks) k_adjoint(Adjoint
 #pragma unroll
           for (int j = 0; j < M; ++j) thb[j] = R(0);
           n = p.nsteps[k] - 1;
+          first_n = n;
           cbase = p.choff[k];
         } else {
           alive = false;
@@ -366,7 +368,20 @@ __global__ void __launch_bounds__(128, Tune<F, R>::adj_blocks) k_adjoint(Adjoint
     if (!__any_sync(FULL, k >= 0 || alive)) break;
     if (k >= 0) {
       if (n >= 0) {
-        const int ch = __ldg(p.chunk_table + cbase + n / L::C);
+        // chunk of step n; on entering a chunk, fetch the id of the next chunk to be visited and
+        // prefetch its lines one step later (the id load then has had a whole step to land)
+        if (n == first_n || n % L::C == L::C - 1) {
+          cur_ch = __ldg(p.chunk_table + cbase + n / L::C);
+          next_ch = (n / L::C >= 1) ? __ldg(p.chunk_table + cbase + n / L::C - 1) : -1;
+          pf_pending = next_ch >= 0;
+        } else if (pf_pending) {
+          const R* q = p.pool + (size_t)next_ch * L::C * L::E;
+#pragma unroll
+          for (int b = 0; b < L::C * L::E * (int)sizeof(R); b += 128)
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const char*>(q) + b));
+          pf_pending = false;
+        }
+        const int ch = cur_ch;
         const R* e = p.pool + ((size_t)ch * L::C + (n % L::C)) * L::E;
         const R h = __ldg(e + 1);
         R y[D];
