@@ -31,7 +31,7 @@ UNIT = "traj/s"
 # mul, fma = 2, div, sqrt, log1p each counted as one operation), and per attempted step of the
 # forward solve: counted from the definitions of the Tsit5 replay step, its reverse sweep and the
 # field's f and vector-Jacobian product (tests/test_flop_counts.py re-derives these numbers).
-FLOPS_ADJOINT_STEP = {"nfw_mn": 1416}
+FLOPS_ADJOINT_STEP = {"nfw_mn": 1254}
 FLOPS_FORWARD_ATTEMPT = {"nfw_mn": 611}
 # FP64 peak: 148 SMs x 64 FP64 FMA lanes/SM/clk x 2 flop x clock (1965 MHz max) = 37.2 TFLOP/s,
 # the datasheet FP64 figure of B200; the same formula at the measured SM clock is reported too.
@@ -103,6 +103,15 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def workload_config(ws, N=1 << 20):
+    return {"workload": "nfw_mn stellar orbits: NFW halo + Miyamoto-Nagai disk, N=%d per GPU, "
+                        "d=6, m=5 per trajectory, fp64, Tsit5 rtol=1e-8 atol=1e-10, t=[0,20]; "
+                        "step = record + loss cotangent + replay gradient" % N,
+            "global_batch": ws * N,
+            "parallelism": "independent trajectories, %d rank(s)" % ws,
+            "l2": "inputs larger than L2 (the record is ~9 GB at 2^20)"}
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -137,9 +146,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": "nfw_mn stellar orbits, N=2^20 (sampled), d=6, m=5, fp64, "
-                                   "Tsit5 rtol=1e-8 atol=1e-10, t=[0,20]",
-                       "global_batch": 1 << 20, "sample": n_sample},
+            "config": dict(workload_config(1), sample="%d trajectories per step" % n_sample),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": nthreads, "kind": "oracle",
                              "sample": "%d trajectories of the 2^20 ensemble per step: record "
                                        "solve + replay gradient" % n_sample},
@@ -333,12 +340,9 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "nfw_mn stellar orbits: NFW halo + Miyamoto-Nagai disk, N=2^20 "
-                               "per GPU, d=6, m=5 per trajectory, fp64, Tsit5 rtol=1e-8 atol=1e-10, "
-                               "t=[0,20]; step = record + loss cotangent + replay gradient",
-                   "global_batch": ws * N, "parallelism": "independent trajectories, %d rank(s)" % ws,
-                   "l2": "inputs larger than L2 (record %.1f GB)" % (info.pool_bytes / 1e9),
-                   "accepted_steps": total_steps, "attempts_forward": attempts},
+        "config": dict(workload_config(ws, N), accepted_steps=total_steps,
+                       attempts_forward=attempts,
+                       record_gb=round(info.pool_bytes / 1e9, 2)),
         "roofline": dominant,
         "roofline_other": other,
         "breakdown_ms": {"forward_only": fwd_ms, "record": rec_ms, "replay_grad": grad_ms,

@@ -356,10 +356,12 @@ gs_status launch_solve(const SolveCall& c) {
   }
 }
 
-// Dynamic shared memory of the adjoint kernel (none at present).
+// Dynamic shared memory of the adjoint kernel: the per-lane stage tape of fields with TAPE > 0
+// (6 stages x TAPE reals x 128 lanes).
 template <class F, class R>
 constexpr size_t adjoint_smem() {
-  return 0;
+  if constexpr (std::is_same_v<F, gs::FMlpWarp>) return 0;
+  else return (size_t)6 * gs::TapeOf<F>::value * BLOCK * sizeof(R);
 }
 
 struct AdjCall {

@@ -213,10 +213,53 @@ struct FNfwMiyamotoNagai {
     dy[4] = -g * y[1];
     dy[5] = -(I.gN + I.gM * I.apB * I.iB) * y[2];
   }
+  // Tape of a stage for the reverse sweep: the five transcendental results of f at that stage,
+  // so that the VJP recomputes only products and sums.
+  static constexpr int TAPE = 5;
+  template <class R> GS_HD static void inter_tape(const R* y, const Theta<R>& t, R* tp) {
+    Inter<R> I;
+    inter(y, t, I);
+    tp[0] = I.ir; tp[1] = I.L; tp[2] = I.isr; tp[3] = I.iB; tp[4] = I.iD;
+  }
+  template <class R>
+  GS_HD static void f_tape(const R* y, const Theta<R>& t, R* dy, R* tp) {
+    Inter<R> I;
+    inter(y, t, I);
+    tp[0] = I.ir; tp[1] = I.L; tp[2] = I.isr; tp[3] = I.iB; tp[4] = I.iD;
+    const R g = I.gN + I.gM;
+    dy[0] = y[3];
+    dy[1] = y[4];
+    dy[2] = y[5];
+    dy[3] = -g * y[0];
+    dy[4] = -g * y[1];
+    dy[5] = -(I.gN + I.gM * I.apB * I.iB) * y[2];
+  }
+  template <class R>
+  GS_HD static void vjp_tape(const R* y, const Theta<R>& t, const R* tp, const R* kb, R* yb,
+                             R* thb) {
+    Inter<R> I;
+    const R x = y[0], yy = y[1], z = y[2];
+    I.R2 = x * x + yy * yy;
+    I.ir = tp[0];
+    I.r = (I.R2 + z * z) * I.ir;
+    I.L = tp[1];
+    I.isr = tp[2];
+    I.gN = t.Mh * (I.ir * I.ir) * (I.L * I.ir - I.isr);
+    I.iB = tp[3];
+    I.apB = t.a + (z * z + t.b2) * I.iB;
+    I.iD = tp[4];
+    I.gM = t.Md * (I.iD * I.iD * I.iD);
+    vjp_from(y, t, I, kb, yb, thb);
+  }
   template <class R>
   GS_HD static void vjp(const R* y, const Theta<R>& t, const R* kb, R* yb, R* thb) {
     Inter<R> I;
     inter(y, t, I);
+    vjp_from(y, t, I, kb, yb, thb);
+  }
+  template <class R>
+  GS_HD static void vjp_from(const R* y, const Theta<R>& t, const Inter<R>& I, const R* kb, R* yb,
+                             R* thb) {
     const R x = y[0], yy = y[1], z = y[2];
     const R ux = kb[3], uy = kb[4], uz = kb[5];
     const R ir2 = I.ir * I.ir;

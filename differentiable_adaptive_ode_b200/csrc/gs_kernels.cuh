@@ -333,6 +333,8 @@ template <class F, class R, int METHOD>
 __global__ void __launch_bounds__(128, Tune<F, R>::adj_blocks) k_adjoint(AdjointParams<R> p) {
   using L = RecLayout<F, R>;
   constexpr int D = F::D, M = F::M;
+  extern __shared__ __align__(16) unsigned char adj_smem[];
+  R* tape = reinterpret_cast<R*>(adj_smem) + threadIdx.x;  // per-lane stage tape (TAPE fields)
   int k = -1;
   bool alive = true;
   int n = 0, first_n = -1, cur_ch = 0, next_ch = -1;
@@ -387,7 +389,7 @@ __global__ void __launch_bounds__(128, Tune<F, R>::adj_blocks) k_adjoint(Adjoint
         R y[D];
 #pragma unroll
         for (int c = 0; c < D; ++c) y[c] = __ldg(e + 2 + c);
-        if constexpr (METHOD == M_TSIT5) tsit5_adjoint_step<F, R>(y, h, th, lam, thb);
+        if constexpr (METHOD == M_TSIT5) tsit5_adjoint_step<F, R>(y, h, th, lam, thb, tape, blockDim.x);
         else ros_adjoint_step<F, R>(y, h, th, lam, thb);
         --n;
       }

@@ -8,6 +8,8 @@
 // Coefficients (not printed on the pages): Tsitouras (2011) for Tsit5, Rang & Angermann (2005)
 // for ROS34PW2 -- the published decimals, rounded to the working precision at compile time.
 #pragma once
+#include <type_traits>
+
 #include "gs_fields.cuh"
 
 namespace gs {
@@ -237,17 +239,34 @@ __device__ __forceinline__ void tsit5_replay_step(const R (&y)[F::D], R h,
 // recompute the stages from the recorded y_n, then sweep them backwards.
 //   kb_i = h (b_i lam + sum_{j>i} a_ji Yb_j),  Yb_i = J_y(Y_i)^T kb_i,  thb += J_th(Y_i)^T kb_i,
 //   lam <- lam + sum_i Yb_i.   (b_7 = 0, so the seventh stage never enters the replay map.)
+// Fields that declare TAPE > 0 hand the reverse sweep the transcendental part of f at each stage
+// (kept in a per-lane shared-memory tape) instead of recomputing it in the VJP.
+template <class F, class = void> struct TapeOf { static constexpr int value = 0; };
+template <class F> struct TapeOf<F, std::void_t<decltype(F::TAPE)>> {
+  static constexpr int value = F::TAPE;
+};
+
+// tape: this lane's slot 0; slot (i, v) at tape[(i * TAPE + v) * tstride] (shared memory).
 template <class F, class R>
 __device__ __forceinline__ void tsit5_adjoint_step(const R (&y)[F::D], R h,
                                                    const typename F::template Theta<R>& th,
-                                                   R (&lam)[F::D], R (&thb)[F::M]) {
+                                                   R (&lam)[F::D], R (&thb)[F::M],
+                                                   R* tape = nullptr, int tstride = 0) {
   constexpr int D = F::D;
+  constexpr int TP = TapeOf<F>::value;
   R Y[6][D];
   {
     R k[5][D];
 #pragma unroll
     for (int c = 0; c < D; ++c) Y[0][c] = y[c];
-    F::f(Y[0], th, k[0]);
+    if constexpr (TP > 0) {
+      R tp[TP > 0 ? TP : 1];
+      F::f_tape(Y[0], th, k[0], tp);
+#pragma unroll
+      for (int v = 0; v < TP; ++v) tape[v * tstride] = tp[v];
+    } else {
+      F::f(Y[0], th, k[0]);
+    }
 #pragma unroll
     for (int i = 1; i < 6; ++i) {
 #pragma unroll
@@ -257,7 +276,15 @@ __device__ __forceinline__ void tsit5_adjoint_step(const R (&y)[F::D], R h,
         for (int j = 1; j < i; ++j) s += ta<R>(i, j) * k[j][c];
         Y[i][c] = y[c] + h * s;
       }
-      if (i < 5) F::f(Y[i], th, k[i]);
+      if constexpr (TP > 0) {
+        R tp[TP > 0 ? TP : 1];
+        if (i < 5) F::f_tape(Y[i], th, k[i], tp);
+        else F::inter_tape(Y[i], th, tp);
+#pragma unroll
+        for (int v = 0; v < TP; ++v) tape[(i * TP + v) * tstride] = tp[v];
+      } else {
+        if (i < 5) F::f(Y[i], th, k[i]);
+      }
     }
   }
   // Reverse sweep.  Yb_j is kept for the stages j > i still to be visited, so that at every
@@ -276,7 +303,14 @@ __device__ __forceinline__ void tsit5_adjoint_step(const R (&y)[F::D], R h,
       for (int j = i + 1; j < 6; ++j) g += ta<R>(j, i) * Yb[j][c];
       kb[c] = h * (tb<R>(i) * lam[c] + g);
     }
-    F::vjp(Y[i], th, kb, Yb[i], thb);
+    if constexpr (TP > 0) {
+      R tp[TP > 0 ? TP : 1];
+#pragma unroll
+      for (int v = 0; v < TP; ++v) tp[v] = tape[(i * TP + v) * tstride];
+      F::vjp_tape(Y[i], th, tp, kb, Yb[i], thb);
+    } else {
+      F::vjp(Y[i], th, kb, Yb[i], thb);
+    }
 #pragma unroll
     for (int c = 0; c < D; ++c) lnew[c] += Yb[i][c];
   }

@@ -1,8 +1,11 @@
 // Host program that tallies the arithmetic of the device fields' f and vector-Jacobian product
-// (add/sub, mul, div, sqrt, log1p per call) by instantiating them with a counting scalar.
+// (add/sub, mul, div, sqrt/rsqrt, log1p per call) by instantiating them with a counting scalar.
+// For a field that hands its VJP the intermediates of f (a stage tape), the VJP is counted
+// without recomputing them: that recomputation is not part of the pullback.
 // Compiled as plain C++ (g++) and run by tests/test_flop_counts.py; prints one JSON object per field.
 #include <cmath>
 #include <cstdio>
+#include <type_traits>
 
 #include "gs_fields.cuh"
 
@@ -24,6 +27,10 @@ inline Cnt sqrt(Cnt a) { T.sqrt++; return Cnt(std::sqrt(a.v)); }
 inline Cnt log1p(Cnt a) { T.log1p++; return Cnt(std::log1p(a.v)); }
 inline Cnt rsqrt(Cnt a) { T.sqrt++; return Cnt(1.0 / std::sqrt(a.v)); }
 
+template <class F, class = void> struct has_pullback : std::false_type {};
+template <class F>
+struct has_pullback<F, std::void_t<decltype(F::TAPE)>> : std::true_type {};
+
 template <class F>
 void run(const char* name, const double* theta, const double* y) {
   Cnt th_src[F::M], yy[F::D], dy[F::D], kb[F::D], yb[F::D], thb[F::M];
@@ -34,9 +41,19 @@ void run(const char* name, const double* theta, const double* y) {
   T = Tally();
   F::f(yy, th, dy);
   Tally tf = T;
-  T = Tally();
-  F::vjp(yy, th, kb, yb, thb);
-  Tally tv = T;
+  Tally tv;
+  if constexpr (has_pullback<F>::value) {
+    // the pullback proper, given f's intermediates at the stage (which f already computed)
+    typename F::template Inter<Cnt> I;
+    F::inter(yy, th, I);
+    T = Tally();
+    F::vjp_from(yy, th, I, kb, yb, thb);
+    tv = T;
+  } else {
+    T = Tally();
+    F::vjp(yy, th, kb, yb, thb);
+    tv = T;
+  }
   std::printf("{\"field\": \"%s\", \"D\": %d, \"M\": %d, "
               "\"f\": {\"add\": %ld, \"mul\": %ld, \"div\": %ld, \"sqrt\": %ld, \"log1p\": %ld}, "
               "\"vjp\": {\"add\": %ld, \"mul\": %ld, \"div\": %ld, \"sqrt\": %ld, \"log1p\": %ld}}\n",
