@@ -334,22 +334,23 @@ gs_status launch_solve(const SolveCall& c) {
     return GS_OK;
   } else {
     if (c.rec) {
-      using L = gs::RecLayout<F, R>;
       p.pool = static_cast<R*>(c.rec->pool);
       p.chunk_traj = c.rec->chunk_traj;
       p.chunk_seq = c.rec->chunk_seq;
       p.pool_chunks = (int)c.rec->pool_chunks;
       p.chunk_count = c.rec->counters + 1;
       p.overflow = c.rec->counters + 2;
-      const size_t smem = (size_t)(BLOCK / 32) * 32 * L::STAGE_STRIDE * sizeof(R);
+      const size_t smem = gs::solve_smem_bytes<F, R, true>();
       auto kern = gs::k_solve<F, R, METHOD, true>;
       GS_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
       const int grid = persistent_grid(kern, smem, c.N);
       kern<<<grid, BLOCK, smem, c.stream>>>(p);
     } else {
       auto kern = gs::k_solve<F, R, METHOD, false>;
-      const int grid = persistent_grid(kern, 0, c.N);
-      kern<<<grid, BLOCK, 0, c.stream>>>(p);
+      const size_t smem = gs::solve_smem_bytes<F, R, false>();
+      GS_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+      const int grid = persistent_grid(kern, smem, c.N);
+      kern<<<grid, BLOCK, smem, c.stream>>>(p);
     }
     GS_CUDA(cudaGetLastError());
     return GS_OK;
@@ -622,7 +623,7 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
     const int used = r->host[1];
     const int overflow = r->host[2];
     if (!overflow) {
-      r->nchunks = used;
+      r->nchunks = std::min<int64_t>(used, r->pool_chunks);  // reserved, some possibly unused
       r->max_steps = r->host[3];
       long long tot;
       std::memcpy(&tot, r->host + 8, sizeof(tot));
@@ -630,7 +631,10 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
       break;
     }
     if (pass == 1) return bail(fail(GS_ERR_CAPACITY, "record pool overflow after resize"));
-    if ((st = ensure_pool(r, (int64_t)used + (used >> 4) + 1024)) != GS_OK) return bail(st);
+    // room for the steps plus every warp's partly used chunk reservation
+    const int64_t warps = (int64_t)(N + 31) / 32;
+    if ((st = ensure_pool(r, (int64_t)used + (used >> 4) + gs::CHUNK_BATCH * std::min<int64_t>(warps, 1 << 16) + 1024)) != GS_OK)
+      return bail(st);
   }
   // chunk offsets and table
   if ((st = scan_counts<1>(r->nsteps, (int)N, C, r->choff, r->tiles, s)) != GS_OK) return bail(st);

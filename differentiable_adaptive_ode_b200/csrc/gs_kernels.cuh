@@ -135,6 +135,27 @@ template <> struct Tune<FNfwMiyamotoNagai, double> {
   static constexpr int adj_blocks = 3, solve_blocks = 3;
 };
 
+// Record chunks are reserved from the global bump counter CHUNK_BATCH at a time per warp.
+constexpr int CHUNK_BATCH = 32;
+
+// Per-warp ring of trajectories whose start-up is done (id, status, starting step, f(y0)).
+constexpr int START_RING = 64;
+template <class F, class R>
+struct StartRing {
+  R f0[F::D][START_RING];
+  R h0[START_RING];
+  int id[START_RING];
+  int st[START_RING];
+};
+template <class F, class R>
+__host__ __device__ constexpr size_t solve_stage_bytes() {
+  return (size_t)4 * 32 * RecLayout<F, R>::STAGE_STRIDE * sizeof(R);
+}
+template <class F, class R, bool REC>
+__host__ __device__ constexpr size_t solve_smem_bytes() {
+  return (REC ? solve_stage_bytes<F, R>() : 0) + 4 * sizeof(StartRing<F, R>);
+}
+
 template <class F, class R, int METHOD, bool REC>
 __global__ void __launch_bounds__(128, Tune<F, R>::solve_blocks) k_solve(SolveParams<R> p) {
   using L = RecLayout<F, R>;
@@ -142,20 +163,21 @@ __global__ void __launch_bounds__(128, Tune<F, R>::solve_blocks) k_solve(SolvePa
   constexpr int order = METHOD == M_TSIT5 ? Tsit5::order : Ros34pw2::order;
   constexpr int qerr = METHOD == M_TSIT5 ? Tsit5::err_order : Ros34pw2::err_order;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  R* stage = nullptr;
-  const int lane = threadIdx.x & 31;
-  if (REC) {
-    const int warp = threadIdx.x >> 5;
-    stage = reinterpret_cast<R*>(smem_raw) + (size_t)warp * 32 * L::STAGE_STRIDE;
-  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // shared memory: [record staging, REC only][start-up ring of this block's warps]
+  R* stage = REC ? reinterpret_cast<R*>(smem_raw) + (size_t)warp * 32 * L::STAGE_STRIDE : nullptr;
   R* mystage = REC ? stage + lane * L::STAGE_STRIDE : nullptr;
+  StartRing<F, R>* ring =
+      reinterpret_cast<StartRing<F, R>*>(smem_raw + (REC ? solve_stage_bytes<F, R>() : 0)) + warp;
 
   const R expo = R(-1.0 / double(qerr));
   const R eps = eps_of<R>();
   const R span = fabs(p.t1 - p.t0);
 
-  int k = -1;           // current trajectory, -1 when the lane needs work
-  bool alive = true;    // false once the work counter is exhausted for this lane
+  int k = -1;                 // current trajectory, -1 when the lane needs work
+  int head = 0, tail = 0;     // this warp's start-up ring (warp-uniform)
+  int cnext = 0, cend = 0;    // this warp's reserved record chunks [cnext, cend) (warp-uniform)
+  bool exhausted = false;     // the work counter has run past N (warp-uniform)
   R t = R(0), h = R(0);
   R y[D], k1[D];
   typename F::template Theta<R> th;
@@ -167,36 +189,69 @@ __global__ void __launch_bounds__(128, Tune<F, R>::solve_blocks) k_solve(SolvePa
   for (int c = 0; c < D; ++c) { y[c] = R(0); k1[c] = R(0); }
 
   for (;;) {
-    // ---- refill retired lanes
-    const bool need = alive && k < 0;
-    if (__any_sync(FULL, need)) {
-      const int id = warp_take(need, p.queue);
-      if (need) {
-        if (id < p.N) {
-          k = id;
-          F::load(th, p.theta + (size_t)p.theta_stride * k);
-#pragma unroll
-          for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
-          t = p.t0;
-          S = 0; Rj = 0; att = 0; last_rej = false; ns = 0; seq = 0;
-        } else {
-          alive = false;
-        }
-      }
-      // start-up of the newly taken trajectories: f(y0), finiteness, starting step
-      if (need && k >= 0) {
+    // ---- refill retired lanes from the warp's start-up ring.  When the ring cannot serve every
+    // lane that needs work, the whole warp takes the next 32 trajectories from the work counter
+    // and runs their start-up (f(y0), finiteness, starting step) together, one per lane -- so
+    // that start-up is paid once per 32 trajectories instead of stalling the warp on one lane.
+    const bool need = k < 0 && !(exhausted && head == tail);
+    const unsigned nm = __ballot_sync(FULL, need);
+    if (nm) {
+      const int want = __popc(nm);
+      if (!exhausted && tail - head < want) {
+        int base = 0;
+        if (lane == 0) base = atomicAdd(p.queue, 32);
+        base = __shfl_sync(FULL, base, 0);
+        if (base + 32 >= p.N) exhausted = true;
+        const int id = base + lane;
+        const bool valid = id < p.N;
         int st = -1;
-        if (!(p.t1 > p.t0)) {
-          st = 0;
-        } else {
-          F::f(y, th, k1);
-          bool finite = true;
+        R h0 = R(0), f0[D];
 #pragma unroll
-          for (int c = 0; c < D; ++c) finite = finite && isfinite(y[c]) && isfinite(k1[c]);
-          if (!finite) st = 3;
-          else h = initial_step<F, R>(y, k1, th, p.t0, p.t1, p.rtol, p.atol, order);
+        for (int c = 0; c < D; ++c) f0[c] = R(0);
+        if (valid) {
+          typename F::template Theta<R> th0;
+          F::load(th0, p.theta + (size_t)p.theta_stride * id);
+          R yy[D];
+#pragma unroll
+          for (int c = 0; c < D; ++c) yy[c] = p.y0[(size_t)id * D + c];
+          if (!(p.t1 > p.t0)) {
+            st = 0;
+          } else {
+            F::f(yy, th0, f0);
+            bool finite = true;
+#pragma unroll
+            for (int c = 0; c < D; ++c) finite = finite && isfinite(yy[c]) && isfinite(f0[c]);
+            if (!finite) st = 3;
+            else h0 = initial_step<F, R>(yy, f0, th0, p.t0, p.t1, p.rtol, p.atol, order);
+          }
         }
-        if (st >= 0) {
+        const unsigned vm = __ballot_sync(FULL, valid);
+        if (valid) {
+          const int slot = (tail + __popc(vm & lanemask_lt())) & (START_RING - 1);
+          ring->id[slot] = id;
+          ring->st[slot] = st;
+          ring->h0[slot] = h0;
+#pragma unroll
+          for (int c = 0; c < D; ++c) ring->f0[c][slot] = f0[c];
+        }
+        tail += __popc(vm);
+        __syncwarp();
+      }
+      const int avail = tail - head;
+      const int rank = __popc(nm & lanemask_lt());
+      if (need && rank < avail) {
+        const int slot = (head + rank) & (START_RING - 1);
+        k = ring->id[slot];
+        const int st = ring->st[slot];
+        h = ring->h0[slot];
+#pragma unroll
+        for (int c = 0; c < D; ++c) k1[c] = ring->f0[c][slot];
+        F::load(th, p.theta + (size_t)p.theta_stride * k);
+#pragma unroll
+        for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
+        t = p.t0;
+        S = 0; Rj = 0; att = 0; last_rej = false; ns = 0; seq = 0;
+        if (st >= 0) {  // finished at start-up: empty interval or non-finite y0 / f(y0)
 #pragma unroll
           for (int c = 0; c < D; ++c) p.y1[(size_t)k * D + c] = y[c];
           if (p.nsteps) p.nsteps[k] = 0;
@@ -205,8 +260,10 @@ __global__ void __launch_bounds__(128, Tune<F, R>::solve_blocks) k_solve(SolvePa
           k = -1;
         }
       }
+      head += want < avail ? want : avail;
+      __syncwarp();
     }
-    if (!__any_sync(FULL, k >= 0 || alive)) break;
+    if (!__any_sync(FULL, k >= 0) && exhausted && head == tail) break;
 
     // ---- one attempted step per active lane
     bool finishing = false;
@@ -281,11 +338,22 @@ __global__ void __launch_bounds__(128, Tune<F, R>::solve_blocks) k_solve(SolvePa
       const int owner = finishing ? fin_traj : k;
       unsigned fm = __ballot_sync(FULL, want);
       if (fm) {
-        const int leader = __ffs(fm) - 1;
-        int base = 0;
-        if (lane == leader) base = atomicAdd(p.chunk_count, __popc(fm));
-        base = __shfl_sync(FULL, base, leader);
-        const int mychunk = base + __popc(fm & lanemask_lt());
+        // chunks come from this warp's reserved block; a new block of CHUNK_BATCH is reserved
+        // from the global bump counter only when the current one runs out
+        const int nwant = __popc(fm), rank = __popc(fm & lanemask_lt());
+        const int avail = cend - cnext;
+        int mychunk;
+        if (nwant > avail) {
+          int nb = 0;
+          if (lane == 0) nb = atomicAdd(p.chunk_count, CHUNK_BATCH);
+          nb = __shfl_sync(FULL, nb, 0);
+          mychunk = rank < avail ? cnext + rank : nb + (rank - avail);
+          cnext = nb + (nwant - avail);
+          cend = nb + CHUNK_BATCH;
+        } else {
+          mychunk = cnext + rank;
+          cnext += nwant;
+        }
         if (want) {
           if (mychunk < p.pool_chunks) {
             p.chunk_traj[mychunk] = owner;
@@ -311,6 +379,10 @@ __global__ void __launch_bounds__(128, Tune<F, R>::solve_blocks) k_solve(SolvePa
       }
     }
   }
+  // chunks reserved but never filled are marked unused for the chunk-table pass
+  if (REC)
+    for (int c = cnext + lane; c < cend; c += 32)
+      if (c < p.pool_chunks) p.chunk_traj[c] = -1;
 }
 
 template <class R>
@@ -550,11 +622,14 @@ __global__ void k_scan_add(long long* out, int N, const long long* tile_base,
   if (i == 0) out[N] = *grand;
 }
 
-// chunk_table[choff[traj] + seq] = chunk
+// chunk_table[choff[traj] + seq] = chunk (reserved-but-unused chunks carry traj = -1)
 __global__ void k_chunk_table(const int* chunk_traj, const int* chunk_seq, int nchunks,
                               const long long* choff, int* table) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c < nchunks) table[choff[chunk_traj[c]] + chunk_seq[c]] = c;
+  if (c < nchunks) {
+    const int k = chunk_traj[c];
+    if (k >= 0) table[choff[k] + chunk_seq[c]] = c;
+  }
 }
 
 // max over S (int), via warp reduce + atomicMax

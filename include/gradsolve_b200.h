@@ -88,7 +88,8 @@ typedef struct {
   int32_t chunk_steps;      /* C: steps per pool chunk */
   int32_t entry_reals;      /* E = 2 + d: reals per recorded step (t_n, h_n, y_n[0..d-1]) */
   int32_t dtype;
-  int64_t nchunks;          /* chunks in use */
+  int64_t nchunks;          /* chunks handed out from the pool (a few may be reserved but
+                               unused; the chunk table lists the used ones) */
   int64_t pool_bytes;       /* device bytes of the step pool */
   /* device pointers owned by the record */
   const int32_t* nsteps;        /* [N] accepted steps S_k */
