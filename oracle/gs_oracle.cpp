@@ -138,6 +138,51 @@ int grad_impl(const ReplayArgs& a) {
   return 0;
 }
 
+struct OutArgs {
+  int method;
+  long long N;
+  int theta_shared;
+  const void* theta;
+  const void* y0;
+  const void* T;
+  const void* H;
+  const int* S;
+  int Smax;
+  double t1;
+  int J;
+  const void* tau;
+  const void* lam;   // [N][J][D] (gradient only)
+  void* out;         // [N][J][D] (outputs only)
+  void* dL_dy0;
+  void* dL_dth;
+  int nthreads;
+};
+
+template <class F, class R>
+int outputs_impl(const OutArgs& a, bool grad) {
+  constexpr int D = F::D, M = F::M;
+  const R* th = static_cast<const R*>(a.theta);
+  const R* y0 = static_cast<const R*>(a.y0);
+  const R* Tm = static_cast<const R*>(a.T);
+  const R* H = static_cast<const R*>(a.H);
+  const R* tau = static_cast<const R*>(a.tau);
+  parallel_for(a.N, a.nthreads, [&](long long k) {
+    const R* thk = th + (a.theta_shared ? 0 : k * M);
+    const size_t off = (size_t)k * a.Smax;
+    if (!grad) {
+      replay_outputs<F, R>(Method(a.method), y0 + k * D, thk, Tm + off, H + off, a.S[k], R(a.t1),
+                           a.J, tau, static_cast<R*>(a.out) + (size_t)k * a.J * D);
+    } else {
+      R* gy = a.dL_dy0 ? static_cast<R*>(a.dL_dy0) + k * D : nullptr;
+      R* gt = a.dL_dth ? static_cast<R*>(a.dL_dth) + k * M : nullptr;
+      replay_outputs_grad<F, R>(Method(a.method), y0 + k * D, thk, Tm + off, H + off, a.S[k],
+                                R(a.t1), a.J, tau,
+                                static_cast<const R*>(a.lam) + (size_t)k * a.J * D, gy, gt);
+    }
+  });
+  return 0;
+}
+
 // Field dispatch: calls fn.template operator()<F>() for the field id; -2 if unknown.
 template <class Fn>
 int with_field(int field, Fn&& fn) {
@@ -210,6 +255,36 @@ int orc_replay_grad(int field, int method, int dtype, long long N, int theta_sha
     using F = decltype(fld);
     if (!method_ok<F>(method)) return -3;
     return dtype == 0 ? grad_impl<F, double>(a) : dtype == 1 ? grad_impl<F, float>(a) : -4;
+  });
+}
+
+// States at requested times tau[J] (ascending, in [t0, t1]) over the padded record (T, H, S):
+// out [N][J][D]; and the gradient of sum_j lam_j . y(tau_j) (lam [N][J][D]).
+int orc_replay_outputs(int field, int method, int dtype, long long N, int theta_shared,
+                       const void* theta, const void* y0, const void* T, const void* H,
+                       const int* S, int Smax, double t1, int J, const void* tau, void* out,
+                       int nthreads) {
+  OutArgs a{method, N, theta_shared, theta, y0, T, H, S, Smax, t1, J, tau, nullptr, out,
+            nullptr, nullptr, nthreads};
+  return with_field(field, [&](auto fld) {
+    using F = decltype(fld);
+    if (!method_ok<F>(method)) return -3;
+    return dtype == 0 ? outputs_impl<F, double>(a, false)
+                      : dtype == 1 ? outputs_impl<F, float>(a, false) : -4;
+  });
+}
+
+int orc_replay_outputs_grad(int field, int method, int dtype, long long N, int theta_shared,
+                            const void* theta, const void* y0, const void* T, const void* H,
+                            const int* S, int Smax, double t1, int J, const void* tau,
+                            const void* lam, void* dL_dy0, void* dL_dth, int nthreads) {
+  OutArgs a{method, N, theta_shared, theta, y0, T, H, S, Smax, t1, J, tau, lam, nullptr,
+            dL_dy0, dL_dth, nthreads};
+  return with_field(field, [&](auto fld) {
+    using F = decltype(fld);
+    if (!method_ok<F>(method)) return -3;
+    return dtype == 0 ? outputs_impl<F, double>(a, true)
+                      : dtype == 1 ? outputs_impl<F, float>(a, true) : -4;
   });
 }
 

@@ -606,4 +606,79 @@ void replay_grad(Method method, const R* y0, const R* th, const R* H, int S, con
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// Outputs at requested times ([GS] §3.4: the replay takes one extra solver step from the
+// preceding mesh point exactly to each requested time, so the state is integrated, not
+// interpolated).  Reading: for tau_j (ascending, t0 <= tau_j <= t1) the preceding mesh point is
+// the last recorded t_n with t_n <= tau_j and tau_j < t_{n+1} (t_S = t1); the output is
+// Phi(y_n, tau_j - t_n), and tau_j = t1 gives y_S.  Tm holds the recorded start times t_n.
+// ------------------------------------------------------------------------------------------
+template <class F, class T>
+void one_step(Method method, const T* y, const T* th, T h, T* ynew) {
+  constexpr int D = F::D;
+  if (method == TSIT5) {
+    T k1[D];
+    F::f(y, th, k1);
+    tsit5_trial<F, T>(y, h, th, k1, ynew, nullptr, nullptr, false);
+  } else {
+    if constexpr (has_jac<F>::value) ros_trial<F, T>(y, h, th, ynew, nullptr, false);
+  }
+}
+
+template <class F, class T>
+void replay_outputs(Method method, const T* y0, const T* th,
+                    const typename base_of<T>::type* Tm, const typename base_of<T>::type* H,
+                    int S, typename base_of<T>::type t1, int J,
+                    const typename base_of<T>::type* tau, T* out) {
+  using R = typename base_of<T>::type;
+  constexpr int D = F::D;
+  T y[D];
+  for (int c = 0; c < D; ++c) y[c] = y0[c];
+  int j = 0;
+  for (int n = 0; n < S; ++n) {
+    const R tnext = (n + 1 < S) ? Tm[n + 1] : t1;
+    while (j < J && tau[j] < tnext) {
+      one_step<F, T>(method, y, th, T(tau[j] - Tm[n]), out + (size_t)j * D);
+      ++j;
+    }
+    T ynew[D];
+    one_step<F, T>(method, y, th, T(H[n]), ynew);
+    for (int c = 0; c < D; ++c) y[c] = ynew[c];
+  }
+  for (; j < J; ++j)
+    for (int c = 0; c < D; ++c) out[(size_t)j * D + c] = y[c];
+}
+
+// Gradient of L = sum_j lam_j . y(tau_j) by its plain definition: forward-mode duals through
+// replay_outputs, contracted with the output cotangents lam [J][D].
+template <class F, class R>
+void replay_outputs_grad(Method method, const R* y0, const R* th, const R* Tm, const R* H, int S,
+                         R t1, int J, const R* tau, const R* lam, R* dL_dy0, R* dL_dth) {
+  constexpr int D = F::D, M = F::M, P = 16;
+  using T = Dual<R, P>;
+  const int ninputs = D + M;
+  std::vector<T> thd(M), out((size_t)J * D);
+  for (int base = 0; base < ninputs; base += P) {
+    T yd[D];
+    for (int c = 0; c < D; ++c) {
+      yd[c] = T(y0[c]);
+      const int dir = c - base;
+      if (dir >= 0 && dir < P) yd[c].g[dir] = R(1);
+    }
+    for (int i = 0; i < M; ++i) {
+      thd[i] = T(th[i]);
+      const int dir = D + i - base;
+      if (dir >= 0 && dir < P) thd[i].g[dir] = R(1);
+    }
+    replay_outputs<F, T>(method, yd, thd.data(), Tm, H, S, t1, J, tau, out.data());
+    for (int dir = 0; dir < P && base + dir < ninputs; ++dir) {
+      R s = R(0);
+      for (int q = 0; q < J * D; ++q) s = s + lam[q] * out[q].g[dir];
+      const int idx = base + dir;
+      if (idx < D) { if (dL_dy0) dL_dy0[idx] = s; }
+      else if (dL_dth) dL_dth[idx - D] = s;
+    }
+  }
+}
+
 }  // namespace orc

@@ -33,6 +33,9 @@ def lib():
                                 vp, vp, vp, i]
         L.orc_replay.argtypes = [i, i, i, ll, i, vp, vp, vp, vp, i, vp, i]
         L.orc_replay_grad.argtypes = [i, i, i, ll, i, vp, vp, vp, vp, i, vp, vp, vp, i]
+        L.orc_replay_outputs.argtypes = [i, i, i, ll, i, vp, vp, vp, vp, vp, i, d, i, vp, vp, i]
+        L.orc_replay_outputs_grad.argtypes = [i, i, i, ll, i, vp, vp, vp, vp, vp, i, d, i, vp, vp,
+                                              vp, vp, i]
         L.orc_rhs.argtypes = [i, ll, i, vp, vp, vp]
         L.orc_jac.argtypes = [i, ll, i, vp, vp, vp]
         L.orc_trial.argtypes = [i, i, vp, vp, d, vp, vp]
@@ -126,6 +129,42 @@ def replay_grad(field, method, theta, y0, H, S, lam, dtype=np.float64, theta_sha
     rc = lib().orc_replay_grad(FIELDS[field], METHODS[method], _dt(dtype), N, int(theta_shared),
                                _p(theta), _p(y0), _p(H), _p(S), H.shape[1], _p(lam), _p(gy),
                                _p(gt), nthreads)
+    assert rc == 0, rc
+    return gy, gt
+
+
+def replay_outputs(field, method, theta, y0, T, H, S, t1, tau, dtype=np.float64,
+                   theta_shared=False, nthreads=1):
+    """States at requested times tau (ascending, in [t0, t1]): one extra step from the preceding
+    recorded mesh point to each tau ([GS] §3.4).  Returns [N, J, D]."""
+    D, M, N, theta, y0 = _prep(field, theta, y0, dtype, theta_shared)
+    T = np.ascontiguousarray(T, dtype=dtype).reshape(N, -1)
+    H = np.ascontiguousarray(H, dtype=dtype).reshape(N, -1)
+    S = np.ascontiguousarray(S, dtype=np.int32)
+    tau = np.ascontiguousarray(tau, dtype=dtype)
+    out = np.zeros((N, len(tau), D), dtype)
+    rc = lib().orc_replay_outputs(FIELDS[field], METHODS[method], _dt(dtype), N,
+                                  int(theta_shared), _p(theta), _p(y0), _p(T), _p(H), _p(S),
+                                  H.shape[1], t1, len(tau), _p(tau), _p(out), nthreads)
+    assert rc == 0, rc
+    return out
+
+
+def replay_outputs_grad(field, method, theta, y0, T, H, S, t1, tau, lam, dtype=np.float64,
+                        theta_shared=False, nthreads=1):
+    """(dL/dy0 [N, D], dL/dtheta [N, M]) of L = sum_k sum_j lam[k, j] . y_k(tau_j)."""
+    D, M, N, theta, y0 = _prep(field, theta, y0, dtype, theta_shared)
+    T = np.ascontiguousarray(T, dtype=dtype).reshape(N, -1)
+    H = np.ascontiguousarray(H, dtype=dtype).reshape(N, -1)
+    S = np.ascontiguousarray(S, dtype=np.int32)
+    tau = np.ascontiguousarray(tau, dtype=dtype)
+    lam = np.ascontiguousarray(lam, dtype=dtype).reshape(N, len(tau), D)
+    gy = np.zeros((N, D), dtype)
+    gt = np.zeros((N, M), dtype)
+    rc = lib().orc_replay_outputs_grad(FIELDS[field], METHODS[method], _dt(dtype), N,
+                                       int(theta_shared), _p(theta), _p(y0), _p(T), _p(H),
+                                       _p(S), H.shape[1], t1, len(tau), _p(tau), _p(lam), _p(gy),
+                                       _p(gt), nthreads)
     assert rc == 0, rc
     return gy, gt
 
