@@ -31,11 +31,15 @@ UNIT = "traj/s"
 # mul, fma = 2, div, sqrt, log1p each counted as one operation), and per attempted step of the
 # forward solve: counted from the definitions of the Tsit5 replay step, its reverse sweep and the
 # field's f and vector-Jacobian product (tests/test_flop_counts.py re-derives these numbers).
-FLOPS_ADJOINT_STEP = {"nfw_mn": 1254}
-FLOPS_FORWARD_ATTEMPT = {"nfw_mn": 611}
+FLOPS_ADJOINT_STEP = {"nfw_mn": 1254, "lorenz63": 432, "lotka_volterra": 344, "mlp": 48400}
+FLOPS_FORWARD_ATTEMPT = {"nfw_mn": 611, "lorenz63": 254, "lotka_volterra": 181, "mlp": 16425}
+# The MLP field (4-32-32-4, tanh) counted by hand: f = 1,280 multiply-adds + 68 bias adds + 64
+# tanh = 2,692 ops; its pullback = the two transposed products (2 x 1,280 flops), the weight
+# outer products (2 x 1,280), 2 x 64 for tanh' and 68 bias cotangents = 5,316 ops; per accepted
+# step 88 d + 6 c_f + 6 c_v = 48,400 (FP32), per attempt 67 d + 6 c_f + 5 = 16,425.
 # FP64 peak: 148 SMs x 64 FP64 FMA lanes/SM/clk x 2 flop x clock (1965 MHz max) = 37.2 TFLOP/s,
 # the datasheet FP64 figure of B200; the same formula at the measured SM clock is reported too.
-SMS, FP64_LANES = 148, 64
+SMS, FP64_LANES, FP32_LANES = 148, 64, 128
 # DRAM bytes (read + write) per accepted step, from one ncu capture of each kernel on the
 # 2^18-trajectory case of this workload; both kernels move a fixed number of bytes per accepted
 # step, so a launch's traffic is this times its accepted steps.  Record kernel: 64 B of record
@@ -48,7 +52,11 @@ LAUNCHES_PER_STEP = 16
 
 
 def fp64_peak_tflops(mhz):
-    return SMS * FP64_LANES * 2 * mhz * 1e6 / 1e12
+    return pipe_peak_tflops(mhz, FP64_LANES)
+
+
+def pipe_peak_tflops(mhz, lanes):
+    return SMS * lanes * 2 * mhz * 1e6 / 1e12
 
 
 class ClockSampler:
@@ -103,13 +111,25 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def workload_config(ws, N=1 << 20):
-    return {"workload": "nfw_mn stellar orbits: NFW halo + Miyamoto-Nagai disk, N=%d per GPU, "
-                        "d=6, m=5 per trajectory, fp64, Tsit5 rtol=1e-8 atol=1e-10, t=[0,20]; "
-                        "step = record + loss cotangent + replay gradient" % N,
+DESCR = {"nfw_mn": "stellar orbits: NFW halo + Miyamoto-Nagai disk",
+         "nfw_mn_f32": "stellar orbits: NFW halo + Miyamoto-Nagai disk",
+         "lorenz63": "Lorenz-63", "lotka_volterra": "Lotka-Volterra",
+         "robertson": "Robertson kinetics (stiff)", "mlp": "neural RHS 4-32-32-4 tanh, shared weights"}
+
+
+def workload_config(ws, N=1 << 20, name="nfw_mn", w=None):
+    if w is None:
+        spec = "d=6, m=5 per trajectory, fp64, Tsit5 rtol=1e-8 atol=1e-10, t=[0,20]"
+    else:
+        spec = "d=%d, m=%d %s, %s, %s rtol=%g atol=%g, t=[%g,%g]" % (
+            w.d, w.m, "shared" if w.theta_shared else "per trajectory",
+            "fp64" if w.dtype == np.float64 else "fp32", w.method, w.rtol, w.atol, w.t0, w.t1)
+    return {"workload": "%s %s, N=%d per GPU, %s; step = record + loss cotangent + replay "
+                        "gradient" % (name, DESCR[name], N, spec),
             "global_batch": ws * N,
             "parallelism": "independent trajectories, %d rank(s)" % ws,
-            "l2": "inputs larger than L2 (the record is ~9 GB at 2^20)"}
+            "l2": "inputs larger than L2 (the record is several GB)" if name.startswith("nfw")
+                  else "record size reported in record_gb"}
 
 
 def dist_env():
@@ -128,15 +148,19 @@ def run_reference(args):
     from oracle import oracle as orc
     nthreads = orc.host_threads()
     n_sample = args.ref_sample
-    w = W.nfw_mn(N=n_sample)
+    w_full = W.by_name(args.workload)
+    w = W.by_name(args.workload, N=n_sample)
     lam = None
     times = []
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
         r = orc.solve(w.field, w.method, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol,
-                      keep_record=True, nthreads=nthreads)
-        lam = W.loss_cotangent(w, r["y1"], w.target)
-        orc.replay_grad(w.field, w.method, w.theta, w.y0, r["H"], r["S"], lam, nthreads=nthreads)
+                      keep_record=True, nthreads=nthreads, dtype=w.dtype,
+                      theta_shared=w.theta_shared)
+        tgt = w.target if w.target is not None else np.zeros_like(r["y1"])
+        lam = W.loss_cotangent(w, r["y1"], tgt)
+        orc.replay_grad(w.field, w.method, w.theta, w.y0, r["H"], r["S"], lam, nthreads=nthreads,
+                        dtype=w.dtype, theta_shared=w.theta_shared)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             times.append(dt)
@@ -144,12 +168,13 @@ def run_reference(args):
     v = n_sample / t
     line = {"metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic",
-            "config": dict(workload_config(1), sample="%d trajectories per step" % n_sample),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64" if w.dtype == np.float64 else "f32", "data": "synthetic",
+            "config": dict(workload_config(1, w_full.N, args.workload, w_full),
+                           sample="%d trajectories per step" % n_sample),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": nthreads, "kind": "oracle",
-                             "sample": "%d trajectories of the 2^20 ensemble per step: record "
-                                       "solve + replay gradient" % n_sample},
+                             "sample": "%d trajectories of the %s ensemble per step: record "
+                                       "solve + replay gradient" % (n_sample, args.workload)},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -175,13 +200,29 @@ def cpu_baseline_sample(seconds_target=15.0):
         n *= 2
 
 
+# Per-workload constants: the field/method, the FP pipe that bounds the hot kernels and the
+# algorithmic operations per unit (counted from the definitions; see the constants above).
+WORKLOADS = {
+    "nfw_mn": dict(dtype="f64", fwd=FLOPS_FORWARD_ATTEMPT["nfw_mn"], adj=FLOPS_ADJOINT_STEP["nfw_mn"]),
+    "nfw_mn_f32": dict(dtype="f32", fwd=FLOPS_FORWARD_ATTEMPT["nfw_mn"],
+                       adj=FLOPS_ADJOINT_STEP["nfw_mn"]),
+    "lorenz63": dict(dtype="f64", fwd=FLOPS_FORWARD_ATTEMPT["lorenz63"],
+                     adj=FLOPS_ADJOINT_STEP["lorenz63"]),
+    "lotka_volterra": dict(dtype="f64", fwd=FLOPS_FORWARD_ATTEMPT["lotka_volterra"],
+                           adj=FLOPS_ADJOINT_STEP["lotka_volterra"]),
+    "robertson": dict(dtype="f64", fwd=None, adj=None),
+    "mlp": dict(dtype="f32", fwd=FLOPS_FORWARD_ATTEMPT["mlp"], adj=FLOPS_ADJOINT_STEP["mlp"]),
+}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--N", type=int, default=1 << 20)
+    ap.add_argument("--workload", default="nfw_mn", choices=sorted(WORKLOADS))
+    ap.add_argument("--N", type=int, default=0, help="trajectories per GPU (0: the workload's)")
     ap.add_argument("--ref-sample", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -205,23 +246,42 @@ def main():
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
 
-    N = args.N
-    w = W.nfw_mn(N=N, seed=4 + 1000 * rank)
-    dt = torch.float64
+    wl = WORKLOADS[args.workload]
+    w = W.by_name(args.workload, N=args.N or None)
+    w = W.by_name(args.workload, N=w.N, seed=w.seed + 1000 * rank)   # each rank: its own ensemble
+    N, d, m = w.N, w.d, w.m
+    f64 = w.dtype == np.float64
+    dt = torch.float64 if f64 else torch.float32
+    rsz = 8 if f64 else 4
+    sys_ = G.system(w.field, w.method, "f64" if f64 else "f32", w.theta_shared)
     th = torch.as_tensor(w.theta, dtype=dt, device=dev)
     y0 = torch.as_tensor(w.y0, dtype=dt, device=dev)
-    target = torch.as_tensor(w.target, dtype=dt, device=dev)
-    mask = torch.as_tensor(w.loss_mask, dtype=dt, device=dev)
-    y1 = torch.empty((N, 6), dtype=dt, device=dev)
-    lam = torch.empty((N, 6), dtype=dt, device=dev)
-    gt = torch.empty((N, 5), dtype=dt, device=dev)
-    gy = torch.empty((N, 6), dtype=dt, device=dev)
-    sys_ = G.system("nfw_mn", "tsit5", "f64")
+    y1 = torch.empty((N, d), dtype=dt, device=dev)
+    # the caller's loss targets: drawn, or solved on the GPU at nominal / teacher parameters
+    if w.target is not None:
+        target = torch.as_tensor(w.target, dtype=dt, device=dev)
+    elif w.target_kind == "nominal_solve":
+        thn = torch.as_tensor(np.tile(w.nominal_theta, (N, 1)), dtype=dt, device=dev)
+        target = torch.empty((N, d), dtype=dt, device=dev)
+        G.gs_solve_forward(sys_, N, thn, y0, w.t0, w.t1, w.rtol, w.atol, target)
+    else:
+        thn = torch.as_tensor(w.nominal_theta, dtype=dt, device=dev)
+        target = torch.empty((N, d), dtype=dt, device=dev)
+        G.gs_solve_forward(sys_, N, thn, y0, w.t0, w.t1, w.rtol, w.atol, target)
+    mask = torch.as_tensor(w.loss_mask if w.loss_mask is not None else np.ones(d), dtype=dt,
+                           device=dev)
+    scale = 2.0 * w.loss_scale
+    lam = torch.empty((N, d), dtype=dt, device=dev)
+    gt = torch.empty((m,) if w.theta_shared else (N, m), dtype=dt, device=dev)
+    gy = torch.empty((N, d), dtype=dt, device=dev)
     rec = G.Record()
+
+    def loss_cotangent():
+        torch.mul(torch.sub(y1, target), mask, out=lam).mul_(scale)
 
     def step():
         G.gs_solve_record(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, rec=rec)
-        torch.mul(torch.sub(y1, target), mask, out=lam).mul_(2.0)     # caller's loss cotangent
+        loss_cotangent()
         G.gs_replay_grad(rec, th, lam, gt, gy)
 
     for _ in range(args.warmup):
@@ -234,8 +294,6 @@ def main():
         torch.cuda.synchronize()
 
     # ---- timed: whole steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
     adj_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     solve_ms = []
@@ -245,14 +303,12 @@ def main():
         stop = torch.cuda.Event(enable_timing=True)
         start.record(stream)
         for i in range(args.steps):
-            ev[i][0].record(stream)
             G.gs_solve_record(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, rec=rec)
             solve_ms.append(rec.info().solve_ms)     # the record kernel alone (library events)
-            torch.mul(torch.sub(y1, target), mask, out=lam).mul_(2.0)
+            loss_cotangent()
             adj_ev[i][0].record(stream)
             G.gs_replay_grad(rec, th, lam, gt, gy)
             adj_ev[i][1].record(stream)
-            ev[i][1].record(stream)
         stop.record(stream)
         barrier()
     total_ms = start.elapsed_time(stop)
@@ -286,13 +342,23 @@ def main():
     attempts = int(S.sum().item() + rj.sum().item())
     rec_ms = timeit(lambda: G.gs_solve_record(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1,
                                               rec=rec))
+    loss_cotangent()
     grad_ms = timeit(lambda: G.gs_replay_grad(rec, th, lam, gt, gy))
+    breakdown = {"forward_only": fwd_ms, "record": rec_ms, "replay_grad": grad_ms, "step": ms_step}
+    if w.field != "mlp":
+        # outputs at 8 requested times ([GS] §3.4) and the gradient of a loss on them
+        tau = [w.t0 + (w.t1 - w.t0) * (j + 1) / 8.0 for j in range(8)]
+        yout = torch.empty((N, len(tau), d), dtype=dt, device=dev)
+        lam_out = (mask.expand(N, len(tau), d) * 0.125).contiguous()
+        breakdown["outputs_8_times"] = timeit(lambda: G.gs_replay_outputs(rec, th, y0, tau, yout))
+        breakdown["replay_grad_outputs_8_times"] = timeit(
+            lambda: G.gs_replay_grad_outputs(rec, th, tau, lam_out, None, gt, gy))
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the region
     h_th = torch.as_tensor(w.theta, dtype=dt).pin_memory()
     h_y0 = torch.as_tensor(w.y0, dtype=dt).pin_memory()
-    h_gt = torch.empty((N, 5), dtype=dt).pin_memory()
-    h_gy = torch.empty((N, 6), dtype=dt).pin_memory()
+    h_gt = torch.empty(tuple(gt.shape), dtype=dt).pin_memory()
+    h_gy = torch.empty((N, d), dtype=dt).pin_memory()
     e2e_steps = max(3, args.steps // 2)
     barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -310,54 +376,57 @@ def main():
         t = torch.tensor([e2e_ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e_ms = float(t.item())
-    h2d = (h_th.numel() + h_y0.numel()) * 8
-    d2h = (h_gt.numel() + h_gy.numel()) * 8
+    h2d = (h_th.numel() + h_y0.numel()) * rsz
+    d2h = (h_gt.numel() + h_gy.numel()) * rsz
 
     clocks = clk.summary()
-    peak_max = fp64_peak_tflops(1965.0)
-    at_clock = fp64_peak_tflops(clocks["sm_mhz"]) if clocks.get("sm_mhz") else None
+    lanes = FP64_LANES if f64 else FP32_LANES
+    peak_max = pipe_peak_tflops(1965.0, lanes)
+    at_clock = pipe_peak_tflops(clocks["sm_mhz"], lanes) if clocks.get("sm_mhz") else None
+    pipe = "FP64" if f64 else "FP32"
 
-    def roof(name, flops, ms, per_unit, unit_name, traffic):
-        achieved = flops / (ms / 1e3) / 1e12
+    def roof(name, per_unit, units, ms, unit_name, traffic):
+        achieved = per_unit * units / (ms / 1e3) / 1e12 if per_unit else None
         return {"kernel": name, "bound": "alu", "achieved": achieved, "peak": peak_max,
-                "unit": "TFLOP/s", "frac": achieved / peak_max, "traffic": traffic,
+                "unit": "TFLOP/s", "frac": achieved / peak_max if achieved else None,
+                "traffic": traffic,
                 "traffic_source": "ncu dram bytes per accepted step on the 2^18 case x steps",
-                "peak_source": "derived: 148 SM x 64 FP64 FMA/clk x 2 x 1965 MHz (FP64 pipe)",
+                "peak_source": "derived: 148 SM x %d %s FMA lanes/clk x 2 x 1965 MHz (%s pipe)"
+                               % (lanes, pipe, pipe),
                 "flops_per_unit": per_unit, "unit_counted": unit_name, "kernel_ms": ms,
-                "frac_at_measured_clock": achieved / at_clock if at_clock else None}
+                "frac_at_measured_clock": achieved / at_clock if (achieved and at_clock) else None}
 
-    rec_ms = statistics.median(solve_ms)
-    roof_rec = roof("k_solve<NfwMiyamotoNagai, double, Tsit5, record>",
-                    attempts * FLOPS_FORWARD_ATTEMPT["nfw_mn"], rec_ms,
-                    FLOPS_FORWARD_ATTEMPT["nfw_mn"], "attempted step",
-                    TRAFFIC_PER_STEP["record"] * total_steps)
-    roof_adj = roof("k_adjoint<NfwMiyamotoNagai, double, Tsit5>",
-                    total_steps * FLOPS_ADJOINT_STEP["nfw_mn"], adj_ms,
-                    FLOPS_ADJOINT_STEP["nfw_mn"], "accepted step",
-                    TRAFFIC_PER_STEP["adjoint"] * total_steps)
-    dominant, other = (roof_rec, roof_adj) if rec_ms >= adj_ms else (roof_adj, roof_rec)
+    method = "Tsit5" if w.method == "tsit5" else "ROS34PW2"
+    rec_kernel_ms = statistics.median(solve_ms)
+    traffic = TRAFFIC_PER_STEP if args.workload == "nfw_mn" else {}
+    roof_rec = roof("k_solve<%s, %s, %s, record>" % (w.field, "double" if f64 else "float", method),
+                    wl["fwd"], attempts, rec_kernel_ms, "attempted step",
+                    traffic.get("record", 0) * total_steps or None)
+    roof_adj = roof("k_adjoint<%s, %s, %s>" % (w.field, "double" if f64 else "float", method),
+                    wl["adj"], total_steps, adj_ms, "accepted step",
+                    traffic.get("adjoint", 0) * total_steps or None)
+    dominant, other = (roof_rec, roof_adj) if rec_kernel_ms >= adj_ms else (roof_adj, roof_rec)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": dict(workload_config(ws, N), accepted_steps=total_steps,
-                       attempts_forward=attempts,
-                       record_gb=round(info.pool_bytes / 1e9, 2)),
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64" if f64 else "f32",
+        "data": "synthetic",
+        "config": dict(workload_config(ws, N, args.workload, w), accepted_steps=total_steps,
+                       attempts_forward=attempts, record_gb=round(info.pool_bytes / 1e9, 2)),
         "roofline": dominant,
         "roofline_other": other,
-        "breakdown_ms": {"forward_only": fwd_ms, "record": rec_ms, "replay_grad": grad_ms,
-                         "step": ms_step},
+        "breakdown_ms": breakdown,
         "forward_traj_per_s": ws * N / (fwd_ms / 1e3),
         "replay_grad_traj_per_s": ws * N / (grad_ms / 1e3),
         "record_traj_per_s": ws * N / (rec_ms / 1e3),
-        "forward_fp64_frac": (attempts * FLOPS_FORWARD_ATTEMPT["nfw_mn"] / (fwd_ms / 1e3) / 1e12)
-        / peak_max,
+        "forward_pipe_frac": (wl["fwd"] * attempts / (fwd_ms / 1e3) / 1e12 / peak_max
+                              if wl["fwd"] else None),
         "e2e": {"value": ws * N / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * LAUNCHES_PER_STEP,
         "clocks": clocks,
     }
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline and args.workload == "nfw_mn":
         line["cpu_baseline"] = cpu_baseline_sample()
     else:
         line["cpu_baseline"] = None

@@ -758,6 +758,149 @@ gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, v
   return st;
 }
 
+}  // extern "C"
+
+namespace {
+
+gs_status check_out_times(const gs_record* rec, int32_t J, const double* tau) {
+  if (!rec) return fail(GS_ERR_INVALID_ARG, "record is NULL");
+  if (J < 1 || J > GS_MAX_OUTPUT_TIMES)
+    return fail(GS_ERR_INVALID_ARG, "J=%d outside [1, %d]", J, GS_MAX_OUTPUT_TIMES);
+  if (!tau) return fail(GS_ERR_INVALID_ARG, "tau is NULL");
+  for (int j = 0; j < J; ++j) {
+    if (!std::isfinite(tau[j])) return fail(GS_ERR_INVALID_ARG, "tau[%d] is not finite", j);
+    if (j > 0 && tau[j] < tau[j - 1])
+      return fail(GS_ERR_INVALID_ARG, "tau must be ascending (tau[%d] < tau[%d])", j, j - 1);
+  }
+  if (rec->sys.field == GS_MLP_4_32_32_4)
+    return fail(GS_ERR_UNSUPPORTED, "outputs at requested times are not built for the MLP field");
+  return GS_OK;
+}
+
+template <class R>
+void fill_times(gs::OutTimes<R>& ot, const gs_record* rec, int32_t J, const double* tau) {
+  ot.J = J;
+  ot.t1 = R(rec->t1);
+  for (int j = 0; j < J; ++j) ot.tau[j] = R(tau[j]);
+}
+
+template <class R>
+void fill_replay_params(gs::ReplayParams<R>& p, const gs_record* rec, const void* theta, int M,
+                        int* queue) {
+  p.N = (int)rec->N;
+  p.theta = static_cast<const R*>(theta);
+  p.theta_stride = rec->sys.theta_shared ? 0 : M;
+  p.nsteps = rec->nsteps;
+  p.choff = rec->choff;
+  p.chunk_table = rec->chunk_table;
+  p.pool = static_cast<R*>(rec->pool);
+  p.queue = queue;
+  p.perm = rec->perm;
+}
+
+}  // namespace
+
+extern "C" {
+
+gs_status gs_replay_outputs(const gs_record* rec, const void* theta, const void* y0, int32_t J,
+                            const double* tau, void* y_out, void* stream) {
+  gs_status st = check_out_times(rec, J, tau);
+  if (st != GS_OK) return st;
+  if (rec->N == 0) return GS_OK;
+  if (!theta || !y0 || !y_out)
+    return fail(GS_ERR_INVALID_ARG, "theta, y0 and y_out must be non-NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* queue = nullptr;
+  GS_CUDA(take_counter(s, &queue));
+  return dispatch(rec->sys, [&]<class F, class R, int METHOD>() {
+    if constexpr (std::is_same_v<F, gs::FMlpWarp>) {
+      return fail(GS_ERR_UNSUPPORTED, "not built for the MLP field");
+    } else {
+      gs::OutParams<R> q{};
+      fill_replay_params<R>(q.rp, rec, theta, F::M, queue);
+      q.rp.y0 = static_cast<const R*>(y0);
+      q.y_out = static_cast<R*>(y_out);
+      fill_times<R>(q.ot, rec, J, tau);
+      auto kern = gs::k_replay_outputs<F, R, METHOD>;
+      kern<<<persistent_grid(kern, 0, rec->N), BLOCK, 0, s>>>(q);
+      GS_CUDA(cudaGetLastError());
+      return GS_OK;
+    }
+  });
+}
+
+gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_t J,
+                                 const double* tau, const void* dL_dyout, const void* dL_dy1,
+                                 void* dL_dtheta, void* dL_dy0, void* stream) {
+  gs_status st = check_out_times(rec, J, tau);
+  if (st != GS_OK) return st;
+  if (rec->N == 0) return GS_OK;
+  if (!theta || !dL_dyout) return fail(GS_ERR_INVALID_ARG, "theta and dL_dyout must be non-NULL");
+  if (!dL_dtheta && !dL_dy0) return fail(GS_ERR_INVALID_ARG, "no output requested");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int M = rec->sys.m;
+  const int64_t N = rec->N;
+  const bool shared = rec->sys.theta_shared && dL_dtheta;
+  const int per_block = 4096;
+  const int nred = (int)((N + per_block - 1) / per_block);
+  gs_record* r = const_cast<gs_record*>(rec);
+  if (shared) {
+    const size_t need = (size_t)N * M * rec->rsz, needp = (size_t)nred * M * rec->rsz;
+    if (r->red_bytes < need) {
+      free_ptr(r->red_scratch);
+      r->red_scratch = nullptr;
+      r->red_bytes = 0;
+      GS_CUDA(cudaMalloc(&r->red_scratch, need));
+      r->red_bytes = need;
+    }
+    if (r->part_bytes < needp) {
+      free_ptr(r->red_partials);
+      r->red_partials = nullptr;
+      r->part_bytes = 0;
+      GS_CUDA(cudaMalloc(&r->red_partials, needp));
+      r->part_bytes = needp;
+    }
+  }
+  int* queue = nullptr;
+  GS_CUDA(take_counter(s, &queue));
+  return dispatch(rec->sys, [&]<class F, class R, int METHOD>() {
+    if constexpr (std::is_same_v<F, gs::FMlpWarp>) {
+      return fail(GS_ERR_UNSUPPORTED, "not built for the MLP field");
+    } else {
+      gs::AdjOutParams<R> q{};
+      gs::AdjointParams<R>& p = q.ap;
+      p.N = (int)N;
+      p.theta = static_cast<const R*>(theta);
+      p.theta_stride = rec->sys.theta_shared ? 0 : F::M;
+      p.dL_dy1 = static_cast<const R*>(dL_dy1);
+      p.dL_dy0 = static_cast<R*>(dL_dy0);
+      p.dL_dtheta = shared ? static_cast<R*>(r->red_scratch) : static_cast<R*>(dL_dtheta);
+      p.nsteps = rec->nsteps;
+      p.choff = rec->choff;
+      p.chunk_table = rec->chunk_table;
+      p.pool = static_cast<const R*>(rec->pool);
+      p.queue = queue;
+      p.perm = rec->perm;
+      q.dL_dyout = static_cast<const R*>(dL_dyout);
+      fill_times<R>(q.ot, rec, J, tau);
+      auto kern = gs::k_adjoint_outputs<F, R, METHOD>;
+      const size_t smem = adjoint_smem<F, R>();
+      if (smem > 48 * 1024)
+        GS_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+      kern<<<persistent_grid(kern, smem, N), BLOCK, smem, s>>>(q);
+      if (shared) {
+        gs::k_reduce_theta<R><<<nred, gs::RED_BLOCK, 0, s>>>(static_cast<const R*>(r->red_scratch),
+                                                            (int)N, M, per_block,
+                                                            static_cast<R*>(r->red_partials));
+        gs::k_reduce_partials<R><<<1, 256, 0, s>>>(static_cast<const R*>(r->red_partials), nred, M,
+                                                   static_cast<R*>(dL_dtheta));
+      }
+      GS_CUDA(cudaGetLastError());
+      return GS_OK;
+    }
+  });
+}
+
 gs_status gs_record_info(const gs_record* rec, gs_record_info_t* out) {
   if (!rec || !out) return fail(GS_ERR_INVALID_ARG, "NULL argument");
   out->N = rec->N;

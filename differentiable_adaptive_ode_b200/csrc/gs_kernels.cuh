@@ -550,6 +550,181 @@ __global__ void __launch_bounds__(128) k_replay_forward(ReplayParams<R> p) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// Outputs at requested times ("gradsolve: fast exact gradients for ODE ensembles on GPUs" §3.4:
+// one extra solver step from the preceding mesh point exactly to each requested time -- the state
+// is integrated, not interpolated).  For ascending tau_j: the output is Phi(y_n, tau_j - t_n) for
+// the first n with tau_j < t_{n+1} (t_S = t1), and y_S when tau_j >= t1.  The requested times
+// travel by value in the kernel parameters.
+// ---------------------------------------------------------------------------------------------
+constexpr int MAX_OUT = 256;
+template <class R>
+struct OutTimes {
+  int J;
+  R t1;
+  R tau[MAX_OUT];
+};
+
+template <class R>
+struct OutParams {
+  ReplayParams<R> rp;   // theta, y0, record, queue, perm (y1 unused)
+  R* y_out;             // [N][J][D]
+  OutTimes<R> ot;
+};
+
+template <class F, class R, int METHOD>
+__device__ __forceinline__ void replay_step(const R (&y)[F::D], R h,
+                                            const typename F::template Theta<R>& th,
+                                            R (&ynew)[F::D]) {
+  if constexpr (METHOD == M_TSIT5) tsit5_replay_step<F, R>(y, h, th, ynew);
+  else ros_replay_step<F, R>(y, h, th, ynew);
+}
+
+template <class F, class R>
+__device__ __forceinline__ const R* rec_entry(const ReplayParams<R>& p, long long cbase, int n) {
+  using L = RecLayout<F, R>;
+  const int ch = p.chunk_table[cbase + n / L::C];
+  return p.pool + ((size_t)ch * L::C + (n % L::C)) * L::E;
+}
+
+template <class F, class R, int METHOD>
+__global__ void __launch_bounds__(128) k_replay_outputs(OutParams<R> q) {
+  constexpr int D = F::D;
+  const ReplayParams<R>& p = q.rp;
+  const int J = q.ot.J;
+  int k = -1;
+  bool alive = true;
+  typename F::template Theta<R> th;
+  for (;;) {
+    const bool need = alive && k < 0;
+    if (__any_sync(FULL, need)) {
+      const int id = warp_take(need, p.queue);
+      if (need) {
+        if (id < p.N) k = p.perm ? p.perm[id] : id;
+        else alive = false;
+      }
+    }
+    if (!__any_sync(FULL, k >= 0 || alive)) break;
+    if (k < 0) continue;
+    F::load(th, p.theta + (size_t)p.theta_stride * k);
+    const int S = p.nsteps[k];
+    const long long cbase = p.choff[k];
+    R* out = q.y_out + (size_t)k * J * D;
+    int j = 0;
+    R y[D], t = R(0), h = R(0);
+#pragma unroll
+    for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
+    for (int n = 0; n < S && j < J; ++n) {
+      const R* e = rec_entry<F, R>(p, cbase, n);
+      t = e[0];
+      h = e[1];
+#pragma unroll
+      for (int c = 0; c < D; ++c) y[c] = e[2 + c];
+      const R tnext = (n + 1 < S) ? rec_entry<F, R>(p, cbase, n + 1)[0] : q.ot.t1;
+      while (j < J && q.ot.tau[j] < tnext) {
+        R yo[D];
+        replay_step<F, R, METHOD>(y, q.ot.tau[j] - t, th, yo);
+#pragma unroll
+        for (int c = 0; c < D; ++c) out[(size_t)j * D + c] = yo[c];
+        ++j;
+      }
+      if (j < J && n == S - 1) {  // the remaining times are at or after t1: the final state
+        R yS[D];
+        replay_step<F, R, METHOD>(y, h, th, yS);
+#pragma unroll
+        for (int c = 0; c < D; ++c) y[c] = yS[c];
+      }
+    }
+    for (; j < J; ++j)
+#pragma unroll
+      for (int c = 0; c < D; ++c) out[(size_t)j * D + c] = y[c];
+    k = -1;
+  }
+}
+
+// Replay adjoint with outputs at requested times: walking the record backwards, the cotangent
+// of each output in the window of step n is pulled back through its extra step from y_n and
+// added to the cotangent of y_n, next to the pullback of the step itself.
+template <class R>
+struct AdjOutParams {
+  AdjointParams<R> ap;  // dL_dy1 may be null here
+  const R* dL_dyout;    // [N][J][D]
+  OutTimes<R> ot;
+};
+
+template <class F, class R, int METHOD>
+__global__ void __launch_bounds__(128, Tune<F, R>::adj_blocks) k_adjoint_outputs(AdjOutParams<R> q) {
+  using L = RecLayout<F, R>;
+  constexpr int D = F::D, M = F::M;
+  extern __shared__ __align__(16) unsigned char adj_smem[];
+  R* tape = reinterpret_cast<R*>(adj_smem) + threadIdx.x;
+  const AdjointParams<R>& p = q.ap;
+  const int J = q.ot.J;
+  int jS = 0;  // outputs before t1 come from steps; the rest are the final state
+  while (jS < J && q.ot.tau[jS] < q.ot.t1) ++jS;
+  int k = -1;
+  bool alive = true;
+  typename F::template Theta<R> th;
+  for (;;) {
+    const bool need = alive && k < 0;
+    if (__any_sync(FULL, need)) {
+      const int id = warp_take(need, p.queue);
+      if (need) {
+        if (id < p.N) k = p.perm ? p.perm[id] : id;
+        else alive = false;
+      }
+    }
+    if (!__any_sync(FULL, k >= 0 || alive)) break;
+    if (k < 0) continue;
+    F::load(th, p.theta + (size_t)p.theta_stride * k);
+    const R* lo = q.dL_dyout + (size_t)k * J * D;
+    R lam[D], thb[M];
+#pragma unroll
+    for (int c = 0; c < D; ++c) lam[c] = p.dL_dy1 ? p.dL_dy1[(size_t)k * D + c] : R(0);
+#pragma unroll
+    for (int i = 0; i < M; ++i) thb[i] = R(0);
+    const int S = p.nsteps[k];
+    for (int j = (S == 0 ? 0 : jS); j < J; ++j)
+#pragma unroll
+      for (int c = 0; c < D; ++c) lam[c] += lo[(size_t)j * D + c];
+    const long long cbase = p.choff[k];
+    int jcur = S == 0 ? 0 : jS;
+    for (int n = S - 1; n >= 0; --n) {
+      const int ch = p.chunk_table[cbase + n / L::C];
+      const R* e = p.pool + ((size_t)ch * L::C + (n % L::C)) * L::E;
+      const R t = e[0], h = e[1];
+      R y[D];
+#pragma unroll
+      for (int c = 0; c < D; ++c) y[c] = e[2 + c];
+      int jlo = jcur;
+      while (jlo > 0 && (n == 0 || q.ot.tau[jlo - 1] >= t)) --jlo;
+      R lacc[D];
+#pragma unroll
+      for (int c = 0; c < D; ++c) lacc[c] = R(0);
+      for (int r = jcur - 1; r >= jlo - 1; --r) {   // r = jlo - 1 is the step itself
+        R lr[D];
+        const R hr = r >= jlo ? q.ot.tau[r] - t : h;
+#pragma unroll
+        for (int c = 0; c < D; ++c) lr[c] = r >= jlo ? lo[(size_t)r * D + c] : lam[c];
+        if constexpr (METHOD == M_TSIT5) tsit5_adjoint_step<F, R>(y, hr, th, lr, thb, tape, blockDim.x);
+        else ros_adjoint_step<F, R>(y, hr, th, lr, thb);
+#pragma unroll
+        for (int c = 0; c < D; ++c) lacc[c] += lr[c];
+      }
+#pragma unroll
+      for (int c = 0; c < D; ++c) lam[c] = lacc[c];
+      jcur = jlo;
+    }
+    if (p.dL_dy0)
+#pragma unroll
+      for (int c = 0; c < D; ++c) p.dL_dy0[(size_t)k * D + c] = lam[c];
+    if (p.dL_dtheta)
+#pragma unroll
+      for (int i = 0; i < M; ++i) p.dL_dtheta[(size_t)k * M + i] = thb[i];
+    k = -1;
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
 // Record finalisation.
 // ---------------------------------------------------------------------------------------------
 // Block-wide exclusive scan of per-trajectory counts (steps, or chunks = ceil(steps / C)).

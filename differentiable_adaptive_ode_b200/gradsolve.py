@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "GS_OK", 1: "GS_ERR_INVALID_ARG", 2: "GS_ERR_CUDA", 3: "GS_ER
 
 # every entry point declared in include/gradsolve_b200.h
 EXPORTS = ("gs_solve_forward", "gs_solve_record", "gs_replay_grad", "gs_replay_forward",
-           "gs_replay_grad_noalloc", "gs_record_info",
+           "gs_replay_grad_noalloc", "gs_replay_outputs", "gs_replay_grad_outputs", "gs_record_info",
            "gs_record_export", "gs_record_import", "gs_record_destroy", "gs_last_error",
            "gs_version")
 
@@ -75,6 +75,9 @@ def lib():
         L.gs_replay_grad.argtypes = [vp, vp, vp, vp, vp, vp]
         L.gs_replay_forward.argtypes = [vp, vp, vp, vp, vp]
         L.gs_replay_grad_noalloc.argtypes = [vp, vp, vp, vp, vp, vp]
+        pd = C.POINTER(C.c_double)
+        L.gs_replay_outputs.argtypes = [vp, vp, vp, C.c_int32, pd, vp, vp]
+        L.gs_replay_grad_outputs.argtypes = [vp, vp, C.c_int32, pd, vp, vp, vp, vp, vp]
         L.gs_record_info.argtypes = [vp, P(GsRecordInfo)]
         L.gs_record_export.argtypes = [vp, vp, vp, vp, vp, vp]
         L.gs_record_import.argtypes = [P(GsSystem), i64, vp, vp, vp, vp, P(vp), vp]
@@ -83,7 +86,8 @@ def lib():
         L.gs_last_error.restype = C.c_char_p
         L.gs_version.restype = C.c_char_p
         for name in ("gs_solve_forward", "gs_solve_record", "gs_replay_grad", "gs_replay_forward",
-                     "gs_replay_grad_noalloc", "gs_record_info",
+                     "gs_replay_grad_noalloc", "gs_replay_outputs", "gs_replay_grad_outputs",
+                     "gs_record_info",
                      "gs_record_export", "gs_record_import"):
             getattr(L, name).restype = C.c_int
         _lib = L
@@ -187,6 +191,28 @@ def gs_replay_grad_noalloc(rec, theta, dL_dy1, dL_dtheta=None, dL_dy0=None, stre
 def gs_replay_forward(rec, theta, y0, y1=None, stream=None):
     """Forward replay over the recorded mesh at theta: refreshes the stored states, fills y1."""
     _check(lib().gs_replay_forward(rec.handle, _ptr(theta), _ptr(y0), _ptr(y1), _stream(stream)))
+
+
+def _times(tau):
+    arr = (C.c_double * len(tau))(*[float(t) for t in tau])
+    return len(tau), arr
+
+
+def gs_replay_outputs(rec, theta, y0, tau, y_out, stream=None):
+    """States at the requested times tau (host sequence, ascending) into y_out [N, J, d]."""
+    J, arr = _times(tau)
+    _check(lib().gs_replay_outputs(rec.handle, _ptr(theta), _ptr(y0), J, arr, _ptr(y_out),
+                                   _stream(stream)))
+
+
+def gs_replay_grad_outputs(rec, theta, tau, dL_dyout, dL_dy1=None, dL_dtheta=None, dL_dy0=None,
+                           stream=None):
+    """Gradient of a loss on the outputs at requested times (dL_dyout [N, J, d]) and optionally
+    on the final state (dL_dy1)."""
+    J, arr = _times(tau)
+    _check(lib().gs_replay_grad_outputs(rec.handle, _ptr(theta), J, arr, _ptr(dL_dyout),
+                                        _ptr(dL_dy1), _ptr(dL_dtheta), _ptr(dL_dy0),
+                                        _stream(stream)))
 
 
 def gs_record_info(rec):

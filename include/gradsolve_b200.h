@@ -143,6 +143,26 @@ gs_status gs_replay_grad(const gs_record* rec, const void* theta, const void* dL
 gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, void* y1,
                             void* stream);
 
+/* States at requested times ([GS] §3.4: one extra solver step from the preceding mesh point
+ * exactly to each requested time -- the returned state is integrated, not interpolated).
+ * tau: HOST array of J times (1 <= J <= GS_MAX_OUTPUT_TIMES), ascending; for tau_j the output is
+ * Phi(y_n, tau_j - t_n) with n the first recorded step with tau_j < t_{n+1} (t_S = t1), and the
+ * final state for tau_j >= t1 (times before t0 are integrated backwards from y0).  Uses the
+ * record's stored states (as gs_replay_grad); y0 [N][d] (device) is the initial state, read for
+ * trajectories with no recorded step.  y_out [N][J][d] (device).  Not built for
+ * GS_MLP_4_32_32_4 (GS_ERR_UNSUPPORTED).  Asynchronous. */
+#define GS_MAX_OUTPUT_TIMES 256
+gs_status gs_replay_outputs(const gs_record* rec, const void* theta, const void* y0, int32_t J,
+                            const double* tau, void* y_out, void* stream);
+
+/* Gradient of a loss on the outputs at requested times (and optionally on the final state):
+ * dL_dyout [N][J][d] (device), dL_dy1 [N][d] (device, nullable); outputs as gs_replay_grad.
+ * Each output's cotangent is pulled back through its extra step from y_n and added to the
+ * cotangent of y_n.  Asynchronous. */
+gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_t J,
+                                 const double* tau, const void* dL_dyout, const void* dL_dy1,
+                                 void* dL_dtheta, void* dL_dy0, void* stream);
+
 /* Replay gradient that allocates no device memory.  The paper has no counterpart: this entry
  * point exists for callers that must not allocate at the moment they ask for a gradient -- code
  * that runs while a stream is being captured into a CUDA graph (allocation is not a capturable

@@ -33,14 +33,25 @@ def ops(t):
     return t["add"] + t["mul"] + t["div"] + t["sqrt"] + t["log1p"]
 
 
-def test_bench_constants_match_counts(counts):
+@pytest.mark.parametrize("field", ["nfw_mn", "lorenz63", "lotka_volterra"])
+def test_bench_constants_match_counts(counts, field):
     import bench
-    c = counts["nfw_mn"]
+    c = counts[field]
     D = c["D"]
     adj = 88 * D + 6 * ops(c["f"]) + 6 * ops(c["vjp"])
     fwd = 67 * D + 6 * ops(c["f"]) + 5
-    assert bench.FLOPS_ADJOINT_STEP["nfw_mn"] == adj
-    assert bench.FLOPS_FORWARD_ATTEMPT["nfw_mn"] == fwd
+    assert bench.FLOPS_ADJOINT_STEP[field] == adj
+    assert bench.FLOPS_FORWARD_ATTEMPT[field] == fwd
+
+
+def test_mlp_hand_count():
+    import bench
+    H, D = 32, 4
+    c_f = 2 * (H * D + H * H + D * H) + (H + H + D) + 2 * H      # products, biases, tanh
+    c_v = 2 * (D * H + H * H + H * D) + 2 * (H * H + H * D + D * H) + 2 * 2 * H + (H + H + D)
+    assert c_f == 2692 and c_v == 5316
+    assert bench.FLOPS_ADJOINT_STEP["mlp"] == 88 * D + 6 * c_f + 6 * c_v
+    assert bench.FLOPS_FORWARD_ATTEMPT["mlp"] == 67 * D + 6 * c_f + 5
 
 
 def test_field_counts_are_plausible(counts):
