@@ -288,6 +288,32 @@ int orc_replay_outputs_grad(int field, int method, int dtype, long long N, int t
   });
 }
 
+// Tangent of the replay's final state along (ydot0 [N][D], thdot [N][M] or [M]) over the padded
+// mesh: y1 [N][D], ydot1 [N][D].
+int orc_replay_jvp(int field, int method, int dtype, long long N, int theta_shared,
+                   const void* theta, const void* y0, const void* thdot, const void* ydot0,
+                   const void* H, const int* S, int Smax, void* y1, void* ydot1, int nthreads) {
+  return with_field(field, [&](auto fld) {
+    using F = decltype(fld);
+    if (!method_ok<F>(method)) return -3;
+    auto run = [&](auto zero) {
+      using R = decltype(zero);
+      constexpr int D = F::D, M = F::M;
+      const R* th = static_cast<const R*>(theta);
+      const R* td = static_cast<const R*>(thdot);
+      parallel_for(N, nthreads, [&](long long k) {
+        const long long to = theta_shared ? 0 : k * M;
+        replay_jvp<F, R>(Method(method), static_cast<const R*>(y0) + k * D, th + to,
+                         static_cast<const R*>(ydot0) + k * D, td + to,
+                         static_cast<const R*>(H) + k * (long long)Smax, S[k],
+                         static_cast<R*>(y1) + k * D, static_cast<R*>(ydot1) + k * D);
+      });
+      return 0;
+    };
+    return dtype == 0 ? run(0.0) : dtype == 1 ? run(0.0f) : -4;
+  });
+}
+
 // f(y; theta) for N states (double only; used by field-level checks).
 int orc_rhs(int field, long long N, int theta_shared, const double* theta, const double* y,
             double* out) {

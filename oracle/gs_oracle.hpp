@@ -681,4 +681,22 @@ void replay_outputs_grad(Method method, const R* y0, const R* th, const R* Tm, c
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// Forward sensitivity along a direction (forward mode through the replay, [GS] §4.4; the
+// in-kernel forward sensitivities of [DA] §2, one direction per pass): the tangent of y_S for
+// the input direction (ydot0, thdot), by one-direction dual numbers through the same chain.
+// ------------------------------------------------------------------------------------------
+template <class F, class R>
+void replay_jvp(Method method, const R* y0, const R* th, const R* ydot0, const R* thdot,
+                const R* H, int S, R* y1, R* ydot1) {
+  constexpr int D = F::D, M = F::M;
+  using T = Dual<R, 1>;
+  T yd[D];
+  std::vector<T> thd(M);
+  for (int c = 0; c < D; ++c) { yd[c] = T(y0[c]); yd[c].g[0] = ydot0[c]; }
+  for (int j = 0; j < M; ++j) { thd[j] = T(th[j]); thd[j].g[0] = thdot[j]; }
+  replay<F, T>(method, yd, thd.data(), H, S);
+  for (int c = 0; c < D; ++c) { y1[c] = yd[c].v; ydot1[c] = yd[c].g[0]; }
+}
+
 }  // namespace orc

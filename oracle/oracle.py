@@ -36,6 +36,7 @@ def lib():
         L.orc_replay_outputs.argtypes = [i, i, i, ll, i, vp, vp, vp, vp, vp, i, d, i, vp, vp, i]
         L.orc_replay_outputs_grad.argtypes = [i, i, i, ll, i, vp, vp, vp, vp, vp, i, d, i, vp, vp,
                                               vp, vp, i]
+        L.orc_replay_jvp.argtypes = [i, i, i, ll, i, vp, vp, vp, vp, vp, vp, i, vp, vp, i]
         L.orc_rhs.argtypes = [i, ll, i, vp, vp, vp]
         L.orc_jac.argtypes = [i, ll, i, vp, vp, vp]
         L.orc_trial.argtypes = [i, i, vp, vp, d, vp, vp]
@@ -167,6 +168,23 @@ def replay_outputs_grad(field, method, theta, y0, T, H, S, t1, tau, lam, dtype=n
                                        _p(gt), nthreads)
     assert rc == 0, rc
     return gy, gt
+
+
+def replay_jvp(field, method, theta, y0, thdot, ydot0, H, S, dtype=np.float64, theta_shared=False,
+               nthreads=1):
+    """(y_S, tangent of y_S along (ydot0, thdot)) over the padded mesh H (forward mode)."""
+    D, M, N, theta, y0 = _prep(field, theta, y0, dtype, theta_shared)
+    thdot = np.ascontiguousarray(thdot, dtype=dtype).reshape(theta.shape)
+    ydot0 = np.ascontiguousarray(ydot0, dtype=dtype).reshape(N, D)
+    H = np.ascontiguousarray(H, dtype=dtype).reshape(N, -1)
+    S = np.ascontiguousarray(S, dtype=np.int32)
+    y1 = np.zeros((N, D), dtype)
+    yd1 = np.zeros((N, D), dtype)
+    rc = lib().orc_replay_jvp(FIELDS[field], METHODS[method], _dt(dtype), N, int(theta_shared),
+                              _p(theta), _p(y0), _p(thdot), _p(ydot0), _p(H), _p(S), H.shape[1],
+                              _p(y1), _p(yd1), nthreads)
+    assert rc == 0, rc
+    return y1, yd1
 
 
 def rhs(field, theta, y, theta_shared=False):
