@@ -69,7 +69,7 @@ MLP_M = 1348
 @dataclass
 class Workload:
     name: str
-    field: str                 # lotka_volterra | lorenz63 | mlp | robertson | nfw_mn
+    field: str                 # lotka_volterra | lorenz63 | mlp | robertson | nfw_mn | log_halo
     method: str                # tsit5 | ros34pw2
     dtype: type                # np.float64 | np.float32
     N: int
@@ -173,9 +173,59 @@ def nfw_mn(N=1 << 20, seed=4, dtype=np.float64, theta_shared=False):
                     loss_mask=mask)
 
 
+LOG_HALO_RC = 0.2
+
+
+def log_halo_vcirc(r, vc=1.0):
+    """Circular speed v_c r / sqrt(R_c^2 + r^2) of the logarithmic halo at radius r (in the plane;
+    used as the velocity scale at any position)."""
+    return vc * r / np.sqrt(LOG_HALO_RC ** 2 + r * r)
+
+
+def log_halo_t1():
+    """3.7 circular periods 2 pi r_m / v_circ(r_m) at the median radius r_m of the shell
+    0.5 <= r <= 2 (uniform in volume): the pages' median of 3.7 orbital periods per orbit."""
+    rm = ((0.5 ** 3 + 2.0 ** 3) / 2.0) ** (1.0 / 3.0)
+    return 3.7 * 2.0 * np.pi * rm / log_halo_vcirc(rm)
+
+
+def log_halo(N=1 << 20, seed=5, dtype=np.float64):
+    """Stars in the flattened logarithmic halo, theta = (v_c, q) = (1, 0.7) shared, R_c = 0.2.
+    Positions uniform in volume in 0.5 <= r <= 2 with an isotropic direction; velocity
+    v_circ(r) (eta t + xi r_hat), t a unit vector perpendicular to r_hat at a uniform angle (orbits
+    in and out of the plane), eta ~ U(0.05, 1) (nearly radial to near-circular), xi ~ U(-0.2, 0.2).
+    rtol = atol = 3.16e-7; t in [0, 3.7 circular periods at the median radius]."""
+    x = _shell_points(seed, S_Y0, N)
+    u = uniform(seed, S_VEL, 3 * N).reshape(N, 3)
+    r = np.linalg.norm(x, axis=1)
+    rh = x / r[:, None]
+    # an orthonormal pair perpendicular to r_hat: e1 = normalise(z_hat x r_hat) (or x_hat when
+    # r_hat is along z), e2 = r_hat x e1
+    e1 = np.cross(np.array([0.0, 0.0, 1.0])[None, :], rh)
+    n1 = np.linalg.norm(e1, axis=1)
+    bad = n1 < 1e-12
+    e1[bad] = np.array([1.0, 0.0, 0.0])
+    n1[bad] = 1.0
+    e1 /= n1[:, None]
+    e2 = np.cross(rh, e1)
+    psi = 2.0 * np.pi * u[:, 0]
+    t = np.cos(psi)[:, None] * e1 + np.sin(psi)[:, None] * e2
+    eta = 0.05 + 0.95 * u[:, 1]
+    xi = -0.2 + 0.4 * u[:, 2]
+    v = log_halo_vcirc(r)[:, None] * (eta[:, None] * t + xi[:, None] * rh)
+    y0 = np.concatenate([x, v], axis=1).astype(dtype)
+    theta = np.array([1.0, 0.7], dtype)
+    target = np.zeros((N, 6))
+    target[:, :3] = _shell_points(seed, S_TARGET, N)
+    mask = np.array([1, 1, 1, 0, 0, 0], np.float64)
+    return Workload("log_halo" + ("_f32" if dtype == np.float32 else ""), "log_halo", "tsit5",
+                    dtype, N, 6, 2, True, theta, y0, 0.0, float(log_halo_t1()), 3.16e-7, 3.16e-7,
+                    seed, target=target, loss_mask=mask)
+
+
 def by_name(name: str, N: Optional[int] = None, **kw) -> Workload:
     table = {"lotka_volterra": lotka_volterra, "lorenz63": lorenz63, "mlp": mlp,
-             "robertson": robertson, "nfw_mn": nfw_mn}
+             "robertson": robertson, "nfw_mn": nfw_mn, "log_halo": log_halo}
     if name == "nfw_mn_f32":
         return nfw_mn(N=N if N else 1 << 20, dtype=np.float32, **kw)
     fn = table[name]

@@ -17,7 +17,7 @@ namespace {
 using namespace orc;
 
 enum FieldId { F_LV = 0, F_LORENZ = 1, F_MLP = 2, F_ROBERTSON = 3, F_NFW = 4, F_LIN1 = 5,
-               F_LIN2 = 6, F_LIN3 = 7 };
+               F_LIN2 = 6, F_LIN3 = 7, F_LOGHALO = 8 };
 
 template <class Fn>
 void parallel_for(long long N, int nthreads, Fn fn) {
@@ -195,6 +195,7 @@ int with_field(int field, Fn&& fn) {
     case F_LIN1: return fn(Linear<1>{});
     case F_LIN2: return fn(Linear<2>{});
     case F_LIN3: return fn(Linear<3>{});
+    case F_LOGHALO: return fn(LogHalo{});
     default: return -2;
   }
 }
@@ -311,6 +312,39 @@ int orc_replay_jvp(int field, int method, int dtype, long long N, int theta_shar
       return 0;
     };
     return dtype == 0 ? run(0.0) : dtype == 1 ? run(0.0f) : -4;
+  });
+}
+
+// Orbit plus forward sensitivities S = dy/dtheta [N][D][M] (Tsit5, control on y alone).
+// S0 [N][D][M] may be NULL (zero start, theta does not enter y0).
+int orc_solve_sens(int field, int dtype, long long N, int theta_shared, const void* theta,
+                   const void* y0, const void* S0, double t0, double t1, double rtol, double atol,
+                   long long max_attempts, void* y1, void* S1, int* S, int* rej, int* status,
+                   int nthreads) {
+  return with_field(field, [&](auto fld) {
+    using F = decltype(fld);
+    if constexpr (F::M > 16) {
+      return -3;  // the dual width is the parameter count: kept to small M
+    } else {
+      auto run = [&](auto zero) {
+        using R = decltype(zero);
+        constexpr int D = F::D, M = F::M;
+        const R* th = static_cast<const R*>(theta);
+        parallel_for(N, nthreads, [&](long long k) {
+          const R* s0 = S0 ? static_cast<const R*>(S0) + k * D * M : nullptr;
+          Record<R> r = solve_sens<F, R>(static_cast<const R*>(y0) + k * D, s0,
+                                         th + (theta_shared ? 0 : k * M), R(t0), R(t1), R(rtol),
+                                         R(atol), max_attempts,
+                                         static_cast<R*>(S1) + k * D * M);
+          for (int c = 0; c < D; ++c) static_cast<R*>(y1)[k * D + c] = r.y1[c];
+          if (S) S[k] = r.S;
+          if (rej) rej[k] = r.rejected;
+          if (status) status[k] = r.status;
+        });
+        return 0;
+      };
+      return dtype == 0 ? run(0.0) : dtype == 1 ? run(0.0f) : -4;
+    }
   });
 }
 

@@ -215,6 +215,29 @@ struct NfwMiyamotoNagai {
   }
 };
 
+// Test particle in an axisymmetric flattened logarithmic halo ([DA] §3; the same potential as
+// the halo-flattening study of [GS] §4.5):  Phi = (1/2) v_c^2 ln(R_c^2 + x^2 + y^2 + z^2/q^2),
+// state (x, y, z, vx, vy, vz), theta = (v_c, q) shared by the stars, core radius R_c = 0.2 fixed
+// (the pages' value; the two differentiated parameters are v_c and q).  -grad Phi written out:
+//   -v_c^2 (x, y, z/q^2) / (R_c^2 + x^2 + y^2 + z^2/q^2).
+struct LogHalo {
+  static constexpr int D = 6, M = 2;
+  static constexpr double Rc = 0.2;
+  template <class T> static void f(const T* y, const T* th, T* dy) {
+    const T x = y[0], yy = y[1], z = y[2];
+    const T vc = th[0], q = th[1];
+    const T zq = z / q;
+    const T Q = cst<T>(Rc * Rc) + x * x + yy * yy + zq * zq;
+    const T g = vc * vc / Q;
+    dy[0] = y[3];
+    dy[1] = y[4];
+    dy[2] = y[5];
+    dy[3] = -(g * x);
+    dy[4] = -(g * yy);
+    dy[5] = -(g * (zq / q));
+  }
+};
+
 // Neural right-hand side: f(y) = W3 tanh(W2 tanh(W1 y + b1) + b2) + b3, sizes 4 -> 32 -> 32 -> 4,
 // all layers with biases ([GS] §2.2: m runs to thousands of weights for a neural RHS).
 // Parameter vector layout (row-major, W[out][in]):
@@ -465,15 +488,18 @@ inline R rms_scaled(const R* v, const R* a, const R* b, int D, R rtol, R atol) {
   return std::sqrt(s / R(D));
 }
 
+// Dc = number of leading state components the step control sees (all of them unless a
+// sensitivity block rides along, see solve_sens).
 template <class F, class R>
-R initial_step(const R* y0, const R* f0, const R* th, R t0, R t1, R rtol, R atol, int p) {
+R initial_step(const R* y0, const R* f0, const R* th, R t0, R t1, R rtol, R atol, int p,
+               int Dc = F::D) {
   constexpr int D = F::D;
   R sc[D];
   for (int i = 0; i < D; ++i) sc[i] = atol + rtol * std::fabs(y0[i]);
   auto norm = [&](const R* v) {
     R s = R(0);
-    for (int i = 0; i < D; ++i) { R q = v[i] / sc[i]; s = s + q * q; }
-    return std::sqrt(s / R(D));
+    for (int i = 0; i < Dc; ++i) { R q = v[i] / sc[i]; s = s + q * q; }
+    return std::sqrt(s / R(Dc));
   };
   const R d0 = norm(y0), d1 = norm(f0);
   R h0 = (d0 < R(1e-5) || d1 < R(1e-5)) ? R(1e-6) : R(0.01) * d0 / d1;
@@ -490,7 +516,7 @@ R initial_step(const R* y0, const R* f0, const R* th, R t0, R t1, R rtol, R atol
 
 template <class F, class R>
 Record<R> solve(Method method, const R* y0, const R* th, R t0, R t1, R rtol, R atol,
-                long long max_attempts, bool keep_record) {
+                long long max_attempts, bool keep_record, int Dc = F::D) {
   constexpr int D = F::D;
   Record<R> rec;
   rec.y1.assign(y0, y0 + D);
@@ -498,13 +524,13 @@ Record<R> solve(Method method, const R* y0, const R* th, R t0, R t1, R rtol, R a
   for (int i = 0; i < D; ++i) y[i] = y0[i];
   if (!(t1 > t0)) return rec;  // empty interval: no step, y1 = y0
   F::f(y, th, k1);
-  for (int i = 0; i < D; ++i)
+  for (int i = 0; i < Dc; ++i)
     if (!std::isfinite(y[i]) || !std::isfinite(k1[i])) { rec.status = 3; return rec; }
   const int p = method == TSIT5 ? Tsit5Tab::order : Ros34pw2Tab::order;
   const int q = method == TSIT5 ? Tsit5Tab::err_order : Ros34pw2Tab::err_order;
   const R expo = R(-1.0 / double(q));
   const R eps = std::numeric_limits<R>::epsilon();
-  R h = initial_step<F, R>(y, k1, th, t0, t1, rtol, atol, p);
+  R h = initial_step<F, R>(y, k1, th, t0, t1, rtol, atol, p, Dc);
   R t = t0;
   bool last_rejected = false;
   while (t < t1) {
@@ -520,7 +546,7 @@ Record<R> solve(Method method, const R* y0, const R* th, R t0, R t1, R rtol, R a
     } else {
       if constexpr (has_jac<F>::value) ros_trial<F, R>(y, h, th, ynew, e, true);
     }
-    const R err = rms_scaled<R>(e, y, ynew, D, rtol, atol);
+    const R err = rms_scaled<R>(e, y, ynew, Dc, rtol, atol);
     if (err <= R(1)) {
       if (keep_record) {
         rec.t.push_back(t);
@@ -697,6 +723,51 @@ void replay_jvp(Method method, const R* y0, const R* th, const R* ydot0, const R
   for (int j = 0; j < M; ++j) { thd[j] = T(th[j]); thd[j].g[0] = thdot[j]; }
   replay<F, T>(method, yd, thd.data(), H, S);
   for (int c = 0; c < D; ++c) { y1[c] = yd[c].v; ydot1[c] = yd[c].g[0]; }
+}
+
+// ------------------------------------------------------------------------------------------
+// Forward sensitivities in the same solve ([DA] §2 and §3: the sensitivity equations integrated
+// together with the orbit, with the step size controlled on the orbit alone).  The augmented
+// state is z = (y, S), S = dy/dtheta stored row-major [D][M]; its right-hand side is
+//   (f(y; theta),  J_y(y) S + J_theta(y)),
+// the second block evaluated as the M directional derivatives of f along (S_{:,p}, e_p) with
+// M-direction dual numbers.  Reading: "controlled on the orbit alone" means that the error test,
+// the starting step and the finiteness check at the start look at the first D components only,
+// so the accepted mesh and y are those of the plain solve.
+// ------------------------------------------------------------------------------------------
+template <class F>
+struct SensAug {
+  static constexpr int D0 = F::D, M = F::M, D = F::D * (1 + F::M);
+  template <class T> static void f(const T* z, const T* th, T* dz) {
+    using DT = Dual<T, M>;
+    DT y[D0], t[M], dy[D0];
+    for (int c = 0; c < D0; ++c) {
+      y[c] = DT(z[c]);
+      for (int p = 0; p < M; ++p) y[c].g[p] = z[D0 + c * M + p];
+    }
+    for (int j = 0; j < M; ++j) { t[j] = DT(th[j]); t[j].g[j] = T(1); }
+    F::f(y, t, dy);
+    for (int c = 0; c < D0; ++c) {
+      dz[c] = dy[c].v;
+      for (int p = 0; p < M; ++p) dz[D0 + c * M + p] = dy[c].g[p];
+    }
+  }
+};
+
+template <class F, class R>
+Record<R> solve_sens(const R* y0, const R* S0, const R* th, R t0, R t1, R rtol, R atol,
+                     long long max_attempts, R* S1) {
+  constexpr int D = F::D, M = F::M;
+  using A = SensAug<F>;
+  R z0[A::D];
+  for (int c = 0; c < D; ++c) z0[c] = y0[c];
+  for (int i = 0; i < D * M; ++i) z0[D + i] = S0 ? S0[i] : R(0);
+  Record<R> za = solve<A, R>(TSIT5, z0, th, t0, t1, rtol, atol, max_attempts, false, D);
+  Record<R> rec;
+  rec.S = za.S; rec.rejected = za.rejected; rec.status = za.status; rec.attempts = za.attempts;
+  rec.y1.assign(za.y1.begin(), za.y1.begin() + D);
+  for (int i = 0; i < D * M; ++i) S1[i] = za.y1[D + i];
+  return rec;
 }
 
 }  // namespace orc

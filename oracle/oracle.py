@@ -16,7 +16,7 @@ import numpy as np
 from . import build_oracle
 
 FIELDS = {"lotka_volterra": 0, "lorenz63": 1, "mlp": 2, "robertson": 3, "nfw_mn": 4,
-          "linear1": 5, "linear2": 6, "linear3": 7}
+          "linear1": 5, "linear2": 6, "linear3": 7, "log_halo": 8}
 METHODS = {"tsit5": 0, "ros34pw2": 1}
 
 _lib = None
@@ -37,6 +37,8 @@ def lib():
         L.orc_replay_outputs_grad.argtypes = [i, i, i, ll, i, vp, vp, vp, vp, vp, i, d, i, vp, vp,
                                               vp, vp, i]
         L.orc_replay_jvp.argtypes = [i, i, i, ll, i, vp, vp, vp, vp, vp, vp, i, vp, vp, i]
+        L.orc_solve_sens.argtypes = [i, i, ll, i, vp, vp, vp, d, d, d, d, ll, vp, vp, vp, vp, vp,
+                                     i]
         L.orc_rhs.argtypes = [i, ll, i, vp, vp, vp]
         L.orc_jac.argtypes = [i, ll, i, vp, vp, vp]
         L.orc_trial.argtypes = [i, i, vp, vp, d, vp, vp]
@@ -185,6 +187,24 @@ def replay_jvp(field, method, theta, y0, thdot, ydot0, H, S, dtype=np.float64, t
                               _p(y1), _p(yd1), nthreads)
     assert rc == 0, rc
     return y1, yd1
+
+
+def solve_sens(field, theta, y0, t0, t1, rtol, atol, S0=None, dtype=np.float64,
+               theta_shared=False, max_attempts=100000, nthreads=1):
+    """Tsit5 solve of the orbit together with S = dy/dtheta [N, D, M], step control on y alone."""
+    D, M, N, theta, y0 = _prep(field, theta, y0, dtype, theta_shared)
+    if S0 is not None:
+        S0 = np.ascontiguousarray(S0, dtype=dtype).reshape(N, D, M)
+    y1 = np.zeros((N, D), dtype)
+    S1 = np.zeros((N, D, M), dtype)
+    S = np.zeros(N, np.int32)
+    rej = np.zeros(N, np.int32)
+    status = np.zeros(N, np.int32)
+    rc = lib().orc_solve_sens(FIELDS[field], _dt(dtype), N, int(theta_shared), _p(theta), _p(y0),
+                              _p(S0), t0, t1, rtol, atol, max_attempts, _p(y1), _p(S1), _p(S),
+                              _p(rej), _p(status), nthreads)
+    assert rc == 0, rc
+    return {"y1": y1, "sens": S1, "S": S, "rejected": rej, "status": status}
 
 
 def rhs(field, theta, y, theta_shared=False):
