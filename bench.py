@@ -31,8 +31,14 @@ UNIT = "traj/s"
 # mul, fma = 2, div, sqrt, log1p each counted as one operation), and per attempted step of the
 # forward solve: counted from the definitions of the Tsit5 replay step, its reverse sweep and the
 # field's f and vector-Jacobian product (tests/test_flop_counts.py re-derives these numbers).
-FLOPS_ADJOINT_STEP = {"nfw_mn": 1254, "lorenz63": 432, "lotka_volterra": 344, "mlp": 48400}
-FLOPS_FORWARD_ATTEMPT = {"nfw_mn": 611, "lorenz63": 254, "lotka_volterra": 181, "mlp": 16425}
+FLOPS_ADJOINT_STEP = {"nfw_mn": 1254, "lorenz63": 432, "lotka_volterra": 344, "mlp": 48400,
+                      "log_halo": 834}
+FLOPS_FORWARD_ATTEMPT = {"nfw_mn": 611, "lorenz63": 254, "lotka_volterra": 181, "mlp": 16425,
+                         "log_halo": 473}
+# Forward sensitivities, per accepted step and all m columns: the tangent of the Tsit5 step,
+# 48 d (stage tangents 35 d, result 13 d) + 6 c_t per column, c_t = the forward-mode rules' extra
+# operations over f (the value part that the kernel recomputes alongside is not counted).
+FLOPS_SENS_STEP = {"log_halo": 912}
 # The MLP field (4-32-32-4, tanh) counted by hand: f = 1,280 multiply-adds + 68 bias adds + 64
 # tanh = 2,692 ops; its pullback = the two transposed products (2 x 1,280 flops), the weight
 # outer products (2 x 1,280), 2 x 64 for tanh' and 68 bias cotangents = 5,316 ops; per accepted
@@ -44,7 +50,7 @@ SMS, FP64_LANES, FP32_LANES = 148, 64, 128
 # 2^18-trajectory case of this workload; both kernels move a fixed number of bytes per accepted
 # step, so a launch's traffic is this times its accepted steps.  Record kernel: 64 B of record
 # per step written plus inputs; adjoint: the 64 B entry read per step plus chunk table and inputs.
-TRAFFIC_PER_STEP = {"record": 65.85, "adjoint": 72.16}
+TRAFFIC_PER_STEP = {"record": 66.52, "adjoint": 70.77}
 # library kernels per step: record = k_solve + 2 k_max_int + 3 prefix scans of 3 kernels each
 # (step offsets, chunk offsets, length bins) + k_chunk_table + k_bin_count + k_bin_scatter (15);
 # replay gradient = k_adjoint (1).
@@ -114,22 +120,24 @@ class ClockSampler:
 DESCR = {"nfw_mn": "stellar orbits: NFW halo + Miyamoto-Nagai disk",
          "nfw_mn_f32": "stellar orbits: NFW halo + Miyamoto-Nagai disk",
          "lorenz63": "Lorenz-63", "lotka_volterra": "Lotka-Volterra",
-         "robertson": "Robertson kinetics (stiff)", "mlp": "neural RHS 4-32-32-4 tanh, shared weights"}
+         "robertson": "Robertson kinetics (stiff)", "mlp": "neural RHS 4-32-32-4 tanh, shared weights",
+         "log_halo": "stellar orbits in a flattened logarithmic halo, theta = (v_c, q) shared"}
 
 
-def workload_config(ws, N=1 << 20, name="nfw_mn", w=None):
+def workload_config(ws, N=1 << 20, name="nfw_mn", w=None, step=None):
     if w is None:
         spec = "d=6, m=5 per trajectory, fp64, Tsit5 rtol=1e-8 atol=1e-10, t=[0,20]"
     else:
         spec = "d=%d, m=%d %s, %s, %s rtol=%g atol=%g, t=[%g,%g]" % (
             w.d, w.m, "shared" if w.theta_shared else "per trajectory",
             "fp64" if w.dtype == np.float64 else "fp32", w.method, w.rtol, w.atol, w.t0, w.t1)
-    return {"workload": "%s %s, N=%d per GPU, %s; step = record + loss cotangent + replay "
-                        "gradient" % (name, DESCR[name], N, spec),
+    step = step or "record + loss cotangent + replay gradient"
+    return {"workload": "%s %s, N=%d per GPU, %s; step = %s" % (name, DESCR[name], N, spec, step),
             "global_batch": ws * N,
             "parallelism": "independent trajectories, %d rank(s)" % ws,
             "l2": "inputs larger than L2 (the record is several GB)" if name.startswith("nfw")
-                  else "record size reported in record_gb"}
+                  else ("flushed between steps" if name == "log_halo"
+                        else "record size reported in record_gb")}
 
 
 def dist_env():
@@ -152,15 +160,20 @@ def run_reference(args):
     w = W.by_name(args.workload, N=n_sample)
     lam = None
     times = []
+    sens = WORKLOADS[args.workload].get("step") == "sens"
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        r = orc.solve(w.field, w.method, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol,
-                      keep_record=True, nthreads=nthreads, dtype=w.dtype,
-                      theta_shared=w.theta_shared)
-        tgt = w.target if w.target is not None else np.zeros_like(r["y1"])
-        lam = W.loss_cotangent(w, r["y1"], tgt)
-        orc.replay_grad(w.field, w.method, w.theta, w.y0, r["H"], r["S"], lam, nthreads=nthreads,
-                        dtype=w.dtype, theta_shared=w.theta_shared)
+        if sens:
+            orc.solve_sens(w.field, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol, dtype=w.dtype,
+                           theta_shared=w.theta_shared, nthreads=nthreads)
+        else:
+            r = orc.solve(w.field, w.method, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol,
+                          keep_record=True, nthreads=nthreads, dtype=w.dtype,
+                          theta_shared=w.theta_shared)
+            tgt = w.target if w.target is not None else np.zeros_like(r["y1"])
+            lam = W.loss_cotangent(w, r["y1"], tgt)
+            orc.replay_grad(w.field, w.method, w.theta, w.y0, r["H"], r["S"], lam,
+                            nthreads=nthreads, dtype=w.dtype, theta_shared=w.theta_shared)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             times.append(dt)
@@ -170,11 +183,14 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64" if w.dtype == np.float64 else "f32", "data": "synthetic",
-            "config": dict(workload_config(1, w_full.N, args.workload, w_full),
+            "config": dict(workload_config(1, w_full.N, args.workload, w_full,
+                                           SENS_STEP if sens else None),
                            sample="%d trajectories per step" % n_sample),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": nthreads, "kind": "oracle",
-                             "sample": "%d trajectories of the %s ensemble per step: record "
-                                       "solve + replay gradient" % (n_sample, args.workload)},
+                             "sample": "%d trajectories of the %s ensemble per step: %s"
+                                       % (n_sample, args.workload,
+                                          "solve with forward sensitivities" if sens else
+                                          "record solve + replay gradient")},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -212,7 +228,178 @@ WORKLOADS = {
                            adj=FLOPS_ADJOINT_STEP["lotka_volterra"]),
     "robertson": dict(dtype="f64", fwd=None, adj=None),
     "mlp": dict(dtype="f32", fwd=FLOPS_FORWARD_ATTEMPT["mlp"], adj=FLOPS_ADJOINT_STEP["mlp"]),
+    "log_halo": dict(dtype="f64", fwd=FLOPS_FORWARD_ATTEMPT["log_halo"],
+                     adj=FLOPS_ADJOINT_STEP["log_halo"], sens=FLOPS_SENS_STEP["log_halo"],
+                     step="sens"),
 }
+SENS_STEP = ("forward solve with the sensitivities S = dy/dtheta (6 x 2 per orbit) in the same "
+             "kernel, step size controlled on the orbit")
+L2_FLUSH_BYTES = 256 << 20
+
+
+def run_sens(args, w, wl, G, torch, dev, stream, ws, rank):
+    """Forward sensitivities ("Differentiable astrophysics at scale" §3): one step = one
+    gs_solve_forward_sens over the ensemble, L2 flushed between steps (inside the timed region)."""
+    N, d, m = w.N, w.d, w.m
+    dt = torch.float64
+    sys_ = G.system(w.field, w.method, "f64", w.theta_shared)
+    th = torch.as_tensor(w.theta, dtype=dt, device=dev)
+    y0 = torch.as_tensor(w.y0, dtype=dt, device=dev)
+    y1 = torch.empty((N, d), dtype=dt, device=dev)
+    S1 = torch.empty((N, d, m), dtype=dt, device=dev)
+    S = torch.empty(N, dtype=torch.int32, device=dev)
+    rj = torch.empty(N, dtype=torch.int32, device=dev)
+    st = torch.empty(N, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def step():
+        G.gs_solve_forward_sens(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, S1, None, S, rj,
+                                st)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if ws > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier()
+    with ClockSampler(dev.index) as clk:
+        start = torch.cuda.Event(enable_timing=True)
+        stop = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(args.steps):
+            flush.zero_()
+            kev[i][0].record(stream)
+            step()
+            kev[i][1].record(stream)
+        stop.record(stream)
+        barrier()
+    total_ms = start.elapsed_time(stop)
+    if ws > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    value = ws * N * args.steps / (total_ms / 1e3)
+    kernel_ms = statistics.median(a.elapsed_time(b) for a, b in kev)
+    assert int((st != 0).sum().item()) == 0, "some trajectory failed"
+    accepted = int(S.sum().item())
+    attempts = accepted + int(rj.sum().item())
+
+    # ---- breakdown (not part of `value`): the orbit alone, and the reverse-mode route (record +
+    # replay gradient of one scalar loss on the final positions) on the same ensemble
+    def timeit(fn, reps=max(3, args.steps // 2)):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    fwd_ms = timeit(lambda: G.gs_solve_forward(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1))
+    rec = G.Record()
+    target = torch.as_tensor(w.target, dtype=dt, device=dev)
+    mask = torch.as_tensor(w.loss_mask, dtype=dt, device=dev)
+    lam = torch.empty((N, d), dtype=dt, device=dev)
+    gt = torch.empty((m,), dtype=dt, device=dev)
+    gy = torch.empty((N, d), dtype=dt, device=dev)
+
+    def reverse():
+        G.gs_solve_record(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, rec=rec)
+        torch.mul(torch.sub(y1, target), mask, out=lam).mul_(2.0)
+        G.gs_replay_grad(rec, th, lam, gt, gy)
+
+    rev_ms = timeit(reverse)
+    rec.close()
+    breakdown = {"sens_step": ms_step, "sens_kernel": kernel_ms, "forward_only": fwd_ms,
+                 "record_plus_replay_grad": rev_ms}
+
+    # ---- end to end through the public API with host buffers (pinned), copies inside the region
+    h_th = torch.as_tensor(w.theta, dtype=dt).pin_memory()
+    h_y0 = torch.as_tensor(w.y0, dtype=dt).pin_memory()
+    h_y1 = torch.empty((N, d), dtype=dt).pin_memory()
+    h_S1 = torch.empty((N, d, m), dtype=dt).pin_memory()
+    e2e_steps = max(3, args.steps // 2)
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        th.copy_(h_th, non_blocking=True)
+        y0.copy_(h_y0, non_blocking=True)
+        step()
+        h_y1.copy_(y1, non_blocking=True)
+        h_S1.copy_(S1, non_blocking=True)
+    b.record(stream)
+    barrier()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    if ws > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    clocks = clk.summary()
+    peak = pipe_peak_tflops(1965.0, FP64_LANES)
+    at_clock = pipe_peak_tflops(clocks["sm_mhz"], FP64_LANES) if clocks.get("sm_mhz") else None
+    flops = wl["fwd"] * attempts + wl["sens"] * accepted
+    achieved = flops / (kernel_ms / 1e3) / 1e12
+    roofline = {"kernel": "k_solve<log_halo, double, Tsit5, sens>", "bound": "alu",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": None,
+                "peak_source": "derived: 148 SM x 64 FP64 FMA lanes/clk x 2 x 1965 MHz (FP64 pipe)",
+                "flops_per_unit": {"attempted step": wl["fwd"], "accepted step (sensitivities)":
+                                   wl["sens"]},
+                "kernel_ms": kernel_ms,
+                "frac_at_measured_clock": achieved / at_clock if at_clock else None}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(workload_config(ws, N, args.workload, w, SENS_STEP),
+                       l2="flushed between steps (%d MiB write inside the timed region)"
+                          % (L2_FLUSH_BYTES >> 20),
+                       accepted_steps=accepted, attempts=attempts),
+        "roofline": roofline,
+        "breakdown_ms": breakdown,
+        "forward_traj_per_s": ws * N / (fwd_ms / 1e3),
+        "e2e": {"value": ws * N / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": (h_th.numel() + h_y0.numel()) * 8,
+                "d2h_bytes_per_step": (h_y1.numel() + h_S1.numel()) * 8},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_sens(w)
+    else:
+        line["cpu_baseline"] = None
+    return line
+
+
+def cpu_baseline_sens(w_full, seconds_target=15.0):
+    """Oracle throughput (solve with forward sensitivities) on a bounded sample, all host threads."""
+    from differentiable_adaptive_ode_b200 import workloads as W
+    from oracle import oracle as orc
+    nthreads = orc.host_threads()
+    n = 256
+    while True:
+        w = W.subset(w_full, np.arange(n))
+        t0 = time.perf_counter()
+        orc.solve_sens(w.field, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol,
+                       theta_shared=w.theta_shared, nthreads=nthreads)
+        dt = time.perf_counter() - t0
+        if dt > seconds_target / 4 or n >= 1 << 16:
+            return {"value": n / dt, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                    "sample": "%d orbits of the 2^20 logarithmic-halo ensemble (solve with "
+                              "forward sensitivities), %.1f s" % (n, dt)}
+        n *= 2
 
 
 def main():
@@ -249,6 +436,13 @@ def main():
     wl = WORKLOADS[args.workload]
     w = W.by_name(args.workload, N=args.N or None)
     w = W.by_name(args.workload, N=w.N, seed=w.seed + 1000 * rank)   # each rank: its own ensemble
+    if wl.get("step") == "sens":
+        line = run_sens(args, w, wl, G, torch, dev, stream, ws, rank)
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return
     N, d, m = w.N, w.d, w.m
     f64 = w.dtype == np.float64
     dt = torch.float64 if f64 else torch.float32

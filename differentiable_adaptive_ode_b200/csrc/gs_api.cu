@@ -53,6 +53,7 @@ bool field_info(int field, FieldInfo* fi) {
     case GS_ROBERTSON: *fi = {3, 3, false, true}; return true;
     case GS_NFW_MN: *fi = {6, 5, true, false}; return true;
     case GS_LINEAR: *fi = {3, 9, true, true}; return true;
+    case GS_LOG_HALO: *fi = {6, 2, true, false}; return true;
     default: return false;
   }
 }
@@ -300,6 +301,8 @@ struct SolveCall {
   int* queue;
   gs_record* rec;  // non-null: record pass
   cudaStream_t stream;
+  const void* sens0 = nullptr;  // forward sensitivities (Tsit5 forward solve only)
+  void* sens1 = nullptr;
 };
 
 template <class F, class R, int METHOD>
@@ -345,6 +348,18 @@ gs_status launch_solve(const SolveCall& c) {
       GS_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
       const int grid = persistent_grid(kern, smem, c.N);
       kern<<<grid, BLOCK, smem, c.stream>>>(p);
+    } else if (c.sens1) {
+      if constexpr (METHOD == gs::M_TSIT5) {
+        p.sens0 = static_cast<const R*>(c.sens0);
+        p.sens1 = static_cast<R*>(c.sens1);
+        auto kern = gs::k_solve<F, R, METHOD, false, true>;
+        const size_t smem = gs::solve_smem_bytes<F, R, false, true>();
+        GS_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        const int grid = persistent_grid(kern, smem, c.N);
+        kern<<<grid, BLOCK, smem, c.stream>>>(p);
+      } else {
+        return fail(GS_ERR_UNSUPPORTED, "forward sensitivities are built for Tsit5 only");
+      }
     } else {
       auto kern = gs::k_solve<F, R, METHOD, false>;
       const size_t smem = gs::solve_smem_bytes<F, R, false>();
@@ -430,6 +445,9 @@ gs_status dispatch(const gs_system& s, Fn&& fn) {
       case GS_LINEAR:
         return f64 ? fn.template operator()<FLinear3, double, M_TSIT5>()
                    : fn.template operator()<FLinear3, float, M_TSIT5>();
+      case GS_LOG_HALO:
+        return f64 ? fn.template operator()<FLogHalo, double, M_TSIT5>()
+                   : fn.template operator()<FLogHalo, float, M_TSIT5>();
       case GS_MLP_4_32_32_4:
         return f64 ? fn.template operator()<FMlpWarp, double, M_TSIT5>()
                    : fn.template operator()<FMlpWarp, float, M_TSIT5>();
@@ -529,6 +547,26 @@ gs_status gs_solve_forward(const gs_system* sys, const gs_options* opt, int64_t 
   GS_CUDA(take_counter(s, &queue));
   SolveCall c{N, theta, sys->theta_shared, y0, t0, t1, rtol, atol, attempts_of(opt), y1,
               nsteps, nrejected, status, queue, nullptr, s};
+  return dispatch(*sys, [&]<class F, class R, int METHOD>() { return launch_solve<F, R, METHOD>(c); });
+}
+
+gs_status gs_solve_forward_sens(const gs_system* sys, const gs_options* opt, int64_t N,
+                                const void* theta, const void* y0, const void* S0, double t0,
+                                double t1, double rtol, double atol, void* y1, void* S1,
+                                int32_t* nsteps, int32_t* nrejected, int32_t* status,
+                                void* stream) {
+  gs_status st = check_common(sys, N, theta, y0, t0, t1, rtol, atol, y1);
+  if (st != GS_OK) return st;
+  if (sys->method != GS_TSIT5 || sys->field == GS_MLP_4_32_32_4)
+    return fail(GS_ERR_UNSUPPORTED,
+                "forward sensitivities are built for the Tsit5 fields other than the MLP");
+  if (N > 0 && !S1) return fail(GS_ERR_INVALID_ARG, "S1 must be non-NULL");
+  if (N == 0) return GS_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* queue = nullptr;
+  GS_CUDA(take_counter(s, &queue));
+  SolveCall c{N, theta, sys->theta_shared, y0, t0, t1, rtol, atol, attempts_of(opt), y1,
+              nsteps, nrejected, status, queue, nullptr, s, S0, S1};
   return dispatch(*sys, [&]<class F, class R, int METHOD>() { return launch_solve<F, R, METHOD>(c); });
 }
 

@@ -286,4 +286,54 @@ struct FNfwMiyamotoNagai {
   }
 };
 
+// ----------------------------------------------------------------------------------------------
+// Test particle in an axisymmetric flattened logarithmic halo ("Differentiable astrophysics at
+// scale" §3): Phi = (1/2) v_c^2 ln(R_c^2 + x^2 + y^2 + z^2/q^2), R_c = 0.2, theta = (v_c, q).
+//   x' = v,  v' = acc = -g w,  w = (x, y, z/q^2),  g = v_c^2 / Q,  Q = R_c^2 + x^2 + y^2 + z^2/q^2.
+// VJP (u = cotangent of v'):  d acc_i/dx_j = (2 g/Q) w_i w_j - g c_j delta_ij, c = (1, 1, 1/q^2);
+//   d acc/dv_c = -(2 v_c/Q) w;  d acc/dq = -(2 g z^2/(q^3 Q)) w + g (0, 0, 2 z/q^3).
+// ----------------------------------------------------------------------------------------------
+struct FLogHalo {
+  static constexpr int D = 6, M = 2;
+  static constexpr double Rc2 = 0.2 * 0.2;
+  template <class R> struct Theta { R vc, q, vc2, iq2; };
+  template <class R> GS_HD static void load(Theta<R>& t, const R* s) {
+    t.vc = s[0]; t.q = s[1];
+    t.vc2 = t.vc * t.vc;
+    const R iq = R(1) / t.q;
+    t.iq2 = iq * iq;
+  }
+  template <class R> GS_HD static void f(const R* y, const Theta<R>& t, R* dy) {
+    const R wz = y[2] * t.iq2;
+    const R Q = R(Rc2) + y[0] * y[0] + y[1] * y[1] + y[2] * wz;
+    const R g = t.vc2 / Q;
+    dy[0] = y[3];
+    dy[1] = y[4];
+    dy[2] = y[5];
+    dy[3] = -g * y[0];
+    dy[4] = -g * y[1];
+    dy[5] = -g * wz;
+  }
+  template <class R>
+  GS_HD static void vjp(const R* y, const Theta<R>& t, const R* kb, R* yb, R* thb) {
+    const R x = y[0], yy = y[1], z = y[2];
+    const R wz = z * t.iq2;
+    const R iQ = R(1) / (R(Rc2) + x * x + yy * yy + z * wz);
+    const R g = t.vc2 * iQ;
+    const R ux = kb[3], uy = kb[4], uz = kb[5];
+    const R uw = ux * x + uy * yy + uz * wz;
+    const R c2 = R(2) * g * iQ * uw;
+    yb[0] = c2 * x - g * ux;
+    yb[1] = c2 * yy - g * uy;
+    yb[2] = c2 * wz - g * t.iq2 * uz;
+    yb[3] = kb[0];
+    yb[4] = kb[1];
+    yb[5] = kb[2];
+    thb[0] -= R(2) * t.vc * iQ * uw;
+    // d/dq: z^2/q^3 = z wz / q and z/q^3 = wz / q
+    const R iq = t.iq2 * t.q;
+    thb[1] += R(2) * g * wz * iq * (uz - z * iQ * uw);
+  }
+};
+
 }  // namespace gs

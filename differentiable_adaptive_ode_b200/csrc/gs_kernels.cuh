@@ -54,6 +54,9 @@ struct SolveParams {
   int pool_chunks;   // capacity in chunks
   int* chunk_count;  // bump allocator
   int* overflow;     // set to 1 when the pool ran out
+  // forward sensitivities (SENS only): S = dy/dtheta, [N][D][M]; sens0 may be null (zero start)
+  const R* sens0;
+  R* sens1;
 };
 
 template <class R> __device__ __forceinline__ R pw(R x, R e);
@@ -151,12 +154,25 @@ template <class F, class R>
 __host__ __device__ constexpr size_t solve_stage_bytes() {
   return (size_t)4 * 32 * RecLayout<F, R>::STAGE_STRIDE * sizeof(R);
 }
-template <class F, class R, bool REC>
+// Per-lane sensitivity matrices of a 128-thread block, entry (c, j) of lane l at
+// [(c * M + j) * 128 + l] (consecutive lanes in consecutive words).
+template <class F, class R>
+__host__ __device__ constexpr size_t solve_sens_bytes() {
+  return (size_t)F::D * F::M * 128 * sizeof(R);
+}
+template <class F, class R, bool REC, bool SENS = false>
 __host__ __device__ constexpr size_t solve_smem_bytes() {
-  return (REC ? solve_stage_bytes<F, R>() : 0) + 4 * sizeof(StartRing<F, R>);
+  return (REC ? solve_stage_bytes<F, R>() : 0) + (SENS ? solve_sens_bytes<F, R>() : 0) +
+         4 * sizeof(StartRing<F, R>);
 }
 
-template <class F, class R, int METHOD, bool REC>
+// SENS = true (Tsit5, no record): the forward sensitivities S = dy/dtheta ride along with the
+// orbit ("Differentiable astrophysics at scale" §2-§3: sensitivity equations integrated in the
+// same kernel, step size controlled on the orbit alone).  The trial, the error test and the
+// controller are exactly those of the plain solve, so the accepted mesh and y1 are the forward
+// solve's; on each accepted step every column S_{:,j} takes the tangent step of that step along
+// (S_{:,j}, e_j).  S lives in shared memory (indexed by the column loop), one slab per lane.
+template <class F, class R, int METHOD, bool REC, bool SENS = false>
 __global__ void __launch_bounds__(128, Tune<F, R>::solve_blocks) k_solve(SolveParams<R> p) {
   using L = RecLayout<F, R>;
   constexpr int D = F::D;
@@ -167,8 +183,14 @@ __global__ void __launch_bounds__(128, Tune<F, R>::solve_blocks) k_solve(SolvePa
   // shared memory: [record staging, REC only][start-up ring of this block's warps]
   R* stage = REC ? reinterpret_cast<R*>(smem_raw) + (size_t)warp * 32 * L::STAGE_STRIDE : nullptr;
   R* mystage = REC ? stage + lane * L::STAGE_STRIDE : nullptr;
+  R* sens = SENS ? reinterpret_cast<R*>(smem_raw + (REC ? solve_stage_bytes<F, R>() : 0)) +
+                       threadIdx.x
+                 : nullptr;
   StartRing<F, R>* ring =
-      reinterpret_cast<StartRing<F, R>*>(smem_raw + (REC ? solve_stage_bytes<F, R>() : 0)) + warp;
+      reinterpret_cast<StartRing<F, R>*>(smem_raw + (REC ? solve_stage_bytes<F, R>() : 0) +
+                                         (SENS ? solve_sens_bytes<F, R>() : 0)) +
+      warp;
+  constexpr int SM = F::M;
 
   const R expo = R(-1.0 / double(qerr));
   const R eps = eps_of<R>();
@@ -251,7 +273,13 @@ __global__ void __launch_bounds__(128, Tune<F, R>::solve_blocks) k_solve(SolvePa
         for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
         t = p.t0;
         S = 0; Rj = 0; att = 0; last_rej = false; ns = 0; seq = 0;
+        if constexpr (SENS) {
+          for (int i = 0; i < D * SM; ++i)
+            sens[i * 128] = p.sens0 ? p.sens0[(size_t)k * D * SM + i] : R(0);
+        }
         if (st >= 0) {  // finished at start-up: empty interval or non-finite y0 / f(y0)
+          if constexpr (SENS)
+            for (int i = 0; i < D * SM; ++i) p.sens1[(size_t)k * D * SM + i] = sens[i * 128];
 #pragma unroll
           for (int c = 0; c < D; ++c) p.y1[(size_t)k * D + c] = y[c];
           if (p.nsteps) p.nsteps[k] = 0;
@@ -302,6 +330,24 @@ __global__ void __launch_bounds__(128, Tune<F, R>::solve_blocks) k_solve(SolvePa
             for (int c = 0; c < D; ++c) e[2 + c] = y[c];
             ++ns;
           }
+          if constexpr (SENS && METHOD == M_TSIT5) {
+            // tangent step of the accepted step for each column j, direction (S_{:,j}, e_j)
+            const R* thk = p.theta + (size_t)p.theta_stride * k;
+#pragma unroll 1
+            for (int j = 0; j < SM; ++j) {
+              Dl<R> src[SM];
+#pragma unroll
+              for (int i = 0; i < SM; ++i) src[i] = Dl<R>(thk[i], i == j ? R(1) : R(0));
+              typename F::template Theta<Dl<R>> thd;
+              F::load(thd, src);
+              R col[D];
+#pragma unroll
+              for (int c = 0; c < D; ++c) col[c] = sens[(c * SM + j) * 128];
+              tsit5_tangent_step<F, R>(y, h, thd, col);
+#pragma unroll
+              for (int c = 0; c < D; ++c) sens[(c * SM + j) * 128] = col[c];
+            }
+          }
           ++S;
           const R facmax = last_rej ? R(1) : R(10);
           R fac = (err == R(0)) ? facmax : R(0.9) * pw<R>(err, expo);
@@ -321,6 +367,8 @@ __global__ void __launch_bounds__(128, Tune<F, R>::solve_blocks) k_solve(SolvePa
         }
       }
       if (st >= 0) {
+        if constexpr (SENS)
+          for (int i = 0; i < D * SM; ++i) p.sens1[(size_t)k * D * SM + i] = sens[i * 128];
 #pragma unroll
         for (int c = 0; c < D; ++c) p.y1[(size_t)k * D + c] = y[c];
         if (p.nsteps) p.nsteps[k] = S;

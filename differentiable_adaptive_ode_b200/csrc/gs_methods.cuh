@@ -10,6 +10,7 @@
 #pragma once
 #include <type_traits>
 
+#include "gs_dual.cuh"
 #include "gs_fields.cuh"
 
 namespace gs {
@@ -232,6 +233,48 @@ __device__ __forceinline__ void tsit5_replay_step(const R (&y)[F::D], R h,
 #pragma unroll
     for (int j = 1; j < 6; ++j) s += tb<R>(j) * k[j][c];
     ynew[c] = y[c] + h * s;
+  }
+}
+
+// Tangent of one Tsit5 step with h fixed, along the input direction (yd, thd.d):
+//   Yd_i = yd + h sum_{j<i} a_ij Kd_j,   Kd_i = J_y(Y_i) Yd_i + J_theta(Y_i) thd,
+//   yd_new = yd + h sum_{i<=6} b_i Kd_i
+// -- the forward-mode derivative of Phi(y, h; theta), i.e. the same Tsit5 step applied to the
+// sensitivity equations S' = J_y S + J_theta.  Each Kd_i comes from f evaluated on dual numbers
+// (value and derivative together), so the stage values Y_i are recomputed alongside.
+template <class F, class R>
+__device__ __forceinline__ void tsit5_tangent_step(const R (&y)[F::D], R h,
+                                                   const typename F::template Theta<Dl<R>>& thd,
+                                                   R (&yd)[F::D]) {
+  constexpr int D = F::D;
+  Dl<R> k[6][D];
+  {
+    Dl<R> Y[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) Y[c] = Dl<R>(y[c], yd[c]);
+    F::f(Y, thd, k[0]);
+  }
+#pragma unroll
+  for (int i = 1; i < 6; ++i) {
+    Dl<R> Y[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+      R sv = ta<R>(i, 0) * k[0][c].v, sd = ta<R>(i, 0) * k[0][c].d;
+#pragma unroll
+      for (int j = 1; j < i; ++j) {
+        sv += ta<R>(i, j) * k[j][c].v;
+        sd += ta<R>(i, j) * k[j][c].d;
+      }
+      Y[c] = Dl<R>(y[c] + h * sv, yd[c] + h * sd);
+    }
+    F::f(Y, thd, k[i]);
+  }
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    R sd = tb<R>(0) * k[0][c].d;
+#pragma unroll
+    for (int j = 1; j < 6; ++j) sd += tb<R>(j) * k[j][c].d;
+    yd[c] = yd[c] + h * sd;
   }
 }
 

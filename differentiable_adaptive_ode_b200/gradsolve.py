@@ -17,16 +17,17 @@ LIB_PATH = os.path.join(PKG, "libgradsolve_b200.so")
 GS_OK, GS_ERR_INVALID_ARG, GS_ERR_CUDA, GS_ERR_CAPACITY, GS_ERR_UNSUPPORTED, GS_ERR_TRAJ_FAILED = range(6)
 GS_F64, GS_F32 = 0, 1
 GS_TSIT5, GS_ROS34PW2 = 0, 1
-FIELDS = {"lotka_volterra": 0, "lorenz63": 1, "mlp": 2, "robertson": 3, "nfw_mn": 4, "linear3": 5}
+FIELDS = {"lotka_volterra": 0, "lorenz63": 1, "mlp": 2, "robertson": 3, "nfw_mn": 4, "linear3": 5,
+          "log_halo": 6}
 # (d, m) of each field, as the library checks them
 FIELD_DIMS = {"lotka_volterra": (2, 4), "lorenz63": (3, 3), "mlp": (4, 1348), "robertson": (3, 3),
-              "nfw_mn": (6, 5), "linear3": (3, 9)}
+              "nfw_mn": (6, 5), "linear3": (3, 9), "log_halo": (6, 2)}
 METHODS = {"tsit5": GS_TSIT5, "ros34pw2": GS_ROS34PW2}
 STATUS_NAMES = {0: "GS_OK", 1: "GS_ERR_INVALID_ARG", 2: "GS_ERR_CUDA", 3: "GS_ERR_CAPACITY",
                 4: "GS_ERR_UNSUPPORTED", 5: "GS_ERR_TRAJ_FAILED"}
 
 # every entry point declared in include/gradsolve_b200.h
-EXPORTS = ("gs_solve_forward", "gs_solve_record", "gs_replay_grad", "gs_replay_forward",
+EXPORTS = ("gs_solve_forward", "gs_solve_forward_sens", "gs_solve_record", "gs_replay_grad", "gs_replay_forward",
            "gs_replay_grad_noalloc", "gs_replay_outputs", "gs_replay_grad_outputs", "gs_record_info",
            "gs_record_export", "gs_record_import", "gs_record_destroy", "gs_last_error",
            "gs_version")
@@ -70,6 +71,8 @@ def lib():
         P = C.POINTER
         L.gs_solve_forward.argtypes = [P(GsSystem), P(GsOptions), i64, vp, vp, d, d, d, d, vp, vp,
                                        vp, vp, vp]
+        L.gs_solve_forward_sens.argtypes = [P(GsSystem), P(GsOptions), i64, vp, vp, vp, d, d, d,
+                                            d, vp, vp, vp, vp, vp, vp]
         L.gs_solve_record.argtypes = [P(GsSystem), P(GsOptions), i64, vp, vp, d, d, d, d,
                                       P(vp), vp, vp, vp]
         L.gs_replay_grad.argtypes = [vp, vp, vp, vp, vp, vp]
@@ -85,7 +88,7 @@ def lib():
         L.gs_record_destroy.restype = None
         L.gs_last_error.restype = C.c_char_p
         L.gs_version.restype = C.c_char_p
-        for name in ("gs_solve_forward", "gs_solve_record", "gs_replay_grad", "gs_replay_forward",
+        for name in ("gs_solve_forward", "gs_solve_forward_sens", "gs_solve_record", "gs_replay_grad", "gs_replay_forward",
                      "gs_replay_grad_noalloc", "gs_replay_outputs", "gs_replay_grad_outputs",
                      "gs_record_info",
                      "gs_record_export", "gs_record_import"):
@@ -138,6 +141,17 @@ def gs_solve_forward(sys, N, theta, y0, t0, t1, rtol, atol, y1, nsteps=None, nre
     _check(lib().gs_solve_forward(C.byref(sys), C.byref(opts), N, _ptr(theta), _ptr(y0), t0, t1,
                                   rtol, atol, _ptr(y1), _ptr(nsteps), _ptr(nrejected),
                                   _ptr(status), _stream(stream)))
+
+
+def gs_solve_forward_sens(sys, N, theta, y0, t0, t1, rtol, atol, y1, S1, S0=None, nsteps=None,
+                          nrejected=None, status=None, opts=None, stream=None):
+    """Forward solve with the sensitivities S = dy/dtheta [N, d, m] integrated alongside (step
+    control on y alone); S0 [N, d, m] optional (zero start)."""
+    opts = opts or options()
+    _check(lib().gs_solve_forward_sens(C.byref(sys), C.byref(opts), N, _ptr(theta), _ptr(y0),
+                                       _ptr(S0), t0, t1, rtol, atol, _ptr(y1), _ptr(S1),
+                                       _ptr(nsteps), _ptr(nrejected), _ptr(status),
+                                       _stream(stream)))
 
 
 class Record:

@@ -56,14 +56,20 @@ typedef enum { GS_TSIT5 = 0, GS_ROS34PW2 = 1 } gs_method;
  *   GS_ROBERTSON       d=3 m=3     theta = (k1, k2, k3), stiff          ([GS] §4.2, §4.5)
  *   GS_NFW_MN          d=6 m=5     test particle in NFW halo + Miyamoto-Nagai disk,
  *                                  theta = (M_h, r_s, M_d, a, b), G = 1
- *   GS_LINEAR          d=3 m=9     y' = A y, theta = A row-major         ([GS] §4.6-4.7) */
+ *   GS_LINEAR          d=3 m=9     y' = A y, theta = A row-major         ([GS] §4.6-4.7)
+ *   GS_LOG_HALO        d=6 m=2     test particle in the flattened logarithmic halo
+ *                                  Phi = v_c^2/2 ln(R_c^2 + x^2 + y^2 + z^2/q^2), R_c = 0.2,
+ *                                  theta = (v_c, q)                     ([DA] §3)
+ * [DA] = "Differentiable astrophysics at scale: solving and differentiating ODE ensembles on the
+ * GPU". */
 typedef enum {
   GS_LOTKA_VOLTERRA = 0,
   GS_LORENZ63 = 1,
   GS_MLP_4_32_32_4 = 2,
   GS_ROBERTSON = 3,
   GS_NFW_MN = 4,
-  GS_LINEAR = 5
+  GS_LINEAR = 5,
+  GS_LOG_HALO = 6
 } gs_field;
 
 typedef struct {
@@ -112,6 +118,25 @@ gs_status gs_solve_forward(const gs_system* sys, const gs_options* opt, int64_t 
                            const void* theta, const void* y0, double t0, double t1, double rtol,
                            double atol, void* y1, int32_t* nsteps, int32_t* nrejected,
                            int32_t* status, void* stream);
+
+/* Forward solve with forward sensitivities ([DA] §2-§3: the sensitivity equations
+ * S' = J_y(y) S + J_theta(y), S = dy/dtheta, integrated in the same kernel as the orbit, with the
+ * step size controlled on the orbit alone).  The trial steps, error test and controller are those
+ * of gs_solve_forward, so y1, nsteps, nrejected and status are identical to its results; on every
+ * accepted step each column S_{:,j} takes the same Tsit5 step of the sensitivity equations along
+ * (S_{:,j}, e_j).  The result is therefore the exact derivative of the discrete solution on the
+ * accepted mesh (the mesh held fixed, as in [GS] §3).
+ * In:  as gs_solve_forward, plus S0 [N][d][m] (device, nullable: zero, i.e. y0 independent of
+ * theta).  For a shared theta, S is still per trajectory: [N][d][m].
+ * Out: y1 [N][d]; S1 [N][d][m] (device, required); nsteps, nrejected, status (nullable).
+ * Built for GS_TSIT5 and every Tsit5 field except GS_MLP_4_32_32_4 (GS_ERR_UNSUPPORTED otherwise).
+ * A non-finite S does not change a trajectory's status (the controller does not see S).
+ * Asynchronous. */
+gs_status gs_solve_forward_sens(const gs_system* sys, const gs_options* opt, int64_t N,
+                                const void* theta, const void* y0, const void* S0, double t0,
+                                double t1, double rtol, double atol, void* y1, void* S1,
+                                int32_t* nsteps, int32_t* nrejected, int32_t* status,
+                                void* stream);
 
 /* Record pass ([GS] §3, Fig. 2): the same adaptive solve, keeping each accepted step
  * (t_n, h_n, y_n) = (start time, step size used, state at the start of the step), n < S_k.

@@ -406,6 +406,15 @@ int orc_count_ops(int field, int what, const double* theta, const double* y, dou
     tally() = OpTally{};
     if (what == 0) {
       F::f(yy, th.data(), out);
+    } else if (what == 3) {
+      // f with one tangent direction (forward-mode rules): value + directional derivative
+      using DC = Dual<Cnt, 1>;
+      std::vector<DC> thd(F::M);
+      DC yd[F::D], od[F::D];
+      for (int j = 0; j < F::M; ++j) { thd[j] = DC(th[j]); thd[j].g[0] = Cnt(j == 0 ? 1.0 : 0.0); }
+      for (int c = 0; c < F::D; ++c) { yd[c] = DC(yy[c]); yd[c].g[0] = Cnt(1.0); }
+      tally() = OpTally{};
+      F::f(yd, thd.data(), od);
     } else if (what == 1) {
       tsit5_trial<F, Cnt>(yy, Cnt(h), th.data(), k1, out, k7, e, true);
     } else {

@@ -92,7 +92,8 @@ inline Dual<R, P> operator/(const Dual<R, P>& a, const Dual<R, P>& b) {
 template <class R, int P>
 inline Dual<R, P> sqrt(const Dual<R, P>& a) {
   Dual<R, P> c;
-  c.v = std::sqrt(a.v);
+  using std::sqrt;  // plain scalars, or the op counter through argument lookup
+  c.v = sqrt(a.v);
   const R d = R(1) / (R(2) * c.v);
   for (int i = 0; i < P; ++i) c.g[i] = a.g[i] * d;
   return c;
@@ -100,7 +101,8 @@ inline Dual<R, P> sqrt(const Dual<R, P>& a) {
 template <class R, int P>
 inline Dual<R, P> log1p(const Dual<R, P>& a) {
   Dual<R, P> c;
-  c.v = std::log1p(a.v);
+  using std::log1p;  // plain scalars, or the op counter through argument lookup
+  c.v = log1p(a.v);
   const R d = R(1) / (R(1) + a.v);
   for (int i = 0; i < P; ++i) c.g[i] = a.g[i] * d;
   return c;
@@ -108,7 +110,8 @@ inline Dual<R, P> log1p(const Dual<R, P>& a) {
 template <class R, int P>
 inline Dual<R, P> tanh(const Dual<R, P>& a) {
   Dual<R, P> c;
-  c.v = std::tanh(a.v);
+  using std::tanh;  // plain scalars, or the op counter through argument lookup
+  c.v = tanh(a.v);
   const R d = R(1) - c.v * c.v;
   for (int i = 0; i < P; ++i) c.g[i] = a.g[i] * d;
   return c;

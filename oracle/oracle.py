@@ -235,12 +235,13 @@ OP_NAMES = ("add", "mul", "div", "sqrt", "log1p", "tanh")
 
 
 def count_ops(field, what, theta, y, h=0.1):
-    """Tally of one f evaluation (what='f'), Tsit5 trial ('tsit5') or ROS34PW2 trial ('ros')."""
+    """Tally of one f evaluation (what='f'), Tsit5 trial ('tsit5'), ROS34PW2 trial ('ros') or f
+    with one tangent direction by the forward-mode rules ('f_dual')."""
     D, M = dims(field)
     theta = np.ascontiguousarray(theta, np.float64).reshape(M)
     y = np.ascontiguousarray(y, np.float64).reshape(D)
     counts = np.zeros(6, np.int64)
-    rc = lib().orc_count_ops(FIELDS[field], {"f": 0, "tsit5": 1, "ros": 2}[what], _p(theta),
+    rc = lib().orc_count_ops(FIELDS[field], {"f": 0, "tsit5": 1, "ros": 2, "f_dual": 3}[what], _p(theta),
                              _p(y), h, _p(counts))
     assert rc == 0, rc
     return dict(zip(OP_NAMES, counts.tolist()))

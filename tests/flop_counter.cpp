@@ -8,6 +8,7 @@
 #include <type_traits>
 
 #include "gs_fields.cuh"
+#include "gs_dual.cuh"
 
 struct Tally { long add = 0, mul = 0, div = 0, sqrt = 0, log1p = 0; };
 static Tally T;
@@ -26,6 +27,7 @@ inline Cnt operator/(Cnt a, Cnt b) { T.div++; return Cnt(a.v / b.v); }
 inline Cnt sqrt(Cnt a) { T.sqrt++; return Cnt(std::sqrt(a.v)); }
 inline Cnt log1p(Cnt a) { T.log1p++; return Cnt(std::log1p(a.v)); }
 inline Cnt rsqrt(Cnt a) { T.sqrt++; return Cnt(1.0 / std::sqrt(a.v)); }
+inline Cnt fma(Cnt a, Cnt b, Cnt c) { T.mul++; T.add++; return Cnt(a.v * b.v + c.v); }
 
 template <class F, class = void> struct has_pullback : std::false_type {};
 template <class F>
@@ -54,11 +56,22 @@ void run(const char* name, const double* theta, const double* y) {
     F::vjp(yy, th, kb, yb, thb);
     tv = T;
   }
+  // f on one-direction dual numbers (the forward-sensitivity stage): value and tangent together
+  using DC = gs::Dl<Cnt>;
+  DC dsrc[F::M], dy_[F::D], ddy[F::D];
+  for (int j = 0; j < F::M; ++j) dsrc[j] = DC(Cnt(theta[j]), Cnt(j == 0 ? 1.0 : 0.0));
+  for (int c = 0; c < F::D; ++c) dy_[c] = DC(Cnt(y[c]), Cnt(0.01 * (c + 1)));
+  typename F::template Theta<DC> thd;
+  F::load(thd, dsrc);
+  T = Tally();
+  F::f(dy_, thd, ddy);
+  Tally td = T;
   std::printf("{\"field\": \"%s\", \"D\": %d, \"M\": %d, "
               "\"f\": {\"add\": %ld, \"mul\": %ld, \"div\": %ld, \"sqrt\": %ld, \"log1p\": %ld}, "
-              "\"vjp\": {\"add\": %ld, \"mul\": %ld, \"div\": %ld, \"sqrt\": %ld, \"log1p\": %ld}}\n",
+              "\"vjp\": {\"add\": %ld, \"mul\": %ld, \"div\": %ld, \"sqrt\": %ld, \"log1p\": %ld}, "
+              "\"fdual\": {\"add\": %ld, \"mul\": %ld, \"div\": %ld, \"sqrt\": %ld, \"log1p\": %ld}}\n",
               name, F::D, F::M, tf.add, tf.mul, tf.div, tf.sqrt, tf.log1p, tv.add, tv.mul, tv.div,
-              tv.sqrt, tv.log1p);
+              tv.sqrt, tv.log1p, td.add, td.mul, td.div, td.sqrt, td.log1p);
 }
 
 int main() {
@@ -70,5 +83,7 @@ int main() {
   run<gs::FLorenz63>("lorenz63", lor_th, lor_y);
   run<gs::FLotkaVolterra>("lotka_volterra", lv_th, lv_y);
   run<gs::FRobertson>("robertson", rob_th, rob_y);
+  const double lh_th[2] = {1.0, 0.7}, lh_y[6] = {0.7, 0.2, 0.4, 0.1, 0.5, 0.05};
+  run<gs::FLogHalo>("log_halo", lh_th, lh_y);
   return 0;
 }

@@ -117,3 +117,21 @@ def rel_rows(a, b, floor):
 
 def small(name, N):
     return W.by_name(name, N=N)
+
+
+def forward_sens(w, S0=None, max_attempts=0):
+    """gs_solve_forward_sens on the workload: y1, S (= dy/dtheta [N, d, m]), counts, status."""
+    t = torch()
+    dt = tdtype(w)
+    th, y0 = dev(w.theta, dt), dev(w.y0, dt)
+    y1 = t.empty((w.N, w.d), dtype=dt, device="cuda")
+    S1 = t.empty((w.N, w.d, w.m), dtype=dt, device="cuda")
+    S = t.empty(w.N, dtype=t.int32, device="cuda")
+    rej = t.empty(w.N, dtype=t.int32, device="cuda")
+    st = t.empty(w.N, dtype=t.int32, device="cuda")
+    G.gs_solve_forward_sens(gsys(w), w.N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, S1,
+                            None if S0 is None else dev(S0, dt), S, rej, st,
+                            opts=G.options(max_attempts))
+    t.cuda.synchronize()
+    return dict(y1=y1.cpu().numpy(), sens=S1.cpu().numpy(), S=S.cpu().numpy(),
+                rejected=rej.cpu().numpy(), status=st.cpu().numpy())

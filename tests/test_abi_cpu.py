@@ -56,6 +56,16 @@ def test_argument_errors_without_device(G):
     assert L.gs_solve_forward(*args(s, 0, rtol=0.0)) == G.GS_ERR_INVALID_ARG
     wrong = G.system("lorenz63", method="ros34pw2")
     assert L.gs_solve_forward(*args(wrong, 10)) == G.GS_ERR_UNSUPPORTED
+    # forward sensitivities: Tsit5 fields other than the MLP only; S1 required
+    sargs = lambda sys_, N, S1=None: (C.byref(sys_), C.byref(o), N, C.c_void_p(8), C.c_void_p(8),
+                                      None, 0.0, 1.0, 1e-6, 1e-9, C.c_void_p(8), S1, None, None,
+                                      None, None)
+    rob = G.system("robertson")
+    assert L.gs_solve_forward_sens(*sargs(rob, 10, C.c_void_p(8))) == G.GS_ERR_UNSUPPORTED
+    mlp = G.system("mlp", dtype="f32", theta_shared=True)
+    assert L.gs_solve_forward_sens(*sargs(mlp, 10, C.c_void_p(8))) == G.GS_ERR_UNSUPPORTED
+    assert L.gs_solve_forward_sens(*sargs(G.system("log_halo", theta_shared=True), 10)) \
+        == G.GS_ERR_INVALID_ARG
     assert L.gs_replay_grad(None, None, None, None, None, None) == G.GS_ERR_INVALID_ARG
     assert L.gs_record_info(None, None) == G.GS_ERR_INVALID_ARG
     L.gs_record_destroy(None)

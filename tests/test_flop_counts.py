@@ -33,7 +33,7 @@ def ops(t):
     return t["add"] + t["mul"] + t["div"] + t["sqrt"] + t["log1p"]
 
 
-@pytest.mark.parametrize("field", ["nfw_mn", "lorenz63", "lotka_volterra"])
+@pytest.mark.parametrize("field", ["nfw_mn", "lorenz63", "lotka_volterra", "log_halo"])
 def test_bench_constants_match_counts(counts, field):
     import bench
     c = counts[field]
@@ -42,6 +42,15 @@ def test_bench_constants_match_counts(counts, field):
     fwd = 67 * D + 6 * ops(c["f"]) + 5
     assert bench.FLOPS_ADJOINT_STEP[field] == adj
     assert bench.FLOPS_FORWARD_ATTEMPT[field] == fwd
+
+
+def test_sens_constant_matches_counts(counts):
+    # tangent of the Tsit5 step per column: stage tangents 35 d + result 13 d, plus six stage
+    # evaluations of f's forward-mode rules beyond f itself (c_t = dual f - f)
+    import bench
+    c = counts["log_halo"]
+    c_t = ops(c["fdual"]) - ops(c["f"])
+    assert bench.FLOPS_SENS_STEP["log_halo"] == c["M"] * (48 * c["D"] + 6 * c_t)
 
 
 def test_mlp_hand_count():
