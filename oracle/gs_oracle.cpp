@@ -202,7 +202,7 @@ int with_field(int field, Fn&& fn) {
 
 template <class F>
 bool method_ok(int method) {
-  if (method == TSIT5) return true;
+  if (method == TSIT5 || method == VERN7) return true;
   if (method == ROS34PW2) return has_jac<F>::value;
   return false;
 }
@@ -384,6 +384,10 @@ int orc_trial(int field, int method, const double* theta, const double* y, doubl
       double k1[F::D], k7[F::D];
       F::f(y, theta, k1);
       tsit5_trial<F, double>(y, h, theta, k1, ynew, k7, e, true);
+    } else if (method == VERN7) {
+      double k1[F::D];
+      F::f(y, theta, k1);
+      vern7_trial<F, double>(y, h, theta, k1, ynew, e, true);
     } else {
       if constexpr (has_jac<F>::value) ros_trial<F, double>(y, h, theta, ynew, e, true);
     }
@@ -435,6 +439,13 @@ void orc_tsit5_tableau(double* C7, double* A49, double* B7, double* BT7) {
     B7[i] = Tsit5Tab::B[i];
     BT7[i] = Tsit5Tab::BT[i];
     for (int j = 0; j < 7; ++j) A49[i * 7 + j] = j < 6 ? Tsit5Tab::A[i][j] : 0.0;
+  }
+}
+void orc_vern7_tableau(double* A100, double* B10, double* BH10) {
+  for (int i = 0; i < 10; ++i) {
+    B10[i] = Vern7Tab::B[i];
+    BH10[i] = Vern7Tab::BH[i];
+    for (int j = 0; j < 10; ++j) A100[i * 10 + j] = j < 9 ? Vern7Tab::A[i][j] : 0.0;
   }
 }
 void orc_ros34pw2_tableau(double* gamma, double* ALPHA16, double* GAMMA16, double* B4,

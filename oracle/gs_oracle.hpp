@@ -339,6 +339,72 @@ struct Ros34pw2Tab {
 };
 
 // ------------------------------------------------------------------------------------------
+// Verner's 7(6) pair ("most efficient" IIa, Verner 2010; the seventh-order Verner pair that
+// [GS] §3.1 offers besides Tsit5 for non-stiff problems): 10 stages, not first-same-as-last.
+// b_2 = b_3 = b_10 = 0; the tenth stage enters only the embedded sixth-order solution b_hat.
+// The decimals are the published ones (checked by the order conditions in the tests).
+// ------------------------------------------------------------------------------------------
+struct Vern7Tab {
+  static constexpr int S = 10;
+  static constexpr int order = 7;
+  static constexpr int err_order = 7;   // embedded order 6, plus one
+  static constexpr double A[10][9] = {
+      {0, 0, 0, 0, 0, 0, 0, 0, 0},
+      {0.005, 0, 0, 0, 0, 0, 0, 0, 0},
+      {-1.0767901234567902, 1.185679012345679, 0, 0, 0, 0, 0, 0, 0},
+      {0.04083333333333333, 0, 0.1225, 0, 0, 0, 0, 0, 0},
+      {0.6389139236255726, 0, -2.455672638223657, 2.272258714598084, 0, 0, 0, 0, 0},
+      {-2.6615773750187572, 0, 10.804513886456137, -8.3539146573962, 0.820487594956657, 0, 0,
+       0, 0},
+      {6.067741434696772, 0, -24.711273635911088, 20.427517930788895, -1.9061579788166472,
+       1.006172249242068, 0, 0, 0},
+      {12.054670076253203, 0, -49.75478495046899, 41.142888638604674, -4.461760149974004,
+       2.042334822239175, -0.09834843665406107, 0, 0},
+      {10.138146522881808, 0, -42.6411360317175, 35.76384003992257, -4.3480228403929075,
+       2.009862268377035, 0.3487490460338272, -0.27143900510483127, 0},
+      {-45.030072034298676, 0, 187.3272437654589, -154.02882369350186, 18.56465306347536,
+       -7.141809679295079, 1.3088085781613787, 0, 0}};
+  static constexpr double B[10] = {0.04715561848627222, 0, 0, 0.25750564298434153,
+                                   0.26216653977412624, 0.15216092656738558, 0.4939969170032485,
+                                   -0.29430311714032503, 0.08131747232495111, 0};
+  static constexpr double BH[10] = {0.044608606606341174, 0, 0, 0.26716403785713727,
+                                    0.22010183001772932, 0.2188431703143157, 0.22898717054112028,
+                                    0, 0, 0.02029518466335628};
+};
+
+// One trial step of Verner 7 from y with step h; k1 = f(y) is passed in (it stays valid across a
+// rejected trial).  Stage states Y_i = y + h sum_{j<i} A_ij k_j (j ascending), the step result
+// y_new = y + h sum_i B_i k_i, the error estimate e = h sum_i (B_i - BH_i) k_i.  With want_err
+// false only stages 1..9 are formed (the replay map: B_10 = 0).
+template <class F, class T>
+void vern7_trial(const T* y, T h, const T* th, const T* k1, T* ynew, T* e, bool want_err) {
+  constexpr int D = F::D;
+  const int nst = want_err ? 10 : 9;
+  T k[10][D];
+  for (int c = 0; c < D; ++c) k[0][c] = k1[c];
+  for (int i = 1; i < nst; ++i) {
+    T Y[D];
+    for (int c = 0; c < D; ++c) {
+      T s = cst<T>(Vern7Tab::A[i][0]) * k[0][c];
+      for (int j = 1; j < i; ++j) s = s + cst<T>(Vern7Tab::A[i][j]) * k[j][c];
+      Y[c] = y[c] + h * s;
+    }
+    F::f(Y, th, k[i]);
+  }
+  for (int c = 0; c < D; ++c) {
+    T s = cst<T>(Vern7Tab::B[0]) * k[0][c];
+    for (int j = 1; j < 9; ++j) s = s + cst<T>(Vern7Tab::B[j]) * k[j][c];
+    ynew[c] = y[c] + h * s;
+  }
+  if (!want_err) return;
+  for (int c = 0; c < D; ++c) {
+    T s = (cst<T>(Vern7Tab::B[0]) - cst<T>(Vern7Tab::BH[0])) * k[0][c];
+    for (int j = 1; j < 10; ++j) s = s + (cst<T>(Vern7Tab::B[j]) - cst<T>(Vern7Tab::BH[j])) * k[j][c];
+    e[c] = h * s;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
 // One trial step of Tsit5 from y with step h.  k1 = f(y) is passed in (first-same-as-last).
 // Writes the step result y_new, the last stage k7 = f(y_new) (the next k1) and the error
 // estimate e = h sum_j BT_j k_j.  Stage states: Y_i = y + h sum_{j<i} A_ij k_j, summed j-ascending.
@@ -451,7 +517,15 @@ void ros_trial(const T* y, T h, const T* th, T* ynew, T* e, bool want_err) {
   }
 }
 
-enum Method { TSIT5 = 0, ROS34PW2 = 1 };
+enum Method { TSIT5 = 0, ROS34PW2 = 1, VERN7 = 2 };
+
+inline int method_order(Method m) {
+  return m == TSIT5 ? Tsit5Tab::order : m == VERN7 ? Vern7Tab::order : Ros34pw2Tab::order;
+}
+inline int method_err_order(Method m) {
+  return m == TSIT5 ? Tsit5Tab::err_order : m == VERN7 ? Vern7Tab::err_order
+                                                       : Ros34pw2Tab::err_order;
+}
 
 // has_jac<F>: stiff fields carry an analytic Jacobian.
 template <class F, class = void> struct has_jac : std::false_type {};
@@ -529,8 +603,8 @@ Record<R> solve(Method method, const R* y0, const R* th, R t0, R t1, R rtol, R a
   F::f(y, th, k1);
   for (int i = 0; i < Dc; ++i)
     if (!std::isfinite(y[i]) || !std::isfinite(k1[i])) { rec.status = 3; return rec; }
-  const int p = method == TSIT5 ? Tsit5Tab::order : Ros34pw2Tab::order;
-  const int q = method == TSIT5 ? Tsit5Tab::err_order : Ros34pw2Tab::err_order;
+  const int p = method_order(method);
+  const int q = method_err_order(method);
   const R expo = R(-1.0 / double(q));
   const R eps = std::numeric_limits<R>::epsilon();
   R h = initial_step<F, R>(y, k1, th, t0, t1, rtol, atol, p, Dc);
@@ -546,6 +620,8 @@ Record<R> solve(Method method, const R* y0, const R* th, R t0, R t1, R rtol, R a
     R ynew[D], k7[D], e[D];
     if (method == TSIT5) {
       tsit5_trial<F, R>(y, h, th, k1, ynew, k7, e, true);
+    } else if (method == VERN7) {
+      vern7_trial<F, R>(y, h, th, k1, ynew, e, true);
     } else {
       if constexpr (has_jac<F>::value) ros_trial<F, R>(y, h, th, ynew, e, true);
     }
@@ -564,6 +640,8 @@ Record<R> solve(Method method, const R* y0, const R* th, R t0, R t1, R rtol, R a
       for (int i = 0; i < D; ++i) y[i] = ynew[i];
       if (method == TSIT5)
         for (int i = 0; i < D; ++i) k1[i] = k7[i];  // first-same-as-last
+      else if (method == VERN7)
+        F::f(y, th, k1);                             // a fresh first stage at the new state
       h = h * fac;
       last_rejected = false;
     } else {
@@ -578,9 +656,24 @@ Record<R> solve(Method method, const R* y0, const R* th, R t0, R t1, R rtol, R a
   return rec;
 }
 
+// One step of the method's one-step map Phi(y, h; theta) (no error estimate): the replay step.
+template <class F, class T>
+void one_step(Method method, const T* y, const T* th, T h, T* ynew) {
+  constexpr int D = F::D;
+  if (method == TSIT5 || method == VERN7) {
+    T k1[D];
+    F::f(y, th, k1);
+    if (method == TSIT5) tsit5_trial<F, T>(y, h, th, k1, ynew, nullptr, nullptr, false);
+    else vern7_trial<F, T>(y, h, th, k1, ynew, nullptr, false);
+  } else {
+    if constexpr (has_jac<F>::value) ros_trial<F, T>(y, h, th, ynew, nullptr, false);
+  }
+}
+
 // ------------------------------------------------------------------------------------------
 // Replay ([GS] §3, Eq. 4): y_{n+1} = Phi(y_n, h_n; theta), n = 0..S-1, with the recorded h_n
-// as data.  For Tsit5, Phi(y, h) = y + h sum_{i<=6} b_i k_i with k_1 = f(y) evaluated afresh.
+// as data.  For Tsit5, Phi(y, h) = y + h sum_{i<=6} b_i k_i with k_1 = f(y) evaluated afresh;
+// for Verner 7, Phi(y, h) = y + h sum_{i<=9} b_i k_i.
 // ------------------------------------------------------------------------------------------
 template <class F, class T>
 void replay(Method method, T* y, const T* th, const typename base_of<T>::type* H, int S) {
@@ -588,13 +681,7 @@ void replay(Method method, T* y, const T* th, const typename base_of<T>::type* H
   for (int n = 0; n < S; ++n) {
     const T h = T(H[n]);
     T ynew[D];
-    if (method == TSIT5) {
-      T k1[D];
-      F::f(y, th, k1);
-      tsit5_trial<F, T>(y, h, th, k1, ynew, nullptr, nullptr, false);
-    } else {
-      if constexpr (has_jac<F>::value) ros_trial<F, T>(y, h, th, ynew, nullptr, false);
-    }
+    one_step<F, T>(method, y, th, h, ynew);
     for (int c = 0; c < D; ++c) y[c] = ynew[c];
   }
 }
@@ -642,17 +729,6 @@ void replay_grad(Method method, const R* y0, const R* th, const R* H, int S, con
 // the last recorded t_n with t_n <= tau_j and tau_j < t_{n+1} (t_S = t1); the output is
 // Phi(y_n, tau_j - t_n), and tau_j = t1 gives y_S.  Tm holds the recorded start times t_n.
 // ------------------------------------------------------------------------------------------
-template <class F, class T>
-void one_step(Method method, const T* y, const T* th, T h, T* ynew) {
-  constexpr int D = F::D;
-  if (method == TSIT5) {
-    T k1[D];
-    F::f(y, th, k1);
-    tsit5_trial<F, T>(y, h, th, k1, ynew, nullptr, nullptr, false);
-  } else {
-    if constexpr (has_jac<F>::value) ros_trial<F, T>(y, h, th, ynew, nullptr, false);
-  }
-}
 
 template <class F, class T>
 void replay_outputs(Method method, const T* y0, const T* th,

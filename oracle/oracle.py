@@ -17,7 +17,7 @@ from . import build_oracle
 
 FIELDS = {"lotka_volterra": 0, "lorenz63": 1, "mlp": 2, "robertson": 3, "nfw_mn": 4,
           "linear1": 5, "linear2": 6, "linear3": 7, "log_halo": 8}
-METHODS = {"tsit5": 0, "ros34pw2": 1}
+METHODS = {"tsit5": 0, "ros34pw2": 1, "vern7": 2}
 
 _lib = None
 
@@ -45,6 +45,7 @@ def lib():
         L.orc_count_ops.argtypes = [i, i, vp, vp, d, vp]
         L.orc_tsit5_tableau.argtypes = [vp, vp, vp, vp]
         L.orc_ros34pw2_tableau.argtypes = [vp, vp, vp, vp, vp]
+        L.orc_vern7_tableau.argtypes = [vp, vp, vp]
         _lib = L
     return _lib
 
@@ -251,6 +252,12 @@ def tsit5_tableau():
     c, A, b, bt = np.zeros(7), np.zeros((7, 7)), np.zeros(7), np.zeros(7)
     lib().orc_tsit5_tableau(_p(c), _p(A), _p(b), _p(bt))
     return c, A, b, bt
+
+
+def vern7_tableau():
+    A, b, bh = np.zeros((10, 10)), np.zeros(10), np.zeros(10)
+    lib().orc_vern7_tableau(_p(A), _p(b), _p(bh))
+    return A, b, bh
 
 
 def ros34pw2_tableau():
