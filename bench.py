@@ -39,6 +39,12 @@ FLOPS_FORWARD_ATTEMPT = {"nfw_mn": 611, "lorenz63": 254, "lotka_volterra": 181, 
 # 48 d (stage tangents 35 d, result 13 d) + 6 c_t per column, c_t = the forward-mode rules' extra
 # operations over f (the value part that the kernel recomputes alongside is not counted).
 FLOPS_SENS_STEP = {"log_halo": 912}
+# Verner 7, counted the same way from its table (nonzero a_ij per stage row 1, 2, 2, 3, 4, 5, 6,
+# 7, 6; b has 7 nonzeros, b - b_hat 8): per attempt 117 d + 10 c_f + 5 (nine new stages and the
+# fresh first stage of the next step); per accepted step of the replay adjoint 160 d + 8 c_f +
+# 9 c_v (stages 2..9 recomputed, nine pullbacks).  c_f, c_v as for Tsit5.
+FLOPS_VERN7_ATTEMPT = {"lorenz63": 436, "nfw_mn": 1047}
+FLOPS_VERN7_ADJOINT = {"lorenz63": 724, "nfw_mn": 2015}
 # The MLP field (4-32-32-4, tanh) counted by hand: f = 1,280 multiply-adds + 68 bias adds + 64
 # tanh = 2,692 ops; its pullback = the two transposed products (2 x 1,280 flops), the weight
 # outer products (2 x 1,280), 2 x 64 for tanh' and 68 bias cotangents = 5,316 ops; per accepted
@@ -66,7 +72,9 @@ def pipe_peak_tflops(mhz, lanes):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms around the timed region.  The
+    sampler is started (and its first sample awaited) before the region begins, and samples taken
+    within 250 ms of the region's ends count, so that short regions still carry a reading."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -74,8 +82,16 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
+        self.samples = []
+        self.t0 = self.t1 = None
+
+    def _reader(self):
+        for line in self.proc.stdout:
+            if line.strip():
+                self.samples.append((time.perf_counter(), line))
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
@@ -83,23 +99,32 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+        if self.proc is not None:
+            self.thread = threading.Thread(target=self._reader, daemon=True)
+            self.thread.start()
+            deadline = time.perf_counter() + 3.0
+            while not self.samples and time.perf_counter() < deadline:
+                time.sleep(0.01)
+        self.t0 = time.perf_counter()
         return self
 
     def __exit__(self, *a):
-        self.lines = []
+        self.t1 = time.perf_counter()
         if self.proc is not None:
+            time.sleep(0.25)
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+            self.thread.join(timeout=5)
 
     def summary(self):
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
+        lines = [l for (ts, l) in self.samples
+                 if self.t0 is not None and self.t0 - 0.25 <= ts <= self.t1 + 0.25]
+        for l in lines:
             f = [x.strip() for x in l.split(",")]
             if len(f) < 9:
                 continue
@@ -121,7 +146,9 @@ DESCR = {"nfw_mn": "stellar orbits: NFW halo + Miyamoto-Nagai disk",
          "nfw_mn_f32": "stellar orbits: NFW halo + Miyamoto-Nagai disk",
          "lorenz63": "Lorenz-63", "lotka_volterra": "Lotka-Volterra",
          "robertson": "Robertson kinetics (stiff)", "mlp": "neural RHS 4-32-32-4 tanh, shared weights",
-         "log_halo": "stellar orbits in a flattened logarithmic halo, theta = (v_c, q) shared"}
+         "log_halo": "stellar orbits in a flattened logarithmic halo, theta = (v_c, q) shared",
+         "lorenz63_vern7": "Lorenz-63, Verner 7(6) pair",
+         "nfw_mn_vern7": "stellar orbits: NFW halo + Miyamoto-Nagai disk, Verner 7(6) pair"}
 
 
 def workload_config(ws, N=1 << 20, name="nfw_mn", w=None, step=None):
@@ -228,6 +255,10 @@ WORKLOADS = {
                            adj=FLOPS_ADJOINT_STEP["lotka_volterra"]),
     "robertson": dict(dtype="f64", fwd=None, adj=None),
     "mlp": dict(dtype="f32", fwd=FLOPS_FORWARD_ATTEMPT["mlp"], adj=FLOPS_ADJOINT_STEP["mlp"]),
+    "lorenz63_vern7": dict(dtype="f64", fwd=FLOPS_VERN7_ATTEMPT["lorenz63"],
+                           adj=FLOPS_VERN7_ADJOINT["lorenz63"]),
+    "nfw_mn_vern7": dict(dtype="f64", fwd=FLOPS_VERN7_ATTEMPT["nfw_mn"],
+                         adj=FLOPS_VERN7_ADJOINT["nfw_mn"]),
     "log_halo": dict(dtype="f64", fwd=FLOPS_FORWARD_ATTEMPT["log_halo"],
                      adj=FLOPS_ADJOINT_STEP["log_halo"], sens=FLOPS_SENS_STEP["log_halo"],
                      step="sens"),
@@ -590,7 +621,7 @@ def main():
                 "flops_per_unit": per_unit, "unit_counted": unit_name, "kernel_ms": ms,
                 "frac_at_measured_clock": achieved / at_clock if (achieved and at_clock) else None}
 
-    method = "Tsit5" if w.method == "tsit5" else "ROS34PW2"
+    method = {"tsit5": "Tsit5", "vern7": "Vern7", "ros34pw2": "ROS34PW2"}[w.method]
     rec_kernel_ms = statistics.median(solve_ms)
     traffic = TRAFFIC_PER_STEP if args.workload == "nfw_mn" else {}
     roof_rec = roof("k_solve<%s, %s, %s, record>" % (w.field, "double" if f64 else "float", method),

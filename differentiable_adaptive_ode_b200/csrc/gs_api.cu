@@ -64,12 +64,14 @@ gs_status check_system(const gs_system* sys) {
   if (!field_info(sys->field, &fi)) return fail(GS_ERR_INVALID_ARG, "unknown field %d", sys->field);
   if (sys->dtype != GS_F64 && sys->dtype != GS_F32)
     return fail(GS_ERR_INVALID_ARG, "unknown dtype %d", sys->dtype);
-  if (sys->method != GS_TSIT5 && sys->method != GS_ROS34PW2)
+  if (sys->method != GS_TSIT5 && sys->method != GS_ROS34PW2 && sys->method != GS_VERN7)
     return fail(GS_ERR_INVALID_ARG, "unknown method %d", sys->method);
   if (sys->d != fi.d || sys->m != fi.m)
     return fail(GS_ERR_INVALID_ARG, "field %d has d=%d m=%d, got d=%d m=%d", sys->field, fi.d,
                 fi.m, sys->d, sys->m);
-  if ((sys->method == GS_TSIT5 && !fi.tsit5) || (sys->method == GS_ROS34PW2 && !fi.ros))
+  if (((sys->method == GS_TSIT5 || sys->method == GS_VERN7) && !fi.tsit5) ||
+      (sys->method == GS_ROS34PW2 && !fi.ros) ||
+      (sys->method == GS_VERN7 && sys->field == GS_MLP_4_32_32_4))
     return fail(GS_ERR_UNSUPPORTED, "field %d is not built for method %d", sys->field, sys->method);
   if (sys->theta_shared != 0 && sys->theta_shared != 1)
     return fail(GS_ERR_INVALID_ARG, "theta_shared must be 0 or 1");
@@ -451,6 +453,25 @@ gs_status dispatch(const gs_system& s, Fn&& fn) {
       case GS_MLP_4_32_32_4:
         return f64 ? fn.template operator()<FMlpWarp, double, M_TSIT5>()
                    : fn.template operator()<FMlpWarp, float, M_TSIT5>();
+      default: break;
+    }
+  } else if (s.method == GS_VERN7) {
+    switch (s.field) {
+      case GS_LOTKA_VOLTERRA:
+        return f64 ? fn.template operator()<FLotkaVolterra, double, M_VERN7>()
+                   : fn.template operator()<FLotkaVolterra, float, M_VERN7>();
+      case GS_LORENZ63:
+        return f64 ? fn.template operator()<FLorenz63, double, M_VERN7>()
+                   : fn.template operator()<FLorenz63, float, M_VERN7>();
+      case GS_NFW_MN:
+        return f64 ? fn.template operator()<FNfwMiyamotoNagai, double, M_VERN7>()
+                   : fn.template operator()<FNfwMiyamotoNagai, float, M_VERN7>();
+      case GS_LINEAR:
+        return f64 ? fn.template operator()<FLinear3, double, M_VERN7>()
+                   : fn.template operator()<FLinear3, float, M_VERN7>();
+      case GS_LOG_HALO:
+        return f64 ? fn.template operator()<FLogHalo, double, M_VERN7>()
+                   : fn.template operator()<FLogHalo, float, M_VERN7>();
       default: break;
     }
   } else {

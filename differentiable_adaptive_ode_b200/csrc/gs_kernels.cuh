@@ -120,7 +120,11 @@ __device__ R initial_step(const R (&y0)[F::D], const R (&f0)[F::D],
   return h;
 }
 
-constexpr int M_TSIT5 = 0, M_ROS = 1;
+constexpr int M_TSIT5 = 0, M_ROS = 1, M_VERN7 = 2;
+template <int METHOD> struct MethodOrder;
+template <> struct MethodOrder<M_TSIT5> { static constexpr int p = Tsit5::order, q = Tsit5::err_order; };
+template <> struct MethodOrder<M_ROS> { static constexpr int p = Ros34pw2::order, q = Ros34pw2::err_order; };
+template <> struct MethodOrder<M_VERN7> { static constexpr int p = Vern7::order, q = Vern7::err_order; };
 
 // Minimum resident 128-thread blocks per SM asked of the compiler (register cap 65536 / (128 b)).
 // Measured on B200 for the stellar field in double precision: the replay adjoint runs 13 % faster
@@ -133,7 +137,8 @@ template <class F, class R> struct Tune { static constexpr int adj_blocks = 1, s
 template <class F, class R> struct Roll { static constexpr bool value = false; };
 template <class R> struct Roll<FNfwMiyamotoNagai, R> { static constexpr bool value = true; };
 // The rolled forward/record kernel of the same field: 3 blocks (170 registers) is 13 % faster on
-// the record pass than unconstrained.
+// the record pass than unconstrained.  (Verner 7 kernels keep nine stage vectors live and are
+// left unconstrained.)
 template <> struct Tune<FNfwMiyamotoNagai, double> {
   static constexpr int adj_blocks = 3, solve_blocks = 3;
 };
@@ -173,11 +178,12 @@ __host__ __device__ constexpr size_t solve_smem_bytes() {
 // solve's; on each accepted step every column S_{:,j} takes the tangent step of that step along
 // (S_{:,j}, e_j).  S lives in shared memory (indexed by the column loop), one slab per lane.
 template <class F, class R, int METHOD, bool REC, bool SENS = false>
-__global__ void __launch_bounds__(128, Tune<F, R>::solve_blocks) k_solve(SolveParams<R> p) {
+__global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve_blocks)
+    k_solve(SolveParams<R> p) {
   using L = RecLayout<F, R>;
   constexpr int D = F::D;
-  constexpr int order = METHOD == M_TSIT5 ? Tsit5::order : Ros34pw2::order;
-  constexpr int qerr = METHOD == M_TSIT5 ? Tsit5::err_order : Ros34pw2::err_order;
+  constexpr int order = MethodOrder<METHOD>::p;
+  constexpr int qerr = MethodOrder<METHOD>::q;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   // shared memory: [record staging, REC only][start-up ring of this block's warps]
@@ -318,6 +324,8 @@ __global__ void __launch_bounds__(128, Tune<F, R>::solve_blocks) k_solve(SolvePa
 #pragma unroll
             for (int c = 0; c < D; ++c) k1[c] = k7[c];
           }
+        } else if constexpr (METHOD == M_VERN7) {
+          err = vern7_trial<F, R>(y, h, th, k1, ynew, p.rtol, p.atol);
         } else {
           err = ros_trial<F, R>(y, h, th, ynew, p.rtol, p.atol);
         }
@@ -355,6 +363,7 @@ __global__ void __launch_bounds__(128, Tune<F, R>::solve_blocks) k_solve(SolvePa
           t = (clipped || t + h >= p.t1) ? p.t1 : t + h;
 #pragma unroll
           for (int c = 0; c < D; ++c) y[c] = ynew[c];
+          if constexpr (METHOD == M_VERN7) F::f(y, th, k1);   // fresh first stage (no FSAL)
           h = h * fac;
           last_rej = false;
           if (t == p.t1) st = 0;
@@ -450,7 +459,8 @@ struct AdjointParams {
 };
 
 template <class F, class R, int METHOD>
-__global__ void __launch_bounds__(128, Tune<F, R>::adj_blocks) k_adjoint(AdjointParams<R> p) {
+__global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_blocks)
+    k_adjoint(AdjointParams<R> p) {
   using L = RecLayout<F, R>;
   constexpr int D = F::D, M = F::M;
   extern __shared__ __align__(16) unsigned char adj_smem[];
@@ -510,6 +520,7 @@ __global__ void __launch_bounds__(128, Tune<F, R>::adj_blocks) k_adjoint(Adjoint
 #pragma unroll
         for (int c = 0; c < D; ++c) y[c] = __ldg(e + 2 + c);
         if constexpr (METHOD == M_TSIT5) tsit5_adjoint_step<F, R>(y, h, th, lam, thb, tape, blockDim.x);
+        else if constexpr (METHOD == M_VERN7) vern7_adjoint_step<F, R>(y, h, th, lam, thb);
         else ros_adjoint_step<F, R>(y, h, th, lam, thb);
         --n;
       }
@@ -529,6 +540,16 @@ __global__ void __launch_bounds__(128, Tune<F, R>::adj_blocks) k_adjoint(Adjoint
 // Forward replay over the recorded mesh at (possibly new) parameters: y_{n+1} = Phi(y_n, h_n),
 // rewriting the stored y_n of every step so that a following k_adjoint differentiates the replay
 // at these parameters; writes y_S to y1.  t_n and h_n are left as recorded.
+// One step of the method's replay map Phi(y, h; theta).
+template <class F, class R, int METHOD>
+__device__ __forceinline__ void replay_step(const R (&y)[F::D], R h,
+                                            const typename F::template Theta<R>& th,
+                                            R (&ynew)[F::D]) {
+  if constexpr (METHOD == M_TSIT5) tsit5_replay_step<F, R>(y, h, th, ynew);
+  else if constexpr (METHOD == M_VERN7) vern7_replay_step<F, R>(y, h, th, ynew);
+  else ros_replay_step<F, R>(y, h, th, ynew);
+}
+
 template <class R>
 struct ReplayParams {
   int N;
@@ -582,8 +603,7 @@ __global__ void __launch_bounds__(128) k_replay_forward(ReplayParams<R> p) {
 #pragma unroll
         for (int c = 0; c < D; ++c) e[2 + c] = y[c];
         R ynew[D];
-        if constexpr (METHOD == M_TSIT5) tsit5_replay_step<F, R>(y, h, th, ynew);
-        else ros_replay_step<F, R>(y, h, th, ynew);
+        replay_step<F, R, METHOD>(y, h, th, ynew);
 #pragma unroll
         for (int c = 0; c < D; ++c) y[c] = ynew[c];
         ++n;
@@ -619,13 +639,6 @@ struct OutParams {
   OutTimes<R> ot;
 };
 
-template <class F, class R, int METHOD>
-__device__ __forceinline__ void replay_step(const R (&y)[F::D], R h,
-                                            const typename F::template Theta<R>& th,
-                                            R (&ynew)[F::D]) {
-  if constexpr (METHOD == M_TSIT5) tsit5_replay_step<F, R>(y, h, th, ynew);
-  else ros_replay_step<F, R>(y, h, th, ynew);
-}
 
 template <class F, class R>
 __device__ __forceinline__ const R* rec_entry(const ReplayParams<R>& p, long long cbase, int n) {
@@ -700,7 +713,8 @@ struct AdjOutParams {
 };
 
 template <class F, class R, int METHOD>
-__global__ void __launch_bounds__(128, Tune<F, R>::adj_blocks) k_adjoint_outputs(AdjOutParams<R> q) {
+__global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_blocks)
+    k_adjoint_outputs(AdjOutParams<R> q) {
   using L = RecLayout<F, R>;
   constexpr int D = F::D, M = F::M;
   extern __shared__ __align__(16) unsigned char adj_smem[];
@@ -754,6 +768,7 @@ __global__ void __launch_bounds__(128, Tune<F, R>::adj_blocks) k_adjoint_outputs
 #pragma unroll
         for (int c = 0; c < D; ++c) lr[c] = r >= jlo ? lo[(size_t)r * D + c] : lam[c];
         if constexpr (METHOD == M_TSIT5) tsit5_adjoint_step<F, R>(y, hr, th, lr, thb, tape, blockDim.x);
+        else if constexpr (METHOD == M_VERN7) vern7_adjoint_step<F, R>(y, hr, th, lr, thb);
         else ros_adjoint_step<F, R>(y, hr, th, lr, thb);
 #pragma unroll
         for (int c = 0; c < D; ++c) lacc[c] += lr[c];

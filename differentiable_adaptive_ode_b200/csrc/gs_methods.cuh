@@ -37,6 +37,46 @@ struct Tsit5 {
                           e7 = 0.015151515151515152;
 };
 
+// Verner's 7(6) pair ("most efficient" IIa, Verner 2010): the seventh-order pair offered next to
+// Tsit5 ("gradsolve: fast exact gradients for ODE ensembles on GPUs" §3.1).  10 stages, not
+// first-same-as-last; b_2 = b_3 = b_10 = 0 and the tenth stage serves only the error estimate.
+// Published decimals.  Zero entries are skipped at compile time in the unrolled stage loops.
+struct Vern7 {
+  static constexpr int order = 7, err_order = 7;
+};
+__host__ __device__ constexpr double vern7_a(int i, int j) {
+  constexpr double A[10][9] = {
+      {0, 0, 0, 0, 0, 0, 0, 0, 0},
+      {0.005, 0, 0, 0, 0, 0, 0, 0, 0},
+      {-1.0767901234567902, 1.185679012345679, 0, 0, 0, 0, 0, 0, 0},
+      {0.04083333333333333, 0, 0.1225, 0, 0, 0, 0, 0, 0},
+      {0.6389139236255726, 0, -2.455672638223657, 2.272258714598084, 0, 0, 0, 0, 0},
+      {-2.6615773750187572, 0, 10.804513886456137, -8.3539146573962, 0.820487594956657, 0, 0,
+       0, 0},
+      {6.067741434696772, 0, -24.711273635911088, 20.427517930788895, -1.9061579788166472,
+       1.006172249242068, 0, 0, 0},
+      {12.054670076253203, 0, -49.75478495046899, 41.142888638604674, -4.461760149974004,
+       2.042334822239175, -0.09834843665406107, 0, 0},
+      {10.138146522881808, 0, -42.6411360317175, 35.76384003992257, -4.3480228403929075,
+       2.009862268377035, 0.3487490460338272, -0.27143900510483127, 0},
+      {-45.030072034298676, 0, 187.3272437654589, -154.02882369350186, 18.56465306347536,
+       -7.141809679295079, 1.3088085781613787, 0, 0}};
+  return A[i][j];
+}
+__host__ __device__ constexpr double vern7_b(int i) {
+  constexpr double B[10] = {0.04715561848627222, 0, 0, 0.25750564298434153, 0.26216653977412624,
+                            0.15216092656738558, 0.4939969170032485, -0.29430311714032503,
+                            0.08131747232495111, 0};
+  return B[i];
+}
+// b - b_hat
+__host__ __device__ constexpr double vern7_e(int i) {
+  constexpr double BH[10] = {0.044608606606341174, 0, 0, 0.26716403785713727,
+                             0.22010183001772932, 0.2188431703143157, 0.22898717054112028, 0, 0,
+                             0.02029518466335628};
+  return vern7_b(i) - BH[i];
+}
+
 // A[i][j] of the explicit stages as a device-evaluable table (i = 0..5 stage index, j < i).
 template <class R> __device__ __forceinline__ R ta(int i, int j) {
   // Resolved at compile time inside fully unrolled loops.
@@ -234,6 +274,138 @@ __device__ __forceinline__ void tsit5_replay_step(const R (&y)[F::D], R h,
     for (int j = 1; j < 6; ++j) s += tb<R>(j) * k[j][c];
     ynew[c] = y[c] + h * s;
   }
+}
+
+// ----------------------------------------------------------------------------------------------
+// Verner 7 one-step maps.  Stage states Y_i = y + h sum_{j<i} a_ij k_j, k_i = f(Y_i).
+// ----------------------------------------------------------------------------------------------
+// Stages 2..NS from y with k1 = f(y) given; k[i] holds slope i (0-based).
+template <class F, class R, int NS>
+__device__ __forceinline__ void vern7_stages(const R (&y)[F::D], R h,
+                                             const typename F::template Theta<R>& th,
+                                             R (&k)[10][F::D]) {
+  constexpr int D = F::D;
+#pragma unroll
+  for (int i = 1; i < NS; ++i) {
+    R Y[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+      R s = R(vern7_a(i, 0)) * k[0][c];
+#pragma unroll
+      for (int j = 1; j < i; ++j)
+        if (vern7_a(i, j) != 0.0) s += R(vern7_a(i, j)) * k[j][c];
+      Y[c] = y[c] + h * s;
+    }
+    F::f(Y, th, k[i]);
+  }
+}
+
+// One Verner 7 trial from y with step h; k1 = f(y) is carried (valid across a rejected trial, and
+// evaluated afresh at the new state after an accepted one: the pair is not first-same-as-last).
+// Returns the scaled RMS error of e = h sum_i (b_i - bh_i) k_i; ynew = y + h sum_i b_i k_i.
+template <class F, class R>
+__device__ __forceinline__ R vern7_trial(const R (&y)[F::D], R h,
+                                         const typename F::template Theta<R>& th,
+                                         const R (&k1)[F::D], R (&ynew)[F::D], R rtol, R atol) {
+  constexpr int D = F::D;
+  R k[10][D];
+#pragma unroll
+  for (int c = 0; c < D; ++c) k[0][c] = k1[c];
+  vern7_stages<F, R, 10>(y, h, th, k);
+  R acc = R(0);
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    R s = R(vern7_b(0)) * k[0][c];
+#pragma unroll
+    for (int j = 1; j < 9; ++j)
+      if (vern7_b(j) != 0.0) s += R(vern7_b(j)) * k[j][c];
+    ynew[c] = y[c] + h * s;
+    R es = R(vern7_e(0)) * k[0][c];
+#pragma unroll
+    for (int j = 1; j < 10; ++j)
+      if (vern7_e(j) != 0.0) es += R(vern7_e(j)) * k[j][c];
+    const R e = h * es;
+    const R sc = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
+    const R q = e / sc;
+    acc += q * q;
+  }
+  return sqrt(acc / R(D));
+}
+
+// The Verner 7 replay map Phi(y, h) = y + h sum_{i<=9} b_i k_i with k_1 = f(y).
+template <class F, class R>
+__device__ __forceinline__ void vern7_replay_step(const R (&y)[F::D], R h,
+                                                  const typename F::template Theta<R>& th,
+                                                  R (&ynew)[F::D]) {
+  constexpr int D = F::D;
+  R k[10][D];
+  F::f(y, th, k[0]);
+  vern7_stages<F, R, 9>(y, h, th, k);
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    R s = R(vern7_b(0)) * k[0][c];
+#pragma unroll
+    for (int j = 1; j < 9; ++j)
+      if (vern7_b(j) != 0.0) s += R(vern7_b(j)) * k[j][c];
+    ynew[c] = y[c] + h * s;
+  }
+}
+
+// Reverse-mode step of the Verner 7 replay map with h fixed (the same rule as the Tsit5 step,
+// nine stages): recompute the stage states from the recorded y_n, then for i = 9..1
+//   kb_i = h (b_i lam + G_i),  Yb_i = J_y(Y_i)^T kb_i,  thb += J_th(Y_i)^T kb_i,
+//   G_j += a_ij Yb_i (j < i),   and finally lam <- lam + sum_i Yb_i.
+template <class F, class R>
+__device__ __forceinline__ void vern7_adjoint_step(const R (&y)[F::D], R h,
+                                                   const typename F::template Theta<R>& th,
+                                                   R (&lam)[F::D], R (&thb)[F::M]) {
+  constexpr int D = F::D;
+  R Y[9][D];
+  {
+    R k[10][D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) Y[0][c] = y[c];
+    F::f(y, th, k[0]);
+#pragma unroll
+    for (int i = 1; i < 9; ++i) {
+#pragma unroll
+      for (int c = 0; c < D; ++c) {
+        R s = R(vern7_a(i, 0)) * k[0][c];
+#pragma unroll
+        for (int j = 1; j < i; ++j)
+          if (vern7_a(i, j) != 0.0) s += R(vern7_a(i, j)) * k[j][c];
+        Y[i][c] = y[c] + h * s;
+      }
+      if (i < 8) F::f(Y[i], th, k[i]);
+    }
+  }
+  R G[8][D], dl[D];
+#pragma unroll
+  for (int c = 0; c < D; ++c) dl[c] = R(0);
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int c = 0; c < D; ++c) G[i][c] = R(0);
+#pragma unroll
+  for (int i = 8; i >= 0; --i) {
+    R kb[D], Yb[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+      R s = (vern7_b(i) != 0.0) ? R(vern7_b(i)) * lam[c] : R(0);
+      if (i < 8) s += G[i][c];
+      kb[c] = h * s;
+    }
+    F::vjp(Y[i], th, kb, Yb, thb);
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+      dl[c] += Yb[c];
+#pragma unroll
+      for (int j = 0; j < i; ++j)
+        if (vern7_a(i, j) != 0.0) G[j][c] += R(vern7_a(i, j)) * Yb[c];
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < D; ++c) lam[c] += dl[c];
 }
 
 // Tangent of one Tsit5 step with h fixed, along the input direction (yd, thd.d):

@@ -47,7 +47,11 @@ typedef enum {
 } gs_status;
 
 typedef enum { GS_F64 = 0, GS_F32 = 1 } gs_dtype;
-typedef enum { GS_TSIT5 = 0, GS_ROS34PW2 = 1 } gs_method;
+/* GS_TSIT5: Tsitouras 5(4), 7 stages, first-same-as-last ([GS] §2.1, the default explicit pair).
+ * GS_ROS34PW2: Rang & Angermann's 4-stage Rosenbrock-Wanner method, order 3(2), for stiff fields.
+ * GS_VERN7: Verner's 7(6) pair, 10 stages, for tight tolerances ([GS] §3.1: the seventh-order
+ * Verner pair offered next to Tsit5); every explicit field except GS_MLP_4_32_32_4. */
+typedef enum { GS_TSIT5 = 0, GS_ROS34PW2 = 1, GS_VERN7 = 2 } gs_method;
 
 /* Built-in fields (all autonomous).  d = state size, m = parameters per trajectory.
  *   GS_LOTKA_VOLTERRA  d=2 m=4     theta = (alpha, beta, gamma, delta)
@@ -74,7 +78,8 @@ typedef enum {
 
 typedef struct {
   int32_t field;        /* gs_field */
-  int32_t method;       /* gs_method: GS_TSIT5 for non-stiff fields, GS_ROS34PW2 for stiff ones */
+  int32_t method;       /* gs_method: GS_TSIT5 or GS_VERN7 for non-stiff fields, GS_ROS34PW2
+                           for stiff ones */
   int32_t dtype;        /* gs_dtype */
   int32_t d, m;         /* must equal the field's sizes (checked) */
   int32_t theta_shared; /* 1: theta is [m] shared by all trajectories; 0: [N][m] */

@@ -11,6 +11,8 @@ c_f and c_v are the op counts (add/sub, mul, div, sqrt or rsqrt, log1p; an FMA c
 field's f and vector-Jacobian product as written in csrc/gs_fields.cuh, tallied by compiling that
 header with a counting scalar (tests/flop_counter.cpp)."""
 import json
+
+import numpy as np
 import os
 import subprocess
 
@@ -51,6 +53,26 @@ def test_sens_constant_matches_counts(counts):
     c = counts["log_halo"]
     c_t = ops(c["fdual"]) - ops(c["f"])
     assert bench.FLOPS_SENS_STEP["log_halo"] == c["M"] * (48 * c["D"] + 6 * c_t)
+
+
+def test_vern7_constants_match_counts(counts, orc):
+    import bench
+    A, b, bh = orc.vern7_tableau()
+    nnz = [int(np.count_nonzero(A[i, :i])) for i in range(1, 10)]
+    assert nnz == [1, 2, 2, 3, 4, 5, 6, 7, 6]
+    nb, ne = int(np.count_nonzero(b[:9])), int(np.count_nonzero(b - bh))
+    # attempt: stage states 2 nnz + 1 each, y_new 2 nb + 1, error 2 ne, scale/quotient/square 5
+    per_c_fwd = sum(2 * n + 1 for n in nnz) + (2 * nb + 1) + 2 * ne + 5
+    # adjoint: stage states 2..9, stage cotangents (3 with b_i != 0, else 1; the last stage 2),
+    # G accumulation 2 per nonzero a_ij of rows 2..9, the nine lam increments and the final add
+    kb = sum(3 if b[i] != 0 else 1 for i in range(8)) + 2
+    per_c_adj = sum(2 * n + 1 for n in nnz[:8]) + kb + 2 * sum(nnz[:8]) + 9 + 1
+    assert (per_c_fwd, per_c_adj) == (117, 160)
+    for field in ("lorenz63", "nfw_mn"):
+        c = counts[field]
+        D = c["D"]
+        assert bench.FLOPS_VERN7_ATTEMPT[field] == 117 * D + 10 * ops(c["f"]) + 5
+        assert bench.FLOPS_VERN7_ADJOINT[field] == 160 * D + 8 * ops(c["f"]) + 9 * ops(c["vjp"])
 
 
 def test_mlp_hand_count():
