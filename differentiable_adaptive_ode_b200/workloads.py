@@ -84,7 +84,7 @@ class Workload:
     atol: float
     seed: int
     target: Optional[np.ndarray] = None   # [N, d] when drawn directly
-    target_kind: str = "given"            # given | nominal_solve | teacher_solve
+    target_kind: str = "given"            # given | nominal_solve | teacher_solve | nominal_y0
     nominal_theta: Optional[np.ndarray] = None
     loss_mask: Optional[np.ndarray] = None  # components of y entering the loss (1) or not (0)
     loss_scale: float = 1.0               # L = loss_scale * sum_k |mask*(y_k - target_k)|^2
@@ -173,6 +173,26 @@ def nfw_mn(N=1 << 20, seed=4, dtype=np.float64, theta_shared=False):
                     loss_mask=mask)
 
 
+HIRES_K = np.array([1.71, 0.43, 8.32, 0.0007, 8.75, 10.03, 0.035, 1.12, 1.745, 280.0, 0.69, 1.81])
+
+
+def hires(N=65536, seed=6):
+    """HIRES (8 components, stiff), rate constants shared at their nominal values; the ensemble
+    varies the initial state (the gradient of interest is with respect to y0):
+    y0 = (u1, 0, 0, 0, 0, 0, 0, 0.0057 u8), u ~ U(0.8, 1.2); t in [0, 321.8122];
+    Rosenbrock23, rtol 1e-6, atol 1e-10.  Loss targets: the final state of the nominal y0."""
+    u = uniform(seed, S_Y0, 2 * N).reshape(N, 2)
+    y0 = np.zeros((N, 8))
+    y0[:, 0] = 0.8 + 0.4 * u[:, 0]
+    y0[:, 7] = 0.0057 * (0.8 + 0.4 * u[:, 1])
+    nominal_y0 = np.array([1.0, 0, 0, 0, 0, 0, 0, 0.0057])
+    w = Workload("hires", "hires", "rosenbrock23", np.float64, N, 8, 12, True, HIRES_K.copy(), y0,
+                 0.0, 321.8122, 1e-6, 1e-10, seed, target_kind="nominal_y0",
+                 nominal_theta=HIRES_K.copy())
+    w.notes["nominal_y0"] = nominal_y0
+    return w
+
+
 LOG_HALO_RC = 0.2
 
 
@@ -225,7 +245,7 @@ def log_halo(N=1 << 20, seed=5, dtype=np.float64):
 
 def by_name(name: str, N: Optional[int] = None, **kw) -> Workload:
     table = {"lotka_volterra": lotka_volterra, "lorenz63": lorenz63, "mlp": mlp,
-             "robertson": robertson, "nfw_mn": nfw_mn, "log_halo": log_halo}
+             "robertson": robertson, "nfw_mn": nfw_mn, "log_halo": log_halo, "hires": hires}
     if name == "nfw_mn_f32":
         return nfw_mn(N=N if N else 1 << 20, dtype=np.float32, **kw)
     if name.endswith("_vern7"):

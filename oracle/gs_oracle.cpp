@@ -17,7 +17,7 @@ namespace {
 using namespace orc;
 
 enum FieldId { F_LV = 0, F_LORENZ = 1, F_MLP = 2, F_ROBERTSON = 3, F_NFW = 4, F_LIN1 = 5,
-               F_LIN2 = 6, F_LIN3 = 7, F_LOGHALO = 8 };
+               F_LIN2 = 6, F_LIN3 = 7, F_LOGHALO = 8, F_HIRES = 9 };
 
 template <class Fn>
 void parallel_for(long long N, int nthreads, Fn fn) {
@@ -196,6 +196,7 @@ int with_field(int field, Fn&& fn) {
     case F_LIN2: return fn(Linear<2>{});
     case F_LIN3: return fn(Linear<3>{});
     case F_LOGHALO: return fn(LogHalo{});
+    case F_HIRES: return fn(Hires{});
     default: return -2;
   }
 }
@@ -203,7 +204,7 @@ int with_field(int field, Fn&& fn) {
 template <class F>
 bool method_ok(int method) {
   if (method == TSIT5 || method == VERN7) return true;
-  if (method == ROS34PW2) return has_jac<F>::value;
+  if (method == ROS34PW2 || method == RB23) return has_jac<F>::value;
   return false;
 }
 
@@ -388,6 +389,8 @@ int orc_trial(int field, int method, const double* theta, const double* y, doubl
       double k1[F::D];
       F::f(y, theta, k1);
       vern7_trial<F, double>(y, h, theta, k1, ynew, e, true);
+    } else if (method == RB23) {
+      if constexpr (has_jac<F>::value) rb23_trial<F, double>(y, h, theta, ynew, e, true);
     } else {
       if constexpr (has_jac<F>::value) ros_trial<F, double>(y, h, theta, ynew, e, true);
     }

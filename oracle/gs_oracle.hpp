@@ -188,6 +188,46 @@ struct Robertson {
   }
 };
 
+// HIRES (Schaefer 1975; Hairer & Wanner II, §IV.10: "high irradiance responses" of
+// photomorphogenesis), the stiff eight-component system of [GS] §4.5 / §4.6.  The twelve rate
+// constants are the parameters, theta = (k1..k12), nominal
+//   (1.71, 0.43, 8.32, 0.0007, 8.75, 10.03, 0.035, 1.12, 1.745, 280, 0.69, 1.81):
+//   y1' = -k1 y1 + k2 y2 + k3 y3 + k4
+//   y2' =  k1 y1 - k5 y2
+//   y3' = -k6 y3 + k2 y4 + k7 y5
+//   y4' =  k3 y2 + k1 y3 - k8 y4
+//   y5' = -k9 y5 + k2 y6 + k2 y7
+//   y6' = -k10 y6 y8 + k11 y4 + k1 y5 - k2 y6 + k11 y7
+//   y7' =  k10 y6 y8 - k12 y7
+//   y8' = -k10 y6 y8 + k12 y7
+struct Hires {
+  static constexpr int D = 8, M = 12;
+  template <class T> static void f(const T* y, const T* k, T* dy) {
+    const T r = k[9] * y[5] * y[7];
+    dy[0] = -(k[0] * y[0]) + k[1] * y[1] + k[2] * y[2] + k[3];
+    dy[1] = k[0] * y[0] - k[4] * y[1];
+    dy[2] = -(k[5] * y[2]) + k[1] * y[3] + k[6] * y[4];
+    dy[3] = k[2] * y[1] + k[0] * y[2] - k[7] * y[3];
+    dy[4] = -(k[8] * y[4]) + k[1] * y[5] + k[1] * y[6];
+    dy[5] = -r + k[10] * y[3] + k[0] * y[4] - k[1] * y[5] + k[10] * y[6];
+    dy[6] = r - k[11] * y[6];
+    dy[7] = -r + k[11] * y[6];
+  }
+  // J = df/dy, row-major, written out from f above.
+  template <class T> static void jac(const T* y, const T* k, T* J) {
+    for (int i = 0; i < 64; ++i) J[i] = T(0);
+    J[0 * 8 + 0] = -k[0]; J[0 * 8 + 1] = k[1];  J[0 * 8 + 2] = k[2];
+    J[1 * 8 + 0] = k[0];  J[1 * 8 + 1] = -k[4];
+    J[2 * 8 + 2] = -k[5]; J[2 * 8 + 3] = k[1];  J[2 * 8 + 4] = k[6];
+    J[3 * 8 + 1] = k[2];  J[3 * 8 + 2] = k[0];  J[3 * 8 + 3] = -k[7];
+    J[4 * 8 + 4] = -k[8]; J[4 * 8 + 5] = k[1];  J[4 * 8 + 6] = k[1];
+    J[5 * 8 + 3] = k[10]; J[5 * 8 + 4] = k[0];  J[5 * 8 + 5] = -(k[9] * y[7]) - k[1];
+    J[5 * 8 + 6] = k[10]; J[5 * 8 + 7] = -(k[9] * y[5]);
+    J[6 * 8 + 5] = k[9] * y[7]; J[6 * 8 + 6] = -k[11]; J[6 * 8 + 7] = k[9] * y[5];
+    J[7 * 8 + 5] = -(k[9] * y[7]); J[7 * 8 + 6] = k[11]; J[7 * 8 + 7] = -(k[9] * y[5]);
+  }
+};
+
 // Test particle in an NFW halo plus a Miyamoto-Nagai disk, G = 1; state (x, y, z, vx, vy, vz),
 // theta = (M_h, r_s, M_d, a, b).
 //   Phi = -M_h ln(1 + r/r_s)/r  -  M_d / sqrt(R^2 + (a + sqrt(z^2 + b^2))^2),  x'' = -grad Phi.
@@ -517,14 +557,60 @@ void ros_trial(const T* y, T h, const T* th, T* ynew, T* e, bool want_err) {
   }
 }
 
-enum Method { TSIT5 = 0, ROS34PW2 = 1, VERN7 = 2 };
+// Rosenbrock23 (Shampine & Reichelt 1997, the pair of MATLAB's ode23s; [GS] §3.1: the
+// second-order linearly implicit method of the fused stiff kernels), autonomous form, exact J:
+//   d = 1/(2 + sqrt 2),  W = I - h d J,  J = f_y(y_n)
+//   F0 = f(y_n),  k1 = W^{-1} F0,  F1 = f(y_n + h k1 / 2),  k2 = W^{-1} (F1 - k1) + k1,
+//   y_{n+1} = y_n + h k2,
+//   F2 = f(y_{n+1}),  k3 = W^{-1} (F2 - e32 (k2 - F1) - 2 (k1 - F0)),  e32 = 6 + sqrt 2,
+//   error estimate e = h (k1 - 2 k2 + k3) / 6.
+struct Rb23Tab {
+  static constexpr int order = 2;
+  static constexpr int err_order = 3;   // the estimate is the local error of the order-2 step
+  static constexpr double d = 0.29289321881345248;    // 1 / (2 + sqrt 2)
+  static constexpr double e32 = 7.4142135623730951;   // 6 + sqrt 2
+};
+
+template <class F, class T>
+void rb23_trial(const T* y, T h, const T* th, T* ynew, T* e, bool want_err) {
+  constexpr int D = F::D;
+  T J[D * D], W[D * D];
+  int piv[D];
+  F::jac(y, th, J);
+  const T hd = h * cst<T>(Rb23Tab::d);
+  for (int r = 0; r < D; ++r)
+    for (int c = 0; c < D; ++c) W[r * D + c] = T(r == c ? 1.0 : 0.0) - hd * J[r * D + c];
+  lu_factor<T, D>(W, piv);
+  T F0[D], k1[D], Y1[D], F1[D], k2[D];
+  F::f(y, th, F0);
+  for (int c = 0; c < D; ++c) k1[c] = F0[c];
+  lu_solve<T, D>(W, piv, k1);
+  for (int c = 0; c < D; ++c) Y1[c] = y[c] + cst<T>(0.5) * h * k1[c];
+  F::f(Y1, th, F1);
+  for (int c = 0; c < D; ++c) k2[c] = F1[c] - k1[c];
+  lu_solve<T, D>(W, piv, k2);
+  for (int c = 0; c < D; ++c) k2[c] = k2[c] + k1[c];
+  for (int c = 0; c < D; ++c) ynew[c] = y[c] + h * k2[c];
+  if (!want_err) return;
+  T F2[D], k3[D];
+  F::f(ynew, th, F2);
+  for (int c = 0; c < D; ++c)
+    k3[c] = F2[c] - cst<T>(Rb23Tab::e32) * (k2[c] - F1[c]) - cst<T>(2.0) * (k1[c] - F0[c]);
+  lu_solve<T, D>(W, piv, k3);
+  for (int c = 0; c < D; ++c)
+    e[c] = h * (k1[c] - cst<T>(2.0) * k2[c] + k3[c]) / cst<T>(6.0);
+}
+
+enum Method { TSIT5 = 0, ROS34PW2 = 1, VERN7 = 2, RB23 = 3 };
 
 inline int method_order(Method m) {
-  return m == TSIT5 ? Tsit5Tab::order : m == VERN7 ? Vern7Tab::order : Ros34pw2Tab::order;
+  return m == TSIT5 ? Tsit5Tab::order : m == VERN7 ? Vern7Tab::order
+                                      : m == RB23 ? Rb23Tab::order : Ros34pw2Tab::order;
 }
 inline int method_err_order(Method m) {
   return m == TSIT5 ? Tsit5Tab::err_order : m == VERN7 ? Vern7Tab::err_order
-                                                       : Ros34pw2Tab::err_order;
+                                          : m == RB23 ? Rb23Tab::err_order
+                                                      : Ros34pw2Tab::err_order;
 }
 
 // has_jac<F>: stiff fields carry an analytic Jacobian.
@@ -622,6 +708,8 @@ Record<R> solve(Method method, const R* y0, const R* th, R t0, R t1, R rtol, R a
       tsit5_trial<F, R>(y, h, th, k1, ynew, k7, e, true);
     } else if (method == VERN7) {
       vern7_trial<F, R>(y, h, th, k1, ynew, e, true);
+    } else if (method == RB23) {
+      if constexpr (has_jac<F>::value) rb23_trial<F, R>(y, h, th, ynew, e, true);
     } else {
       if constexpr (has_jac<F>::value) ros_trial<F, R>(y, h, th, ynew, e, true);
     }
@@ -665,6 +753,8 @@ void one_step(Method method, const T* y, const T* th, T h, T* ynew) {
     F::f(y, th, k1);
     if (method == TSIT5) tsit5_trial<F, T>(y, h, th, k1, ynew, nullptr, nullptr, false);
     else vern7_trial<F, T>(y, h, th, k1, ynew, nullptr, false);
+  } else if (method == RB23) {
+    if constexpr (has_jac<F>::value) rb23_trial<F, T>(y, h, th, ynew, nullptr, false);
   } else {
     if constexpr (has_jac<F>::value) ros_trial<F, T>(y, h, th, ynew, nullptr, false);
   }

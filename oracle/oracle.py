@@ -16,8 +16,8 @@ import numpy as np
 from . import build_oracle
 
 FIELDS = {"lotka_volterra": 0, "lorenz63": 1, "mlp": 2, "robertson": 3, "nfw_mn": 4,
-          "linear1": 5, "linear2": 6, "linear3": 7, "log_halo": 8}
-METHODS = {"tsit5": 0, "ros34pw2": 1, "vern7": 2}
+          "linear1": 5, "linear2": 6, "linear3": 7, "log_halo": 8, "hires": 9}
+METHODS = {"tsit5": 0, "ros34pw2": 1, "vern7": 2, "rosenbrock23": 3}
 
 _lib = None
 

@@ -37,10 +37,21 @@ def test_vern7_record_forward_and_gradient(orc, name, N):
     assert np.all(out["status"] == 0) and np.all(ref["status"] == 0)
     assert np.array_equal(ex["S"], ref["S"])
     assert U.rel_rows(out["y1"], ref["y1"], w.atol).max() <= 1e-9
-    for k in range(min(N, 40)):
-        S = ex["S"][k]
-        dh = np.max(np.abs(ex["H"][k, :S] - ref["H"][k, :S])) / np.max(np.abs(ref["H"][k, :S]))
-        assert dh <= 1e-6, (k, dh)
+    # step sizes: the Verner controller's step sequence sits on a wider rounding floor than
+    # Tsit5's (its error estimate cancels terms of size |a_ij| ~ 190): the bar is the oracle's own
+    # spread under a one-ulp change of y0 (same counts, measured 2e-3 on the stellar ensemble)
+    yp = w.y0 * (1 + np.finfo(np.float64).eps)
+    ref2 = orc.solve(w.field, w.method, w.theta, yp, w.t0, w.t1, w.rtol, w.atol,
+                     theta_shared=w.theta_shared, keep_record=True, nthreads=8)
+
+    def dh(Ha, Hb, S):
+        return np.max(np.abs(Ha[:S] - Hb[:S])) / np.max(np.abs(Hb[:S]))
+
+    same = np.flatnonzero(ref2["S"] == ref["S"])
+    spread = max([dh(ref2["H"][k], ref["H"][k], ref["S"][k]) for k in same] + [1e-7])
+    gpu = max(dh(ex["H"][k], ref["H"][k], ex["S"][k]) for k in range(N))
+    print("vern7 step sizes: gpu %.3g, oracle 1-ulp spread %.3g" % (gpu, spread))
+    assert gpu <= max(1e-6, 3 * spread)
     fw = U.forward(w)
     assert np.array_equal(fw["S"], ex["S"]) and np.array_equal(fw["y1"], out["y1"])
     assert np.array_equal(fw["rejected"], ref["rejected"])
