@@ -148,6 +148,8 @@ DESCR = {"nfw_mn": "stellar orbits: NFW halo + Miyamoto-Nagai disk",
          "robertson": "Robertson kinetics (stiff)", "mlp": "neural RHS 4-32-32-4 tanh, shared weights",
          "log_halo": "stellar orbits in a flattened logarithmic halo, theta = (v_c, q) shared",
          "lorenz63_vern7": "Lorenz-63, Verner 7(6) pair",
+         "robertson_rb23": "Robertson kinetics (stiff), Rosenbrock23",
+         "hires": "HIRES kinetics (stiff, 8 components), Rosenbrock23, shared rate constants",
          "nfw_mn_vern7": "stellar orbits: NFW halo + Miyamoto-Nagai disk, Verner 7(6) pair"}
 
 
@@ -254,6 +256,8 @@ WORKLOADS = {
     "lotka_volterra": dict(dtype="f64", fwd=FLOPS_FORWARD_ATTEMPT["lotka_volterra"],
                            adj=FLOPS_ADJOINT_STEP["lotka_volterra"]),
     "robertson": dict(dtype="f64", fwd=None, adj=None),
+    "robertson_rb23": dict(dtype="f64", fwd=None, adj=None),
+    "hires": dict(dtype="f64", fwd=None, adj=None),
     "mlp": dict(dtype="f32", fwd=FLOPS_FORWARD_ATTEMPT["mlp"], adj=FLOPS_ADJOINT_STEP["mlp"]),
     "lorenz63_vern7": dict(dtype="f64", fwd=FLOPS_VERN7_ATTEMPT["lorenz63"],
                            adj=FLOPS_VERN7_ADJOINT["lorenz63"]),
@@ -485,6 +489,10 @@ def main():
     # the caller's loss targets: drawn, or solved on the GPU at nominal / teacher parameters
     if w.target is not None:
         target = torch.as_tensor(w.target, dtype=dt, device=dev)
+    elif w.target_kind == "nominal_y0":
+        y0n = torch.as_tensor(np.tile(w.notes["nominal_y0"], (N, 1)), dtype=dt, device=dev)
+        target = torch.empty((N, d), dtype=dt, device=dev)
+        G.gs_solve_forward(sys_, N, th, y0n, w.t0, w.t1, w.rtol, w.atol, target)
     elif w.target_kind == "nominal_solve":
         thn = torch.as_tensor(np.tile(w.nominal_theta, (N, 1)), dtype=dt, device=dev)
         target = torch.empty((N, d), dtype=dt, device=dev)
@@ -621,7 +629,8 @@ def main():
                 "flops_per_unit": per_unit, "unit_counted": unit_name, "kernel_ms": ms,
                 "frac_at_measured_clock": achieved / at_clock if (achieved and at_clock) else None}
 
-    method = {"tsit5": "Tsit5", "vern7": "Vern7", "ros34pw2": "ROS34PW2"}[w.method]
+    method = {"tsit5": "Tsit5", "vern7": "Vern7", "ros34pw2": "ROS34PW2",
+              "rosenbrock23": "Rosenbrock23"}[w.method]
     rec_kernel_ms = statistics.median(solve_ms)
     traffic = TRAFFIC_PER_STEP if args.workload == "nfw_mn" else {}
     roof_rec = roof("k_solve<%s, %s, %s, record>" % (w.field, "double" if f64 else "float", method),

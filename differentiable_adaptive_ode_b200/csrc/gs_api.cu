@@ -54,6 +54,7 @@ bool field_info(int field, FieldInfo* fi) {
     case GS_NFW_MN: *fi = {6, 5, true, false}; return true;
     case GS_LINEAR: *fi = {3, 9, true, true}; return true;
     case GS_LOG_HALO: *fi = {6, 2, true, false}; return true;
+    case GS_HIRES: *fi = {8, 12, false, true}; return true;
     default: return false;
   }
 }
@@ -64,13 +65,14 @@ gs_status check_system(const gs_system* sys) {
   if (!field_info(sys->field, &fi)) return fail(GS_ERR_INVALID_ARG, "unknown field %d", sys->field);
   if (sys->dtype != GS_F64 && sys->dtype != GS_F32)
     return fail(GS_ERR_INVALID_ARG, "unknown dtype %d", sys->dtype);
-  if (sys->method != GS_TSIT5 && sys->method != GS_ROS34PW2 && sys->method != GS_VERN7)
+  if (sys->method != GS_TSIT5 && sys->method != GS_ROS34PW2 && sys->method != GS_VERN7 &&
+      sys->method != GS_ROSENBROCK23)
     return fail(GS_ERR_INVALID_ARG, "unknown method %d", sys->method);
   if (sys->d != fi.d || sys->m != fi.m)
     return fail(GS_ERR_INVALID_ARG, "field %d has d=%d m=%d, got d=%d m=%d", sys->field, fi.d,
                 fi.m, sys->d, sys->m);
   if (((sys->method == GS_TSIT5 || sys->method == GS_VERN7) && !fi.tsit5) ||
-      (sys->method == GS_ROS34PW2 && !fi.ros) ||
+      ((sys->method == GS_ROS34PW2 || sys->method == GS_ROSENBROCK23) && !fi.ros) ||
       (sys->method == GS_VERN7 && sys->field == GS_MLP_4_32_32_4))
     return fail(GS_ERR_UNSUPPORTED, "field %d is not built for method %d", sys->field, sys->method);
   if (sys->theta_shared != 0 && sys->theta_shared != 1)
@@ -474,11 +476,27 @@ gs_status dispatch(const gs_system& s, Fn&& fn) {
                    : fn.template operator()<FLogHalo, float, M_VERN7>();
       default: break;
     }
+  } else if (s.method == GS_ROSENBROCK23) {
+    switch (s.field) {
+      case GS_ROBERTSON:
+        return f64 ? fn.template operator()<FRobertson, double, M_RB23>()
+                   : fn.template operator()<FRobertson, float, M_RB23>();
+      case GS_HIRES:
+        return f64 ? fn.template operator()<FHires, double, M_RB23>()
+                   : fn.template operator()<FHires, float, M_RB23>();
+      case GS_LINEAR:
+        return f64 ? fn.template operator()<FLinear3, double, M_RB23>()
+                   : fn.template operator()<FLinear3, float, M_RB23>();
+      default: break;
+    }
   } else {
     switch (s.field) {
       case GS_ROBERTSON:
         return f64 ? fn.template operator()<FRobertson, double, M_ROS>()
                    : fn.template operator()<FRobertson, float, M_ROS>();
+      case GS_HIRES:
+        return f64 ? fn.template operator()<FHires, double, M_ROS>()
+                   : fn.template operator()<FHires, float, M_ROS>();
       case GS_LINEAR:
         return f64 ? fn.template operator()<FLinear3, double, M_ROS>()
                    : fn.template operator()<FLinear3, float, M_ROS>();

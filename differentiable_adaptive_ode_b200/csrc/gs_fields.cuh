@@ -129,6 +129,94 @@ struct FRobertson {
 };
 
 // ----------------------------------------------------------------------------------------------
+// HIRES (Schaefer 1975; Hairer & Wanner II §IV.10), stiff, theta = the twelve rate constants
+// k = (1.71, 0.43, 8.32, 0.0007, 8.75, 10.03, 0.035, 1.12, 1.745, 280, 0.69, 1.81) nominal:
+//   f0 = -k0 y0 + k1 y1 + k2 y2 + k3          f4 = -k8 y4 + k1 y5 + k1 y6
+//   f1 =  k0 y0 - k4 y1                        f5 = -r + k10 y3 + k0 y4 - k1 y5 + k10 y6
+//   f2 = -k5 y2 + k1 y3 + k6 y4                f6 =  r - k11 y6
+//   f3 =  k2 y1 + k0 y2 - k7 y3                f7 = -r + k11 y6,      r = k9 y5 y7.
+// J depends on y only through r (entries (5|6|7, 5|7)), linearly: its derivatives are constants.
+// ----------------------------------------------------------------------------------------------
+struct FHires {
+  static constexpr int D = 8, M = 12;
+  template <class R> struct Theta { R k[12]; };
+  template <class R> GS_HD static void load(Theta<R>& t, const R* s) {
+#pragma unroll
+    for (int i = 0; i < 12; ++i) t.k[i] = s[i];
+  }
+  template <class R> GS_HD static void f(const R* y, const Theta<R>& t, R* dy) {
+    const R* k = t.k;
+    const R r = k[9] * y[5] * y[7];
+    dy[0] = -k[0] * y[0] + k[1] * y[1] + k[2] * y[2] + k[3];
+    dy[1] = k[0] * y[0] - k[4] * y[1];
+    dy[2] = -k[5] * y[2] + k[1] * y[3] + k[6] * y[4];
+    dy[3] = k[2] * y[1] + k[0] * y[2] - k[7] * y[3];
+    dy[4] = -k[8] * y[4] + k[1] * y[5] + k[1] * y[6];
+    dy[5] = -r + k[10] * y[3] + k[0] * y[4] - k[1] * y[5] + k[10] * y[6];
+    dy[6] = r - k[11] * y[6];
+    dy[7] = -r + k[11] * y[6];
+  }
+  template <class R> GS_HD static void jac(const R* y, const Theta<R>& t, R* J) {
+    const R* k = t.k;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) J[i] = R(0);
+    J[0] = -k[0];  J[1] = k[1];  J[2] = k[2];
+    J[8] = k[0];   J[9] = -k[4];
+    J[18] = -k[5]; J[19] = k[1]; J[20] = k[6];
+    J[25] = k[2];  J[26] = k[0]; J[27] = -k[7];
+    J[36] = -k[8]; J[37] = k[1]; J[38] = k[1];
+    const R a = k[9] * y[7], b = k[9] * y[5];
+    J[43] = k[10]; J[44] = k[0]; J[45] = -a - k[1]; J[46] = k[10]; J[47] = -b;
+    J[53] = a;     J[54] = -k[11]; J[55] = b;
+    J[61] = -a;    J[62] = k[11];  J[63] = -b;
+  }
+  template <class R>
+  GS_HD static void vjp(const R* y, const Theta<R>& t, const R* u, R* yb, R* thb) {
+    const R* k = t.k;
+    const R w = u[6] - u[5] - u[7];   // cotangent of r
+    yb[0] = k[0] * (u[1] - u[0]);
+    yb[1] = k[1] * u[0] - k[4] * u[1] + k[2] * u[3];
+    yb[2] = k[2] * u[0] - k[5] * u[2] + k[0] * u[3];
+    yb[3] = k[1] * u[2] - k[7] * u[3] + k[10] * u[5];
+    yb[4] = k[6] * u[2] - k[8] * u[4] + k[0] * u[5];
+    yb[5] = k[1] * (u[4] - u[5]) + k[9] * y[7] * w;
+    yb[6] = k[1] * u[4] + k[10] * u[5] + k[11] * (u[7] - u[6]);
+    yb[7] = k[9] * y[5] * w;
+    thb[0] += y[0] * (u[1] - u[0]) + y[2] * u[3] + y[4] * u[5];
+    thb[1] += y[1] * u[0] + y[3] * u[2] + (y[5] + y[6]) * u[4] - y[5] * u[5];
+    thb[2] += y[2] * u[0] + y[1] * u[3];
+    thb[3] += u[0];
+    thb[4] -= y[1] * u[1];
+    thb[5] -= y[2] * u[2];
+    thb[6] += y[4] * u[2];
+    thb[7] -= y[3] * u[3];
+    thb[8] -= y[4] * u[4];
+    thb[9] += y[5] * y[7] * w;
+    thb[10] += (y[3] + y[6]) * u[5];
+    thb[11] += y[6] * (u[7] - u[6]);
+  }
+  template <class R>
+  GS_HD static void jac_vjp(const R* y, const Theta<R>& t, const R* Jb, R* yb, R* thb) {
+    const R* k = t.k;
+    const R wa = Jb[53] - Jb[45] - Jb[61];   // entries carrying a = k9 y7
+    const R wb = Jb[55] - Jb[47] - Jb[63];   // entries carrying b = k9 y5
+    yb[7] += k[9] * wa;
+    yb[5] += k[9] * wb;
+    thb[0] += Jb[8] - Jb[0] + Jb[26] + Jb[44];
+    thb[1] += Jb[1] + Jb[19] + Jb[37] + Jb[38] - Jb[45];
+    thb[2] += Jb[2] + Jb[25];
+    thb[4] -= Jb[9];
+    thb[5] -= Jb[18];
+    thb[6] += Jb[20];
+    thb[7] -= Jb[27];
+    thb[8] -= Jb[36];
+    thb[9] += y[7] * wa + y[5] * wb;
+    thb[10] += Jb[43] + Jb[46];
+    thb[11] += Jb[62] - Jb[54];
+  }
+};
+
+// ----------------------------------------------------------------------------------------------
 // Linear test field y' = A y, theta = A (row-major 3x3); J = A.
 // ----------------------------------------------------------------------------------------------
 struct FLinear3 {

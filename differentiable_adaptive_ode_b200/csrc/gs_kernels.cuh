@@ -120,11 +120,12 @@ __device__ R initial_step(const R (&y0)[F::D], const R (&f0)[F::D],
   return h;
 }
 
-constexpr int M_TSIT5 = 0, M_ROS = 1, M_VERN7 = 2;
+constexpr int M_TSIT5 = 0, M_ROS = 1, M_VERN7 = 2, M_RB23 = 3;
 template <int METHOD> struct MethodOrder;
 template <> struct MethodOrder<M_TSIT5> { static constexpr int p = Tsit5::order, q = Tsit5::err_order; };
 template <> struct MethodOrder<M_ROS> { static constexpr int p = Ros34pw2::order, q = Ros34pw2::err_order; };
 template <> struct MethodOrder<M_VERN7> { static constexpr int p = Vern7::order, q = Vern7::err_order; };
+template <> struct MethodOrder<M_RB23> { static constexpr int p = Rb23::order, q = Rb23::err_order; };
 
 // Minimum resident 128-thread blocks per SM asked of the compiler (register cap 65536 / (128 b)).
 // Measured on B200 for the stellar field in double precision: the replay adjoint runs 13 % faster
@@ -326,6 +327,13 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
           }
         } else if constexpr (METHOD == M_VERN7) {
           err = vern7_trial<F, R>(y, h, th, k1, ynew, p.rtol, p.atol);
+        } else if constexpr (METHOD == M_RB23) {
+          R F2[D];
+          err = rb23_trial<F, R>(y, h, th, k1, ynew, F2, p.rtol, p.atol);
+          if (err <= R(1)) {
+#pragma unroll
+            for (int c = 0; c < D; ++c) k1[c] = F2[c];   // first-same-as-last
+          }
         } else {
           err = ros_trial<F, R>(y, h, th, ynew, p.rtol, p.atol);
         }
@@ -521,6 +529,7 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
         for (int c = 0; c < D; ++c) y[c] = __ldg(e + 2 + c);
         if constexpr (METHOD == M_TSIT5) tsit5_adjoint_step<F, R>(y, h, th, lam, thb, tape, blockDim.x);
         else if constexpr (METHOD == M_VERN7) vern7_adjoint_step<F, R>(y, h, th, lam, thb);
+        else if constexpr (METHOD == M_RB23) rb23_adjoint_step<F, R>(y, h, th, lam, thb);
         else ros_adjoint_step<F, R>(y, h, th, lam, thb);
         --n;
       }
@@ -547,6 +556,7 @@ __device__ __forceinline__ void replay_step(const R (&y)[F::D], R h,
                                             R (&ynew)[F::D]) {
   if constexpr (METHOD == M_TSIT5) tsit5_replay_step<F, R>(y, h, th, ynew);
   else if constexpr (METHOD == M_VERN7) vern7_replay_step<F, R>(y, h, th, ynew);
+  else if constexpr (METHOD == M_RB23) rb23_replay_step<F, R>(y, h, th, ynew);
   else ros_replay_step<F, R>(y, h, th, ynew);
 }
 
@@ -769,6 +779,7 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
         for (int c = 0; c < D; ++c) lr[c] = r >= jlo ? lo[(size_t)r * D + c] : lam[c];
         if constexpr (METHOD == M_TSIT5) tsit5_adjoint_step<F, R>(y, hr, th, lr, thb, tape, blockDim.x);
         else if constexpr (METHOD == M_VERN7) vern7_adjoint_step<F, R>(y, hr, th, lr, thb);
+        else if constexpr (METHOD == M_RB23) rb23_adjoint_step<F, R>(y, hr, th, lr, thb);
         else ros_adjoint_step<F, R>(y, hr, th, lr, thb);
 #pragma unroll
         for (int c = 0; c < D; ++c) lacc[c] += lr[c];

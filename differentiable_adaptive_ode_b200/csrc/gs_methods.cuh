@@ -741,6 +741,154 @@ __device__ __forceinline__ void ros_replay_step(const R (&y)[F::D], R h,
   }
 }
 
+// ----------------------------------------------------------------------------------------------
+// Rosenbrock23 (Shampine & Reichelt 1997, the pair of MATLAB's ode23s; "gradsolve: fast exact
+// gradients for ODE ensembles on GPUs" §3.1: the second-order linearly implicit method of the
+// fused stiff kernels), autonomous form with the exact J = f_y(y_n), d = 1/(2 + sqrt 2):
+//   W = I - h d J;  F0 = f(y_n);  k1 = W^{-1} F0;  F1 = f(y_n + h k1/2);
+//   k2 = W^{-1} (F1 - k1) + k1;  y_{n+1} = y_n + h k2;
+//   F2 = f(y_{n+1});  k3 = W^{-1} (F2 - e32 (k2 - F1) - 2 (k1 - F0));  e = h (k1 - 2 k2 + k3)/6.
+// F2 is the next step's F0 (first-same-as-last).
+// ----------------------------------------------------------------------------------------------
+struct Rb23 {
+  static constexpr int order = 2, err_order = 3;
+  static constexpr double d = 0.29289321881345248;    // 1 / (2 + sqrt 2)
+  static constexpr double e32 = 7.4142135623730951;   // 6 + sqrt 2
+};
+
+template <class F, class R>
+__device__ __forceinline__ void rb23_matrix(const R (&y)[F::D], R h,
+                                            const typename F::template Theta<R>& th,
+                                            R (&J)[F::D * F::D], SmallLU<R, F::D>& lu) {
+  constexpr int D = F::D;
+  F::jac(y, th, J);
+  const R hd = h * R(Rb23::d);
+  R Mx[D][D];
+#pragma unroll
+  for (int r = 0; r < D; ++r)
+#pragma unroll
+    for (int c = 0; c < D; ++c) Mx[r][c] = (r == c ? R(1) : R(0)) - hd * J[r * D + c];
+  lu.factor(Mx);
+}
+
+// k1, F1 and k2 of the step from y (F0 = f(y) given).
+template <class F, class R>
+__device__ __forceinline__ void rb23_stages(const R (&y)[F::D], R h,
+                                            const typename F::template Theta<R>& th,
+                                            const SmallLU<R, F::D>& lu, const R (&F0)[F::D],
+                                            R (&k1)[F::D], R (&F1)[F::D], R (&k2)[F::D]) {
+  constexpr int D = F::D;
+  lu.solve(F0, k1);
+  R Y1[D], r[D];
+#pragma unroll
+  for (int c = 0; c < D; ++c) Y1[c] = y[c] + R(0.5) * h * k1[c];
+  F::f(Y1, th, F1);
+#pragma unroll
+  for (int c = 0; c < D; ++c) r[c] = F1[c] - k1[c];
+  lu.solve(r, k2);
+#pragma unroll
+  for (int c = 0; c < D; ++c) k2[c] = k2[c] + k1[c];
+}
+
+// One Rosenbrock23 trial from y with F0 = f(y) carried; returns the scaled RMS error and
+// F2 = f(y_new) (the next F0 when the step is accepted).
+template <class F, class R>
+__device__ __forceinline__ R rb23_trial(const R (&y)[F::D], R h,
+                                        const typename F::template Theta<R>& th,
+                                        const R (&F0)[F::D], R (&ynew)[F::D], R (&F2)[F::D],
+                                        R rtol, R atol) {
+  constexpr int D = F::D;
+  R J[D * D];
+  SmallLU<R, D> lu;
+  rb23_matrix<F, R>(y, h, th, J, lu);
+  R k1[D], F1[D], k2[D];
+  rb23_stages<F, R>(y, h, th, lu, F0, k1, F1, k2);
+#pragma unroll
+  for (int c = 0; c < D; ++c) ynew[c] = y[c] + h * k2[c];
+  F::f(ynew, th, F2);
+  R r[D], k3[D];
+#pragma unroll
+  for (int c = 0; c < D; ++c)
+    r[c] = F2[c] - R(Rb23::e32) * (k2[c] - F1[c]) - R(2) * (k1[c] - F0[c]);
+  lu.solve(r, k3);
+  R acc = R(0);
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    const R e = h * (k1[c] - R(2) * k2[c] + k3[c]) / R(6);
+    const R sc = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
+    const R q = e / sc;
+    acc += q * q;
+  }
+  return sqrt(acc / R(D));
+}
+
+// The Rosenbrock23 replay map y + h k2 (no error estimate).
+template <class F, class R>
+__device__ __forceinline__ void rb23_replay_step(const R (&y)[F::D], R h,
+                                                 const typename F::template Theta<R>& th,
+                                                 R (&ynew)[F::D]) {
+  constexpr int D = F::D;
+  R J[D * D];
+  SmallLU<R, D> lu;
+  rb23_matrix<F, R>(y, h, th, J, lu);
+  R F0[D], k1[D], F1[D], k2[D];
+  F::f(y, th, F0);
+  rb23_stages<F, R>(y, h, th, lu, F0, k1, F1, k2);
+#pragma unroll
+  for (int c = 0; c < D; ++c) ynew[c] = y[c] + h * k2[c];
+}
+
+// Reverse-mode step of the Rosenbrock23 replay map with h fixed.  With u = k2 - k1
+// (W u = F1 - k1) and lam the cotangent of y_{n+1}:
+//   k2b = h lam;  mu2 = W^{-T} k2b;  F1b = mu2;  k1b = k2b - mu2;  Jb = h d mu2 u^T
+//   Y1b = J_y(Y1)^T mu2 (thb += J_th(Y1)^T mu2);  yb = lam + Y1b;  k1b += h Y1b / 2
+//   mu1 = W^{-T} k1b;  Jb += h d mu1 k1^T;  yb += J_y(y)^T mu1 (thb += J_th(y)^T mu1)
+//   yb += Jb : dJ/dy,  thb += Jb : dJ/dtheta;   lam <- yb.
+template <class F, class R>
+__device__ __forceinline__ void rb23_adjoint_step(const R (&y)[F::D], R h,
+                                                  const typename F::template Theta<R>& th,
+                                                  R (&lam)[F::D], R (&thb)[F::M]) {
+  constexpr int D = F::D;
+  R J[D * D];
+  SmallLU<R, D> lu;
+  rb23_matrix<F, R>(y, h, th, J, lu);
+  R F0[D], k1[D], F1[D], k2[D];
+  F::f(y, th, F0);
+  rb23_stages<F, R>(y, h, th, lu, F0, k1, F1, k2);
+  const R hd = h * R(Rb23::d);
+  R Jb[D * D], yb[D], k2b[D], mu[D], k1b[D], tmp[D];
+#pragma unroll
+  for (int c = 0; c < D; ++c) { yb[c] = lam[c]; k2b[c] = h * lam[c]; }
+  lu.solve_t(k2b, mu);                               // mu2
+#pragma unroll
+  for (int r = 0; r < D; ++r)
+#pragma unroll
+    for (int c = 0; c < D; ++c) Jb[r * D + c] = hd * mu[r] * (k2[c] - k1[c]);
+  R Y1[D];
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    k1b[c] = k2b[c] - mu[c];
+    Y1[c] = y[c] + R(0.5) * h * k1[c];
+  }
+  F::vjp(Y1, th, mu, tmp, thb);                      // Y1b
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    yb[c] += tmp[c];
+    k1b[c] += R(0.5) * h * tmp[c];
+  }
+  lu.solve_t(k1b, mu);                               // mu1
+#pragma unroll
+  for (int r = 0; r < D; ++r)
+#pragma unroll
+    for (int c = 0; c < D; ++c) Jb[r * D + c] += hd * mu[r] * k1[c];
+  F::vjp(y, th, mu, tmp, thb);
+#pragma unroll
+  for (int c = 0; c < D; ++c) yb[c] += tmp[c];
+  F::jac_vjp(y, th, Jb, yb, thb);
+#pragma unroll
+  for (int c = 0; c < D; ++c) lam[c] = yb[c];
+}
+
 // Reverse-mode step of the ROS34PW2 replay map with h fixed.  With M = I - gamma h J,
 // r_i = h f(Y_i) + h J G_i, M k_i = r_i, the backward pass for stage i = 4..1 is
 //   mu_i = M^{-T} kb_i                          (one transpose solve, same LU)

@@ -16,13 +16,14 @@ LIB_PATH = os.path.join(PKG, "libgradsolve_b200.so")
 
 GS_OK, GS_ERR_INVALID_ARG, GS_ERR_CUDA, GS_ERR_CAPACITY, GS_ERR_UNSUPPORTED, GS_ERR_TRAJ_FAILED = range(6)
 GS_F64, GS_F32 = 0, 1
-GS_TSIT5, GS_ROS34PW2, GS_VERN7 = 0, 1, 2
+GS_TSIT5, GS_ROS34PW2, GS_VERN7, GS_ROSENBROCK23 = 0, 1, 2, 3
 FIELDS = {"lotka_volterra": 0, "lorenz63": 1, "mlp": 2, "robertson": 3, "nfw_mn": 4, "linear3": 5,
-          "log_halo": 6}
+          "log_halo": 6, "hires": 7}
 # (d, m) of each field, as the library checks them
 FIELD_DIMS = {"lotka_volterra": (2, 4), "lorenz63": (3, 3), "mlp": (4, 1348), "robertson": (3, 3),
-              "nfw_mn": (6, 5), "linear3": (3, 9), "log_halo": (6, 2)}
-METHODS = {"tsit5": GS_TSIT5, "ros34pw2": GS_ROS34PW2, "vern7": GS_VERN7}
+              "nfw_mn": (6, 5), "linear3": (3, 9), "log_halo": (6, 2), "hires": (8, 12)}
+METHODS = {"tsit5": GS_TSIT5, "ros34pw2": GS_ROS34PW2, "vern7": GS_VERN7,
+           "rosenbrock23": GS_ROSENBROCK23}
 STATUS_NAMES = {0: "GS_OK", 1: "GS_ERR_INVALID_ARG", 2: "GS_ERR_CUDA", 3: "GS_ERR_CAPACITY",
                 4: "GS_ERR_UNSUPPORTED", 5: "GS_ERR_TRAJ_FAILED"}
 
@@ -110,7 +111,7 @@ def _check(code, allow=()):
 def system(field, method=None, dtype="f64", theta_shared=False):
     d, m = FIELD_DIMS[field]
     if method is None:
-        method = "ros34pw2" if field == "robertson" else "tsit5"
+        method = "ros34pw2" if field in ("robertson", "hires") else "tsit5"
     return GsSystem(FIELDS[field], METHODS[method], GS_F64 if dtype in ("f64", "float64") else GS_F32,
                     d, m, int(bool(theta_shared)))
 

@@ -248,11 +248,13 @@ def by_name(name: str, N: Optional[int] = None, **kw) -> Workload:
              "robertson": robertson, "nfw_mn": nfw_mn, "log_halo": log_halo, "hires": hires}
     if name == "nfw_mn_f32":
         return nfw_mn(N=N if N else 1 << 20, dtype=np.float32, **kw)
-    if name.endswith("_vern7"):
-        # the same ensemble integrated with the Verner 7(6) pair instead of Tsit5
-        w = by_name(name[:-len("_vern7")], N=N, **kw)
-        w.name, w.method = name, "vern7"
-        return w
+    for suffix, method in (("_vern7", "vern7"), ("_rb23", "rosenbrock23"),
+                           ("_ros34pw2", "ros34pw2")):
+        if name.endswith(suffix):
+            # the same ensemble integrated with another method of the same kind
+            w = by_name(name[:-len(suffix)], N=N, **kw)
+            w.name, w.method = name, method
+            return w
     fn = table[name]
     return fn(N=N, **kw) if N else fn(**kw)
 

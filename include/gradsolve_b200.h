@@ -50,8 +50,10 @@ typedef enum { GS_F64 = 0, GS_F32 = 1 } gs_dtype;
 /* GS_TSIT5: Tsitouras 5(4), 7 stages, first-same-as-last ([GS] §2.1, the default explicit pair).
  * GS_ROS34PW2: Rang & Angermann's 4-stage Rosenbrock-Wanner method, order 3(2), for stiff fields.
  * GS_VERN7: Verner's 7(6) pair, 10 stages, for tight tolerances ([GS] §3.1: the seventh-order
- * Verner pair offered next to Tsit5); every explicit field except GS_MLP_4_32_32_4. */
-typedef enum { GS_TSIT5 = 0, GS_ROS34PW2 = 1, GS_VERN7 = 2 } gs_method;
+ * Verner pair offered next to Tsit5); every explicit field except GS_MLP_4_32_32_4.
+ * GS_ROSENBROCK23: Shampine & Reichelt's linearly implicit order-2(3) pair ([GS] §3.1: the
+ * second-order Rosenbrock23 method of the fused stiff kernels), for the stiff fields. */
+typedef enum { GS_TSIT5 = 0, GS_ROS34PW2 = 1, GS_VERN7 = 2, GS_ROSENBROCK23 = 3 } gs_method;
 
 /* Built-in fields (all autonomous).  d = state size, m = parameters per trajectory.
  *   GS_LOTKA_VOLTERRA  d=2 m=4     theta = (alpha, beta, gamma, delta)
@@ -64,6 +66,9 @@ typedef enum { GS_TSIT5 = 0, GS_ROS34PW2 = 1, GS_VERN7 = 2 } gs_method;
  *   GS_LOG_HALO        d=6 m=2     test particle in the flattened logarithmic halo
  *                                  Phi = v_c^2/2 ln(R_c^2 + x^2 + y^2 + z^2/q^2), R_c = 0.2,
  *                                  theta = (v_c, q)                     ([DA] §3)
+ *   GS_HIRES           d=8 m=12    stiff HIRES kinetics, theta = the 12 rate constants
+ *                                  (1.71, 0.43, 8.32, 7e-4, 8.75, 10.03, 0.035, 1.12, 1.745,
+ *                                  280, 0.69, 1.81 nominal)             ([GS] §4.5-4.6)
  * [DA] = "Differentiable astrophysics at scale: solving and differentiating ODE ensembles on the
  * GPU". */
 typedef enum {
@@ -73,13 +78,14 @@ typedef enum {
   GS_ROBERTSON = 3,
   GS_NFW_MN = 4,
   GS_LINEAR = 5,
-  GS_LOG_HALO = 6
+  GS_LOG_HALO = 6,
+  GS_HIRES = 7
 } gs_field;
 
 typedef struct {
   int32_t field;        /* gs_field */
-  int32_t method;       /* gs_method: GS_TSIT5 or GS_VERN7 for non-stiff fields, GS_ROS34PW2
-                           for stiff ones */
+  int32_t method;       /* gs_method: GS_TSIT5 or GS_VERN7 for non-stiff fields, GS_ROS34PW2 or
+                           GS_ROSENBROCK23 for stiff ones */
   int32_t dtype;        /* gs_dtype */
   int32_t d, m;         /* must equal the field's sizes (checked) */
   int32_t theta_shared; /* 1: theta is [m] shared by all trajectories; 0: [N][m] */
