@@ -45,6 +45,31 @@ FLOPS_SENS_STEP = {"log_halo": 912}
 # 9 c_v (stages 2..9 recomputed, nine pullbacks).  c_f, c_v as for Tsit5.
 FLOPS_VERN7_ATTEMPT = {"lorenz63": 436, "nfw_mn": 1047}
 FLOPS_VERN7_ADJOINT = {"lorenz63": 724, "nfw_mn": 2015}
+# Stiff fields: (d, c_f, c_v, c_J, c_Jv) -- f, its pullback, the Jacobian and the contraction of a
+# Jacobian cotangent with dJ/d(y, theta), counted like c_f and c_v.
+STIFF_COUNTS = {"robertson": (3, 8, 20, 9, 22), "hires": (8, 38, 77, 3, 32)}
+
+
+def lu_ops(d):
+    """Dense LU without the pivot search: per column one reciprocal, k multipliers and 2 k^2 for
+    the update of the k x k trailing block."""
+    return sum(1 + k + 2 * k * k for k in range(d))
+
+
+def stiff_flops(method, field):
+    """Operations per attempted step and per accepted step of the replay adjoint, counted from the
+    step's definition (one solve = 2 d^2 - d):
+      ROS34PW2 attempt  c_J + 4 c_f + 17 d^2 + 53 d + LU(d) + 6
+      ROS34PW2 adjoint  c_J + c_Jv + 4 c_f + 4 c_v + 51 d^2 + 92 d + LU(d) + 1
+      Rosenbrock23 attempt  c_J + 2 c_f + 7 d^2 + 20 d + LU(d) + 7
+      Rosenbrock23 adjoint  c_J + c_Jv + 2 c_f + 2 c_v + 12 d^2 + 12 d + LU(d) + 3"""
+    d, cf, cv, cj, cjv = STIFF_COUNTS[field]
+    lu = lu_ops(d)
+    if method == "ros34pw2":
+        return (cj + 4 * cf + 17 * d * d + 53 * d + lu + 6,
+                cj + cjv + 4 * cf + 4 * cv + 51 * d * d + 92 * d + lu + 1)
+    return (cj + 2 * cf + 7 * d * d + 20 * d + lu + 7,
+            cj + cjv + 2 * cf + 2 * cv + 12 * d * d + 12 * d + lu + 3)
 # The MLP field (4-32-32-4, tanh) counted by hand: f = 1,280 multiply-adds + 68 bias adds + 64
 # tanh = 2,692 ops; its pullback = the two transposed products (2 x 1,280 flops), the weight
 # outer products (2 x 1,280), 2 x 64 for tanh' and 68 bias cotangents = 5,316 ops; per accepted
@@ -255,9 +280,12 @@ WORKLOADS = {
                      adj=FLOPS_ADJOINT_STEP["lorenz63"]),
     "lotka_volterra": dict(dtype="f64", fwd=FLOPS_FORWARD_ATTEMPT["lotka_volterra"],
                            adj=FLOPS_ADJOINT_STEP["lotka_volterra"]),
-    "robertson": dict(dtype="f64", fwd=None, adj=None),
-    "robertson_rb23": dict(dtype="f64", fwd=None, adj=None),
-    "hires": dict(dtype="f64", fwd=None, adj=None),
+    "robertson": dict(dtype="f64", fwd=stiff_flops("ros34pw2", "robertson")[0],
+                      adj=stiff_flops("ros34pw2", "robertson")[1]),
+    "robertson_rb23": dict(dtype="f64", fwd=stiff_flops("rosenbrock23", "robertson")[0],
+                           adj=stiff_flops("rosenbrock23", "robertson")[1]),
+    "hires": dict(dtype="f64", fwd=stiff_flops("rosenbrock23", "hires")[0],
+                  adj=stiff_flops("rosenbrock23", "hires")[1]),
     "mlp": dict(dtype="f32", fwd=FLOPS_FORWARD_ATTEMPT["mlp"], adj=FLOPS_ADJOINT_STEP["mlp"]),
     "lorenz63_vern7": dict(dtype="f64", fwd=FLOPS_VERN7_ATTEMPT["lorenz63"],
                            adj=FLOPS_VERN7_ADJOINT["lorenz63"]),

@@ -33,6 +33,10 @@ template <class F, class = void> struct has_pullback : std::false_type {};
 template <class F>
 struct has_pullback<F, std::void_t<decltype(F::TAPE)>> : std::true_type {};
 
+template <class F, class = void> struct has_jac : std::false_type {};
+template <class F>
+struct has_jac<F, std::void_t<decltype(&F::template jac<double>)>> : std::true_type {};
+
 template <class F>
 void run(const char* name, const double* theta, const double* y) {
   Cnt th_src[F::M], yy[F::D], dy[F::D], kb[F::D], yb[F::D], thb[F::M];
@@ -66,7 +70,23 @@ void run(const char* name, const double* theta, const double* y) {
   T = Tally();
   F::f(dy_, thd, ddy);
   Tally td = T;
-  std::printf("{\"field\": \"%s\", \"D\": %d, \"M\": %d, "
+  // Jacobian and the contraction of a Jacobian cotangent with its derivatives (stiff fields)
+  Tally tj, tjv;
+  if constexpr (has_jac<F>::value) {
+    Cnt J[F::D * F::D], Jb[F::D * F::D], yb2[F::D], thb2[F::M];
+    for (int i = 0; i < F::D * F::D; ++i) Jb[i] = Cnt(0.01 * (i + 1));
+    for (int c = 0; c < F::D; ++c) yb2[c] = Cnt(0);
+    for (int j = 0; j < F::M; ++j) thb2[j] = Cnt(0);
+    T = Tally();
+    F::jac(yy, th, J);
+    tj = T;
+    T = Tally();
+    F::jac_vjp(yy, th, Jb, yb2, thb2);
+    tjv = T;
+  }
+  std::printf("{\"jac\": %ld, \"jac_vjp\": %ld, ", tj.add + tj.mul + tj.div + tj.sqrt + tj.log1p,
+              tjv.add + tjv.mul + tjv.div + tjv.sqrt + tjv.log1p);
+  std::printf("\"field\": \"%s\", \"D\": %d, \"M\": %d, "
               "\"f\": {\"add\": %ld, \"mul\": %ld, \"div\": %ld, \"sqrt\": %ld, \"log1p\": %ld}, "
               "\"vjp\": {\"add\": %ld, \"mul\": %ld, \"div\": %ld, \"sqrt\": %ld, \"log1p\": %ld}, "
               "\"fdual\": {\"add\": %ld, \"mul\": %ld, \"div\": %ld, \"sqrt\": %ld, \"log1p\": %ld}}\n",
@@ -85,5 +105,9 @@ int main() {
   run<gs::FRobertson>("robertson", rob_th, rob_y);
   const double lh_th[2] = {1.0, 0.7}, lh_y[6] = {0.7, 0.2, 0.4, 0.1, 0.5, 0.05};
   run<gs::FLogHalo>("log_halo", lh_th, lh_y);
+  const double hi_th[12] = {1.71, 0.43, 8.32, 0.0007, 8.75, 10.03, 0.035, 1.12, 1.745, 280, 0.69,
+                            1.81};
+  const double hi_y[8] = {0.7, 0.01, 0.02, 0.03, 0.04, 0.05, 0.06, 0.007};
+  run<gs::FHires>("hires", hi_th, hi_y);
   return 0;
 }

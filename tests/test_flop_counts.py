@@ -75,6 +75,20 @@ def test_vern7_constants_match_counts(counts, orc):
         assert bench.FLOPS_VERN7_ADJOINT[field] == 160 * D + 8 * ops(c["f"]) + 9 * ops(c["vjp"])
 
 
+def test_stiff_counts_and_formulas(counts):
+    import bench
+    for field in ("robertson", "hires"):
+        c = counts[field]
+        assert bench.STIFF_COUNTS[field] == (c["D"], ops(c["f"]), ops(c["vjp"]), c["jac"],
+                                             c["jac_vjp"])
+    # the 3 x 3 elimination: column 0: 1 reciprocal + 2 multipliers + 2 x 2 x 2; column 1:
+    # 1 + 1 + 2; column 2: 1
+    assert bench.lu_ops(3) == 16
+    assert bench.stiff_flops("ros34pw2", "robertson") == (375, 895)
+    assert bench.stiff_flops("rosenbrock23", "robertson") == (171, 250)
+    assert bench.stiff_flops("rosenbrock23", "hires") == (1010, 1448)
+
+
 def test_mlp_hand_count():
     import bench
     H, D = 32, 4
