@@ -337,6 +337,10 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
         } else {
           err = ros_trial<F, R>(y, h, th, ynew, p.rtol, p.atol);
         }
+        // the controller's factor 0.9 err^(-1/q), formed once for both outcomes: when a warp holds
+        // accepted and rejected lanes together (nearly always) it would otherwise run the power
+        // function on both paths
+        const R fpow = R(0.9) * pw<R>(err, expo);
         if (err <= R(1)) {
           if (REC) {
             R* e = mystage + ns * L::E;
@@ -366,7 +370,7 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
           }
           ++S;
           const R facmax = last_rej ? R(1) : R(10);
-          R fac = (err == R(0)) ? facmax : R(0.9) * pw<R>(err, expo);
+          R fac = (err == R(0)) ? facmax : fpow;
           fac = fmin(facmax, fmax(R(0.2), fac));
           t = (clipped || t + h >= p.t1) ? p.t1 : t + h;
 #pragma unroll
@@ -377,7 +381,7 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
           if (t == p.t1) st = 0;
         } else {
           ++Rj;
-          R fac = isfinite(err) ? R(0.9) * pw<R>(err, expo) : R(0.2);
+          R fac = isfinite(err) ? fpow : R(0.2);
           fac = fmin(R(10), fmax(R(0.2), fac));
           h = h * fac;
           last_rej = true;
