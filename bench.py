@@ -81,7 +81,16 @@ SMS, FP64_LANES, FP32_LANES = 148, 64, 128
 # 2^18-trajectory case of this workload; both kernels move a fixed number of bytes per accepted
 # step, so a launch's traffic is this times its accepted steps.  Record kernel: 64 B of record
 # per step written plus inputs; adjoint: the 64 B entry read per step plus chunk table and inputs.
-TRAFFIC_PER_STEP = {"record": 66.52, "adjoint": 70.77}
+TRAFFIC_PER_STEP = {
+    "nfw_mn": {"record": 66.52, "adjoint": 70.77},
+    "robertson": {"record": 38.9, "adjoint": 46.2},
+    "robertson_rb23": {"record": 39.8, "adjoint": 47.2},
+    "hires": {"record": 373.4, "adjoint": 99.1},          # record: spill traffic (d = 8 LU)
+    "lorenz63_vern7": {"adjoint": 46.4},                   # its record pass stays partly in L2
+}
+# forward sensitivities: DRAM bytes per trajectory (inputs and outputs; nothing per step), from
+# the ncu capture of the 2^18-orbit case
+TRAFFIC_SENS_PER_TRAJ = {"log_halo": 49.5}
 # library kernels per step: record = k_solve + 2 k_max_int + 3 prefix scans of 3 kernels each
 # (step offsets, chunk offsets, length bins) + k_chunk_table + k_bin_count + k_bin_scatter (15);
 # replay gradient = k_adjoint (1).
@@ -416,7 +425,8 @@ def run_sens(args, w, wl, G, torch, dev, stream, ws, rank):
     achieved = flops / (kernel_ms / 1e3) / 1e12
     roofline = {"kernel": "k_solve<log_halo, double, Tsit5, sens>", "bound": "alu",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": None,
+                "traffic": TRAFFIC_SENS_PER_TRAJ[args.workload] * N,
+                "traffic_source": "ncu dram bytes per trajectory on the 2^18 case x trajectories",
                 "peak_source": "derived: 148 SM x 64 FP64 FMA lanes/clk x 2 x 1965 MHz (FP64 pipe)",
                 "flops_per_unit": {"attempted step": wl["fwd"], "accepted step (sensitivities)":
                                    wl["sens"]},
@@ -651,7 +661,7 @@ def main():
         return {"kernel": name, "bound": "alu", "achieved": achieved, "peak": peak_max,
                 "unit": "TFLOP/s", "frac": achieved / peak_max if achieved else None,
                 "traffic": traffic,
-                "traffic_source": "ncu dram bytes per accepted step on the 2^18 case x steps",
+                "traffic_source": "ncu dram bytes per accepted step of one capture x steps",
                 "peak_source": "derived: 148 SM x %d %s FMA lanes/clk x 2 x 1965 MHz (%s pipe)"
                                % (lanes, pipe, pipe),
                 "flops_per_unit": per_unit, "unit_counted": unit_name, "kernel_ms": ms,
@@ -660,7 +670,7 @@ def main():
     method = {"tsit5": "Tsit5", "vern7": "Vern7", "ros34pw2": "ROS34PW2",
               "rosenbrock23": "Rosenbrock23"}[w.method]
     rec_kernel_ms = statistics.median(solve_ms)
-    traffic = TRAFFIC_PER_STEP if args.workload == "nfw_mn" else {}
+    traffic = TRAFFIC_PER_STEP.get(args.workload, {})
     roof_rec = roof("k_solve<%s, %s, %s, record>" % (w.field, "double" if f64 else "float", method),
                     wl["fwd"], attempts, rec_kernel_ms, "attempted step",
                     traffic.get("record", 0) * total_steps or None)

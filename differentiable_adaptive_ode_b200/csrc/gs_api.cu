@@ -184,6 +184,7 @@ struct gs_record {
   // visiting order of the replay kernels (longest records first) and its counting-sort scratch
   int* perm = nullptr;
   int64_t perm_cap = 0;
+  int64_t perm_n = 0;   // ensemble size the current perm was built for (0: none)
   int* bins = nullptr;          // [nb] counts, then [nb] cursors
   long long* binoff = nullptr;  // [nb + 1]
   long long* btiles = nullptr;
@@ -285,6 +286,7 @@ gs_status build_perm(gs_record* r, cudaStream_t s) {
   gs::k_bin_scatter<<<grid, 256, 0, s>>>(r->nsteps, (int)N, r->max_steps, r->binoff,
                                          r->bins + nb, r->perm);
   GS_CUDA(cudaGetLastError());
+  r->perm_n = N;
   return GS_OK;
 }
 
@@ -307,6 +309,7 @@ struct SolveCall {
   cudaStream_t stream;
   const void* sens0 = nullptr;  // forward sensitivities (Tsit5 forward solve only)
   void* sens1 = nullptr;
+  const int* order = nullptr;   // visiting order of the trajectories (null: index order)
 };
 
 template <class F, class R, int METHOD>
@@ -323,6 +326,7 @@ gs_status launch_solve(const SolveCall& c) {
   p.nrejected = c.nrejected;
   p.status = c.status;
   p.queue = c.queue;
+  p.order = c.order;
   if constexpr (std::is_same_v<F, gs::FMlpWarp>) {
     if (c.rec) {
       p.pool = static_cast<R*>(c.rec->pool);
@@ -646,6 +650,7 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
     r->pool = nullptr; r->chunk_traj = r->chunk_seq = r->chunk_table = nullptr;
     r->pool_chunks = r->chunk_arrays_cap = 0;
   }
+  const bool order_ok = !fresh && r->perm && r->perm_n == N;
   r->sys = *sys;
   r->N = N;
   r->C = C;
@@ -675,6 +680,10 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
       return bail(fail(GS_ERR_CUDA, "cudaMemsetAsync failed"));
     SolveCall c{N, theta, sys->theta_shared, y0, t0, t1, rtol, atol, attempts_of(opt), y1,
                 r->nsteps, nullptr, status_out, r->counters, r, s};
+    // a record that is made again for an ensemble of the same size starts its trajectories in the
+    // previous solve's longest-first order: long trajectories begin early instead of forming the
+    // tail of the launch.  Scheduling only -- every trajectory's result is independent of it.
+    if (order_ok) c.order = r->perm;
     cudaEventRecord(r->ev0, s);
     st = dispatch(*sys, [&]<class F, class R, int METHOD>() { return launch_solve<F, R, METHOD>(c); });
     if (st != GS_OK) return bail(st);

@@ -47,6 +47,7 @@ struct SolveParams {
   int* nrejected;
   int* status;
   int* queue;        // work counter
+  const int* order;  // trajectory visited at queue position q (null: q itself)
   // record (REC only)
   R* pool;
   int* chunk_traj;
@@ -231,8 +232,9 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
         if (lane == 0) base = atomicAdd(p.queue, 32);
         base = __shfl_sync(FULL, base, 0);
         if (base + 32 >= p.N) exhausted = true;
-        const int id = base + lane;
-        const bool valid = id < p.N;
+        const int q = base + lane;
+        const bool valid = q < p.N;
+        const int id = (valid && p.order) ? p.order[q] : q;
         int st = -1;
         R h0 = R(0), f0[D];
 #pragma unroll

@@ -154,7 +154,9 @@ gs_status gs_solve_forward_sens(const gs_system* sys, const gs_options* opt, int
  * *rec: if NULL on entry a new record is created; otherwise its storage is reused (grown when
  * needed) and its contents replaced.  y1 [N][d] (device, required), status [N] (nullable).
  * Synchronises the stream once to size the record; if the pool was too small the solve is run
- * again with exactly the needed size.  Returns GS_ERR_TRAJ_FAILED (with the record complete)
+ * again with exactly the needed size.  A record made again for an ensemble of the same size
+ * starts its trajectories in the previous solve's longest-first order (scheduling only: results
+ * do not depend on the order).  Returns GS_ERR_TRAJ_FAILED (with the record complete)
  * when some trajectory status != 0. */
 gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N,
                           const void* theta, const void* y0, double t0, double t1, double rtol,
