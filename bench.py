@@ -82,7 +82,7 @@ SMS, FP64_LANES, FP32_LANES = 148, 64, 128
 # step, so a launch's traffic is this times its accepted steps.  Record kernel: 64 B of record
 # per step written plus inputs; adjoint: the 64 B entry read per step plus chunk table and inputs.
 TRAFFIC_PER_STEP = {
-    "nfw_mn": {"record": 66.52, "adjoint": 70.77},
+    "nfw_mn": {"record": 68.3, "adjoint": 70.77},
     "robertson": {"record": 38.9, "adjoint": 46.2},
     "robertson_rb23": {"record": 39.8, "adjoint": 47.2},
     "hires": {"record": 373.4, "adjoint": 99.1},          # record: spill traffic (d = 8 LU)
@@ -90,7 +90,7 @@ TRAFFIC_PER_STEP = {
 }
 # forward sensitivities: DRAM bytes per trajectory (inputs and outputs; nothing per step), from
 # the ncu capture of the 2^18-orbit case
-TRAFFIC_SENS_PER_TRAJ = {"log_halo": 49.5}
+TRAFFIC_SENS_PER_TRAJ = {"log_halo": 50.8}
 # library kernels per step: record = k_solve + 2 k_max_int + 3 prefix scans of 3 kernels each
 # (step offsets, chunk offsets, length bins) + k_chunk_table + k_bin_count + k_bin_scatter (15);
 # replay gradient = k_adjoint (1).
@@ -323,10 +323,15 @@ def run_sens(args, w, wl, G, torch, dev, stream, ws, rank):
     rj = torch.empty(N, dtype=torch.int32, device=dev)
     st = torch.empty(N, dtype=torch.int32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    # the caller's start order: orbits by decreasing attempts of the previous solve (scheduling
+    # only), formed on the device after every step
+    order = torch.arange(N, dtype=torch.int32, device=dev)
+    opts = G.options(start_order=order)
 
     def step():
         G.gs_solve_forward_sens(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, S1, None, S, rj,
-                                st)
+                                st, opts=opts)
+        order.copy_(torch.argsort(S + rj, descending=True))
 
     for _ in range(args.warmup):
         flush.zero_()

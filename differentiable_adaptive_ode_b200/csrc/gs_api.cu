@@ -590,6 +590,7 @@ gs_status gs_solve_forward(const gs_system* sys, const gs_options* opt, int64_t 
   GS_CUDA(take_counter(s, &queue));
   SolveCall c{N, theta, sys->theta_shared, y0, t0, t1, rtol, atol, attempts_of(opt), y1,
               nsteps, nrejected, status, queue, nullptr, s};
+  c.order = opt ? opt->start_order : nullptr;
   return dispatch(*sys, [&]<class F, class R, int METHOD>() { return launch_solve<F, R, METHOD>(c); });
 }
 
@@ -610,6 +611,7 @@ gs_status gs_solve_forward_sens(const gs_system* sys, const gs_options* opt, int
   GS_CUDA(take_counter(s, &queue));
   SolveCall c{N, theta, sys->theta_shared, y0, t0, t1, rtol, atol, attempts_of(opt), y1,
               nsteps, nrejected, status, queue, nullptr, s, S0, S1};
+  c.order = opt ? opt->start_order : nullptr;
   return dispatch(*sys, [&]<class F, class R, int METHOD>() { return launch_solve<F, R, METHOD>(c); });
 }
 
@@ -683,7 +685,8 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
     // a record that is made again for an ensemble of the same size starts its trajectories in the
     // previous solve's longest-first order: long trajectories begin early instead of forming the
     // tail of the launch.  Scheduling only -- every trajectory's result is independent of it.
-    if (order_ok) c.order = r->perm;
+    if (opt && opt->start_order) c.order = opt->start_order;
+    else if (order_ok) c.order = r->perm;
     cudaEventRecord(r->ev0, s);
     st = dispatch(*sys, [&]<class F, class R, int METHOD>() { return launch_solve<F, R, METHOD>(c); });
     if (st != GS_OK) return bail(st);

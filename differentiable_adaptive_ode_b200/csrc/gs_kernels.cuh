@@ -233,8 +233,12 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
         base = __shfl_sync(FULL, base, 0);
         if (base + 32 >= p.N) exhausted = true;
         const int q = base + lane;
-        const bool valid = q < p.N;
-        const int id = (valid && p.order) ? p.order[q] : q;
+        int id = q;
+        bool valid = q < p.N;
+        if (valid && p.order) {
+          id = p.order[q];
+          valid = id >= 0 && id < p.N;   // a caller's order entry outside the ensemble is skipped
+        }
         int st = -1;
         R h0 = R(0), f0[D];
 #pragma unroll

@@ -40,7 +40,8 @@ class GsSystem(C.Structure):
 
 
 class GsOptions(C.Structure):
-    _fields_ = [("max_attempts", C.c_int64), ("record_capacity_steps", C.c_int64)]
+    _fields_ = [("max_attempts", C.c_int64), ("record_capacity_steps", C.c_int64),
+                ("start_order", C.c_void_p)]
 
 
 class GsRecordInfo(C.Structure):
@@ -116,8 +117,11 @@ def system(field, method=None, dtype="f64", theta_shared=False):
                     d, m, int(bool(theta_shared)))
 
 
-def options(max_attempts=0, record_capacity_steps=0):
-    return GsOptions(max_attempts, record_capacity_steps)
+def options(max_attempts=0, record_capacity_steps=0, start_order=None):
+    """start_order: optional int32 device tensor [N], the order in which trajectories are started
+    (scheduling only).  The tensor must stay alive while the call's work runs."""
+    return GsOptions(max_attempts, record_capacity_steps,
+                     None if start_order is None else start_order.data_ptr())
 
 
 def _ptr(t):

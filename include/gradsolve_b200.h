@@ -94,6 +94,13 @@ typedef struct {
 typedef struct {
   int64_t max_attempts;          /* per trajectory; <= 0 means the default 100000 */
   int64_t record_capacity_steps; /* initial record pool size in steps; 0 = automatic */
+  const int32_t* start_order;    /* device [N] or NULL: trajectory started at queue position q
+                                    is start_order[q].  Scheduling only (results do not depend
+                                    on it): a permutation that starts long trajectories first
+                                    shortens the tail of a launch.  Entries outside [0, N) are
+                                    skipped; a non-permutation leaves some outputs unwritten.
+                                    gs_solve_record falls back to the previous record's
+                                    longest-first order when NULL (see there). */
 } gs_options;
 
 typedef struct gs_record gs_record; /* opaque, library-owned, device resident */

@@ -128,3 +128,26 @@ def test_sens_edges_and_argument_checks():
                                 U.dev(rob.y0, torch.float64), 0.0, 1.0, 1e-6, 1e-6, out,
                                 torch.empty((4, 3, 3), dtype=torch.float64, device="cuda"))
     assert e.value.code == G.GS_ERR_UNSUPPORTED
+
+
+def test_start_order_changes_nothing_but_the_schedule():
+    import torch
+    w = U.small("log_halo", 2000)
+    base = U.forward_sens(w)
+    dt = torch.float64
+    th, y0 = U.dev(w.theta, dt), U.dev(w.y0, dt)
+    for order in (np.arange(w.N)[::-1], np.random.default_rng(4).permutation(w.N)):
+        o = torch.as_tensor(order.astype(np.int32), device="cuda")
+        y1 = torch.empty((w.N, w.d), dtype=dt, device="cuda")
+        S1 = torch.empty((w.N, w.d, w.m), dtype=dt, device="cuda")
+        S = torch.empty(w.N, dtype=torch.int32, device="cuda")
+        G.gs_solve_forward_sens(U.gsys(w), w.N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, S1, None,
+                                S, opts=G.options(start_order=o))
+        y1f = torch.empty_like(y1)
+        G.gs_solve_forward(U.gsys(w), w.N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1f,
+                           opts=G.options(start_order=o))
+        torch.cuda.synchronize()
+        assert np.array_equal(y1.cpu().numpy(), base["y1"])
+        assert np.array_equal(y1f.cpu().numpy(), base["y1"])
+        assert np.array_equal(S1.cpu().numpy(), base["sens"])
+        assert np.array_equal(S.cpu().numpy(), base["S"])
