@@ -1007,6 +1007,7 @@ gs_status gs_record_info(const gs_record* rec, gs_record_info_t* out) {
   out->chunk_table = rec->chunk_table;
   out->pool = rec->pool;
   out->solve_ms = rec->solve_ms;
+  out->order = rec->perm_n == rec->N ? rec->perm : nullptr;
   return GS_OK;
 }
 

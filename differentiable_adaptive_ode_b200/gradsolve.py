@@ -49,7 +49,8 @@ class GsRecordInfo(C.Structure):
                 ("chunk_steps", C.c_int32), ("entry_reals", C.c_int32), ("dtype", C.c_int32),
                 ("nchunks", C.c_int64), ("pool_bytes", C.c_int64), ("nsteps", C.c_void_p),
                 ("status", C.c_void_p), ("offsets", C.c_void_p), ("chunk_offsets", C.c_void_p),
-                ("chunk_table", C.c_void_p), ("pool", C.c_void_p), ("solve_ms", C.c_double)]
+                ("chunk_table", C.c_void_p), ("pool", C.c_void_p), ("solve_ms", C.c_double),
+                ("order", C.c_void_p)]
 
 
 class GradsolveError(RuntimeError):

@@ -126,6 +126,9 @@ typedef struct {
                                    pool + (c*C + slot)*E reals, entry = (t, h, y[0..d-1]) */
   double solve_ms;              /* device time of the solve kernel(s) of the last
                                    gs_solve_record (CUDA events around the launch), 0 if none */
+  const int32_t* order;          /* [N] trajectories by decreasing accepted-step count (the
+                                   replay's visiting order); usable as gs_options.start_order
+                                   for later solves of the same ensemble */
 } gs_record_info_t;
 
 /* Forward-only solve ([GS] §4.1: one thread per trajectory, final state only).

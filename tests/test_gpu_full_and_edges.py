@@ -201,3 +201,21 @@ def test_rerecord_in_previous_order_is_bitwise_identical():
     for key in ("S", "T", "H", "Y", "offsets"):
         assert np.array_equal(ex1[key], ex2[key]), key
     assert np.array_equal(g1[0], g2[0]) and np.array_equal(g1[1], g2[1])
+
+
+def test_record_info_order_is_longest_first_permutation():
+    import torch
+
+    class _Dev:  # a view of a library-owned device array through the CUDA array interface
+        def __init__(self, ptr, n):
+            self.__cuda_array_interface__ = {"shape": (n,), "typestr": "<i4",
+                                             "data": (ptr, True), "version": 3}
+
+    w = W.lorenz63(N=777)
+    rec, _ = U.record(w)
+    info = rec.info()
+    ex = U.export_padded(w, rec)
+    assert info.order
+    o = torch.as_tensor(_Dev(info.order, w.N), device="cuda").cpu().numpy()
+    assert np.array_equal(np.sort(o), np.arange(w.N))
+    assert np.all(np.diff(ex["S"][o]) <= 0)
