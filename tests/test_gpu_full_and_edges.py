@@ -209,7 +209,7 @@ def test_record_info_order_is_longest_first_permutation():
     class _Dev:  # a view of a library-owned device array through the CUDA array interface
         def __init__(self, ptr, n):
             self.__cuda_array_interface__ = {"shape": (n,), "typestr": "<i4",
-                                             "data": (ptr, True), "version": 3}
+                                             "data": (ptr, False), "version": 3}
 
     w = W.lorenz63(N=777)
     rec, _ = U.record(w)
