@@ -1,6 +1,8 @@
-"""Builds the CUDA library libgradsolve_b200.so in-tree for sm_100a with nvcc.
+"""Builds the CUDA library libgradsolve_b200.so in-tree for sm_100a with nvcc, and its checked
+variant libgradsolve_b200_checked.so (-DGS_CHECKED: accesses through a record's chunk table are
+bounds-checked, counted and redirected; see gs_checked_violations).
 
-    python -m differentiable_adaptive_ode_b200.build [--force]
+    python -m differentiable_adaptive_ode_b200.build [--force] [--checked] [-v]
 """
 import os
 import subprocess
@@ -11,6 +13,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libgradsolve_b200.so")
+CHECKED_LIB = os.path.join(PKG, "libgradsolve_b200_checked.so")
 SOURCES = ["gs_api.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -28,19 +31,23 @@ def nvcc():
     return "nvcc"
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and os.path.exists(LIB):
-        if os.path.getmtime(LIB) >= max(os.path.getmtime(p) for p in _deps()):
-            return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    lib = CHECKED_LIB if checked else LIB
+    if not force and os.path.exists(lib):
+        if os.path.getmtime(lib) >= max(os.path.getmtime(p) for p in _deps()):
+            return lib
+    tmp = lib + ".tmp%d" % os.getpid()
     cmd = [nvcc(), "-std=c++20", "-O3", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
            "-I" + INCLUDE, "-o", tmp] + [os.path.join(CSRC, s) for s in SOURCES]
+    if checked:
+        cmd.insert(1, "-DGS_CHECKED")
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                checked="--checked" in sys.argv))

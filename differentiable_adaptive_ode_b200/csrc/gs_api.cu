@@ -246,6 +246,11 @@ gs_status ensure_pool(gs_record* r, int64_t chunks) {
 }
 
 // exclusive scan of nsteps (MODE 0) or chunk counts (MODE 1) into out[0..N]
+// Allocated sizes of a record's pool and chunk table (bounds of the checked build).
+gs::RecBounds bounds_of(const gs_record* r) {
+  return gs::RecBounds{(long long)r->chunk_arrays_cap, (long long)r->pool_chunks};
+}
+
 template <int MODE>
 gs_status scan_counts(const int* S, int N, int C, long long* out, long long* tiles,
                       cudaStream_t st) {
@@ -417,6 +422,7 @@ gs_status launch_adjoint(const AdjCall& c) {
   p.pool = static_cast<const R*>(r->pool);
   p.queue = c.queue;
   p.perm = r->perm;
+  p.bounds = bounds_of(r);
   auto kern = gs::k_adjoint<F, R, METHOD>;
   const size_t smem = adjoint_smem<F, R>();
   if (smem > 48 * 1024)
@@ -562,6 +568,7 @@ static gs_status replay_grad_mlp(const gs_record* rec, const void* theta, const 
     p.chunk_table = rec->chunk_table;
     p.pool = static_cast<const R*>(rec->pool);
     p.perm = rec->perm;
+    p.bounds = bounds_of(rec);
     kern<<<grid, BLOCK, 0, s>>>(p);
     if (partials)
       gs::k_reduce_partials<R><<<(gs::MLP_M + 255) / 256, 256, 0, s>>>(partials, nwarps, gs::MLP_M,
@@ -729,7 +736,7 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
   if ((st = scan_counts<1>(r->nsteps, (int)N, C, r->choff, r->tiles, s)) != GS_OK) return bail(st);
   if (r->nchunks > 0)
     gs::k_chunk_table<<<(int)((r->nchunks + 255) / 256), 256, 0, s>>>(
-        r->chunk_traj, r->chunk_seq, (int)r->nchunks, r->choff, r->chunk_table);
+        r->chunk_traj, r->chunk_seq, (int)r->nchunks, r->choff, r->chunk_table, bounds_of(r));
   if (cudaGetLastError() != cudaSuccess) return bail(fail(GS_ERR_CUDA, "chunk table launch failed"));
   if ((st = build_perm(r, s)) != GS_OK) return bail(st);
   *rec = r;
@@ -821,6 +828,7 @@ gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, v
       p.pool = static_cast<R*>(rec->pool);
       p.queue = queue;
       p.perm = rec->perm;
+      p.bounds = bounds_of(rec);
       auto kern = gs::k_replay_forward_mlp<R>;
       kern<<<persistent_grid(kern, 0, rec->N * 32), BLOCK, 0, s>>>(p);
       GS_CUDA(cudaGetLastError());
@@ -837,6 +845,7 @@ gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, v
     p.pool = static_cast<R*>(rec->pool);
     p.queue = queue;
     p.perm = rec->perm;
+    p.bounds = bounds_of(rec);
     auto kern = gs::k_replay_forward<F, R, METHOD>;
     const int grid = persistent_grid(kern, 0, rec->N);
     kern<<<grid, BLOCK, 0, s>>>(p);
@@ -885,6 +894,7 @@ void fill_replay_params(gs::ReplayParams<R>& p, const gs_record* rec, const void
   p.pool = static_cast<R*>(rec->pool);
   p.queue = queue;
   p.perm = rec->perm;
+  p.bounds = bounds_of(rec);
 }
 
 }  // namespace
@@ -970,6 +980,7 @@ gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_
       p.pool = static_cast<const R*>(rec->pool);
       p.queue = queue;
       p.perm = rec->perm;
+      p.bounds = bounds_of(rec);
       q.dL_dyout = static_cast<const R*>(dL_dyout);
       fill_times<R>(q.ot, rec, J, tau);
       auto kern = gs::k_adjoint_outputs<F, R, METHOD>;
@@ -988,6 +999,20 @@ gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_
       return GS_OK;
     }
   });
+}
+
+gs_status gs_checked_violations(int64_t* count) {
+#ifdef GS_CHECKED
+  if (!count) return fail(GS_ERR_INVALID_ARG, "count must be non-NULL");
+  unsigned long long v = 0, z = 0;
+  GS_CUDA(cudaMemcpyFromSymbol(&v, gs::g_gs_violations, sizeof(v)));
+  GS_CUDA(cudaMemcpyToSymbol(gs::g_gs_violations, &z, sizeof(z)));
+  *count = (int64_t)v;
+  return GS_OK;
+#else
+  (void)count;
+  return fail(GS_ERR_UNSUPPORTED, "not a checked build (compile with -DGS_CHECKED)");
+#endif
 }
 
 gs_status gs_record_info(const gs_record* rec, gs_record_info_t* out) {
@@ -1024,12 +1049,14 @@ gs_status gs_record_export(const gs_record* rec, void* T, void* H, void* Y, int6
     gs::k_export<double><<<nb, 256, 0, s>>>(static_cast<const double*>(rec->pool), rec->chunk_table,
                                             rec->choff, rec->offsets, (int)rec->N, rec->sys.d,
                                             rec->C, rec->total_steps, static_cast<double*>(T),
-                                            static_cast<double*>(H), static_cast<double*>(Y));
+                                            static_cast<double*>(H), static_cast<double*>(Y),
+                                            bounds_of(rec));
   else
     gs::k_export<float><<<nb, 256, 0, s>>>(static_cast<const float*>(rec->pool), rec->chunk_table,
                                            rec->choff, rec->offsets, (int)rec->N, rec->sys.d,
                                            rec->C, rec->total_steps, static_cast<float*>(T),
-                                           static_cast<float*>(H), static_cast<float*>(Y));
+                                           static_cast<float*>(H), static_cast<float*>(Y),
+                                           bounds_of(rec));
   GS_CUDA(cudaGetLastError());
   return GS_OK;
 }
@@ -1091,13 +1118,13 @@ gs_status gs_record_import(const gs_system* sys, int64_t N, const int32_t* nstep
                                                 (int)N, sys->d, C, r->total_steps,
                                                 static_cast<const double*>(T),
                                                 static_cast<const double*>(H),
-                                                static_cast<const double*>(Y));
+                                                static_cast<const double*>(Y), bounds_of(r));
       else
         gs::k_import<float><<<nb, 256, 0, s>>>(static_cast<float*>(r->pool), r->choff, r->offsets,
                                                (int)N, sys->d, C, r->total_steps,
                                                static_cast<const float*>(T),
                                                static_cast<const float*>(H),
-                                               static_cast<const float*>(Y));
+                                               static_cast<const float*>(Y), bounds_of(r));
       if (cudaGetLastError() != cudaSuccess) return bail(fail(GS_ERR_CUDA, "import launch failed"));
     }
     if ((st = build_perm(r, s)) != GS_OK) return bail(st);
@@ -1189,6 +1216,7 @@ gs_status noalloc_adjoint(const gs_record* r, const void* theta, const void* dL_
     p.pool = static_cast<const R*>(r->pool);
     p.queue = reinterpret_cast<int*>(scratch);
     p.perm = r->perm;
+    p.bounds = bounds_of(r);
     auto kern = gs::k_adjoint<F, R, METHOD>;
     const size_t smem = adjoint_smem<F, R>();
     int nb = 0;

@@ -26,6 +26,46 @@ namespace gs {
 
 constexpr unsigned FULL = 0xffffffffu;
 
+// ---------------------------------------------------------------------------------------------
+// Bounds of a record's device arrays, for the checked build (-DGS_CHECKED): every access through
+// the chunk table is checked against the allocated sizes; an out-of-range index is counted in
+// g_gs_violations and the access is redirected to a small scratch entry, so the kernel stays in
+// bounds and finishes (the result is then wrong and the count says so).  The normal build
+// compiles the checks away.
+// ---------------------------------------------------------------------------------------------
+struct RecBounds {
+  long long table_cap;   // entries allocated for the chunk table
+  long long pool_chunks; // chunks allocated in the pool
+};
+#ifdef GS_CHECKED
+__device__ unsigned long long g_gs_violations;
+__device__ double g_gs_scratch_entry[64];
+__device__ __forceinline__ void gs_violation() { atomicAdd(&g_gs_violations, 1ull); }
+#endif
+
+// Chunk id at chunk-table position ti (checked build: -1 when ti is outside the table).
+__device__ __forceinline__ int chunk_at(const int* table, long long ti, const RecBounds& b) {
+#ifdef GS_CHECKED
+  if (ti < 0 || ti >= b.table_cap) {
+    gs_violation();
+    return -1;
+  }
+#endif
+  return __ldg(table + ti);
+}
+// Entry of step n (slot n % C) in chunk ch (checked build: the scratch entry when ch is not a
+// chunk of the pool).
+template <class L, class R>
+__device__ __forceinline__ R* chunk_entry(R* pool, int ch, int n, const RecBounds& b) {
+#ifdef GS_CHECKED
+  if (ch < 0 || ch >= b.pool_chunks) {
+    gs_violation();
+    return reinterpret_cast<R*>(g_gs_scratch_entry);
+  }
+#endif
+  return pool + ((size_t)ch * L::C + (n % L::C)) * L::E;
+}
+
 // Record chunk: C accepted steps of one trajectory, entry = (t, h, y[0..D-1]) contiguous.
 template <class F, class R>
 struct RecLayout {
@@ -474,6 +514,7 @@ struct AdjointParams {
   const R* pool;
   int* queue;
   const int* perm;          // visiting order (longest records first); nullable = identity
+  RecBounds bounds;
 };
 
 template <class F, class R, int METHOD>
@@ -521,8 +562,11 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
         // chunk of step n; on entering a chunk, fetch the id of the next chunk to be visited and
         // prefetch its lines one step later (the id load then has had a whole step to land)
         if (n == first_n || n % L::C == L::C - 1) {
-          cur_ch = __ldg(p.chunk_table + cbase + n / L::C);
-          next_ch = (n / L::C >= 1) ? __ldg(p.chunk_table + cbase + n / L::C - 1) : -1;
+          cur_ch = chunk_at(p.chunk_table, cbase + n / L::C, p.bounds);
+          next_ch = (n / L::C >= 1) ? chunk_at(p.chunk_table, cbase + n / L::C - 1, p.bounds) : -1;
+#ifdef GS_CHECKED
+          if (next_ch >= p.bounds.pool_chunks) next_ch = -1;
+#endif
           pf_pending = next_ch >= 0;
         } else if (pf_pending) {
           const R* q = p.pool + (size_t)next_ch * L::C * L::E;
@@ -531,8 +575,7 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
             asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const char*>(q) + b));
           pf_pending = false;
         }
-        const int ch = cur_ch;
-        const R* e = p.pool + ((size_t)ch * L::C + (n % L::C)) * L::E;
+        const R* e = chunk_entry<L>(p.pool, cur_ch, n, p.bounds);
         const R h = __ldg(e + 1);
         R y[D];
 #pragma unroll
@@ -583,6 +626,7 @@ struct ReplayParams {
   R* pool;
   int* queue;
   const int* perm;
+  RecBounds bounds;
 };
 
 template <class F, class R, int METHOD>
@@ -617,8 +661,8 @@ __global__ void __launch_bounds__(128) k_replay_forward(ReplayParams<R> p) {
     if (!__any_sync(FULL, k >= 0 || alive)) break;
     if (k >= 0) {
       if (n < S) {
-        const int ch = p.chunk_table[cbase + n / L::C];
-        R* e = p.pool + ((size_t)ch * L::C + (n % L::C)) * L::E;
+        R* e = chunk_entry<L>(p.pool, chunk_at(p.chunk_table, cbase + n / L::C, p.bounds), n,
+                              p.bounds);
         const R h = e[1];
 #pragma unroll
         for (int c = 0; c < D; ++c) e[2 + c] = y[c];
@@ -663,8 +707,8 @@ struct OutParams {
 template <class F, class R>
 __device__ __forceinline__ const R* rec_entry(const ReplayParams<R>& p, long long cbase, int n) {
   using L = RecLayout<F, R>;
-  const int ch = p.chunk_table[cbase + n / L::C];
-  return p.pool + ((size_t)ch * L::C + (n % L::C)) * L::E;
+  return chunk_entry<L>(p.pool, chunk_at(p.chunk_table, cbase + n / L::C, p.bounds), n,
+                        p.bounds);
 }
 
 template <class F, class R, int METHOD>
@@ -771,8 +815,8 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
     const long long cbase = p.choff[k];
     int jcur = S == 0 ? 0 : jS;
     for (int n = S - 1; n >= 0; --n) {
-      const int ch = p.chunk_table[cbase + n / L::C];
-      const R* e = p.pool + ((size_t)ch * L::C + (n % L::C)) * L::E;
+      const R* e = chunk_entry<L>(p.pool, chunk_at(p.chunk_table, cbase + n / L::C, p.bounds), n,
+                                  p.bounds);
       const R t = e[0], h = e[1];
       R y[D];
 #pragma unroll
@@ -883,11 +927,20 @@ __global__ void k_scan_add(long long* out, int N, const long long* tile_base,
 
 // chunk_table[choff[traj] + seq] = chunk (reserved-but-unused chunks carry traj = -1)
 __global__ void k_chunk_table(const int* chunk_traj, const int* chunk_seq, int nchunks,
-                              const long long* choff, int* table) {
+                              const long long* choff, int* table, RecBounds b) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c < nchunks) {
     const int k = chunk_traj[c];
-    if (k >= 0) table[choff[k] + chunk_seq[c]] = c;
+    if (k >= 0) {
+      const long long ti = choff[k] + chunk_seq[c];
+#ifdef GS_CHECKED
+      if (ti < 0 || ti >= b.table_cap) {
+        gs_violation();
+        return;
+      }
+#endif
+      table[ti] = c;
+    }
   }
 }
 
@@ -905,7 +958,7 @@ __global__ void k_max_int(const int* S, int N, int* out) {
 template <class R>
 __global__ void k_export(const R* pool, const int* table, const long long* choff,
                          const long long* offsets, int N, int D, int C, long long total, R* T,
-                         R* H, R* Y) {
+                         R* H, R* Y, RecBounds b) {
   const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (g >= total) return;
   // binary search the trajectory owning step g
@@ -917,8 +970,15 @@ __global__ void k_export(const R* pool, const int* table, const long long* choff
   const int k = lo;
   const long long n = g - offsets[k];
   const int E = 2 + D;
-  const int ch = table[choff[k] + n / C];
+  const long long ti = choff[k] + n / C;
+  const int ch = table[ti];
   const R* e = pool + ((size_t)ch * C + (n % C)) * E;
+#ifdef GS_CHECKED
+  if (ti < 0 || ti >= b.table_cap || ch < 0 || ch >= b.pool_chunks) {
+    gs_violation();
+    return;
+  }
+#endif
   if (T) T[g] = e[0];
   if (H) H[g] = e[1];
   if (Y) for (int c = 0; c < D; ++c) Y[g * D + c] = e[2 + c];
@@ -928,7 +988,8 @@ __global__ void k_export(const R* pool, const int* table, const long long* choff
 // (chunk id = choff[k] + n / C, so chunk_table is the identity).
 template <class R>
 __global__ void k_import(R* pool, const long long* choff, const long long* offsets, int N, int D,
-                         int C, long long total, const R* T, const R* H, const R* Y) {
+                         int C, long long total, const R* T, const R* H, const R* Y,
+                         RecBounds b) {
   const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (g >= total) return;
   int lo = 0, hi = N - 1;
@@ -940,6 +1001,12 @@ __global__ void k_import(R* pool, const long long* choff, const long long* offse
   const long long n = g - offsets[k];
   const int E = 2 + D;
   const long long ch = choff[k] + n / C;
+#ifdef GS_CHECKED
+  if (ch < 0 || ch >= b.pool_chunks) {
+    gs_violation();
+    return;
+  }
+#endif
   R* e = pool + ((size_t)ch * C + (n % C)) * E;
   e[0] = T ? T[g] : R(0);
   e[1] = H[g];

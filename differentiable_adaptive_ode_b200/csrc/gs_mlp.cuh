@@ -338,8 +338,8 @@ __global__ void __launch_bounds__(128) k_replay_forward_mlp(ReplayParams<R> p) {
     const int S = p.nsteps[k];
     const long long cbase = p.choff[k];
     for (int n = 0; n < S; ++n) {
-      const int ch = p.chunk_table[cbase + n / L::C];
-      R* e = p.pool + ((size_t)ch * L::C + (n % L::C)) * L::E;
+      R* e = chunk_entry<L>(p.pool, chunk_at(p.chunk_table, cbase + n / L::C, p.bounds), n,
+                            p.bounds);
       const R h = e[1];
       __syncwarp();
       if (lane < D) e[2 + lane] = y[lane];
@@ -389,6 +389,7 @@ struct MlpAdjParams {
   const int* chunk_table;
   const R* pool;
   const int* perm;
+  RecBounds bounds;
 };
 
 template <class R>
@@ -410,8 +411,8 @@ __global__ void __launch_bounds__(128) k_adjoint_mlp(MlpAdjParams<R> p) {
     for (int c = 0; c < D; ++c) lam[c] = p.dL_dy1[(size_t)k * D + c];
     const long long cbase = p.choff[k];
     for (int n = p.nsteps[k] - 1; n >= 0; --n) {
-      const int ch = p.chunk_table[cbase + n / L::C];
-      const R* e = p.pool + ((size_t)ch * L::C + (n % L::C)) * L::E;
+      const R* e = chunk_entry<L>(p.pool, chunk_at(p.chunk_table, cbase + n / L::C, p.bounds),
+                                  n, p.bounds);
       const R h = e[1];
       R y[D];
 #pragma unroll

@@ -13,6 +13,9 @@ import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libgradsolve_b200.so")
+CHECKED_LIB_PATH = os.path.join(PKG, "libgradsolve_b200_checked.so")
+if os.environ.get("GRADSOLVE_B200_CHECKED") == "1":   # the bounds-checked build of the library
+    LIB_PATH = CHECKED_LIB_PATH
 
 GS_OK, GS_ERR_INVALID_ARG, GS_ERR_CUDA, GS_ERR_CAPACITY, GS_ERR_UNSUPPORTED, GS_ERR_TRAJ_FAILED = range(6)
 GS_F64, GS_F32 = 0, 1
@@ -28,10 +31,10 @@ STATUS_NAMES = {0: "GS_OK", 1: "GS_ERR_INVALID_ARG", 2: "GS_ERR_CUDA", 3: "GS_ER
                 4: "GS_ERR_UNSUPPORTED", 5: "GS_ERR_TRAJ_FAILED"}
 
 # every entry point declared in include/gradsolve_b200.h
-EXPORTS = ("gs_solve_forward", "gs_solve_forward_sens", "gs_solve_record", "gs_replay_grad", "gs_replay_forward",
-           "gs_replay_grad_noalloc", "gs_replay_outputs", "gs_replay_grad_outputs", "gs_record_info",
-           "gs_record_export", "gs_record_import", "gs_record_destroy", "gs_last_error",
-           "gs_version")
+EXPORTS = ("gs_solve_forward", "gs_solve_forward_sens", "gs_solve_record", "gs_replay_grad",
+           "gs_replay_forward", "gs_replay_grad_noalloc", "gs_replay_outputs",
+           "gs_replay_grad_outputs", "gs_record_info", "gs_record_export", "gs_record_import",
+           "gs_record_destroy", "gs_last_error", "gs_version", "gs_checked_violations")
 
 
 class GsSystem(C.Structure):
@@ -85,6 +88,8 @@ def lib():
         L.gs_replay_outputs.argtypes = [vp, vp, vp, C.c_int32, pd, vp, vp]
         L.gs_replay_grad_outputs.argtypes = [vp, vp, C.c_int32, pd, vp, vp, vp, vp, vp]
         L.gs_record_info.argtypes = [vp, P(GsRecordInfo)]
+        L.gs_checked_violations.argtypes = [P(C.c_int64)]
+        L.gs_checked_violations.restype = C.c_int
         L.gs_record_export.argtypes = [vp, vp, vp, vp, vp, vp]
         L.gs_record_import.argtypes = [P(GsSystem), i64, vp, vp, vp, vp, P(vp), vp]
         L.gs_record_destroy.argtypes = [vp]
@@ -251,6 +256,13 @@ def gs_record_import(sys, N, nsteps, T, H, Y, stream=None):
     _check(lib().gs_record_import(C.byref(sys), N, _ptr(nsteps), _ptr(T), _ptr(H), _ptr(Y),
                                   C.byref(rec.handle), _stream(stream)))
     return rec
+
+
+def checked_violations():
+    """Out-of-range record accesses counted by the checked build since the last call."""
+    v = C.c_int64(0)
+    _check(lib().gs_checked_violations(C.byref(v)))
+    return v.value
 
 
 def version():

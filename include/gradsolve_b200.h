@@ -232,6 +232,13 @@ gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_
 gs_status gs_replay_grad_noalloc(const gs_record* rec, const void* theta, const void* dL_dy1,
                                  void* dL_dtheta, void* dL_dy0, void* stream);
 
+/* Checked build (compiled with -DGS_CHECKED into libgradsolve_b200_checked.so): every access
+ * through a record's chunk table is checked against the allocated pool and table, and an
+ * out-of-range one is counted and redirected to scratch memory instead of touching memory
+ * outside the record.  Returns, in *count, the number counted since the previous call (the
+ * counter is then reset).  Synchronises the device.  The normal build returns GS_ERR_UNSUPPORTED. */
+gs_status gs_checked_violations(int64_t* count);
+
 /* Sizes and device pointers of a record (no synchronisation). */
 gs_status gs_record_info(const gs_record* rec, gs_record_info_t* out);
 

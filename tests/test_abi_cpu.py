@@ -77,3 +77,18 @@ def test_binding_refuses_without_library(monkeypatch):
     monkeypatch.setattr(gradsolve, "LIB_PATH", "/nonexistent/libgradsolve_b200.so")
     with pytest.raises(RuntimeError):
         gradsolve.lib()
+
+
+def test_normal_build_has_no_violation_counter(G):
+    import ctypes as C
+    v = C.c_int64(0)
+    assert G.lib().gs_checked_violations(C.byref(v)) == G.GS_ERR_UNSUPPORTED
+
+
+def test_checked_build_compiles_and_exports():
+    import ctypes as C
+    from differentiable_adaptive_ode_b200 import build
+    path = build.build(checked=True)
+    L = C.CDLL(path)
+    for name in declared():
+        assert hasattr(L, name), name

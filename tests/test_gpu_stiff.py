@@ -76,3 +76,31 @@ def test_hires_reference_solution_on_gpu():
     fw = U.forward(w)
     assert np.all(fw["status"] == 0)
     assert np.max(np.abs(fw["y1"][0] - ref) / ref) < 1e-8
+
+
+@pytest.mark.parametrize("name,rtol,atol,t1", [("robertson_rb23", 1e-4, 1e-8, 1.0),
+                                               ("lorenz63_vern7", 1e-5, 1e-6, None)])
+def test_fp32_methods_on_their_own_mesh(orc, name, rtol, atol, t1):
+    # fp32 reading: states against the fp32 oracle replay of the GPU's own mesh, gradients against
+    # the exact (fp64) derivative of the replay over that mesh.  (Robertson over [0, 1e4] is out
+    # of reach in fp32: the step-size floor 16 eps |t1 - t0| = 0.02 is above the initial
+    # transient's steps, so every trajectory ends with status 2; the test takes [0, 1].)
+    w = U.small(name, 300)
+    w.dtype, w.rtol, w.atol = np.float32, rtol, atol
+    if t1 is not None:
+        w.t1 = t1
+    rec, out = U.record(w)
+    assert np.all(out["status"] == 0)
+    ex = U.export_padded(w, rec)
+    yrep = orc.replay(w.field, w.method, w.theta, w.y0, ex["H"], ex["S"], dtype=np.float32,
+                      theta_shared=w.theta_shared)
+    err = U.rel_rows(out["y1"], yrep, atol)
+    assert np.quantile(err, 0.99) <= 1e-4 and err.max() <= 1e-3, err.max()
+    lam = np.random.default_rng(12).normal(size=(w.N, w.d))
+    gy, gt = U.replay_grad(w, rec, lam)
+    ry, rt = orc.replay_grad(w.field, w.method, w.theta.astype(np.float32).astype(np.float64),
+                             w.y0.astype(np.float32).astype(np.float64),
+                             ex["H"].astype(np.float64), ex["S"], lam, nthreads=8)
+    for got, want in ((gy, ry), (gt, rt)):
+        rel = U.rel_rows(got, want, 1e-300)
+        assert np.quantile(rel, 0.99) <= 1e-3 and rel.max() <= 1e-2, rel.max()
