@@ -88,6 +88,16 @@ TRAFFIC_PER_STEP = {
     "hires": {"record": 373.4, "adjoint": 99.1},          # record: spill traffic (d = 8 LU)
     "lorenz63_vern7": {"adjoint": 46.4},                   # its record pass stays partly in L2
 }
+# FP64 pipe occupancy (sm__pipe_fp64_cycles_active, % of peak) of the same captures: how busy the
+# pipe is, transcendental sequences included, next to the algorithmic fraction
+PIPE_BUSY_NCU = {
+    "nfw_mn": {"record": 0.404, "adjoint": 0.568},
+    "robertson": {"record": 0.415, "adjoint": 0.354},
+    "robertson_rb23": {"record": 0.342, "adjoint": 0.343},
+    "hires": {"record": 0.177, "adjoint": 0.204},
+    "lorenz63_vern7": {"record": 0.457, "adjoint": 0.552},
+    "log_halo": {"sens": 0.617},
+}
 # forward sensitivities: DRAM bytes per trajectory (inputs and outputs; nothing per step), from
 # the ncu capture of the 2^18-orbit case
 TRAFFIC_SENS_PER_TRAJ = {"log_halo": 50.8}
@@ -456,6 +466,7 @@ def run_sens(args, w, wl, G, torch, dev, stream, ws, rank):
     achieved = flops / (kernel_ms / 1e3) / 1e12
     roofline = {"kernel": "k_solve<log_halo, double, Tsit5, sens>", "bound": "alu",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "pipe_busy_ncu": PIPE_BUSY_NCU.get(args.workload, {}).get("sens"),
                 "traffic": TRAFFIC_SENS_PER_TRAJ[args.workload] * N,
                 "traffic_source": "ncu dram bytes per trajectory on the 2^18 case x trajectories",
                 "peak_source": "derived: 148 SM x 64 FP64 FMA lanes/clk x 2 x 1965 MHz (FP64 pipe)",
@@ -714,9 +725,10 @@ def main():
     at_clock = pipe_peak_tflops(clocks["sm_mhz"], lanes) if clocks.get("sm_mhz") else None
     pipe = "FP64" if f64 else "FP32"
 
-    def roof(name, per_unit, units, ms, unit_name, traffic):
+    def roof(name, per_unit, units, ms, unit_name, traffic, busy=None):
         achieved = per_unit * units / (ms / 1e3) / 1e12 if per_unit else None
         return {"kernel": name, "bound": "alu", "achieved": achieved, "peak": peak_max,
+                "pipe_busy_ncu": busy,
                 "unit": "TFLOP/s", "frac": achieved / peak_max if achieved else None,
                 "traffic": traffic,
                 "traffic_source": "ncu dram bytes per accepted step of one capture x steps",
@@ -731,10 +743,12 @@ def main():
     traffic = TRAFFIC_PER_STEP.get(args.workload, {})
     roof_rec = roof("k_solve<%s, %s, %s, record>" % (w.field, "double" if f64 else "float", method),
                     wl["fwd"], attempts, rec_kernel_ms, "attempted step",
-                    traffic.get("record", 0) * total_steps or None)
+                    traffic.get("record", 0) * total_steps or None,
+                    PIPE_BUSY_NCU.get(args.workload, {}).get("record"))
     roof_adj = roof("k_adjoint<%s, %s, %s>" % (w.field, "double" if f64 else "float", method),
                     wl["adj"], total_steps, adj_ms, "accepted step",
-                    traffic.get("adjoint", 0) * total_steps or None)
+                    traffic.get("adjoint", 0) * total_steps or None,
+                    PIPE_BUSY_NCU.get(args.workload, {}).get("adjoint"))
     dominant, other = (roof_rec, roof_adj) if rec_kernel_ms >= adj_ms else (roof_adj, roof_rec)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,

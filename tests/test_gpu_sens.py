@@ -151,3 +151,19 @@ def test_start_order_changes_nothing_but_the_schedule():
         assert np.array_equal(y1f.cpu().numpy(), base["y1"])
         assert np.array_equal(S1.cpu().numpy(), base["sens"])
         assert np.array_equal(S.cpu().numpy(), base["S"])
+
+
+def test_sens_non_finite_parameters_and_attempt_cap():
+    # per-trajectory theta with a NaN: that trajectory ends at start-up with status 3 and its S is
+    # the starting S0 (zero); the others are unaffected.  A cap of 5 attempts gives status 1.
+    w = U.small("lorenz63", 16)
+    w.theta = w.theta.copy()
+    w.theta[5, 1] = np.nan
+    g = U.forward_sens(w)
+    assert g["status"][5] == 3 and np.all(np.delete(g["status"], 5) == 0)
+    assert np.all(g["sens"][5] == 0)
+    ok = U.forward_sens(U.small("lorenz63", 16))
+    keep = np.delete(np.arange(16), 5)
+    assert np.array_equal(g["sens"][keep], ok["sens"][keep])
+    capped = U.forward_sens(U.small("lorenz63", 16), max_attempts=5)
+    assert np.all(capped["status"] == 1) and np.all(capped["S"] + capped["rejected"] == 5)
