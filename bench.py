@@ -592,10 +592,18 @@ def main():
     def loss_cotangent():
         torch.mul(torch.sub(y1, target), mask, out=lam).mul_(scale)
 
+    # a parameter vector shared by the whole ensemble is shared across ranks too: its cotangent is
+    # summed over the ranks' ensembles (the one exchange of the path; m values)
+    reduce_shared = ws > 1 and w.theta_shared
+    if reduce_shared:
+        from differentiable_adaptive_ode_b200.ensemble import allreduce_theta_bar
+
     def step():
         G.gs_solve_record(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, rec=rec)
         loss_cotangent()
         G.gs_replay_grad(rec, th, lam, gt, gy)
+        if reduce_shared:
+            allreduce_theta_bar(gt)
 
     for _ in range(args.warmup):
         step()
@@ -622,6 +630,8 @@ def main():
             adj_ev[i][0].record(stream)
             G.gs_replay_grad(rec, th, lam, gt, gy)
             adj_ev[i][1].record(stream)
+            if reduce_shared:
+                allreduce_theta_bar(gt)
         stop.record(stream)
         barrier()
     total_ms = start.elapsed_time(stop)
@@ -689,6 +699,8 @@ def main():
                               rec=q["rec"])
             torch.mul(torch.sub(q["y1"], target), mask, out=q["lam"]).mul_(scale)
             G.gs_replay_grad(q["rec"], q["th"], q["lam"], q["gt"], q["gy"])
+            if reduce_shared:
+                allreduce_theta_bar(q["gt"])
             q["h_gt"].copy_(q["gt"], non_blocking=True)
             q["h_gy"].copy_(q["gy"], non_blocking=True)
 
