@@ -1,6 +1,7 @@
 // gs_api.cu -- the C ABI declared in include/gradsolve_b200.h: argument checks, record lifecycle,
 // kernel launches.  Every entry point returns a status; nothing here aborts.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -16,6 +17,13 @@
 #include "gradsolve_b200.h"
 #include "gs_kernels.cuh"
 #include "gs_mlp.cuh"
+
+// NVTX range over one entry point (header-only NVTX v3): profilers show each library call as a
+// named range around its kernels.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 
 namespace {
 
@@ -589,6 +597,7 @@ gs_status gs_solve_forward(const gs_system* sys, const gs_options* opt, int64_t 
                            const void* theta, const void* y0, double t0, double t1, double rtol,
                            double atol, void* y1, int32_t* nsteps, int32_t* nrejected,
                            int32_t* status, void* stream) {
+  NvtxRange nvtx_range("gs_solve_forward");
   gs_status st = check_common(sys, N, theta, y0, t0, t1, rtol, atol, y1);
   if (st != GS_OK) return st;
   if (N == 0) return GS_OK;
@@ -606,6 +615,7 @@ gs_status gs_solve_forward_sens(const gs_system* sys, const gs_options* opt, int
                                 double t1, double rtol, double atol, void* y1, void* S1,
                                 int32_t* nsteps, int32_t* nrejected, int32_t* status,
                                 void* stream) {
+  NvtxRange nvtx_range("gs_solve_forward_sens");
   gs_status st = check_common(sys, N, theta, y0, t0, t1, rtol, atol, y1);
   if (st != GS_OK) return st;
   if (sys->method != GS_TSIT5 || sys->field == GS_MLP_4_32_32_4)
@@ -625,6 +635,7 @@ gs_status gs_solve_forward_sens(const gs_system* sys, const gs_options* opt, int
 gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N,
                           const void* theta, const void* y0, double t0, double t1, double rtol,
                           double atol, gs_record** rec, void* y1, int32_t* status, void* stream) {
+  NvtxRange nvtx_range("gs_solve_record");
   gs_status st = check_common(sys, N, theta, y0, t0, t1, rtol, atol, y1);
   if (st != GS_OK) return st;
   if (!rec) return fail(GS_ERR_INVALID_ARG, "rec must be non-NULL");
@@ -749,6 +760,7 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
 
 gs_status gs_replay_grad(const gs_record* rec, const void* theta, const void* dL_dy1,
                          void* dL_dtheta, void* dL_dy0, void* stream) {
+  NvtxRange nvtx_range("gs_replay_grad");
   if (!rec) return fail(GS_ERR_INVALID_ARG, "record is NULL");
   if (rec->N == 0) return GS_OK;
   if (!theta || !dL_dy1) return fail(GS_ERR_INVALID_ARG, "theta and dL_dy1 must be non-NULL");
@@ -797,6 +809,7 @@ gs_status gs_replay_grad(const gs_record* rec, const void* theta, const void* dL
 
 gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, void* y1,
                             void* stream) {
+  NvtxRange nvtx_range("gs_replay_forward");
   if (!rec) return fail(GS_ERR_INVALID_ARG, "record is NULL");
   if (rec->N == 0) return GS_OK;
   if (!theta || !y0) return fail(GS_ERR_INVALID_ARG, "theta and y0 must be non-NULL");
@@ -903,6 +916,7 @@ extern "C" {
 
 gs_status gs_replay_outputs(const gs_record* rec, const void* theta, const void* y0, int32_t J,
                             const double* tau, void* y_out, void* stream) {
+  NvtxRange nvtx_range("gs_replay_outputs");
   gs_status st = check_out_times(rec, J, tau);
   if (st != GS_OK) return st;
   if (rec->N == 0) return GS_OK;
@@ -931,6 +945,7 @@ gs_status gs_replay_outputs(const gs_record* rec, const void* theta, const void*
 gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_t J,
                                  const double* tau, const void* dL_dyout, const void* dL_dy1,
                                  void* dL_dtheta, void* dL_dy0, void* stream) {
+  NvtxRange nvtx_range("gs_replay_grad_outputs");
   gs_status st = check_out_times(rec, J, tau);
   if (st != GS_OK) return st;
   if (rec->N == 0) return GS_OK;
@@ -1038,6 +1053,7 @@ gs_status gs_record_info(const gs_record* rec, gs_record_info_t* out) {
 
 gs_status gs_record_export(const gs_record* rec, void* T, void* H, void* Y, int64_t* offsets,
                            void* stream) {
+  NvtxRange nvtx_range("gs_record_export");
   if (!rec) return fail(GS_ERR_INVALID_ARG, "record is NULL");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (offsets && rec->N >= 0)
@@ -1063,6 +1079,7 @@ gs_status gs_record_export(const gs_record* rec, void* T, void* H, void* Y, int6
 
 gs_status gs_record_import(const gs_system* sys, int64_t N, const int32_t* nsteps, const void* T,
                            const void* H, const void* Y, gs_record** rec, void* stream) {
+  NvtxRange nvtx_range("gs_record_import");
   gs_status st = check_system(sys);
   if (st != GS_OK) return st;
   if (!rec) return fail(GS_ERR_INVALID_ARG, "rec must be non-NULL");
@@ -1240,6 +1257,7 @@ gs_status noalloc_adjoint(const gs_record* r, const void* theta, const void* dL_
 extern "C" gs_status gs_replay_grad_noalloc(const gs_record* rec, const void* theta,
                                             const void* dL_dy1, void* dL_dtheta, void* dL_dy0,
                                             void* stream) {
+  NvtxRange nvtx_range("gs_replay_grad_noalloc");
   if (!rec) return fail(GS_ERR_INVALID_ARG, "record is NULL");
   if (rec->N == 0) return GS_OK;
   if (!theta || !dL_dy1) return fail(GS_ERR_INVALID_ARG, "theta and dL_dy1 must be non-NULL");

@@ -174,6 +174,22 @@ class Record:
     def info(self):
         return gs_record_info(self)
 
+    def order(self):
+        """The record's longest-first trajectory order as an int32 CUDA tensor that views the
+        library-owned array (valid until the record is made again or freed), or None; usable as
+        options(start_order=...) for later solves of the same ensemble."""
+        import torch
+        inf = self.info()
+        if not inf.order or inf.N == 0:
+            return None
+
+        class _View:
+            def __init__(self, ptr, n):
+                self.__cuda_array_interface__ = {"shape": (n,), "typestr": "<i4",
+                                                 "data": (ptr, False), "version": 3}
+
+        return torch.as_tensor(_View(inf.order, int(inf.N)), device="cuda")
+
     def close(self):
         if self.handle and self.handle.value:
             lib().gs_record_destroy(self.handle)

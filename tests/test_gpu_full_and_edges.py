@@ -204,18 +204,19 @@ def test_rerecord_in_previous_order_is_bitwise_identical():
 
 
 def test_record_info_order_is_longest_first_permutation():
-    import torch
-
-    class _Dev:  # a view of a library-owned device array through the CUDA array interface
-        def __init__(self, ptr, n):
-            self.__cuda_array_interface__ = {"shape": (n,), "typestr": "<i4",
-                                             "data": (ptr, False), "version": 3}
-
     w = W.lorenz63(N=777)
     rec, _ = U.record(w)
-    info = rec.info()
     ex = U.export_padded(w, rec)
-    assert info.order
-    o = torch.as_tensor(_Dev(info.order, w.N), device="cuda").cpu().numpy()
+    assert rec.info().order
+    o = rec.order().cpu().numpy()
     assert np.array_equal(np.sort(o), np.arange(w.N))
     assert np.all(np.diff(ex["S"][o]) <= 0)
+    # used as the start order of a forward solve: the same results
+    f0 = U.forward(w)
+    import torch
+    y1 = torch.empty((w.N, w.d), dtype=torch.float64, device="cuda")
+    G.gs_solve_forward(U.gsys(w), w.N, U.dev(w.theta, torch.float64), U.dev(w.y0, torch.float64),
+                       w.t0, w.t1, w.rtol, w.atol, y1,
+                       opts=G.options(start_order=rec.order().clone()))
+    torch.cuda.synchronize()
+    assert np.array_equal(y1.cpu().numpy(), f0["y1"])
