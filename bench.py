@@ -228,14 +228,10 @@ def run_reference(args):
     from differentiable_adaptive_ode_b200 import workloads as W
     from oracle import oracle as orc
     nthreads = orc.host_threads()
-    n_sample = args.ref_sample
     w_full = W.by_name(args.workload)
-    w = W.by_name(args.workload, N=n_sample)
-    lam = None
-    times = []
     sens = WORKLOADS[args.workload].get("step") == "sens"
-    for i in range(args.warmup + args.steps):
-        t0 = time.perf_counter()
+
+    def one_step(w):
         if sens:
             orc.solve_sens(w.field, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol, dtype=w.dtype,
                            theta_shared=w.theta_shared, nthreads=nthreads)
@@ -247,6 +243,20 @@ def run_reference(args):
             lam = W.loss_cotangent(w, r["y1"], tgt)
             orc.replay_grad(w.field, w.method, w.theta, w.y0, r["H"], r["S"], lam,
                             nthreads=nthreads, dtype=w.dtype, theta_shared=w.theta_shared)
+
+    n_sample = args.ref_sample
+    if n_sample <= 0:
+        # a sample of about 3 s of host work per step (so that the whole run stays within
+        # minutes), from a 64-trajectory calibration, between 64 and 4096 trajectories
+        t0 = time.perf_counter()
+        one_step(W.by_name(args.workload, N=64))
+        per = (time.perf_counter() - t0) / 64
+        n_sample = int(min(4096, max(64, 3.0 / max(per, 1e-9))))
+    w = W.by_name(args.workload, N=n_sample)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        one_step(w)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             times.append(dt)
@@ -525,7 +535,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="nfw_mn", choices=sorted(WORKLOADS))
     ap.add_argument("--N", type=int, default=0, help="trajectories per GPU (0: the workload's)")
-    ap.add_argument("--ref-sample", type=int, default=1024)
+    ap.add_argument("--ref-sample", type=int, default=0,
+                    help="trajectories per reference step (0: about 3 s of host work)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.impl == "reference":
