@@ -247,10 +247,10 @@ def run_reference(args):
     n_sample = args.ref_sample
     if n_sample <= 0:
         # a sample of about 3 s of host work per step (so that the whole run stays within
-        # minutes), from a 64-trajectory calibration, between 64 and 4096 trajectories
+        # minutes), from a 256-trajectory calibration, between 64 and 4096 trajectories
         t0 = time.perf_counter()
-        one_step(W.by_name(args.workload, N=64))
-        per = (time.perf_counter() - t0) / 64
+        one_step(W.by_name(args.workload, N=256))
+        per = (time.perf_counter() - t0) / 256
         n_sample = int(min(4096, max(64, 3.0 / max(per, 1e-9))))
     w = W.by_name(args.workload, N=n_sample)
     times = []
