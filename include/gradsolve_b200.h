@@ -9,10 +9,13 @@
  *   the fixed-step replay over that mesh with the mesh held fixed as data (§3: d Psi(theta;
  *   sg[R(theta0)]) / d theta, Eq. 4), with respect to theta, y0 or both.  The loss is a scalar
  *   L = sum_k l(y_k(t1; theta)) (§2.2), so the caller passes dL/dy1 and receives the pull-back.
- *   Non-stiff problems use the Tsit5 5(4) pair with first-same-as-last reuse (§2.1, §3.1); stiff
- *   problems a linearly implicit Rosenbrock-Wanner step, here ROS34PW2, whose stages solve with
- *   I - gamma h J and whose backward pass uses one transpose solve per stage and differentiates J
- *   (§3.2).  One GPU thread integrates one trajectory with its state in registers (§2.4, §4.1).
+ *   Non-stiff problems use the Tsit5 5(4) pair with first-same-as-last reuse (§2.1, §3.1) or
+ *   Verner's 7(6) pair; stiff problems a linearly implicit Rosenbrock-Wanner step (ROS34PW2 or
+ *   Rosenbrock23), whose stages solve with I - gamma h J and whose backward pass uses transpose
+ *   solves with the same factorisation and differentiates J (§3.2).  One GPU thread integrates
+ *   one trajectory with its state in registers (§2.4, §4.1); the neural field takes one warp.
+ *   gs_solve_forward_sens integrates forward sensitivities dy/dtheta with the orbit instead
+ *   ([DA] = "Differentiable astrophysics at scale", §2-§3).
  *
  * Conventions (all entry points):
  *   - Real arrays are double (GS_F64) or float (GS_F32) per gs_system.dtype, row-major:
