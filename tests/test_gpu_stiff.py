@@ -104,3 +104,31 @@ def test_fp32_methods_on_their_own_mesh(orc, name, rtol, atol, t1):
     for got, want in ((gy, ry), (gt, rt)):
         rel = U.rel_rows(got, want, 1e-300)
         assert np.quantile(rel, 0.99) <= 1e-3 and rel.max() <= 1e-2, rel.max()
+
+
+@pytest.mark.parametrize("name", ["robertson_rb23", "hires"])
+def test_stiff_outputs_at_requested_times(orc, name):
+    import torch
+    w = U.small(name, 64)
+    rec, out = U.record(w)
+    ex = U.export_padded(w, rec)
+    tau = np.array([w.t0 + (w.t1 - w.t0) * f for f in (0.001, 0.1, 0.5, 1.0)])
+    dt = torch.float64
+    yo = torch.empty((w.N, len(tau), w.d), dtype=dt, device="cuda")
+    G.gs_replay_outputs(rec, U.dev(w.theta, dt), U.dev(w.y0, dt), tau, yo)
+    lo = np.random.default_rng(13).normal(size=(w.N, len(tau), w.d))
+    gy = torch.empty((w.N, w.d), dtype=dt, device="cuda")
+    gt = torch.empty((w.m,) if w.theta_shared else (w.N, w.m), dtype=dt, device="cuda")
+    G.gs_replay_grad_outputs(rec, U.dev(w.theta, dt), tau, U.dev(lo, dt), None, gt, gy)
+    torch.cuda.synchronize()
+    want = orc.replay_outputs(w.field, w.method, w.theta, w.y0, ex["T"], ex["H"], ex["S"], w.t1,
+                              tau, theta_shared=w.theta_shared, nthreads=8)
+    assert U.rel_rows(yo.cpu().numpy().reshape(w.N, -1), want.reshape(w.N, -1),
+                      w.atol).max() <= 1e-9
+    ry, rt = orc.replay_outputs_grad(w.field, w.method, w.theta, w.y0, ex["T"], ex["H"], ex["S"],
+                                     w.t1, tau, lo, theta_shared=w.theta_shared, nthreads=8)
+    assert U.rel_rows(gy.cpu().numpy(), ry, 1e-300).max() <= 1e-8
+    got_t = gt.cpu().numpy()
+    if w.theta_shared:
+        got_t, rt = got_t[None, :], rt.sum(0, keepdims=True)
+    assert U.rel_rows(got_t, rt, 1e-300).max() <= 1e-8
