@@ -22,7 +22,9 @@ from differentiable_adaptive_ode_b200 import workloads as W  # noqa: E402
 from oracle import oracle as orc  # noqa: E402
 
 CASES = [("lotka_volterra", 4), ("lorenz63", 4), ("robertson", 2), ("nfw_mn", 4),
-         ("nfw_mn_f32", 4), ("mlp", 2)]
+         ("nfw_mn_f32", 4), ("mlp", 2), ("lorenz63_vern7", 3), ("robertson_rb23", 2),
+         ("hires", 1), ("log_halo", 3)]
+SENS_CASES = [("log_halo", 3), ("lorenz63", 2)]
 
 
 def compute(name, N):
@@ -39,11 +41,22 @@ def compute(name, N):
                 dL_dy0=gy.tolist(), dL_dtheta=gt.tolist())
 
 
+def compute_sens(name, N):
+    w = W.by_name(name, N=N)
+    r = orc.solve_sens(w.field, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol,
+                       theta_shared=w.theta_shared)
+    return dict(S=r["S"].tolist(), rejected=r["rejected"].tolist(), y1=r["y1"].tolist(),
+                sens=r["sens"].tolist())
+
+
 def main():
     out = {"source": "oracle/ (CPU), seeds of differentiable_adaptive_ode_b200.workloads",
            "lam": "numpy default_rng(12345).normal(size=(N, d))", "cases": {}}
     for name, N in CASES:
         out["cases"][name] = dict(N=N, **compute(name, N))
+    out["sens_cases"] = {}
+    for name, N in SENS_CASES:
+        out["sens_cases"][name] = dict(N=N, **compute_sens(name, N))
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "oracle_small_cases.json")
     with open(path, "w") as f:
         json.dump(out, f, indent=1)

@@ -21,3 +21,9 @@ def test_oracle_reproduces_golden_anchors():
         for key in ("y1", "dL_dy0", "dL_dtheta"):
             a, b = np.asarray(got[key]), np.asarray(case[key])
             assert np.max(np.abs(a - b)) <= rtol * max(1.0, np.max(np.abs(b))), (name, key)
+    for name, case in gold.get("sens_cases", {}).items():
+        got = make_golden.compute_sens(name, case["N"])
+        assert got["S"] == case["S"] and got["rejected"] == case["rejected"], name
+        for key in ("y1", "sens"):
+            a, b = np.asarray(got[key]), np.asarray(case[key])
+            assert np.max(np.abs(a - b)) <= 1e-12 * max(1.0, np.max(np.abs(b))), (name, key)
