@@ -82,11 +82,11 @@ SMS, FP64_LANES, FP32_LANES = 148, 64, 128
 # step, so a launch's traffic is this times its accepted steps.  Record kernel: 64 B of record
 # per step written plus inputs; adjoint: the 64 B entry read per step plus chunk table and inputs.
 TRAFFIC_PER_STEP = {
-    "nfw_mn": {"record": 68.3, "adjoint": 70.77},
-    "robertson": {"record": 38.9, "adjoint": 46.2},
-    "robertson_rb23": {"record": 39.8, "adjoint": 47.2},
-    "hires": {"record": 373.4, "adjoint": 99.1},          # record: spill traffic (d = 8 LU)
-    "lorenz63_vern7": {"adjoint": 46.4},                   # its record pass stays partly in L2
+    "nfw_mn": {"record": 68.3, "adjoint": 70.4},
+    "robertson": {"record": 38.9, "adjoint": 42.2},
+    "robertson_rb23": {"record": 39.8, "adjoint": 42.4},
+    "hires": {"record": 82.1, "adjoint": 88.7},
+    "lorenz63_vern7": {"adjoint": 45.2},                   # its record pass stays partly in L2
 }
 # FP64 pipe occupancy (sm__pipe_fp64_cycles_active, % of peak) of the same captures: how busy the
 # pipe is, transcendental sequences included, next to the algorithmic fraction
