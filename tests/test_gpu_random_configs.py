@@ -1,8 +1,10 @@
 """GPU parity on randomly drawn configurations (seeded): field, method, tolerances, interval and
 ensemble size vary together, and every draw must meet the fp64 bars against the oracle — counts
-identical on at least 99.9 % of trajectories, final states 1e-9, replay gradients on the GPU's
+identical on at least 99.9 % of trajectories, replay gradients on the GPU's
 own mesh 1e-8 ("gradsolve: fast exact gradients for ODE ensembles on GPUs" §3: the derivative of
-the recorded fixed-mesh chain)."""
+the recorded fixed-mesh chain), the final state against the oracle's replay of the GPU's mesh
+1e-11, and against the oracle's own adaptive solve 1e-9 or ten times the oracle's spread under a
+one-ulp change of y0, whichever is wider."""
 import numpy as np
 import pytest
 
@@ -45,7 +47,19 @@ def test_random_configuration(orc, draw):
     assert np.all(out["status"] == 0) and np.all(ref["status"] == 0)
     same = ex["S"] == ref["S"]
     assert same.mean() >= 0.999, (name, w.method, same.mean())
-    assert U.rel_rows(out["y1"][same], ref["y1"][same], w.atol).max() <= 1e-9
+    # on the GPU's own mesh the oracle's replay reproduces the GPU's final state to rounding
+    yrep = orc.replay(w.field, w.method, w.theta, w.y0, ex["H"], ex["S"],
+                      theta_shared=w.theta_shared, nthreads=8)
+    assert U.rel_rows(out["y1"], yrep, w.atol).max() <= 1e-11
+    # adaptive against adaptive: 1e-9, or ten times the oracle's own spread under a one-ulp change
+    # of y0 where that is wider (the Verner controller at loose tolerances moves step sizes by up
+    # to 1e-3 on the same count, measured; the final state moves with them)
+    spread_ref = orc.solve(w.field, w.method, w.theta, w.y0 * (1 + np.finfo(float).eps), w.t0,
+                           w.t1, w.rtol, w.atol, theta_shared=w.theta_shared, nthreads=8)
+    both = same & (spread_ref["S"] == ref["S"])
+    spread = U.rel_rows(spread_ref["y1"][both], ref["y1"][both], w.atol).max()
+    err = U.rel_rows(out["y1"][same], ref["y1"][same], w.atol).max()
+    assert err <= max(1e-9, 10 * spread), (err, spread)
     lam = rng.normal(size=(w.N, w.d))
     gy, gt = U.replay_grad(w, rec, lam)
     ry, rt = orc.replay_grad(w.field, w.method, w.theta, w.y0, ex["H"], ex["S"], lam,
