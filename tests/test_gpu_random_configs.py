@@ -3,7 +3,7 @@ ensemble size vary together, and every draw must meet the fp64 bars against the 
 identical on at least 99.9 % of trajectories, replay gradients on the GPU's
 own mesh 1e-8 ("gradsolve: fast exact gradients for ODE ensembles on GPUs" §3: the derivative of
 the recorded fixed-mesh chain), the final state against the oracle's replay of the GPU's mesh
-1e-11, and against the oracle's own adaptive solve 1e-9 or ten times the oracle's spread under a
+1e-10, and against the oracle's own adaptive solve 1e-9 or ten times the oracle's spread under a
 one-ulp change of y0, whichever is wider."""
 import numpy as np
 import pytest
@@ -50,7 +50,7 @@ def test_random_configuration(orc, draw):
     # on the GPU's own mesh the oracle's replay reproduces the GPU's final state to rounding
     yrep = orc.replay(w.field, w.method, w.theta, w.y0, ex["H"], ex["S"],
                       theta_shared=w.theta_shared, nthreads=8)
-    assert U.rel_rows(out["y1"], yrep, w.atol).max() <= 1e-11
+    assert U.rel_rows(out["y1"], yrep, w.atol).max() <= 1e-10
     # adaptive against adaptive: 1e-9, or ten times the oracle's own spread under a one-ulp change
     # of y0 where that is wider (the Verner controller at loose tolerances moves step sizes by up
     # to 1e-3 on the same count, measured; the final state moves with them)
