@@ -96,11 +96,11 @@ PIPE_BUSY_NCU = {
     "robertson_rb23": {"record": 0.342, "adjoint": 0.343},
     "hires": {"record": 0.177, "adjoint": 0.204},
     "lorenz63_vern7": {"record": 0.457, "adjoint": 0.552},
-    "log_halo": {"sens": 0.617},
+    "log_halo": {"sens": 0.710},
 }
 # forward sensitivities: DRAM bytes per trajectory (inputs and outputs; nothing per step), from
 # the ncu capture of the 2^18-orbit case
-TRAFFIC_SENS_PER_TRAJ = {"log_halo": 50.8}
+TRAFFIC_SENS_PER_TRAJ = {"log_halo": 91.1}
 # library kernels per step: record = k_solve + 2 k_max_int + 3 prefix scans of 3 kernels each
 # (step offsets, chunk offsets, length bins) + k_chunk_table + k_bin_count + k_bin_scatter (15);
 # replay gradient = k_adjoint (1).
