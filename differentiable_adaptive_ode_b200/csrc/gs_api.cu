@@ -394,11 +394,11 @@ gs_status launch_solve(const SolveCall& c) {
 }
 
 // Dynamic shared memory of the adjoint kernel: the per-lane stage tape of fields with TAPE > 0
-// (6 stages x TAPE reals x 128 lanes).
-template <class F, class R>
+// (6 stages for Tsit5, 9 for Verner 7, x TAPE reals x 128 lanes).
+template <class F, class R, int METHOD>
 constexpr size_t adjoint_smem() {
   if constexpr (std::is_same_v<F, gs::FMlpWarp>) return 0;
-  else return (size_t)6 * gs::TapeOf<F>::value * BLOCK * sizeof(R);
+  else return (size_t)(METHOD == gs::M_VERN7 ? 9 : 6) * gs::TapeOf<F>::value * BLOCK * sizeof(R);
 }
 
 struct AdjCall {
@@ -432,7 +432,7 @@ gs_status launch_adjoint(const AdjCall& c) {
   p.perm = r->perm;
   p.bounds = bounds_of(r);
   auto kern = gs::k_adjoint<F, R, METHOD>;
-  const size_t smem = adjoint_smem<F, R>();
+  const size_t smem = adjoint_smem<F, R, METHOD>();
   if (smem > 48 * 1024)
     GS_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   const int grid = persistent_grid(kern, smem, r->N);
@@ -999,7 +999,7 @@ gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_
       q.dL_dyout = static_cast<const R*>(dL_dyout);
       fill_times<R>(q.ot, rec, J, tau);
       auto kern = gs::k_adjoint_outputs<F, R, METHOD>;
-      const size_t smem = adjoint_smem<F, R>();
+      const size_t smem = adjoint_smem<F, R, METHOD>();
       if (smem > 48 * 1024)
         GS_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
       kern<<<persistent_grid(kern, smem, N), BLOCK, smem, s>>>(q);
@@ -1235,7 +1235,7 @@ gs_status noalloc_adjoint(const gs_record* r, const void* theta, const void* dL_
     p.perm = r->perm;
     p.bounds = bounds_of(r);
     auto kern = gs::k_adjoint<F, R, METHOD>;
-    const size_t smem = adjoint_smem<F, R>();
+    const size_t smem = adjoint_smem<F, R, METHOD>();
     int nb = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, BLOCK, smem) != cudaSuccess || nb < 1)
       nb = 1;

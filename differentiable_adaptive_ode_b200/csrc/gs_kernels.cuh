@@ -654,7 +654,7 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
 #pragma unroll
         for (int c = 0; c < D; ++c) y[c] = __ldg(e + 2 + c);
         if constexpr (METHOD == M_TSIT5) tsit5_adjoint_step<F, R>(y, h, th, lam, thb, tape, blockDim.x);
-        else if constexpr (METHOD == M_VERN7) vern7_adjoint_step<F, R>(y, h, th, lam, thb);
+        else if constexpr (METHOD == M_VERN7) vern7_adjoint_step<F, R>(y, h, th, lam, thb, tape, blockDim.x);
         else if constexpr (METHOD == M_RB23) rb23_adjoint_step<F, R>(y, h, th, lam, thb);
         else ros_adjoint_step<F, R>(y, h, th, lam, thb);
         --n;
@@ -905,7 +905,7 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
 #pragma unroll
         for (int c = 0; c < D; ++c) lr[c] = r >= jlo ? lo[(size_t)r * D + c] : lam[c];
         if constexpr (METHOD == M_TSIT5) tsit5_adjoint_step<F, R>(y, hr, th, lr, thb, tape, blockDim.x);
-        else if constexpr (METHOD == M_VERN7) vern7_adjoint_step<F, R>(y, hr, th, lr, thb);
+        else if constexpr (METHOD == M_VERN7) vern7_adjoint_step<F, R>(y, hr, th, lr, thb, tape, blockDim.x);
         else if constexpr (METHOD == M_RB23) rb23_adjoint_step<F, R>(y, hr, th, lr, thb);
         else ros_adjoint_step<F, R>(y, hr, th, lr, thb);
 #pragma unroll

@@ -276,6 +276,13 @@ __device__ __forceinline__ void tsit5_replay_step(const R (&y)[F::D], R h,
   }
 }
 
+// TAPE of a field: how many transcendental intermediates of f one stage keeps for its VJP
+// (0 when the field declares none).
+template <class F, class = void> struct TapeOf { static constexpr int value = 0; };
+template <class F> struct TapeOf<F, std::void_t<decltype(F::TAPE)>> {
+  static constexpr int value = F::TAPE;
+};
+
 // ----------------------------------------------------------------------------------------------
 // Verner 7 one-step maps.  Stage states Y_i = y + h sum_{j<i} a_ij k_j, k_i = f(Y_i).
 // ----------------------------------------------------------------------------------------------
@@ -355,17 +362,28 @@ __device__ __forceinline__ void vern7_replay_step(const R (&y)[F::D], R h,
 // nine stages): recompute the stage states from the recorded y_n, then for i = 9..1
 //   kb_i = h (b_i lam + G_i),  Yb_i = J_y(Y_i)^T kb_i,  thb += J_th(Y_i)^T kb_i,
 //   G_j += a_ij Yb_i (j < i),   and finally lam <- lam + sum_i Yb_i.
+// Fields that declare TAPE > 0 keep the transcendental part of f at each of the nine stages in
+// the per-lane shared-memory tape (slot (i, v) at tape[(i * TAPE + v) * tstride]) for the VJPs.
 template <class F, class R>
 __device__ __forceinline__ void vern7_adjoint_step(const R (&y)[F::D], R h,
                                                    const typename F::template Theta<R>& th,
-                                                   R (&lam)[F::D], R (&thb)[F::M]) {
+                                                   R (&lam)[F::D], R (&thb)[F::M],
+                                                   R* tape = nullptr, int tstride = 0) {
   constexpr int D = F::D;
+  constexpr int TP = TapeOf<F>::value;
   R Y[9][D];
   {
     R k[10][D];
 #pragma unroll
     for (int c = 0; c < D; ++c) Y[0][c] = y[c];
-    F::f(y, th, k[0]);
+    if constexpr (TP > 0) {
+      R tp[TP > 0 ? TP : 1];
+      F::f_tape(Y[0], th, k[0], tp);
+#pragma unroll
+      for (int v = 0; v < TP; ++v) tape[v * tstride] = tp[v];
+    } else {
+      F::f(y, th, k[0]);
+    }
 #pragma unroll
     for (int i = 1; i < 9; ++i) {
 #pragma unroll
@@ -376,7 +394,15 @@ __device__ __forceinline__ void vern7_adjoint_step(const R (&y)[F::D], R h,
           if (vern7_a(i, j) != 0.0) s += R(vern7_a(i, j)) * k[j][c];
         Y[i][c] = y[c] + h * s;
       }
-      if (i < 8) F::f(Y[i], th, k[i]);
+      if constexpr (TP > 0) {
+        R tp[TP > 0 ? TP : 1];
+        if (i < 8) F::f_tape(Y[i], th, k[i], tp);
+        else F::inter_tape(Y[i], th, tp);
+#pragma unroll
+        for (int v = 0; v < TP; ++v) tape[(i * TP + v) * tstride] = tp[v];
+      } else {
+        if (i < 8) F::f(Y[i], th, k[i]);
+      }
     }
   }
   R G[8][D], dl[D];
@@ -395,7 +421,14 @@ __device__ __forceinline__ void vern7_adjoint_step(const R (&y)[F::D], R h,
       if (i < 8) s += G[i][c];
       kb[c] = h * s;
     }
-    F::vjp(Y[i], th, kb, Yb, thb);
+    if constexpr (TP > 0) {
+      R tp[TP > 0 ? TP : 1];
+#pragma unroll
+      for (int v = 0; v < TP; ++v) tp[v] = tape[(i * TP + v) * tstride];
+      F::vjp_tape(Y[i], th, tp, kb, Yb, thb);
+    } else {
+      F::vjp(Y[i], th, kb, Yb, thb);
+    }
 #pragma unroll
     for (int c = 0; c < D; ++c) {
       dl[c] += Yb[c];
@@ -456,10 +489,6 @@ __device__ __forceinline__ void tsit5_tangent_step(const R (&y)[F::D], R h,
 //   lam <- lam + sum_i Yb_i.   (b_7 = 0, so the seventh stage never enters the replay map.)
 // Fields that declare TAPE > 0 hand the reverse sweep the transcendental part of f at each stage
 // (kept in a per-lane shared-memory tape) instead of recomputing it in the VJP.
-template <class F, class = void> struct TapeOf { static constexpr int value = 0; };
-template <class F> struct TapeOf<F, std::void_t<decltype(F::TAPE)>> {
-  static constexpr int value = F::TAPE;
-};
 
 // tape: this lane's slot 0; slot (i, v) at tape[(i * TAPE + v) * tstride] (shared memory).
 template <class F, class R>
