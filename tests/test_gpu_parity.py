@@ -165,7 +165,7 @@ def test_gradient_on_imported_oracle_record(orc, name, N):
     assert U.rel_rows(gt, rt, 1e-300).max() <= 1e-8
 
 
-@pytest.mark.parametrize("method", ["tsit5", "ros34pw2"])
+@pytest.mark.parametrize("method", ["tsit5", "ros34pw2", "vern7", "rosenbrock23"])
 def test_linear_field_both_methods(orc, method):
     rng = np.random.default_rng(9)
     N = 160
@@ -203,11 +203,12 @@ def test_shared_theta_reduction(orc, name):
     assert np.array_equal(gt, gt2) and np.array_equal(gy, gy2)
 
 
-def test_gradient_at_other_theta_on_fixed_mesh(orc):
+@pytest.mark.parametrize("name", ["lorenz63", "lorenz63_vern7", "robertson_rb23"])
+def test_gradient_at_other_theta_on_fixed_mesh(orc, name):
     # one record made at theta0 serves a gradient at theta on the same mesh ([GS] §3: the
     # derivative of Psi(theta; sg[R(theta0)])): forward replay at theta, then the backward sweep
     import torch
-    w = U.small("lorenz63", 200)
+    w = U.small(name, 200)
     rec, out = U.record(w)
     ex = U.export_padded(w, rec)
     th2 = w.theta * 1.01
