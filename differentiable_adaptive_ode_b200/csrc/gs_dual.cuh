@@ -19,6 +19,35 @@
 
 namespace gs {
 
+// log(1 + x) for x > -1, given a and b with a * b = 1 / (1 + x) to a few ulps (a reciprocal that
+// the caller has at hand).  fp64: w = fl(1 + x) and its rounding error c, 1 + x = w + c exactly
+// (Knuth's TwoSum, branch-free); then log(1 + x) = log(w) + c / w up to (c / w)^2 <= 2^-106, and
+// 1 / w = a * b to a few ulps suffices for the small correction.  The result stays within about
+// 2 ulps (CUDA's log is within 1) at the cost of one log, six adds and a multiply-add, with no
+// division.  The sums are rounded one by one on the device, which the exactness of c needs; a
+// caller whose x is a product forms it with mul_rn, so that no kernel fuses that product into
+// the sums (the forward-only and recording solvers then stay bit-for-bit alike).  fp32 keeps
+// log1pf.
+GS_DHD double log1p_q(double x, double a, double b) {
+#ifdef __CUDA_ARCH__
+  const double w = __dadd_rn(1.0, x);
+  const double xv = __dsub_rn(w, 1.0);
+  const double c = __dadd_rn(__dsub_rn(1.0, __dsub_rn(w, xv)), __dsub_rn(x, xv));
+#else
+  const double w = 1.0 + x;
+  const double xv = w - 1.0;
+  const double c = (1.0 - (w - xv)) + (x - xv);
+#endif
+  return fma(c, a * b, log(w));
+}
+GS_DHD float log1p_q(float x, float, float) { return log1pf(x); }
+
+// a * b rounded on its own: in fp64 on the device the product is never fused into a later sum.
+template <class R> GS_DHD R mul_rn(R a, R b) { return a * b; }
+#ifdef __CUDA_ARCH__
+template <> GS_DHD double mul_rn<double>(double a, double b) { return __dmul_rn(a, b); }
+#endif
+
 template <class R>
 struct Dl {
   R v, d;
@@ -54,6 +83,11 @@ struct Dl {
   friend GS_DHD Dl sqrt(const Dl& a) {
     const R s = sqrt(a.v);
     return Dl(s, R(0.5) * a.d / s);
+  }
+  // d log(1 + x) = dx / (1 + x) = dx * (p * q) when p * q = 1 / (1 + x)
+  friend GS_DHD Dl log1p_q(const Dl& x, const Dl& p, const Dl& q) {
+    const R iw = p.v * q.v;
+    return Dl(log1p_q(x.v, p.v, q.v), x.d * iw);
   }
   friend GS_DHD Dl log1p(const Dl& a) {
     return Dl(log1p(a.v), a.d / (R(1) + a.v));

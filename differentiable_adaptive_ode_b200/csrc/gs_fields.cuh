@@ -26,6 +26,7 @@
 inline double rsqrt(double x) { return 1.0 / std::sqrt(x); }
 inline float rsqrt(float x) { return 1.0f / std::sqrt(x); }
 #endif
+#include "gs_dual.cuh"
 
 namespace gs {
 
@@ -281,8 +282,8 @@ struct FNfwMiyamotoNagai {
     const R r2 = I.R2 + z * z;
     I.ir = rsqrt(r2);
     I.r = r2 * I.ir;
-    I.L = log1p(I.r * t.irs);
     I.isr = R(1) / (t.rs + I.r);
+    I.L = log1p_q(mul_rn(I.r, t.irs), t.rs, I.isr);  // rs / (rs + r) = 1 / (1 + r / rs)
     I.gN = t.Mh * (I.ir * I.ir) * (I.L * I.ir - I.isr);
     const R B2 = z * z + t.b2;
     I.iB = rsqrt(B2);

@@ -26,6 +26,8 @@ inline Cnt operator*(Cnt a, Cnt b) { T.mul++; return Cnt(a.v * b.v); }
 inline Cnt operator/(Cnt a, Cnt b) { T.div++; return Cnt(a.v / b.v); }
 inline Cnt sqrt(Cnt a) { T.sqrt++; return Cnt(std::sqrt(a.v)); }
 inline Cnt log1p(Cnt a) { T.log1p++; return Cnt(std::log1p(a.v)); }
+// the fields' log1p evaluation given a reciprocal of 1 + x (log1p_q) is one log1p of the formula
+inline Cnt log1p_q(Cnt a, Cnt, Cnt) { T.log1p++; return Cnt(std::log1p(a.v)); }
 inline Cnt rsqrt(Cnt a) { T.sqrt++; return Cnt(1.0 / std::sqrt(a.v)); }
 inline Cnt fma(Cnt a, Cnt b, Cnt c) { T.mul++; T.add++; return Cnt(a.v * b.v + c.v); }
 
