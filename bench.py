@@ -82,7 +82,7 @@ SMS, FP64_LANES, FP32_LANES = 148, 64, 128
 # step, so a launch's traffic is this times its accepted steps.  Record kernel: 64 B of record
 # per step written plus inputs; adjoint: the 64 B entry read per step plus chunk table and inputs.
 TRAFFIC_PER_STEP = {
-    "nfw_mn": {"record": 68.5, "adjoint": 70.4},
+    "nfw_mn": {"record": 68.5, "adjoint": 70.7},
     "robertson": {"record": 38.9, "adjoint": 42.2},
     "robertson_rb23": {"record": 39.8, "adjoint": 42.4},
     "hires": {"record": 82.1, "adjoint": 88.7},
@@ -91,7 +91,7 @@ TRAFFIC_PER_STEP = {
 # FP64 pipe occupancy (sm__pipe_fp64_cycles_active, % of peak) of the same captures: how busy the
 # pipe is, transcendental sequences included, next to the algorithmic fraction
 PIPE_BUSY_NCU = {
-    "nfw_mn": {"record": 0.457, "adjoint": 0.570},
+    "nfw_mn": {"record": 0.465, "adjoint": 0.631},
     "robertson": {"record": 0.415, "adjoint": 0.354},
     "robertson_rb23": {"record": 0.342, "adjoint": 0.343},
     "hires": {"record": 0.177, "adjoint": 0.204},
