@@ -184,6 +184,12 @@ template <class R> struct Roll<FNfwMiyamotoNagai, R> { static constexpr bool val
 template <> struct Tune<FNfwMiyamotoNagai, double> {
   static constexpr int adj_blocks = 3, solve_blocks = 3;
 };
+// fp32: the reverse sweep at 4 blocks/SM (128 registers, from 141) 1.60 -> 1.45 ms at 2^20; the
+// solve kernels (112 registers, 4 blocks already) lose at 5 (2.91 -> 3.02 ms record), and 4
+// blocks of the fp64 kernels (spilling) lose too (record 20.4 -> 24.4, adjoint 13.6 -> 15.0).
+template <> struct Tune<FNfwMiyamotoNagai, float> {
+  static constexpr int adj_blocks = 4, solve_blocks = 1;
+};
 // The forward-sensitivity solve of the logarithmic halo in double precision: 3 blocks/SM
 // (168 registers) against 2 unconstrained (228): 31.5 -> 28.7 ms at 2^20 orbits.
 template <> struct Tune<FLogHalo, double> {
