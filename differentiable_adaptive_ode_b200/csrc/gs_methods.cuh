@@ -599,9 +599,13 @@ template <class R> __device__ __forceinline__ R rbe(int i) {
 
 // In-register LU of a D x D matrix with partial pivoting (largest |entry|, ties to the lowest
 // row).  The permutation is kept as a row map p[] so that solves index without data movement.
+// The pivots' reciprocals are formed once (the factorisation needs them anyway) and every solve
+// multiplies by them: a Rosenbrock step solves three or four times with one factorisation, and
+// an fp64 division costs several times a multiply on the FP64 pipe.
 template <class R, int D>
 struct SmallLU {
   R lu[D][D];
+  R dinv[D];  // reciprocals of U's diagonal, formed once by factor(): the solves multiply
   int p[D];
   __device__ __forceinline__ void factor(const R (&A)[D][D]) {
 #pragma unroll
@@ -622,6 +626,7 @@ struct SmallLU {
         }
       }
       const R inv = R(1) / lu[col][col];
+      dinv[col] = inv;
 #pragma unroll
       for (int r = col + 1; r < D; ++r) {
         const R l = lu[r][col] * inv;
@@ -648,7 +653,7 @@ struct SmallLU {
     for (int r = D - 1; r >= 0; --r) {
 #pragma unroll
       for (int c = r + 1; c < D; ++c) x[r] -= lu[r][c] * x[c];
-      x[r] = x[r] / lu[r][r];
+      x[r] = x[r] * dinv[r];
     }
   }
   // x = A^{-T} b:  A^T = U^T L^T P, so solve U^T z = b, L^T w = z, x = P^T w.
@@ -659,7 +664,7 @@ struct SmallLU {
       R v = bb[r];
 #pragma unroll
       for (int c = 0; c < r; ++c) v -= lu[c][r] * z[c];
-      z[r] = v / lu[r][r];
+      z[r] = v * dinv[r];
     }
 #pragma unroll
     for (int r = D - 1; r >= 0; --r)
