@@ -83,18 +83,18 @@ SMS, FP64_LANES, FP32_LANES = 148, 64, 128
 # per step written plus inputs; adjoint: the 64 B entry read per step plus chunk table and inputs.
 TRAFFIC_PER_STEP = {
     "nfw_mn": {"record": 68.5, "adjoint": 70.7},
-    "robertson": {"record": 38.9, "adjoint": 42.2},
-    "robertson_rb23": {"record": 39.8, "adjoint": 42.4},
-    "hires": {"record": 82.1, "adjoint": 88.7},
+    "robertson": {"record": 38.9, "adjoint": 42.4},
+    "robertson_rb23": {"record": 39.8, "adjoint": 47.1},
+    "hires": {"record": 83.1, "adjoint": 89.4},
     "lorenz63_vern7": {"adjoint": 45.2},                   # its record pass stays partly in L2
 }
 # FP64 pipe occupancy (sm__pipe_fp64_cycles_active, % of peak) of the same captures: how busy the
 # pipe is, transcendental sequences included, next to the algorithmic fraction
 PIPE_BUSY_NCU = {
     "nfw_mn": {"record": 0.465, "adjoint": 0.631},
-    "robertson": {"record": 0.415, "adjoint": 0.354},
-    "robertson_rb23": {"record": 0.342, "adjoint": 0.343},
-    "hires": {"record": 0.177, "adjoint": 0.204},
+    "robertson": {"record": 0.416, "adjoint": 0.427},
+    "robertson_rb23": {"record": 0.328, "adjoint": 0.387},
+    "hires": {"record": 0.196, "adjoint": 0.217},
     "lorenz63_vern7": {"record": 0.457, "adjoint": 0.552},
     "log_halo": {"sens": 0.710},
 }
