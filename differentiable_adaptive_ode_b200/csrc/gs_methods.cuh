@@ -15,6 +15,56 @@
 
 namespace gs {
 
+// The step's scaled RMS error sqrt(mean_c (e_c / sc_c)^2) (the accept test of an embedded pair).
+template <class R, int D>
+__device__ __forceinline__ R scaled_rms(const R (&e)[D], const R (&sc)[D]) {
+  R s2 = R(0);
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    const R q = e[c] / sc[c];
+    s2 = fma(q, q, s2);
+  }
+  return sqrt(s2 / R(D));
+}
+// fp64: the D reciprocals 1/sc_c from ONE division by Montgomery's simultaneous inversion
+// (P. L. Montgomery, "Speeding the Pollard and elliptic curve methods of factorization", Math.
+// Comp. 48, 1987): prefix products P_c = sc_0 ... sc_c, one reciprocal of P_{D-1}, then backwards
+// 1/sc_c = P_{c-1} / P_c and 1/P_{c-1} = sc_c / P_c.  Each reciprocal carries at most about 3D
+// roundings (below 1e-14 relative for D <= 8), far below what the step control resolves.  Where
+// a prefix product leaves the normal range (scales near 0 or huge, non-finite values) the step
+// takes the per-component divisions instead, so those cases behave exactly as before.
+template <int D>
+__device__ __forceinline__ double scaled_rms(const double (&e)[D], const double (&sc)[D]) {
+  constexpr double lo = 2.2250738585072014e-308, hi = 1.7976931348623157e308;  // normal range
+  double P[D];
+  P[0] = sc[0];
+  bool ok = (P[0] >= lo) && (P[0] <= hi);
+#pragma unroll
+  for (int c = 1; c < D; ++c) {
+    P[c] = P[c - 1] * sc[c];
+    ok = ok && (P[c] >= lo) && (P[c] <= hi);
+  }
+  double s2 = 0.0;
+  if (ok) {
+    double inv = 1.0 / P[D - 1];
+#pragma unroll
+    for (int c = D - 1; c > 0; --c) {
+      const double q = e[c] * (inv * P[c - 1]);
+      inv = inv * sc[c];
+      s2 = fma(q, q, s2);
+    }
+    const double q0 = e[0] * inv;
+    s2 = fma(q0, q0, s2);
+  } else {
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+      const double q = e[c] / sc[c];
+      s2 = fma(q, q, s2);
+    }
+  }
+  return sqrt(s2 * (1.0 / D));
+}
+
 struct Tsit5 {
   static constexpr int order = 5, err_order = 5;
   // a_ij, i = 2..7, j < i; row 7 equals b (b_7 = 0).
@@ -190,15 +240,13 @@ __device__ __forceinline__ R tsit5_trial_rolled(const R (&y)[F::D], R h,
       for (int c = 0; c < D; ++c) acc[m][c] = fma(hc, kk[c], acc[m + 1][c]);
     }
   }
-  R s2 = R(0);
+  R ev[D], sc[D];
 #pragma unroll
   for (int c = 0; c < D; ++c) {
-    const R e = h * er[c];
-    const R sc = fma(rtol, fmax(fabs(y[c]), fabs(ynew[c])), atol);
-    const R q = e / sc;
-    s2 = fma(q, q, s2);
+    ev[c] = h * er[c];
+    sc[c] = fma(rtol, fmax(fabs(y[c]), fabs(ynew[c])), atol);
   }
-  return sqrt(s2 / R(D));
+  return scaled_rms(ev, sc);
 }
 
 // One Tsit5 trial from y with step h; k1 = f(y) is carried (first-same-as-last).  Produces the
@@ -232,7 +280,7 @@ __device__ __forceinline__ R tsit5_trial(const R (&y)[F::D], R h, const typename
     ynew[c] = y[c] + h * s;
   }
   F::f(ynew, th, k7);
-  R acc = R(0);
+  R ev[D], sc[D];
 #pragma unroll
   for (int c = 0; c < D; ++c) {
     R s = te<R>(0) * k[0][c];
@@ -240,11 +288,10 @@ __device__ __forceinline__ R tsit5_trial(const R (&y)[F::D], R h, const typename
     for (int j = 1; j < 6; ++j) s += te<R>(j) * k[j][c];
     s += te<R>(6) * k7[c];
     const R e = h * s;
-    const R sc = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
-    const R q = e / sc;
-    acc += q * q;
+    ev[c] = e;
+    sc[c] = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
   }
-  return sqrt(acc / R(D));
+  return scaled_rms(ev, sc);
 }
 
 // The Tsit5 replay map Phi(y, h) = y + h sum_{i<=6} b_i k_i with k_1 = f(y) (no error estimate).
@@ -319,7 +366,7 @@ __device__ __forceinline__ R vern7_trial(const R (&y)[F::D], R h,
 #pragma unroll
   for (int c = 0; c < D; ++c) k[0][c] = k1[c];
   vern7_stages<F, R, 10>(y, h, th, k);
-  R acc = R(0);
+  R ev[D], sc[D];
 #pragma unroll
   for (int c = 0; c < D; ++c) {
     R s = R(vern7_b(0)) * k[0][c];
@@ -332,11 +379,10 @@ __device__ __forceinline__ R vern7_trial(const R (&y)[F::D], R h,
     for (int j = 1; j < 10; ++j)
       if (vern7_e(j) != 0.0) es += R(vern7_e(j)) * k[j][c];
     const R e = h * es;
-    const R sc = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
-    const R q = e / sc;
-    acc += q * q;
+    ev[c] = e;
+    sc[c] = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
   }
-  return sqrt(acc / R(D));
+  return scaled_rms(ev, sc);
 }
 
 // The Verner 7 replay map Phi(y, h) = y + h sum_{i<=9} b_i k_i with k_1 = f(y).
@@ -737,7 +783,7 @@ __device__ __forceinline__ R ros_trial(const R (&y)[F::D], R h,
   ros_matrix<F, R>(y, h, th, J, lu);
   R k[4][D];
   ros_stages<F, R>(y, h, th, J, lu, k);
-  R acc = R(0);
+  R ev[D], sc[D];
 #pragma unroll
   for (int c = 0; c < D; ++c) {
     R s = rb<R>(0) * k[0][c];
@@ -748,11 +794,10 @@ __device__ __forceinline__ R ros_trial(const R (&y)[F::D], R h,
       e += rbe<R>(i) * k[i][c];
     }
     ynew[c] = y[c] + s;
-    const R sc = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
-    const R q = e / sc;
-    acc += q * q;
+    ev[c] = e;
+    sc[c] = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
   }
-  return sqrt(acc / R(D));
+  return scaled_rms(ev, sc);
 }
 
 // The ROS34PW2 replay map (no error estimate).
@@ -845,15 +890,14 @@ __device__ __forceinline__ R rb23_trial(const R (&y)[F::D], R h,
   for (int c = 0; c < D; ++c)
     r[c] = F2[c] - R(Rb23::e32) * (k2[c] - F1[c]) - R(2) * (k1[c] - F0[c]);
   lu.solve(r, k3);
-  R acc = R(0);
+  R ev[D], sc[D];
 #pragma unroll
   for (int c = 0; c < D; ++c) {
-    const R e = h * (k1[c] - R(2) * k2[c] + k3[c]) / R(6);
-    const R sc = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
-    const R q = e / sc;
-    acc += q * q;
+    const R e = h * (k1[c] - R(2) * k2[c] + k3[c]) * R(1.0 / 6.0);
+    ev[c] = e;
+    sc[c] = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
   }
-  return sqrt(acc / R(D));
+  return scaled_rms(ev, sc);
 }
 
 // The Rosenbrock23 replay map y + h k2 (no error estimate).
