@@ -81,8 +81,11 @@ SMS, FP64_LANES, FP32_LANES = 148, 64, 128
 # 2^18-trajectory case of this workload; both kernels move a fixed number of bytes per accepted
 # step, so a launch's traffic is this times its accepted steps.  Record kernel: 64 B of record
 # per step written plus inputs; adjoint: the 64 B entry read per step plus chunk table and inputs.
+# The stellar record and adjoint figures were captured after the last change to those kernels;
+# the other workloads' record and sensitivity figures precede the one-division error norm, a
+# change of arithmetic only that leaves the bytes each step moves (its record entry) as they were.
 TRAFFIC_PER_STEP = {
-    "nfw_mn": {"record": 68.5, "adjoint": 70.7},
+    "nfw_mn": {"record": 68.4, "adjoint": 70.7},
     "robertson": {"record": 38.9, "adjoint": 42.4},
     "robertson_rb23": {"record": 39.8, "adjoint": 47.1},
     "hires": {"record": 83.1, "adjoint": 89.4},
@@ -91,7 +94,7 @@ TRAFFIC_PER_STEP = {
 # FP64 pipe occupancy (sm__pipe_fp64_cycles_active, % of peak) of the same captures: how busy the
 # pipe is, transcendental sequences included, next to the algorithmic fraction
 PIPE_BUSY_NCU = {
-    "nfw_mn": {"record": 0.465, "adjoint": 0.631},
+    "nfw_mn": {"record": 0.493, "adjoint": 0.631},
     "robertson": {"record": 0.416, "adjoint": 0.427},
     "robertson_rb23": {"record": 0.328, "adjoint": 0.387},
     "hires": {"record": 0.196, "adjoint": 0.217},
