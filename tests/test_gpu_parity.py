@@ -184,6 +184,33 @@ def test_linear_field_both_methods(orc, method):
     assert U.rel_rows(gt, rt, 1e-300).max() <= 1e-8
 
 
+@pytest.mark.parametrize("method", ["tsit5", "rosenbrock23"])
+def test_linear_decay_to_tiny_error_scales(orc, method):
+    """States decaying to ~1e-195 with atol = 1e-300: the error scales atol + rtol |y| fall to
+    ~1e-200, so the products of the scales that give the error norm's reciprocals from one
+    division underflow part way through every trajectory, and the solver takes the per-component
+    divisions from there on.  Both stretches must match the oracle (plain divisions throughout)."""
+    rng = np.random.default_rng(19)
+    N = 64
+    # eigenvalues within about -1.5 +- 0.1: |y(300)| between ~1e-210 and ~1e-180 (no subnormals);
+    # the one-division form holds while the scales stay above ~1e-103 (t below ~150) and gives
+    # way to the per-component divisions from about t = 150 to 230 on
+    A = rng.normal(size=(N, 3, 3)) * 0.05 - 1.5 * np.eye(3)[None]
+    y0 = rng.normal(size=(N, 3))
+    w = W.Workload("linear3", "linear3", method, np.float64, N, 3, 9, False, A.reshape(N, 9), y0,
+                   0.0, 300.0, 1e-6, 1e-300, 0)
+    rec, out = U.record(w)
+    ex = U.export_padded(w, rec)
+    ref = _oracle_solve(orc, w)
+    assert np.all(np.abs(out["y1"]).max(axis=1) < 1e-150)     # the scales did leave the range
+    _check_states(w, dict(S=ex["S"], y1=out["y1"]), ref)
+    lam = rng.normal(size=(N, 3))
+    gy, gt = U.replay_grad(w, rec, lam)
+    ry, rt = orc.replay_grad("linear3", method, w.theta, w.y0, ex["H"], ex["S"], lam)
+    assert U.rel_rows(gy, ry, 1e-300).max() <= 1e-8
+    assert U.rel_rows(gt, rt, 1e-300).max() <= 1e-8
+
+
 @pytest.mark.parametrize("name", ["nfw_mn", "lotka_volterra"])
 def test_shared_theta_reduction(orc, name):
     w = U.small(name, 700)
