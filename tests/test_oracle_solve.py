@@ -220,3 +220,78 @@ def test_fp32_solve_tracks_fp64(orc):
     assert np.all(r32["status"] == 0)
     err = np.max(np.abs(r32["y1"] - r64["y1"]), axis=1) / np.max(np.abs(r64["y1"]), axis=1)
     assert np.median(err) < 1e-3
+
+
+def _rk_poly(z, A, v):
+    """1 + sum_q z^q v^T A^(q-1) 1: what the weights v of an explicit RK method give on y' = z y
+    over one step (z = h lambda); with v = b - b_hat, 1 + the error estimate's factor."""
+    s, u = 1.0, np.ones(A.shape[0])
+    for q in range(1, A.shape[0] + 1):
+        s += z ** q * (v @ u)
+        u = A @ u
+    return s
+
+
+def _scalar_step(method, orc):
+    """(R, E)(h, lam): step factor and error-estimate factor of one step on y' = lam y, y = 1."""
+    if method == "tsit5":
+        c, A, b, bt = orc.tsit5_tableau()
+        return lambda h, lam: (_rk_poly(h * lam, A, b), _rk_poly(h * lam, A, bt) - 1.0)
+    if method == "vern7":
+        A, b, bh = orc.vern7_tableau()
+        return lambda h, lam: (_rk_poly(h * lam, A, b), _rk_poly(h * lam, A, b - bh) - 1.0)
+    if method == "ros34pw2":
+        g, al, ga, b, bh = orc.ros34pw2_tableau()
+        beta = al + ga
+
+        def ros(h, lam):
+            z, K = h * lam, []
+            for i in range(4):                  # (1 - g z) K_i = z (1 + sum_j beta_ij K_j)
+                K.append(z / (1 - g * z) * (1 + sum(beta[i, j] * K[j] for j in range(i))))
+            return 1 + sum(b[i] * K[i] for i in range(4)), sum((b[i] - bh[i]) * K[i] for i in range(4))
+        return ros
+    # Rosenbrock23 (Shampine & Reichelt): W = 1 - d h lam, slopes k1, k2, k3, e = h (k1 - 2k2 + k3)/6
+    d, e32 = 1 / (2 + np.sqrt(2)), 6 + np.sqrt(2)
+
+    def rb23(h, lam):
+        W = 1 - d * h * lam
+        F0 = lam
+        k1 = F0 / W
+        F1 = lam * (1 + h * k1 / 2)
+        k2 = (F1 - k1) / W + k1
+        y1 = 1 + h * k2
+        k3 = (lam * y1 - e32 * (k2 - F1) - 2 * (k1 - F0)) / W
+        return y1, h * (k1 - 2 * k2 + k3) / 6
+    return rb23
+
+
+@pytest.mark.parametrize("method,q", [("tsit5", 5), ("vern7", 7), ("ros34pw2", 3),
+                                      ("rosenbrock23", 3)])
+def test_controller_settles_at_its_fixed_point(orc, method, q):
+    # On y' = lam y with a pure relative tolerance the scaled error of a step depends on h alone:
+    # err(h) = |E(h lam)| / (rtol max(1, |R(h lam)|)).  The I-controller h <- 0.9 err^(-1/q) h
+    # therefore settles where 0.9 err^(-1/q) = 1, i.e. err(h*) = 0.9^q; h* is found here by
+    # bisection on the closed-form factors, independently of the solver's loop.  A wrong safety
+    # factor, exponent or error norm moves the recorded steps off h*.
+    lam, rtol = -1.0, 1e-6 if method != "vern7" else 1e-8
+    step = _scalar_step(method, orc)
+    r = orc.solve("linear1", method, [[lam]], [[1.0]], 0.0, 40.0, rtol, 1e-300, keep_record=True)
+    S = int(r["S"][0])
+    H = r["H"][0, :S]
+    assert r["status"][0] == 0 and r["rejected"][0] == 0 and S > 100
+
+    def err(h):
+        R, E = step(h, lam)
+        return abs(E) / (rtol * max(1.0, abs(R)))
+    lo, hi = 1e-9, 4 * H.max()
+    assert err(lo) < 0.9 ** q < err(hi)
+    for _ in range(200):
+        mid = 0.5 * (lo + hi)
+        lo, hi = (mid, hi) if err(mid) < 0.9 ** q else (lo, mid)
+    h_star = 0.5 * (lo + hi)
+    settled = H[S // 2:S - 1]               # past the start-up, before the step clipped to t1
+    assert np.max(np.abs(settled - h_star)) <= 1e-7 * h_star, (h_star, settled[:3])
+    # and the start-up grows the step by at most the factor cap of 10 per accepted step
+    assert np.all(H[1:S - 1] <= 10 * H[:S - 2] * (1 + 1e-12))
+    if method == "rosenbrock23":            # a tiny first step: the cap itself is reached
+        assert abs(H[1] / H[0] - 10.0) < 1e-12
