@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <initializer_list>
 #include <atomic>
 #include <mutex>
 #include <new>
@@ -537,6 +538,33 @@ gs_status check_common(const gs_system* sys, int64_t N, const void* theta, const
   return GS_OK;
 }
 
+// The caller's arrays must be readable by this device's kernels: plain (unregistered) host memory,
+// or another device's memory, would make a kernel fault instead of returning an error.  Only a
+// positive identification rejects a pointer (device, managed and page-locked host memory pass;
+// when the runtime cannot tell, the pointer passes too).
+struct NamedPtr { const void* p; const char* name; };
+gs_status check_device(std::initializer_list<NamedPtr> ptrs) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return GS_OK;
+  }
+  for (const NamedPtr& a : ptrs) {
+    if (!a.p) continue;
+    cudaPointerAttributes at{};
+    if (cudaPointerGetAttributes(&at, a.p) != cudaSuccess) {
+      cudaGetLastError();
+      continue;
+    }
+    if (at.type == cudaMemoryTypeUnregistered)
+      return fail(GS_ERR_INVALID_ARG, "%s is host memory: a device pointer is required", a.name);
+    if (at.type == cudaMemoryTypeDevice && at.device != dev)
+      return fail(GS_ERR_INVALID_ARG, "%s is memory of device %d, the current device is %d",
+                  a.name, at.device, dev);
+  }
+  return GS_OK;
+}
+
 long long attempts_of(const gs_options* opt) {
   return (opt && opt->max_attempts > 0) ? (long long)opt->max_attempts : 100000LL;
 }
@@ -601,6 +629,10 @@ gs_status gs_solve_forward(const gs_system* sys, const gs_options* opt, int64_t 
   gs_status st = check_common(sys, N, theta, y0, t0, t1, rtol, atol, y1);
   if (st != GS_OK) return st;
   if (N == 0) return GS_OK;
+  st = check_device({{theta, "theta"}, {y0, "y0"}, {y1, "y1"}, {nsteps, "nsteps"},
+                     {nrejected, "nrejected"}, {status, "status"},
+                     {opt ? opt->start_order : nullptr, "start_order"}});
+  if (st != GS_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* queue = nullptr;
   GS_CUDA(take_counter(s, &queue));
@@ -623,6 +655,10 @@ gs_status gs_solve_forward_sens(const gs_system* sys, const gs_options* opt, int
                 "forward sensitivities are built for the Tsit5 fields other than the MLP");
   if (N > 0 && !S1) return fail(GS_ERR_INVALID_ARG, "S1 must be non-NULL");
   if (N == 0) return GS_OK;
+  st = check_device({{theta, "theta"}, {y0, "y0"}, {S0, "S0"}, {y1, "y1"}, {S1, "S1"},
+                     {nsteps, "nsteps"}, {nrejected, "nrejected"}, {status, "status"},
+                     {opt ? opt->start_order : nullptr, "start_order"}});
+  if (st != GS_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* queue = nullptr;
   GS_CUDA(take_counter(s, &queue));
@@ -639,6 +675,11 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
   gs_status st = check_common(sys, N, theta, y0, t0, t1, rtol, atol, y1);
   if (st != GS_OK) return st;
   if (!rec) return fail(GS_ERR_INVALID_ARG, "rec must be non-NULL");
+  if (N > 0) {
+    st = check_device({{theta, "theta"}, {y0, "y0"}, {y1, "y1"}, {status, "status"},
+                       {opt ? opt->start_order : nullptr, "start_order"}});
+    if (st != GS_OK) return st;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   gs_record* r = *rec;
   bool fresh = false;
@@ -765,6 +806,9 @@ gs_status gs_replay_grad(const gs_record* rec, const void* theta, const void* dL
   if (rec->N == 0) return GS_OK;
   if (!theta || !dL_dy1) return fail(GS_ERR_INVALID_ARG, "theta and dL_dy1 must be non-NULL");
   if (!dL_dtheta && !dL_dy0) return fail(GS_ERR_INVALID_ARG, "no output requested");
+  gs_status st = check_device({{theta, "theta"}, {dL_dy1, "dL_dy1"}, {dL_dtheta, "dL_dtheta"},
+                               {dL_dy0, "dL_dy0"}});
+  if (st != GS_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int M = rec->sys.m;
   const int64_t N = rec->N;
@@ -813,6 +857,8 @@ gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, v
   if (!rec) return fail(GS_ERR_INVALID_ARG, "record is NULL");
   if (rec->N == 0) return GS_OK;
   if (!theta || !y0) return fail(GS_ERR_INVALID_ARG, "theta and y0 must be non-NULL");
+  const gs_status dst = check_device({{theta, "theta"}, {y0, "y0"}, {y1, "y1"}});
+  if (dst != GS_OK) return dst;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   void* y1buf = y1;
   if (!y1buf) {
@@ -922,6 +968,8 @@ gs_status gs_replay_outputs(const gs_record* rec, const void* theta, const void*
   if (rec->N == 0) return GS_OK;
   if (!theta || !y0 || !y_out)
     return fail(GS_ERR_INVALID_ARG, "theta, y0 and y_out must be non-NULL");
+  st = check_device({{theta, "theta"}, {y0, "y0"}, {y_out, "y_out"}});
+  if (st != GS_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* queue = nullptr;
   GS_CUDA(take_counter(s, &queue));
@@ -951,6 +999,9 @@ gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_
   if (rec->N == 0) return GS_OK;
   if (!theta || !dL_dyout) return fail(GS_ERR_INVALID_ARG, "theta and dL_dyout must be non-NULL");
   if (!dL_dtheta && !dL_dy0) return fail(GS_ERR_INVALID_ARG, "no output requested");
+  st = check_device({{theta, "theta"}, {dL_dyout, "dL_dyout"}, {dL_dy1, "dL_dy1"},
+                     {dL_dtheta, "dL_dtheta"}, {dL_dy0, "dL_dy0"}});
+  if (st != GS_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int M = rec->sys.m;
   const int64_t N = rec->N;
@@ -1055,6 +1106,8 @@ gs_status gs_record_export(const gs_record* rec, void* T, void* H, void* Y, int6
                            void* stream) {
   NvtxRange nvtx_range("gs_record_export");
   if (!rec) return fail(GS_ERR_INVALID_ARG, "record is NULL");
+  gs_status st = check_device({{T, "T"}, {H, "H"}, {Y, "Y"}, {offsets, "offsets"}});
+  if (st != GS_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (offsets && rec->N >= 0)
     GS_CUDA(cudaMemcpyAsync(offsets, rec->offsets, (rec->N + 1) * sizeof(long long),
@@ -1085,6 +1138,10 @@ gs_status gs_record_import(const gs_system* sys, int64_t N, const int32_t* nstep
   if (!rec) return fail(GS_ERR_INVALID_ARG, "rec must be non-NULL");
   if (N < 0 || N > 0x7fffffffLL) return fail(GS_ERR_INVALID_ARG, "N out of range");
   if (N > 0 && (!nsteps || !H || !Y)) return fail(GS_ERR_INVALID_ARG, "nsteps, H, Y required");
+  if (N > 0) {
+    st = check_device({{nsteps, "nsteps"}, {T, "T"}, {H, "H"}, {Y, "Y"}});
+    if (st != GS_OK) return st;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   gs_record* r = new (std::nothrow) gs_record();
   if (!r) return fail(GS_ERR_CAPACITY, "out of host memory");

@@ -127,12 +127,14 @@ def options(max_attempts=0, record_capacity_steps=0, start_order=None):
     """start_order: optional int32 device tensor [N], the order in which trajectories are started
     (scheduling only).  The tensor must stay alive while the call's work runs."""
     return GsOptions(max_attempts, record_capacity_steps,
-                     None if start_order is None else start_order.data_ptr())
+                     None if start_order is None else _ptr(start_order).value)
 
 
 def _ptr(t):
     if t is None:
         return None
+    if not t.is_cuda:
+        raise ValueError("tensors must be on a CUDA device (got %s)" % t.device)
     if not t.is_contiguous():
         raise ValueError("tensors must be contiguous")
     return C.c_void_p(t.data_ptr())

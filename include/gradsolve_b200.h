@@ -21,7 +21,10 @@
  *   - Real arrays are double (GS_F64) or float (GS_F32) per gs_system.dtype, row-major:
  *     y0, y1, dL_dy1, dL_dy0: [N][d];  theta, dL_dtheta: [N][m], or [m] when theta_shared.
  *   - Array pointers are DEVICE pointers owned by the caller, unless stated otherwise.  The record
- *     (gs_record) is owned by the library and freed by gs_record_destroy.
+ *     (gs_record) is owned by the library and freed by gs_record_destroy.  Before launching, the
+ *     entry points ask the runtime what each array is and return GS_ERR_INVALID_ARG for plain
+ *     (unregistered) host memory or another device's memory, which a kernel could not read;
+ *     device, managed and page-locked host memory pass (gs_replay_grad_noalloc skips the query).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued on it; calls
  *     return when the work is enqueued, except where a host synchronisation is stated.
  *   - Errors: every entry point returns a gs_status and never aborts or exits; gs_last_error()

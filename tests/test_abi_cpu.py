@@ -92,3 +92,17 @@ def test_checked_build_compiles_and_exports():
     L = C.CDLL(path)
     for name in declared():
         assert hasattr(L, name), name
+
+
+def test_binding_refuses_host_tensors(G):
+    # a host tensor's address is not readable by the kernels: the binding refuses it before the
+    # library is called (the library itself also asks the runtime, on a GPU machine)
+    torch = pytest.importorskip("torch")
+    s = G.system("lorenz63")
+    th = torch.zeros((4, 3), dtype=torch.float64)
+    y0 = torch.zeros((4, 3), dtype=torch.float64)
+    y1 = torch.empty_like(y0)
+    with pytest.raises(ValueError, match="CUDA device"):
+        G.gs_solve_forward(s, 4, th, y0, 0.0, 1.0, 1e-6, 1e-9, y1)
+    with pytest.raises(ValueError, match="CUDA device"):
+        G.options(start_order=torch.arange(4, dtype=torch.int32))
