@@ -204,6 +204,11 @@ struct gs_record {
   size_t red_bytes = 0, part_bytes = 0;
   void* y1_scratch = nullptr;    // y_S of gs_replay_forward when the caller passes no y1
   size_t y1_bytes = 0;
+  // the theta the stored states y_n were computed at ([N][m], or [m] when shared); counters[8]
+  // is the flag the device comparison with a caller's theta raises
+  void* theta_kept = nullptr;
+  size_t theta_kept_bytes = 0;
+  bool theta_known = false;      // false after an import: the first use replays the states
   // device time of the solve kernel of the last record pass
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
   double solve_ms = 0;
@@ -571,6 +576,102 @@ long long attempts_of(const gs_options* opt) {
 
 }  // namespace
 
+// ------------------------------------------------------------------------------------------------
+// The theta of the stored states.  Beside the states y_n, a record keeps a copy of the theta they
+// were computed at (set by the record pass and by gs_replay_forward).  Every call that reads the
+// stored states at a caller's theta first compares the two bit for bit on the device; when they
+// differ, the mesh is replayed forward at the caller's theta from the stored y_0, rewriting the
+// stored states (t_n and h_n are kept).  The result of such a call is therefore always that of
+// the replay Psi(theta; sg[h]) over the recorded mesh ("gradsolve: fast exact gradients for ODE
+// ensembles on GPUs", §3: the mesh is data; §4.8: one mesh serves the gradients of a whole fit).
+// An equal theta costs one read of both copies and a replay launch that exits at once.
+// ------------------------------------------------------------------------------------------------
+namespace {
+
+size_t theta_bytes(const gs_record* r) {
+  return (size_t)(r->sys.theta_shared ? 1 : std::max<int64_t>(r->N, 1)) * r->sys.m * r->rsz;
+}
+
+gs_status ensure_theta_kept(gs_record* r) {
+  const size_t need = theta_bytes(r);
+  if (r->theta_kept_bytes >= need) return GS_OK;
+  free_ptr(r->theta_kept);
+  r->theta_kept = nullptr;
+  r->theta_kept_bytes = 0;
+  GS_CUDA(cudaMalloc(&r->theta_kept, need));
+  r->theta_kept_bytes = need;
+  return GS_OK;
+}
+
+// The stored states are now those of `theta`.
+gs_status keep_theta(gs_record* r, const void* theta, cudaStream_t s) {
+  GS_CUDA(cudaMemcpyAsync(r->theta_kept, theta, theta_bytes(r), cudaMemcpyDeviceToDevice, s));
+  r->theta_known = true;
+  return GS_OK;
+}
+
+// Makes the stored states those of `theta`.  `queue`: a work counter for the replay kernel, zeroed
+// on stream s.  With `fixed_grid` (the entry point that allocates nothing) the grid comes from the
+// occupancy query and `sms` alone, without the per-device context.
+gs_status refresh_states(gs_record* r, const void* theta, int* queue, bool fixed_grid, int sms,
+                         cudaStream_t s) {
+  if (r->N == 0 || r->total_steps == 0) return GS_OK;  // no stored state
+  if (!r->theta_kept) return fail(GS_ERR_INVALID_ARG, "record holds no parameter copy");
+  int* stale = r->counters + 8;
+  GS_CUDA(cudaMemsetAsync(stale, r->theta_known ? 0 : 1, sizeof(int), s));
+  const long long count = (long long)(theta_bytes(r) / r->rsz);
+  const int cgrid = (int)std::max(1LL, std::min<long long>((count + 255) / 256, 8LL * sms));
+  if (r->rsz == 8)
+    gs::k_theta_check<double><<<cgrid, 256, 0, s>>>(static_cast<const double*>(theta),
+                                                   static_cast<double*>(r->theta_kept), count, stale);
+  else
+    gs::k_theta_check<float><<<cgrid, 256, 0, s>>>(static_cast<const float*>(theta),
+                                                  static_cast<float*>(r->theta_kept), count, stale);
+  GS_CUDA(cudaGetLastError());
+  r->theta_known = true;
+  return dispatch(r->sys, [&]<class F, class R, int METHOD>() {
+    gs::ReplayParams<R> p{};
+    p.N = (int)r->N;
+    p.theta = static_cast<const R*>(theta);
+    p.theta_stride = r->sys.theta_shared ? 0 : r->sys.m;
+    p.y0 = nullptr;  // from the stored y_0
+    p.y1 = nullptr;
+    p.nsteps = r->nsteps;
+    p.choff = r->choff;
+    p.chunk_table = r->chunk_table;
+    p.pool = static_cast<R*>(r->pool);
+    p.queue = queue;
+    p.perm = r->perm;
+    p.bounds = bounds_of(r);
+    p.gate = stale;
+    auto launch = [&](auto kern, long long units) -> gs_status {
+      int grid = 1;
+      if (fixed_grid) {
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, BLOCK, 0) != cudaSuccess ||
+            nb < 1)
+          nb = 1;
+        grid = (int)std::max(1LL, std::min((long long)sms * nb, (units + BLOCK - 1) / BLOCK));
+      } else {
+        grid = persistent_grid(kern, 0, units);
+      }
+      kern<<<grid, BLOCK, 0, s>>>(p);
+      GS_CUDA(cudaGetLastError());
+      return GS_OK;
+    };
+    if constexpr (std::is_same_v<F, gs::FMlpWarp>) return launch(gs::k_replay_forward_mlp<R>, r->N * 32);
+    else return launch(gs::k_replay_forward<F, R, METHOD>, r->N);
+  });
+}
+
+int device_sms() {
+  cudaError_t e;
+  DeviceCtx* c = device_ctx(&e);
+  return c ? c->sms : 148;
+}
+
+}  // namespace
+
 // Replay adjoint of the MLP field: one warp per trajectory, per-warp weight-cotangent partials,
 // then a fixed-order sum over warps.
 static gs_status replay_grad_mlp(const gs_record* rec, const void* theta, const void* dL_dy1,
@@ -791,6 +892,8 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
         r->chunk_traj, r->chunk_seq, (int)r->nchunks, r->choff, r->chunk_table, bounds_of(r));
   if (cudaGetLastError() != cudaSuccess) return bail(fail(GS_ERR_CUDA, "chunk table launch failed"));
   if ((st = build_perm(r, s)) != GS_OK) return bail(st);
+  if ((st = ensure_theta_kept(r)) != GS_OK || (st = keep_theta(r, theta, s)) != GS_OK)
+    return bail(st);
   *rec = r;
   if (r->host[4] != 0) {
     fail(GS_ERR_TRAJ_FAILED, "some trajectories did not reach t1 (max status %d)", r->host[4]);
@@ -812,11 +915,14 @@ gs_status gs_replay_grad(const gs_record* rec, const void* theta, const void* dL
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int M = rec->sys.m;
   const int64_t N = rec->N;
+  gs_record* r = const_cast<gs_record*>(rec);
+  int* rq = nullptr;
+  GS_CUDA(take_counter(s, &rq));
+  if ((st = refresh_states(r, theta, rq, false, device_sms(), s)) != GS_OK) return st;
   if (rec->sys.field == GS_MLP_4_32_32_4) return replay_grad_mlp(rec, theta, dL_dy1, dL_dtheta, dL_dy0, s);
   const bool shared = rec->sys.theta_shared && dL_dtheta;
   const int per_block = 4096;
   const int nred = (int)((N + per_block - 1) / per_block);
-  gs_record* r = const_cast<gs_record*>(rec);
   if (shared) {
     const size_t need = (size_t)N * M * rec->rsz, needp = (size_t)nred * M * rec->rsz;
     if (r->red_bytes < need) {
@@ -912,7 +1018,8 @@ gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, v
     return GS_OK;
     }
   });
-  return st;
+  if (st != GS_OK) return st;
+  return keep_theta(rec, theta, s);  // the stored states are now those of theta
 }
 
 }  // extern "C"
@@ -973,6 +1080,10 @@ gs_status gs_replay_outputs(const gs_record* rec, const void* theta, const void*
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* queue = nullptr;
   GS_CUDA(take_counter(s, &queue));
+  int* rq = nullptr;
+  GS_CUDA(take_counter(s, &rq));
+  st = refresh_states(const_cast<gs_record*>(rec), theta, rq, false, device_sms(), s);
+  if (st != GS_OK) return st;
   return dispatch(rec->sys, [&]<class F, class R, int METHOD>() {
     if constexpr (std::is_same_v<F, gs::FMlpWarp>) {
       return fail(GS_ERR_UNSUPPORTED, "not built for the MLP field");
@@ -1009,6 +1120,9 @@ gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_
   const int per_block = 4096;
   const int nred = (int)((N + per_block - 1) / per_block);
   gs_record* r = const_cast<gs_record*>(rec);
+  int* rq = nullptr;
+  GS_CUDA(take_counter(s, &rq));
+  if ((st = refresh_states(r, theta, rq, false, device_sms(), s)) != GS_OK) return st;
   if (shared) {
     const size_t need = (size_t)N * M * rec->rsz, needp = (size_t)nred * M * rec->rsz;
     if (r->red_bytes < need) {
@@ -1202,7 +1316,9 @@ gs_status gs_record_import(const gs_system* sys, int64_t N, const int32_t* nstep
       if (cudaGetLastError() != cudaSuccess) return bail(fail(GS_ERR_CUDA, "import launch failed"));
     }
     if ((st = build_perm(r, s)) != GS_OK) return bail(st);
+    if ((st = ensure_theta_kept(r)) != GS_OK) return bail(st);
   }
+  r->theta_known = false;  // the states' theta is not known: the first use replays them
   *rec = r;
   return GS_OK;
 }
@@ -1217,6 +1333,7 @@ void gs_record_destroy(gs_record* r) {
   free_ptr(r->nsteps); free_ptr(r->status); free_ptr(r->offsets); free_ptr(r->choff);
   free_ptr(r->tiles); free_ptr(r->counters);
   free_ptr(r->red_scratch); free_ptr(r->red_partials); free_ptr(r->y1_scratch);
+  free_ptr(r->theta_kept);
   free_ptr(r->perm); free_ptr(r->bins); free_ptr(r->binoff); free_ptr(r->btiles);
   if (r->host) cudaFreeHost(r->host);
   if (r->ev0) cudaEventDestroy(r->ev0);
@@ -1230,8 +1347,9 @@ void gs_record_destroy(gs_record* r) {
 // ------------------------------------------------------------------------------------------------
 // gs_replay_grad_noalloc: the replay gradient with its scratch in a fixed device array, for
 // callers that cannot allocate device memory when they ask for a gradient.
-// Layout of the array: [0, 256) work counter; then theta-bar per trajectory [N][m]; then the
-// block partials [nred][m] of the shared-theta sum.
+// Layout of the array: [0, 256) work counters (the adjoint's at byte 0, the forward replay's at
+// byte 64); then theta-bar per trajectory [N][m]; then the block partials [nred][m] of the
+// shared-theta sum.
 // ------------------------------------------------------------------------------------------------
 static __device__ __align__(256) unsigned char g_noalloc_scratch[GS_NOALLOC_SCRATCH_BYTES];
 
@@ -1293,12 +1411,13 @@ gs_status noalloc_adjoint(const gs_record* r, const void* theta, const void* dL_
     p.bounds = bounds_of(r);
     auto kern = gs::k_adjoint<F, R, METHOD>;
     const size_t smem = adjoint_smem<F, R, METHOD>();
+    if (smem > 48 * 1024)
+      GS_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     int nb = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, BLOCK, smem) != cudaSuccess || nb < 1)
       nb = 1;
     const long long grid =
         std::max(1LL, std::min((long long)sms * nb, (long long)((N + BLOCK - 1) / BLOCK)));
-    GS_CUDA(cudaMemsetAsync(scratch, 0, sizeof(int), s));  // the counter starts at zero
     kern<<<(int)grid, BLOCK, smem, s>>>(p);
     if (shared) {
       gs::k_reduce_theta<R><<<nred, gs::RED_BLOCK, 0, s>>>(traj, (int)N, M, per_block, partials);
@@ -1321,6 +1440,9 @@ extern "C" gs_status gs_replay_grad_noalloc(const gs_record* rec, const void* th
   if (!dL_dtheta && !dL_dy0) return fail(GS_ERR_INVALID_ARG, "no output requested");
   if (rec->sys.field == GS_MLP_4_32_32_4)
     return fail(GS_ERR_UNSUPPORTED, "gs_replay_grad_noalloc does not take the MLP field");
+  gs_status st = check_device({{theta, "theta"}, {dL_dy1, "dL_dy1"}, {dL_dtheta, "dL_dtheta"},
+                               {dL_dy0, "dL_dy0"}});
+  if (st != GS_OK) return st;
   const bool shared = rec->sys.theta_shared && dL_dtheta;
   const size_t nred = (size_t)((rec->N + 4095) / 4096);
   const size_t need = 256 + (shared ? ((size_t)rec->N + nred) * rec->sys.m * rec->rsz : 0);
@@ -1330,13 +1452,17 @@ extern "C" gs_status gs_replay_grad_noalloc(const gs_record* rec, const void* th
                 "array holds %u bytes (use gs_replay_grad)",
                 need, (long long)rec->N, rec->sys.m, GS_NOALLOC_SCRATCH_BYTES);
   NoallocDevice* d = nullptr;
-  gs_status st = noalloc_setup(&d);
+  st = noalloc_setup(&d);
   if (st != GS_OK) return st;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev != rec->device)
     return fail(GS_ERR_INVALID_ARG, "record belongs to device %d, current is %d", rec->device, dev);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  GS_CUDA(cudaMemsetAsync(d->ptr, 0, 128, s));  // both work counters start at zero
+  st = refresh_states(const_cast<gs_record*>(rec), theta, reinterpret_cast<int*>(d->ptr + 64),
+                      true, d->sms, s);
+  if (st != GS_OK) return st;
   return dispatch(rec->sys, [&]<class F, class R, int METHOD>() {
     return noalloc_adjoint<F, R, METHOD>(rec, theta, dL_dy1, dL_dtheta, dL_dy0, d->ptr, d->sms, s);
   });

@@ -19,6 +19,7 @@
 // the stages from it).
 #pragma once
 #include <cstdint>
+#include <type_traits>
 
 #include "gs_methods.cuh"
 
@@ -697,8 +698,8 @@ struct ReplayParams {
   int N;
   const R* theta;
   int theta_stride;
-  const R* y0;
-  R* y1;
+  const R* y0;              // null: each trajectory starts from its stored y_0 (entry 0)
+  R* y1;                    // nullable
   const int* nsteps;
   const long long* choff;
   const int* chunk_table;
@@ -706,12 +707,14 @@ struct ReplayParams {
   int* queue;
   const int* perm;
   RecBounds bounds;
+  const int* gate = nullptr;  // k_replay_forward*: when set and *gate == 0 the kernel does nothing
 };
 
 template <class F, class R, int METHOD>
 __global__ void __launch_bounds__(128) k_replay_forward(ReplayParams<R> p) {
   using L = RecLayout<F, R>;
   constexpr int D = F::D;
+  if (p.gate && *p.gate == 0) return;
   int k = -1, n = 0, S = 0;
   bool alive = true;
   long long cbase = 0;
@@ -727,11 +730,18 @@ __global__ void __launch_bounds__(128) k_replay_forward(ReplayParams<R> p) {
         if (id < p.N) {
           k = p.perm ? p.perm[id] : id;
           F::load(th, p.theta + (size_t)p.theta_stride * k);
-#pragma unroll
-          for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
           n = 0;
           S = p.nsteps[k];
           cbase = p.choff[k];
+          if (p.y0) {
+#pragma unroll
+            for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
+          } else if (S > 0) {
+            const R* e0 = chunk_entry<L>(p.pool, chunk_at(p.chunk_table, cbase, p.bounds), 0,
+                                         p.bounds);
+#pragma unroll
+            for (int c = 0; c < D; ++c) y[c] = e0[2 + c];
+          }
         } else {
           alive = false;
         }
@@ -752,8 +762,9 @@ __global__ void __launch_bounds__(128) k_replay_forward(ReplayParams<R> p) {
         ++n;
       }
       if (n >= S) {
+        if (p.y1)
 #pragma unroll
-        for (int c = 0; c < D; ++c) p.y1[(size_t)k * D + c] = y[c];
+          for (int c = 0; c < D; ++c) p.y1[(size_t)k * D + c] = y[c];
         k = -1;
       }
     }
@@ -1021,6 +1032,26 @@ __global__ void k_chunk_table(const int* chunk_traj, const int* chunk_seq, int n
       table[ti] = c;
     }
   }
+}
+
+// The stored states of a record belong to the theta kept beside them.  Compares the caller's
+// theta with that copy bit for bit; any difference sets *stale (the caller zeroes it, or sets it
+// to force a replay) and the copy takes the caller's values.
+template <class R>
+__global__ void k_theta_check(const R* theta, R* kept, long long count, int* stale) {
+  using U = typename std::conditional<sizeof(R) == 8, unsigned long long, unsigned>::type;
+  const U* a = reinterpret_cast<const U*>(theta);
+  U* b = reinterpret_cast<U*>(kept);
+  bool diff = false;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < count;
+       i += (long long)gridDim.x * blockDim.x) {
+    const U v = a[i];
+    if (v != b[i]) {
+      b[i] = v;
+      diff = true;
+    }
+  }
+  if (__any_sync(FULL, diff) && (threadIdx.x & 31) == 0) *stale = 1;
 }
 
 // max over S (int), via warp reduce + atomicMax

@@ -323,6 +323,7 @@ __global__ void __launch_bounds__(128) k_replay_forward_mlp(ReplayParams<R> p) {
   using L = MlpLayout<R>;
   constexpr int D = MLP_D;
   __shared__ R slots[4][32];
+  if (p.gate && *p.gate == 0) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   MlpLane<R> W;
   W.load(p.theta, slots[warp]);
@@ -332,11 +333,18 @@ __global__ void __launch_bounds__(128) k_replay_forward_mlp(ReplayParams<R> p) {
     id = __shfl_sync(FULL, id, 0);
     if (id >= p.N) break;
     const int k = p.perm ? p.perm[id] : id;
-    R y[D];
-#pragma unroll
-    for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
     const int S = p.nsteps[k];
     const long long cbase = p.choff[k];
+    R y[D];
+    if (p.y0) {
+#pragma unroll
+      for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
+    } else {
+      if (S == 0) continue;  // nothing stored and nothing to rewrite
+      const R* e0 = chunk_entry<L>(p.pool, chunk_at(p.chunk_table, cbase, p.bounds), 0, p.bounds);
+#pragma unroll
+      for (int c = 0; c < D; ++c) y[c] = e0[2 + c];
+    }
     for (int n = 0; n < S; ++n) {
       R* e = chunk_entry<L>(p.pool, chunk_at(p.chunk_table, cbase + n / L::C, p.bounds), n,
                             p.bounds);
@@ -370,7 +378,7 @@ __global__ void __launch_bounds__(128) k_replay_forward_mlp(ReplayParams<R> p) {
 #pragma unroll
       for (int c = 0; c < D; ++c) y[c] = ynew[c];
     }
-    if (lane < D) p.y1[(size_t)k * D + lane] = y[lane];
+    if (p.y1 && lane < D) p.y1[(size_t)k * D + lane] = y[lane];
   }
 }
 

@@ -24,7 +24,7 @@
  *     (gs_record) is owned by the library and freed by gs_record_destroy.  Before launching, the
  *     entry points ask the runtime what each array is and return GS_ERR_INVALID_ARG for plain
  *     (unregistered) host memory or another device's memory, which a kernel could not read;
- *     device, managed and page-locked host memory pass (gs_replay_grad_noalloc skips the query).
+ *     device, managed and page-locked host memory pass.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued on it; calls
  *     return when the work is enqueued, except where a host synchronisation is stated.
  *   - Errors: every entry point returns a gs_status and never aborts or exits; gs_last_error()
@@ -179,12 +179,15 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
                           double atol, gs_record** rec, void* y1, int32_t* status, void* stream);
 
 /* Replay gradient ([GS] §3): the exact reverse-mode derivative of the replay over the recorded
- * mesh with the mesh held fixed as data.  The backward sweep recomputes each step's stages from
- * the state stored for that step ([GS] §3.3: one accepted state kept per step): the states of the
- * record pass, or of the latest gs_replay_forward.  With the stored states made at theta0 and
- * `theta` = theta0 the result is d Psi(theta0; sg[R(theta0)]) / d theta.  For a gradient at another
- * theta on the same mesh (d Psi(theta; sg[R(theta0)]) / d theta), call gs_replay_forward(theta)
- * first.
+ * mesh with the mesh held fixed as data, at `theta`: d Psi(theta; sg[R(theta0)]) / d theta, where
+ * R(theta0) is the recorded mesh, for `theta` equal to the recorded theta0 or not ([GS] §3; §4.8:
+ * one mesh serves the gradients of a whole fit).  The backward sweep recomputes each step's stages
+ * from the state stored for that step ([GS] §3.3: one accepted state kept per step).  The record
+ * keeps the theta its stored states were made at (the record pass's, or the latest
+ * gs_replay_forward's); the call compares it with `theta` bit for bit on the device and, when they
+ * differ, first replays the mesh forward at `theta` from the stored y_0, rewriting the stored
+ * states in place (t_n, h_n kept; nothing allocated).  Calls on one record must be ordered on one
+ * stream (they share its states).
  * In:  theta (as for the solve), dL_dy1 [N][d].  Out (each nullable, at least one non-NULL):
  * dL_dy0 [N][d]; dL_dtheta [N][m], or [m] = sum over the ensemble when theta is shared (summed in
  * a fixed order: bitwise reproducible).  Asynchronous. */
@@ -192,8 +195,8 @@ gs_status gs_replay_grad(const gs_record* rec, const void* theta, const void* dL
                          void* dL_dtheta, void* dL_dy0, void* stream);
 
 /* Forward replay ([GS] §3, Eq. 4): y_{n+1} = Phi(y_n, h_n; theta) over the recorded mesh from y0,
- * storing each y_n in the record (t_n and h_n are kept) and y_S in y1 [N][d] (device, nullable).
- * Asynchronous. */
+ * storing each y_n in the record (t_n and h_n are kept) and y_S in y1 [N][d] (device, nullable);
+ * the record then holds the states of `theta` (and of this y0).  Asynchronous. */
 gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, void* y1,
                             void* stream);
 
@@ -202,8 +205,9 @@ gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, v
  * tau: HOST array of J times (1 <= J <= GS_MAX_OUTPUT_TIMES), ascending; for tau_j the output is
  * Phi(y_n, tau_j - t_n) with n the first recorded step with tau_j < t_{n+1} (t_S = t1), and the
  * final state for tau_j >= t1 (times before t0 are integrated backwards from y0).  Uses the
- * record's stored states (as gs_replay_grad); y0 [N][d] (device) is the initial state, read for
- * trajectories with no recorded step.  y_out [N][J][d] (device).  Not built for
+ * record's stored states, replayed first when `theta` is not the theta they were made at (as
+ * gs_replay_grad); y0 [N][d] (device) is the initial state, read for trajectories with no
+ * recorded step.  y_out [N][J][d] (device).  Not built for
  * GS_MLP_4_32_32_4 (GS_ERR_UNSUPPORTED).  Asynchronous. */
 #define GS_MAX_OUTPUT_TIMES 256
 gs_status gs_replay_outputs(const gs_record* rec, const void* theta, const void* y0, int32_t J,
@@ -212,7 +216,7 @@ gs_status gs_replay_outputs(const gs_record* rec, const void* theta, const void*
 /* Gradient of a loss on the outputs at requested times (and optionally on the final state):
  * dL_dyout [N][J][d] (device), dL_dy1 [N][d] (device, nullable); outputs as gs_replay_grad.
  * Each output's cotangent is pulled back through its extra step from y_n and added to the
- * cotangent of y_n.  Asynchronous. */
+ * cotangent of y_n.  The stored states follow `theta` as in gs_replay_grad.  Asynchronous. */
 gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_t J,
                                  const double* tau, const void* dL_dyout, const void* dL_dy1,
                                  void* dL_dtheta, void* dL_dy0, void* stream);
@@ -230,10 +234,14 @@ gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_
  * fixed array of GS_NOALLOC_SCRATCH_BYTES (8 MiB) inside the library, held by every GPU that
  * loads the library until the process exits.  A record whose shared-theta scratch would not fit
  * (about N*m <= 1.04e6 in double, 2.09e6 in float) is rejected with GS_ERR_CAPACITY.
+ * Like gs_replay_grad it differentiates at `theta` even when the stored states were made at
+ * another theta, replaying them into the record's own slots first.
  * The first call on a device looks up that array's device address (a one-time set-up per
- * device); make that first call before any stream capture begins.  All calls share the one
- * array and the counter is cleared at the start of each call: calls that overlap on the GPU (on
- * different streams, or from different threads) race and must not be issued.  Asynchronous. */
+ * device), and the first call for each (field, method, dtype) combination loads that
+ * combination's kernels; make those first calls before any stream capture begins.  All calls
+ * share the one array and its work counters are cleared at the start of each call: calls that
+ * overlap on the GPU (on different streams, or from different threads) race and must not be
+ * issued.  Asynchronous. */
 #define GS_NOALLOC_SCRATCH_BYTES (8u << 20)
 gs_status gs_replay_grad_noalloc(const gs_record* rec, const void* theta, const void* dL_dy1,
                                  void* dL_dtheta, void* dL_dy0, void* stream);
@@ -255,7 +263,9 @@ gs_status gs_record_export(const gs_record* rec, void* T, void* H, void* Y, int6
 
 /* Build a record from contiguous ragged arrays (device): nsteps [N] int32, T [total] (nullable,
  * zeros when NULL), H [total], Y [total][d] with total = sum nsteps.  Lets one mesh be replayed
- * by another producer's record or reused across many gradients ([GS] §4.8).  Synchronises once. */
+ * by another producer's record or reused across many gradients ([GS] §4.8).  The theta of the
+ * imported states is unknown to the library, so the first call that takes a theta replays them
+ * from each trajectory's first state Y[offsets[k]].  Synchronises once. */
 gs_status gs_record_import(const gs_system* sys, int64_t N, const int32_t* nsteps, const void* T,
                            const void* H, const void* Y, gs_record** rec, void* stream);
 

@@ -6,7 +6,9 @@ allocations, or a loop in which an allocation would synchronise the device.  The
 point keeps its scratch in a fixed array inside the library instead.  These tests call it through
 the C ABI and check that it returns what gs_replay_grad returns, on two calls in a row (the array
 keeps the previous call's contents, so the second call shows that what must start at zero is
-cleared), and that a problem too large for the array is refused with a clear error.
+cleared), that the second call changes the device's free memory by nothing, and that a problem
+too large for the array is refused with a clear error.  The no-alloc calls come first on each
+record, so they cannot lean on anything gs_replay_grad allocated for it.
 
 This file is collected last on purpose: it passes alone in a fresh process and after the others.
 """
@@ -30,21 +32,30 @@ def _cuda():
     G.lib()
 
 
-def _both(w, rec, lam):
+def _both(w, rec, lam, theta=None):
+    """Two no-alloc calls in a row on a record no other gradient call has touched, then
+    gs_replay_grad for reference.  The second no-alloc call must leave the device's free memory
+    exactly as it found it (the first may still load the variant's kernels)."""
     torch = U.torch()
     dt = U.tdtype(w)
-    th, lam_t = U.dev(w.theta, dt), U.dev(lam, dt)
+    th = U.dev(w.theta if theta is None else theta, dt)
+    lam_t = U.dev(lam, dt)
     shape_t = (w.m,) if w.theta_shared else (w.N, w.m)
+    bufs = [(torch.full(shape_t, np.nan, dtype=dt, device="cuda"),
+             torch.full((w.N, w.d), np.nan, dtype=dt, device="cuda")) for _ in range(2)]
+    torch.cuda.synchronize()
+    outs = []
+    for i, (gt, gy) in enumerate(bufs):     # the two calls share the fixed scratch
+        free_before = torch.cuda.mem_get_info()[0]
+        G.gs_replay_grad_noalloc(rec, th, lam_t, gt, gy)
+        torch.cuda.synchronize()
+        if i == 1:
+            assert torch.cuda.mem_get_info()[0] == free_before
+        outs.append((gt.cpu().numpy(), gy.cpu().numpy()))
     ref_t = torch.empty(shape_t, dtype=dt, device="cuda")
     ref_y = torch.empty((w.N, w.d), dtype=dt, device="cuda")
     G.gs_replay_grad(rec, th, lam_t, ref_t, ref_y)
-    outs = []
-    for _ in range(2):                      # two calls in a row share the fixed scratch
-        gt = torch.full(shape_t, np.nan, dtype=dt, device="cuda")
-        gy = torch.full((w.N, w.d), np.nan, dtype=dt, device="cuda")
-        G.gs_replay_grad_noalloc(rec, th, lam_t, gt, gy)
-        torch.cuda.synchronize()
-        outs.append((gt.cpu().numpy(), gy.cpu().numpy()))
+    torch.cuda.synchronize()
     return (ref_t.cpu().numpy(), ref_y.cpu().numpy()), outs
 
 
@@ -71,6 +82,17 @@ def test_no_alloc_matches_replay_grad_per_trajectory_theta():
     rec, _ = U.record(w)
     lam = np.random.default_rng(12).normal(size=(w.N, w.d))
     (rt, ry), outs = _both(w, rec, lam)
+    for gt, gy in outs:
+        assert _close(gt, rt) and _close(gy, ry)
+
+
+def test_no_alloc_at_a_theta_other_than_the_recorded_one():
+    # the stored states were made at theta0; both entry points must differentiate the replay at
+    # the theta they are given (the no-alloc one replays the states into the record's own slots)
+    w = W.nfw_mn(N=700)
+    rec, _ = U.record(w)
+    lam = np.random.default_rng(13).normal(size=(w.N, w.d))
+    (rt, ry), outs = _both(w, rec, lam, theta=w.theta * 1.01)
     for gt, gy in outs:
         assert _close(gt, rt) and _close(gy, ry)
 
