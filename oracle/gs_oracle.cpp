@@ -399,7 +399,9 @@ int orc_trial(int field, int method, const double* theta, const double* y, doubl
 }
 
 // Arithmetic tally of one f evaluation (what=0), one Tsit5 trial step with error estimate
-// (what=1) or one Rosenbrock trial step (what=2), at state y and parameters theta.
+// (what=1), one Rosenbrock trial step (what=2), f on one-direction dual numbers (what=3), or the
+// reverse sweep of f's vector-Jacobian product with respect to (y, theta) taken by a plain
+// reverse-mode pass over f's operations (what=4), at state y and parameters theta.
 // counts = {add, mul, div, sqrt, log1p, tanh}.
 int orc_count_ops(int field, int what, const double* theta, const double* y, double h,
                   long long* counts) {
@@ -422,6 +424,20 @@ int orc_count_ops(int field, int what, const double* theta, const double* y, dou
       for (int c = 0; c < F::D; ++c) { yd[c] = DC(yy[c]); yd[c].g[0] = Cnt(1.0); }
       tally() = OpTally{};
       F::f(yd, thd.data(), od);
+    } else if (what == 4) {
+      std::vector<Tap> tht(F::M);
+      Tap yt[F::D], ot[F::D];
+      tape().clear();
+      for (int c = 0; c < F::D; ++c) yt[c] = Tap::leaf(y[c]);
+      for (int j = 0; j < F::M; ++j) tht[j] = Tap::leaf(theta[j]);
+      F::f(yt, tht.data(), ot);
+      int outs[F::D];
+      for (int c = 0; c < F::D; ++c) outs[c] = ot[c].id;
+      const OpTally t = tally_reverse_sweep(outs, F::D);
+      tape().clear();
+      counts[0] = t.add; counts[1] = t.mul; counts[2] = t.div;
+      counts[3] = t.sqrt; counts[4] = t.log1p; counts[5] = t.tanh;
+      return 0;
     } else if (what == 1) {
       tsit5_trial<F, Cnt>(yy, Cnt(h), th.data(), k1, out, k7, e, true);
     } else {

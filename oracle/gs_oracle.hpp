@@ -149,6 +149,80 @@ inline Cnt tanh(Cnt a) { tally().tanh++; return Cnt(std::tanh(a.v)); }
 inline double value_of(Cnt a) { return a.v; }
 
 // ------------------------------------------------------------------------------------------
+// Reverse-mode tape: a double that records every operation whose result depends on a marked
+// input, so that the work of a plain reverse sweep (the definitional pullback of f, adjoints
+// accumulated into zero-initialised slots) can be tallied.  Used to bound the operation count of
+// a vector-Jacobian product independently of any hand-written one.
+// ------------------------------------------------------------------------------------------
+enum TapOp { TAP_LEAF, TAP_ADD, TAP_SUB, TAP_NEG, TAP_MUL, TAP_DIV, TAP_SQRT, TAP_LOG1P, TAP_TANH };
+struct TapNode { TapOp op; int a, b; };
+inline std::vector<TapNode>& tape() { static thread_local std::vector<TapNode> t; return t; }
+struct Tap {
+  double v;
+  int id;  // node on the tape, -1 for a value that depends on no marked input
+  Tap() : v(0), id(-1) {}
+  Tap(double x) : v(x), id(-1) {}
+  static Tap leaf(double x) {
+    tape().push_back({TAP_LEAF, -1, -1});
+    Tap t(x);
+    t.id = (int)tape().size() - 1;
+    return t;
+  }
+};
+template <> struct base_of<Tap> { using type = double; };
+inline Tap tap_node(double v, TapOp op, int a, int b) {
+  Tap t(v);
+  if (a < 0 && b < 0) return t;
+  tape().push_back({op, a, b});
+  t.id = (int)tape().size() - 1;
+  return t;
+}
+inline Tap operator+(Tap a, Tap b) { return tap_node(a.v + b.v, TAP_ADD, a.id, b.id); }
+inline Tap operator-(Tap a, Tap b) { return tap_node(a.v - b.v, TAP_SUB, a.id, b.id); }
+inline Tap operator-(Tap a) { return tap_node(-a.v, TAP_NEG, a.id, -1); }
+inline Tap operator*(Tap a, Tap b) { return tap_node(a.v * b.v, TAP_MUL, a.id, b.id); }
+inline Tap operator/(Tap a, Tap b) { return tap_node(a.v / b.v, TAP_DIV, a.id, b.id); }
+inline Tap sqrt(Tap a) { return tap_node(std::sqrt(a.v), TAP_SQRT, a.id, -1); }
+inline Tap log1p(Tap a) { return tap_node(std::log1p(a.v), TAP_LOG1P, a.id, -1); }
+inline Tap tanh(Tap a) { return tap_node(std::tanh(a.v), TAP_TANH, a.id, -1); }
+inline double value_of(Tap a) { return a.v; }
+
+// Operations of the reverse sweep over the tape, from the given output nodes back to the leaves,
+// for the nodes on a path between them.  Per node, with z its result and zb its adjoint:
+//   z = a +- b:  ab += zb, bb +-= zb                  1 add per marked operand
+//   z = -a:      ab -= zb                             1 add
+//   z = a b:     ab += zb b, bb += zb a               1 mul + 1 add per marked operand
+//   z = a / b:   t = zb / b;  ab += t;  bb -= t z     1 div, + 1 add (a), + 1 mul + 1 add (b)
+//   z = sqrt a:  ab += 0.5 (zb / z)                   1 div + 1 mul + 1 add
+//   z = log1p a: ab += zb / (1 + a)                   2 add + 1 div
+//   z = tanh a:  ab += zb (1 - z z)                   2 mul + 2 add
+inline OpTally tally_reverse_sweep(const int* outputs, int nout) {
+  const std::vector<TapNode>& t = tape();
+  std::vector<char> live(t.size(), 0);
+  for (int i = 0; i < nout; ++i)
+    if (outputs[i] >= 0) live[outputs[i]] = 1;
+  OpTally c;
+  for (int n = (int)t.size() - 1; n >= 0; --n) {
+    if (!live[n]) continue;
+    const TapNode& d = t[n];
+    const bool ua = d.a >= 0, ub = d.b >= 0;
+    if (ua) live[d.a] = 1;
+    if (ub) live[d.b] = 1;
+    switch (d.op) {
+      case TAP_LEAF: break;
+      case TAP_ADD: case TAP_SUB: c.add += ua + ub; break;
+      case TAP_NEG: c.add += 1; break;
+      case TAP_MUL: c.mul += ua + ub; c.add += ua + ub; break;
+      case TAP_DIV: c.div += 1; c.add += ua + ub; c.mul += ub; break;
+      case TAP_SQRT: c.div += 1; c.mul += 1; c.add += 1; break;
+      case TAP_LOG1P: c.add += 2; c.div += 1; break;
+      case TAP_TANH: c.mul += 2; c.add += 2; break;
+    }
+  }
+  return c;
+}
+
+// ------------------------------------------------------------------------------------------
 // Fields.  Each is autonomous: dy/dt = f(y; theta).  D = state size, M = parameter count.
 // ------------------------------------------------------------------------------------------
 

@@ -237,12 +237,13 @@ OP_NAMES = ("add", "mul", "div", "sqrt", "log1p", "tanh")
 
 def count_ops(field, what, theta, y, h=0.1):
     """Tally of one f evaluation (what='f'), Tsit5 trial ('tsit5'), ROS34PW2 trial ('ros') or f
-    with one tangent direction by the forward-mode rules ('f_dual')."""
+    with one tangent direction by the forward-mode rules ('f_dual'), or the plain reverse sweep
+    of f's vector-Jacobian product with respect to (y, theta) ('vjp_reverse')."""
     D, M = dims(field)
     theta = np.ascontiguousarray(theta, np.float64).reshape(M)
     y = np.ascontiguousarray(y, np.float64).reshape(D)
     counts = np.zeros(6, np.int64)
-    rc = lib().orc_count_ops(FIELDS[field], {"f": 0, "tsit5": 1, "ros": 2, "f_dual": 3}[what], _p(theta),
+    rc = lib().orc_count_ops(FIELDS[field], {"f": 0, "tsit5": 1, "ros": 2, "f_dual": 3, "vjp_reverse": 4}[what], _p(theta),
                              _p(y), h, _p(counts))
     assert rc == 0, rc
     return dict(zip(OP_NAMES, counts.tolist()))

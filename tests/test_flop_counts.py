@@ -104,3 +104,26 @@ def test_field_counts_are_plausible(counts):
     assert ops(counts["lorenz63"]["f"]) == 8
     assert counts["nfw_mn"]["f"]["log1p"] == 1 and counts["nfw_mn"]["f"]["sqrt"] == 3
     assert counts["nfw_mn"]["f"]["div"] == 1
+
+
+@pytest.mark.parametrize("field", ["nfw_mn", "lorenz63", "lotka_volterra", "log_halo",
+                                   "robertson", "hires"])
+def test_vjp_counts_within_the_plain_reverse_sweep(counts, orc, field):
+    # The vector-Jacobian products the throughput figures charge (c_v, counted from the kernels'
+    # own source) must not exceed what a plain reverse-mode sweep over the oracle's f costs: the
+    # oracle tapes its own f and tallies the adjoint rules of every recorded operation.  A
+    # hand-written pullback doing redundant work would exceed that bound and inflate the reported
+    # fraction of peak; this pins c_v from outside the kernel source.
+    D, M = orc.dims(field)
+    rng = np.random.default_rng(4)
+    rev = orc.count_ops(field, "vjp_reverse", rng.uniform(0.5, 1.5, M), rng.uniform(0.5, 1.5, D))
+    kernel = ops(counts[field]["vjp"])
+    print("%s: c_v kernel %d, plain reverse sweep %d" % (field, kernel, sum(rev.values())))
+    assert kernel <= sum(rev.values())
+
+
+def test_mlp_vjp_count_within_the_plain_reverse_sweep(orc):
+    D, M = orc.dims("mlp")
+    rng = np.random.default_rng(5)
+    rev = orc.count_ops("mlp", "vjp_reverse", rng.normal(size=M) * 0.2, rng.normal(size=D))
+    assert 5316 <= sum(rev.values())   # the hand count of test_mlp_hand_count
