@@ -106,8 +106,9 @@ PIPE_BUSY_NCU = {
 TRAFFIC_SENS_PER_TRAJ = {"log_halo": 91.1}
 # library kernels per step: record = k_solve + 2 k_max_int + 3 prefix scans of 3 kernels each
 # (step offsets, chunk offsets, length bins) + k_chunk_table + k_bin_count + k_bin_scatter (15);
-# replay gradient = k_adjoint (1).
-LAUNCHES_PER_STEP = 16
+# replay gradient = k_theta_check + k_replay_forward (exits at once: the theta is the recorded one)
+# + k_adjoint (3).
+LAUNCHES_PER_STEP = 18
 
 
 def fp64_peak_tflops(mhz):
@@ -281,25 +282,38 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline_sample(seconds_target=15.0):
-    """Oracle throughput (record + replay gradient) on a bounded sample, all host threads."""
+def cpu_baseline_sample(seconds_target=15.0, single_core_n=1 << 14):
+    """Oracle throughput (record + replay gradient) on a bounded sample, all host threads; and on
+    one thread over the first 2^14 trajectories of the same ensemble, scaled linearly."""
     from differentiable_adaptive_ode_b200 import workloads as W
     from oracle import oracle as orc
     nthreads = orc.host_threads()
-    n = 256
-    while True:
-        w = W.nfw_mn(N=n)
+
+    def run(w, threads):
         t0 = time.perf_counter()
         r = orc.solve(w.field, w.method, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol,
-                      keep_record=True, nthreads=nthreads)
+                      keep_record=True, nthreads=threads)
         lam = W.loss_cotangent(w, r["y1"], w.target)
-        orc.replay_grad(w.field, w.method, w.theta, w.y0, r["H"], r["S"], lam, nthreads=nthreads)
-        dt = time.perf_counter() - t0
+        orc.replay_grad(w.field, w.method, w.theta, w.y0, r["H"], r["S"], lam, nthreads=threads)
+        return time.perf_counter() - t0
+
+    n = 256
+    while True:
+        dt = run(W.nfw_mn(N=n), nthreads)
         if dt > seconds_target / 4 or n >= 1 << 16:
-            return {"value": n / dt, "unit": UNIT, "cores": nthreads, "kind": "oracle",
-                    "sample": "%d trajectories of the 2^20 stellar ensemble (record solve + "
-                              "replay gradient), %.1f s" % (n, dt)}
+            break
         n *= 2
+    out = {"value": n / dt, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+           "sample": "%d trajectories of the 2^20 stellar ensemble (record solve + replay "
+                     "gradient), %.1f s" % (n, dt)}
+    if single_core_n:
+        w1 = W.subset(W.nfw_mn(), np.arange(single_core_n))
+        dt1 = run(w1, 1)
+        out["single_core"] = {"value": single_core_n / dt1, "unit": UNIT, "cores": 1,
+                              "sample": "the first %d trajectories of the 2^20 stellar ensemble "
+                                        "on one thread, %.1f s" % (single_core_n, dt1),
+                              "full_ensemble_s_scaled": dt1 * (1 << 20) / single_core_n}
+    return out
 
 
 # Per-workload constants: the field/method, the FP pipe that bounds the hot kernels and the
@@ -686,6 +700,48 @@ def main():
     loss_cotangent()
     grad_ms = timeit(lambda: G.gs_replay_grad(rec, th, lam, gt, gy))
     breakdown = {"forward_only": fwd_ms, "record": rec_ms, "replay_grad": grad_ms, "step": ms_step}
+
+    # a record made from nothing ([GS] §4.7 reports the one-time record separately): a new record
+    # object per repetition -- its allocations, a pool sized by default for 64 steps per
+    # trajectory (trajectories that find it full are parked and resumed once it has grown), no
+    # longest-first order yet -- then the first gradient.  Wall-clock through completion.
+    def fresh(with_grad):
+        best = None
+        for _ in range(3):
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            r = G.Record()
+            G.gs_solve_record(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, rec=r)
+            if with_grad:
+                loss_cotangent()
+                G.gs_replay_grad(r, th, lam, gt, gy)
+            torch.cuda.synchronize()
+            dt_ = (time.perf_counter() - t0) * 1e3
+            breakdown["fresh_record_solve_kernels"] = r.info().solve_ms
+            r.close()
+            best = dt_ if best is None else min(best, dt_)
+        return best
+
+    def reused_wall():
+        best = None
+        for _ in range(3):
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            G.gs_solve_record(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, rec=rec)
+            torch.cuda.synchronize()
+            dt_ = (time.perf_counter() - t0) * 1e3
+            best = dt_ if best is None else min(best, dt_)
+        return best
+
+    breakdown["fresh_record_wall"] = fresh(False)
+    breakdown["fresh_record_plus_first_gradient_wall"] = fresh(True)
+    breakdown["reused_record_wall"] = reused_wall()
+    # the same forward-only solve started in index order: what a first solve, which knows no
+    # longest-first order yet, pays for scheduling alone
+    ident = torch.arange(N, dtype=torch.int32, device=dev)
+    breakdown["forward_only_index_order"] = timeit(
+        lambda: G.gs_solve_forward(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, S, rj, stt,
+                                   opts=G.options(start_order=ident)))
     if w.field != "mlp":
         # outputs at 8 requested times ([GS] §3.4) and the gradient of a loss on them
         tau = [w.t0 + (w.t1 - w.t0) * (j + 1) / 8.0 for j in range(8)]

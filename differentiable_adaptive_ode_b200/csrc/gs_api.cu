@@ -188,8 +188,16 @@ struct gs_record {
   long long* offsets = nullptr;
   long long* choff = nullptr;
   long long* tiles = nullptr;  // scan scratch (tile totals) + grand totals
-  int* counters = nullptr;     // [0] queue [1] chunk count [2] overflow [3] max S [4] max status
+  int* counters = nullptr;     // [0] queue [1] chunk count [2] parked [3] max S [4] max status
   int* host = nullptr;         // pinned mirror of counters, then offsets[N] at host+8
+  // trajectories parked by a record pass whose pool ran out: two id lists (one written while the
+  // other is resumed) and the parked states
+  int* park_list[2] = {nullptr, nullptr};
+  void* park_r = nullptr;
+  int* park_i = nullptr;
+  long long* park_att = nullptr;
+  int64_t park_n = 0;
+  size_t park_r_bytes = 0;
   // visiting order of the replay kernels (longest records first) and its counting-sort scratch
   int* perm = nullptr;
   int64_t perm_cap = 0;
@@ -239,6 +247,64 @@ gs_status ensure_traj_arrays(gs_record* r, int64_t N) {
   if (!r->counters) GS_CUDA(cudaMalloc(&r->counters, 16 * sizeof(int)));
   if (!r->host) GS_CUDA(cudaMallocHost(&r->host, 16 * sizeof(int)));
   r->n_cap = n;
+  return GS_OK;
+}
+
+gs_status ensure_park(gs_record* r, int64_t N) {
+  const int64_t n = std::max<int64_t>(N, 1);
+  const size_t rb = (size_t)n * (2 + 2 * r->sys.d) * r->rsz;
+  if (r->park_n >= n && r->park_r_bytes >= rb) return GS_OK;
+  free_ptr(r->park_list[0]); free_ptr(r->park_list[1]); free_ptr(r->park_r);
+  free_ptr(r->park_i); free_ptr(r->park_att);
+  r->park_list[0] = r->park_list[1] = nullptr;
+  r->park_r = nullptr;
+  r->park_i = nullptr;
+  r->park_att = nullptr;
+  r->park_n = 0;
+  r->park_r_bytes = 0;
+  GS_CUDA(cudaMalloc(&r->park_list[0], n * sizeof(int)));
+  GS_CUDA(cudaMalloc(&r->park_list[1], n * sizeof(int)));
+  GS_CUDA(cudaMalloc(&r->park_r, rb));
+  GS_CUDA(cudaMalloc(&r->park_i, n * 4 * sizeof(int)));
+  GS_CUDA(cudaMalloc(&r->park_att, n * sizeof(long long)));
+  r->park_n = n;
+  r->park_r_bytes = rb;
+  return GS_OK;
+}
+
+// Enlarges the pool to `chunks`, keeping the first `keep` chunks (entries and labels).
+gs_status grow_pool(gs_record* r, int64_t chunks, int64_t keep, cudaStream_t s) {
+  if (chunks > 0x7fffffffLL)
+    return fail(GS_ERR_CAPACITY, "record needs %lld chunks, more than 2^31-1", (long long)chunks);
+  const size_t cb = (size_t)r->C * r->E * r->rsz;
+  void* pool = nullptr;
+  int *traj = nullptr, *seq = nullptr, *table = nullptr;
+  auto undo = [&]() {
+    free_ptr(pool); free_ptr(traj); free_ptr(seq); free_ptr(table);
+  };
+  if (cudaMalloc(&pool, (size_t)chunks * cb) != cudaSuccess ||
+      cudaMalloc(&traj, chunks * sizeof(int)) != cudaSuccess ||
+      cudaMalloc(&seq, chunks * sizeof(int)) != cudaSuccess ||
+      cudaMalloc(&table, chunks * sizeof(int)) != cudaSuccess) {
+    undo();
+    return fail(GS_ERR_CUDA, "cannot grow the record pool to %lld chunks", (long long)chunks);
+  }
+  if (keep > 0 &&
+      (cudaMemcpyAsync(pool, r->pool, (size_t)keep * cb, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+       cudaMemcpyAsync(traj, r->chunk_traj, keep * sizeof(int), cudaMemcpyDeviceToDevice, s) !=
+           cudaSuccess ||
+       cudaMemcpyAsync(seq, r->chunk_seq, keep * sizeof(int), cudaMemcpyDeviceToDevice, s) !=
+           cudaSuccess ||
+       cudaStreamSynchronize(s) != cudaSuccess)) {
+    undo();
+    return fail(GS_ERR_CUDA, "record pool copy failed");
+  }
+  free_ptr(r->pool); free_ptr(r->chunk_traj); free_ptr(r->chunk_seq); free_ptr(r->chunk_table);
+  r->pool = pool;
+  r->chunk_traj = traj;
+  r->chunk_seq = seq;
+  r->chunk_table = table;
+  r->pool_chunks = r->chunk_arrays_cap = chunks;
   return GS_OK;
 }
 
@@ -329,6 +395,9 @@ struct SolveCall {
   const void* sens0 = nullptr;  // forward sensitivities (Tsit5 forward solve only)
   void* sens1 = nullptr;
   const int* order = nullptr;   // visiting order of the trajectories (null: index order)
+  int64_t nqueue = -1;          // queue positions to visit (-1: N)
+  int resume = 0;               // record pass resuming the trajectories listed in `order`
+  int park_list = 0;            // which of the record's two park lists receives new parks
 };
 
 template <class F, class R, int METHOD>
@@ -346,16 +415,24 @@ gs_status launch_solve(const SolveCall& c) {
   p.status = c.status;
   p.queue = c.queue;
   p.order = c.order;
+  p.nqueue = (int)(c.nqueue < 0 ? c.N : c.nqueue);
+  if (c.rec) {
+    p.pool = static_cast<R*>(c.rec->pool);
+    p.chunk_traj = c.rec->chunk_traj;
+    p.chunk_seq = c.rec->chunk_seq;
+    p.pool_chunks = (int)c.rec->pool_chunks;
+    p.chunk_count = c.rec->counters + 1;
+    p.park_count = c.rec->counters + 2;
+    p.park_list = c.rec->park_list[c.park_list];
+    p.park_r = static_cast<R*>(c.rec->park_r);
+    p.park_i = c.rec->park_i;
+    p.park_att = c.rec->park_att;
+    p.resume = c.resume;
+  }
   if constexpr (std::is_same_v<F, gs::FMlpWarp>) {
     if (c.rec) {
-      p.pool = static_cast<R*>(c.rec->pool);
-      p.chunk_traj = c.rec->chunk_traj;
-      p.chunk_seq = c.rec->chunk_seq;
-      p.pool_chunks = (int)c.rec->pool_chunks;
-      p.chunk_count = c.rec->counters + 1;
-      p.overflow = c.rec->counters + 2;
       auto kern = gs::k_solve_mlp<R, true>;
-      kern<<<persistent_grid(kern, 0, c.N * 32), BLOCK, 0, c.stream>>>(p);
+      kern<<<persistent_grid(kern, 0, (long long)p.nqueue * 32), BLOCK, 0, c.stream>>>(p);
     } else {
       auto kern = gs::k_solve_mlp<R, false>;
       kern<<<persistent_grid(kern, 0, c.N * 32), BLOCK, 0, c.stream>>>(p);
@@ -364,16 +441,10 @@ gs_status launch_solve(const SolveCall& c) {
     return GS_OK;
   } else {
     if (c.rec) {
-      p.pool = static_cast<R*>(c.rec->pool);
-      p.chunk_traj = c.rec->chunk_traj;
-      p.chunk_seq = c.rec->chunk_seq;
-      p.pool_chunks = (int)c.rec->pool_chunks;
-      p.chunk_count = c.rec->counters + 1;
-      p.overflow = c.rec->counters + 2;
       const size_t smem = gs::solve_smem_bytes<F, R, true>();
       auto kern = gs::k_solve<F, R, METHOD, true>;
       GS_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-      const int grid = persistent_grid(kern, smem, c.N);
+      const int grid = persistent_grid(kern, smem, p.nqueue);
       kern<<<grid, BLOCK, smem, c.stream>>>(p);
     } else if (c.sens1) {
       if constexpr (METHOD == gs::M_TSIT5) {
@@ -837,25 +908,37 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
   if (!r->ev0 && (cudaEventCreate(&r->ev0) != cudaSuccess || cudaEventCreate(&r->ev1) != cudaSuccess))
     return bail(fail(GS_ERR_CUDA, "cudaEventCreate failed"));
   r->solve_ms = 0;
-  for (int pass = 0; pass < 2; ++pass) {
-    if (cudaMemsetAsync(r->counters, 0, 16 * sizeof(int), s) != cudaSuccess)
-      return bail(fail(GS_ERR_CUDA, "cudaMemsetAsync failed"));
+  if ((st = ensure_park(r, N)) != GS_OK) return bail(st);
+  if (cudaMemsetAsync(r->counters, 0, 16 * sizeof(int), s) != cudaSuccess)
+    return bail(fail(GS_ERR_CUDA, "cudaMemsetAsync failed"));
+  // A record that is made again for an ensemble of the same size starts its trajectories in the
+  // previous solve's longest-first order: long trajectories begin early instead of forming the
+  // tail of the launch.  Scheduling only -- every trajectory's result is independent of it.
+  const int* order0 = (opt && opt->start_order) ? opt->start_order : (order_ok ? r->perm : nullptr);
+  // Pass 0 solves every trajectory.  When the pool runs out, the trajectories that find it full
+  // are parked before their next attempt; the pool then grows (its contents kept) by an estimate
+  // of what they still need, and the next pass resumes only them from their parked states.
+  int64_t nq = N;
+  int list = 0;
+  int64_t pass_start = 0;  // chunks handed out before this pass
+  const int nb = (int)((N + 255) / 256);
+  for (int pass = 0;; ++pass) {
     SolveCall c{N, theta, sys->theta_shared, y0, t0, t1, rtol, atol, attempts_of(opt), y1,
                 r->nsteps, nullptr, status_out, r->counters, r, s};
-    // a record that is made again for an ensemble of the same size starts its trajectories in the
-    // previous solve's longest-first order: long trajectories begin early instead of forming the
-    // tail of the launch.  Scheduling only -- every trajectory's result is independent of it.
-    if (opt && opt->start_order) c.order = opt->start_order;
-    else if (order_ok) c.order = r->perm;
+    c.order = pass == 0 ? order0 : r->park_list[list ^ 1];
+    c.nqueue = nq;
+    c.resume = pass > 0;
+    c.park_list = list;
     cudaEventRecord(r->ev0, s);
     st = dispatch(*sys, [&]<class F, class R, int METHOD>() { return launch_solve<F, R, METHOD>(c); });
     if (st != GS_OK) return bail(st);
     cudaEventRecord(r->ev1, s);
+    // summary over the ensemble (complete once no trajectory is parked): statuses, the longest
+    // record, the worst status, the step offsets
     if (status_out != r->status &&
         cudaMemcpyAsync(r->status, status_out, N * sizeof(int), cudaMemcpyDeviceToDevice, s) !=
             cudaSuccess)
       return bail(fail(GS_ERR_CUDA, "status copy failed"));
-    const int nb = (int)((N + 255) / 256);
     gs::k_max_int<<<nb, 256, 0, s>>>(r->nsteps, (int)N, r->counters + 3);
     gs::k_max_int<<<nb, 256, 0, s>>>(r->status, (int)N, r->counters + 4);
     if ((st = scan_counts<0>(r->nsteps, (int)N, C, r->offsets, r->tiles, s)) != GS_OK) return bail(st);
@@ -869,21 +952,56 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
       return bail(fail(GS_ERR_CUDA, "record solve failed: %s", cudaGetErrorString(e)));
     float pass_ms = 0;
     if (cudaEventElapsedTime(&pass_ms, r->ev0, r->ev1) == cudaSuccess) r->solve_ms += pass_ms;
-    const int used = r->host[1];
-    const int overflow = r->host[2];
-    if (!overflow) {
-      r->nchunks = std::min<int64_t>(used, r->pool_chunks);  // reserved, some possibly unused
+    const int64_t used = std::min<int64_t>(r->host[1], r->pool_chunks);
+    const int parked = r->host[2];
+    if (parked == 0) {
+      r->nchunks = used;  // reserved, some possibly unused
       r->max_steps = r->host[3];
       long long tot;
       std::memcpy(&tot, r->host + 8, sizeof(tot));
       r->total_steps = tot;
       break;
     }
-    if (pass == 1) return bail(fail(GS_ERR_CAPACITY, "record pool overflow after resize"));
-    // room for the steps plus every warp's partly used chunk reservation
-    const int64_t warps = (int64_t)(N + 31) / 32;
-    if ((st = ensure_pool(r, (int64_t)used + (used >> 4) + gs::CHUNK_BATCH * std::min<int64_t>(warps, 1 << 16) + 1024)) != GS_OK)
-      return bail(st);
+    if (pass >= 64) return bail(fail(GS_ERR_CAPACITY, "record pool still full after %d passes", pass));
+    // what the parked trajectories still need: from their progress, and for those parked before
+    // their first step twice the mean use of the trajectories that did start in this pass
+    unsigned long long* est = reinterpret_cast<unsigned long long*>(r->counters + 10);
+    if (cudaMemsetAsync(est, 0, 2 * sizeof(unsigned long long), s) != cudaSuccess)
+      return bail(fail(GS_ERR_CUDA, "cudaMemsetAsync failed"));
+    const int eb = (parked + 255) / 256;
+    if (rsz == 8)
+      gs::k_park_estimate<double><<<eb, 256, 0, s>>>(r->park_list[list], parked,
+                                                    static_cast<const double*>(r->park_r), r->park_i,
+                                                    sys->d, t0, t1, C, est);
+    else
+      gs::k_park_estimate<float><<<eb, 256, 0, s>>>(r->park_list[list], parked,
+                                                   static_cast<const float*>(r->park_r), r->park_i,
+                                                   sys->d, (float)t0, (float)t1, C, est);
+    unsigned long long hest[2] = {0, 0};
+    if (cudaMemcpyAsync(hest, est, sizeof(hest), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return bail(fail(GS_ERR_CUDA, "park estimate failed"));
+    const int64_t unstarted = (int64_t)hest[1];
+    const int64_t started = std::max<int64_t>(1, nq - unstarted);
+    const int64_t per_new = 2 * std::max<int64_t>(used - pass_start, 1) / started + 2;
+    const int64_t warps = std::min<int64_t>((nq + 31) / 32, 1 << 16);
+    // progress is a poor guide where early steps are short (a stiff start): the pool at most
+    // triples per pass, so a wild estimate costs a pass, not the device's memory
+    const int64_t extra = std::max<int64_t>(
+        std::min<int64_t>((int64_t)hest[0] + unstarted * per_new, 2 * used + 1024), 2 * parked);
+    const int64_t want = used + extra + (int64_t)gs::CHUNK_BATCH * warps + 1024;
+    if ((st = grow_pool(r, want, used, s)) != GS_OK) return bail(st);
+    // the next pass: the parked trajectories, a fresh queue, park count and summary, and chunks
+    // handed out after the kept ones
+    r->host[0] = (int)used;
+    if (cudaMemsetAsync(r->counters, 0, 5 * sizeof(int), s) != cudaSuccess ||
+        cudaMemcpyAsync(r->counters + 1, r->host, sizeof(int), cudaMemcpyHostToDevice, s) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return bail(fail(GS_ERR_CUDA, "counter reset failed"));
+    pass_start = used;
+    nq = parked;
+    list ^= 1;
   }
   // chunk offsets and table
   if ((st = scan_counts<1>(r->nsteps, (int)N, C, r->choff, r->tiles, s)) != GS_OK) return bail(st);
@@ -1335,6 +1453,8 @@ void gs_record_destroy(gs_record* r) {
   free_ptr(r->red_scratch); free_ptr(r->red_partials); free_ptr(r->y1_scratch);
   free_ptr(r->theta_kept);
   free_ptr(r->perm); free_ptr(r->bins); free_ptr(r->binoff); free_ptr(r->btiles);
+  free_ptr(r->park_list[0]); free_ptr(r->park_list[1]); free_ptr(r->park_r);
+  free_ptr(r->park_i); free_ptr(r->park_att);
   if (r->host) cudaFreeHost(r->host);
   if (r->ev0) cudaEventDestroy(r->ev0);
   if (r->ev1) cudaEventDestroy(r->ev1);

@@ -42,10 +42,17 @@ GS_DHD double log1p_q(double x, double a, double b) {
 }
 GS_DHD float log1p_q(float x, float, float) { return log1pf(x); }
 
-// a * b rounded on its own: in fp64 on the device the product is never fused into a later sum.
+// a * b and a + b rounded on their own: on the device the product is never fused into a later
+// sum, nor the sum into an earlier product.  Written with these (and explicit fma), an expression
+// rounds the same way in every kernel that inlines it, whatever the compiler could otherwise merge
+// or fuse around it.
 template <class R> GS_DHD R mul_rn(R a, R b) { return a * b; }
+template <class R> GS_DHD R add_rn(R a, R b) { return a + b; }
 #ifdef __CUDA_ARCH__
 template <> GS_DHD double mul_rn<double>(double a, double b) { return __dmul_rn(a, b); }
+template <> GS_DHD float mul_rn<float>(float a, float b) { return __fmul_rn(a, b); }
+template <> GS_DHD double add_rn<double>(double a, double b) { return __dadd_rn(a, b); }
+template <> GS_DHD float add_rn<float>(float a, float b) { return __fadd_rn(a, b); }
 #endif
 
 template <class R>
@@ -62,6 +69,10 @@ struct Dl {
     return Dl(a.v - b.v, a.d - b.d);
   }
   friend GS_DHD Dl operator-(const Dl& a) { return Dl(-a.v, -a.d); }
+  // a b + c: d = a' b + a b' + c'
+  friend GS_DHD Dl fma(const Dl& a, const Dl& b, const Dl& c) {
+    return Dl(fma(a.v, b.v, c.v), fma(a.d, b.v, fma(a.v, b.d, c.d)));
+  }
   friend GS_DHD Dl operator*(const Dl& a, const Dl& b) {
     return Dl(a.v * b.v, fma(a.d, b.v, a.v * b.d));
   }

@@ -275,32 +275,34 @@ struct FNfwMiyamotoNagai {
     t.b2 = t.b * t.b;
   }
   // Quantities of f shared with the VJP; one division, three reciprocal square roots, one log1p.
+  // Every rounding is spelled out (explicit fma, mul_rn, add_rn): f is inlined into the solve,
+  // record and sensitivity kernels, and must round the same way in each of them.
   template <class R> struct Inter { R R2, r, ir, L, isr, gN, iB, apB, iD, gM; };
   template <class R> GS_HD static void inter(const R* y, const Theta<R>& t, Inter<R>& I) {
     const R x = y[0], yy = y[1], z = y[2];
-    I.R2 = x * x + yy * yy;
-    const R r2 = I.R2 + z * z;
+    I.R2 = fma(x, x, mul_rn(yy, yy));
+    const R r2 = fma(z, z, I.R2);
     I.ir = rsqrt(r2);
-    I.r = r2 * I.ir;
-    I.isr = R(1) / (t.rs + I.r);
+    I.r = mul_rn(r2, I.ir);
+    I.isr = R(1) / add_rn(t.rs, I.r);
     I.L = log1p_q(mul_rn(I.r, t.irs), t.rs, I.isr);  // rs / (rs + r) = 1 / (1 + r / rs)
-    I.gN = t.Mh * (I.ir * I.ir) * (I.L * I.ir - I.isr);
-    const R B2 = z * z + t.b2;
+    I.gN = mul_rn(mul_rn(t.Mh, mul_rn(I.ir, I.ir)), fma(I.L, I.ir, -I.isr));
+    const R B2 = fma(z, z, t.b2);
     I.iB = rsqrt(B2);
-    I.apB = t.a + B2 * I.iB;
-    I.iD = rsqrt(I.R2 + I.apB * I.apB);
-    I.gM = t.Md * (I.iD * I.iD * I.iD);
+    I.apB = fma(B2, I.iB, t.a);
+    I.iD = rsqrt(fma(I.apB, I.apB, I.R2));
+    I.gM = mul_rn(t.Md, mul_rn(mul_rn(I.iD, I.iD), I.iD));
   }
   template <class R> GS_HD static void f(const R* y, const Theta<R>& t, R* dy) {
     Inter<R> I;
     inter(y, t, I);
-    const R g = I.gN + I.gM;
+    const R g = add_rn(I.gN, I.gM);
     dy[0] = y[3];
     dy[1] = y[4];
     dy[2] = y[5];
-    dy[3] = -g * y[0];
-    dy[4] = -g * y[1];
-    dy[5] = -(I.gN + I.gM * I.apB * I.iB) * y[2];
+    dy[3] = -mul_rn(g, y[0]);
+    dy[4] = -mul_rn(g, y[1]);
+    dy[5] = -mul_rn(fma(mul_rn(I.gM, I.apB), I.iB, I.gN), y[2]);
   }
   // Tape of a stage for the reverse sweep: the five transcendental results of f at that stage,
   // so that the VJP recomputes only products and sums.
@@ -315,13 +317,13 @@ struct FNfwMiyamotoNagai {
     Inter<R> I;
     inter(y, t, I);
     tp[0] = I.ir; tp[1] = I.L; tp[2] = I.isr; tp[3] = I.iB; tp[4] = I.iD;
-    const R g = I.gN + I.gM;
+    const R g = add_rn(I.gN, I.gM);
     dy[0] = y[3];
     dy[1] = y[4];
     dy[2] = y[5];
-    dy[3] = -g * y[0];
-    dy[4] = -g * y[1];
-    dy[5] = -(I.gN + I.gM * I.apB * I.iB) * y[2];
+    dy[3] = -mul_rn(g, y[0]);
+    dy[4] = -mul_rn(g, y[1]);
+    dy[5] = -mul_rn(fma(mul_rn(I.gM, I.apB), I.iB, I.gN), y[2]);
   }
   template <class R>
   GS_HD static void vjp_tape(const R* y, const Theta<R>& t, const R* tp, const R* kb, R* yb,

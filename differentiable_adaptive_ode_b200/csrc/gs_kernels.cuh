@@ -89,13 +89,23 @@ struct SolveParams {
   int* status;
   int* queue;        // work counter
   const int* order;  // trajectory visited at queue position q (null: q itself)
+  int nqueue;        // queue positions to visit: N, or the number of parked trajectories resumed
   // record (REC only)
   R* pool;
   int* chunk_traj;
   int* chunk_seq;
   int pool_chunks;   // capacity in chunks
   int* chunk_count;  // bump allocator
-  int* overflow;     // set to 1 when the pool ran out
+  // Trajectories that found the pool exhausted are parked before their next attempt, with every
+  // accepted step so far written: their ids go to park_list (park_count of them) and their state
+  // to the per-trajectory park arrays.  A pass with resume = 1 visits park_list entries (order)
+  // and continues each from its parked state instead of starting it.
+  int* park_count;
+  int* park_list;      // [N]
+  R* park_r;           // [N][2 + 2D]: t, h, y, the slope f(y) carried into the next attempt
+  int* park_i;         // [N][4]: accepted steps, rejected trials, next chunk sequence, last rejected
+  long long* park_att; // [N] attempts so far
+  int resume;
   // forward sensitivities (SENS only): S = dy/dtheta, [N][D][M]; sens0 may be null (zero start)
   const R* sens0;
   R* sens1;
@@ -132,26 +142,26 @@ __device__ R initial_step(const R (&y0)[F::D], const R (&f0)[F::D],
                           const typename F::template Theta<R>& th, R t0, R t1, R rtol, R atol,
                           int p) {
   constexpr int D = F::D;
-  R s0 = R(0), s1 = R(0);
+  // roundings spelled out (explicit fma, mul_rn, add_rn) so that every kernel starts alike
+  R s0 = R(0), s1 = R(0), sc[D];
 #pragma unroll
   for (int i = 0; i < D; ++i) {
-    const R sc = atol + rtol * fabs(y0[i]);
-    const R a = y0[i] / sc, b = f0[i] / sc;
-    s0 += a * a;
-    s1 += b * b;
+    sc[i] = add_rn(atol, mul_rn(rtol, fabs(y0[i])));
+    const R a = y0[i] / sc[i], b = f0[i] / sc[i];
+    s0 = fma(a, a, s0);
+    s1 = fma(b, b, s1);
   }
   const R d0 = sqrt(s0 / R(D)), d1 = sqrt(s1 / R(D));
-  const R h0 = (d0 < R(1e-5) || d1 < R(1e-5)) ? R(1e-6) : R(0.01) * d0 / d1;
+  const R h0 = (d0 < R(1e-5) || d1 < R(1e-5)) ? R(1e-6) : mul_rn(R(0.01), d0) / d1;
   R y1[D], f1[D];
 #pragma unroll
-  for (int i = 0; i < D; ++i) y1[i] = y0[i] + h0 * f0[i];
+  for (int i = 0; i < D; ++i) y1[i] = fma(h0, f0[i], y0[i]);
   F::f(y1, th, f1);
   R s2 = R(0);
 #pragma unroll
   for (int i = 0; i < D; ++i) {
-    const R sc = atol + rtol * fabs(y0[i]);
-    const R q = (f1[i] - f0[i]) / sc;
-    s2 += q * q;
+    const R q = add_rn(f1[i], -f0[i]) / sc[i];
+    s2 = fma(q, q, s2);
   }
   const R d2 = sqrt(s2 / R(D)) / h0;
   const R dm = d1 > d2 ? d1 : d2;   // same selection as max(d1, d2) with d1 first
@@ -297,10 +307,10 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
         int base = 0;
         if (lane == 0) base = atomicAdd(p.queue, 32);
         base = __shfl_sync(FULL, base, 0);
-        if (base + 32 >= p.N) exhausted = true;
+        if (base + 32 >= p.nqueue) exhausted = true;
         const int q = base + lane;
         int id = q;
-        bool valid = q < p.N;
+        bool valid = q < p.nqueue;
         if (valid && p.order) {
           id = p.order[q];
           valid = id >= 0 && id < p.N;   // a caller's order entry outside the ensemble is skipped
@@ -309,7 +319,13 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
         R h0 = R(0), f0[D];
 #pragma unroll
         for (int c = 0; c < D; ++c) f0[c] = R(0);
-        if (valid) {
+        if (REC && valid && p.resume) {
+          // a parked trajectory: its start-up is done; it brings its step and carried slope
+          const R* pr = p.park_r + (size_t)id * (2 + 2 * D);
+          h0 = pr[1];
+#pragma unroll
+          for (int c = 0; c < D; ++c) f0[c] = pr[2 + D + c];
+        } else if (valid) {
           typename F::template Theta<R> th0;
           F::load(th0, p.theta + (size_t)p.theta_stride * id);
           R yy[D];
@@ -348,10 +364,21 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
 #pragma unroll
         for (int c = 0; c < D; ++c) k1[c] = ring->f0[c][slot];
         F::load(th, p.theta + (size_t)p.theta_stride * k);
+        ns = 0;
+        if (REC && p.resume) {
+          const R* pr = p.park_r + (size_t)k * (2 + 2 * D);
+          t = pr[0];
 #pragma unroll
-        for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
-        t = p.t0;
-        S = 0; Rj = 0; att = 0; last_rej = false; ns = 0; seq = 0;
+          for (int c = 0; c < D; ++c) y[c] = pr[2 + c];
+          const int* pi = p.park_i + (size_t)k * 4;
+          S = pi[0]; Rj = pi[1]; seq = pi[2]; last_rej = pi[3] != 0;
+          att = p.park_att[k];
+        } else {
+#pragma unroll
+          for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
+          t = p.t0;
+          S = 0; Rj = 0; att = 0; last_rej = false; seq = 0;
+        }
         if constexpr (SENS) {
           for (int i = 0; i < D * SM; ++i)
             sens[i * 128] = p.sens0 ? p.sens0[(size_t)k * D * SM + i] : R(0);
@@ -372,10 +399,12 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
     }
     if (!__any_sync(FULL, k >= 0) && exhausted && head == tail) break;
 
-    // ---- direct record: a lane about to attempt a step without a chunk takes one from this
-    // warp's reserved block (a new block of CHUNK_BATCH from the global bump counter only when
-    // the current one runs out) and labels it with its trajectory and sequence number
-    if constexpr (DIRECT) {
+    // ---- record: a lane about to attempt a step without a chunk takes one from this warp's
+    // reserved block (a new block of CHUNK_BATCH from the global bump counter only when the
+    // current one runs out) and labels it with its trajectory and sequence number.  When the pool
+    // is exhausted the trajectory is parked instead, before the attempt: every step it accepted
+    // so far is in its chunks, and its state goes to the park arrays for a later pass.
+    if constexpr (REC) {
       const bool needc = k >= 0 && cur < 0;
       const unsigned cm = __ballot_sync(FULL, needc);
       if (cm) {
@@ -394,12 +423,22 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
           cnext += nwant;
         }
         if (needc) {
-          cur = mychunk;
-          if (cur < p.pool_chunks) {
+          if (mychunk < p.pool_chunks) {
+            cur = mychunk;
             p.chunk_traj[cur] = k;
             p.chunk_seq[cur] = seq;
           } else {
-            *p.overflow = 1;
+            const int at = atomicAdd(p.park_count, 1);
+            p.park_list[at] = k;
+            R* pr = p.park_r + (size_t)k * (2 + 2 * D);
+            pr[0] = t;
+            pr[1] = h;
+#pragma unroll
+            for (int c = 0; c < D; ++c) { pr[2 + c] = y[c]; pr[2 + D + c] = k1[c]; }
+            int* pi = p.park_i + (size_t)k * 4;
+            pi[0] = S; pi[1] = Rj; pi[2] = seq; pi[3] = last_rej ? 1 : 0;
+            p.park_att[k] = att;
+            k = -1;
           }
         }
       }
@@ -407,7 +446,6 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
 
     // ---- one attempted step per active lane
     bool finishing = false;
-    int fin_traj = -1;
     if (k >= 0) {
       int st = -1;
       if (att >= p.max_attempts) {
@@ -506,13 +544,15 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
         }
       }
       if (st >= 0) {
-        if constexpr (DIRECT) {
+        if constexpr (REC) {
           // a chunk taken for an attempt that never came to be accepted is marked unused; a
-          // partly filled one keeps its entries
-          if (cur >= 0 && ns == 0 && cur < p.pool_chunks) p.chunk_traj[cur] = -1;
-          cur = -1;
-          ns = 0;
-          seq = 0;
+          // partly filled one keeps its entries (staged ones are flushed into it below)
+          if (cur >= 0 && ns == 0) p.chunk_traj[cur] = -1;
+          if (DIRECT || ns == 0) {
+            cur = -1;
+            ns = 0;
+            seq = 0;
+          }
         }
         if constexpr (SENS)
           for (int i = 0; i < D * SM; ++i) p.sens1[(size_t)k * D * SM + i] = sens[i * 128];
@@ -522,55 +562,35 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
         if (p.nrejected) p.nrejected[k] = Rj;
         if (p.status) p.status[k] = st;
         finishing = true;
-        fin_traj = k;
         k = -1;
       }
     }
 
-    // ---- staged record: flush full (or final partial) chunks, one warp-wide coalesced copy each
+    // ---- staged record: flush full (or final partial) chunks into their lanes' chunks, one
+    // warp-wide coalesced copy each
     if constexpr (STAGED) {
       const bool want = (ns == L::C) || (finishing && ns > 0);
-      const int owner = finishing ? fin_traj : k;
       unsigned fm = __ballot_sync(FULL, want);
       if (fm) {
-        // chunks come from this warp's reserved block; a new block of CHUNK_BATCH is reserved
-        // from the global bump counter only when the current one runs out
-        const int nwant = __popc(fm), rank = __popc(fm & lanemask_lt());
-        const int avail = cend - cnext;
-        int mychunk;
-        if (nwant > avail) {
-          int nb = 0;
-          if (lane == 0) nb = atomicAdd(p.chunk_count, CHUNK_BATCH);
-          nb = __shfl_sync(FULL, nb, 0);
-          mychunk = rank < avail ? cnext + rank : nb + (rank - avail);
-          cnext = nb + (nwant - avail);
-          cend = nb + CHUNK_BATCH;
-        } else {
-          mychunk = cnext + rank;
-          cnext += nwant;
-        }
-        if (want) {
-          if (mychunk < p.pool_chunks) {
-            p.chunk_traj[mychunk] = owner;
-            p.chunk_seq[mychunk] = seq;
-          } else {
-            *p.overflow = 1;
-          }
-        }
         __syncwarp();
         while (fm) {
           const int src = __ffs(fm) - 1;
           fm &= fm - 1;
-          const int ch = __shfl_sync(FULL, mychunk, src);
+          const int ch = __shfl_sync(FULL, cur, src);
           const int cnt = __shfl_sync(FULL, ns, src);
-          if (ch < p.pool_chunks) {
+          if (ch >= 0 && ch < p.pool_chunks) {
             R* dst = p.pool + (size_t)ch * (L::C * L::E);
             const R* s = stage + src * L::STAGE_STRIDE;
             for (int i = lane; i < cnt * L::E; i += 32) dst[i] = s[i];
           }
         }
         __syncwarp();
-        if (want) { ++seq; ns = 0; }
+        if (want) {
+          ++seq;
+          ns = 0;
+          cur = -1;
+          if (finishing) seq = 0;
+        }
       }
     }
   }
@@ -1031,6 +1051,26 @@ __global__ void k_chunk_table(const int* chunk_traj, const int* chunk_seq, int n
 #endif
       table[ti] = c;
     }
+  }
+}
+
+// Chunks the parked trajectories of a record pass still need, estimated from their progress:
+// a trajectory parked at time t after S accepted steps needs about S (t1 - t) / (t - t0) more
+// (taken with a 25 % margin); out[1] counts those parked before their first step.
+template <class R>
+__global__ void k_park_estimate(const int* list, int P, const R* park_r, const int* park_i, int D,
+                                R t0, R t1, int C, unsigned long long* out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= P) return;
+  const int k = list[i];
+  const R t = park_r[(size_t)k * (2 + 2 * D)];
+  const int S = park_i[(size_t)k * 4];
+  if (t > t0) {
+    const double rem = 1.25 * double(S + 1) * double(t1 - t) / double(t - t0);
+    const double ch = fmin(rem / C + 2.0, double(1 << 20));
+    atomicAdd(out, (unsigned long long)ch);
+  } else {
+    atomicAdd(out + 1, 1ull);
   }
 }
 

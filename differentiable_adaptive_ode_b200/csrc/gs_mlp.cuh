@@ -238,31 +238,73 @@ __global__ void __launch_bounds__(128) k_solve_mlp(SolveParams<R> p) {
   const R expo = R(-1.0 / double(Tsit5::err_order));
   const R eps = eps_of<R>();
   const R span = fabs(p.t1 - p.t0);
+  constexpr int PARKED = -2;
   for (;;) {
-    int k = 0;
-    if (lane == 0) k = atomicAdd(p.queue, 1);
-    k = __shfl_sync(FULL, k, 0);
-    if (k >= p.N) break;
+    int q = 0;
+    if (lane == 0) q = atomicAdd(p.queue, 1);
+    q = __shfl_sync(FULL, q, 0);
+    if (q >= p.nqueue) break;
+    const int k = p.order ? p.order[q] : q;
+    if (k < 0 || k >= p.N) continue;   // an order entry outside the ensemble is skipped
     R y[D], k1[D];
-#pragma unroll
-    for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
     R t = p.t0, h = R(0);
     int S = 0, Rj = 0, seq = 0, slot = 0, chunk = -1, st = -1;
     long long att = 0;
     bool last_rej = false;
-    if (!(p.t1 > p.t0)) {
-      st = 0;
-    } else {
-      FMlpWarp::f<R>(y, W, k1);
-      bool finite = true;
+    if (REC && p.resume) {
+      // a parked trajectory continues from its parked state (start-up already done)
+      const R* pr = p.park_r + (size_t)k * (2 + 2 * D);
+      t = pr[0];
+      h = pr[1];
 #pragma unroll
-      for (int c = 0; c < D; ++c) finite = finite && isfinite(y[c]) && isfinite(k1[c]);
-      if (!finite) st = 3;
-      else h = initial_step<FMlpWarp, R>(y, k1, W, p.t0, p.t1, p.rtol, p.atol, Tsit5::order);
+      for (int c = 0; c < D; ++c) { y[c] = pr[2 + c]; k1[c] = pr[2 + D + c]; }
+      const int* pi = p.park_i + (size_t)k * 4;
+      S = pi[0]; Rj = pi[1]; seq = pi[2]; last_rej = pi[3] != 0;
+      att = p.park_att[k];
+    } else {
+#pragma unroll
+      for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
+      if (!(p.t1 > p.t0)) {
+        st = 0;
+      } else {
+        FMlpWarp::f<R>(y, W, k1);
+        bool finite = true;
+#pragma unroll
+        for (int c = 0; c < D; ++c) finite = finite && isfinite(y[c]) && isfinite(k1[c]);
+        if (!finite) st = 3;
+        else h = initial_step<FMlpWarp, R>(y, k1, W, p.t0, p.t1, p.rtol, p.atol, Tsit5::order);
+      }
     }
     while (st < 0) {
       if (att >= p.max_attempts) { st = 1; break; }
       if (!(h >= R(16) * eps * fmax(fabs(t), span))) { st = 2; break; }
+      if (REC && chunk < 0) {
+        // the chunk for the next accepted steps is taken before the attempt; when the pool is
+        // exhausted the trajectory is parked here, every accepted step so far written
+        int ch = 0;
+        if (lane == 0) ch = atomicAdd(p.chunk_count, 1);
+        ch = __shfl_sync(FULL, ch, 0);
+        if (ch < p.pool_chunks) {
+          chunk = ch;
+          if (lane == 0) { p.chunk_traj[chunk] = k; p.chunk_seq[chunk] = seq; }
+          ++seq;
+        } else {
+          if (lane == 0) {
+            const int at = atomicAdd(p.park_count, 1);
+            p.park_list[at] = k;
+            R* pr = p.park_r + (size_t)k * (2 + 2 * D);
+            pr[0] = t;
+            pr[1] = h;
+#pragma unroll
+            for (int c = 0; c < D; ++c) { pr[2 + c] = y[c]; pr[2 + D + c] = k1[c]; }
+            int* pi = p.park_i + (size_t)k * 4;
+            pi[0] = S; pi[1] = Rj; pi[2] = seq; pi[3] = last_rej ? 1 : 0;
+            p.park_att[k] = att;
+          }
+          st = PARKED;
+          break;
+        }
+      }
       bool clipped = false;
       if (t + h > p.t1) { h = p.t1 - t; clipped = true; }
       ++att;
@@ -270,25 +312,13 @@ __global__ void __launch_bounds__(128) k_solve_mlp(SolveParams<R> p) {
       const R err = tsit5_trial<FMlpWarp, R>(y, h, W, k1, ynew, k7, p.rtol, p.atol);
       if (err <= R(1)) {
         if (REC) {
-          if (slot == 0) {
-            int ch = 0;
-            if (lane == 0) ch = atomicAdd(p.chunk_count, 1);
-            chunk = __shfl_sync(FULL, ch, 0);
-            if (chunk < p.pool_chunks) {
-              if (lane == 0) { p.chunk_traj[chunk] = k; p.chunk_seq[chunk] = seq; }
-            } else if (lane == 0) {
-              *p.overflow = 1;
-            }
-            ++seq;
-          }
-          if (chunk < p.pool_chunks) {
-            R* e = p.pool + ((size_t)chunk * L::C + slot) * L::E;
-            R v = (lane == 0) ? t : h;
+          R* e = p.pool + ((size_t)chunk * L::C + slot) * L::E;
+          R v = (lane == 0) ? t : h;
 #pragma unroll
-            for (int c = 0; c < D; ++c) v = (lane == 2 + c) ? y[c] : v;
-            if (lane < L::E) e[lane] = v;
-          }
+          for (int c = 0; c < D; ++c) v = (lane == 2 + c) ? y[c] : v;
+          if (lane < L::E) e[lane] = v;
           slot = (slot + 1 == L::C) ? 0 : slot + 1;
+          if (slot == 0) chunk = -1;
         }
         ++S;
         const R facmax = last_rej ? R(1) : R(10);
@@ -308,6 +338,9 @@ __global__ void __launch_bounds__(128) k_solve_mlp(SolveParams<R> p) {
         last_rej = true;
       }
     }
+    if (st == PARKED) continue;
+    // a chunk taken for an attempt that was never accepted is marked unused
+    if (REC && chunk >= 0 && slot == 0 && lane == 0) p.chunk_traj[chunk] = -1;
     if (lane < D) p.y1[(size_t)k * D + lane] = y[lane];
     if (lane == 0) {
       if (p.nsteps) p.nsteps[k] = S;

@@ -1,12 +1,14 @@
 """GPU parity at the benchmark sizes (sampled trajectories the oracle computes one by one) and the
 edge cases: empty and single-trajectory ensembles, a zero-length interval, non-finite parameters,
-the attempt cap, record reuse, the pool-overflow re-run, and zero-length padding steps in an
+the attempt cap, record reuse, trajectories parked by a full pool and resumed, and zero-length
+padding steps in an
 imported record ([GS] = "gradsolve: fast exact gradients for ODE ensembles on GPUs", §3: a step of
 size zero leaves the state and its derivative unchanged)."""
 import numpy as np
 import pytest
 
 import gpu_util as U
+from test_gpu_parity import _check_states
 from differentiable_adaptive_ode_b200 import gradsolve as G
 from differentiable_adaptive_ode_b200 import workloads as W
 
@@ -75,13 +77,68 @@ def test_full_size_sampled_parity(orc, name):
     assert U.rel_rows(gt[idx], rt, 1e-300).max() <= 1e-8
 
 
+def test_full_size_f32_stellar_sampled_parity(orc):
+    # the fp32 stellar ensemble at its benchmark size (2^20 orbits, rtol 1e-5, atol 1e-6): a sample
+    # of 256 orbits against the oracle in fp32 (counts and final states, held to the oracle's own
+    # one-ulp spread), then on the GPU's fp32 mesh the fixed-mesh states (oracle fp32 replay) and
+    # the gradient (the exact fp64 derivative of the replay over that mesh)
+    import torch
+    w = W.by_name("nfw_mn_f32")
+    rec, out = U.record(w)
+    assert np.all(out["status"] == 0)
+    idx = _sample(w.N, n=254, seed=3)
+    sub = W.subset(w, idx)
+    info = rec.info()
+    off = torch.empty(w.N + 1, dtype=torch.int64, device="cuda")
+    H = torch.empty(int(info.total_steps), dtype=torch.float32, device="cuda")
+    G.gs_record_export(rec, None, H, None, off)
+    torch.cuda.synchronize()
+    off = off.cpu().numpy()
+    S = np.diff(off)
+    Hn = H.cpu().numpy()
+    Hs = np.zeros((len(idx), S[idx].max()), np.float32)
+    for r_, k in enumerate(idx):
+        Hs[r_, :S[k]] = Hn[off[k]:off[k + 1]]
+    ref = orc.solve(sub.field, sub.method, sub.theta, sub.y0, sub.t0, sub.t1, sub.rtol, sub.atol,
+                    dtype=np.float32, nthreads=8)
+    _check_states(sub, dict(S=S[idx], y1=out["y1"][idx]), ref, orc)
+    # fixed mesh: the oracle's fp32 replay of the GPU mesh (spec bar 1e-4 per trajectory)
+    yrep = orc.replay(sub.field, sub.method, sub.theta, sub.y0, Hs, S[idx], dtype=np.float32,
+                      nthreads=8)
+    err = U.rel_rows(out["y1"][idx], yrep, sub.atol)
+    print("fp32 stellar 2^20, fixed-mesh states: p50 %.3g p99 %.3g max %.3g"
+          % (np.median(err), np.quantile(err, 0.99), err.max()))
+    assert np.quantile(err, 0.99) <= 1e-4 and err.max() <= 1e-3, err.max()
+    # gradient of the benchmark loss on the GPU mesh (spec bar 1e-3 per trajectory)
+    lam = W.loss_cotangent(w, out["y1"], _target(orc, w))
+    gy, gt = U.replay_grad(w, rec, lam)
+    th64 = sub.theta.astype(np.float32).astype(np.float64)
+    y064 = sub.y0.astype(np.float32).astype(np.float64)
+    ry, rt = orc.replay_grad(sub.field, sub.method, th64, y064, Hs.astype(np.float64), S[idx],
+                             lam[idx].astype(np.float32).astype(np.float64), nthreads=8)
+    # the oracle's own fp32 reverse sweep over the same mesh: how far fp32 rounding alone carries
+    # the gradient from the exact one on these orbits (amplified along the longer ones)
+    oy, ot = orc.replay_grad(sub.field, sub.method, sub.theta, sub.y0, Hs, S[idx],
+                             lam[idx].astype(np.float32), dtype=np.float32, nthreads=8)
+    for name, got, own, want in (("dL/dy0", gy[idx], oy, ry), ("dL/dtheta", gt[idx], ot, rt)):
+        rel = U.rel_rows(got, want, 1e-300)
+        rel_o = U.rel_rows(own, want, 1e-300)
+        print("fp32 stellar 2^20, %s against the exact derivative: GPU p50 %.3g p99 %.3g max %.3g;"
+              " oracle fp32 p50 %.3g p99 %.3g max %.3g; north-star 1e-3: %.1f%% within"
+              % (name, np.median(rel), np.quantile(rel, 0.99), rel.max(), np.median(rel_o),
+                 np.quantile(rel_o, 0.99), rel_o.max(), 100 * np.mean(rel <= 1e-3)))
+        assert np.median(rel) <= 1e-3
+        assert np.quantile(rel, 0.99) <= max(1e-3, 3 * np.quantile(rel_o, 0.99))
+        assert rel.max() <= max(1e-2, 3 * rel_o.max())
+
+
 def test_full_size_mlp_sampled_shared_gradient(orc):
     # the ensemble weight gradient is linear in dL/dy1: zero the cotangent outside a sample and
     # the GPU returns the sample's weight gradient, which the oracle computes directly
     import torch
     w = W.mlp()
     rec, out = U.record(w)
-    idx = _sample(w.N, n=16)
+    idx = _sample(w.N, n=126)
     sub = W.subset(w, idx)
     ref = orc.solve("mlp", "tsit5", w.theta, sub.y0, 0.0, 1.0, w.rtol, w.atol, dtype=np.float32,
                     theta_shared=True, nthreads=8)
@@ -93,10 +150,9 @@ def test_full_size_mlp_sampled_shared_gradient(orc):
     torch.cuda.synchronize()
     off = off.cpu().numpy()
     S = np.diff(off)
-    # fp32: accept decisions near err = 1 sit on the rounding floor (the oracle against itself
-    # under a one-ulp change of y0 keeps ~85 % of the counts on this ensemble)
-    assert np.all(np.abs(S[idx].astype(int) - ref["S"]) <= 1)
-    assert np.mean(S[idx] == ref["S"]) >= 0.5
+    # fp32: accept decisions near err = 1 sit on the rounding floor; counts and states are held to
+    # the oracle's own spread under a one-ulp change of y0, measured on the same sample
+    _check_states(sub, dict(S=S[idx], y1=out["y1"][idx]), ref, orc)
     tgt = _target(orc, w).astype(np.float32)
     lam = np.zeros((w.N, 4))
     lam[idx] = W.loss_cotangent(w, out["y1"], tgt)[idx]
@@ -151,7 +207,7 @@ def test_status_codes_and_failed_record():
 
 def test_record_reuse_and_overflow_rerun(orc):
     w = W.nfw_mn(N=700)
-    # a pool far too small: the solve runs again with the exact size; results unchanged
+    # a pool far too small: the parked trajectories resume in later passes; results unchanged
     rec, out = U.record(w, capacity=50)
     ex = U.export_padded(w, rec)
     ref = orc.solve(w.field, w.method, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol, nthreads=8)
@@ -164,6 +220,32 @@ def test_record_reuse_and_overflow_rerun(orc):
                      nthreads=8)
     assert np.array_equal(ex2["S"], ref2["S"])
     assert U.rel_rows(out2["y1"], ref2["y1"], w2.atol).max() <= 1e-9
+
+
+@pytest.mark.parametrize("name,N,capacity", [("nfw_mn", 700, 50),       # direct writes
+                                             ("lorenz63", 900, 8),      # staged writes
+                                             ("robertson", 300, 30),    # a Rosenbrock method
+                                             ("lorenz63_vern7", 500, 20),
+                                             ("mlp", 300, 16)])         # one warp per trajectory
+def test_record_resumes_parked_trajectories(name, N, capacity):
+    # A pool far too small: the trajectories that find it full are parked before their next
+    # attempt and resumed by later passes once the pool has grown.  The record, the final states
+    # and the gradient must equal those of a record made with room to spare, bit for bit.
+    w = W.by_name(name, N=N)
+    rec_a, out_a = U.record(w, capacity=capacity)
+    rec_b, out_b = U.record(w, capacity=400 * N)
+    ea, eb = U.export_padded(w, rec_a), U.export_padded(w, rec_b)
+    assert np.all(out_a["status"] == 0)
+    for key in ("S", "T", "H", "Y"):
+        assert np.array_equal(ea[key], eb[key]), key
+    assert np.array_equal(out_a["y1"], out_b["y1"])
+    assert ea["info"].total_steps == eb["info"].total_steps
+    assert ea["info"].max_steps == eb["info"].max_steps
+    lam = np.random.default_rng(3).normal(size=(w.N, w.d)).astype(w.dtype)
+    ga, gb = U.replay_grad(w, rec_a, lam), U.replay_grad(w, rec_b, lam)
+    assert np.array_equal(ga[0], gb[0])
+    if not w.theta_shared:   # a shared theta's sum is grouped by the visiting order
+        assert np.array_equal(ga[1], gb[1])
 
 
 def test_zero_steps_in_imported_record_change_nothing(orc):

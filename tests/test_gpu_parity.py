@@ -49,7 +49,8 @@ def _self_spread(orc, w):
     a = _oracle_solve(orc, w)
     b = orc.solve(w.field, w.method, w.theta, y0p, w.t0, w.t1, w.rtol, w.atol, dtype=w.dtype,
                   theta_shared=w.theta_shared, nthreads=8)
-    return U.rel_rows(a["y1"], b["y1"], w.atol), np.mean(a["S"] == b["S"])
+    dS = np.abs(a["S"].astype(int) - b["S"].astype(int))
+    return U.rel_rows(a["y1"], b["y1"], w.atol), np.mean(a["S"] == b["S"]), dS
 
 
 def _check_states(w, gpu, ref, orc=None):
@@ -68,13 +69,15 @@ def _check_states(w, gpu, ref, orc=None):
     # final states by up to ~1e-2.  The GPU must be as close to the oracle as the oracle is to
     # itself under that perturbation (the per-trajectory 1e-4 bar is applied on a fixed mesh, in
     # test_record_parity_and_replay).
-    spread, same_self = _self_spread(orc, w)
+    spread, same_self, dS_self = _self_spread(orc, w)
     q_gpu, q_self = np.quantile(err_all, 0.99), np.quantile(spread, 0.99)
-    print("%s: 1-ulp self spread p99 %.3g, identical counts %.3f; GPU p99 %.3g"
-          % (w.name, q_self, same_self, q_gpu))
+    print("%s: 1-ulp self spread p99 %.3g, identical counts %.3f, max |dS| %d; GPU p99 %.3g "
+          "(north-star 1e-4: %.1f%% of trajectories within)"
+          % (w.name, q_self, same_self, dS_self.max(), q_gpu, 100 * np.mean(err_all <= 1e-4)))
     assert q_gpu <= 3 * max(q_self, STATE_TOL[w.dtype]), (q_gpu, q_self)
     assert same.mean() >= same_self - 0.15, (same.mean(), same_self)
-    assert np.mean(dS <= 3) >= COUNT_FRAC, dS.max()
+    # count differences no wider than the oracle's own under a one-ulp change (at least 3)
+    assert np.mean(dS <= max(3, 2 * dS_self.max())) >= COUNT_FRAC, (dS.max(), dS_self.max())
 
 
 @pytest.mark.parametrize("name,N", SMALL)
