@@ -190,9 +190,11 @@ struct gs_record {
   long long* tiles = nullptr;  // scan scratch (tile totals) + grand totals
   int* counters = nullptr;     // [0] queue [1] chunk count [2] parked [3] max S [4] max status
   int* host = nullptr;         // pinned mirror of counters, then offsets[N] at host+8
-  // trajectories parked by a record pass whose pool ran out: two id lists (one written while the
-  // other is resumed) and the parked states
-  int* park_list[2] = {nullptr, nullptr};
+  // trajectories parked by a record pass (the pool ran out, or their first slice was done): their
+  // ids, their states, and their order for the next pass
+  int* park_list = nullptr;
+  int* park_key = nullptr;       // estimated remaining steps of each parked trajectory
+  int* park_order = nullptr;     // the parked trajectories by decreasing estimate
   void* park_r = nullptr;
   int* park_i = nullptr;
   long long* park_att = nullptr;
@@ -254,19 +256,21 @@ gs_status ensure_park(gs_record* r, int64_t N) {
   const int64_t n = std::max<int64_t>(N, 1);
   const size_t rb = (size_t)n * (2 + 2 * r->sys.d) * r->rsz;
   if (r->park_n >= n && r->park_r_bytes >= rb) return GS_OK;
-  free_ptr(r->park_list[0]); free_ptr(r->park_list[1]); free_ptr(r->park_r);
-  free_ptr(r->park_i); free_ptr(r->park_att);
-  r->park_list[0] = r->park_list[1] = nullptr;
+  free_ptr(r->park_list); free_ptr(r->park_r);
+  free_ptr(r->park_i); free_ptr(r->park_att); free_ptr(r->park_key); free_ptr(r->park_order);
+  r->park_list = nullptr;
+  r->park_key = r->park_order = nullptr;
   r->park_r = nullptr;
   r->park_i = nullptr;
   r->park_att = nullptr;
   r->park_n = 0;
   r->park_r_bytes = 0;
-  GS_CUDA(cudaMalloc(&r->park_list[0], n * sizeof(int)));
-  GS_CUDA(cudaMalloc(&r->park_list[1], n * sizeof(int)));
+  GS_CUDA(cudaMalloc(&r->park_list, n * sizeof(int)));
   GS_CUDA(cudaMalloc(&r->park_r, rb));
   GS_CUDA(cudaMalloc(&r->park_i, n * 4 * sizeof(int)));
   GS_CUDA(cudaMalloc(&r->park_att, n * sizeof(long long)));
+  GS_CUDA(cudaMalloc(&r->park_key, n * sizeof(int)));
+  GS_CUDA(cudaMalloc(&r->park_order, n * sizeof(int)));
   r->park_n = n;
   r->park_r_bytes = rb;
   return GS_OK;
@@ -342,6 +346,31 @@ gs_status scan_counts(const int* S, int N, int C, long long* out, long long* til
   return GS_OK;
 }
 
+// out[j] = the j-th of the n entries of keys (values in [0, kmax]) in decreasing order: the
+// entry's index, or ids[index] when ids is given.  Counting sort in the record's bin scratch.
+gs_status counting_sort_desc(gs_record* r, const int* keys, int64_t n, int kmax, const int* ids,
+                             int* out, cudaStream_t s) {
+  if (n <= 0) return GS_OK;
+  const int64_t nb = (int64_t)kmax + 1;
+  if (r->bins_cap < nb) {
+    free_ptr(r->bins); free_ptr(r->binoff); free_ptr(r->btiles);
+    r->bins = nullptr; r->binoff = r->btiles = nullptr;
+    r->bins_cap = 0;
+    GS_CUDA(cudaMalloc(&r->bins, 2 * nb * sizeof(int)));
+    GS_CUDA(cudaMalloc(&r->binoff, (nb + 1) * sizeof(long long)));
+    GS_CUDA(cudaMalloc(&r->btiles, (nb / gs::SCAN_BLOCK + 3) * sizeof(long long)));
+    r->bins_cap = nb;
+  }
+  GS_CUDA(cudaMemsetAsync(r->bins, 0, 2 * nb * sizeof(int), s));
+  const int grid = (int)((n + 255) / 256);
+  gs::k_bin_count<<<grid, 256, 0, s>>>(keys, (int)n, kmax, r->bins);
+  gs_status st = scan_counts<0>(r->bins, (int)nb, 1, r->binoff, r->btiles, s);
+  if (st != GS_OK) return st;
+  gs::k_bin_scatter<<<grid, 256, 0, s>>>(keys, (int)n, kmax, r->binoff, r->bins + nb, out, ids);
+  GS_CUDA(cudaGetLastError());
+  return GS_OK;
+}
+
 // perm = trajectories by decreasing S (needs r->nsteps, r->max_steps).
 gs_status build_perm(gs_record* r, cudaStream_t s) {
   const int64_t N = r->N;
@@ -353,24 +382,8 @@ gs_status build_perm(gs_record* r, cudaStream_t s) {
     GS_CUDA(cudaMalloc(&r->perm, N * sizeof(int)));
     r->perm_cap = N;
   }
-  const int64_t nb = (int64_t)r->max_steps + 1;
-  if (r->bins_cap < nb) {
-    free_ptr(r->bins); free_ptr(r->binoff); free_ptr(r->btiles);
-    r->bins = nullptr; r->binoff = r->btiles = nullptr;
-    r->bins_cap = 0;
-    GS_CUDA(cudaMalloc(&r->bins, 2 * nb * sizeof(int)));
-    GS_CUDA(cudaMalloc(&r->binoff, (nb + 1) * sizeof(long long)));
-    GS_CUDA(cudaMalloc(&r->btiles, (nb / gs::SCAN_BLOCK + 3) * sizeof(long long)));
-    r->bins_cap = nb;
-  }
-  GS_CUDA(cudaMemsetAsync(r->bins, 0, 2 * nb * sizeof(int), s));
-  const int grid = (int)((N + 255) / 256);
-  gs::k_bin_count<<<grid, 256, 0, s>>>(r->nsteps, (int)N, r->max_steps, r->bins);
-  gs_status st = scan_counts<0>(r->bins, (int)nb, 1, r->binoff, r->btiles, s);
+  gs_status st = counting_sort_desc(r, r->nsteps, N, r->max_steps, nullptr, r->perm, s);
   if (st != GS_OK) return st;
-  gs::k_bin_scatter<<<grid, 256, 0, s>>>(r->nsteps, (int)N, r->max_steps, r->binoff,
-                                         r->bins + nb, r->perm);
-  GS_CUDA(cudaGetLastError());
   r->perm_n = N;
   return GS_OK;
 }
@@ -397,7 +410,7 @@ struct SolveCall {
   const int* order = nullptr;   // visiting order of the trajectories (null: index order)
   int64_t nqueue = -1;          // queue positions to visit (-1: N)
   int resume = 0;               // record pass resuming the trajectories listed in `order`
-  int park_list = 0;            // which of the record's two park lists receives new parks
+  int slice = 0;                // record pass: attempts per trajectory before it is parked (0: all)
 };
 
 template <class F, class R, int METHOD>
@@ -423,11 +436,12 @@ gs_status launch_solve(const SolveCall& c) {
     p.pool_chunks = (int)c.rec->pool_chunks;
     p.chunk_count = c.rec->counters + 1;
     p.park_count = c.rec->counters + 2;
-    p.park_list = c.rec->park_list[c.park_list];
+    p.park_list = c.rec->park_list;
     p.park_r = static_cast<R*>(c.rec->park_r);
     p.park_i = c.rec->park_i;
     p.park_att = c.rec->park_att;
     p.resume = c.resume;
+    p.slice = c.slice;
   }
   if constexpr (std::is_same_v<F, gs::FMlpWarp>) {
     if (c.rec) {
@@ -892,11 +906,25 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
   r->t0 = t0;
   r->t1 = t1;
   if ((st = ensure_traj_arrays(r, N)) != GS_OK) return bail(st);
+  // A record that is made again for an ensemble of the same size starts its trajectories in the
+  // previous solve's longest-first order: long trajectories begin early instead of forming the
+  // tail of the launch.  Scheduling only -- every trajectory's result is independent of it.
+  const int* order0 = (opt && opt->start_order) ? opt->start_order : (order_ok ? r->perm : nullptr);
+  // With no order at hand (a first solve of this ensemble), every trajectory first takes a short
+  // slice of SLICE attempts; the rest of the record then resumes them by decreasing estimate of
+  // their remaining steps (from the progress of the slice), and the pool is sized from the same
+  // estimate.  The one-warp-per-trajectory neural field, and small ensembles, start in index order.
+  constexpr int SLICE = 16;
+  const bool slice_mode = !order0 && N >= 4096 && sys->field != GS_MLP_4_32_32_4;
+  const int64_t warps = std::min<int64_t>((std::max<int64_t>(N, 1) + 31) / 32, 1 << 16);
   int64_t want_chunks = r->pool_chunks;
   if (want_chunks == 0) {
-    const int64_t steps = (opt && opt->record_capacity_steps > 0) ? opt->record_capacity_steps
-                                                                   : std::max<int64_t>(N, 1) * 64;
-    want_chunks = (steps + C - 1) / C + std::max<int64_t>(N, 1);
+    if (opt && opt->record_capacity_steps > 0)
+      want_chunks = (opt->record_capacity_steps + C - 1) / C + std::max<int64_t>(N, 1);
+    else if (slice_mode)  // the slice: at most SLICE + C - 1 accepted steps, one chunk to spare
+      want_chunks = N * ((SLICE + 2 * C - 2) / C + 1) + (int64_t)gs::CHUNK_BATCH * warps + 1024;
+    else
+      want_chunks = (std::max<int64_t>(N, 1) * 64 + C - 1) / C + std::max<int64_t>(N, 1);
   }
   if ((st = ensure_pool(r, want_chunks)) != GS_OK) return bail(st);
   if (N == 0) {
@@ -911,24 +939,22 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
   if ((st = ensure_park(r, N)) != GS_OK) return bail(st);
   if (cudaMemsetAsync(r->counters, 0, 16 * sizeof(int), s) != cudaSuccess)
     return bail(fail(GS_ERR_CUDA, "cudaMemsetAsync failed"));
-  // A record that is made again for an ensemble of the same size starts its trajectories in the
-  // previous solve's longest-first order: long trajectories begin early instead of forming the
-  // tail of the launch.  Scheduling only -- every trajectory's result is independent of it.
-  const int* order0 = (opt && opt->start_order) ? opt->start_order : (order_ok ? r->perm : nullptr);
-  // Pass 0 solves every trajectory.  When the pool runs out, the trajectories that find it full
-  // are parked before their next attempt; the pool then grows (its contents kept) by an estimate
-  // of what they still need, and the next pass resumes only them from their parked states.
+  // Pass 0 takes every trajectory (in slice mode for SLICE attempts each).  Trajectories that are
+  // parked -- their slice spent, or the pool found full -- resume in the next pass from their
+  // parked states, by decreasing estimate of their remaining steps, after the pool has grown
+  // (its contents kept) by the estimate of what they still need.
   int64_t nq = N;
-  int list = 0;
   int64_t pass_start = 0;  // chunks handed out before this pass
   const int nb = (int)((N + 255) / 256);
+  constexpr int KMAX = 1 << 16;
   for (int pass = 0;; ++pass) {
+    const bool sliced = slice_mode && pass == 0;
     SolveCall c{N, theta, sys->theta_shared, y0, t0, t1, rtol, atol, attempts_of(opt), y1,
                 r->nsteps, nullptr, status_out, r->counters, r, s};
-    c.order = pass == 0 ? order0 : r->park_list[list ^ 1];
+    c.order = pass == 0 ? order0 : r->park_order;
     c.nqueue = nq;
     c.resume = pass > 0;
-    c.park_list = list;
+    c.slice = sliced ? SLICE : 0;
     cudaEventRecord(r->ev0, s);
     st = dispatch(*sys, [&]<class F, class R, int METHOD>() { return launch_solve<F, R, METHOD>(c); });
     if (st != GS_OK) return bail(st);
@@ -963,20 +989,25 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
       break;
     }
     if (pass >= 64) return bail(fail(GS_ERR_CAPACITY, "record pool still full after %d passes", pass));
-    // what the parked trajectories still need: from their progress, and for those parked before
-    // their first step twice the mean use of the trajectories that did start in this pass
+    // what the parked trajectories still need (from their progress; for those parked before
+    // their first step twice the mean use of the trajectories that did start in this pass), and
+    // their order for the next pass: largest estimate first
     unsigned long long* est = reinterpret_cast<unsigned long long*>(r->counters + 10);
     if (cudaMemsetAsync(est, 0, 2 * sizeof(unsigned long long), s) != cudaSuccess)
       return bail(fail(GS_ERR_CUDA, "cudaMemsetAsync failed"));
     const int eb = (parked + 255) / 256;
     if (rsz == 8)
-      gs::k_park_estimate<double><<<eb, 256, 0, s>>>(r->park_list[list], parked,
+      gs::k_park_estimate<double><<<eb, 256, 0, s>>>(r->park_list, parked,
                                                     static_cast<const double*>(r->park_r), r->park_i,
-                                                    sys->d, t0, t1, C, est);
+                                                    sys->d, t0, t1, C, est, r->park_key, KMAX);
     else
-      gs::k_park_estimate<float><<<eb, 256, 0, s>>>(r->park_list[list], parked,
+      gs::k_park_estimate<float><<<eb, 256, 0, s>>>(r->park_list, parked,
                                                    static_cast<const float*>(r->park_r), r->park_i,
-                                                   sys->d, (float)t0, (float)t1, C, est);
+                                                   sys->d, (float)t0, (float)t1, C, est,
+                                                   r->park_key, KMAX);
+    if ((st = counting_sort_desc(r, r->park_key, parked, KMAX, r->park_list, r->park_order, s)) !=
+        GS_OK)
+      return bail(st);
     unsigned long long hest[2] = {0, 0};
     if (cudaMemcpyAsync(hest, est, sizeof(hest), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
@@ -984,13 +1015,17 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
     const int64_t unstarted = (int64_t)hest[1];
     const int64_t started = std::max<int64_t>(1, nq - unstarted);
     const int64_t per_new = 2 * std::max<int64_t>(used - pass_start, 1) / started + 2;
-    const int64_t warps = std::min<int64_t>((nq + 31) / 32, 1 << 16);
-    // progress is a poor guide where early steps are short (a stiff start): the pool at most
-    // triples per pass, so a wild estimate costs a pass, not the device's memory
-    const int64_t extra = std::max<int64_t>(
-        std::min<int64_t>((int64_t)hest[0] + unstarted * per_new, 2 * used + 1024), 2 * parked);
+    int64_t extra = std::max<int64_t>((int64_t)hest[0] + unstarted * per_new, 2 * (int64_t)parked);
+    // after a pool found full the pool at most triples per pass, so that a wild estimate costs a
+    // pass, not the device's memory; and never beyond 80 % of the free device memory
+    if (!sliced) extra = std::min<int64_t>(extra, std::max<int64_t>(2 * used + 1024, 2 * (int64_t)parked));
+    size_t free_b = 0, total_b = 0;
+    const int64_t chunk_b = (int64_t)C * E * (int64_t)rsz + 3 * (int64_t)sizeof(int);
+    if (cudaMemGetInfo(&free_b, &total_b) == cudaSuccess)
+      extra = std::min<int64_t>(extra, std::max<int64_t>((int64_t)(free_b * 0.8) / chunk_b,
+                                                         2 * (int64_t)parked));
     const int64_t want = used + extra + (int64_t)gs::CHUNK_BATCH * warps + 1024;
-    if ((st = grow_pool(r, want, used, s)) != GS_OK) return bail(st);
+    if (want > r->pool_chunks && (st = grow_pool(r, want, used, s)) != GS_OK) return bail(st);
     // the next pass: the parked trajectories, a fresh queue, park count and summary, and chunks
     // handed out after the kept ones
     r->host[0] = (int)used;
@@ -1001,7 +1036,6 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
       return bail(fail(GS_ERR_CUDA, "counter reset failed"));
     pass_start = used;
     nq = parked;
-    list ^= 1;
   }
   // chunk offsets and table
   if ((st = scan_counts<1>(r->nsteps, (int)N, C, r->choff, r->tiles, s)) != GS_OK) return bail(st);
@@ -1453,8 +1487,8 @@ void gs_record_destroy(gs_record* r) {
   free_ptr(r->red_scratch); free_ptr(r->red_partials); free_ptr(r->y1_scratch);
   free_ptr(r->theta_kept);
   free_ptr(r->perm); free_ptr(r->bins); free_ptr(r->binoff); free_ptr(r->btiles);
-  free_ptr(r->park_list[0]); free_ptr(r->park_list[1]); free_ptr(r->park_r);
-  free_ptr(r->park_i); free_ptr(r->park_att);
+  free_ptr(r->park_list); free_ptr(r->park_r);
+  free_ptr(r->park_i); free_ptr(r->park_att); free_ptr(r->park_key); free_ptr(r->park_order);
   if (r->host) cudaFreeHost(r->host);
   if (r->ev0) cudaEventDestroy(r->ev0);
   if (r->ev1) cudaEventDestroy(r->ev1);

@@ -106,6 +106,9 @@ struct SolveParams {
   int* park_i;         // [N][4]: accepted steps, rejected trials, next chunk sequence, last rejected
   long long* park_att; // [N] attempts so far
   int resume;
+  // > 0: a trajectory that has made this many attempts in the pass is parked at its next chunk
+  // boundary (a first slice of every trajectory, whose progress orders the rest of the record)
+  int slice;
   // forward sensitivities (SENS only): S = dy/dtheta, [N][D][M]; sens0 may be null (zero start)
   const R* sens0;
   R* sens1;
@@ -243,6 +246,25 @@ template <class F, class R, bool REC, bool SENS = false>
 __host__ __device__ constexpr size_t solve_smem_bytes() {
   return ((REC && !RecDirect<F, R>::value) ? solve_stage_bytes<F, R>() : 0) +
          (SENS ? solve_sens_bytes<F, R>() : 0) + 4 * sizeof(StartRing<F, R>);
+}
+
+// Parks trajectory k: its id goes to the park list and its state (everything the next attempt
+// needs) to the park arrays, from which a later record pass resumes it.
+template <class F, class R>
+__device__ __forceinline__ void park_state(const SolveParams<R>& p, int k, R t, R h,
+                                           const R (&y)[F::D], const R (&k1)[F::D], int S, int Rj,
+                                           int seq, bool last_rej, long long att) {
+  constexpr int D = F::D;
+  const int at = atomicAdd(p.park_count, 1);
+  p.park_list[at] = k;
+  R* pr = p.park_r + (size_t)k * (2 + 2 * D);
+  pr[0] = t;
+  pr[1] = h;
+#pragma unroll
+  for (int c = 0; c < D; ++c) { pr[2 + c] = y[c]; pr[2 + D + c] = k1[c]; }
+  int* pi = p.park_i + (size_t)k * 4;
+  pi[0] = S; pi[1] = Rj; pi[2] = seq; pi[3] = last_rej ? 1 : 0;
+  p.park_att[k] = att;
 }
 
 // SENS = true (Tsit5, no record): the forward sensitivities S = dy/dtheta ride along with the
@@ -405,7 +427,10 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
     // is exhausted the trajectory is parked instead, before the attempt: every step it accepted
     // so far is in its chunks, and its state goes to the park arrays for a later pass.
     if constexpr (REC) {
-      const bool needc = k >= 0 && cur < 0;
+      // the slice of the first pass: a trajectory with p.slice attempts made is parked instead
+      // of taking a chunk (first passes start every trajectory afresh, so attempts count from 0)
+      const bool sliced = p.slice > 0 && att >= p.slice;
+      const bool needc = k >= 0 && cur < 0 && !sliced;
       const unsigned cm = __ballot_sync(FULL, needc);
       if (cm) {
         const int nwant = __popc(cm), rank = __popc(cm & lanemask_lt());
@@ -428,19 +453,14 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
             p.chunk_traj[cur] = k;
             p.chunk_seq[cur] = seq;
           } else {
-            const int at = atomicAdd(p.park_count, 1);
-            p.park_list[at] = k;
-            R* pr = p.park_r + (size_t)k * (2 + 2 * D);
-            pr[0] = t;
-            pr[1] = h;
-#pragma unroll
-            for (int c = 0; c < D; ++c) { pr[2 + c] = y[c]; pr[2 + D + c] = k1[c]; }
-            int* pi = p.park_i + (size_t)k * 4;
-            pi[0] = S; pi[1] = Rj; pi[2] = seq; pi[3] = last_rej ? 1 : 0;
-            p.park_att[k] = att;
+            park_state<F, R>(p, k, t, h, y, k1, S, Rj, seq, last_rej, att);
             k = -1;
           }
         }
+      }
+      if (k >= 0 && cur < 0 && sliced) {
+        park_state<F, R>(p, k, t, h, y, k1, S, Rj, seq, last_rej, att);
+        k = -1;
       }
     }
 
@@ -1056,21 +1076,27 @@ __global__ void k_chunk_table(const int* chunk_traj, const int* chunk_seq, int n
 
 // Chunks the parked trajectories of a record pass still need, estimated from their progress:
 // a trajectory parked at time t after S accepted steps needs about S (t1 - t) / (t - t0) more
-// (taken with a 25 % margin); out[1] counts those parked before their first step.
+// (at most 64 S; taken with a 25 % margin); out[1] counts those parked before their first step.  With `keys`,
+// keys[i] = that estimate of the remaining steps of list[i], capped at kmax (kmax for a
+// trajectory without progress): the order in which the next pass takes them, largest first.
 template <class R>
 __global__ void k_park_estimate(const int* list, int P, const R* park_r, const int* park_i, int D,
-                                R t0, R t1, int C, unsigned long long* out) {
+                                R t0, R t1, int C, unsigned long long* out, int* keys, int kmax) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= P) return;
   const int k = list[i];
   const R t = park_r[(size_t)k * (2 + 2 * D)];
   const int S = park_i[(size_t)k * 4];
   if (t > t0) {
-    const double rem = 1.25 * double(S + 1) * double(t1 - t) / double(t - t0);
-    const double ch = fmin(rem / C + 2.0, double(1 << 20));
+    // progress in time is a poor guide after a stiff start (tiny early steps): at most 64 times
+    // the steps taken so far
+    const double rem = fmin(double(S + 1) * double(t1 - t) / double(t - t0), 64.0 * (S + 1));
+    const double ch = fmin(1.25 * rem / C + 2.0, double(1 << 20));
     atomicAdd(out, (unsigned long long)ch);
+    if (keys) keys[i] = (int)fmin(rem, double(kmax));
   } else {
     atomicAdd(out + 1, 1ull);
+    if (keys) keys[i] = kmax;
   }
 }
 
@@ -1170,12 +1196,13 @@ __global__ void k_bin_count(const int* S, int N, int smax, int* bins) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < N) atomicAdd(&bins[smax - S[i]], 1);
 }
+// perm[position] = i (or ids[i] when ids is given), positions by decreasing S[i]
 __global__ void k_bin_scatter(const int* S, int N, int smax, const long long* binoff, int* cursor,
-                              int* perm) {
+                              int* perm, const int* ids) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < N) {
     const int b = smax - S[i];
-    perm[binoff[b] + atomicAdd(&cursor[b], 1)] = i;
+    perm[binoff[b] + atomicAdd(&cursor[b], 1)] = ids ? ids[i] : i;
   }
 }
 

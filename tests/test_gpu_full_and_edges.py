@@ -248,6 +248,35 @@ def test_record_resumes_parked_trajectories(name, N, capacity):
         assert np.array_equal(ga[1], gb[1])
 
 
+@pytest.mark.parametrize("name,N", [("nfw_mn", 6000), ("lorenz63", 8192), ("robertson", 4500),
+                                    ("nfw_mn_f32", 5000), ("hires", 4096)])
+def test_first_record_in_slices_equals_ordered_record(name, N):
+    # A first record of an ensemble (no order known) runs a slice of every trajectory, then
+    # resumes them by decreasing estimate of their remaining steps, in a pool sized from that
+    # estimate.  Scheduling only: it must equal, bit for bit, a record started from a caller's
+    # order in one pass.
+    import torch
+    w = W.by_name(name, N=N)
+    rec_a, out_a = U.record(w)
+    dt = U.tdtype(w)
+    y1 = torch.empty((w.N, w.d), dtype=dt, device="cuda")
+    order = torch.arange(w.N, dtype=torch.int32, device="cuda")
+    rec_b = G.gs_solve_record(U.gsys(w), w.N, U.dev(w.theta, dt), U.dev(w.y0, dt), w.t0, w.t1,
+                              w.rtol, w.atol, y1,
+                              opts=G.options(record_capacity_steps=400 * w.N, start_order=order))
+    torch.cuda.synchronize()
+    ea, eb = U.export_padded(w, rec_a), U.export_padded(w, rec_b)
+    for key in ("S", "T", "H", "Y"):
+        assert np.array_equal(ea[key], eb[key]), key
+    assert np.array_equal(out_a["y1"], y1.cpu().numpy())
+    assert ea["info"].max_steps == eb["info"].max_steps
+    lam = np.random.default_rng(4).normal(size=(w.N, w.d)).astype(w.dtype)
+    ga, gb = U.replay_grad(w, rec_a, lam), U.replay_grad(w, rec_b, lam)
+    assert np.array_equal(ga[0], gb[0])
+    if not w.theta_shared:
+        assert np.array_equal(ga[1], gb[1])
+
+
 def test_zero_steps_in_imported_record_change_nothing(orc):
     w = W.lorenz63(N=50)
     ref = orc.solve(w.field, w.method, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol, keep_record=True)
