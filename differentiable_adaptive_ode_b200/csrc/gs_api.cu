@@ -93,12 +93,16 @@ gs_status check_system(const gs_system* sys) {
 
 // Per-device library state, created on first use and kept until exit: the SM count, a ring of
 // work-queue counters (each call takes its own slot, zeroes it on its stream and hands it to its
-// kernel, so calls on different streams never share a counter), and cached occupancy figures.
+// kernel, so calls on different streams never share a counter), cached occupancy figures, and
+// the stream-ordered memory pool that records draw their device storage from.  The pool keeps
+// the storage of destroyed records for the next ones (a new record then costs no driver
+// allocation, and destroying one no synchronous free) until gs_memory_trim hands it back.
 struct DeviceCtx {
   std::once_flag once;
   cudaError_t init_err = cudaSuccess;
   int sms = 148;
   int* ring = nullptr;
+  cudaMemPool_t mempool = nullptr;
   std::atomic<unsigned> next{0};
   std::mutex occ_mu;
   std::unordered_map<const void*, int> occ;
@@ -119,9 +123,31 @@ DeviceCtx* device_ctx(cudaError_t* err) {
   std::call_once(c.once, [&]() {
     c.init_err = cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev);
     if (c.init_err == cudaSuccess) c.init_err = cudaMalloc(&c.ring, RING * sizeof(int));
+    if (c.init_err == cudaSuccess) {
+      cudaMemPoolProps props = {};
+      props.allocType = cudaMemAllocationTypePinned;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      c.init_err = cudaMemPoolCreate(&c.mempool, &props);
+    }
+    if (c.init_err == cudaSuccess) {
+      uint64_t keep = UINT64_MAX;  // released storage stays in the pool until trimmed
+      c.init_err = cudaMemPoolSetAttribute(c.mempool, cudaMemPoolAttrReleaseThreshold, &keep);
+    }
   });
   *err = c.init_err;
   return c.init_err == cudaSuccess ? &c : nullptr;
+}
+
+// Device storage of a record: from the device's pool, ordered on stream s (usable by work on s
+// at once, by other streams after s has reached this point).
+template <class T>
+cudaError_t dalloc(T** p, size_t bytes, cudaStream_t s) {
+  cudaError_t e;
+  DeviceCtx* c = device_ctx(&e);
+  if (!c) return e;
+  return cudaMallocFromPoolAsync(reinterpret_cast<void**>(p), std::max<size_t>(bytes, 1), c->mempool,
+                                 s);
 }
 
 // A zeroed work counter for one launch on stream s.
@@ -189,7 +215,7 @@ struct gs_record {
   long long* choff = nullptr;
   long long* tiles = nullptr;  // scan scratch (tile totals) + grand totals
   int* counters = nullptr;     // [0] queue [1] chunk count [2] parked [3] max S [4] max status
-  int* host = nullptr;         // pinned mirror of counters, then offsets[N] at host+8
+  int host[16] = {};           // read-back of counters, then offsets[N] at host+8
   // trajectories parked by a record pass (the pool ran out, or their first slice was done): their
   // ids, their states, and their order for the next pass
   int* park_list = nullptr;
@@ -229,35 +255,36 @@ struct gs_record {
 
 namespace {
 
-void free_ptr(void* p) {
-  if (p) cudaFree(p);
+// Returns record storage to the pool once the work queued on stream s before this point is done.
+void free_ptr(void* p, cudaStream_t s) {
+  if (p) cudaFreeAsync(p, s);
 }
 
-gs_status ensure_traj_arrays(gs_record* r, int64_t N) {
+gs_status ensure_traj_arrays(gs_record* r, int64_t N, cudaStream_t s) {
   if (r->n_cap >= N && r->counters) return GS_OK;
-  free_ptr(r->nsteps); free_ptr(r->status); free_ptr(r->offsets); free_ptr(r->choff);
-  free_ptr(r->tiles);
+  free_ptr(r->nsteps, s); free_ptr(r->status, s); free_ptr(r->offsets, s); free_ptr(r->choff, s);
+  free_ptr(r->tiles, s);
   r->nsteps = r->status = nullptr;
   r->offsets = r->choff = r->tiles = nullptr;
   const int64_t n = std::max<int64_t>(N, 1);
   const int64_t ntiles = (n + gs::SCAN_BLOCK - 1) / gs::SCAN_BLOCK;
-  GS_CUDA(cudaMalloc(&r->nsteps, n * sizeof(int)));
-  GS_CUDA(cudaMalloc(&r->status, n * sizeof(int)));
-  GS_CUDA(cudaMalloc(&r->offsets, (n + 1) * sizeof(long long)));
-  GS_CUDA(cudaMalloc(&r->choff, (n + 1) * sizeof(long long)));
-  GS_CUDA(cudaMalloc(&r->tiles, (ntiles + 2) * sizeof(long long)));
-  if (!r->counters) GS_CUDA(cudaMalloc(&r->counters, 16 * sizeof(int)));
-  if (!r->host) GS_CUDA(cudaMallocHost(&r->host, 16 * sizeof(int)));
+  GS_CUDA(dalloc(&r->nsteps, n * sizeof(int), s));
+  GS_CUDA(dalloc(&r->status, n * sizeof(int), s));
+  GS_CUDA(dalloc(&r->offsets, (n + 1) * sizeof(long long), s));
+  GS_CUDA(dalloc(&r->choff, (n + 1) * sizeof(long long), s));
+  GS_CUDA(dalloc(&r->tiles, (ntiles + 2) * sizeof(long long), s));
+  if (!r->counters) GS_CUDA(dalloc(&r->counters, 16 * sizeof(int), s));
   r->n_cap = n;
   return GS_OK;
 }
 
-gs_status ensure_park(gs_record* r, int64_t N) {
+gs_status ensure_park(gs_record* r, int64_t N, cudaStream_t s) {
   const int64_t n = std::max<int64_t>(N, 1);
   const size_t rb = (size_t)n * (2 + 2 * r->sys.d) * r->rsz;
   if (r->park_n >= n && r->park_r_bytes >= rb) return GS_OK;
-  free_ptr(r->park_list); free_ptr(r->park_r);
-  free_ptr(r->park_i); free_ptr(r->park_att); free_ptr(r->park_key); free_ptr(r->park_order);
+  free_ptr(r->park_list, s); free_ptr(r->park_r, s);
+  free_ptr(r->park_i, s); free_ptr(r->park_att, s); free_ptr(r->park_key, s);
+  free_ptr(r->park_order, s);
   r->park_list = nullptr;
   r->park_key = r->park_order = nullptr;
   r->park_r = nullptr;
@@ -265,12 +292,12 @@ gs_status ensure_park(gs_record* r, int64_t N) {
   r->park_att = nullptr;
   r->park_n = 0;
   r->park_r_bytes = 0;
-  GS_CUDA(cudaMalloc(&r->park_list, n * sizeof(int)));
-  GS_CUDA(cudaMalloc(&r->park_r, rb));
-  GS_CUDA(cudaMalloc(&r->park_i, n * 4 * sizeof(int)));
-  GS_CUDA(cudaMalloc(&r->park_att, n * sizeof(long long)));
-  GS_CUDA(cudaMalloc(&r->park_key, n * sizeof(int)));
-  GS_CUDA(cudaMalloc(&r->park_order, n * sizeof(int)));
+  GS_CUDA(dalloc(&r->park_list, n * sizeof(int), s));
+  GS_CUDA(dalloc(&r->park_r, rb, s));
+  GS_CUDA(dalloc(&r->park_i, n * 4 * sizeof(int), s));
+  GS_CUDA(dalloc(&r->park_att, n * sizeof(long long), s));
+  GS_CUDA(dalloc(&r->park_key, n * sizeof(int), s));
+  GS_CUDA(dalloc(&r->park_order, n * sizeof(int), s));
   r->park_n = n;
   r->park_r_bytes = rb;
   return GS_OK;
@@ -284,12 +311,12 @@ gs_status grow_pool(gs_record* r, int64_t chunks, int64_t keep, cudaStream_t s) 
   void* pool = nullptr;
   int *traj = nullptr, *seq = nullptr, *table = nullptr;
   auto undo = [&]() {
-    free_ptr(pool); free_ptr(traj); free_ptr(seq); free_ptr(table);
+    free_ptr(pool, s); free_ptr(traj, s); free_ptr(seq, s); free_ptr(table, s);
   };
-  if (cudaMalloc(&pool, (size_t)chunks * cb) != cudaSuccess ||
-      cudaMalloc(&traj, chunks * sizeof(int)) != cudaSuccess ||
-      cudaMalloc(&seq, chunks * sizeof(int)) != cudaSuccess ||
-      cudaMalloc(&table, chunks * sizeof(int)) != cudaSuccess) {
+  if (dalloc(&pool, (size_t)chunks * cb, s) != cudaSuccess ||
+      dalloc(&traj, chunks * sizeof(int), s) != cudaSuccess ||
+      dalloc(&seq, chunks * sizeof(int), s) != cudaSuccess ||
+      dalloc(&table, chunks * sizeof(int), s) != cudaSuccess) {
     undo();
     return fail(GS_ERR_CUDA, "cannot grow the record pool to %lld chunks", (long long)chunks);
   }
@@ -298,12 +325,12 @@ gs_status grow_pool(gs_record* r, int64_t chunks, int64_t keep, cudaStream_t s) 
        cudaMemcpyAsync(traj, r->chunk_traj, keep * sizeof(int), cudaMemcpyDeviceToDevice, s) !=
            cudaSuccess ||
        cudaMemcpyAsync(seq, r->chunk_seq, keep * sizeof(int), cudaMemcpyDeviceToDevice, s) !=
-           cudaSuccess ||
-       cudaStreamSynchronize(s) != cudaSuccess)) {
+           cudaSuccess)) {
     undo();
     return fail(GS_ERR_CUDA, "record pool copy failed");
   }
-  free_ptr(r->pool); free_ptr(r->chunk_traj); free_ptr(r->chunk_seq); free_ptr(r->chunk_table);
+  free_ptr(r->pool, s); free_ptr(r->chunk_traj, s); free_ptr(r->chunk_seq, s);
+  free_ptr(r->chunk_table, s);
   r->pool = pool;
   r->chunk_traj = traj;
   r->chunk_seq = seq;
@@ -312,19 +339,20 @@ gs_status grow_pool(gs_record* r, int64_t chunks, int64_t keep, cudaStream_t s) 
   return GS_OK;
 }
 
-gs_status ensure_pool(gs_record* r, int64_t chunks) {
+gs_status ensure_pool(gs_record* r, int64_t chunks, cudaStream_t s) {
   if (chunks > 0x7fffffffLL)
     return fail(GS_ERR_CAPACITY, "record needs %lld chunks, more than 2^31-1", (long long)chunks);
   if (r->pool_chunks >= chunks && r->chunk_arrays_cap >= chunks) return GS_OK;
-  free_ptr(r->pool); free_ptr(r->chunk_traj); free_ptr(r->chunk_seq); free_ptr(r->chunk_table);
+  free_ptr(r->pool, s); free_ptr(r->chunk_traj, s); free_ptr(r->chunk_seq, s);
+  free_ptr(r->chunk_table, s);
   r->pool = nullptr;
   r->chunk_traj = r->chunk_seq = r->chunk_table = nullptr;
   r->pool_chunks = r->chunk_arrays_cap = 0;
   const int64_t c = std::max<int64_t>(chunks, 1);
-  GS_CUDA(cudaMalloc(&r->pool, (size_t)c * r->C * r->E * r->rsz));
-  GS_CUDA(cudaMalloc(&r->chunk_traj, c * sizeof(int)));
-  GS_CUDA(cudaMalloc(&r->chunk_seq, c * sizeof(int)));
-  GS_CUDA(cudaMalloc(&r->chunk_table, c * sizeof(int)));
+  GS_CUDA(dalloc(&r->pool, (size_t)c * r->C * r->E * r->rsz, s));
+  GS_CUDA(dalloc(&r->chunk_traj, c * sizeof(int), s));
+  GS_CUDA(dalloc(&r->chunk_seq, c * sizeof(int), s));
+  GS_CUDA(dalloc(&r->chunk_table, c * sizeof(int), s));
   r->pool_chunks = r->chunk_arrays_cap = c;
   return GS_OK;
 }
@@ -353,12 +381,12 @@ gs_status counting_sort_desc(gs_record* r, const int* keys, int64_t n, int kmax,
   if (n <= 0) return GS_OK;
   const int64_t nb = (int64_t)kmax + 1;
   if (r->bins_cap < nb) {
-    free_ptr(r->bins); free_ptr(r->binoff); free_ptr(r->btiles);
+    free_ptr(r->bins, s); free_ptr(r->binoff, s); free_ptr(r->btiles, s);
     r->bins = nullptr; r->binoff = r->btiles = nullptr;
     r->bins_cap = 0;
-    GS_CUDA(cudaMalloc(&r->bins, 2 * nb * sizeof(int)));
-    GS_CUDA(cudaMalloc(&r->binoff, (nb + 1) * sizeof(long long)));
-    GS_CUDA(cudaMalloc(&r->btiles, (nb / gs::SCAN_BLOCK + 3) * sizeof(long long)));
+    GS_CUDA(dalloc(&r->bins, 2 * nb * sizeof(int), s));
+    GS_CUDA(dalloc(&r->binoff, (nb + 1) * sizeof(long long), s));
+    GS_CUDA(dalloc(&r->btiles, (nb / gs::SCAN_BLOCK + 3) * sizeof(long long), s));
     r->bins_cap = nb;
   }
   GS_CUDA(cudaMemsetAsync(r->bins, 0, 2 * nb * sizeof(int), s));
@@ -376,10 +404,10 @@ gs_status build_perm(gs_record* r, cudaStream_t s) {
   const int64_t N = r->N;
   if (N <= 0) return GS_OK;
   if (r->perm_cap < N) {
-    free_ptr(r->perm);
+    free_ptr(r->perm, s);
     r->perm = nullptr;
     r->perm_cap = 0;
-    GS_CUDA(cudaMalloc(&r->perm, N * sizeof(int)));
+    GS_CUDA(dalloc(&r->perm, N * sizeof(int), s));
     r->perm_cap = N;
   }
   gs_status st = counting_sort_desc(r, r->nsteps, N, r->max_steps, nullptr, r->perm, s);
@@ -677,13 +705,13 @@ size_t theta_bytes(const gs_record* r) {
   return (size_t)(r->sys.theta_shared ? 1 : std::max<int64_t>(r->N, 1)) * r->sys.m * r->rsz;
 }
 
-gs_status ensure_theta_kept(gs_record* r) {
+gs_status ensure_theta_kept(gs_record* r, cudaStream_t s) {
   const size_t need = theta_bytes(r);
   if (r->theta_kept_bytes >= need) return GS_OK;
-  free_ptr(r->theta_kept);
+  free_ptr(r->theta_kept, s);
   r->theta_kept = nullptr;
   r->theta_kept_bytes = 0;
-  GS_CUDA(cudaMalloc(&r->theta_kept, need));
+  GS_CUDA(dalloc(&r->theta_kept, need, s));
   r->theta_kept_bytes = need;
   return GS_OK;
 }
@@ -771,10 +799,10 @@ static gs_status replay_grad_mlp(const gs_record* rec, const void* theta, const 
     if (dL_dtheta) {
       const size_t need = (size_t)nwarps * gs::MLP_M * sizeof(R);
       if (r->part_bytes < need) {
-        free_ptr(r->red_partials);
+        free_ptr(r->red_partials, s);
         r->red_partials = nullptr;
         r->part_bytes = 0;
-        GS_CUDA(cudaMalloc(&r->red_partials, need));
+        GS_CUDA(dalloc(&r->red_partials, need, s));
         r->part_bytes = need;
       }
       partials = static_cast<R*>(r->red_partials);
@@ -893,7 +921,8 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
   const size_t rsz = sys->dtype == GS_F64 ? 8 : 4;
   if (!fresh && (r->C != C || r->E != E || r->rsz != rsz)) {
     // a different layout: drop the old pool
-    free_ptr(r->pool); free_ptr(r->chunk_traj); free_ptr(r->chunk_seq); free_ptr(r->chunk_table);
+    free_ptr(r->pool, s); free_ptr(r->chunk_traj, s); free_ptr(r->chunk_seq, s);
+    free_ptr(r->chunk_table, s);
     r->pool = nullptr; r->chunk_traj = r->chunk_seq = r->chunk_table = nullptr;
     r->pool_chunks = r->chunk_arrays_cap = 0;
   }
@@ -905,7 +934,7 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
   r->rsz = rsz;
   r->t0 = t0;
   r->t1 = t1;
-  if ((st = ensure_traj_arrays(r, N)) != GS_OK) return bail(st);
+  if ((st = ensure_traj_arrays(r, N, s)) != GS_OK) return bail(st);
   // A record that is made again for an ensemble of the same size starts its trajectories in the
   // previous solve's longest-first order: long trajectories begin early instead of forming the
   // tail of the launch.  Scheduling only -- every trajectory's result is independent of it.
@@ -926,7 +955,7 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
     else
       want_chunks = (std::max<int64_t>(N, 1) * 64 + C - 1) / C + std::max<int64_t>(N, 1);
   }
-  if ((st = ensure_pool(r, want_chunks)) != GS_OK) return bail(st);
+  if ((st = ensure_pool(r, want_chunks, s)) != GS_OK) return bail(st);
   if (N == 0) {
     r->nchunks = r->total_steps = 0;
     r->max_steps = 0;
@@ -936,7 +965,7 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
   if (!r->ev0 && (cudaEventCreate(&r->ev0) != cudaSuccess || cudaEventCreate(&r->ev1) != cudaSuccess))
     return bail(fail(GS_ERR_CUDA, "cudaEventCreate failed"));
   r->solve_ms = 0;
-  if ((st = ensure_park(r, N)) != GS_OK) return bail(st);
+  if ((st = ensure_park(r, N, s)) != GS_OK) return bail(st);
   if (cudaMemsetAsync(r->counters, 0, 16 * sizeof(int), s) != cudaSuccess)
     return bail(fail(GS_ERR_CUDA, "cudaMemsetAsync failed"));
   // Pass 0 takes every trajectory (in slice mode for SLICE attempts each).  Trajectories that are
@@ -1021,9 +1050,20 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
     if (!sliced) extra = std::min<int64_t>(extra, std::max<int64_t>(2 * used + 1024, 2 * (int64_t)parked));
     size_t free_b = 0, total_b = 0;
     const int64_t chunk_b = (int64_t)C * E * (int64_t)rsz + 3 * (int64_t)sizeof(int);
-    if (cudaMemGetInfo(&free_b, &total_b) == cudaSuccess)
+    if (cudaMemGetInfo(&free_b, &total_b) == cudaSuccess) {
+      // storage the pool holds but no record uses counts as free
+      cudaError_t ce;
+      DeviceCtx* dc = device_ctx(&ce);
+      uint64_t held = 0, inuse = 0;
+      if (dc && cudaMemPoolGetAttribute(dc->mempool, cudaMemPoolAttrReservedMemCurrent, &held) ==
+                    cudaSuccess &&
+          cudaMemPoolGetAttribute(dc->mempool, cudaMemPoolAttrUsedMemCurrent, &inuse) ==
+              cudaSuccess &&
+          held > inuse)
+        free_b += held - inuse;
       extra = std::min<int64_t>(extra, std::max<int64_t>((int64_t)(free_b * 0.8) / chunk_b,
                                                          2 * (int64_t)parked));
+    }
     const int64_t want = used + extra + (int64_t)gs::CHUNK_BATCH * warps + 1024;
     if (want > r->pool_chunks && (st = grow_pool(r, want, used, s)) != GS_OK) return bail(st);
     // the next pass: the parked trajectories, a fresh queue, park count and summary, and chunks
@@ -1044,7 +1084,7 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
         r->chunk_traj, r->chunk_seq, (int)r->nchunks, r->choff, r->chunk_table, bounds_of(r));
   if (cudaGetLastError() != cudaSuccess) return bail(fail(GS_ERR_CUDA, "chunk table launch failed"));
   if ((st = build_perm(r, s)) != GS_OK) return bail(st);
-  if ((st = ensure_theta_kept(r)) != GS_OK || (st = keep_theta(r, theta, s)) != GS_OK)
+  if ((st = ensure_theta_kept(r, s)) != GS_OK || (st = keep_theta(r, theta, s)) != GS_OK)
     return bail(st);
   *rec = r;
   if (r->host[4] != 0) {
@@ -1078,17 +1118,17 @@ gs_status gs_replay_grad(const gs_record* rec, const void* theta, const void* dL
   if (shared) {
     const size_t need = (size_t)N * M * rec->rsz, needp = (size_t)nred * M * rec->rsz;
     if (r->red_bytes < need) {
-      free_ptr(r->red_scratch);
+      free_ptr(r->red_scratch, s);
       r->red_scratch = nullptr;
       r->red_bytes = 0;
-      GS_CUDA(cudaMalloc(&r->red_scratch, need));
+      GS_CUDA(dalloc(&r->red_scratch, need, s));
       r->red_bytes = need;
     }
     if (r->part_bytes < needp) {
-      free_ptr(r->red_partials);
+      free_ptr(r->red_partials, s);
       r->red_partials = nullptr;
       r->part_bytes = 0;
-      GS_CUDA(cudaMalloc(&r->red_partials, needp));
+      GS_CUDA(dalloc(&r->red_partials, needp, s));
       r->part_bytes = needp;
     }
   }
@@ -1122,10 +1162,10 @@ gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, v
   if (!y1buf) {
     const size_t need = (size_t)rec->N * rec->sys.d * rec->rsz;
     if (rec->y1_bytes < need) {
-      free_ptr(rec->y1_scratch);
+      free_ptr(rec->y1_scratch, s);
       rec->y1_scratch = nullptr;
       rec->y1_bytes = 0;
-      GS_CUDA(cudaMalloc(&rec->y1_scratch, need));
+      GS_CUDA(dalloc(&rec->y1_scratch, need, s));
       rec->y1_bytes = need;
     }
     y1buf = rec->y1_scratch;
@@ -1278,17 +1318,17 @@ gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_
   if (shared) {
     const size_t need = (size_t)N * M * rec->rsz, needp = (size_t)nred * M * rec->rsz;
     if (r->red_bytes < need) {
-      free_ptr(r->red_scratch);
+      free_ptr(r->red_scratch, s);
       r->red_scratch = nullptr;
       r->red_bytes = 0;
-      GS_CUDA(cudaMalloc(&r->red_scratch, need));
+      GS_CUDA(dalloc(&r->red_scratch, need, s));
       r->red_bytes = need;
     }
     if (r->part_bytes < needp) {
-      free_ptr(r->red_partials);
+      free_ptr(r->red_partials, s);
       r->red_partials = nullptr;
       r->part_bytes = 0;
-      GS_CUDA(cudaMalloc(&r->red_partials, needp));
+      GS_CUDA(dalloc(&r->red_partials, needp, s));
       r->part_bytes = needp;
     }
   }
@@ -1427,7 +1467,7 @@ gs_status gs_record_import(const gs_system* sys, int64_t N, const int32_t* nstep
   r->C = C;
   r->E = E;
   r->rsz = sys->dtype == GS_F64 ? 8 : 4;
-  if ((st = ensure_traj_arrays(r, N)) != GS_OK) return bail(st);
+  if ((st = ensure_traj_arrays(r, N, s)) != GS_OK) return bail(st);
   if (N > 0) {
     if (cudaMemcpyAsync(r->nsteps, nsteps, N * sizeof(int), cudaMemcpyDeviceToDevice, s) !=
             cudaSuccess ||
@@ -1449,7 +1489,7 @@ gs_status gs_record_import(const gs_system* sys, int64_t N, const int32_t* nstep
     r->total_steps = tot[0];
     r->nchunks = tot[1];
     r->max_steps = r->host[3];
-    if ((st = ensure_pool(r, std::max<int64_t>(r->nchunks, 1))) != GS_OK) return bail(st);
+    if ((st = ensure_pool(r, std::max<int64_t>(r->nchunks, 1), s)) != GS_OK) return bail(st);
     if (r->nchunks > 0) {
       gs::k_iota<<<(int)((r->nchunks + 255) / 256), 256, 0, s>>>(r->chunk_table, (int)r->nchunks);
       const int nb = (int)((r->total_steps + 255) / 256);
@@ -1468,7 +1508,7 @@ gs_status gs_record_import(const gs_system* sys, int64_t N, const int32_t* nstep
       if (cudaGetLastError() != cudaSuccess) return bail(fail(GS_ERR_CUDA, "import launch failed"));
     }
     if ((st = build_perm(r, s)) != GS_OK) return bail(st);
-    if ((st = ensure_theta_kept(r)) != GS_OK) return bail(st);
+    if ((st = ensure_theta_kept(r, s)) != GS_OK) return bail(st);
   }
   r->theta_known = false;  // the states' theta is not known: the first use replays them
   *rec = r;
@@ -1480,20 +1520,32 @@ void gs_record_destroy(gs_record* r) {
   int prev = 0;
   cudaGetDevice(&prev);
   cudaSetDevice(r->device);
-  cudaDeviceSynchronize();
-  free_ptr(r->pool); free_ptr(r->chunk_traj); free_ptr(r->chunk_seq); free_ptr(r->chunk_table);
-  free_ptr(r->nsteps); free_ptr(r->status); free_ptr(r->offsets); free_ptr(r->choff);
-  free_ptr(r->tiles); free_ptr(r->counters);
-  free_ptr(r->red_scratch); free_ptr(r->red_partials); free_ptr(r->y1_scratch);
-  free_ptr(r->theta_kept);
-  free_ptr(r->perm); free_ptr(r->bins); free_ptr(r->binoff); free_ptr(r->btiles);
-  free_ptr(r->park_list); free_ptr(r->park_r);
-  free_ptr(r->park_i); free_ptr(r->park_att); free_ptr(r->park_key); free_ptr(r->park_order);
-  if (r->host) cudaFreeHost(r->host);
+  cudaDeviceSynchronize();  // nothing queued may still use the storage handed back below
+  cudaStream_t s = 0;
+  free_ptr(r->pool, s); free_ptr(r->chunk_traj, s); free_ptr(r->chunk_seq, s);
+  free_ptr(r->chunk_table, s);
+  free_ptr(r->nsteps, s); free_ptr(r->status, s); free_ptr(r->offsets, s); free_ptr(r->choff, s);
+  free_ptr(r->tiles, s); free_ptr(r->counters, s);
+  free_ptr(r->red_scratch, s); free_ptr(r->red_partials, s); free_ptr(r->y1_scratch, s);
+  free_ptr(r->theta_kept, s);
+  free_ptr(r->perm, s); free_ptr(r->bins, s); free_ptr(r->binoff, s); free_ptr(r->btiles, s);
+  free_ptr(r->park_list, s); free_ptr(r->park_r, s);
+  free_ptr(r->park_i, s); free_ptr(r->park_att, s); free_ptr(r->park_key, s);
+  free_ptr(r->park_order, s);
   if (r->ev0) cudaEventDestroy(r->ev0);
   if (r->ev1) cudaEventDestroy(r->ev1);
   cudaSetDevice(prev);
   delete r;
+}
+
+gs_status gs_memory_trim(int64_t keep_bytes) {
+  cudaError_t e;
+  DeviceCtx* c = device_ctx(&e);
+  if (!c) return fail(GS_ERR_CUDA, "device context: %s", cudaGetErrorString(e));
+  if (keep_bytes < 0) keep_bytes = 0;
+  GS_CUDA(cudaDeviceSynchronize());
+  GS_CUDA(cudaMemPoolTrimTo(c->mempool, (size_t)keep_bytes));
+  return GS_OK;
 }
 
 }  // extern "C"

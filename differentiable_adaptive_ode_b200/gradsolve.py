@@ -34,7 +34,8 @@ STATUS_NAMES = {0: "GS_OK", 1: "GS_ERR_INVALID_ARG", 2: "GS_ERR_CUDA", 3: "GS_ER
 EXPORTS = ("gs_solve_forward", "gs_solve_forward_sens", "gs_solve_record", "gs_replay_grad",
            "gs_replay_forward", "gs_replay_grad_noalloc", "gs_replay_outputs",
            "gs_replay_grad_outputs", "gs_record_info", "gs_record_export", "gs_record_import",
-           "gs_record_destroy", "gs_last_error", "gs_version", "gs_checked_violations")
+           "gs_record_destroy", "gs_memory_trim", "gs_last_error", "gs_version",
+           "gs_checked_violations")
 
 
 class GsSystem(C.Structure):
@@ -94,6 +95,8 @@ def lib():
         L.gs_record_import.argtypes = [P(GsSystem), i64, vp, vp, vp, vp, P(vp), vp]
         L.gs_record_destroy.argtypes = [vp]
         L.gs_record_destroy.restype = None
+        L.gs_memory_trim.argtypes = [i64]
+        L.gs_memory_trim.restype = C.c_int
         L.gs_last_error.restype = C.c_char_p
         L.gs_version.restype = C.c_char_p
         for name in ("gs_solve_forward", "gs_solve_forward_sens", "gs_solve_record", "gs_replay_grad", "gs_replay_forward",
@@ -281,6 +284,11 @@ def checked_violations():
     v = C.c_int64(0)
     _check(lib().gs_checked_violations(C.byref(v)))
     return v.value
+
+
+def gs_memory_trim(keep_bytes=0):
+    """Hand the record storage the device's pool keeps beyond keep_bytes back to the device."""
+    _check(lib().gs_memory_trim(int(keep_bytes)))
 
 
 def version():

@@ -26,7 +26,9 @@
  *     (unregistered) host memory or another device's memory, which a kernel could not read;
  *     device, managed and page-locked host memory pass.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is enqueued on it; calls
- *     return when the work is enqueued, except where a host synchronisation is stated.
+ *     return when the work is enqueued, except where a host synchronisation is stated.  Calls on
+ *     one record use its device storage and must be ordered: on one stream, or with the caller
+ *     synchronising between streams.
  *   - Errors: every entry point returns a gs_status and never aborts or exits; gs_last_error()
  *     returns a message for the calling thread's most recent failure.
  *   - Per-trajectory status codes (status arrays): 0 ok; 1 max_attempts reached; 2 step size
@@ -269,8 +271,18 @@ gs_status gs_record_export(const gs_record* rec, void* T, void* H, void* Y, int6
 gs_status gs_record_import(const gs_system* sys, int64_t N, const int32_t* nsteps, const void* T,
                            const void* H, const void* Y, gs_record** rec, void* stream);
 
-/* Free a record (NULL is ignored).  Synchronises the record's device. */
+/* Free a record (NULL is ignored).  Synchronises the record's device.  The record's device
+ * storage returns to the device's record pool, where the next records take it (see
+ * gs_memory_trim). */
 void gs_record_destroy(gs_record* rec);
+
+/* Records draw their device storage from a stream-ordered memory pool per device, which keeps the
+ * storage of destroyed records (and of records that grew) for later records instead of handing
+ * it back to the device: a new record then costs no driver allocation and destroying one no
+ * synchronous free.  gs_memory_trim(keep_bytes) hands what the pool holds beyond keep_bytes (and
+ * beyond what live records use) back to the current device.  Synchronises the device.  Not part
+ * of the method ([GS] has no counterpart): memory management of the library. */
+gs_status gs_memory_trim(int64_t keep_bytes);
 
 /* Message of the calling thread's last failure ("" if none). */
 const char* gs_last_error(void);

@@ -277,6 +277,30 @@ def test_first_record_in_slices_equals_ordered_record(name, N):
         assert np.array_equal(ga[1], gb[1])
 
 
+def test_record_storage_is_reused_and_trimmed():
+    # a destroyed record's device storage goes back to the library's pool and the next record
+    # takes it; gs_memory_trim hands the pool's idle storage back to the device; records made
+    # before and after either are the same
+    import torch
+    w = W.lorenz63(N=1 << 16)
+    rec, out = U.record(w)
+    ref = U.export_padded(w, rec)
+    rec.close()
+    rec2, out2 = U.record(w)
+    ex2 = U.export_padded(w, rec2)
+    rec2.close()
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info()[0]
+    G.gs_memory_trim(0)
+    assert torch.cuda.mem_get_info()[0] > free_before   # the two records' storage was handed back
+    rec3, out3 = U.record(w)
+    ex3 = U.export_padded(w, rec3)
+    for e in (ex2, ex3):
+        for key in ("S", "H", "Y"):
+            assert np.array_equal(e[key], ref[key]), key
+    assert np.array_equal(out2["y1"], out["y1"]) and np.array_equal(out3["y1"], out["y1"])
+
+
 def test_zero_steps_in_imported_record_change_nothing(orc):
     w = W.lorenz63(N=50)
     ref = orc.solve(w.field, w.method, w.theta, w.y0, w.t0, w.t1, w.rtol, w.atol, keep_record=True)
