@@ -117,6 +117,38 @@ struct SolveParams {
 template <class R> __device__ __forceinline__ R pw(R x, R e);
 template <> __device__ __forceinline__ double pw<double>(double x, double e) { return pow(x, e); }
 template <> __device__ __forceinline__ float pw<float>(float x, float e) { return powf(x, e); }
+// y^Q for a small positive integer Q, by repeated multiplication
+template <int Q>
+__device__ __forceinline__ double ipow(double y) {
+  if constexpr (Q == 1) return y;
+  else if constexpr (Q % 2 == 0) { const double h = ipow<Q / 2>(y); return h * h; }
+  else return ipow<Q - 1>(y) * y;
+}
+
+// The step controller's factor 0.9 err^(-1/Q), which the controller clamps to [0.2, 10] (or to
+// [0.2, 1] right after a reject): only err within [(0.09)^Q, 4.5^Q] -- inside [1e-10, 1e10] for
+// Q <= 7 -- reaches the clamp's interior, so err is clamped to [1e-10, 1e10] first, which leaves
+// every clamped factor as it was (non-finite and zero err never use this value).  fp64: Newton's
+// iteration on g(y) = err y^Q - 1, y <- y + (y / Q)(1 - err y^Q), from a float estimate good to
+// ~1e-7; quadratic convergence takes two steps below the double rounding, so the factor is within
+// about an ulp of the exactly rounded power, for a dozen FP64 operations instead of a general
+// power function.  fp32 keeps powf.
+template <class R, int Q> __device__ __forceinline__ R ctrl_factor(R err);
+template <int Q>
+__device__ __forceinline__ double ctrl_factor_d(double err) {
+  const double x = fmin(fmax(err, 1e-10), 1e10);
+  double y = (double)exp2f(-__log2f((float)x) / float(Q));
+#pragma unroll
+  for (int it = 0; it < 2; ++it) y = fma(y * (1.0 / Q), fma(-x, ipow<Q>(y), 1.0), y);
+  return 0.9 * y;
+}
+template <> __device__ __forceinline__ double ctrl_factor<double, 3>(double e) { return ctrl_factor_d<3>(e); }
+template <> __device__ __forceinline__ double ctrl_factor<double, 5>(double e) { return ctrl_factor_d<5>(e); }
+template <> __device__ __forceinline__ double ctrl_factor<double, 7>(double e) { return ctrl_factor_d<7>(e); }
+template <> __device__ __forceinline__ float ctrl_factor<float, 3>(float e) { return 0.9f * powf(e, float(-1.0 / 3)); }
+template <> __device__ __forceinline__ float ctrl_factor<float, 5>(float e) { return 0.9f * powf(e, float(-1.0 / 5)); }
+template <> __device__ __forceinline__ float ctrl_factor<float, 7>(float e) { return 0.9f * powf(e, float(-1.0 / 7)); }
+
 template <class R> __device__ __forceinline__ R eps_of();
 template <> __device__ __forceinline__ double eps_of<double>() { return 2.220446049250313e-16; }
 template <> __device__ __forceinline__ float eps_of<float>() { return 1.1920929e-07f; }
@@ -298,7 +330,6 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
   int cur = -1;               // direct record: chunk receiving this lane's next entries
   constexpr int SM = F::M;
 
-  const R expo = R(-1.0 / double(qerr));
   const R eps = eps_of<R>();
   const R span = fabs(p.t1 - p.t0);
 
@@ -503,7 +534,7 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
         // the controller's factor 0.9 err^(-1/q), formed once for both outcomes: when a warp holds
         // accepted and rejected lanes together (nearly always) it would otherwise run the power
         // function on both paths
-        const R fpow = R(0.9) * pw<R>(err, expo);
+        const R fpow = ctrl_factor<R, qerr>(err);
         if (err <= R(1)) {
           if constexpr (DIRECT) {
             if (cur < p.pool_chunks) {

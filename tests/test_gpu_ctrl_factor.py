@@ -1,0 +1,42 @@
+"""Accuracy of the step controller's factor as the solve kernels form it (gs::ctrl_factor).
+
+The I-controller ("gradsolve: fast exact gradients for ODE ensembles on GPUs", §2.1: a controller
+proposes the next step from the error estimate) multiplies h by clamp(0.9 err^(-1/q), 0.2, 10).
+The kernels take err^(-1/q) by two Newton steps on err y^q = 1 from a float estimate, after
+clamping err to [1e-10, 1e10].  Bound: the float estimate is good to ~1e-7; each step squares the
+relative error times (q + 1)/2, so the second leaves ~1e-26, and what remains is the rounding of
+the last step and of the product with 0.9 -- within 2 ulps, checked against a long-double
+reference with CUDA's pow beside it.  The clamp: below (0.09)^q the factor must be at least 10
+and above 4.5^q at most 0.2, so that the controller's clamped factor is unchanged by it.
+"""
+import json
+import os
+import shutil
+import subprocess
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+HERE = os.path.dirname(os.path.abspath(__file__))
+CSRC = os.path.join(os.path.dirname(HERE), "differentiable_adaptive_ode_b200", "csrc")
+
+
+def test_controller_factor_within_2_ulps(tmp_path):
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    exe = str(tmp_path / "ctrl_factor_check")
+    subprocess.run([nvcc, "-std=c++20", "-O3", "-gencode", "arch=compute_100a,code=sm_100a",
+                    "-I", CSRC, "-o", exe, os.path.join(HERE, "ctrl_factor_check.cu")],
+                   check=True, timeout=900)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    res = json.loads(r.stdout.strip().splitlines()[-1])
+    assert res["n"] > 100000
+    for q in ("q3", "q5", "q7"):
+        assert res[q]["clamp_ok"] == 1, res
+        assert res[q]["ulp"] <= 2.0, res
+        # the comparison column: CUDA's pow takes the exponent -1/q rounded to a double, which
+        # moves x^(-1/q) by |ln x| 2^-54 relative (up to ~1.6 ulp at the ends of [1e-14, 1e14])
+        assert res[q]["pow_ulp"] <= 4.0, res
