@@ -81,29 +81,31 @@ SMS, FP64_LANES, FP32_LANES = 148, 64, 128
 # 2^18-trajectory case of this workload; both kernels move a fixed number of bytes per accepted
 # step, so a launch's traffic is this times its accepted steps.  Record kernel: 64 B of record
 # per step written plus inputs; adjoint: the 64 B entry read per step plus chunk table and inputs.
-# The stellar record and adjoint figures were captured after the last change to those kernels;
-# the other workloads' record and sensitivity figures precede the one-division error norm, a
-# change of arithmetic only that leaves the bytes each step moves (its record entry) as they were.
+# The stellar figures were captured after the last change to those kernels.  The other
+# workloads' record kernels (and the sensitivity solve) have changed since their captures (record
+# chunks taken before each attempt, trajectories parked and resumed, the controller's power), so
+# their record and sensitivity figures are withheld (None) until captured again; their replay
+# adjoints are unchanged since theirs.
 TRAFFIC_PER_STEP = {
-    "nfw_mn": {"record": 68.4, "adjoint": 70.7},
-    "robertson": {"record": 38.9, "adjoint": 42.4},
-    "robertson_rb23": {"record": 39.8, "adjoint": 47.1},
-    "hires": {"record": 83.1, "adjoint": 89.4},
+    "nfw_mn": {"record": 68.5, "adjoint": 70.8},
+    "robertson": {"record": None, "adjoint": 42.4},
+    "robertson_rb23": {"record": None, "adjoint": 47.1},
+    "hires": {"record": None, "adjoint": 89.4},
     "lorenz63_vern7": {"adjoint": 45.2},                   # its record pass stays partly in L2
 }
 # FP64 pipe occupancy (sm__pipe_fp64_cycles_active, % of peak) of the same captures: how busy the
 # pipe is, transcendental sequences included, next to the algorithmic fraction
 PIPE_BUSY_NCU = {
-    "nfw_mn": {"record": 0.493, "adjoint": 0.631},
-    "robertson": {"record": 0.416, "adjoint": 0.427},
-    "robertson_rb23": {"record": 0.328, "adjoint": 0.387},
-    "hires": {"record": 0.196, "adjoint": 0.217},
-    "lorenz63_vern7": {"record": 0.457, "adjoint": 0.552},
-    "log_halo": {"sens": 0.710},
+    "nfw_mn": {"record": 0.544, "adjoint": 0.733},
+    "robertson": {"record": None, "adjoint": 0.427},
+    "robertson_rb23": {"record": None, "adjoint": 0.387},
+    "hires": {"record": None, "adjoint": 0.217},
+    "lorenz63_vern7": {"record": None, "adjoint": 0.552},
+    "log_halo": {"sens": None},
 }
 # forward sensitivities: DRAM bytes per trajectory (inputs and outputs; nothing per step), from
-# the ncu capture of the 2^18-orbit case
-TRAFFIC_SENS_PER_TRAJ = {"log_halo": 91.1}
+# an ncu capture of the 2^18-orbit case (withheld: the kernel changed since)
+TRAFFIC_SENS_PER_TRAJ = {"log_halo": None}
 # library kernels per step: record = k_solve + 2 k_max_int + 3 prefix scans of 3 kernels each
 # (step offsets, chunk offsets, length bins) + k_chunk_table + k_bin_count + k_bin_scatter (15);
 # replay gradient = k_theta_check + k_replay_forward (exits at once: the theta is the recorded one)
@@ -494,7 +496,8 @@ def run_sens(args, w, wl, G, torch, dev, stream, ws, rank):
     roofline = {"kernel": "k_solve<log_halo, double, Tsit5, sens>", "bound": "alu",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "pipe_busy_ncu": PIPE_BUSY_NCU.get(args.workload, {}).get("sens"),
-                "traffic": TRAFFIC_SENS_PER_TRAJ[args.workload] * N,
+                "traffic": (TRAFFIC_SENS_PER_TRAJ[args.workload] * N
+                            if TRAFFIC_SENS_PER_TRAJ.get(args.workload) else None),
                 "traffic_source": "ncu dram bytes per trajectory on the 2^18 case x trajectories",
                 "peak_source": "derived: 148 SM x 64 FP64 FMA lanes/clk x 2 x 1965 MHz (FP64 pipe)",
                 "flops_per_unit": {"attempted step": wl["fwd"], "accepted step (sensitivities)":
@@ -829,11 +832,11 @@ def main():
     traffic = TRAFFIC_PER_STEP.get(args.workload, {})
     roof_rec = roof("k_solve<%s, %s, %s, record>" % (w.field, "double" if f64 else "float", method),
                     wl["fwd"], attempts, rec_kernel_ms, "attempted step",
-                    traffic.get("record", 0) * total_steps or None,
+                    (traffic.get("record") or 0) * total_steps or None,
                     PIPE_BUSY_NCU.get(args.workload, {}).get("record"))
     roof_adj = roof("k_adjoint<%s, %s, %s>" % (w.field, "double" if f64 else "float", method),
                     wl["adj"], total_steps, adj_ms, "accepted step",
-                    traffic.get("adjoint", 0) * total_steps or None,
+                    (traffic.get("adjoint") or 0) * total_steps or None,
                     PIPE_BUSY_NCU.get(args.workload, {}).get("adjoint"))
     dominant, other = (roof_rec, roof_adj) if rec_kernel_ms >= adj_ms else (roof_adj, roof_rec)
     line = {

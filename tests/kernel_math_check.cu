@@ -1,0 +1,136 @@
+// Accuracy check of the kernels' own fp64 arithmetic helpers against long-double host references:
+//  - the step controller's factor 0.9 err^(-1/Q) (gs::ctrl_factor: two Newton steps on
+//    err y^Q = 1 from a float estimate, after clamping err to [1e-10, 1e10]), beside CUDA's pow,
+//    and the clamp's claim: below (0.09)^Q the factor is at least 10 and above 4.5^Q at most 0.2,
+//    so the controller's clamped factor is the same as with the unclamped power;
+//  - the Newton-refined reciprocal and reciprocal square root (gs::rcp_nr, gs::rsqrt_nr), beside
+//    CUDA's division and rsqrt, over normal positive arguments from 2^-1000 to 2^1000.
+//
+// Built and run by tests/test_gpu_kernel_math.py.  Prints one JSON object:
+//   {"n": ..., "q3": {"ulp": max, "pow_ulp": max, "clamp_ok": 0|1}, "q5": ..., "q7": ...,
+//    "rcp": {"ulp": max, "cuda_ulp": max}, "rsqrt": {...}}
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <vector>
+
+#include "gs_kernels.cuh"
+
+__global__ void k_recip(const double* __restrict__ x, double* __restrict__ out, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    out[4 * i + 0] = gs::rcp_nr(x[i]);
+    out[4 * i + 1] = 1.0 / x[i];
+    out[4 * i + 2] = gs::rsqrt_nr(x[i]);
+    out[4 * i + 3] = rsqrt(x[i]);
+  }
+}
+
+template <int Q>
+__global__ void k_eval(const double* __restrict__ x, double* __restrict__ f,
+                       double* __restrict__ p, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    f[i] = gs::ctrl_factor<double, Q>(x[i]);
+    p[i] = 0.9 * pow(x[i], -1.0 / Q);
+  }
+}
+
+static bool ok(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) std::fprintf(stderr, "%s: %s\n", what, cudaGetErrorString(e));
+  return e == cudaSuccess;
+}
+
+template <int Q>
+static bool run(const std::vector<double>& x, double* ulp, double* pow_ulp, int* clamp_ok) {
+  const int n = int(x.size());
+  const size_t bytes = x.size() * sizeof(double);
+  double *dx = nullptr, *df = nullptr, *dp = nullptr;
+  if (!ok(cudaMalloc(&dx, bytes), "malloc") || !ok(cudaMalloc(&df, bytes), "malloc") ||
+      !ok(cudaMalloc(&dp, bytes), "malloc"))
+    return false;
+  if (!ok(cudaMemcpy(dx, x.data(), bytes, cudaMemcpyHostToDevice), "h2d")) return false;
+  k_eval<Q><<<(n + 255) / 256, 256>>>(dx, df, dp, n);
+  if (!ok(cudaGetLastError(), "launch") || !ok(cudaDeviceSynchronize(), "sync")) return false;
+  std::vector<double> f(x.size()), p(x.size());
+  if (!ok(cudaMemcpy(f.data(), df, bytes, cudaMemcpyDeviceToHost), "d2h") ||
+      !ok(cudaMemcpy(p.data(), dp, bytes, cudaMemcpyDeviceToHost), "d2h"))
+    return false;
+  cudaFree(dx); cudaFree(df); cudaFree(dp);
+  *ulp = 0;
+  *pow_ulp = 0;
+  *clamp_ok = 1;
+  const long double lo = powl(0.09L, Q), hi = powl(4.5L, Q);
+  for (size_t i = 0; i < x.size(); ++i) {
+    const long double xi = x[i];
+    if (xi < lo) { if (!(f[i] >= 10.0)) *clamp_ok = 0; continue; }
+    if (xi > hi) { if (!(f[i] <= 0.2)) *clamp_ok = 0; continue; }
+    const long double ref = (long double)0.9 * powl(xi, -1.0L / Q);
+    int ex;
+    std::frexp(double(ref), &ex);
+    const double u = std::ldexp(1.0, ex - 53);
+    const double e1 = double(fabsl((long double)f[i] - ref)) / u;
+    const double e2 = double(fabsl((long double)p[i] - ref)) / u;
+    if (!(e1 <= *ulp)) *ulp = e1;  // NaN propagates as a failure
+    if (e2 > *pow_ulp) *pow_ulp = e2;
+  }
+  return true;
+}
+
+static bool run_recip(double* u_rcp, double* c_rcp, double* u_rs, double* c_rs, int* n_out) {
+  std::vector<double> x;
+  for (int e = -1000; e < 1000; ++e)
+    for (int k = 0; k < 64; ++k) x.push_back(std::ldexp(1.0 + k / 64.0 + 1.0 / 4099.0, e));
+  const int n = int(x.size());
+  *n_out = n;
+  double *dx = nullptr, *dout = nullptr;
+  if (!ok(cudaMalloc(&dx, n * sizeof(double)), "malloc") ||
+      !ok(cudaMalloc(&dout, 4 * n * sizeof(double)), "malloc"))
+    return false;
+  if (!ok(cudaMemcpy(dx, x.data(), n * sizeof(double), cudaMemcpyHostToDevice), "h2d")) return false;
+  k_recip<<<(n + 255) / 256, 256>>>(dx, dout, n);
+  if (!ok(cudaGetLastError(), "launch") || !ok(cudaDeviceSynchronize(), "sync")) return false;
+  std::vector<double> out(4 * x.size());
+  if (!ok(cudaMemcpy(out.data(), dout, 4 * n * sizeof(double), cudaMemcpyDeviceToHost), "d2h"))
+    return false;
+  cudaFree(dx); cudaFree(dout);
+  *u_rcp = *c_rcp = *u_rs = *c_rs = 0;
+  auto ulps = [](long double v, long double ref) {
+    int ex;
+    std::frexp(double(ref), &ex);
+    return double(fabsl(v - ref)) / std::ldexp(1.0, ex - 53);
+  };
+  for (int i = 0; i < n; ++i) {
+    const long double xi = x[i];
+    const long double r1 = 1.0L / xi, r2 = 1.0L / sqrtl(xi);
+    const double a = ulps(out[4 * i], r1), b = ulps(out[4 * i + 1], r1);
+    const double c = ulps(out[4 * i + 2], r2), d = ulps(out[4 * i + 3], r2);
+    if (!(a <= *u_rcp)) *u_rcp = a;
+    if (b > *c_rcp) *c_rcp = b;
+    if (!(c <= *u_rs)) *u_rs = c;
+    if (d > *c_rs) *c_rs = d;
+  }
+  return true;
+}
+
+int main() {
+  // err from 1e-14 to 1e14, 4096 points per decade, plus the clamp's edges
+  std::vector<double> x;
+  for (int i = 0; i <= 28 * 4096; ++i) x.push_back(std::pow(10.0, -14.0 + i / 4096.0));
+  for (double e : {1e-10, 1e10, 0.5, 1.0, 2.0}) x.push_back(e);
+  double u3, p3, u5, p5, u7, p7;
+  int c3, c5, c7;
+  if (!run<3>(x, &u3, &p3, &c3) || !run<5>(x, &u5, &p5, &c5) || !run<7>(x, &u7, &p7, &c7))
+    return 1;
+  double ur, cr, us, cs;
+  int nr;
+  if (!run_recip(&ur, &cr, &us, &cs, &nr)) return 1;
+  std::printf("{\"n\": %d, \"q3\": {\"ulp\": %.4f, \"pow_ulp\": %.4f, \"clamp_ok\": %d}, "
+              "\"q5\": {\"ulp\": %.4f, \"pow_ulp\": %.4f, \"clamp_ok\": %d}, "
+              "\"q7\": {\"ulp\": %.4f, \"pow_ulp\": %.4f, \"clamp_ok\": %d}, "
+              "\"n_recip\": %d, \"rcp\": {\"ulp\": %.4f, \"cuda_ulp\": %.4f}, "
+              "\"rsqrt\": {\"ulp\": %.4f, \"cuda_ulp\": %.4f}}\n",
+              int(x.size()), u3, p3, c3, u5, p5, c5, u7, p7, c7, nr, ur, cr, us, cs);
+  return 0;
+}

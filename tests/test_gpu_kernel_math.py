@@ -1,4 +1,6 @@
-"""Accuracy of the step controller's factor as the solve kernels form it (gs::ctrl_factor).
+"""Accuracy of the kernels' own fp64 arithmetic helpers: the step controller's factor
+(gs::ctrl_factor) and the Newton-refined reciprocal and reciprocal square root of the stellar
+field (gs::rcp_nr, gs::rsqrt_nr).
 
 The I-controller ("gradsolve: fast exact gradients for ODE ensembles on GPUs", §2.1: a controller
 proposes the next step from the error estimate) multiplies h by clamp(0.9 err^(-1/q), 0.2, 10).
@@ -8,6 +10,9 @@ relative error times (q + 1)/2, so the second leaves ~1e-26, and what remains is
 the last step and of the product with 0.9 -- within 2 ulps, checked against a long-double
 reference with CUDA's pow beside it.  The clamp: below (0.09)^q the factor must be at least 10
 and above 4.5^q at most 0.2, so that the controller's clamped factor is unchanged by it.
+The reciprocal and reciprocal square root start from the hardware approximations (relative error
+near 2^-22); two Newton steps leave the rounding of the last step, within 1.5 ulps (checked over
+2^-1000 .. 2^1000 against long double, CUDA's correctly rounded division and its rsqrt beside).
 """
 import json
 import os
@@ -21,14 +26,14 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(os.path.dirname(HERE), "differentiable_adaptive_ode_b200", "csrc")
 
 
-def test_controller_factor_within_2_ulps(tmp_path):
+def test_kernel_math_helpers_within_bounds(tmp_path):
     torch = pytest.importorskip("torch")
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
-    exe = str(tmp_path / "ctrl_factor_check")
+    exe = str(tmp_path / "kernel_math_check")
     subprocess.run([nvcc, "-std=c++20", "-O3", "-gencode", "arch=compute_100a,code=sm_100a",
-                    "-I", CSRC, "-o", exe, os.path.join(HERE, "ctrl_factor_check.cu")],
+                    "-I", CSRC, "-o", exe, os.path.join(HERE, "kernel_math_check.cu")],
                    check=True, timeout=900)
     r = subprocess.run([exe], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr
@@ -40,3 +45,7 @@ def test_controller_factor_within_2_ulps(tmp_path):
         # the comparison column: CUDA's pow takes the exponent -1/q rounded to a double, which
         # moves x^(-1/q) by |ln x| 2^-54 relative (up to ~1.6 ulp at the ends of [1e-14, 1e14])
         assert res[q]["pow_ulp"] <= 4.0, res
+    assert res["n_recip"] > 100000
+    for f in ("rcp", "rsqrt"):
+        assert res[f]["ulp"] <= 1.5, res
+        assert res[f]["cuda_ulp"] <= 1.5, res
