@@ -10,6 +10,7 @@
 #include <cstring>
 #include <initializer_list>
 #include <atomic>
+#include <map>
 #include <mutex>
 #include <new>
 #include <string>
@@ -94,18 +95,23 @@ gs_status check_system(const gs_system* sys) {
 // Per-device library state, created on first use and kept until exit: the SM count, a ring of
 // work-queue counters (each call takes its own slot, zeroes it on its stream and hands it to its
 // kernel, so calls on different streams never share a counter), cached occupancy figures, and
-// the stream-ordered memory pool that records draw their device storage from.  The pool keeps
-// the storage of destroyed records for the next ones (a new record then costs no driver
-// allocation, and destroying one no synchronous free) until gs_memory_trim hands it back.
+// the cache of record storage: blocks released by records (destroyed, or regrown) are kept here
+// for the next records instead of going back to the driver, so that a new record costs no
+// allocation and destroying one no cudaFree (about 6 ms for 12 GB), until gs_memory_trim hands
+// them back.  New storage comes from cudaMalloc (about 2 ms for 12 GB; a stream-ordered memory
+// pool took 83 ms to grow by the same amount the first time, measured on B200).
 struct DeviceCtx {
   std::once_flag once;
   cudaError_t init_err = cudaSuccess;
   int sms = 148;
   int* ring = nullptr;
-  cudaMemPool_t mempool = nullptr;
   std::atomic<unsigned> next{0};
   std::mutex occ_mu;
   std::unordered_map<const void*, int> occ;
+  std::mutex mem_mu;
+  std::multimap<size_t, void*> cached;      // released blocks by size
+  std::unordered_map<void*, size_t> sizes;  // every block handed out or cached, by address
+  size_t cached_bytes = 0;
 };
 constexpr int MAX_DEVICES = 64;
 constexpr unsigned RING = 4096;
@@ -123,31 +129,57 @@ DeviceCtx* device_ctx(cudaError_t* err) {
   std::call_once(c.once, [&]() {
     c.init_err = cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev);
     if (c.init_err == cudaSuccess) c.init_err = cudaMalloc(&c.ring, RING * sizeof(int));
-    if (c.init_err == cudaSuccess) {
-      cudaMemPoolProps props = {};
-      props.allocType = cudaMemAllocationTypePinned;
-      props.location.type = cudaMemLocationTypeDevice;
-      props.location.id = dev;
-      c.init_err = cudaMemPoolCreate(&c.mempool, &props);
-    }
-    if (c.init_err == cudaSuccess) {
-      uint64_t keep = UINT64_MAX;  // released storage stays in the pool until trimmed
-      c.init_err = cudaMemPoolSetAttribute(c.mempool, cudaMemPoolAttrReleaseThreshold, &keep);
-    }
   });
   *err = c.init_err;
   return c.init_err == cudaSuccess ? &c : nullptr;
 }
 
-// Device storage of a record: from the device's pool, ordered on stream s (usable by work on s
-// at once, by other streams after s has reached this point).
+// Hands cached blocks back to the driver until at most `keep` bytes stay cached (largest first).
+cudaError_t release_cached(DeviceCtx* c, size_t keep) {
+  std::lock_guard<std::mutex> lk(c->mem_mu);
+  cudaError_t e = cudaSuccess;
+  while (c->cached_bytes > keep && !c->cached.empty()) {
+    auto it = std::prev(c->cached.end());
+    const cudaError_t f = cudaFree(it->second);
+    if (f != cudaSuccess) e = f;
+    c->cached_bytes -= it->first;
+    c->sizes.erase(it->second);
+    c->cached.erase(it);
+  }
+  return e;
+}
+
+// Device storage of a record, usable by any stream: the smallest cached block that holds `bytes`
+// without wasting more than half of itself, else new storage from cudaMalloc (after handing the
+// cache back to the driver if the device is out of memory).
 template <class T>
-cudaError_t dalloc(T** p, size_t bytes, cudaStream_t s) {
+cudaError_t dalloc(T** p, size_t bytes, cudaStream_t) {
   cudaError_t e;
   DeviceCtx* c = device_ctx(&e);
   if (!c) return e;
-  return cudaMallocFromPoolAsync(reinterpret_cast<void**>(p), std::max<size_t>(bytes, 1), c->mempool,
-                                 s);
+  bytes = std::max<size_t>(bytes, 256);
+  {
+    std::lock_guard<std::mutex> lk(c->mem_mu);
+    auto it = c->cached.lower_bound(bytes);
+    if (it != c->cached.end() && it->first <= 2 * bytes) {
+      *p = static_cast<T*>(it->second);
+      c->cached_bytes -= it->first;
+      c->cached.erase(it);
+      return cudaSuccess;
+    }
+  }
+  void* q = nullptr;
+  e = cudaMalloc(&q, bytes);
+  if (e == cudaErrorMemoryAllocation) {
+    cudaGetLastError();  // clear the error before trying again
+    release_cached(c, 0);
+    e = cudaMalloc(&q, bytes);
+  }
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(c->mem_mu);
+  c->sizes[q] = bytes;
+  *p = static_cast<T*>(q);
+  return cudaSuccess;
 }
 
 // A zeroed work counter for one launch on stream s.
@@ -255,9 +287,22 @@ struct gs_record {
 
 namespace {
 
-// Returns record storage to the pool once the work queued on stream s before this point is done.
-void free_ptr(void* p, cudaStream_t s) {
-  if (p) cudaFreeAsync(p, s);
+// Returns record storage to the device's cache.  The device is synchronised first (as cudaFree
+// would): no queued work may still use a block that the next record could take.
+void free_ptr(void* p, cudaStream_t) {
+  if (!p) return;
+  cudaError_t e;
+  DeviceCtx* c = device_ctx(&e);
+  if (!c) return;
+  cudaDeviceSynchronize();
+  std::lock_guard<std::mutex> lk(c->mem_mu);
+  auto it = c->sizes.find(p);
+  if (it == c->sizes.end()) {  // not a block of this device's cache
+    cudaFree(p);
+    return;
+  }
+  c->cached.emplace(it->second, p);
+  c->cached_bytes += it->second;
 }
 
 gs_status ensure_traj_arrays(gs_record* r, int64_t N, cudaStream_t s) {
@@ -390,11 +435,23 @@ gs_status counting_sort_desc(gs_record* r, const int* keys, int64_t n, int kmax,
     r->bins_cap = nb;
   }
   GS_CUDA(cudaMemsetAsync(r->bins, 0, 2 * nb * sizeof(int), s));
-  const int grid = (int)((n + 255) / 256);
-  gs::k_bin_count<<<grid, 256, 0, s>>>(keys, (int)n, kmax, r->bins);
+  // up to 4,097 bins a block keeps its own histogram in shared memory (32 KB for the scatter)
+  const bool small = nb <= 4097;
+  const int threads = small ? 1024 : 256;
+  const int grid = (int)((n + threads - 1) / threads);
+  if (small)
+    gs::k_bin_count_smem<<<grid, threads, nb * sizeof(int), s>>>(keys, (int)n, kmax, r->bins);
+  else
+    gs::k_bin_count<<<grid, threads, 0, s>>>(keys, (int)n, kmax, r->bins);
   gs_status st = scan_counts<0>(r->bins, (int)nb, 1, r->binoff, r->btiles, s);
   if (st != GS_OK) return st;
-  gs::k_bin_scatter<<<grid, 256, 0, s>>>(keys, (int)n, kmax, r->binoff, r->bins + nb, out, ids);
+  if (small)
+    gs::k_bin_scatter_smem<<<grid, threads, 2 * nb * sizeof(int), s>>>(keys, (int)n, kmax,
+                                                                      r->binoff, r->bins + nb,
+                                                                      out, ids);
+  else
+    gs::k_bin_scatter<<<grid, threads, 0, s>>>(keys, (int)n, kmax, r->binoff, r->bins + nb, out,
+                                               ids);
   GS_CUDA(cudaGetLastError());
   return GS_OK;
 }
@@ -975,7 +1032,7 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
   int64_t nq = N;
   int64_t pass_start = 0;  // chunks handed out before this pass
   const int nb = (int)((N + 255) / 256);
-  constexpr int KMAX = 1 << 16;
+  constexpr int KMAX = 4096;  // remaining-step keys beyond this count as the longest
   for (int pass = 0;; ++pass) {
     const bool sliced = slice_mode && pass == 0;
     SolveCall c{N, theta, sys->theta_shared, y0, t0, t1, rtol, atol, attempts_of(opt), y1,
@@ -1051,16 +1108,13 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
     size_t free_b = 0, total_b = 0;
     const int64_t chunk_b = (int64_t)C * E * (int64_t)rsz + 3 * (int64_t)sizeof(int);
     if (cudaMemGetInfo(&free_b, &total_b) == cudaSuccess) {
-      // storage the pool holds but no record uses counts as free
+      // storage the cache holds counts as free
       cudaError_t ce;
       DeviceCtx* dc = device_ctx(&ce);
-      uint64_t held = 0, inuse = 0;
-      if (dc && cudaMemPoolGetAttribute(dc->mempool, cudaMemPoolAttrReservedMemCurrent, &held) ==
-                    cudaSuccess &&
-          cudaMemPoolGetAttribute(dc->mempool, cudaMemPoolAttrUsedMemCurrent, &inuse) ==
-              cudaSuccess &&
-          held > inuse)
-        free_b += held - inuse;
+      if (dc) {
+        std::lock_guard<std::mutex> lk(dc->mem_mu);
+        free_b += dc->cached_bytes;
+      }
       extra = std::min<int64_t>(extra, std::max<int64_t>((int64_t)(free_b * 0.8) / chunk_b,
                                                          2 * (int64_t)parked));
     }
@@ -1544,7 +1598,7 @@ gs_status gs_memory_trim(int64_t keep_bytes) {
   if (!c) return fail(GS_ERR_CUDA, "device context: %s", cudaGetErrorString(e));
   if (keep_bytes < 0) keep_bytes = 0;
   GS_CUDA(cudaDeviceSynchronize());
-  GS_CUDA(cudaMemPoolTrimTo(c->mempool, (size_t)keep_bytes));
+  GS_CUDA(release_cached(c, (size_t)keep_bytes));
   return GS_OK;
 }
 

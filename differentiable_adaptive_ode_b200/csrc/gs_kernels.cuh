@@ -1114,20 +1114,31 @@ template <class R>
 __global__ void k_park_estimate(const int* list, int P, const R* park_r, const int* park_i, int D,
                                 R t0, R t1, int C, unsigned long long* out, int* keys, int kmax) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= P) return;
-  const int k = list[i];
-  const R t = park_r[(size_t)k * (2 + 2 * D)];
-  const int S = park_i[(size_t)k * 4];
-  if (t > t0) {
-    // progress in time is a poor guide after a stiff start (tiny early steps): at most 64 times
-    // the steps taken so far
-    const double rem = fmin(double(S + 1) * double(t1 - t) / double(t - t0), 64.0 * (S + 1));
-    const double ch = fmin(1.25 * rem / C + 2.0, double(1 << 20));
-    atomicAdd(out, (unsigned long long)ch);
-    if (keys) keys[i] = (int)fmin(rem, double(kmax));
-  } else {
-    atomicAdd(out + 1, 1ull);
-    if (keys) keys[i] = kmax;
+  unsigned long long chunks = 0, fresh = 0;
+  if (i < P) {
+    const int k = list[i];
+    const R t = park_r[(size_t)k * (2 + 2 * D)];
+    const int S = park_i[(size_t)k * 4];
+    if (t > t0) {
+      // progress in time is a poor guide after a stiff start (tiny early steps): at most 64
+      // times the steps taken so far
+      const double rem = fmin(double(S + 1) * double(t1 - t) / double(t - t0), 64.0 * (S + 1));
+      chunks = (unsigned long long)fmin(1.25 * rem / C + 2.0, double(1 << 20));
+      if (keys) keys[i] = (int)fmin(rem, double(kmax));
+    } else {
+      fresh = 1;
+      if (keys) keys[i] = kmax;
+    }
+  }
+  // one atomic per warp for each sum (the block is a whole number of warps)
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    chunks += __shfl_xor_sync(FULL, chunks, o);
+    fresh += __shfl_xor_sync(FULL, fresh, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    if (chunks) atomicAdd(out, chunks);
+    if (fresh) atomicAdd(out + 1, fresh);
   }
 }
 
@@ -1227,6 +1238,19 @@ __global__ void k_bin_count(const int* S, int N, int smax, int* bins) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < N) atomicAdd(&bins[smax - S[i]], 1);
 }
+// The same counts through a per-block histogram in shared memory ([smax + 1] ints), added to the
+// global one once per nonzero bin: a handful of hot bins no longer serialise every element's
+// atomic in L2.
+__global__ void k_bin_count_smem(const int* S, int N, int smax, int* bins) {
+  extern __shared__ int hist[];
+  for (int j = threadIdx.x; j <= smax; j += blockDim.x) hist[j] = 0;
+  __syncthreads();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < N) atomicAdd(&hist[smax - S[i]], 1);
+  __syncthreads();
+  for (int j = threadIdx.x; j <= smax; j += blockDim.x)
+    if (hist[j]) atomicAdd(&bins[j], hist[j]);
+}
 // perm[position] = i (or ids[i] when ids is given), positions by decreasing S[i]
 __global__ void k_bin_scatter(const int* S, int N, int smax, const long long* binoff, int* cursor,
                               int* perm, const int* ids) {
@@ -1235,6 +1259,26 @@ __global__ void k_bin_scatter(const int* S, int N, int smax, const long long* bi
     const int b = smax - S[i];
     perm[binoff[b] + atomicAdd(&cursor[b], 1)] = ids ? ids[i] : i;
   }
+}
+// The same scatter with one global reservation per block and nonzero bin: ranks within the block
+// from a shared-memory histogram ([2 (smax + 1)] ints: counts, then the block's bases).
+__global__ void k_bin_scatter_smem(const int* S, int N, int smax, const long long* binoff,
+                                   int* cursor, int* perm, const int* ids) {
+  extern __shared__ int hist[];
+  int* base = hist + smax + 1;
+  for (int j = threadIdx.x; j <= smax; j += blockDim.x) hist[j] = 0;
+  __syncthreads();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  int b = 0, rank = 0;
+  if (i < N) {
+    b = smax - S[i];
+    rank = atomicAdd(&hist[b], 1);
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j <= smax; j += blockDim.x)
+    if (hist[j]) base[j] = atomicAdd(&cursor[j], hist[j]);
+  __syncthreads();
+  if (i < N) perm[binoff[b] + base[b] + rank] = ids ? ids[i] : i;
 }
 
 __global__ void k_iota(int* a, int n) {

@@ -272,16 +272,17 @@ gs_status gs_record_import(const gs_system* sys, int64_t N, const int32_t* nstep
                            const void* H, const void* Y, gs_record** rec, void* stream);
 
 /* Free a record (NULL is ignored).  Synchronises the record's device.  The record's device
- * storage returns to the device's record pool, where the next records take it (see
+ * storage goes to the device's cache of record storage, where the next records take it (see
  * gs_memory_trim). */
 void gs_record_destroy(gs_record* rec);
 
-/* Records draw their device storage from a stream-ordered memory pool per device, which keeps the
- * storage of destroyed records (and of records that grew) for later records instead of handing
- * it back to the device: a new record then costs no driver allocation and destroying one no
- * synchronous free.  gs_memory_trim(keep_bytes) hands what the pool holds beyond keep_bytes (and
- * beyond what live records use) back to the current device.  Synchronises the device.  Not part
- * of the method ([GS] has no counterpart): memory management of the library. */
+/* Records keep their device storage in a cache per device: storage released by a destroyed record
+ * (or by a record that grew) stays reserved for later records instead of going back to the
+ * device, so a new record costs no allocation and destroying one no cudaFree.  New storage comes
+ * from cudaMalloc; when the device runs out of memory the cache is handed back first.
+ * gs_memory_trim(keep_bytes) hands cached storage beyond keep_bytes back to the current device
+ * (storage of live records is not touched).  Synchronises the device.  Not part of the method
+ * ([GS] has no counterpart): memory management of the library. */
 gs_status gs_memory_trim(int64_t keep_bytes);
 
 /* Message of the calling thread's last failure ("" if none). */
