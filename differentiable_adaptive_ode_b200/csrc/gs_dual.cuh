@@ -56,28 +56,27 @@ template <> GS_DHD float add_rn<float>(float a, float b) { return __fadd_rn(a, b
 #endif
 
 // 1/x and 1/sqrt(x) for normal, positive, finite x: the hardware's approximations
-// (rcp.approx.ftz.f64, rsqrt.approx.ftz.f64: relative error near 2^-22) refined by two Newton
-// steps for the reciprocal, y <- y + y (1 - x y), and for the reciprocal square root,
-// y <- y + (y / 2)(1 - x y^2).  Each step squares the relative error, so two leave only the
-// rounding of the last step: within about an ulp of the exact value (checked against long
-// double), without the special-case paths of a general division or rsqrt.  Other scalar types
-// (float, dual numbers, the counting scalar) take the plain operations.
+// (rcp.approx.ftz.f64, rsqrt.approx.ftz.f64: relative error near 2^-22) refined by one
+// third-order step (the series of (1 - e)^(-1) and (1 - e)^(-1/2) to second order in the
+// residual): with e = 1 - x y, 1/x = y (1 + e + e^2 + ...); with e = 1 - x y^2,
+// 1/sqrt(x) = y (1 + e/2 + 3 e^2/8 + ...).  The dropped terms are below e^3 <= 2^-63 relative,
+// so what remains is the rounding of the few operations: within about an ulp of the exact value
+// (checked against long double), without the special-case paths of a general division or rsqrt.
+// Other scalar types (float, dual numbers, the counting scalar) take the plain operations.
 template <class R> GS_DHD R rsqrt_nr(R x) { return rsqrt(x); }
 template <class R> GS_DHD R rcp_nr(R x) { return R(1) / x; }
 #ifdef __CUDA_ARCH__
 template <> __device__ __forceinline__ double rsqrt_nr<double>(double x) {
   double y;
   asm("rsqrt.approx.ftz.f64 %0, %1;" : "=d"(y) : "d"(x));
-#pragma unroll
-  for (int i = 0; i < 2; ++i) y = fma(0.5 * y, fma(-x * y, y, 1.0), y);
-  return y;
+  const double e = fma(-x * y, y, 1.0);
+  return fma(y * fma(0.375, e, 0.5), e, y);
 }
 template <> __device__ __forceinline__ double rcp_nr<double>(double x) {
   double y;
   asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(y) : "d"(x));
-#pragma unroll
-  for (int i = 0; i < 2; ++i) y = fma(y, fma(-x, y, 1.0), y);
-  return y;
+  const double e = fma(-x, y, 1.0);
+  return fma(y, fma(e, e, e), y);
 }
 #endif
 

@@ -278,9 +278,9 @@ struct FNfwMiyamotoNagai {
   // Every rounding is spelled out (explicit fma, mul_rn, add_rn): f is inlined into the solve,
   // record and sensitivity kernels, and must round the same way in each of them.  Its operands
   // are normal and positive (r^2 > 0, z^2 + b^2 >= b^2, r_s + r >= r_s), so the reciprocal and
-  // the reciprocal square roots take the Newton-refined hardware approximations (rcp_nr,
-  // rsqrt_nr): measured on the 2^20 stellar ensemble, record 16.2 -> 15.7 ms, replay adjoint
-  // 12.6 -> 11.9 ms, against CUDA's division and rsqrt.
+  // the reciprocal square roots take the refined hardware approximations (rcp_nr, rsqrt_nr):
+  // measured on the 2^20 stellar ensemble against CUDA's division and rsqrt, record 16.2 -> 15.1
+  // ms, replay adjoint 12.6 -> 11.6 ms.
   template <class R> struct Inter { R R2, r, ir, L, isr, gN, iB, apB, iD, gM; };
   template <class R> GS_HD static void inter(const R* y, const Theta<R>& t, Inter<R>& I) {
     const R x = y[0], yy = y[1], z = y[2];

@@ -3,7 +3,7 @@
 //    err y^Q = 1 from a float estimate, after clamping err to [1e-10, 1e10]), beside CUDA's pow,
 //    and the clamp's claim: below (0.09)^Q the factor is at least 10 and above 4.5^Q at most 0.2,
 //    so the controller's clamped factor is the same as with the unclamped power;
-//  - the Newton-refined reciprocal and reciprocal square root (gs::rcp_nr, gs::rsqrt_nr), beside
+//  - the refined reciprocal and reciprocal square root (gs::rcp_nr, gs::rsqrt_nr), beside
 //    CUDA's division and rsqrt, over normal positive arguments from 2^-1000 to 2^1000.
 //
 // Built and run by tests/test_gpu_kernel_math.py.  Prints one JSON object:

@@ -1,5 +1,5 @@
 """Accuracy of the kernels' own fp64 arithmetic helpers: the step controller's factor
-(gs::ctrl_factor) and the Newton-refined reciprocal and reciprocal square root of the stellar
+(gs::ctrl_factor) and the refined reciprocal and reciprocal square root of the stellar
 field (gs::rcp_nr, gs::rsqrt_nr).
 
 The I-controller ("gradsolve: fast exact gradients for ODE ensembles on GPUs", §2.1: a controller
@@ -11,8 +11,10 @@ the last step and of the product with 0.9 -- within 2 ulps, checked against a lo
 reference with CUDA's pow beside it.  The clamp: below (0.09)^q the factor must be at least 10
 and above 4.5^q at most 0.2, so that the controller's clamped factor is unchanged by it.
 The reciprocal and reciprocal square root start from the hardware approximations (relative error
-near 2^-22); two Newton steps leave the rounding of the last step, within 1.5 ulps (checked over
-2^-1000 .. 2^1000 against long double, CUDA's correctly rounded division and its rsqrt beside).
+near 2^-22) and take one third-order correction (the residual's series to second order), whose
+dropped terms are below 2^-63: what remains is the rounding of the few operations, within 1.5
+ulps (checked over 2^-1000 .. 2^1000 against long double, CUDA's correctly rounded division and
+its rsqrt beside).
 """
 import json
 import os
