@@ -96,7 +96,7 @@ TRAFFIC_PER_STEP = {
 # FP64 pipe occupancy (sm__pipe_fp64_cycles_active, % of peak) of the same captures: how busy the
 # pipe is, transcendental sequences included, next to the algorithmic fraction
 PIPE_BUSY_NCU = {
-    "nfw_mn": {"record": 0.544, "adjoint": 0.733},
+    "nfw_mn": {"record": 0.528, "adjoint": 0.718},
     "robertson": {"record": None, "adjoint": 0.427},
     "robertson_rb23": {"record": None, "adjoint": 0.387},
     "hires": {"record": None, "adjoint": 0.217},

@@ -401,7 +401,7 @@ struct FLogHalo {
   template <class R> GS_HD static void f(const R* y, const Theta<R>& t, R* dy) {
     const R wz = y[2] * t.iq2;
     const R Q = R(Rc2) + y[0] * y[0] + y[1] * y[1] + y[2] * wz;
-    const R g = t.vc2 / Q;
+    const R g = mul_rn(t.vc2, rcp_nr(Q));  // Q >= R_c^2 > 0
     dy[0] = y[3];
     dy[1] = y[4];
     dy[2] = y[5];
@@ -413,7 +413,7 @@ struct FLogHalo {
   GS_HD static void vjp(const R* y, const Theta<R>& t, const R* kb, R* yb, R* thb) {
     const R x = y[0], yy = y[1], z = y[2];
     const R wz = z * t.iq2;
-    const R iQ = R(1) / (R(Rc2) + x * x + yy * yy + z * wz);
+    const R iQ = rcp_nr(R(Rc2) + x * x + yy * yy + z * wz);
     const R g = t.vc2 * iQ;
     const R ux = kb[3], uy = kb[4], uz = kb[5];
     const R uw = ux * x + uy * yy + uz * wz;

@@ -277,6 +277,33 @@ def test_first_record_in_slices_equals_ordered_record(name, N):
         assert np.array_equal(ga[1], gb[1])
 
 
+def test_sliced_first_record_with_attempt_cap_and_failures():
+    # a first record of 5,000 trajectories (sliced, then resumed) where the attempt cap (40) ends
+    # most trajectories after they were parked and resumed, and a few fail at start-up (non-finite
+    # theta): statuses, counts, final states and the record equal the plain forward solve's and
+    # those of a record started from a caller's order (no slice)
+    import torch
+    w = W.nfw_mn(N=5000)
+    w.theta = w.theta.copy()
+    w.theta[[7, 4321], 1] = np.nan
+    fw = U.forward(w, max_attempts=40)
+    rec_a, out_a = U.record(w, allow_failed=True, max_attempts=40)
+    ea = U.export_padded(w, rec_a)
+    assert np.array_equal(out_a["status"], fw["status"])
+    assert np.sum(fw["status"] == 1) > 1000 and np.all(fw["status"][[7, 4321]] == 3)
+    assert np.array_equal(ea["S"], fw["S"])
+    assert np.array_equal(out_a["y1"], fw["y1"])
+    dt = U.tdtype(w)
+    y1 = torch.empty((w.N, w.d), dtype=dt, device="cuda")
+    order = torch.arange(w.N, dtype=torch.int32, device="cuda")
+    rec_b = G.gs_solve_record(U.gsys(w), w.N, U.dev(w.theta, dt), U.dev(w.y0, dt), w.t0, w.t1,
+                              w.rtol, w.atol, y1, opts=G.options(40, 400 * w.N, order),
+                              allow_failed=True)
+    eb = U.export_padded(w, rec_b)
+    for key in ("S", "T", "H", "Y"):
+        assert np.array_equal(ea[key], eb[key]), key
+
+
 def test_record_storage_is_reused_and_trimmed():
     # a destroyed record's device storage goes back to the library's pool and the next record
     # takes it; gs_memory_trim hands the pool's idle storage back to the device; records made
