@@ -32,13 +32,13 @@ UNIT = "traj/s"
 # forward solve: counted from the definitions of the Tsit5 replay step, its reverse sweep and the
 # field's f and vector-Jacobian product (tests/test_flop_counts.py re-derives these numbers).
 FLOPS_ADJOINT_STEP = {"nfw_mn": 1254, "lorenz63": 432, "lotka_volterra": 344, "mlp": 48400,
-                      "log_halo": 834}
+                      "log_halo": 840}
 FLOPS_FORWARD_ATTEMPT = {"nfw_mn": 611, "lorenz63": 254, "lotka_volterra": 181, "mlp": 16425,
-                         "log_halo": 473}
+                         "log_halo": 479}
 # Forward sensitivities, per accepted step and all m columns: the tangent of the Tsit5 step,
 # 48 d (stage tangents 35 d, result 13 d) + 6 c_t per column, c_t = the forward-mode rules' extra
 # operations over f (the value part that the kernel recomputes alongside is not counted).
-FLOPS_SENS_STEP = {"log_halo": 912}
+FLOPS_SENS_STEP = {"log_halo": 948}
 # Verner 7, counted the same way from its table (nonzero a_ij per stage row 1, 2, 2, 3, 4, 5, 6,
 # 7, 6; b has 7 nonzeros, b - b_hat 8): per attempt 117 d + 10 c_f + 5 (nine new stages and the
 # fresh first stage of the next step); per accepted step of the replay adjoint 160 d + 8 c_f +
@@ -88,8 +88,8 @@ SMS, FP64_LANES, FP32_LANES = 148, 64, 128
 # adjoints are unchanged since theirs.
 TRAFFIC_PER_STEP = {
     "nfw_mn": {"record": 68.5, "adjoint": 70.8},
-    "robertson": {"record": None, "adjoint": 42.4},
-    "robertson_rb23": {"record": None, "adjoint": 47.1},
+    "robertson": {"record": 38.9, "adjoint": 42.2},
+    "robertson_rb23": {"record": 39.8, "adjoint": 43.7},
     "hires": {"record": None, "adjoint": 89.4},
     "lorenz63_vern7": {"adjoint": 45.2},                   # its record pass stays partly in L2
 }
@@ -97,15 +97,15 @@ TRAFFIC_PER_STEP = {
 # pipe is, transcendental sequences included, next to the algorithmic fraction
 PIPE_BUSY_NCU = {
     "nfw_mn": {"record": 0.528, "adjoint": 0.718},
-    "robertson": {"record": None, "adjoint": 0.427},
-    "robertson_rb23": {"record": None, "adjoint": 0.387},
+    "robertson": {"record": 0.387, "adjoint": 0.425},
+    "robertson_rb23": {"record": 0.259, "adjoint": 0.393},
     "hires": {"record": None, "adjoint": 0.217},
-    "lorenz63_vern7": {"record": None, "adjoint": 0.552},
-    "log_halo": {"sens": None},
+    "lorenz63_vern7": {"record": 0.439, "adjoint": 0.552},
+    "log_halo": {"sens": 0.790},
 }
 # forward sensitivities: DRAM bytes per trajectory (inputs and outputs; nothing per step), from
-# an ncu capture of the 2^18-orbit case (withheld: the kernel changed since)
-TRAFFIC_SENS_PER_TRAJ = {"log_halo": None}
+# an ncu capture of the 2^18-orbit case
+TRAFFIC_SENS_PER_TRAJ = {"log_halo": 94.3}
 # library kernels per step: record = k_solve + 2 k_max_int + 3 prefix scans of 3 kernels each
 # (step offsets, chunk offsets, length bins) + k_chunk_table + k_bin_count + k_bin_scatter (15);
 # replay gradient = k_theta_check + k_replay_forward (exits at once: the theta is the recorded one)
