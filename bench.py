@@ -87,7 +87,7 @@ SMS, FP64_LANES, FP32_LANES = 148, 64, 128
 # their record and sensitivity figures are withheld (None) until captured again; their replay
 # adjoints are unchanged since theirs.
 TRAFFIC_PER_STEP = {
-    "nfw_mn": {"record": 68.5, "adjoint": 70.8},
+    "nfw_mn": {"record": 68.3, "adjoint": 71.0},
     "robertson": {"record": 38.9, "adjoint": 42.2},
     "robertson_rb23": {"record": 39.8, "adjoint": 43.7},
     "hires": {"record": None, "adjoint": 89.4},
@@ -96,7 +96,7 @@ TRAFFIC_PER_STEP = {
 # FP64 pipe occupancy (sm__pipe_fp64_cycles_active, % of peak) of the same captures: how busy the
 # pipe is, transcendental sequences included, next to the algorithmic fraction
 PIPE_BUSY_NCU = {
-    "nfw_mn": {"record": 0.528, "adjoint": 0.718},
+    "nfw_mn": {"record": 0.560, "adjoint": 0.723},
     "robertson": {"record": 0.387, "adjoint": 0.425},
     "robertson_rb23": {"record": 0.259, "adjoint": 0.393},
     "hires": {"record": None, "adjoint": 0.217},

@@ -255,6 +255,31 @@ template <class F, class R> struct RecDirect { static constexpr bool value = fal
 template <class R> struct RecDirect<FNfwMiyamotoNagai, R> { static constexpr bool value = true; };
 template <class R> struct RecDirect<FHires, R> { static constexpr bool value = true; };
 
+// One record entry (t, h, y) written from a lane's registers.  When the entry fills whole
+// 16-byte words (the pool is 256-byte aligned and entries are contiguous), it goes out as 16-byte
+// vector stores: half (fp64) or a quarter (fp32) of the store instructions, and of the requests
+// that the L1 must process for a warp whose 32 lanes write 32 different chunks.
+template <class R, int E>
+__device__ __forceinline__ void store_entry(R* e, R t, R h, const R (&y)[E - 2]) {
+  if constexpr (E * sizeof(R) % 16 == 0 && sizeof(R) == 8) {
+    double2* v = reinterpret_cast<double2*>(e);
+    v[0] = make_double2(t, h);
+#pragma unroll
+    for (int c = 0; c < (E - 2) / 2; ++c) v[1 + c] = make_double2(y[2 * c], y[2 * c + 1]);
+  } else if constexpr (E * sizeof(R) % 16 == 0 && sizeof(R) == 4 && E % 4 == 0) {
+    float4* v = reinterpret_cast<float4*>(e);
+    v[0] = make_float4(t, h, y[0], y[1]);
+#pragma unroll
+    for (int c = 0; c < (E - 4) / 4; ++c)
+      v[1 + c] = make_float4(y[2 + 4 * c], y[3 + 4 * c], y[4 + 4 * c], y[5 + 4 * c]);
+  } else {
+    e[0] = t;
+    e[1] = h;
+#pragma unroll
+    for (int c = 0; c < E - 2; ++c) e[2 + c] = y[c];
+  }
+}
+
 // Per-warp ring of trajectories whose start-up is done (id, status, starting step, f(y0)).
 constexpr int START_RING = 64;
 template <class F, class R>
@@ -539,10 +564,7 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::solve
           if constexpr (DIRECT) {
             if (cur < p.pool_chunks) {
               R* e = p.pool + ((size_t)cur * L::C + ns) * L::E;
-              e[0] = t;
-              e[1] = h;
-#pragma unroll
-              for (int c = 0; c < D; ++c) e[2 + c] = y[c];
+              store_entry<R, L::E>(e, t, h, y);
             }
             if (++ns == L::C) {   // chunk full: the next attempt takes a new one
               ++seq;

@@ -213,26 +213,29 @@ __device__ __forceinline__ R tsit5_trial_rolled(const R (&y)[F::D], R h,
                                                 R (&k7)[F::D], R rtol, R atol) {
   constexpr int D = F::D;
   const auto& T = tsit5_tab<R>();
-  R acc[6][D], er[D];
+  R acc[6][D], er[D], hc1[6];
 #pragma unroll
-  for (int m = 0; m < 6; ++m) {
-    const R hc = h * T.fwd[1][m];
+  for (int m = 0; m < 6; ++m) hc1[m] = h * T.fwd[1][m];
 #pragma unroll
-    for (int c = 0; c < D; ++c) acc[m][c] = fma(hc, k1[c], y[c]);
+  for (int c = 0; c < D; ++c) {
+    const R yc = y[c], kc = k1[c];
+#pragma unroll
+    for (int m = 0; m < 6; ++m) acc[m][c] = fma(hc1[m], kc, yc);
+    er[c] = T.e[1] * kc;
   }
-#pragma unroll
-  for (int c = 0; c < D; ++c) er[c] = T.e[1] * k1[c];
+  // The last stage (i = 7) evaluates f at y_new itself and opens no further stage, so the loop
+  // leaves with acc[0] = y_new and kk = f(y_new), copied out after it: no value other than acc
+  // and er is carried from one pass of the body to the next.  (Copying them out inside the loop,
+  // on its last pass, kept y_new and k7 live across every pass: the stellar record kernel spilled
+  // at 168 registers, and ran 15.1 ms against 13.3 ms this way at 2^20 trajectories.)
+  R kk[D];
 #pragma unroll 1
   for (int i = 2; i <= 7; ++i) {
-    R kk[D];
     F::f(acc[0], th, kk);
     const R ei = T.e[i];
 #pragma unroll
     for (int c = 0; c < D; ++c) er[c] = fma(ei, kk[c], er[c]);
-    if (i == 7) {
-#pragma unroll
-      for (int c = 0; c < D; ++c) { ynew[c] = acc[0][c]; k7[c] = kk[c]; }
-    }
+    if (i == 7) break;
 #pragma unroll
     for (int m = 0; m < 5; ++m) {
       const R hc = h * T.fwd[i][m];
@@ -240,11 +243,14 @@ __device__ __forceinline__ R tsit5_trial_rolled(const R (&y)[F::D], R h,
       for (int c = 0; c < D; ++c) acc[m][c] = fma(hc, kk[c], acc[m + 1][c]);
     }
   }
+#pragma unroll
+  for (int c = 0; c < D; ++c) { ynew[c] = acc[0][c]; k7[c] = kk[c]; }
   R ev[D], sc[D];
 #pragma unroll
   for (int c = 0; c < D; ++c) {
+    const R yc = y[c];
     ev[c] = h * er[c];
-    sc[c] = fma(rtol, fmax(fabs(y[c]), fabs(ynew[c])), atol);
+    sc[c] = fma(rtol, fmax(fabs(yc), fabs(ynew[c])), atol);
   }
   return scaled_rms(ev, sc);
 }

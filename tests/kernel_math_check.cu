@@ -4,11 +4,15 @@
 //    and the clamp's claim: below (0.09)^Q the factor is at least 10 and above 4.5^Q at most 0.2,
 //    so the controller's clamped factor is the same as with the unclamped power;
 //  - the refined reciprocal and reciprocal square root (gs::rcp_nr, gs::rsqrt_nr), beside
-//    CUDA's division and rsqrt, over normal positive arguments from 2^-1000 to 2^1000.
+//    CUDA's division and rsqrt, over normal positive arguments from 2^-1000 to 2^1000;
+//  - the table-driven logarithm (gs::log_tab) beside CUDA's log: positive normal arguments
+//    across the whole range, densely over [1, 16] (where the stellar field evaluates it), near 1,
+//    next to every breakpoint c_j +- 1/256 of the table, and the special arguments.
 //
 // Built and run by tests/test_gpu_kernel_math.py.  Prints one JSON object:
 //   {"n": ..., "q3": {"ulp": max, "pow_ulp": max, "clamp_ok": 0|1}, "q5": ..., "q7": ...,
-//    "rcp": {"ulp": max, "cuda_ulp": max}, "rsqrt": {...}}
+//    "rcp": {"ulp": max, "cuda_ulp": max}, "rsqrt": {...},
+//    "n_log": ..., "log": {"ulp": max, "cuda_ulp": max, "special_ok": 0|1}}
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -24,6 +28,14 @@ __global__ void k_recip(const double* __restrict__ x, double* __restrict__ out, 
     out[4 * i + 1] = 1.0 / x[i];
     out[4 * i + 2] = gs::rsqrt_nr(x[i]);
     out[4 * i + 3] = rsqrt(x[i]);
+  }
+}
+
+__global__ void k_log(const double* __restrict__ x, double* __restrict__ out, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    out[2 * i + 0] = gs::log_tab(x[i]);
+    out[2 * i + 1] = log(x[i]);
   }
 }
 
@@ -114,6 +126,58 @@ static bool run_recip(double* u_rcp, double* c_rcp, double* u_rs, double* c_rs, 
   return true;
 }
 
+static bool run_log(double* u_log, double* c_log, int* special_ok, int* n_out) {
+  std::vector<double> x;
+  for (int e = -1022; e < 1024; ++e)
+    for (int k = 0; k < 64; ++k) x.push_back(std::ldexp(1.0 + k / 64.0 + 1.0 / 7919.0, e));
+  for (int k = 0; k < 400000; ++k) x.push_back(1.0 + 15.0 * k / 400000.0 + 1e-9 * (k % 7));
+  for (int k = 0; k < 100000; ++k) x.push_back(1.0 + std::ldexp(1.0, -6) * k / 100000.0);
+  for (int k = 0; k < 100000; ++k) x.push_back(1.0 - std::ldexp(1.0, -7) * k / 100000.0);
+  for (int k = 1; k < 53; ++k) { x.push_back(1.0 + std::ldexp(1.0, -k)); x.push_back(1.0 - std::ldexp(1.0, -k - 1)); }
+  for (int e = -2; e < 4; ++e)
+    for (int j = 0; j < 256; ++j)
+      for (int d = -4; d <= 4; ++d)
+        x.push_back(std::ldexp(1.0 + (j + 0.5) / 256.0 + d * 0x1p-52, e));
+  x.push_back(2.2250738585072014e-308);
+  x.push_back(1.7976931348623157e308);
+  const int nreg = int(x.size());
+  // special arguments, checked separately: +inf, +0, -1, NaN, a subnormal
+  const double specials[] = {HUGE_VAL, 0.0, -1.0, std::nan(""), 4.9e-324};
+  for (double v : specials) x.push_back(v);
+  const int n = int(x.size());
+  *n_out = nreg;
+  double *dx = nullptr, *dout = nullptr;
+  if (!ok(cudaMalloc(&dx, n * sizeof(double)), "malloc") ||
+      !ok(cudaMalloc(&dout, 2 * n * sizeof(double)), "malloc"))
+    return false;
+  if (!ok(cudaMemcpy(dx, x.data(), n * sizeof(double), cudaMemcpyHostToDevice), "h2d")) return false;
+  k_log<<<(n + 255) / 256, 256>>>(dx, dout, n);
+  if (!ok(cudaGetLastError(), "launch") || !ok(cudaDeviceSynchronize(), "sync")) return false;
+  std::vector<double> out(2 * x.size());
+  if (!ok(cudaMemcpy(out.data(), dout, 2 * n * sizeof(double), cudaMemcpyDeviceToHost), "d2h"))
+    return false;
+  cudaFree(dx); cudaFree(dout);
+  *u_log = *c_log = 0;
+  for (int i = 0; i < nreg; ++i) {
+    const long double ref = logl((long double)x[i]);
+    if (ref == 0) {                       // log 1 = 0 exactly
+      if (out[2 * i] != 0.0) *u_log = 1e9;
+      continue;
+    }
+    int ex;
+    std::frexp(double(ref), &ex);
+    const double u = std::ldexp(1.0, ex - 53);
+    const double a = double(fabsl((long double)out[2 * i] - ref)) / u;
+    const double b = double(fabsl((long double)out[2 * i + 1] - ref)) / u;
+    if (!(a <= *u_log)) *u_log = a;       // NaN propagates as a failure
+    if (b > *c_log) *c_log = b;
+  }
+  const double* sp = out.data() + 2 * nreg;
+  *special_ok = (sp[0] == HUGE_VAL) && (sp[2] == -HUGE_VAL) && std::isnan(sp[4]) &&
+                std::isnan(sp[6]) && std::isnan(sp[8]);
+  return true;
+}
+
 int main() {
   // err from 1e-14 to 1e14, 4096 points per decade, plus the clamp's edges
   std::vector<double> x;
@@ -126,11 +190,15 @@ int main() {
   double ur, cr, us, cs;
   int nr;
   if (!run_recip(&ur, &cr, &us, &cs, &nr)) return 1;
+  double ul, cl;
+  int sl, nl;
+  if (!run_log(&ul, &cl, &sl, &nl)) return 1;
   std::printf("{\"n\": %d, \"q3\": {\"ulp\": %.4f, \"pow_ulp\": %.4f, \"clamp_ok\": %d}, "
               "\"q5\": {\"ulp\": %.4f, \"pow_ulp\": %.4f, \"clamp_ok\": %d}, "
               "\"q7\": {\"ulp\": %.4f, \"pow_ulp\": %.4f, \"clamp_ok\": %d}, "
               "\"n_recip\": %d, \"rcp\": {\"ulp\": %.4f, \"cuda_ulp\": %.4f}, "
-              "\"rsqrt\": {\"ulp\": %.4f, \"cuda_ulp\": %.4f}}\n",
-              int(x.size()), u3, p3, c3, u5, p5, c5, u7, p7, c7, nr, ur, cr, us, cs);
+              "\"rsqrt\": {\"ulp\": %.4f, \"cuda_ulp\": %.4f}, "
+              "\"n_log\": %d, \"log\": {\"ulp\": %.4f, \"cuda_ulp\": %.4f, \"special_ok\": %d}}\n",
+              int(x.size()), u3, p3, c3, u5, p5, c5, u7, p7, c7, nr, ur, cr, us, cs, nl, ul, cl, sl);
   return 0;
 }

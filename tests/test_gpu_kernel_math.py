@@ -1,6 +1,6 @@
 """Accuracy of the kernels' own fp64 arithmetic helpers: the step controller's factor
-(gs::ctrl_factor) and the refined reciprocal and reciprocal square root of the stellar
-field (gs::rcp_nr, gs::rsqrt_nr).
+(gs::ctrl_factor), the refined reciprocal and reciprocal square root of the stellar field
+(gs::rcp_nr, gs::rsqrt_nr) and its table-driven logarithm (gs::log_tab).
 
 The I-controller ("gradsolve: fast exact gradients for ODE ensembles on GPUs", §2.1: a controller
 proposes the next step from the error estimate) multiplies h by clamp(0.9 err^(-1/q), 0.2, 10).
@@ -15,6 +15,9 @@ near 2^-22) and take one third-order correction (the residual's series to second
 dropped terms are below 2^-63: what remains is the rounding of the few operations, within 1.5
 ulps (checked over 2^-1000 .. 2^1000 against long double, CUDA's correctly rounded division and
 its rsqrt beside).
+The logarithm of the stellar field (gs::log_tab, Tang's table-driven method) is within half an
+ulp plus its few roundings: the bar is 0.6 ulp (CUDA's log, beside it, within 1), with +inf,
++0, a negative argument, NaN and a subnormal mapped to +inf, -inf and NaN.
 """
 import json
 import os
@@ -51,3 +54,7 @@ def test_kernel_math_helpers_within_bounds(tmp_path):
     for f in ("rcp", "rsqrt"):
         assert res[f]["ulp"] <= 1.5, res
         assert res[f]["cuda_ulp"] <= 1.5, res
+    assert res["n_log"] > 500000
+    assert res["log"]["ulp"] <= 0.6, res
+    assert res["log"]["cuda_ulp"] <= 1.0, res
+    assert res["log"]["special_ok"] == 1, res
