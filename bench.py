@@ -707,10 +707,11 @@ def main():
     # a record made from nothing ([GS] §4.7 reports the one-time record separately): a new record
     # object per repetition -- its allocations, a pool sized by default for 64 steps per
     # trajectory (trajectories that find it full are parked and resumed once it has grown), no
-    # longest-first order yet -- then the first gradient.  Wall-clock through completion.
+    # longest-first order yet -- then the first gradient.  Wall-clock through completion, the best
+    # of five (host-side costs -- allocation, the driver -- vary from one repetition to the next).
     def fresh(with_grad):
         best = None
-        for _ in range(3):
+        for _ in range(5):
             torch.cuda.synchronize()
             t0 = time.perf_counter()
             r = G.Record()
@@ -727,7 +728,7 @@ def main():
 
     def reused_wall():
         best = None
-        for _ in range(3):
+        for _ in range(5):
             torch.cuda.synchronize()
             t0 = time.perf_counter()
             G.gs_solve_record(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, rec=rec)

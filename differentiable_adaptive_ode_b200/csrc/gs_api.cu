@@ -112,6 +112,7 @@ struct DeviceCtx {
   std::multimap<size_t, void*> cached;      // released blocks by size
   std::unordered_map<void*, size_t> sizes;  // every block handed out or cached, by address
   size_t cached_bytes = 0;
+  size_t total_mem = 0;                     // device memory, read once
 };
 constexpr int MAX_DEVICES = 64;
 constexpr unsigned RING = 4096;
@@ -129,6 +130,11 @@ DeviceCtx* device_ctx(cudaError_t* err) {
   std::call_once(c.once, [&]() {
     c.init_err = cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev);
     if (c.init_err == cudaSuccess) c.init_err = cudaMalloc(&c.ring, RING * sizeof(int));
+    size_t free_b = 0;
+    if (c.init_err == cudaSuccess && cudaMemGetInfo(&free_b, &c.total_mem) != cudaSuccess) {
+      cudaGetLastError();
+      c.total_mem = 0;
+    }
   });
   *err = c.init_err;
   return c.init_err == cudaSuccess ? &c : nullptr;
@@ -840,6 +846,22 @@ int device_sms() {
   return c ? c->sms : 148;
 }
 
+// The estimate of what the parked trajectories of a record pass still need (gs::k_park_estimate),
+// for the first P entries of the park list, or for as many as the device counter `count` holds
+// (at most P) when it is non-null.
+void launch_park_estimate(gs_record* r, int P, const int* count, int d, double t0, double t1,
+                          int C, unsigned long long* est, int kmax, cudaStream_t s) {
+  const int eb = (std::max(P, 1) + 255) / 256;
+  if (r->rsz == 8)
+    gs::k_park_estimate<double><<<eb, 256, 0, s>>>(r->park_list, P, count,
+                                                  static_cast<const double*>(r->park_r), r->park_i,
+                                                  d, t0, t1, C, est, r->park_key, kmax);
+  else
+    gs::k_park_estimate<float><<<eb, 256, 0, s>>>(r->park_list, P, count,
+                                                 static_cast<const float*>(r->park_r), r->park_i, d,
+                                                 (float)t0, (float)t1, C, est, r->park_key, kmax);
+}
+
 }  // namespace
 
 // Replay adjoint of the MLP field: one warp per trajectory, per-warp weight-cotangent partials,
@@ -1054,7 +1076,16 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
     gs::k_max_int<<<nb, 256, 0, s>>>(r->nsteps, (int)N, r->counters + 3);
     gs::k_max_int<<<nb, 256, 0, s>>>(r->status, (int)N, r->counters + 4);
     if ((st = scan_counts<0>(r->nsteps, (int)N, C, r->offsets, r->tiles, s)) != GS_OK) return bail(st);
-    if (cudaMemcpyAsync(r->host, r->counters, 8 * sizeof(int), cudaMemcpyDeviceToHost, s) !=
+    // a slice parks (nearly) every trajectory: the estimate of what they still need is queued
+    // right behind the pass, with the parked count read on the device, and comes back with the
+    // summary in one synchronisation
+    unsigned long long* est = reinterpret_cast<unsigned long long*>(r->counters + 10);
+    if (sliced) {
+      if (cudaMemsetAsync(est, 0, 2 * sizeof(unsigned long long), s) != cudaSuccess)
+        return bail(fail(GS_ERR_CUDA, "cudaMemsetAsync failed"));
+      launch_park_estimate(r, (int)nq, r->counters + 2, sys->d, t0, t1, C, est, KMAX, s);
+    }
+    if (cudaMemcpyAsync(r->host, r->counters, 14 * sizeof(int), cudaMemcpyDeviceToHost, s) !=
             cudaSuccess ||
         cudaMemcpyAsync(r->host + 8, r->offsets + N, sizeof(long long), cudaMemcpyDeviceToHost, s) !=
             cudaSuccess)
@@ -1078,56 +1109,69 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
     // what the parked trajectories still need (from their progress; for those parked before
     // their first step twice the mean use of the trajectories that did start in this pass), and
     // their order for the next pass: largest estimate first
-    unsigned long long* est = reinterpret_cast<unsigned long long*>(r->counters + 10);
-    if (cudaMemsetAsync(est, 0, 2 * sizeof(unsigned long long), s) != cudaSuccess)
-      return bail(fail(GS_ERR_CUDA, "cudaMemsetAsync failed"));
-    const int eb = (parked + 255) / 256;
-    if (rsz == 8)
-      gs::k_park_estimate<double><<<eb, 256, 0, s>>>(r->park_list, parked,
-                                                    static_cast<const double*>(r->park_r), r->park_i,
-                                                    sys->d, t0, t1, C, est, r->park_key, KMAX);
-    else
-      gs::k_park_estimate<float><<<eb, 256, 0, s>>>(r->park_list, parked,
-                                                   static_cast<const float*>(r->park_r), r->park_i,
-                                                   sys->d, (float)t0, (float)t1, C, est,
-                                                   r->park_key, KMAX);
+    unsigned long long hest[2] = {0, 0};
+    if (sliced) {
+      std::memcpy(hest, r->host + 10, sizeof(hest));
+    } else {
+      if (cudaMemsetAsync(est, 0, 2 * sizeof(unsigned long long), s) != cudaSuccess)
+        return bail(fail(GS_ERR_CUDA, "cudaMemsetAsync failed"));
+      launch_park_estimate(r, parked, nullptr, sys->d, t0, t1, C, est, KMAX, s);
+      if (cudaMemcpyAsync(hest, est, sizeof(hest), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+          cudaStreamSynchronize(s) != cudaSuccess)
+        return bail(fail(GS_ERR_CUDA, "park estimate failed"));
+    }
+    // the next pass's order (queued; only that pass reads it)
     if ((st = counting_sort_desc(r, r->park_key, parked, KMAX, r->park_list, r->park_order, s)) !=
         GS_OK)
       return bail(st);
-    unsigned long long hest[2] = {0, 0};
-    if (cudaMemcpyAsync(hest, est, sizeof(hest), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaStreamSynchronize(s) != cudaSuccess)
-      return bail(fail(GS_ERR_CUDA, "park estimate failed"));
     const int64_t unstarted = (int64_t)hest[1];
     const int64_t started = std::max<int64_t>(1, nq - unstarted);
     const int64_t per_new = 2 * std::max<int64_t>(used - pass_start, 1) / started + 2;
     int64_t extra = std::max<int64_t>((int64_t)hest[0] + unstarted * per_new, 2 * (int64_t)parked);
     // after a pool found full the pool at most triples per pass, so that a wild estimate costs a
-    // pass, not the device's memory; and never beyond 80 % of the free device memory
+    // pass, not the device's memory
     if (!sliced) extra = std::min<int64_t>(extra, std::max<int64_t>(2 * used + 1024, 2 * (int64_t)parked));
-    size_t free_b = 0, total_b = 0;
+    // and never beyond 80 % of the device memory that is free (the cache's blocks count as
+    // free).  Asking the driver costs 0.1-0.8 ms, so it is asked only when the pool would take
+    // an eighth of the device or more, or when growing without asking failed.
     const int64_t chunk_b = (int64_t)C * E * (int64_t)rsz + 3 * (int64_t)sizeof(int);
-    if (cudaMemGetInfo(&free_b, &total_b) == cudaSuccess) {
-      // storage the cache holds counts as free
+    auto cap_by_free = [&](int64_t x) {
+      size_t free_b = 0, total_b = 0;
+      if (cudaMemGetInfo(&free_b, &total_b) != cudaSuccess) {
+        cudaGetLastError();
+        return x;
+      }
       cudaError_t ce;
       DeviceCtx* dc = device_ctx(&ce);
       if (dc) {
         std::lock_guard<std::mutex> lk(dc->mem_mu);
         free_b += dc->cached_bytes;
       }
-      extra = std::min<int64_t>(extra, std::max<int64_t>((int64_t)(free_b * 0.8) / chunk_b,
-                                                         2 * (int64_t)parked));
+      return std::min<int64_t>(x, std::max<int64_t>((int64_t)(free_b * 0.8) / chunk_b,
+                                                    2 * (int64_t)parked));
+    };
+    cudaError_t ce;
+    const DeviceCtx* dc = device_ctx(&ce);
+    const size_t total_mem = dc ? dc->total_mem : 0;
+    const bool asked = total_mem == 0 || (double)(used + extra) * chunk_b >= 0.125 * total_mem;
+    if (asked) extra = cap_by_free(extra);
+    int64_t want = used + extra + (int64_t)gs::CHUNK_BATCH * warps + 1024;
+    if (want > r->pool_chunks) {
+      st = grow_pool(r, want, used, s);
+      if (st != GS_OK && !asked) {
+        cudaGetLastError();
+        extra = cap_by_free(extra);
+        want = used + extra + (int64_t)gs::CHUNK_BATCH * warps + 1024;
+        st = want > r->pool_chunks ? grow_pool(r, want, used, s) : GS_OK;
+      }
+      if (st != GS_OK) return bail(st);
     }
-    const int64_t want = used + extra + (int64_t)gs::CHUNK_BATCH * warps + 1024;
-    if (want > r->pool_chunks && (st = grow_pool(r, want, used, s)) != GS_OK) return bail(st);
     // the next pass: the parked trajectories, a fresh queue, park count and summary, and chunks
     // handed out after the kept ones
-    r->host[0] = (int)used;
-    if (cudaMemsetAsync(r->counters, 0, 5 * sizeof(int), s) != cudaSuccess ||
-        cudaMemcpyAsync(r->counters + 1, r->host, sizeof(int), cudaMemcpyHostToDevice, s) !=
-            cudaSuccess ||
-        cudaStreamSynchronize(s) != cudaSuccess)
+    if (cudaMemsetAsync(r->counters, 0, 5 * sizeof(int), s) != cudaSuccess)
       return bail(fail(GS_ERR_CUDA, "counter reset failed"));
+    gs::k_set_int<<<1, 1, 0, s>>>(r->counters + 1, (int)used);
+    if (cudaGetLastError() != cudaSuccess) return bail(fail(GS_ERR_CUDA, "counter reset failed"));
     pass_start = used;
     nq = parked;
   }

@@ -1133,11 +1133,15 @@ __global__ void k_chunk_table(const int* chunk_traj, const int* chunk_seq, int n
 // keys[i] = that estimate of the remaining steps of list[i], capped at kmax (kmax for a
 // trajectory without progress): the order in which the next pass takes them, largest first.
 template <class R>
-__global__ void k_park_estimate(const int* list, int P, const R* park_r, const int* park_i, int D,
-                                R t0, R t1, int C, unsigned long long* out, int* keys, int kmax) {
+__global__ void k_park_estimate(const int* list, int P, const int* count, const R* park_r,
+                                const int* park_i, int D, R t0, R t1, int C,
+                                unsigned long long* out, int* keys, int kmax) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   unsigned long long chunks = 0, fresh = 0;
-  if (i < P) {
+  // the number of parked trajectories: P, or (count non-null) read on the device by a launch
+  // sized for at most P, queued behind the pass before the host has read it
+  const int n = count ? min(*count, P) : P;
+  if (i < n) {
     const int k = list[i];
     const R t = park_r[(size_t)k * (2 + 2 * D)];
     const int S = park_i[(size_t)k * 4];
@@ -1163,6 +1167,9 @@ __global__ void k_park_estimate(const int* list, int P, const R* park_r, const i
     if (fresh) atomicAdd(out + 1, fresh);
   }
 }
+
+// *p = v, queued on a stream (no host buffer to keep alive until the copy has run).
+__global__ void k_set_int(int* p, int v) { *p = v; }
 
 // The stored states of a record belong to the theta kept beside them.  Compares the caller's
 // theta with that copy bit for bit; any difference sets *stale (the caller zeroes it, or sets it
