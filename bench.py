@@ -50,10 +50,43 @@ FLOPS_VERN7_ADJOINT = {"lorenz63": 724, "nfw_mn": 2015}
 STIFF_COUNTS = {"robertson": (3, 8, 20, 9, 22), "hires": (8, 38, 77, 3, 32)}
 
 
+# Jacobian sparsity patterns the fields declare to the kernels (bit c of row r: J[r][c] can be
+# nonzero); the LU of the iteration matrix then works on that pattern and its fill-in only.
+JAC_PATTERN = {"hires": (0x07, 0x03, 0x1C, 0x0E, 0x70, 0xF8, 0xE0, 0xE0)}
+
+
 def lu_ops(d):
     """Dense LU without the pivot search: per column one reciprocal, k multipliers and 2 k^2 for
     the update of the k x k trailing block."""
     return sum(1 + k + 2 * k * k for k in range(d))
+
+
+def pattern_ops(field, d):
+    """(nnz(J), operations of one triangular solve pair, operations of the LU) on the field's
+    Jacobian pattern with the fill-in of elimination without row exchanges; the dense figures
+    (d^2, 2 d^2 - d, lu_ops(d)) for a field without a declared pattern.  Per column of the LU: one
+    reciprocal, m multipliers and 2 m u updates (m rows below, u columns right in the pattern);
+    a solve: 2 per strictly lower and strictly upper entry, and d multiplications by the pivots'
+    reciprocals."""
+    rows = JAC_PATTERN.get(field)
+    if rows is None:
+        return d * d, 2 * d * d - d, lu_ops(d)
+    J = [[bool((rows[r] >> c) & 1) for c in range(d)] for r in range(d)]
+    f = [[J[r][c] or r == c for c in range(d)] for r in range(d)]
+    for col in range(d):
+        for i in range(col + 1, d):
+            if f[i][col]:
+                for j in range(col + 1, d):
+                    if f[col][j]:
+                        f[i][j] = True
+    lu = 0
+    for col in range(d):
+        m = sum(f[r][col] for r in range(col + 1, d))
+        u = sum(f[col][q] for q in range(col + 1, d))
+        lu += 1 + m + 2 * m * u
+    nl = sum(f[r][c] for r in range(d) for c in range(r))
+    nu = sum(f[r][c] for r in range(d) for c in range(r + 1, d))
+    return sum(map(sum, J)), 2 * (nl + nu) + d, lu
 
 
 def stiff_flops(method, field):
@@ -62,14 +95,22 @@ def stiff_flops(method, field):
       ROS34PW2 attempt  c_J + 4 c_f + 17 d^2 + 53 d + LU(d) + 6
       ROS34PW2 adjoint  c_J + c_Jv + 4 c_f + 4 c_v + 51 d^2 + 92 d + LU(d) + 1
       Rosenbrock23 attempt  c_J + 2 c_f + 7 d^2 + 20 d + LU(d) + 7
-      Rosenbrock23 adjoint  c_J + c_Jv + 2 c_f + 2 c_v + 12 d^2 + 12 d + LU(d) + 3"""
+      Rosenbrock23 adjoint  c_J + c_Jv + 2 c_f + 2 c_v + 12 d^2 + 12 d + LU(d) + 3
+    Rosenbrock23's d^2 terms are the iteration matrix (d^2 + d), three solves in the attempt and
+    four (two of them transposed) in the adjoint, and the adjoint's two outer products into the
+    Jacobian cotangent (3 d^2): on a field with a declared Jacobian pattern they become nnz(J) + d,
+    the pattern's solves and 3 nnz(J), and LU(d) the pattern's elimination (pattern_ops) -- the
+    work of the kernels, which touch nothing else.  (ROS34PW2 is counted dense: its J G products
+    run over every entry, and no patterned field takes it.)"""
     d, cf, cv, cj, cjv = STIFF_COUNTS[field]
-    lu = lu_ops(d)
     if method == "ros34pw2":
+        lu = lu_ops(d)
         return (cj + 4 * cf + 17 * d * d + 53 * d + lu + 6,
                 cj + cjv + 4 * cf + 4 * cv + 51 * d * d + 92 * d + lu + 1)
-    return (cj + 2 * cf + 7 * d * d + 20 * d + lu + 7,
-            cj + cjv + 2 * cf + 2 * cv + 12 * d * d + 12 * d + lu + 3)
+    nnz, solve, lu = pattern_ops(field, d)
+    w = nnz + d
+    return (cj + 2 * cf + w + 3 * solve + 22 * d + lu + 7,
+            cj + cjv + 2 * cf + 2 * cv + w + 4 * solve + 3 * nnz + 15 * d + lu + 3)
 # The MLP field (4-32-32-4, tanh) counted by hand: f = 1,280 multiply-adds + 68 bias adds + 64
 # tanh = 2,692 ops; its pullback = the two transposed products (2 x 1,280 flops), the weight
 # outer products (2 x 1,280), 2 x 64 for tanh' and 68 bias cotangents = 5,316 ops; per accepted
@@ -90,7 +131,7 @@ TRAFFIC_PER_STEP = {
     "nfw_mn": {"record": 68.3, "adjoint": 71.0},
     "robertson": {"record": 38.9, "adjoint": 42.2},
     "robertson_rb23": {"record": 39.8, "adjoint": 43.7},
-    "hires": {"record": None, "adjoint": 89.4},
+    "hires": {"record": 80.5, "adjoint": 81.6},            # captured at 16,384 trajectories
     "lorenz63_vern7": {"adjoint": 45.2},                   # its record pass stays partly in L2
 }
 # FP64 pipe occupancy (sm__pipe_fp64_cycles_active, % of peak) of the same captures: how busy the
@@ -99,7 +140,7 @@ PIPE_BUSY_NCU = {
     "nfw_mn": {"record": 0.560, "adjoint": 0.723},
     "robertson": {"record": 0.387, "adjoint": 0.425},
     "robertson_rb23": {"record": 0.259, "adjoint": 0.393},
-    "hires": {"record": None, "adjoint": 0.217},
+    "hires": {"record": 0.204, "adjoint": 0.248},          # 16,384 trajectories: one wave
     "lorenz63_vern7": {"record": 0.439, "adjoint": 0.552},
     "log_halo": {"sens": 0.790},
 }

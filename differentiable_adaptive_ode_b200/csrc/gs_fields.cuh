@@ -157,6 +157,11 @@ struct FHires {
     dy[6] = r - k[11] * y[6];
     dy[7] = -r + k[11] * y[6];
   }
+  // Structural nonzeros of jac: bit c of row r (the iteration matrices' LU skips the rest).
+  GS_HD static constexpr bool jac_nz(int r, int c) {
+    constexpr unsigned rows[8] = {0x07, 0x03, 0x1C, 0x0E, 0x70, 0xF8, 0xE0, 0xE0};
+    return r >= 0 && r < 8 && c >= 0 && c < 8 && ((rows[r] >> c) & 1u) != 0;
+  }
   template <class R> GS_HD static void jac(const R* y, const Theta<R>& t, R* J) {
     const R* k = t.k;
 #pragma unroll

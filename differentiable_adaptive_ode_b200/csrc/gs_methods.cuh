@@ -649,6 +649,43 @@ template <class R> __device__ __forceinline__ R rbe(int i) {
   return R(B[i]) - R(BH[i]);
 }
 
+// Structural nonzeros of a field's Jacobian: every entry, unless the field declares its pattern
+// with jac_nz(r, c) (false: J[r][c] is zero for every state and parameter).
+template <class F, class = void>
+struct JacPattern {
+  static constexpr bool dense = true;
+  GS_HD static constexpr bool nz(int, int) { return true; }
+};
+template <class F>
+struct JacPattern<F, std::void_t<decltype(F::jac_nz(0, 0))>> {
+  static constexpr bool dense = false;
+  GS_HD static constexpr bool nz(int r, int c) { return F::jac_nz(r, c); }
+};
+// Entries of the LU factors of I - c J that elimination without row exchanges can make nonzero:
+// J's pattern with the diagonal, closed under elimination (fill-in).
+template <int D, class P>
+GS_HD constexpr bool lu_nz(int r, int c) {
+  bool f[D][D] = {};
+  for (int i = 0; i < D; ++i)
+    for (int j = 0; j < D; ++j) f[i][j] = i == j || P::nz(i, j);
+  for (int col = 0; col < D; ++col)
+    for (int i = col + 1; i < D; ++i)
+      if (f[i][col])
+        for (int j = col + 1; j < D; ++j)
+          if (f[col][j]) f[i][j] = true;
+  return f[r][c];
+}
+// fn(std::integral_constant<int, i>{}) for i = 0 .. N-1: loop indices usable in constant
+// expressions (if constexpr on the pattern).
+template <class Fn, int... I>
+__device__ __forceinline__ void static_for_seq(Fn& fn, std::integer_sequence<int, I...>) {
+  (fn(std::integral_constant<int, I>{}), ...);
+}
+template <int N, class Fn>
+__device__ __forceinline__ void static_for(Fn&& fn) {
+  static_for_seq(fn, std::make_integer_sequence<int, N>{});
+}
+
 // In-register LU of a D x D matrix with partial pivoting (largest |entry|, ties to the lowest
 // row).  The permutation is kept as a row map p[] so that solves index without data movement.
 // The pivots' reciprocals are formed once (the factorisation needs them anyway) and every solve
@@ -661,12 +698,69 @@ template <class R> __device__ __forceinline__ R rbe(int i) {
 // fields nearly never need one (none in 6,500 sampled steps of HIRES and Robertson, which keep
 // their diagonal dominant), and the results are those of the exchanging code in every case.
 // Every update is an explicit FMA, so that all kernels using it round alike.
-template <class R, int D>
+// With a declared Jacobian pattern P (HIRES: 25 of 64 entries), factor_shifted takes the entries
+// of the factors that can be nonzero only (the fill-in known at compile time, every loop index a
+// constant): about a tenth of the dense elimination's operations for HIRES and a third of the
+// solves', and a fraction of the registers.  It makes no row exchange: should partial pivoting
+// want one at some column, ok turns false and the caller makes that step again with the dense
+// LU (with_field_lu below) -- the same results as the dense code either way.
+template <class R, int D, class P = JacPattern<void>>
 struct SmallLU {
   R lu[D][D];
   R dinv[D];  // reciprocals of U's diagonal, formed once by factor(): the solves multiply
   int p[D];
   bool swapped;  // some row exchange was made: p is not the identity
+  bool ok;  // patterned factorisation: no row exchange was wanted (always true when dense)
+
+  // factors I - c J (J row-major, D x D)
+  __device__ __forceinline__ void factor_shifted(const R (&J)[D * D], R c) {
+    if constexpr (P::dense) {
+      R A[D][D];
+#pragma unroll
+      for (int r = 0; r < D; ++r)
+#pragma unroll
+        for (int q = 0; q < D; ++q) A[r][q] = fma(-c, J[r * D + q], r == q ? R(1) : R(0));
+      factor(A);
+      ok = true;
+    } else {
+      static_for<D>([&](auto ri) {
+        constexpr int r = decltype(ri)::value;
+        static_for<D>([&](auto qi) {
+          constexpr int q = decltype(qi)::value;
+          if constexpr (lu_nz<D, P>(r, q)) {
+            if constexpr (r == q || P::nz(r, q))
+              lu[r][q] = fma(-c, J[r * D + q], r == q ? R(1) : R(0));
+            else
+              lu[r][q] = R(0);  // fill-in
+          }
+        });
+      });
+      bool need = false;
+      static_for<D>([&](auto ci) {
+        constexpr int col = decltype(ci)::value;
+        static_for<D>([&](auto ri) {
+          constexpr int r = decltype(ri)::value;
+          if constexpr (r > col && lu_nz<D, P>(r, col))
+            need = need || (fabs(lu[r][col]) > fabs(lu[col][col]));
+        });
+        const R inv = R(1) / lu[col][col];
+        dinv[col] = inv;
+        static_for<D>([&](auto ri) {
+          constexpr int r = decltype(ri)::value;
+          if constexpr (r > col && lu_nz<D, P>(r, col)) {
+            const R l = lu[r][col] * inv;
+            lu[r][col] = l;
+            static_for<D>([&](auto qi) {
+              constexpr int q = decltype(qi)::value;
+              if constexpr (q > col && lu_nz<D, P>(col, q))
+                lu[r][q] = fma(-l, lu[col][q], lu[r][q]);
+            });
+          }
+        });
+      });
+      ok = !need;
+    }
+  }
   __device__ __forceinline__ void factor(const R (&A)[D][D]) {
     swapped = false;
 #pragma unroll
@@ -706,62 +800,119 @@ struct SmallLU {
   }
   // x = A^{-1} b   (P A = L U)
   __device__ __forceinline__ void solve(const R (&bb)[D], R (&x)[D]) const {
-    if (swapped) {
-#pragma unroll
-      for (int r = 0; r < D; ++r) {
-        R v = R(0);
-#pragma unroll
-        for (int s = 0; s < D; ++s) v = (p[r] == s) ? bb[s] : v;
-        x[r] = v;
-      }
-    } else {
+    if constexpr (!P::dense) {
 #pragma unroll
       for (int r = 0; r < D; ++r) x[r] = bb[r];
-    }
+      static_for<D>([&](auto ri) {
+        constexpr int r = decltype(ri)::value;
+        static_for<D>([&](auto qi) {
+          constexpr int q = decltype(qi)::value;
+          if constexpr (q < r && lu_nz<D, P>(r, q)) x[r] = fma(-lu[r][q], x[q], x[r]);
+        });
+      });
+      static_for<D>([&](auto ki) {
+        constexpr int r = D - 1 - decltype(ki)::value;
+        static_for<D>([&](auto qi) {
+          constexpr int q = decltype(qi)::value;
+          if constexpr (q > r && lu_nz<D, P>(r, q)) x[r] = fma(-lu[r][q], x[q], x[r]);
+        });
+        x[r] = x[r] * dinv[r];
+      });
+    } else {
+      if (swapped) {
 #pragma unroll
-    for (int r = 1; r < D; ++r)
+        for (int r = 0; r < D; ++r) {
+          R v = R(0);
 #pragma unroll
-      for (int c = 0; c < r; ++c) x[r] = fma(-lu[r][c], x[c], x[r]);
+          for (int s = 0; s < D; ++s) v = (p[r] == s) ? bb[s] : v;
+          x[r] = v;
+        }
+      } else {
 #pragma unroll
-    for (int r = D - 1; r >= 0; --r) {
+        for (int r = 0; r < D; ++r) x[r] = bb[r];
+      }
 #pragma unroll
-      for (int c = r + 1; c < D; ++c) x[r] = fma(-lu[r][c], x[c], x[r]);
-      x[r] = x[r] * dinv[r];
+      for (int r = 1; r < D; ++r)
+#pragma unroll
+        for (int c = 0; c < r; ++c) x[r] = fma(-lu[r][c], x[c], x[r]);
+#pragma unroll
+      for (int r = D - 1; r >= 0; --r) {
+#pragma unroll
+        for (int c = r + 1; c < D; ++c) x[r] = fma(-lu[r][c], x[c], x[r]);
+        x[r] = x[r] * dinv[r];
+      }
     }
   }
   // x = A^{-T} b:  A^T = U^T L^T P, so solve U^T z = b, L^T w = z, x = P^T w.
   __device__ __forceinline__ void solve_t(const R (&bb)[D], R (&x)[D]) const {
-    R z[D];
-#pragma unroll
-    for (int r = 0; r < D; ++r) {
-      R v = bb[r];
-#pragma unroll
-      for (int c = 0; c < r; ++c) v = fma(-lu[c][r], z[c], v);
-      z[r] = v * dinv[r];
-    }
-#pragma unroll
-    for (int r = D - 1; r >= 0; --r)
-#pragma unroll
-      for (int c = r + 1; c < D; ++c) z[r] = fma(-lu[c][r], z[c], z[r]);
-    if (swapped) {
-#pragma unroll
-      for (int s = 0; s < D; ++s) {
-        R v = R(0);
-#pragma unroll
-        for (int r = 0; r < D; ++r) v = (p[r] == s) ? z[r] : v;
-        x[s] = v;
-      }
+    if constexpr (!P::dense) {
+      static_for<D>([&](auto ri) {
+        constexpr int r = decltype(ri)::value;
+        R v = bb[r];
+        static_for<D>([&](auto qi) {
+          constexpr int q = decltype(qi)::value;
+          if constexpr (q < r && lu_nz<D, P>(q, r)) v = fma(-lu[q][r], x[q], v);
+        });
+        x[r] = v * dinv[r];
+      });
+      static_for<D>([&](auto ki) {
+        constexpr int r = D - 1 - decltype(ki)::value;
+        static_for<D>([&](auto qi) {
+          constexpr int q = decltype(qi)::value;
+          if constexpr (q > r && lu_nz<D, P>(q, r)) x[r] = fma(-lu[q][r], x[q], x[r]);
+        });
+      });
     } else {
+      R z[D];
 #pragma unroll
-      for (int s = 0; s < D; ++s) x[s] = z[s];
+      for (int r = 0; r < D; ++r) {
+        R v = bb[r];
+#pragma unroll
+        for (int c = 0; c < r; ++c) v = fma(-lu[c][r], z[c], v);
+        z[r] = v * dinv[r];
+      }
+#pragma unroll
+      for (int r = D - 1; r >= 0; --r)
+#pragma unroll
+        for (int c = r + 1; c < D; ++c) z[r] = fma(-lu[c][r], z[c], z[r]);
+      if (swapped) {
+#pragma unroll
+        for (int s = 0; s < D; ++s) {
+          R v = R(0);
+#pragma unroll
+          for (int r = 0; r < D; ++r) v = (p[r] == s) ? z[r] : v;
+          x[s] = v;
+        }
+      } else {
+#pragma unroll
+        for (int s = 0; s < D; ++s) x[s] = z[s];
+      }
     }
   }
 };
 
-template <class F, class R>
+// Runs step(lu) -- a Rosenbrock step that factors its iteration matrix into lu first and returns
+// false, before writing any output, when lu reports that partial pivoting would exchange rows --
+// with the LU of the field's Jacobian pattern, and again with the dense LU when that one would
+// have exchanged rows.  Fields without a declared pattern take the dense LU only.
+template <class F, class R, class Step>
+__device__ __forceinline__ void with_field_lu(Step&& step) {
+  if constexpr (JacPattern<F>::dense) {
+    SmallLU<R, F::D> lu;
+    step(lu);
+  } else {
+    SmallLU<R, F::D, JacPattern<F>> lu;
+    if (!step(lu)) {
+      SmallLU<R, F::D> ld;
+      step(ld);
+    }
+  }
+}
+
+template <class F, class R, class LU>
 __device__ __forceinline__ void ros_stages(const R (&y)[F::D], R h,
                                            const typename F::template Theta<R>& th,
-                                           const R (&J)[F::D * F::D], const SmallLU<R, F::D>& lu,
+                                           const R (&J)[F::D * F::D], const LU& lu,
                                            R (&k)[4][F::D]) {
   constexpr int D = F::D;
 #pragma unroll
@@ -790,19 +941,12 @@ __device__ __forceinline__ void ros_stages(const R (&y)[F::D], R h,
   }
 }
 
-template <class F, class R>
+template <class F, class R, class LU>
 __device__ __forceinline__ void ros_matrix(const R (&y)[F::D], R h,
                                            const typename F::template Theta<R>& th,
-                                           R (&J)[F::D * F::D], SmallLU<R, F::D>& lu) {
-  constexpr int D = F::D;
+                                           R (&J)[F::D * F::D], LU& lu) {
   F::jac(y, th, J);
-  const R gh = R(Ros34pw2::gamma) * h;
-  R Mx[D][D];
-#pragma unroll
-  for (int r = 0; r < D; ++r)
-#pragma unroll
-    for (int c = 0; c < D; ++c) Mx[r][c] = (r == c ? R(1) : R(0)) - gh * J[r * D + c];
-  lu.factor(Mx);
+  lu.factor_shifted(J, R(Ros34pw2::gamma) * h);
 }
 
 template <class F, class R>
@@ -810,26 +954,31 @@ __device__ __forceinline__ R ros_trial(const R (&y)[F::D], R h,
                                        const typename F::template Theta<R>& th,
                                        R (&ynew)[F::D], R rtol, R atol) {
   constexpr int D = F::D;
-  R J[D * D];
-  SmallLU<R, D> lu;
-  ros_matrix<F, R>(y, h, th, J, lu);
-  R k[4][D];
-  ros_stages<F, R>(y, h, th, J, lu, k);
-  R ev[D], sc[D];
+  R err_out = R(0);
+  with_field_lu<F, R>([&](auto& lu) {
+    R J[D * D];
+    ros_matrix<F, R>(y, h, th, J, lu);
+    if (!lu.ok) return false;
+    R k[4][D];
+    ros_stages<F, R>(y, h, th, J, lu, k);
+    R ev[D], sc[D];
 #pragma unroll
-  for (int c = 0; c < D; ++c) {
-    R s = rb<R>(0) * k[0][c];
-    R e = rbe<R>(0) * k[0][c];
+    for (int c = 0; c < D; ++c) {
+      R s = rb<R>(0) * k[0][c];
+      R e = rbe<R>(0) * k[0][c];
 #pragma unroll
-    for (int i = 1; i < 4; ++i) {
-      s += rb<R>(i) * k[i][c];
-      e += rbe<R>(i) * k[i][c];
+      for (int i = 1; i < 4; ++i) {
+        s += rb<R>(i) * k[i][c];
+        e += rbe<R>(i) * k[i][c];
+      }
+      ynew[c] = y[c] + s;
+      ev[c] = e;
+      sc[c] = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
     }
-    ynew[c] = y[c] + s;
-    ev[c] = e;
-    sc[c] = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
-  }
-  return scaled_rms(ev, sc);
+    err_out = scaled_rms(ev, sc);
+    return true;
+  });
+  return err_out;
 }
 
 // The ROS34PW2 replay map (no error estimate).
@@ -838,18 +987,21 @@ __device__ __forceinline__ void ros_replay_step(const R (&y)[F::D], R h,
                                                 const typename F::template Theta<R>& th,
                                                 R (&ynew)[F::D]) {
   constexpr int D = F::D;
-  R J[D * D];
-  SmallLU<R, D> lu;
-  ros_matrix<F, R>(y, h, th, J, lu);
-  R k[4][D];
-  ros_stages<F, R>(y, h, th, J, lu, k);
+  with_field_lu<F, R>([&](auto& lu) {
+    R J[D * D];
+    ros_matrix<F, R>(y, h, th, J, lu);
+    if (!lu.ok) return false;
+    R k[4][D];
+    ros_stages<F, R>(y, h, th, J, lu, k);
 #pragma unroll
-  for (int c = 0; c < D; ++c) {
-    R s = rb<R>(0) * k[0][c];
+    for (int c = 0; c < D; ++c) {
+      R s = rb<R>(0) * k[0][c];
 #pragma unroll
-    for (int i = 1; i < 4; ++i) s += rb<R>(i) * k[i][c];
-    ynew[c] = y[c] + s;
-  }
+      for (int i = 1; i < 4; ++i) s += rb<R>(i) * k[i][c];
+      ynew[c] = y[c] + s;
+    }
+    return true;
+  });
 }
 
 // ----------------------------------------------------------------------------------------------
@@ -867,26 +1019,19 @@ struct Rb23 {
   static constexpr double e32 = 7.4142135623730951;   // 6 + sqrt 2
 };
 
-template <class F, class R>
+template <class F, class R, class LU>
 __device__ __forceinline__ void rb23_matrix(const R (&y)[F::D], R h,
                                             const typename F::template Theta<R>& th,
-                                            R (&J)[F::D * F::D], SmallLU<R, F::D>& lu) {
-  constexpr int D = F::D;
+                                            R (&J)[F::D * F::D], LU& lu) {
   F::jac(y, th, J);
-  const R hd = h * R(Rb23::d);
-  R Mx[D][D];
-#pragma unroll
-  for (int r = 0; r < D; ++r)
-#pragma unroll
-    for (int c = 0; c < D; ++c) Mx[r][c] = (r == c ? R(1) : R(0)) - hd * J[r * D + c];
-  lu.factor(Mx);
+  lu.factor_shifted(J, h * R(Rb23::d));
 }
 
 // k1, F1 and k2 of the step from y (F0 = f(y) given).
-template <class F, class R>
+template <class F, class R, class LU>
 __device__ __forceinline__ void rb23_stages(const R (&y)[F::D], R h,
                                             const typename F::template Theta<R>& th,
-                                            const SmallLU<R, F::D>& lu, const R (&F0)[F::D],
+                                            const LU& lu, const R (&F0)[F::D],
                                             R (&k1)[F::D], R (&F1)[F::D], R (&k2)[F::D]) {
   constexpr int D = F::D;
   lu.solve(F0, k1);
@@ -909,27 +1054,32 @@ __device__ __forceinline__ R rb23_trial(const R (&y)[F::D], R h,
                                         const R (&F0)[F::D], R (&ynew)[F::D], R (&F2)[F::D],
                                         R rtol, R atol) {
   constexpr int D = F::D;
-  R J[D * D];
-  SmallLU<R, D> lu;
-  rb23_matrix<F, R>(y, h, th, J, lu);
-  R k1[D], F1[D], k2[D];
-  rb23_stages<F, R>(y, h, th, lu, F0, k1, F1, k2);
+  R err_out = R(0);
+  with_field_lu<F, R>([&](auto& lu) {
+    R J[D * D];
+    rb23_matrix<F, R>(y, h, th, J, lu);
+    if (!lu.ok) return false;
+    R k1[D], F1[D], k2[D];
+    rb23_stages<F, R>(y, h, th, lu, F0, k1, F1, k2);
 #pragma unroll
-  for (int c = 0; c < D; ++c) ynew[c] = y[c] + h * k2[c];
-  F::f(ynew, th, F2);
-  R r[D], k3[D];
+    for (int c = 0; c < D; ++c) ynew[c] = y[c] + h * k2[c];
+    F::f(ynew, th, F2);
+    R r[D], k3[D];
 #pragma unroll
-  for (int c = 0; c < D; ++c)
-    r[c] = F2[c] - R(Rb23::e32) * (k2[c] - F1[c]) - R(2) * (k1[c] - F0[c]);
-  lu.solve(r, k3);
-  R ev[D], sc[D];
+    for (int c = 0; c < D; ++c)
+      r[c] = F2[c] - R(Rb23::e32) * (k2[c] - F1[c]) - R(2) * (k1[c] - F0[c]);
+    lu.solve(r, k3);
+    R ev[D], sc[D];
 #pragma unroll
-  for (int c = 0; c < D; ++c) {
-    const R e = h * (k1[c] - R(2) * k2[c] + k3[c]) * R(1.0 / 6.0);
-    ev[c] = e;
-    sc[c] = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
-  }
-  return scaled_rms(ev, sc);
+    for (int c = 0; c < D; ++c) {
+      const R e = h * (k1[c] - R(2) * k2[c] + k3[c]) * R(1.0 / 6.0);
+      ev[c] = e;
+      sc[c] = atol + rtol * fmax(fabs(y[c]), fabs(ynew[c]));
+    }
+    err_out = scaled_rms(ev, sc);
+    return true;
+  });
+  return err_out;
 }
 
 // The Rosenbrock23 replay map y + h k2 (no error estimate).
@@ -938,14 +1088,17 @@ __device__ __forceinline__ void rb23_replay_step(const R (&y)[F::D], R h,
                                                  const typename F::template Theta<R>& th,
                                                  R (&ynew)[F::D]) {
   constexpr int D = F::D;
-  R J[D * D];
-  SmallLU<R, D> lu;
-  rb23_matrix<F, R>(y, h, th, J, lu);
-  R F0[D], k1[D], F1[D], k2[D];
-  F::f(y, th, F0);
-  rb23_stages<F, R>(y, h, th, lu, F0, k1, F1, k2);
+  with_field_lu<F, R>([&](auto& lu) {
+    R J[D * D];
+    rb23_matrix<F, R>(y, h, th, J, lu);
+    if (!lu.ok) return false;
+    R F0[D], k1[D], F1[D], k2[D];
+    F::f(y, th, F0);
+    rb23_stages<F, R>(y, h, th, lu, F0, k1, F1, k2);
 #pragma unroll
-  for (int c = 0; c < D; ++c) ynew[c] = y[c] + h * k2[c];
+    for (int c = 0; c < D; ++c) ynew[c] = y[c] + h * k2[c];
+    return true;
+  });
 }
 
 // Reverse-mode step of the Rosenbrock23 replay map with h fixed.  With u = k2 - k1
@@ -959,44 +1112,47 @@ __device__ __forceinline__ void rb23_adjoint_step(const R (&y)[F::D], R h,
                                                   const typename F::template Theta<R>& th,
                                                   R (&lam)[F::D], R (&thb)[F::M]) {
   constexpr int D = F::D;
-  R J[D * D];
-  SmallLU<R, D> lu;
-  rb23_matrix<F, R>(y, h, th, J, lu);
-  R F0[D], k1[D], F1[D], k2[D];
-  F::f(y, th, F0);
-  rb23_stages<F, R>(y, h, th, lu, F0, k1, F1, k2);
-  const R hd = h * R(Rb23::d);
-  R Jb[D * D], yb[D], k2b[D], mu[D], k1b[D], tmp[D];
+  with_field_lu<F, R>([&](auto& lu) {
+    R J[D * D];
+    rb23_matrix<F, R>(y, h, th, J, lu);
+    if (!lu.ok) return false;
+    R F0[D], k1[D], F1[D], k2[D];
+    F::f(y, th, F0);
+    rb23_stages<F, R>(y, h, th, lu, F0, k1, F1, k2);
+    const R hd = h * R(Rb23::d);
+    R Jb[D * D], yb[D], k2b[D], mu[D], k1b[D], tmp[D];
 #pragma unroll
-  for (int c = 0; c < D; ++c) { yb[c] = lam[c]; k2b[c] = h * lam[c]; }
-  lu.solve_t(k2b, mu);                               // mu2
+    for (int c = 0; c < D; ++c) { yb[c] = lam[c]; k2b[c] = h * lam[c]; }
+    lu.solve_t(k2b, mu);                               // mu2
 #pragma unroll
-  for (int r = 0; r < D; ++r)
+    for (int r = 0; r < D; ++r)
 #pragma unroll
-    for (int c = 0; c < D; ++c) Jb[r * D + c] = hd * mu[r] * (k2[c] - k1[c]);
-  R Y1[D];
+      for (int c = 0; c < D; ++c) Jb[r * D + c] = hd * mu[r] * (k2[c] - k1[c]);
+    R Y1[D];
 #pragma unroll
-  for (int c = 0; c < D; ++c) {
-    k1b[c] = k2b[c] - mu[c];
-    Y1[c] = y[c] + R(0.5) * h * k1[c];
-  }
-  F::vjp(Y1, th, mu, tmp, thb);                      // Y1b
+    for (int c = 0; c < D; ++c) {
+      k1b[c] = k2b[c] - mu[c];
+      Y1[c] = y[c] + R(0.5) * h * k1[c];
+    }
+    F::vjp(Y1, th, mu, tmp, thb);                      // Y1b
 #pragma unroll
-  for (int c = 0; c < D; ++c) {
-    yb[c] += tmp[c];
-    k1b[c] += R(0.5) * h * tmp[c];
-  }
-  lu.solve_t(k1b, mu);                               // mu1
+    for (int c = 0; c < D; ++c) {
+      yb[c] += tmp[c];
+      k1b[c] += R(0.5) * h * tmp[c];
+    }
+    lu.solve_t(k1b, mu);                               // mu1
 #pragma unroll
-  for (int r = 0; r < D; ++r)
+    for (int r = 0; r < D; ++r)
 #pragma unroll
-    for (int c = 0; c < D; ++c) Jb[r * D + c] += hd * mu[r] * k1[c];
-  F::vjp(y, th, mu, tmp, thb);
+      for (int c = 0; c < D; ++c) Jb[r * D + c] += hd * mu[r] * k1[c];
+    F::vjp(y, th, mu, tmp, thb);
 #pragma unroll
-  for (int c = 0; c < D; ++c) yb[c] += tmp[c];
-  F::jac_vjp(y, th, Jb, yb, thb);
+    for (int c = 0; c < D; ++c) yb[c] += tmp[c];
+    F::jac_vjp(y, th, Jb, yb, thb);
 #pragma unroll
-  for (int c = 0; c < D; ++c) lam[c] = yb[c];
+    for (int c = 0; c < D; ++c) lam[c] = yb[c];
+    return true;
+  });
 }
 
 // Reverse-mode step of the ROS34PW2 replay map with h fixed.  With M = I - gamma h J,
@@ -1012,66 +1168,69 @@ __device__ __forceinline__ void ros_adjoint_step(const R (&y)[F::D], R h,
                                                  const typename F::template Theta<R>& th,
                                                  R (&lam)[F::D], R (&thb)[F::M]) {
   constexpr int D = F::D;
-  R J[D * D];
-  SmallLU<R, D> lu;
-  ros_matrix<F, R>(y, h, th, J, lu);
-  R k[4][D];
-  ros_stages<F, R>(y, h, th, J, lu, k);
-  R kb[4][D], Jb[D * D], yb[D];
+  with_field_lu<F, R>([&](auto& lu) {
+    R J[D * D];
+    ros_matrix<F, R>(y, h, th, J, lu);
+    if (!lu.ok) return false;
+    R k[4][D];
+    ros_stages<F, R>(y, h, th, J, lu, k);
+    R kb[4][D], Jb[D * D], yb[D];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int c = 0; c < D; ++c) kb[i][c] = rb<R>(i) * lam[c];
+      for (int c = 0; c < D; ++c) kb[i][c] = rb<R>(i) * lam[c];
 #pragma unroll
-  for (int i = 0; i < D * D; ++i) Jb[i] = R(0);
+    for (int i = 0; i < D * D; ++i) Jb[i] = R(0);
 #pragma unroll
-  for (int c = 0; c < D; ++c) yb[c] = lam[c];
-  const R gh = R(Ros34pw2::gamma) * h;
+    for (int c = 0; c < D; ++c) yb[c] = lam[c];
+    const R gh = R(Ros34pw2::gamma) * h;
 #pragma unroll
-  for (int i = 3; i >= 0; --i) {
-    R mu[D];
-    lu.solve_t(kb[i], mu);
-    R Y[D], G[D];
-#pragma unroll
-    for (int c = 0; c < D; ++c) {
-      R u = R(0), g = R(0);
-#pragma unroll
-      for (int j = 0; j < i; ++j) {
-        u += ral<R>(i, j) * k[j][c];
-        g += rga<R>(i, j) * k[j][c];
-      }
-      Y[c] = y[c] + u;
-      G[c] = g;
-    }
-#pragma unroll
-    for (int r = 0; r < D; ++r)
-#pragma unroll
-      for (int c = 0; c < D; ++c) Jb[r * D + c] += mu[r] * (gh * k[i][c] + h * G[c]);
-    R fb[D], Yb[D];
-#pragma unroll
-    for (int c = 0; c < D; ++c) fb[c] = h * mu[c];
-    F::vjp(Y, th, fb, Yb, thb);
-    if (i > 0) {
-      R Jtmu[D];
+    for (int i = 3; i >= 0; --i) {
+      R mu[D];
+      lu.solve_t(kb[i], mu);
+      R Y[D], G[D];
 #pragma unroll
       for (int c = 0; c < D; ++c) {
-        R s = R(0);
+        R u = R(0), g = R(0);
 #pragma unroll
-        for (int r = 0; r < D; ++r) s += J[r * D + c] * mu[r];
-        Jtmu[c] = h * s;
+        for (int j = 0; j < i; ++j) {
+          u += ral<R>(i, j) * k[j][c];
+          g += rga<R>(i, j) * k[j][c];
+        }
+        Y[c] = y[c] + u;
+        G[c] = g;
       }
 #pragma unroll
-      for (int j = 0; j < i; ++j)
+      for (int r = 0; r < D; ++r)
 #pragma unroll
-        for (int c = 0; c < D; ++c)
-          kb[j][c] += ral<R>(i, j) * Yb[c] + rga<R>(i, j) * Jtmu[c];
+        for (int c = 0; c < D; ++c) Jb[r * D + c] += mu[r] * (gh * k[i][c] + h * G[c]);
+      R fb[D], Yb[D];
+#pragma unroll
+      for (int c = 0; c < D; ++c) fb[c] = h * mu[c];
+      F::vjp(Y, th, fb, Yb, thb);
+      if (i > 0) {
+        R Jtmu[D];
+#pragma unroll
+        for (int c = 0; c < D; ++c) {
+          R s = R(0);
+#pragma unroll
+          for (int r = 0; r < D; ++r) s += J[r * D + c] * mu[r];
+          Jtmu[c] = h * s;
+        }
+#pragma unroll
+        for (int j = 0; j < i; ++j)
+#pragma unroll
+          for (int c = 0; c < D; ++c)
+            kb[j][c] += ral<R>(i, j) * Yb[c] + rga<R>(i, j) * Jtmu[c];
+      }
+#pragma unroll
+      for (int c = 0; c < D; ++c) yb[c] += Yb[c];
     }
+    F::jac_vjp(y, th, Jb, yb, thb);
 #pragma unroll
-    for (int c = 0; c < D; ++c) yb[c] += Yb[c];
-  }
-  F::jac_vjp(y, th, Jb, yb, thb);
-#pragma unroll
-  for (int c = 0; c < D; ++c) lam[c] = yb[c];
+    for (int c = 0; c < D; ++c) lam[c] = yb[c];
+    return true;
+  });
 }
 
 }  // namespace gs

@@ -18,6 +18,11 @@ its rsqrt beside).
 The logarithm of the stellar field (gs::log_tab, Tang's table-driven method) is within half an
 ulp plus its few roundings: the bar is 0.6 ulp (CUDA's log, beside it, within 1), with +inf,
 +0, a negative argument, NaN and a subnormal mapped to +inf, -inf and NaN.
+The LU of a patterned iteration matrix (HIRES's Jacobian pattern: only the entries the fill-in
+reaches, no row exchange) reports a wanted exchange exactly when the dense LU makes one, gives
+the dense solutions of W x = b and W^T x = b bit for bit otherwise, and a step run through
+with_field_lu (patterned, else dense) gives the dense solution in every case: 20,000 random
+matrices of that pattern, half of them made to need row exchanges; residuals at rounding level.
 """
 import json
 import os
@@ -58,3 +63,12 @@ def test_kernel_math_helpers_within_bounds(tmp_path):
     assert res["log"]["ulp"] <= 0.6, res
     assert res["log"]["cuda_ulp"] <= 1.0, res
     assert res["log"]["special_ok"] == 1, res
+    # the patterned LU asks for the dense one exactly when pivoting exchanges rows, equals it
+    # otherwise, and a step through with_field_lu gives the dense solution in every case
+    assert res["lu"]["n"] == 20000, res
+    assert res["lu"]["fallback"] >= 2000 and res["lu"]["n"] - res["lu"]["fallback"] >= 2000, res
+    assert res["lu"]["flag_mismatch"] == 0, res
+    assert res["lu"]["mismatch"] == 0, res
+    # backward error of partial pivoting: n 2^(n-1) u = 8 * 128 * 2^-53 ~ 1.1e-13 for n = 8 (the
+    # growth bound), with the residual's own rounding: a decade of room
+    assert res["lu"]["resid"] <= 1e-12, res
