@@ -40,7 +40,7 @@ struct RecBounds {
 };
 #ifdef GS_CHECKED
 __device__ unsigned long long g_gs_violations;
-__device__ double g_gs_scratch_entry[64];
+__device__ __align__(16) double g_gs_scratch_entry[64];  // 16-byte loads and stores of entries
 __device__ __forceinline__ void gs_violation() { atomicAdd(&g_gs_violations, 1ull); }
 #endif
 
@@ -278,6 +278,35 @@ __device__ __forceinline__ void store_entry(R* e, R t, R h, const R (&y)[E - 2])
 #pragma unroll
     for (int c = 0; c < E - 2; ++c) e[2 + c] = y[c];
   }
+}
+
+// One record entry's step size and state read by a replay kernel (read-only path): as 16-byte
+// loads when the entry fills whole 16-byte words (fp64 entries of an even number of reals), the
+// counterpart of store_entry.
+template <class R, int E>
+__device__ __forceinline__ void load_entry(const R* e, R& t, R& h, R (&y)[E - 2]) {
+  if constexpr (E * sizeof(R) % 16 == 0 && sizeof(R) == 8) {
+    const double2* v = reinterpret_cast<const double2*>(e);
+    const double2 th = __ldg(v);
+    t = th.x;
+    h = th.y;
+#pragma unroll
+    for (int c = 0; c < (E - 2) / 2; ++c) {
+      const double2 w = __ldg(v + 1 + c);
+      y[2 * c] = w.x;
+      y[2 * c + 1] = w.y;
+    }
+  } else {
+    t = __ldg(e);
+    h = __ldg(e + 1);
+#pragma unroll
+    for (int c = 0; c < E - 2; ++c) y[c] = __ldg(e + 2 + c);
+  }
+}
+template <class R, int E>
+__device__ __forceinline__ void load_entry(const R* e, R& h, R (&y)[E - 2]) {
+  R t;
+  load_entry<R, E>(e, t, h, y);
 }
 
 // Per-warp ring of trajectories whose start-up is done (id, status, starting step, f(y0)).
@@ -749,10 +778,8 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
           pf_pending = false;
         }
         const R* e = chunk_entry<L>(p.pool, cur_ch, n, p.bounds);
-        const R h = __ldg(e + 1);
-        R y[D];
-#pragma unroll
-        for (int c = 0; c < D; ++c) y[c] = __ldg(e + 2 + c);
+        R h, y[D];
+        load_entry<R, L::E>(e, h, y);
         if constexpr (METHOD == M_TSIT5) tsit5_adjoint_step<F, R>(y, h, th, lam, thb, tape, blockDim.x);
         else if constexpr (METHOD == M_VERN7) vern7_adjoint_step<F, R>(y, h, th, lam, thb, tape, blockDim.x);
         else if constexpr (METHOD == M_RB23) rb23_adjoint_step<F, R>(y, h, th, lam, thb);
@@ -896,6 +923,7 @@ __device__ __forceinline__ const R* rec_entry(const ReplayParams<R>& p, long lon
 
 template <class F, class R, int METHOD>
 __global__ void __launch_bounds__(128) k_replay_outputs(OutParams<R> q) {
+  using L = RecLayout<F, R>;
   constexpr int D = F::D;
   const ReplayParams<R>& p = q.rp;
   const int J = q.ot.J;
@@ -922,11 +950,7 @@ __global__ void __launch_bounds__(128) k_replay_outputs(OutParams<R> q) {
 #pragma unroll
     for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
     for (int n = 0; n < S && j < J; ++n) {
-      const R* e = rec_entry<F, R>(p, cbase, n);
-      t = e[0];
-      h = e[1];
-#pragma unroll
-      for (int c = 0; c < D; ++c) y[c] = e[2 + c];
+      load_entry<R, L::E>(rec_entry<F, R>(p, cbase, n), t, h, y);
       const R tnext = (n + 1 < S) ? rec_entry<F, R>(p, cbase, n + 1)[0] : q.ot.t1;
       while (j < J && q.ot.tau[j] < tnext) {
         R yo[D];
@@ -1000,10 +1024,8 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
     for (int n = S - 1; n >= 0; --n) {
       const R* e = chunk_entry<L>(p.pool, chunk_at(p.chunk_table, cbase + n / L::C, p.bounds), n,
                                   p.bounds);
-      const R t = e[0], h = e[1];
-      R y[D];
-#pragma unroll
-      for (int c = 0; c < D; ++c) y[c] = e[2 + c];
+      R t, h, y[D];
+      load_entry<R, L::E>(e, t, h, y);
       int jlo = jcur;
       while (jlo > 0 && (n == 0 || q.ot.tau[jlo - 1] >= t)) --jlo;
       R lacc[D];
