@@ -1151,7 +1151,7 @@ __global__ void k_chunk_table(const int* chunk_traj, const int* chunk_seq, int n
 
 // Chunks the parked trajectories of a record pass still need, estimated from their progress:
 // a trajectory parked at time t after S accepted steps needs about S (t1 - t) / (t - t0) more
-// (at most 64 S; taken with a 25 % margin); out[1] counts those parked before their first step.  With `keys`,
+// (at most 128 S; taken with a 25 % margin); out[1] counts those parked before their first step.  With `keys`,
 // keys[i] = that estimate of the remaining steps of list[i], capped at kmax (kmax for a
 // trajectory without progress): the order in which the next pass takes them, largest first.
 template <class R>
@@ -1168,9 +1168,9 @@ __global__ void k_park_estimate(const int* list, int P, const int* count, const 
     const R t = park_r[(size_t)k * (2 + 2 * D)];
     const int S = park_i[(size_t)k * 4];
     if (t > t0) {
-      // progress in time is a poor guide after a stiff start (tiny early steps): at most 64
+      // progress in time is a poor guide after a stiff start (tiny early steps): at most 128
       // times the steps taken so far
-      const double rem = fmin(double(S + 1) * double(t1 - t) / double(t - t0), 64.0 * (S + 1));
+      const double rem = fmin(double(S + 1) * double(t1 - t) / double(t - t0), 128.0 * (S + 1));
       chunks = (unsigned long long)fmin(1.25 * rem / C + 2.0, double(1 << 20));
       if (keys) keys[i] = (int)fmin(rem, double(kmax));
     } else {
