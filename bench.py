@@ -126,7 +126,7 @@ SMS, FP64_LANES, FP32_LANES = 148, 64, 128
 # change leaves stale is withheld as None until captured again); the Verner 7 Lorenz record
 # keeps part of its record in L2 at the captured size, so it has none.
 TRAFFIC_PER_STEP = {
-    "nfw_mn": {"record": 68.3, "adjoint": 71.1},
+    "nfw_mn": {"record": 67.3, "adjoint": 85.1},
     "robertson": {"record": 38.9, "adjoint": 42.2},
     "robertson_rb23": {"record": 39.8, "adjoint": 43.6},
     "hires": {"record": 80.5, "adjoint": 81.6},            # captured at 16,384 trajectories
@@ -135,7 +135,7 @@ TRAFFIC_PER_STEP = {
 # FP64 pipe occupancy (sm__pipe_fp64_cycles_active, % of peak) of the same captures: how busy the
 # pipe is, transcendental sequences included, next to the algorithmic fraction
 PIPE_BUSY_NCU = {
-    "nfw_mn": {"record": 0.560, "adjoint": 0.743},
+    "nfw_mn": {"record": 0.564, "adjoint": 0.741},
     "robertson": {"record": 0.408, "adjoint": 0.474},
     "robertson_rb23": {"record": 0.299, "adjoint": 0.459},
     "hires": {"record": 0.204, "adjoint": 0.253},          # 16,384 trajectories: one wave

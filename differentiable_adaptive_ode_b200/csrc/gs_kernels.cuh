@@ -67,11 +67,29 @@ __device__ __forceinline__ R* chunk_entry(R* pool, int ch, int n, const RecBound
   return pool + ((size_t)ch * L::C + (n % L::C)) * L::E;
 }
 
-// Record chunk: C accepted steps of one trajectory, entry = (t, h, y[0..D-1]) contiguous.
+// Record writes, two forms.  Direct: each accepted step's entry goes straight from the lane's
+// registers into its current chunk (taken from the warp's block before the attempt), with no
+// staging and no flush.  Staged: the entry is staged in shared memory and a full chunk is
+// copied out by the whole warp as one coalesced block.  Measured on B200 at 2^20 trajectories
+// (record call): the stellar field, whose step is long, 24.8 -> 22.1 ms direct (fp32 3.21 ->
+// 2.89); Lorenz-63, whose step is short and whose record rate is high, 5.44 staged against 6.13
+// direct.  Fields with long steps take the direct form.
+template <class F, class R> struct RecDirect { static constexpr bool value = false; };
+template <class R> struct RecDirect<FNfwMiyamotoNagai, R> { static constexpr bool value = true; };
+template <class R> struct RecDirect<FHires, R> { static constexpr bool value = true; };
+
+// Record chunk: C accepted steps of one trajectory, entry = (t, h, y[0..D-1]) contiguous: 8 steps
+// for entries under 48 bytes, and for direct fields while the chunk stays within 512 bytes (no
+// shared-memory stage to hold it; half the chunks to hand out, label and list in the chunk table
+// and half the chunk changes of the replay kernels: the stellar step 24.33 -> 24.12 ms at 2^20);
+// 4 otherwise (HIRES's 80-byte entries: 8 measured slower in its record kernel, 8.45 -> 8.79 ms).
 template <class F, class R>
 struct RecLayout {
   static constexpr int E = 2 + F::D;                                     // reals per step
-  static constexpr int C = (E * int(sizeof(R)) >= 48) ? 4 : 8;           // steps per chunk
+  static constexpr int C = (E * int(sizeof(R)) < 48 ||
+                            (RecDirect<F, R>::value && 8 * E * int(sizeof(R)) <= 512))
+                               ? 8
+                               : 4;                                      // steps per chunk
   static constexpr int STAGE_STRIDE = C * E + 1;                         // per-lane smem stride
 };
 
@@ -244,17 +262,6 @@ template <> struct Tune<FLogHalo, double> {
 
 // Record chunks are reserved from the global bump counter CHUNK_BATCH at a time per warp.
 constexpr int CHUNK_BATCH = 32;
-// Record writes, two forms.  Direct: each accepted step's entry goes straight from the lane's
-// registers into its current chunk (taken from the warp's block before the attempt), with no
-// staging and no flush.  Staged: the entry is staged in shared memory and a full chunk is
-// copied out by the whole warp as one coalesced block.  Measured on B200 at 2^20 trajectories
-// (record call): the stellar field, whose step is long, 24.8 -> 22.1 ms direct (fp32 3.21 ->
-// 2.89); Lorenz-63, whose step is short and whose record rate is high, 5.44 staged against 6.13
-// direct.  Fields with long steps take the direct form.
-template <class F, class R> struct RecDirect { static constexpr bool value = false; };
-template <class R> struct RecDirect<FNfwMiyamotoNagai, R> { static constexpr bool value = true; };
-template <class R> struct RecDirect<FHires, R> { static constexpr bool value = true; };
-
 // One record entry (t, h, y) written from a lane's registers.  When the entry fills whole
 // 16-byte words (the pool is 256-byte aligned and entries are contiguous), it goes out as 16-byte
 // vector stores: half (fp64) or a quarter (fp32) of the store instructions, and of the requests
