@@ -278,6 +278,8 @@ struct gs_record {
   size_t red_bytes = 0, part_bytes = 0;
   void* y1_scratch = nullptr;    // y_S of gs_replay_forward when the caller passes no y1
   size_t y1_bytes = 0;
+  void* out_scratch = nullptr;   // output cotangents pulled back to their steps [N][J][d]
+  size_t out_bytes = 0;
   // the theta the stored states y_n were computed at ([N][m], or [m] when shared); counters[8]
   // is the flag the device comparison with a caller's theta raises
   void* theta_kept = nullptr;
@@ -1430,6 +1432,18 @@ gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_
       r->part_bytes = needp;
     }
   }
+  // outputs before t1 (compared in the record's precision, as the kernels compare them)
+  const bool f32 = rec->rsz == sizeof(float);
+  int jS = 0;
+  while (jS < J && (f32 ? (float)tau[jS] < (float)rec->t1 : tau[jS] < rec->t1)) ++jS;
+  const size_t need_g = (size_t)N * jS * rec->sys.d * rec->rsz;
+  if (r->out_bytes < need_g) {
+    free_ptr(r->out_scratch, s);
+    r->out_scratch = nullptr;
+    r->out_bytes = 0;
+    GS_CUDA(dalloc(&r->out_scratch, need_g, s));
+    r->out_bytes = need_g;
+  }
   int* queue = nullptr;
   GS_CUDA(take_counter(s, &queue));
   return dispatch(rec->sys, [&]<class F, class R, int METHOD>() {
@@ -1453,8 +1467,16 @@ gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_
       p.bounds = bounds_of(rec);
       q.dL_dyout = static_cast<const R*>(dL_dyout);
       fill_times<R>(q.ot, rec, J, tau);
-      auto kern = gs::k_adjoint_outputs<F, R, METHOD>;
+      q.jS = jS;
+      q.G = static_cast<R*>(r->out_scratch);
       const size_t smem = adjoint_smem<F, R, METHOD>();
+      if (jS > 0) {  // the output pullbacks, then the walk that adds them
+        auto first = gs::k_output_pullbacks<F, R, METHOD>;
+        if (smem > 48 * 1024)
+          GS_CUDA(cudaFuncSetAttribute(first, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        first<<<(unsigned)((N + BLOCK - 1) / BLOCK), BLOCK, smem, s>>>(q);
+      }
+      auto kern = gs::k_adjoint_outputs<F, R, METHOD>;
       if (smem > 48 * 1024)
         GS_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
       kern<<<persistent_grid(kern, smem, N), BLOCK, smem, s>>>(q);
@@ -1625,6 +1647,7 @@ void gs_record_destroy(gs_record* r) {
   free_ptr(r->nsteps, s); free_ptr(r->status, s); free_ptr(r->offsets, s); free_ptr(r->choff, s);
   free_ptr(r->tiles, s); free_ptr(r->counters, s);
   free_ptr(r->red_scratch, s); free_ptr(r->red_partials, s); free_ptr(r->y1_scratch, s);
+  free_ptr(r->out_scratch, s);
   free_ptr(r->theta_kept, s);
   free_ptr(r->perm, s); free_ptr(r->bins, s); free_ptr(r->binoff, s); free_ptr(r->btiles, s);
   free_ptr(r->park_list, s); free_ptr(r->park_r, s);

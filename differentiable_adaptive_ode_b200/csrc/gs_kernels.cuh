@@ -921,8 +921,8 @@ struct OutParams {
 };
 
 
-template <class F, class R>
-__device__ __forceinline__ const R* rec_entry(const ReplayParams<R>& p, long long cbase, int n) {
+template <class F, class R, class P>
+__device__ __forceinline__ const R* rec_entry(const P& p, long long cbase, int n) {
   using L = RecLayout<F, R>;
   return chunk_entry<L>(p.pool, chunk_at(p.chunk_table, cbase + n / L::C, p.bounds), n,
                         p.bounds);
@@ -980,16 +980,88 @@ __global__ void __launch_bounds__(128) k_replay_outputs(OutParams<R> q) {
   }
 }
 
-// Replay adjoint with outputs at requested times: walking the record backwards, the cotangent
-// of each output in the window of step n is pulled back through its extra step from y_n and
-// added to the cotangent of y_n, next to the pullback of the step itself.
+// One step of the method's replay adjoint: lam <- the pullback of lam through the step from y
+// with size h, theta-bar accumulated (the tape is the Tsit5 and Verner 7 stage tape).
+template <class F, class R, int METHOD>
+__device__ __forceinline__ void adjoint_step(const R (&y)[F::D], R h,
+                                             const typename F::template Theta<R>& th,
+                                             R (&lam)[F::D], R (&thb)[F::M], R* tape) {
+  if constexpr (METHOD == M_TSIT5) tsit5_adjoint_step<F, R>(y, h, th, lam, thb, tape, blockDim.x);
+  else if constexpr (METHOD == M_VERN7) vern7_adjoint_step<F, R>(y, h, th, lam, thb, tape, blockDim.x);
+  else if constexpr (METHOD == M_RB23) rb23_adjoint_step<F, R>(y, h, th, lam, thb);
+  else ros_adjoint_step<F, R>(y, h, th, lam, thb);
+}
+
 template <class R>
 struct AdjOutParams {
   AdjointParams<R> ap;  // dL_dy1 may be null here
   const R* dL_dyout;    // [N][J][D]
   OutTimes<R> ot;
+  int jS;               // outputs 0 .. jS - 1 are before t1 (the rest are the final state)
+  R* G;                 // [N][jS][D]: the output cotangents pulled back to their window states
 };
 
+// Replay adjoint with outputs at requested times, first pass.  Output j < jS of trajectory k is
+// the state reached by one extra step from the recorded state y_n of the last step with
+// t_n <= tau_j (step 0 if there is none), of size tau_j - t_n.  Its cotangent mu_j therefore
+// reaches y_n as g_j, the pullback of mu_j through that extra step, and reaches theta as that
+// pullback's theta-bar term.  Neither depends on the cotangent of the steps after n, so all of
+// them are taken here, before the walk over the record: every lane takes the same jS pullbacks
+// (the times are shared by all trajectories), so a warp takes them in lockstep, where taking them
+// inside the walk would stall the whole warp on nearly every step for the one lane that meets an
+// output.  g_j goes to G; the theta-bar terms, summed, to dL_dtheta[k], where the walk starts.
+template <class F, class R, int METHOD>
+__global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_blocks)
+    k_output_pullbacks(AdjOutParams<R> q) {
+  using L = RecLayout<F, R>;
+  constexpr int D = F::D, M = F::M;
+  extern __shared__ __align__(16) unsigned char adj_smem[];
+  R* tape = reinterpret_cast<R*>(adj_smem) + threadIdx.x;
+  const AdjointParams<R>& p = q.ap;
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= p.N) return;
+  const int S = p.nsteps[k];
+  R thb[M];
+#pragma unroll
+  for (int i = 0; i < M; ++i) thb[i] = R(0);
+  if (S > 0) {
+    typename F::template Theta<R> th;
+    F::load(th, p.theta + (size_t)p.theta_stride * k);
+    const long long cbase = p.choff[k];
+    const R* lo = q.dL_dyout + (size_t)k * q.ot.J * D;
+    int n = 0;
+    for (int j = 0; j < q.jS; ++j) {
+      const R tau = q.ot.tau[j];
+      // the last step n with t_n <= tau: the times ascend, so it is at or after the previous
+      // output's step (whose t_n <= tau_{j-1} <= tau_j); step 0 when no recorded time is <= tau
+      int a = n, b = S - 1;
+      while (a < b) {
+        const int m = (a + b + 1) >> 1;
+        if (rec_entry<F, R>(p, cbase, m)[0] <= tau) a = m;
+        else b = m - 1;
+      }
+      n = a;
+      R t, h, y[D], mu[D];
+      load_entry<R, L::E>(rec_entry<F, R>(p, cbase, n), t, h, y);
+#pragma unroll
+      for (int c = 0; c < D; ++c) mu[c] = lo[(size_t)j * D + c];
+      adjoint_step<F, R, METHOD>(y, tau - t, th, mu, thb, tape);
+#pragma unroll
+      for (int c = 0; c < D; ++c) q.G[((size_t)k * q.jS + j) * D + c] = mu[c];
+    }
+  }
+  if (p.dL_dtheta)
+#pragma unroll
+    for (int i = 0; i < M; ++i) p.dL_dtheta[(size_t)k * M + i] = thb[i];
+}
+
+// Replay adjoint with outputs at requested times, second pass: the walk of k_adjoint (one
+// recorded step per active lane per pass of the loop, a lane refilled with the next trajectory,
+// longest records first, as soon as its own is done), started from dL/dy1 plus the cotangents of
+// the outputs at or after t1 and from the first pass's theta-bar, with the first pass's g_j added
+// to the cotangent of y_n at each output's step n.  The window test is the first pass's: going
+// down from step S - 1, output j belongs to the first step with t_n <= tau_j, and to step 0 if
+// none.
 template <class F, class R, int METHOD>
 __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_blocks)
     k_adjoint_outputs(AdjOutParams<R> q) {
@@ -998,69 +1070,89 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
   extern __shared__ __align__(16) unsigned char adj_smem[];
   R* tape = reinterpret_cast<R*>(adj_smem) + threadIdx.x;
   const AdjointParams<R>& p = q.ap;
-  const int J = q.ot.J;
-  int jS = 0;  // outputs before t1 come from steps; the rest are the final state
-  while (jS < J && q.ot.tau[jS] < q.ot.t1) ++jS;
-  int k = -1;
-  bool alive = true;
+  const int J = q.ot.J, jS = q.jS;
+  const bool thb_from_first = jS > 0 && p.dL_dtheta;
+  int k = -1, n = -1, first_n = -1, jcur = 0, cur_ch = 0, next_ch = -1;
+  bool alive = true, pf_pending = false;
+  long long cbase = 0;
+  R lam[D], thb[M];
   typename F::template Theta<R> th;
+#pragma unroll
+  for (int c = 0; c < D; ++c) lam[c] = R(0);
+#pragma unroll
+  for (int i = 0; i < M; ++i) thb[i] = R(0);
   for (;;) {
     const bool need = alive && k < 0;
     if (__any_sync(FULL, need)) {
       const int id = warp_take(need, p.queue);
       if (need) {
-        if (id < p.N) k = p.perm ? p.perm[id] : id;
-        else alive = false;
+        if (id < p.N) {
+          k = p.perm ? p.perm[id] : id;
+          F::load(th, p.theta + (size_t)p.theta_stride * k);
+          const R* lo = q.dL_dyout + (size_t)k * J * D;
+#pragma unroll
+          for (int c = 0; c < D; ++c) lam[c] = p.dL_dy1 ? p.dL_dy1[(size_t)k * D + c] : R(0);
+#pragma unroll
+          for (int i = 0; i < M; ++i) thb[i] = thb_from_first ? p.dL_dtheta[(size_t)k * M + i] : R(0);
+          const int S = p.nsteps[k];
+          jcur = S == 0 ? 0 : jS;
+          for (int jj = jcur; jj < J; ++jj)
+#pragma unroll
+            for (int c = 0; c < D; ++c) lam[c] += lo[(size_t)jj * D + c];
+          n = S - 1;
+          first_n = n;
+          cbase = p.choff[k];
+        } else {
+          alive = false;
+        }
       }
     }
     if (!__any_sync(FULL, k >= 0 || alive)) break;
-    if (k < 0) continue;
-    F::load(th, p.theta + (size_t)p.theta_stride * k);
-    const R* lo = q.dL_dyout + (size_t)k * J * D;
-    R lam[D], thb[M];
+    if (k >= 0) {
+      if (n >= 0) {
+        // chunk of step n, and the next chunk's lines prefetched one step after entering one
+        if (n == first_n || n % L::C == L::C - 1) {
+          cur_ch = chunk_at(p.chunk_table, cbase + n / L::C, p.bounds);
+          next_ch = (n / L::C >= 1) ? chunk_at(p.chunk_table, cbase + n / L::C - 1, p.bounds) : -1;
+#ifdef GS_CHECKED
+          if (next_ch >= p.bounds.pool_chunks) next_ch = -1;
+#endif
+          pf_pending = next_ch >= 0;
+        } else if (pf_pending) {
+          const R* pq = p.pool + (size_t)next_ch * L::C * L::E;
 #pragma unroll
-    for (int c = 0; c < D; ++c) lam[c] = p.dL_dy1 ? p.dL_dy1[(size_t)k * D + c] : R(0);
+          for (int b = 0; b < L::C * L::E * (int)sizeof(R); b += 128)
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const char*>(pq) + b));
+          pf_pending = false;
+        }
+        const R* e = chunk_entry<L>(p.pool, cur_ch, n, p.bounds);
+        R t, h, y[D];
+        load_entry<R, L::E>(e, t, h, y);
+        int jlo = jcur;
+        while (jlo > 0 && (n == 0 || q.ot.tau[jlo - 1] >= t)) --jlo;
+        // the stored pullbacks of this step's outputs, fetched while the step is pulled back
+        for (int r = jlo; r < jcur; ++r) {
+          const char* g = reinterpret_cast<const char*>(q.G + ((size_t)k * jS + r) * D);
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(g));
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(g + D * sizeof(R) - 1));
+        }
+        adjoint_step<F, R, METHOD>(y, h, th, lam, thb, tape);
+        for (int r = jlo; r < jcur; ++r)
 #pragma unroll
-    for (int i = 0; i < M; ++i) thb[i] = R(0);
-    const int S = p.nsteps[k];
-    for (int j = (S == 0 ? 0 : jS); j < J; ++j)
-#pragma unroll
-      for (int c = 0; c < D; ++c) lam[c] += lo[(size_t)j * D + c];
-    const long long cbase = p.choff[k];
-    int jcur = S == 0 ? 0 : jS;
-    for (int n = S - 1; n >= 0; --n) {
-      const R* e = chunk_entry<L>(p.pool, chunk_at(p.chunk_table, cbase + n / L::C, p.bounds), n,
-                                  p.bounds);
-      R t, h, y[D];
-      load_entry<R, L::E>(e, t, h, y);
-      int jlo = jcur;
-      while (jlo > 0 && (n == 0 || q.ot.tau[jlo - 1] >= t)) --jlo;
-      R lacc[D];
-#pragma unroll
-      for (int c = 0; c < D; ++c) lacc[c] = R(0);
-      for (int r = jcur - 1; r >= jlo - 1; --r) {   // r = jlo - 1 is the step itself
-        R lr[D];
-        const R hr = r >= jlo ? q.ot.tau[r] - t : h;
-#pragma unroll
-        for (int c = 0; c < D; ++c) lr[c] = r >= jlo ? lo[(size_t)r * D + c] : lam[c];
-        if constexpr (METHOD == M_TSIT5) tsit5_adjoint_step<F, R>(y, hr, th, lr, thb, tape, blockDim.x);
-        else if constexpr (METHOD == M_VERN7) vern7_adjoint_step<F, R>(y, hr, th, lr, thb, tape, blockDim.x);
-        else if constexpr (METHOD == M_RB23) rb23_adjoint_step<F, R>(y, hr, th, lr, thb);
-        else ros_adjoint_step<F, R>(y, hr, th, lr, thb);
-#pragma unroll
-        for (int c = 0; c < D; ++c) lacc[c] += lr[c];
+          for (int c = 0; c < D; ++c) lam[c] += q.G[((size_t)k * jS + r) * D + c];
+        jcur = jlo;
+        --n;
       }
+      if (n < 0) {
+        if (p.dL_dy0)
 #pragma unroll
-      for (int c = 0; c < D; ++c) lam[c] = lacc[c];
-      jcur = jlo;
+          for (int c = 0; c < D; ++c) p.dL_dy0[(size_t)k * D + c] = lam[c];
+        if (p.dL_dtheta)
+#pragma unroll
+          for (int i = 0; i < M; ++i) p.dL_dtheta[(size_t)k * M + i] = thb[i];
+        k = -1;
+      }
     }
-    if (p.dL_dy0)
-#pragma unroll
-      for (int c = 0; c < D; ++c) p.dL_dy0[(size_t)k * D + c] = lam[c];
-    if (p.dL_dtheta)
-#pragma unroll
-      for (int i = 0; i < M; ++i) p.dL_dtheta[(size_t)k * M + i] = thb[i];
-    k = -1;
   }
 }
 

@@ -114,3 +114,74 @@ def test_outputs_argument_checks():
         G.gs_replay_outputs(recm, U.dev(m.theta, torch.float32), U.dev(m.y0, torch.float32),
                             [0.5], torch.empty((4, 1, 4), dtype=torch.float32, device="cuda"))
     assert e.value.code == G.GS_ERR_UNSUPPORTED
+
+
+def test_outputs_gradient_windows_and_edges(orc):
+    """The gradient's corner cases: many times with repeats, so that one step's window holds
+    several outputs and some outputs fall on mesh points; a time before t0 (integrated backwards
+    from y0, so in step 0's window); one of the two gradients asked for at a time; every time at
+    or after t1 (the walk alone with the final state's cotangent); an ensemble that leaves the
+    last 128-lane block partly empty."""
+    torch = U.torch()
+    w = U.small("lorenz63", 257)
+    rec, _ = U.record(w)
+    ex = U.export_padded(w, rec)
+    rng = np.random.default_rng(11)
+    T0 = ex["T"][0, :ex["S"][0]]
+    tau = np.concatenate([[w.t0 - 0.05 * (w.t1 - w.t0)], rng.uniform(w.t0, w.t1, 40), T0[1:6],
+                          T0[2:4], [w.t1, w.t1]])
+    tau = np.sort(tau)
+    lam_out = rng.normal(size=(w.N, len(tau), w.d))
+    ry, rt = orc.replay_outputs_grad(w.field, w.method, w.theta, w.y0, ex["T"], ex["H"], ex["S"],
+                                     w.t1, tau, lam_out, nthreads=8)
+    gy, gt = _gpu_grad(w, rec, tau, lam_out, None)
+    assert U.rel_rows(gy, ry, 1e-300).max() <= 1e-8
+    assert U.rel_rows(gt, rt, 1e-300).max() <= 1e-8
+    # one gradient at a time
+    th, lo = U.dev(w.theta, torch.float64), U.dev(lam_out, torch.float64)
+    gt1 = torch.empty((w.N, w.m), dtype=torch.float64, device="cuda")
+    G.gs_replay_grad_outputs(rec, th, tau, lo, None, gt1, None)
+    gy1 = torch.empty((w.N, w.d), dtype=torch.float64, device="cuda")
+    G.gs_replay_grad_outputs(rec, th, tau, lo, None, None, gy1)
+    torch.cuda.synchronize()
+    assert U.rel_rows(gt1.cpu().numpy(), rt, 1e-300).max() <= 1e-8
+    assert U.rel_rows(gy1.cpu().numpy(), ry, 1e-300).max() <= 1e-8
+    # every time at or after t1: the gradient of the final state against the summed cotangent
+    tau2 = np.array([w.t1, w.t1 * 1.25])
+    lam2 = rng.normal(size=(w.N, 2, w.d))
+    gy2, gt2 = _gpu_grad(w, rec, tau2, lam2, None)
+    ry2, rt2 = orc.replay_grad(w.field, w.method, w.theta, w.y0, ex["H"], ex["S"], lam2.sum(1),
+                               nthreads=8)
+    assert U.rel_rows(gy2, ry2, 1e-300).max() <= 1e-8
+    assert U.rel_rows(gt2, rt2, 1e-300).max() <= 1e-8
+
+
+def test_full_size_outputs_gradient_sampled(orc):
+    """The stellar ensemble at its benchmark size (2^20 orbits) with the 8 times the benchmark
+    asks for (the last one t1): the gradient of the loss on the outputs for sampled orbits against
+    the oracle on their own recorded meshes, through the same launches as the benchmark."""
+    torch = U.torch()
+    w = W.by_name("nfw_mn")
+    rec, _ = U.record(w)
+    tau = [w.t0 + (w.t1 - w.t0) * (j + 1) / 8.0 for j in range(8)]
+    lam_out = np.random.default_rng(12).normal(size=(w.N, len(tau), w.d))
+    gy, gt = _gpu_grad(w, rec, tau, lam_out, None)
+    tot = int(rec.info().total_steps)
+    T = torch.empty(tot, dtype=torch.float64, device="cuda")
+    H = torch.empty(tot, dtype=torch.float64, device="cuda")
+    off = torch.empty(w.N + 1, dtype=torch.int64, device="cuda")
+    G.gs_record_export(rec, T, H, None, off)
+    torch.cuda.synchronize()
+    off = off.cpu().numpy()
+    rng = np.random.default_rng(13)
+    idx = np.unique(np.concatenate([[0, w.N - 1], rng.choice(w.N, size=24, replace=False)]))
+    S = (off[idx + 1] - off[idx]).astype(np.int32)
+    Ts, Hs = np.zeros((len(idx), S.max())), np.zeros((len(idx), S.max()))
+    for r_, k in enumerate(idx):
+        Ts[r_, :S[r_]] = T[off[k]:off[k + 1]].cpu().numpy()
+        Hs[r_, :S[r_]] = H[off[k]:off[k + 1]].cpu().numpy()
+    sub = W.subset(w, idx)
+    ry, rt = orc.replay_outputs_grad(sub.field, sub.method, sub.theta, sub.y0, Ts, Hs, S, w.t1,
+                                     np.array(tau), lam_out[idx], nthreads=8)
+    assert U.rel_rows(gy[idx], ry, 1e-300).max() <= 1e-8
+    assert U.rel_rows(gt[idx], rt, 1e-300).max() <= 1e-8
