@@ -1333,6 +1333,15 @@ gs_status check_out_times(const gs_record* rec, int32_t J, const double* tau) {
   return GS_OK;
 }
 
+// How many of the ascending times are before t1, compared in the record's precision as the kernels
+// compare them.
+int outputs_before_t1(const gs_record* rec, int32_t J, const double* tau) {
+  const bool f32 = rec->rsz == sizeof(float);
+  int jS = 0;
+  while (jS < J && (f32 ? (float)tau[jS] < (float)rec->t1 : tau[jS] < rec->t1)) ++jS;
+  return jS;
+}
+
 template <class R>
 void fill_times(gs::OutTimes<R>& ot, const gs_record* rec, int32_t J, const double* tau) {
   ot.J = J;
@@ -1370,8 +1379,6 @@ gs_status gs_replay_outputs(const gs_record* rec, const void* theta, const void*
   st = check_device({{theta, "theta"}, {y0, "y0"}, {y_out, "y_out"}});
   if (st != GS_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int* queue = nullptr;
-  GS_CUDA(take_counter(s, &queue));
   int* rq = nullptr;
   GS_CUDA(take_counter(s, &rq));
   st = refresh_states(const_cast<gs_record*>(rec), theta, rq, false, device_sms(), s);
@@ -1381,12 +1388,12 @@ gs_status gs_replay_outputs(const gs_record* rec, const void* theta, const void*
       return fail(GS_ERR_UNSUPPORTED, "not built for the MLP field");
     } else {
       gs::OutParams<R> q{};
-      fill_replay_params<R>(q.rp, rec, theta, F::M, queue);
+      fill_replay_params<R>(q.rp, rec, theta, F::M, nullptr);
       q.rp.y0 = static_cast<const R*>(y0);
       q.y_out = static_cast<R*>(y_out);
       fill_times<R>(q.ot, rec, J, tau);
-      auto kern = gs::k_replay_outputs<F, R, METHOD>;
-      kern<<<persistent_grid(kern, 0, rec->N), BLOCK, 0, s>>>(q);
+      q.jS = outputs_before_t1(rec, J, tau);
+      gs::k_replay_outputs<F, R, METHOD><<<(unsigned)((rec->N + BLOCK - 1) / BLOCK), BLOCK, 0, s>>>(q);
       GS_CUDA(cudaGetLastError());
       return GS_OK;
     }
@@ -1432,10 +1439,7 @@ gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_
       r->part_bytes = needp;
     }
   }
-  // outputs before t1 (compared in the record's precision, as the kernels compare them)
-  const bool f32 = rec->rsz == sizeof(float);
-  int jS = 0;
-  while (jS < J && (f32 ? (float)tau[jS] < (float)rec->t1 : tau[jS] < rec->t1)) ++jS;
+  const int jS = outputs_before_t1(rec, J, tau);
   const size_t need_g = (size_t)N * jS * rec->sys.d * rec->rsz;
   if (r->out_bytes < need_g) {
     free_ptr(r->out_scratch, s);

@@ -915,9 +915,10 @@ struct OutTimes {
 
 template <class R>
 struct OutParams {
-  ReplayParams<R> rp;   // theta, y0, record, queue, perm (y1 unused)
+  ReplayParams<R> rp;   // theta, y0, record (y1, queue and perm unused)
   R* y_out;             // [N][J][D]
   OutTimes<R> ot;
+  int jS;               // outputs 0 .. jS - 1 are before t1 (the rest are the final state)
 };
 
 
@@ -928,55 +929,63 @@ __device__ __forceinline__ const R* rec_entry(const P& p, long long cbase, int n
                         p.bounds);
 }
 
+// The recorded step output time tau is taken from: the last step n in [from, S) with
+// t_n <= tau, or `from` when there is none (from = 0: a time before t0 is taken from step 0).
+// Binary search over the recorded times, which ascend with n; the caller passes, as `from`, the
+// step of an earlier (not later) time, whose t_n <= tau.
+template <class F, class R, class P>
+__device__ __forceinline__ int output_step(const P& p, long long cbase, int from, int S, R tau) {
+  int a = from, b = S - 1;
+  while (a < b) {
+    const int m = (a + b + 1) >> 1;
+    if (rec_entry<F, R>(p, cbase, m)[0] <= tau) a = m;
+    else b = m - 1;
+  }
+  return a;
+}
+
+// States at requested times.  Output j of trajectory k with tau_j < t1 is one extra step, of size
+// tau_j - t_n, from the recorded state y_n of its step n (output_step); the outputs at or after t1
+// are the final state, one step of size h_{S-1} from y_{S-1}; with no recorded step every output
+// is y0.  The record keeps every y_n, so no walk over it is needed: each output reads one entry
+// after its search.  Every lane takes the same jS extra steps (the times are shared), so a warp
+// takes them in lockstep.  One lane per trajectory.
 template <class F, class R, int METHOD>
 __global__ void __launch_bounds__(128) k_replay_outputs(OutParams<R> q) {
   using L = RecLayout<F, R>;
   constexpr int D = F::D;
   const ReplayParams<R>& p = q.rp;
-  const int J = q.ot.J;
-  int k = -1;
-  bool alive = true;
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= p.N) return;
+  const int J = q.ot.J, jS = q.jS;
+  const int S = p.nsteps[k];
+  R* out = q.y_out + (size_t)k * J * D;
+  if (S == 0) {
+    for (int j = 0; j < J; ++j)
+#pragma unroll
+      for (int c = 0; c < D; ++c) out[(size_t)j * D + c] = p.y0[(size_t)k * D + c];
+    return;
+  }
   typename F::template Theta<R> th;
-  for (;;) {
-    const bool need = alive && k < 0;
-    if (__any_sync(FULL, need)) {
-      const int id = warp_take(need, p.queue);
-      if (need) {
-        if (id < p.N) k = p.perm ? p.perm[id] : id;
-        else alive = false;
-      }
-    }
-    if (!__any_sync(FULL, k >= 0 || alive)) break;
-    if (k < 0) continue;
-    F::load(th, p.theta + (size_t)p.theta_stride * k);
-    const int S = p.nsteps[k];
-    const long long cbase = p.choff[k];
-    R* out = q.y_out + (size_t)k * J * D;
-    int j = 0;
-    R y[D], t = R(0), h = R(0);
+  F::load(th, p.theta + (size_t)p.theta_stride * k);
+  const long long cbase = p.choff[k];
+  int n = 0;
+  for (int j = 0; j < jS; ++j) {
+    const R tau = q.ot.tau[j];
+    n = output_step<F, R>(p, cbase, n, S, tau);
+    R t, h, y[D], yo[D];
+    load_entry<R, L::E>(rec_entry<F, R>(p, cbase, n), t, h, y);
+    replay_step<F, R, METHOD>(y, tau - t, th, yo);
 #pragma unroll
-    for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
-    for (int n = 0; n < S && j < J; ++n) {
-      load_entry<R, L::E>(rec_entry<F, R>(p, cbase, n), t, h, y);
-      const R tnext = (n + 1 < S) ? rec_entry<F, R>(p, cbase, n + 1)[0] : q.ot.t1;
-      while (j < J && q.ot.tau[j] < tnext) {
-        R yo[D];
-        replay_step<F, R, METHOD>(y, q.ot.tau[j] - t, th, yo);
+    for (int c = 0; c < D; ++c) out[(size_t)j * D + c] = yo[c];
+  }
+  if (jS < J) {
+    R t, h, y[D], yS[D];
+    load_entry<R, L::E>(rec_entry<F, R>(p, cbase, S - 1), t, h, y);
+    replay_step<F, R, METHOD>(y, h, th, yS);
+    for (int j = jS; j < J; ++j)
 #pragma unroll
-        for (int c = 0; c < D; ++c) out[(size_t)j * D + c] = yo[c];
-        ++j;
-      }
-      if (j < J && n == S - 1) {  // the remaining times are at or after t1: the final state
-        R yS[D];
-        replay_step<F, R, METHOD>(y, h, th, yS);
-#pragma unroll
-        for (int c = 0; c < D; ++c) y[c] = yS[c];
-      }
-    }
-    for (; j < J; ++j)
-#pragma unroll
-      for (int c = 0; c < D; ++c) out[(size_t)j * D + c] = y[c];
-    k = -1;
+      for (int c = 0; c < D; ++c) out[(size_t)j * D + c] = yS[c];
   }
 }
 
@@ -1032,15 +1041,7 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
     int n = 0;
     for (int j = 0; j < q.jS; ++j) {
       const R tau = q.ot.tau[j];
-      // the last step n with t_n <= tau: the times ascend, so it is at or after the previous
-      // output's step (whose t_n <= tau_{j-1} <= tau_j); step 0 when no recorded time is <= tau
-      int a = n, b = S - 1;
-      while (a < b) {
-        const int m = (a + b + 1) >> 1;
-        if (rec_entry<F, R>(p, cbase, m)[0] <= tau) a = m;
-        else b = m - 1;
-      }
-      n = a;
+      n = output_step<F, R>(p, cbase, n, S, tau);
       R t, h, y[D], mu[D];
       load_entry<R, L::E>(rec_entry<F, R>(p, cbase, n), t, h, y);
 #pragma unroll
