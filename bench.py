@@ -785,14 +785,13 @@ def main():
     breakdown["forward_only_index_order"] = timeit(
         lambda: G.gs_solve_forward(sys_, N, th, y0, w.t0, w.t1, w.rtol, w.atol, y1, S, rj, stt,
                                    opts=G.options(start_order=ident)))
-    if w.field != "mlp":
-        # outputs at 8 requested times ([GS] §3.4) and the gradient of a loss on them
-        tau = [w.t0 + (w.t1 - w.t0) * (j + 1) / 8.0 for j in range(8)]
-        yout = torch.empty((N, len(tau), d), dtype=dt, device=dev)
-        lam_out = (mask.expand(N, len(tau), d) * 0.125).contiguous()
-        breakdown["outputs_8_times"] = timeit(lambda: G.gs_replay_outputs(rec, th, y0, tau, yout))
-        breakdown["replay_grad_outputs_8_times"] = timeit(
-            lambda: G.gs_replay_grad_outputs(rec, th, tau, lam_out, None, gt, gy))
+    # outputs at 8 requested times ([GS] §3.4) and the gradient of a loss on them
+    tau = [w.t0 + (w.t1 - w.t0) * (j + 1) / 8.0 for j in range(8)]
+    yout = torch.empty((N, len(tau), d), dtype=dt, device=dev)
+    lam_out = (mask.expand(N, len(tau), d) * 0.125).contiguous()
+    breakdown["outputs_8_times"] = timeit(lambda: G.gs_replay_outputs(rec, th, y0, tau, yout))
+    breakdown["replay_grad_outputs_8_times"] = timeit(
+        lambda: G.gs_replay_grad_outputs(rec, th, tau, lam_out, None, gt, gy))
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the region.
     # Two stream pipelines with their own buffers and records, steps alternating between them, so

@@ -1328,8 +1328,6 @@ gs_status check_out_times(const gs_record* rec, int32_t J, const double* tau) {
     if (j > 0 && tau[j] < tau[j - 1])
       return fail(GS_ERR_INVALID_ARG, "tau must be ascending (tau[%d] < tau[%d])", j, j - 1);
   }
-  if (rec->sys.field == GS_MLP_4_32_32_4)
-    return fail(GS_ERR_UNSUPPORTED, "outputs at requested times are not built for the MLP field");
   return GS_OK;
 }
 
@@ -1364,6 +1362,68 @@ void fill_replay_params(gs::ReplayParams<R>& p, const gs_record* rec, const void
   p.bounds = bounds_of(rec);
 }
 
+// Gradient of a loss on the outputs at requested times, MLP field: the output pullbacks, then the
+// walk that adds them, both one warp per trajectory on the same grid (warp gw carries its weight-
+// cotangent partial from the first pass into the second), then a fixed-order sum over warps.
+static gs_status replay_grad_outputs_mlp(const gs_record* rec, const void* theta, int32_t J,
+                                         const double* tau, const void* dL_dyout,
+                                         const void* dL_dy1, void* dL_dtheta, void* dL_dy0,
+                                         cudaStream_t s) {
+  gs_record* r = const_cast<gs_record*>(rec);
+  const int jS = outputs_before_t1(rec, J, tau);
+  const size_t need_g = (size_t)rec->N * jS * rec->sys.d * rec->rsz;
+  if (r->out_bytes < need_g) {
+    free_ptr(r->out_scratch, s);
+    r->out_scratch = nullptr;
+    r->out_bytes = 0;
+    GS_CUDA(dalloc(&r->out_scratch, need_g, s));
+    r->out_bytes = need_g;
+  }
+  auto run = [&](auto zero) -> gs_status {
+    using R = decltype(zero);
+    auto walk = gs::k_adjoint_outputs_mlp<R>;
+    const int grid = persistent_grid(walk, 0, rec->N * 32);
+    const int nwarps = grid * (BLOCK / 32);
+    R* partials = nullptr;
+    if (dL_dtheta) {
+      const size_t need = (size_t)nwarps * gs::MLP_M * sizeof(R);
+      if (r->part_bytes < need) {
+        free_ptr(r->red_partials, s);
+        r->red_partials = nullptr;
+        r->part_bytes = 0;
+        GS_CUDA(dalloc(&r->red_partials, need, s));
+        r->part_bytes = need;
+      }
+      partials = static_cast<R*>(r->red_partials);
+    }
+    gs::MlpOutAdjParams<R> q{};
+    gs::MlpAdjParams<R>& p = q.ap;
+    p.N = (int)rec->N;
+    p.theta = static_cast<const R*>(theta);
+    p.dL_dy1 = static_cast<const R*>(dL_dy1);
+    p.dL_dy0 = static_cast<R*>(dL_dy0);
+    p.partials = partials;
+    p.nsteps = rec->nsteps;
+    p.choff = rec->choff;
+    p.chunk_table = rec->chunk_table;
+    p.pool = static_cast<const R*>(rec->pool);
+    p.perm = rec->perm;
+    p.bounds = bounds_of(rec);
+    q.dL_dyout = static_cast<const R*>(dL_dyout);
+    fill_times<R>(q.ot, rec, J, tau);
+    q.jS = jS;
+    q.G = static_cast<R*>(r->out_scratch);
+    if (jS > 0) gs::k_output_pullbacks_mlp<R><<<grid, BLOCK, 0, s>>>(q);
+    walk<<<grid, BLOCK, 0, s>>>(q);
+    if (partials)
+      gs::k_reduce_partials<R><<<(gs::MLP_M + 255) / 256, 256, 0, s>>>(partials, nwarps, gs::MLP_M,
+                                                                    static_cast<R*>(dL_dtheta));
+    GS_CUDA(cudaGetLastError());
+    return GS_OK;
+  };
+  return rec->sys.dtype == GS_F64 ? run(0.0) : run(0.0f);
+}
+
 }  // namespace
 
 extern "C" {
@@ -1384,19 +1444,20 @@ gs_status gs_replay_outputs(const gs_record* rec, const void* theta, const void*
   st = refresh_states(const_cast<gs_record*>(rec), theta, rq, false, device_sms(), s);
   if (st != GS_OK) return st;
   return dispatch(rec->sys, [&]<class F, class R, int METHOD>() {
+    gs::OutParams<R> q{};
+    fill_replay_params<R>(q.rp, rec, theta, F::M, nullptr);
+    q.rp.y0 = static_cast<const R*>(y0);
+    q.y_out = static_cast<R*>(y_out);
+    fill_times<R>(q.ot, rec, J, tau);
+    q.jS = outputs_before_t1(rec, J, tau);
     if constexpr (std::is_same_v<F, gs::FMlpWarp>) {
-      return fail(GS_ERR_UNSUPPORTED, "not built for the MLP field");
+      auto kern = gs::k_replay_outputs_mlp<R>;  // one warp per trajectory
+      kern<<<persistent_grid(kern, 0, rec->N * 32), BLOCK, 0, s>>>(q);
     } else {
-      gs::OutParams<R> q{};
-      fill_replay_params<R>(q.rp, rec, theta, F::M, nullptr);
-      q.rp.y0 = static_cast<const R*>(y0);
-      q.y_out = static_cast<R*>(y_out);
-      fill_times<R>(q.ot, rec, J, tau);
-      q.jS = outputs_before_t1(rec, J, tau);
       gs::k_replay_outputs<F, R, METHOD><<<(unsigned)((rec->N + BLOCK - 1) / BLOCK), BLOCK, 0, s>>>(q);
-      GS_CUDA(cudaGetLastError());
-      return GS_OK;
     }
+    GS_CUDA(cudaGetLastError());
+    return GS_OK;
   });
 }
 
@@ -1422,6 +1483,8 @@ gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_
   int* rq = nullptr;
   GS_CUDA(take_counter(s, &rq));
   if ((st = refresh_states(r, theta, rq, false, device_sms(), s)) != GS_OK) return st;
+  if (rec->sys.field == GS_MLP_4_32_32_4)
+    return replay_grad_outputs_mlp(rec, theta, J, tau, dL_dyout, dL_dy1, dL_dtheta, dL_dy0, s);
   if (shared) {
     const size_t need = (size_t)N * M * rec->rsz, needp = (size_t)nred * M * rec->rsz;
     if (r->red_bytes < need) {
@@ -1452,7 +1515,7 @@ gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_
   GS_CUDA(take_counter(s, &queue));
   return dispatch(rec->sys, [&]<class F, class R, int METHOD>() {
     if constexpr (std::is_same_v<F, gs::FMlpWarp>) {
-      return fail(GS_ERR_UNSUPPORTED, "not built for the MLP field");
+      return fail(GS_ERR_UNSUPPORTED, "the MLP field takes replay_grad_outputs_mlp");
     } else {
       gs::AdjOutParams<R> q{};
       gs::AdjointParams<R>& p = q.ap;

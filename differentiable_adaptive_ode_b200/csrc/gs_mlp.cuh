@@ -126,6 +126,21 @@ struct MlpBar {
     b1 = R(0);
     b2 = R(0);
   }
+  // read back a partial that store wrote (b3b into every lane, as it accumulates there)
+  __device__ void load(const R* in) {
+    const int i = threadIdx.x & 31;
+#pragma unroll
+    for (int c = 0; c < MLP_D; ++c) w1[c] = in[MLP_OW1 + i * MLP_D + c];
+    b1 = in[MLP_OB1 + i];
+#pragma unroll
+    for (int j = 0; j < MLP_H; ++j) w2[j] = in[MLP_OW2 + i * MLP_H + j];
+    b2 = in[MLP_OB2 + i];
+#pragma unroll
+    for (int o = 0; o < MLP_D; ++o) {
+      w3[o] = in[MLP_OW3 + o * MLP_H + i];
+      b3[o] = in[MLP_OB3 + o];
+    }
+  }
   // write this warp's partial (M values) to out
   __device__ void store(R* out) const {
     const int i = threadIdx.x & 31;
@@ -350,6 +365,42 @@ __global__ void __launch_bounds__(128) k_solve_mlp(SolveParams<R> p) {
   }
 }
 
+// One Tsit5 step of the replay map for the MLP field: every lane of the warp, y replicated.
+template <class R>
+__device__ __forceinline__ void mlp_replay_step(const MlpLane<R>& W, const R (&y)[MLP_D], R h,
+                                                R (&ynew)[MLP_D]) {
+  constexpr int D = MLP_D;
+  R kk[6][D], Y[D];
+  FMlpWarp::f<R>(y, W, kk[0]);
+#pragma unroll
+  for (int i = 1; i < 6; ++i) {
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+      R s = ta<R>(i, 0) * kk[0][c];
+#pragma unroll
+      for (int j = 1; j < i; ++j) s += ta<R>(i, j) * kk[j][c];
+      Y[c] = y[c] + h * s;
+    }
+    FMlpWarp::f<R>(Y, W, kk[i]);
+  }
+#pragma unroll
+  for (int c = 0; c < D; ++c) {
+    R s = tb<R>(0) * kk[0][c];
+#pragma unroll
+    for (int j = 1; j < 6; ++j) s += tb<R>(j) * kk[j][c];
+    ynew[c] = y[c] + h * s;
+  }
+}
+
+// Lane c (< D) writes component c of a vector that every lane holds.
+template <class R>
+__device__ __forceinline__ void mlp_lane_store(R* out, const R (&v)[MLP_D]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int c = 0; c < MLP_D; ++c)
+    if (lane == c) out[c] = v[c];
+}
+
 // Forward replay over the recorded mesh (rewrites the stored y_n), one warp per trajectory.
 template <class R>
 __global__ void __launch_bounds__(128) k_replay_forward_mlp(ReplayParams<R> p) {
@@ -384,30 +435,8 @@ __global__ void __launch_bounds__(128) k_replay_forward_mlp(ReplayParams<R> p) {
       const R h = e[1];
       __syncwarp();
       if (lane < D) e[2 + lane] = y[lane];
-      R k1[D], ynew[D];
-      FMlpWarp::f<R>(y, W, k1);
-      R Y[D];
-      R kk[6][D];
-#pragma unroll
-      for (int c = 0; c < D; ++c) kk[0][c] = k1[c];
-#pragma unroll
-      for (int i = 1; i < 6; ++i) {
-#pragma unroll
-        for (int c = 0; c < D; ++c) {
-          R s = ta<R>(i, 0) * kk[0][c];
-#pragma unroll
-          for (int j = 1; j < i; ++j) s += ta<R>(i, j) * kk[j][c];
-          Y[c] = y[c] + h * s;
-        }
-        FMlpWarp::f<R>(Y, W, kk[i]);
-      }
-#pragma unroll
-      for (int c = 0; c < D; ++c) {
-        R s = tb<R>(0) * kk[0][c];
-#pragma unroll
-        for (int j = 1; j < 6; ++j) s += tb<R>(j) * kk[j][c];
-        ynew[c] = y[c] + h * s;
-      }
+      R ynew[D];
+      mlp_replay_step<R>(W, y, h, ynew);
 #pragma unroll
       for (int c = 0; c < D; ++c) y[c] = ynew[c];
     }
@@ -461,6 +490,151 @@ __global__ void __launch_bounds__(128) k_adjoint_mlp(MlpAdjParams<R> p) {
       mlp_adjoint_step<R>(W, y, h, lam, bar);
     }
     if (p.dL_dy0 && lane < D) p.dL_dy0[(size_t)k * D + lane] = lam[lane];
+  }
+  if (p.partials) bar.store(p.partials + (size_t)gw * MLP_M);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Outputs at requested times and their gradient ("gradsolve: fast exact gradients for ODE
+// ensembles on GPUs" §3.4: one extra solver step from the preceding mesh point exactly to each
+// requested time), one warp per trajectory.  The rule is the other fields' (k_replay_outputs,
+// k_output_pullbacks, k_adjoint_outputs): output j < jS is one step of size tau_j - t_n from the
+// recorded y_n of its step n (output_step), the rest are the final state, and y0 when nothing is
+// recorded.  Warp w takes trajectories w, w + nwarps, ...; every lane takes the same search and
+// steps, so the warp stays converged for the field's shuffles.
+// ------------------------------------------------------------------------------------------------
+template <class R>
+__global__ void __launch_bounds__(128) k_replay_outputs_mlp(OutParams<R> q) {
+  constexpr int D = MLP_D;
+  __shared__ R slots[4][32];
+  const ReplayParams<R>& p = q.rp;
+  const int warp = threadIdx.x >> 5;
+  const int J = q.ot.J, jS = q.jS;
+  MlpLane<R> W;
+  W.load(p.theta, slots[warp]);
+  for (int k = blockIdx.x * 4 + warp; k < p.N; k += gridDim.x * 4) {
+    const int S = p.nsteps[k];
+    R* out = q.y_out + (size_t)k * J * D;
+    if (S == 0) {
+      R y[D];
+#pragma unroll
+      for (int c = 0; c < D; ++c) y[c] = p.y0[(size_t)k * D + c];
+      for (int j = 0; j < J; ++j) mlp_lane_store<R>(out + (size_t)j * D, y);
+      continue;
+    }
+    const long long cbase = p.choff[k];
+    int n = 0;
+    for (int j = 0; j < jS; ++j) {
+      const R tau = q.ot.tau[j];
+      n = output_step<FMlpWarp, R>(p, cbase, n, S, tau);
+      const R* e = rec_entry<FMlpWarp, R>(p, cbase, n);
+      R y[D], yo[D];
+#pragma unroll
+      for (int c = 0; c < D; ++c) y[c] = e[2 + c];
+      mlp_replay_step<R>(W, y, tau - e[0], yo);
+      mlp_lane_store<R>(out + (size_t)j * D, yo);
+    }
+    if (jS < J) {
+      const R* e = rec_entry<FMlpWarp, R>(p, cbase, S - 1);
+      R y[D], yS[D];
+#pragma unroll
+      for (int c = 0; c < D; ++c) y[c] = e[2 + c];
+      mlp_replay_step<R>(W, y, e[1], yS);
+      for (int j = jS; j < J; ++j) mlp_lane_store<R>(out + (size_t)j * D, yS);
+    }
+  }
+}
+
+template <class R>
+struct MlpOutAdjParams {
+  MlpAdjParams<R> ap;   // dL_dy1 may be null here
+  const R* dL_dyout;    // [N][J][D]
+  OutTimes<R> ot;
+  int jS;               // outputs 0 .. jS - 1 are before t1
+  R* G;                 // [N][jS][D]: the output cotangents pulled back to their window states
+};
+
+// First pass: each output's cotangent pulled back through its extra step (to G) and that
+// pullback's weight cotangent (into the warp's partial, which the second pass continues).
+template <class R>
+__global__ void __launch_bounds__(128) k_output_pullbacks_mlp(MlpOutAdjParams<R> q) {
+  constexpr int D = MLP_D;
+  __shared__ R slots[4][32];
+  const MlpAdjParams<R>& p = q.ap;
+  const int warp = threadIdx.x >> 5;
+  const int gw = blockIdx.x * 4 + warp;
+  const int nwarps = gridDim.x * 4;
+  MlpLane<R> W;
+  W.load(p.theta, slots[warp]);
+  MlpBar<R> bar;
+  bar.zero();
+  for (int k = gw; k < p.N; k += nwarps) {
+    const int S = p.nsteps[k];
+    if (S == 0) continue;
+    const long long cbase = p.choff[k];
+    const R* lo = q.dL_dyout + (size_t)k * q.ot.J * D;
+    int n = 0;
+    for (int j = 0; j < q.jS; ++j) {
+      const R tau = q.ot.tau[j];
+      n = output_step<FMlpWarp, R>(p, cbase, n, S, tau);
+      const R* e = rec_entry<FMlpWarp, R>(p, cbase, n);
+      R y[D], mu[D];
+#pragma unroll
+      for (int c = 0; c < D; ++c) {
+        y[c] = e[2 + c];
+        mu[c] = lo[(size_t)j * D + c];
+      }
+      mlp_adjoint_step<R>(W, y, tau - e[0], mu, bar);
+      mlp_lane_store<R>(q.G + ((size_t)k * q.jS + j) * D, mu);
+    }
+  }
+  if (p.partials) bar.store(p.partials + (size_t)gw * MLP_M);
+}
+
+// Second pass: k_adjoint_mlp's walk from dL/dy1 plus the cotangents of the outputs at or after t1,
+// adding at each output's step its pulled-back cotangent from the first pass (same grid, so warp
+// gw continues its own partial).
+template <class R>
+__global__ void __launch_bounds__(128) k_adjoint_outputs_mlp(MlpOutAdjParams<R> q) {
+  constexpr int D = MLP_D;
+  __shared__ R slots[4][32];
+  const MlpAdjParams<R>& p = q.ap;
+  const int warp = threadIdx.x >> 5;
+  const int gw = blockIdx.x * 4 + warp;
+  const int nwarps = gridDim.x * 4;
+  const int J = q.ot.J, jS = q.jS;
+  MlpLane<R> W;
+  W.load(p.theta, slots[warp]);
+  MlpBar<R> bar;
+  if (jS > 0 && p.partials) bar.load(p.partials + (size_t)gw * MLP_M);
+  else bar.zero();
+  for (int id = gw; id < p.N; id += nwarps) {
+    const int k = p.perm ? p.perm[id] : id;
+    const int S = p.nsteps[k];
+    const R* lo = q.dL_dyout + (size_t)k * J * D;
+    R lam[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) lam[c] = p.dL_dy1 ? p.dL_dy1[(size_t)k * D + c] : R(0);
+    int jcur = S == 0 ? 0 : jS;
+    for (int jj = jcur; jj < J; ++jj)
+#pragma unroll
+      for (int c = 0; c < D; ++c) lam[c] += lo[(size_t)jj * D + c];
+    const long long cbase = p.choff[k];
+    for (int n = S - 1; n >= 0; --n) {
+      const R* e = rec_entry<FMlpWarp, R>(p, cbase, n);
+      const R t = e[0], h = e[1];
+      R y[D];
+#pragma unroll
+      for (int c = 0; c < D; ++c) y[c] = e[2 + c];
+      mlp_adjoint_step<R>(W, y, h, lam, bar);
+      int jlo = jcur;
+      while (jlo > 0 && (n == 0 || q.ot.tau[jlo - 1] >= t)) --jlo;
+      for (int r = jlo; r < jcur; ++r)
+#pragma unroll
+        for (int c = 0; c < D; ++c) lam[c] += q.G[((size_t)k * jS + r) * D + c];
+      jcur = jlo;
+    }
+    if (p.dL_dy0) mlp_lane_store<R>(p.dL_dy0 + (size_t)k * D, lam);
   }
   if (p.partials) bar.store(p.partials + (size_t)gw * MLP_M);
 }

@@ -209,8 +209,8 @@ gs_status gs_replay_forward(gs_record* rec, const void* theta, const void* y0, v
  * final state for tau_j >= t1 (times before t0 are integrated backwards from y0).  Uses the
  * record's stored states, replayed first when `theta` is not the theta they were made at (as
  * gs_replay_grad); y0 [N][d] (device) is the initial state, read for trajectories with no
- * recorded step.  y_out [N][J][d] (device).  Not built for
- * GS_MLP_4_32_32_4 (GS_ERR_UNSUPPORTED).  Asynchronous. */
+ * recorded step.  y_out [N][J][d] (device).  Every field, the MLP field included.
+ * Asynchronous. */
 #define GS_MAX_OUTPUT_TIMES 256
 gs_status gs_replay_outputs(const gs_record* rec, const void* theta, const void* y0, int32_t J,
                             const double* tau, void* y_out, void* stream);

@@ -30,15 +30,17 @@ def main():
         out[name + ":grad"] = float(np.abs(gy).sum() + np.abs(gt).sum())
         ex = U.export_padded(w, rec)
         out[name + ":export"] = float(np.abs(ex["H"]).sum() + np.abs(ex["Y"]).sum())
+        tau = [w.t0 + (w.t1 - w.t0) * f for f in (0.25, 0.5, 0.9)]
+        yo = torch.empty((w.N, 3, w.d), dtype=dt, device="cuda")
+        G.gs_replay_outputs(rec, U.dev(w.theta, dt), U.dev(w.y0, dt), tau, yo)
+        gy2 = torch.empty((w.N, w.d), dtype=dt, device="cuda")
+        gt2 = torch.empty((w.m,) if w.theta_shared else (w.N, w.m), dtype=dt, device="cuda")
+        G.gs_replay_grad_outputs(rec, U.dev(w.theta, dt), tau,
+                                 U.dev(np.ones((w.N, 3, w.d)), dt), None, gt2, gy2)
+        torch.cuda.synchronize()
+        out[name + ":outputs"] = float(yo.abs().sum().item() + gy2.abs().sum().item() +
+                                       gt2.abs().sum().item())
         if name != "mlp":
-            tau = [w.t0 + (w.t1 - w.t0) * f for f in (0.25, 0.5, 0.9)]
-            yo = torch.empty((w.N, 3, w.d), dtype=dt, device="cuda")
-            G.gs_replay_outputs(rec, U.dev(w.theta, dt), U.dev(w.y0, dt), tau, yo)
-            gy2 = torch.empty((w.N, w.d), dtype=dt, device="cuda")
-            G.gs_replay_grad_outputs(rec, U.dev(w.theta, dt), tau,
-                                     U.dev(np.ones((w.N, 3, w.d)), dt), None, None, gy2)
-            torch.cuda.synchronize()
-            out[name + ":outputs"] = float(yo.abs().sum().item() + gy2.abs().sum().item())
             # import the exported arrays and differentiate again
             rec2 = U.import_record(w, ex["S"], ex["T"], ex["H"], ex["Y"])
             gy3, _ = U.replay_grad(w, rec2, lam)

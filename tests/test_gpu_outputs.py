@@ -108,12 +108,60 @@ def test_outputs_argument_checks():
     with pytest.raises(G.GradsolveError) as e:
         G.gs_replay_outputs(rec, th, U.dev(w.y0, torch.float64), [], out)
     assert e.value.code == G.GS_ERR_INVALID_ARG
-    m = W.mlp(N=4)
-    recm, _ = U.record(m)
-    with pytest.raises(G.GradsolveError) as e:
-        G.gs_replay_outputs(recm, U.dev(m.theta, torch.float32), U.dev(m.y0, torch.float32),
-                            [0.5], torch.empty((4, 1, 4), dtype=torch.float32, device="cuda"))
-    assert e.value.code == G.GS_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("dtype", [np.float64, np.float32])
+def test_mlp_outputs_and_gradient(orc, dtype):
+    """The neural field (weights shared by the ensemble, one warp per trajectory): outputs at
+    requested times and the gradient of a loss on them against the oracle on the GPU's own mesh;
+    fp32 against the fp64 oracle on the fp32 mesh with the fp32 gradient bar of the replay
+    gradient's test."""
+    w = W.mlp(N=40)
+    w.theta = w.theta.copy()
+    w.theta[128:160] = np.linspace(-0.2, 0.2, 32)       # non-zero biases exercise every block
+    w.theta[1184:1216] = np.linspace(0.1, -0.1, 32)
+    w.theta[1344:1348] = [0.05, -0.05, 0.1, 0.0]
+    w.dtype = dtype
+    if dtype == np.float64:
+        w.rtol, w.atol = 1e-8, 1e-10
+    rec, out = U.record(w)
+    ex = U.export_padded(w, rec)
+    tau = _times(w, ex)
+    T, H = ex["T"].astype(np.float64), ex["H"].astype(np.float64)
+    got = _gpu_outputs(w, rec, tau)
+    ref = orc.replay_outputs("mlp", "tsit5", w.theta, w.y0.astype(dtype).astype(np.float64), T, H,
+                             ex["S"], w.t1, tau, theta_shared=True, nthreads=8)
+    err = U.rel_rows(got.reshape(w.N, -1), ref.reshape(w.N, -1), w.atol)
+    if dtype == np.float64:
+        assert err.max() <= 1e-9, err.max()
+        assert U.rel_rows(got[:, -1], out["y1"], w.atol).max() <= 1e-12
+    else:
+        assert np.quantile(err, 0.99) <= 1e-4 and err.max() <= 1e-3, err.max()
+    rng = np.random.default_rng(8)
+    lam_out = rng.normal(size=(w.N, len(tau), w.d))
+    lam1 = rng.normal(size=(w.N, w.d))
+    gy, gt = _gpu_grad(w, rec, tau, lam_out, lam1)
+    ry, rt = orc.replay_outputs_grad("mlp", "tsit5", w.theta, w.y0, T, H, ex["S"], w.t1, tau,
+                                     lam_out, theta_shared=True, nthreads=8)
+    ry1, rt1 = orc.replay_grad("mlp", "tsit5", w.theta, w.y0, H, ex["S"], lam1, theta_shared=True,
+                               nthreads=8)
+    tol = 1e-8 if dtype == np.float64 else 1e-3
+    rs = (rt + rt1).sum(0)
+    assert gt.shape == (1348,)
+    assert np.max(np.abs(gt - rs)) <= tol * np.max(np.abs(rs)), np.max(np.abs(gt - rs))
+    assert np.quantile(U.rel_rows(gy, ry + ry1, 1e-300), 0.99) <= tol
+    # the ensemble sum is reproducible bit for bit; every time at or after t1 (no first pass)
+    gy2, gt2 = _gpu_grad(w, rec, tau, lam_out, lam1)
+    assert np.array_equal(gt, gt2) and np.array_equal(gy, gy2)
+    tau2 = np.array([w.t1, w.t1 * 1.25])
+    lam2 = rng.normal(size=(w.N, 2, w.d))
+    gy3, gt3 = _gpu_grad(w, rec, tau2, lam2, None)
+    gy4, gt4 = U.replay_grad(w, rec, lam2.sum(1))
+    # (the two kernels may run different grids, so the warp partials are summed in another
+    # grouping; in fp32 the summed cotangent is also rounded once here and twice there)
+    tight = 1e-12 if dtype == np.float64 else 1e-5
+    assert np.max(np.abs(gt3 - gt4)) <= tight * np.max(np.abs(gt4))
+    assert np.max(np.abs(gy3 - gy4)) <= tight * np.max(np.abs(gy4))
 
 
 def test_outputs_gradient_windows_and_edges(orc):
