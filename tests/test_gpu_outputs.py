@@ -206,12 +206,13 @@ def test_outputs_gradient_windows_and_edges(orc):
 
 def test_full_size_outputs_gradient_sampled(orc):
     """The stellar ensemble at its benchmark size (2^20 orbits) with the 8 times the benchmark
-    asks for (the last one t1): the gradient of the loss on the outputs for sampled orbits against
-    the oracle on their own recorded meshes, through the same launches as the benchmark."""
+    asks for (the last one t1): the outputs and the gradient of a loss on them for sampled orbits
+    against the oracle on their own recorded meshes, through the same launches as the benchmark."""
     torch = U.torch()
     w = W.by_name("nfw_mn")
     rec, _ = U.record(w)
     tau = [w.t0 + (w.t1 - w.t0) * (j + 1) / 8.0 for j in range(8)]
+    yout = _gpu_outputs(w, rec, tau)
     lam_out = np.random.default_rng(12).normal(size=(w.N, len(tau), w.d))
     gy, gt = _gpu_grad(w, rec, tau, lam_out, None)
     tot = int(rec.info().total_steps)
@@ -229,6 +230,10 @@ def test_full_size_outputs_gradient_sampled(orc):
         Ts[r_, :S[r_]] = T[off[k]:off[k + 1]].cpu().numpy()
         Hs[r_, :S[r_]] = H[off[k]:off[k + 1]].cpu().numpy()
     sub = W.subset(w, idx)
+    ro = orc.replay_outputs(sub.field, sub.method, sub.theta, sub.y0, Ts, Hs, S, w.t1,
+                            np.array(tau), nthreads=8)
+    err = U.rel_rows(yout[idx].reshape(len(idx), -1), ro.reshape(len(idx), -1), w.atol)
+    assert err.max() <= 1e-9, err.max()
     ry, rt = orc.replay_outputs_grad(sub.field, sub.method, sub.theta, sub.y0, Ts, Hs, S, w.t1,
                                      np.array(tau), lam_out[idx], nthreads=8)
     assert U.rel_rows(gy[idx], ry, 1e-300).max() <= 1e-8
