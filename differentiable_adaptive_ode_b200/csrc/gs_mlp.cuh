@@ -23,6 +23,7 @@
 namespace gs {
 
 constexpr int MLP_H = 32, MLP_D = 4, MLP_M = 1348;
+static_assert(MLP_D == 4, "warp_sum4 reduces the four outputs of the field");
 constexpr int MLP_OW1 = 0, MLP_OB1 = 128, MLP_OW2 = 160, MLP_OB2 = 1184, MLP_OW3 = 1216,
               MLP_OB3 = 1344;
 
@@ -57,23 +58,59 @@ struct MlpLane {
   }
 };
 
-// Butterfly sum; addition being commutative, every lane ends with the same bits, and the value is
-// broadcast from lane 0 as well so that the replicated state can never drift between lanes.
-template <class R> __device__ __forceinline__ R warp_sum(R v) {
+// The four sums over the warp of four per-lane values, every lane receiving all four.  A
+// reduce-scatter butterfly: over the first two exchanges (lane distance 16, then 8) the lanes
+// split the four sums between them, each lane keeping one and passing the others on; the last
+// three exchanges (4, 2, 1) finish the sum each lane kept; then each sum is broadcast from a lane
+// that holds it (lanes 0, 8, 16, 24 hold sums 0, 1, 2, 3).  10 shuffles, where four separate
+// butterflies with broadcasts take 24.  Addition being commutative, every lane that finishes a
+// sum holds the same bits, and the broadcast gives every lane the same value, so the state that
+// the lanes replicate cannot drift between them.
+template <class R>
+__device__ __forceinline__ void warp_sum4(const R (&v)[4], R (&sum)[4]) {
+  const int lane = threadIdx.x & 31;
+  const bool up16 = lane & 16, up8 = lane & 8;
+  // distance 16: the lower half keeps sums 0 and 1, the upper half sums 2 and 3
+  R a0 = up16 ? v[2] : v[0], a1 = up16 ? v[3] : v[1];
+  const R s0 = up16 ? v[0] : v[2], s1 = up16 ? v[1] : v[3];
+  a0 += __shfl_xor_sync(FULL, s0, 16);
+  a1 += __shfl_xor_sync(FULL, s1, 16);
+  // distance 8: of its two, a lane keeps the first if bit 3 of its index is clear
+  R k = up8 ? a1 : a0;
+  k += __shfl_xor_sync(FULL, up8 ? a0 : a1, 8);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-  return __shfl_sync(FULL, v, 0);
+  for (int o = 4; o > 0; o >>= 1) k += __shfl_xor_sync(FULL, k, o);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) sum[c] = __shfl_sync(FULL, k, 8 * c);
 }
 
-// Broadcast the 32 lane values v through shared memory; out[j] = v of lane j.
+// Broadcast the 32 lane values v through shared memory; out[j] = v of lane j.  The slot is
+// 16-byte aligned and read back as 16-byte vectors (every lane reads the same words: a broadcast).
 template <class R>
 __device__ __forceinline__ void warp_gather(R* slot, R v, R (&out)[MLP_H]) {
   const int i = threadIdx.x & 31;
   __syncwarp();
   slot[i] = v;
   __syncwarp();
+  if constexpr (sizeof(R) == 4) {
+    const float4* s4 = reinterpret_cast<const float4*>(slot);
 #pragma unroll
-  for (int j = 0; j < MLP_H; ++j) out[j] = slot[j];
+    for (int q = 0; q < MLP_H / 4; ++q) {
+      const float4 t = s4[q];
+      out[4 * q] = t.x;
+      out[4 * q + 1] = t.y;
+      out[4 * q + 2] = t.z;
+      out[4 * q + 3] = t.w;
+    }
+  } else {
+    const double2* s2 = reinterpret_cast<const double2*>(slot);
+#pragma unroll
+    for (int q = 0; q < MLP_H / 2; ++q) {
+      const double2 t = s2[q];
+      out[2 * q] = t.x;
+      out[2 * q + 1] = t.y;
+    }
+  }
 }
 
 template <class R> __device__ __forceinline__ R tanh_r(R x);
@@ -95,8 +132,12 @@ __device__ __forceinline__ void mlp_f(const MlpLane<R>& W, const R (&y)[MLP_D], 
 #pragma unroll
   for (int j = 0; j < MLP_H; ++j) z2 += W.w2r[j] * hv[j];
   h2 = tanh_r<R>(z2);
+  R part[MLP_D], sum[MLP_D];
 #pragma unroll
-  for (int o = 0; o < MLP_D; ++o) dy[o] = W.b3[o] + warp_sum<R>(W.w3c[o] * h2);
+  for (int o = 0; o < MLP_D; ++o) part[o] = W.w3c[o] * h2;
+  warp_sum4<R>(part, sum);
+#pragma unroll
+  for (int o = 0; o < MLP_D; ++o) dy[o] = W.b3[o] + sum[o];
 }
 
 // Field adaptor so that the generic Tsit5 trial step can drive the warp-cooperative f.
@@ -219,11 +260,13 @@ __device__ __forceinline__ void mlp_adjoint_step(const MlpLane<R>& W, const R (&
     for (int j = 0; j < MLP_H; ++j) h1b += W.w2c[j] * zv[j];
     const R z1b = h1b * (R(1) - H1[i] * H1[i]);
     tb_.b1 += z1b;
+    R part[D];
 #pragma unroll
     for (int c = 0; c < D; ++c) {
       tb_.w1[c] += z1b * Y[i][c];
-      Yb[i][c] = warp_sum<R>(W.w1[c] * z1b);
+      part[c] = W.w1[c] * z1b;
     }
+    warp_sum4<R>(part, Yb[i]);
 #pragma unroll
     for (int c = 0; c < D; ++c) lnew[c] += Yb[i][c];
   }
@@ -246,7 +289,7 @@ template <class R, bool REC>
 __global__ void __launch_bounds__(128) k_solve_mlp(SolveParams<R> p) {
   using L = MlpLayout<R>;
   constexpr int D = MLP_D;
-  __shared__ R slots[4][32];
+  __shared__ __align__(16) R slots[4][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   MlpLane<R> W;
   W.load(p.theta, slots[warp]);
@@ -406,7 +449,7 @@ template <class R>
 __global__ void __launch_bounds__(128) k_replay_forward_mlp(ReplayParams<R> p) {
   using L = MlpLayout<R>;
   constexpr int D = MLP_D;
-  __shared__ R slots[4][32];
+  __shared__ __align__(16) R slots[4][32];
   if (p.gate && *p.gate == 0) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   MlpLane<R> W;
@@ -466,7 +509,7 @@ template <class R>
 __global__ void __launch_bounds__(128) k_adjoint_mlp(MlpAdjParams<R> p) {
   using L = MlpLayout<R>;
   constexpr int D = MLP_D;
-  __shared__ R slots[4][32];
+  __shared__ __align__(16) R slots[4][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gw = blockIdx.x * 4 + warp;
   const int nwarps = gridDim.x * 4;
@@ -506,7 +549,7 @@ __global__ void __launch_bounds__(128) k_adjoint_mlp(MlpAdjParams<R> p) {
 template <class R>
 __global__ void __launch_bounds__(128) k_replay_outputs_mlp(OutParams<R> q) {
   constexpr int D = MLP_D;
-  __shared__ R slots[4][32];
+  __shared__ __align__(16) R slots[4][32];
   const ReplayParams<R>& p = q.rp;
   const int warp = threadIdx.x >> 5;
   const int J = q.ot.J, jS = q.jS;
@@ -559,7 +602,7 @@ struct MlpOutAdjParams {
 template <class R>
 __global__ void __launch_bounds__(128) k_output_pullbacks_mlp(MlpOutAdjParams<R> q) {
   constexpr int D = MLP_D;
-  __shared__ R slots[4][32];
+  __shared__ __align__(16) R slots[4][32];
   const MlpAdjParams<R>& p = q.ap;
   const int warp = threadIdx.x >> 5;
   const int gw = blockIdx.x * 4 + warp;
@@ -597,7 +640,7 @@ __global__ void __launch_bounds__(128) k_output_pullbacks_mlp(MlpOutAdjParams<R>
 template <class R>
 __global__ void __launch_bounds__(128) k_adjoint_outputs_mlp(MlpOutAdjParams<R> q) {
   constexpr int D = MLP_D;
-  __shared__ R slots[4][32];
+  __shared__ __align__(16) R slots[4][32];
   const MlpAdjParams<R>& p = q.ap;
   const int warp = threadIdx.x >> 5;
   const int gw = blockIdx.x * 4 + warp;
