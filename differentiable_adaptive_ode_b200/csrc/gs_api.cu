@@ -278,8 +278,6 @@ struct gs_record {
   size_t red_bytes = 0, part_bytes = 0;
   void* y1_scratch = nullptr;    // y_S of gs_replay_forward when the caller passes no y1
   size_t y1_bytes = 0;
-  void* out_scratch = nullptr;   // output cotangents pulled back to their steps [N][J][d]
-  size_t out_bytes = 0;
   // the theta the stored states y_n were computed at ([N][m], or [m] when shared); counters[8]
   // is the flag the device comparison with a caller's theta raises
   void* theta_kept = nullptr;
@@ -1362,27 +1360,18 @@ void fill_replay_params(gs::ReplayParams<R>& p, const gs_record* rec, const void
   p.bounds = bounds_of(rec);
 }
 
-// Gradient of a loss on the outputs at requested times, MLP field: the output pullbacks, then the
-// walk that adds them, both one warp per trajectory on the same grid (warp gw carries its weight-
-// cotangent partial from the first pass into the second), then a fixed-order sum over warps.
+// Gradient of a loss on the outputs at requested times, MLP field: one warp per trajectory
+// (the extra pullbacks taken where the walk meets them), per-warp weight-cotangent partials, then a
+// fixed-order sum over warps.
 static gs_status replay_grad_outputs_mlp(const gs_record* rec, const void* theta, int32_t J,
                                          const double* tau, const void* dL_dyout,
                                          const void* dL_dy1, void* dL_dtheta, void* dL_dy0,
                                          cudaStream_t s) {
   gs_record* r = const_cast<gs_record*>(rec);
-  const int jS = outputs_before_t1(rec, J, tau);
-  const size_t need_g = (size_t)rec->N * jS * rec->sys.d * rec->rsz;
-  if (r->out_bytes < need_g) {
-    free_ptr(r->out_scratch, s);
-    r->out_scratch = nullptr;
-    r->out_bytes = 0;
-    GS_CUDA(dalloc(&r->out_scratch, need_g, s));
-    r->out_bytes = need_g;
-  }
   auto run = [&](auto zero) -> gs_status {
     using R = decltype(zero);
-    auto walk = gs::k_adjoint_outputs_mlp<R>;
-    const int grid = persistent_grid(walk, 0, rec->N * 32);
+    auto kern = gs::k_adjoint_outputs_mlp<R>;
+    const int grid = persistent_grid(kern, 0, rec->N * 32);
     const int nwarps = grid * (BLOCK / 32);
     R* partials = nullptr;
     if (dL_dtheta) {
@@ -1411,10 +1400,8 @@ static gs_status replay_grad_outputs_mlp(const gs_record* rec, const void* theta
     p.bounds = bounds_of(rec);
     q.dL_dyout = static_cast<const R*>(dL_dyout);
     fill_times<R>(q.ot, rec, J, tau);
-    q.jS = jS;
-    q.G = static_cast<R*>(r->out_scratch);
-    if (jS > 0) gs::k_output_pullbacks_mlp<R><<<grid, BLOCK, 0, s>>>(q);
-    walk<<<grid, BLOCK, 0, s>>>(q);
+    q.jS = outputs_before_t1(rec, J, tau);
+    kern<<<grid, BLOCK, 0, s>>>(q);
     if (partials)
       gs::k_reduce_partials<R><<<(gs::MLP_M + 255) / 256, 256, 0, s>>>(partials, nwarps, gs::MLP_M,
                                                                     static_cast<R*>(dL_dtheta));
@@ -1503,14 +1490,6 @@ gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_
     }
   }
   const int jS = outputs_before_t1(rec, J, tau);
-  const size_t need_g = (size_t)N * jS * rec->sys.d * rec->rsz;
-  if (r->out_bytes < need_g) {
-    free_ptr(r->out_scratch, s);
-    r->out_scratch = nullptr;
-    r->out_bytes = 0;
-    GS_CUDA(dalloc(&r->out_scratch, need_g, s));
-    r->out_bytes = need_g;
-  }
   int* queue = nullptr;
   GS_CUDA(take_counter(s, &queue));
   return dispatch(rec->sys, [&]<class F, class R, int METHOD>() {
@@ -1535,14 +1514,8 @@ gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_
       q.dL_dyout = static_cast<const R*>(dL_dyout);
       fill_times<R>(q.ot, rec, J, tau);
       q.jS = jS;
-      q.G = static_cast<R*>(r->out_scratch);
-      const size_t smem = adjoint_smem<F, R, METHOD>();
-      if (jS > 0) {  // the output pullbacks, then the walk that adds them
-        auto first = gs::k_output_pullbacks<F, R, METHOD>;
-        if (smem > 48 * 1024)
-          GS_CUDA(cudaFuncSetAttribute(first, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-        first<<<(unsigned)((N + BLOCK - 1) / BLOCK), BLOCK, smem, s>>>(q);
-      }
+      // the stage tape, then each lane's cotangent slot for the passes that take an output
+      const size_t smem = adjoint_smem<F, R, METHOD>() + (size_t)F::D * BLOCK * sizeof(R);
       auto kern = gs::k_adjoint_outputs<F, R, METHOD>;
       if (smem > 48 * 1024)
         GS_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
@@ -1714,7 +1687,6 @@ void gs_record_destroy(gs_record* r) {
   free_ptr(r->nsteps, s); free_ptr(r->status, s); free_ptr(r->offsets, s); free_ptr(r->choff, s);
   free_ptr(r->tiles, s); free_ptr(r->counters, s);
   free_ptr(r->red_scratch, s); free_ptr(r->red_partials, s); free_ptr(r->y1_scratch, s);
-  free_ptr(r->out_scratch, s);
   free_ptr(r->theta_kept, s);
   free_ptr(r->perm, s); free_ptr(r->bins, s); free_ptr(r->binoff, s); free_ptr(r->btiles, s);
   free_ptr(r->park_list, s); free_ptr(r->park_r, s);

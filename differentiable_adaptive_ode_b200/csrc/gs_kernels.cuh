@@ -1007,62 +1007,24 @@ struct AdjOutParams {
   const R* dL_dyout;    // [N][J][D]
   OutTimes<R> ot;
   int jS;               // outputs 0 .. jS - 1 are before t1 (the rest are the final state)
-  R* G;                 // [N][jS][D]: the output cotangents pulled back to their window states
 };
 
-// Replay adjoint with outputs at requested times, first pass.  Output j < jS of trajectory k is
-// the state reached by one extra step from the recorded state y_n of the last step with
-// t_n <= tau_j (step 0 if there is none), of size tau_j - t_n.  Its cotangent mu_j therefore
-// reaches y_n as g_j, the pullback of mu_j through that extra step, and reaches theta as that
-// pullback's theta-bar term.  Neither depends on the cotangent of the steps after n, so all of
-// them are taken here, before the walk over the record: every lane takes the same jS pullbacks
-// (the times are shared by all trajectories), so a warp takes them in lockstep, where taking them
-// inside the walk would stall the whole warp on nearly every step for the one lane that meets an
-// output.  g_j goes to G; the theta-bar terms, summed, to dL_dtheta[k], where the walk starts.
-template <class F, class R, int METHOD>
-__global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_blocks)
-    k_output_pullbacks(AdjOutParams<R> q) {
-  using L = RecLayout<F, R>;
-  constexpr int D = F::D, M = F::M;
-  extern __shared__ __align__(16) unsigned char adj_smem[];
-  R* tape = reinterpret_cast<R*>(adj_smem) + threadIdx.x;
-  const AdjointParams<R>& p = q.ap;
-  const int k = blockIdx.x * blockDim.x + threadIdx.x;
-  if (k >= p.N) return;
-  const int S = p.nsteps[k];
-  R thb[M];
-#pragma unroll
-  for (int i = 0; i < M; ++i) thb[i] = R(0);
-  if (S > 0) {
-    typename F::template Theta<R> th;
-    F::load(th, p.theta + (size_t)p.theta_stride * k);
-    const long long cbase = p.choff[k];
-    const R* lo = q.dL_dyout + (size_t)k * q.ot.J * D;
-    int n = 0;
-    for (int j = 0; j < q.jS; ++j) {
-      const R tau = q.ot.tau[j];
-      n = output_step<F, R>(p, cbase, n, S, tau);
-      R t, h, y[D], mu[D];
-      load_entry<R, L::E>(rec_entry<F, R>(p, cbase, n), t, h, y);
-#pragma unroll
-      for (int c = 0; c < D; ++c) mu[c] = lo[(size_t)j * D + c];
-      adjoint_step<F, R, METHOD>(y, tau - t, th, mu, thb, tape);
-#pragma unroll
-      for (int c = 0; c < D; ++c) q.G[((size_t)k * q.jS + j) * D + c] = mu[c];
-    }
-  }
-  if (p.dL_dtheta)
-#pragma unroll
-    for (int i = 0; i < M; ++i) p.dL_dtheta[(size_t)k * M + i] = thb[i];
-}
-
-// Replay adjoint with outputs at requested times, second pass: the walk of k_adjoint (one
-// recorded step per active lane per pass of the loop, a lane refilled with the next trajectory,
-// longest records first, as soon as its own is done), started from dL/dy1 plus the cotangents of
-// the outputs at or after t1 and from the first pass's theta-bar, with the first pass's g_j added
-// to the cotangent of y_n at each output's step n.  The window test is the first pass's: going
-// down from step S - 1, output j belongs to the first step with t_n <= tau_j, and to step 0 if
-// none.
+// Replay adjoint with outputs at requested times ("gradsolve: fast exact gradients for ODE
+// ensembles on GPUs" §3.4).  Output j < jS of trajectory k is one extra step, of size tau_j - t_n,
+// from the recorded state y_n of the first step n (going down the record) with t_n <= tau_j, and
+// of step 0 if there is none; the outputs at or after t1 are the final state.  So the cotangent of
+// y_n is the pullback of the later steps' cotangent through step n, plus, for each output of that
+// step, the pullback of the output's cotangent through its extra step.
+//
+// The walk of k_adjoint (one pullback per active lane per pass of the loop, a lane refilled with
+// the next trajectory, longest records first, as soon as its own is done), in which a lane's pass
+// pulls back either its next recorded step or, after a step that holds outputs, one of those
+// outputs' extra steps.  Both are the same adjoint step of the same y_n with another step size and
+// cotangent, so the warp takes them together in one call: a lane that meets an output costs the
+// others nothing, where an extra call for it would stall the warp on nearly every pass (with 8
+// outputs over about 130 steps, some lane of a 32-lane warp meets one on most passes).  During an
+// output's pass the lane's cotangent waits in its shared-memory slot and the output's cotangent
+// takes its place in the call; the result is added to it afterwards.
 template <class F, class R, int METHOD>
 __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_blocks)
     k_adjoint_outputs(AdjOutParams<R> q) {
@@ -1070,12 +1032,18 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
   constexpr int D = F::D, M = F::M;
   extern __shared__ __align__(16) unsigned char adj_smem[];
   R* tape = reinterpret_cast<R*>(adj_smem) + threadIdx.x;
+  // after the stage tape of the Tsit5 and Verner 7 sweeps (TAPE reals per stage and lane), this
+  // lane's cotangent slot: D reals at stride blockDim.x
+  constexpr int TAPE_REALS = (METHOD == M_VERN7 ? 9 : (METHOD == M_TSIT5 ? 6 : 0)) * TapeOf<F>::value;
+  R* stash = reinterpret_cast<R*>(adj_smem) + TAPE_REALS * blockDim.x + threadIdx.x;
   const AdjointParams<R>& p = q.ap;
   const int J = q.ot.J, jS = q.jS;
-  const bool thb_from_first = jS > 0 && p.dL_dtheta;
-  int k = -1, n = -1, first_n = -1, jcur = 0, cur_ch = 0, next_ch = -1;
+  // per lane: trajectory k, step n; the outputs jcur .. J - 1 are taken; after the pullback of a
+  // step that holds outputs jlo .. jcur - 1, r counts them down (r >= jlo: output r is next)
+  int k = -1, n = -1, first_n = -1, jcur = 0, jlo = 0, r = -1, cur_ch = 0, next_ch = -1;
   bool alive = true, pf_pending = false;
   long long cbase = 0;
+  const R* lo = nullptr;
   R lam[D], thb[M];
   typename F::template Theta<R> th;
 #pragma unroll
@@ -1090,11 +1058,11 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
         if (id < p.N) {
           k = p.perm ? p.perm[id] : id;
           F::load(th, p.theta + (size_t)p.theta_stride * k);
-          const R* lo = q.dL_dyout + (size_t)k * J * D;
+          lo = q.dL_dyout + (size_t)k * J * D;
 #pragma unroll
           for (int c = 0; c < D; ++c) lam[c] = p.dL_dy1 ? p.dL_dy1[(size_t)k * D + c] : R(0);
 #pragma unroll
-          for (int i = 0; i < M; ++i) thb[i] = thb_from_first ? p.dL_dtheta[(size_t)k * M + i] : R(0);
+          for (int i = 0; i < M; ++i) thb[i] = R(0);
           const int S = p.nsteps[k];
           jcur = S == 0 ? 0 : jS;
           for (int jj = jcur; jj < J; ++jj)
@@ -1102,6 +1070,7 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
             for (int c = 0; c < D; ++c) lam[c] += lo[(size_t)jj * D + c];
           n = S - 1;
           first_n = n;
+          r = -1;
           cbase = p.choff[k];
         } else {
           alive = false;
@@ -1111,38 +1080,50 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
     if (!__any_sync(FULL, k >= 0 || alive)) break;
     if (k >= 0) {
       if (n >= 0) {
-        // chunk of step n, and the next chunk's lines prefetched one step after entering one
-        if (n == first_n || n % L::C == L::C - 1) {
-          cur_ch = chunk_at(p.chunk_table, cbase + n / L::C, p.bounds);
-          next_ch = (n / L::C >= 1) ? chunk_at(p.chunk_table, cbase + n / L::C - 1, p.bounds) : -1;
+        const bool out = r >= 0;  // this pass: output r's extra step from y_n
+        if (!out) {
+          // chunk of step n, and the next chunk's lines prefetched one step after entering one
+          if (n == first_n || n % L::C == L::C - 1) {
+            cur_ch = chunk_at(p.chunk_table, cbase + n / L::C, p.bounds);
+            next_ch = (n / L::C >= 1) ? chunk_at(p.chunk_table, cbase + n / L::C - 1, p.bounds) : -1;
 #ifdef GS_CHECKED
-          if (next_ch >= p.bounds.pool_chunks) next_ch = -1;
+            if (next_ch >= p.bounds.pool_chunks) next_ch = -1;
 #endif
-          pf_pending = next_ch >= 0;
-        } else if (pf_pending) {
-          const R* pq = p.pool + (size_t)next_ch * L::C * L::E;
+            pf_pending = next_ch >= 0;
+          } else if (pf_pending) {
+            const R* pq = p.pool + (size_t)next_ch * L::C * L::E;
 #pragma unroll
-          for (int b = 0; b < L::C * L::E * (int)sizeof(R); b += 128)
-            asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const char*>(pq) + b));
-          pf_pending = false;
+            for (int b = 0; b < L::C * L::E * (int)sizeof(R); b += 128)
+              asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const char*>(pq) + b));
+            pf_pending = false;
+          }
         }
         const R* e = chunk_entry<L>(p.pool, cur_ch, n, p.bounds);
         R t, h, y[D];
         load_entry<R, L::E>(e, t, h, y);
-        int jlo = jcur;
-        while (jlo > 0 && (n == 0 || q.ot.tau[jlo - 1] >= t)) --jlo;
-        // the stored pullbacks of this step's outputs, fetched while the step is pulled back
-        for (int r = jlo; r < jcur; ++r) {
-          const char* g = reinterpret_cast<const char*>(q.G + ((size_t)k * jS + r) * D);
-          asm volatile("prefetch.global.L1 [%0];" ::"l"(g));
-          asm volatile("prefetch.global.L1 [%0];" ::"l"(g + D * sizeof(R) - 1));
+        if (out) {
+#pragma unroll
+          for (int c = 0; c < D; ++c) {
+            stash[c * blockDim.x] = lam[c];
+            lam[c] = lo[(size_t)r * D + c];
+          }
+          h = q.ot.tau[r] - t;
         }
         adjoint_step<F, R, METHOD>(y, h, th, lam, thb, tape);
-        for (int r = jlo; r < jcur; ++r)
+        if (out) {
 #pragma unroll
-          for (int c = 0; c < D; ++c) lam[c] += q.G[((size_t)k * jS + r) * D + c];
-        jcur = jlo;
-        --n;
+          for (int c = 0; c < D; ++c) lam[c] += stash[c * blockDim.x];
+          if (--r < jlo) {  // the step's outputs are taken: on to step n - 1
+            jcur = jlo;
+            r = -1;
+            --n;
+          }
+        } else {
+          jlo = jcur;
+          while (jlo > 0 && (n == 0 || q.ot.tau[jlo - 1] >= t)) --jlo;
+          if (jlo < jcur) r = jcur - 1;
+          else --n;
+        }
       }
       if (n < 0) {
         if (p.dL_dy0)

@@ -167,21 +167,6 @@ struct MlpBar {
     b1 = R(0);
     b2 = R(0);
   }
-  // read back a partial that store wrote (b3b into every lane, as it accumulates there)
-  __device__ void load(const R* in) {
-    const int i = threadIdx.x & 31;
-#pragma unroll
-    for (int c = 0; c < MLP_D; ++c) w1[c] = in[MLP_OW1 + i * MLP_D + c];
-    b1 = in[MLP_OB1 + i];
-#pragma unroll
-    for (int j = 0; j < MLP_H; ++j) w2[j] = in[MLP_OW2 + i * MLP_H + j];
-    b2 = in[MLP_OB2 + i];
-#pragma unroll
-    for (int o = 0; o < MLP_D; ++o) {
-      w3[o] = in[MLP_OW3 + o * MLP_H + i];
-      b3[o] = in[MLP_OB3 + o];
-    }
-  }
   // write this warp's partial (M values) to out
   __device__ void store(R* out) const {
     const int i = threadIdx.x & 31;
@@ -541,10 +526,10 @@ __global__ void __launch_bounds__(128) k_adjoint_mlp(MlpAdjParams<R> p) {
 // Outputs at requested times and their gradient ("gradsolve: fast exact gradients for ODE
 // ensembles on GPUs" §3.4: one extra solver step from the preceding mesh point exactly to each
 // requested time), one warp per trajectory.  The rule is the other fields' (k_replay_outputs,
-// k_output_pullbacks, k_adjoint_outputs): output j < jS is one step of size tau_j - t_n from the
-// recorded y_n of its step n (output_step), the rest are the final state, and y0 when nothing is
-// recorded.  Warp w takes trajectories w, w + nwarps, ...; every lane takes the same search and
-// steps, so the warp stays converged for the field's shuffles.
+// k_adjoint_outputs): output j < jS is one step of size tau_j - t_n from the recorded y_n of its
+// step n (output_step), the rest are the final state, and y0 when nothing is recorded.  Warp w
+// takes trajectories w, w + nwarps, ...; every lane takes the same search and steps, so the warp
+// stays converged for the field's shuffles.
 // ------------------------------------------------------------------------------------------------
 template <class R>
 __global__ void __launch_bounds__(128) k_replay_outputs_mlp(OutParams<R> q) {
@@ -594,49 +579,12 @@ struct MlpOutAdjParams {
   const R* dL_dyout;    // [N][J][D]
   OutTimes<R> ot;
   int jS;               // outputs 0 .. jS - 1 are before t1
-  R* G;                 // [N][jS][D]: the output cotangents pulled back to their window states
 };
 
-// First pass: each output's cotangent pulled back through its extra step (to G) and that
-// pullback's weight cotangent (into the warp's partial, which the second pass continues).
-template <class R>
-__global__ void __launch_bounds__(128) k_output_pullbacks_mlp(MlpOutAdjParams<R> q) {
-  constexpr int D = MLP_D;
-  __shared__ __align__(16) R slots[4][32];
-  const MlpAdjParams<R>& p = q.ap;
-  const int warp = threadIdx.x >> 5;
-  const int gw = blockIdx.x * 4 + warp;
-  const int nwarps = gridDim.x * 4;
-  MlpLane<R> W;
-  W.load(p.theta, slots[warp]);
-  MlpBar<R> bar;
-  bar.zero();
-  for (int k = gw; k < p.N; k += nwarps) {
-    const int S = p.nsteps[k];
-    if (S == 0) continue;
-    const long long cbase = p.choff[k];
-    const R* lo = q.dL_dyout + (size_t)k * q.ot.J * D;
-    int n = 0;
-    for (int j = 0; j < q.jS; ++j) {
-      const R tau = q.ot.tau[j];
-      n = output_step<FMlpWarp, R>(p, cbase, n, S, tau);
-      const R* e = rec_entry<FMlpWarp, R>(p, cbase, n);
-      R y[D], mu[D];
-#pragma unroll
-      for (int c = 0; c < D; ++c) {
-        y[c] = e[2 + c];
-        mu[c] = lo[(size_t)j * D + c];
-      }
-      mlp_adjoint_step<R>(W, y, tau - e[0], mu, bar);
-      mlp_lane_store<R>(q.G + ((size_t)k * q.jS + j) * D, mu);
-    }
-  }
-  if (p.partials) bar.store(p.partials + (size_t)gw * MLP_M);
-}
-
-// Second pass: k_adjoint_mlp's walk from dL/dy1 plus the cotangents of the outputs at or after t1,
-// adding at each output's step its pulled-back cotangent from the first pass (same grid, so warp
-// gw continues its own partial).
+// Gradient: k_adjoint_mlp's walk from dL/dy1 plus the cotangents of the outputs at or after t1;
+// after the pullback of a step that holds outputs, each of them is pulled back through its extra
+// step from the same y_n and added.  A warp works on one trajectory, so the extra pullbacks leave
+// no lane idle.
 template <class R>
 __global__ void __launch_bounds__(128) k_adjoint_outputs_mlp(MlpOutAdjParams<R> q) {
   constexpr int D = MLP_D;
@@ -649,8 +597,7 @@ __global__ void __launch_bounds__(128) k_adjoint_outputs_mlp(MlpOutAdjParams<R> 
   MlpLane<R> W;
   W.load(p.theta, slots[warp]);
   MlpBar<R> bar;
-  if (jS > 0 && p.partials) bar.load(p.partials + (size_t)gw * MLP_M);
-  else bar.zero();
+  bar.zero();
   for (int id = gw; id < p.N; id += nwarps) {
     const int k = p.perm ? p.perm[id] : id;
     const int S = p.nsteps[k];
@@ -663,19 +610,36 @@ __global__ void __launch_bounds__(128) k_adjoint_outputs_mlp(MlpOutAdjParams<R> 
 #pragma unroll
       for (int c = 0; c < D; ++c) lam[c] += lo[(size_t)jj * D + c];
     const long long cbase = p.choff[k];
-    for (int n = S - 1; n >= 0; --n) {
+    // one adjoint step per pass: step n itself, or (r >= jlo) the extra step of output r from the
+    // same y_n; one call site keeps one copy of the step in the kernel
+    int n = S - 1, r = -1, jlo = jcur;
+    while (n >= 0) {
       const R* e = rec_entry<FMlpWarp, R>(p, cbase, n);
-      const R t = e[0], h = e[1];
-      R y[D];
+      const R t = e[0];
+      const bool out = r >= 0;
+      R y[D], v[D];
 #pragma unroll
-      for (int c = 0; c < D; ++c) y[c] = e[2 + c];
-      mlp_adjoint_step<R>(W, y, h, lam, bar);
-      int jlo = jcur;
-      while (jlo > 0 && (n == 0 || q.ot.tau[jlo - 1] >= t)) --jlo;
-      for (int r = jlo; r < jcur; ++r)
+      for (int c = 0; c < D; ++c) {
+        y[c] = e[2 + c];
+        v[c] = out ? lo[(size_t)r * D + c] : lam[c];
+      }
+      mlp_adjoint_step<R>(W, y, out ? q.ot.tau[r] - t : e[1], v, bar);
+      if (out) {
 #pragma unroll
-        for (int c = 0; c < D; ++c) lam[c] += q.G[((size_t)k * jS + r) * D + c];
-      jcur = jlo;
+        for (int c = 0; c < D; ++c) lam[c] += v[c];
+        if (--r < jlo) {  // the step's outputs are taken: on to step n - 1
+          jcur = jlo;
+          r = -1;
+          --n;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < D; ++c) lam[c] = v[c];
+        jlo = jcur;
+        while (jlo > 0 && (n == 0 || q.ot.tau[jlo - 1] >= t)) --jlo;
+        if (jlo < jcur) r = jcur - 1;
+        else --n;
+      }
     }
     if (p.dL_dy0) mlp_lane_store<R>(p.dL_dy0 + (size_t)k * D, lam);
   }

@@ -218,9 +218,7 @@ gs_status gs_replay_outputs(const gs_record* rec, const void* theta, const void*
 /* Gradient of a loss on the outputs at requested times (and optionally on the final state):
  * dL_dyout [N][J][d] (device), dL_dy1 [N][d] (device, nullable); outputs as gs_replay_grad.
  * Each output's cotangent is pulled back through its extra step from y_n and added to the
- * cotangent of y_n.  The stored states follow `theta` as in gs_replay_grad.  Those pullbacks go to
- * a scratch of N * (outputs before t1) * d values that the record allocates on first need and
- * keeps until it is destroyed (besides gs_replay_grad's scratch).  Asynchronous. */
+ * cotangent of y_n.  The stored states follow `theta` as in gs_replay_grad.  Asynchronous. */
 gs_status gs_replay_grad_outputs(const gs_record* rec, const void* theta, int32_t J,
                                  const double* tau, const void* dL_dyout, const void* dL_dy1,
                                  void* dL_dtheta, void* dL_dy0, void* stream);
