@@ -187,6 +187,21 @@ def test_empty_and_single_and_zero_interval():
     lam = np.random.default_rng(0).normal(size=(5, 3))
     gy, gt = U.replay_grad(w0, rec0, lam)
     assert np.array_equal(gy, lam) and np.all(gt == 0)
+    # ... and with no recorded step every output is y0 and the outputs' cotangents reach y0
+    # unchanged (summed with dL/dy1), theta not at all
+    tau = [0.0, 0.5]
+    th, y0 = U.dev(w0.theta, torch.float64), U.dev(w0.y0, torch.float64)
+    yo = torch.empty((5, 2, 3), dtype=torch.float64, device="cuda")
+    G.gs_replay_outputs(rec0, th, y0, tau, yo)
+    lo = np.random.default_rng(1).normal(size=(5, 2, 3))
+    gy2 = torch.empty((5, 3), dtype=torch.float64, device="cuda")
+    gt2 = torch.empty((5, 3), dtype=torch.float64, device="cuda")
+    G.gs_replay_grad_outputs(rec0, th, tau, U.dev(lo, torch.float64), U.dev(lam, torch.float64),
+                             gt2, gy2)
+    torch.cuda.synchronize()
+    assert np.array_equal(yo.cpu().numpy(), np.repeat(w0.y0[:, None, :], 2, axis=1))
+    assert np.array_equal(gy2.cpu().numpy(), lam + lo[:, 0] + lo[:, 1])
+    assert np.all(gt2.cpu().numpy() == 0)
 
 
 def test_status_codes_and_failed_record():
