@@ -94,6 +94,27 @@ def test_outputs_shared_theta_and_fp32(orc):
                              ex32["S"], w32.t1, tau32, dtype=np.float32, nthreads=8)
     err = U.rel_rows(got.reshape(300, -1), ref.reshape(300, -1), w32.atol)
     assert np.quantile(err, 0.99) <= 1e-4 and err.max() <= 1e-3
+    # fp32 gradient of a loss on the outputs against the exact (fp64) derivative over the GPU's
+    # fp32 mesh.  Cotangents of random sign enter at nine times and partly cancel, so fp32
+    # rounding alone moves a few trajectories' dL/dtheta by more than 1e-3: the oracle's own fp32
+    # derivative on this mesh does (p99 1.2e-3).  Bars: the ensemble within 1e-3; 99 % of the
+    # trajectories within 1e-3 or twice the fp32 oracle's 99th percentile, whichever is larger;
+    # the worst within 1e-2.
+    lo32 = np.random.default_rng(9).normal(size=(300, len(tau32), w32.d))
+    gy, gt = _gpu_grad(w32, rec32, tau32, lo32, None)
+    T64, H64 = ex32["T"].astype(np.float64), ex32["H"].astype(np.float64)
+    ry, rt = orc.replay_outputs_grad(w32.field, w32.method, w32.theta, w32.y0, T64, H64,
+                                     ex32["S"], w32.t1, tau32, lo32, nthreads=8)
+    qy, qt = orc.replay_outputs_grad(w32.field, w32.method, w32.theta, w32.y0, ex32["T"],
+                                     ex32["H"], ex32["S"], w32.t1, tau32, lo32, dtype=np.float32,
+                                     nthreads=8)
+    for got_, want, own in ((gy, ry, qy), (gt, rt, qt)):
+        rel = U.rel_rows(got_, want, 1e-300)
+        spread = np.quantile(U.rel_rows(own, want, 1e-300), 0.99)
+        ens = np.linalg.norm(got_ - want) / np.linalg.norm(want)
+        assert ens <= 1e-3, ens
+        assert np.quantile(rel, 0.99) <= max(1e-3, 2 * spread), (np.quantile(rel, 0.99), spread)
+        assert rel.max() <= 1e-2, rel.max()
 
 
 def test_outputs_argument_checks():
