@@ -1044,6 +1044,7 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
   bool alive = true, pf_pending = false;
   long long cbase = 0;
   const R* lo = nullptr;
+  R tau_next = R(0);  // tau[jcur - 1]: the time of the next output going down (jcur > 0)
   R lam[D], thb[M];
   typename F::template Theta<R> th;
 #pragma unroll
@@ -1068,6 +1069,7 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
           for (int jj = jcur; jj < J; ++jj)
 #pragma unroll
             for (int c = 0; c < D; ++c) lam[c] += lo[(size_t)jj * D + c];
+          tau_next = jcur > 0 ? q.ot.tau[jcur - 1] : R(0);
           n = S - 1;
           first_n = n;
           r = -1;
@@ -1115,14 +1117,16 @@ __global__ void __launch_bounds__(128, METHOD == M_VERN7 ? 1 : Tune<F, R>::adj_b
           for (int c = 0; c < D; ++c) lam[c] += stash[c * blockDim.x];
           if (--r < jlo) {  // the step's outputs are taken: on to step n - 1
             jcur = jlo;
+            tau_next = jcur > 0 ? q.ot.tau[jcur - 1] : R(0);
             r = -1;
             --n;
           }
-        } else {
-          jlo = jcur;
+        } else if (jcur > 0 && (n == 0 || tau_next >= t)) {  // the step holds outputs
+          jlo = jcur - 1;
           while (jlo > 0 && (n == 0 || q.ot.tau[jlo - 1] >= t)) --jlo;
-          if (jlo < jcur) r = jcur - 1;
-          else --n;
+          r = jcur - 1;
+        } else {
+          --n;
         }
       }
       if (n < 0) {
