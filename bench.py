@@ -145,11 +145,11 @@ PIPE_BUSY_NCU = {
 # forward sensitivities: DRAM bytes per trajectory (inputs and outputs; nothing per step), from
 # an ncu capture of the 2^18-orbit case
 TRAFFIC_SENS_PER_TRAJ = {"log_halo": 94.3}
-# library kernels per step: record = k_solve + 2 k_max_int + 3 prefix scans of 3 kernels each
-# (step offsets, chunk offsets, length bins) + k_chunk_table + k_bin_count + k_bin_scatter (15);
-# replay gradient = k_theta_check + k_replay_forward (exits at once: the theta is the recorded one)
-# + k_adjoint (3).
-LAUNCHES_PER_STEP = 18
+# library kernels per step: record = k_solve + the pass summary (3 kernels: step and chunk
+# offsets side by side, longest record, worst status) + k_chunk_table + the longest-first order
+# (k_bin_count, the one-block scan of the length bins, k_bin_scatter) (8); replay gradient =
+# k_theta_check + k_replay_forward (exits at once: the theta is the recorded one) + k_adjoint (3).
+LAUNCHES_PER_STEP = 11
 
 
 def fp64_peak_tflops(mhz):

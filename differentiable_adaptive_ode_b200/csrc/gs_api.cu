@@ -323,7 +323,7 @@ gs_status ensure_traj_arrays(gs_record* r, int64_t N, cudaStream_t s) {
   GS_CUDA(dalloc(&r->status, n * sizeof(int), s));
   GS_CUDA(dalloc(&r->offsets, (n + 1) * sizeof(long long), s));
   GS_CUDA(dalloc(&r->choff, (n + 1) * sizeof(long long), s));
-  GS_CUDA(dalloc(&r->tiles, (ntiles + 2) * sizeof(long long), s));
+  GS_CUDA(dalloc(&r->tiles, 2 * (ntiles + 2) * sizeof(long long), s));  // two scans side by side
   if (!r->counters) GS_CUDA(dalloc(&r->counters, 16 * sizeof(int), s));
   r->n_cap = n;
   return GS_OK;
@@ -414,6 +414,18 @@ gs::RecBounds bounds_of(const gs_record* r) {
   return gs::RecBounds{(long long)r->chunk_arrays_cap, (long long)r->pool_chunks};
 }
 
+// The summary of a record pass: step offsets, chunk offsets, the largest step count and status
+// (into counters[3] and counters[4], zeroed by the caller) in three kernels.
+gs_status summarise_pass(gs_record* r, const int* status, int N, int C, cudaStream_t st) {
+  const int ntiles = (N + gs::SCAN_BLOCK - 1) / gs::SCAN_BLOCK;
+  gs::k_summary_tiles<<<ntiles, gs::SCAN_BLOCK, 0, st>>>(r->nsteps, status, N, C, r->offsets,
+                                                         r->choff, r->tiles, r->counters + 3);
+  gs::k_summary_totals<<<1, gs::SCAN_BLOCK, 0, st>>>(r->tiles, ntiles);
+  gs::k_summary_add<<<(N + 255) / 256, 256, 0, st>>>(r->offsets, r->choff, N, r->tiles, ntiles);
+  GS_CUDA(cudaGetLastError());
+  return GS_OK;
+}
+
 template <int MODE>
 gs_status scan_counts(const int* S, int N, int C, long long* out, long long* tiles,
                       cudaStream_t st) {
@@ -449,8 +461,13 @@ gs_status counting_sort_desc(gs_record* r, const int* keys, int64_t n, int kmax,
     gs::k_bin_count_smem<<<grid, threads, nb * sizeof(int), s>>>(keys, (int)n, kmax, r->bins);
   else
     gs::k_bin_count<<<grid, threads, 0, s>>>(keys, (int)n, kmax, r->bins);
-  gs_status st = scan_counts<0>(r->bins, (int)nb, 1, r->binoff, r->btiles, s);
-  if (st != GS_OK) return st;
+  if (small) {
+    gs::k_scan_one_block<<<1, gs::SCAN_BLOCK, 0, s>>>(r->bins, (int)nb, r->binoff);
+    GS_CUDA(cudaGetLastError());
+  } else {
+    gs_status st = scan_counts<0>(r->bins, (int)nb, 1, r->binoff, r->btiles, s);
+    if (st != GS_OK) return st;
+  }
   if (small)
     gs::k_bin_scatter_smem<<<grid, threads, 2 * nb * sizeof(int), s>>>(keys, (int)n, kmax,
                                                                       r->binoff, r->bins + nb,
@@ -1053,7 +1070,6 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
   // (its contents kept) by the estimate of what they still need.
   int64_t nq = N;
   int64_t pass_start = 0;  // chunks handed out before this pass
-  const int nb = (int)((N + 255) / 256);
   constexpr int KMAX = 4096;  // remaining-step keys beyond this count as the longest
   for (int pass = 0;; ++pass) {
     const bool sliced = slice_mode && pass == 0;
@@ -1068,14 +1084,12 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
     if (st != GS_OK) return bail(st);
     cudaEventRecord(r->ev1, s);
     // summary over the ensemble (complete once no trajectory is parked): statuses, the longest
-    // record, the worst status, the step offsets
+    // record, the worst status, the step and chunk offsets
     if (status_out != r->status &&
         cudaMemcpyAsync(r->status, status_out, N * sizeof(int), cudaMemcpyDeviceToDevice, s) !=
             cudaSuccess)
       return bail(fail(GS_ERR_CUDA, "status copy failed"));
-    gs::k_max_int<<<nb, 256, 0, s>>>(r->nsteps, (int)N, r->counters + 3);
-    gs::k_max_int<<<nb, 256, 0, s>>>(r->status, (int)N, r->counters + 4);
-    if ((st = scan_counts<0>(r->nsteps, (int)N, C, r->offsets, r->tiles, s)) != GS_OK) return bail(st);
+    if ((st = summarise_pass(r, status_out, (int)N, C, s)) != GS_OK) return bail(st);
     // a slice parks (nearly) every trajectory: the estimate of what they still need is queued
     // right behind the pass, with the parked count read on the device, and comes back with the
     // summary in one synchronisation
@@ -1175,8 +1189,7 @@ gs_status gs_solve_record(const gs_system* sys, const gs_options* opt, int64_t N
     pass_start = used;
     nq = parked;
   }
-  // chunk offsets and table
-  if ((st = scan_counts<1>(r->nsteps, (int)N, C, r->choff, r->tiles, s)) != GS_OK) return bail(st);
+  // chunk table (the chunk offsets came with the last pass's summary)
   if (r->nchunks > 0)
     gs::k_chunk_table<<<(int)((r->nchunks + 255) / 256), 256, 0, s>>>(
         r->chunk_traj, r->chunk_seq, (int)r->nchunks, r->choff, r->chunk_table, bounds_of(r));

@@ -1208,11 +1208,92 @@ __global__ void __launch_bounds__(SCAN_BLOCK) k_scan_totals(long long* tile_tot,
   if (threadIdx.x == 0) *grand = carry;
 }
 
+// Exclusive scan of n counts by one block, tile after tile with a carry: out[0..n), out[n] = the
+// total.  For short arrays (the length bins of the longest-first order), one launch instead of
+// three.
+__global__ void __launch_bounds__(SCAN_BLOCK) k_scan_one_block(const int* in, int n,
+                                                               long long* out) {
+  long long carry = 0;
+  for (int b0 = 0; b0 < n; b0 += SCAN_BLOCK) {
+    const int i = b0 + threadIdx.x;
+    long long tot;
+    const long long ex = block_exclusive_scan(i < n ? (long long)in[i] : 0LL, &tot);
+    if (i < n) out[i] = carry + ex;
+    carry += tot;
+  }
+  if (threadIdx.x == 0) out[n] = carry;
+}
+
 __global__ void k_scan_add(long long* out, int N, const long long* tile_base,
                            const long long* grand) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < N) out[i] += tile_base[i / SCAN_BLOCK];
   if (i == 0) out[N] = *grand;
+}
+
+// The summary of a record pass in one three-kernel scan: the exclusive scans of the step counts
+// (step offsets) and of the chunk counts ceil(S / C) (chunk offsets) side by side, and the largest
+// step count and status (atomicMax into maxes[0] and maxes[1], which the caller zeroes).  The tile
+// scratch holds two halves of ntiles + 2: tile totals, then the grand total.
+__global__ void __launch_bounds__(SCAN_BLOCK) k_summary_tiles(const int* S, const int* status,
+                                                              int N, int C, long long* off,
+                                                              long long* choff, long long* tiles,
+                                                              int* maxes) {
+  const int i = blockIdx.x * SCAN_BLOCK + threadIdx.x;
+  const int ntiles = gridDim.x;
+  const int sv = i < N ? S[i] : 0;
+  long long tot_s, tot_c;
+  const long long ex_s = block_exclusive_scan((long long)sv, &tot_s);
+  const long long ex_c = block_exclusive_scan((long long)((sv + C - 1) / C), &tot_c);
+  if (i < N) {
+    off[i] = ex_s;
+    choff[i] = ex_c;
+  }
+  if (threadIdx.x == 0) {
+    tiles[blockIdx.x] = tot_s;
+    tiles[ntiles + 2 + blockIdx.x] = tot_c;
+  }
+  int ms = sv, mt = i < N ? status[i] : 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ms = max(ms, __shfl_xor_sync(FULL, ms, o));
+    mt = max(mt, __shfl_xor_sync(FULL, mt, o));
+  }
+  if ((threadIdx.x & 31) == 0) {
+    atomicMax(maxes, ms);
+    atomicMax(maxes + 1, mt);
+  }
+}
+
+__global__ void __launch_bounds__(SCAN_BLOCK) k_summary_totals(long long* tiles, int ntiles) {
+#pragma unroll 1
+  for (int h = 0; h < 2; ++h) {
+    long long* t = tiles + h * (ntiles + 2);
+    long long carry = 0;
+    for (int b0 = 0; b0 < ntiles; b0 += SCAN_BLOCK) {
+      const int i = b0 + threadIdx.x;
+      long long tot;
+      const long long v = i < ntiles ? t[i] : 0;
+      const long long ex = block_exclusive_scan(v, &tot);
+      if (i < ntiles) t[i] = carry + ex;
+      carry += tot;
+    }
+    if (threadIdx.x == 0) t[ntiles] = carry;
+  }
+}
+
+__global__ void k_summary_add(long long* off, long long* choff, int N, const long long* tiles,
+                              int ntiles) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const long long* tc = tiles + ntiles + 2;
+  if (i < N) {
+    off[i] += tiles[i / SCAN_BLOCK];
+    choff[i] += tc[i / SCAN_BLOCK];
+  }
+  if (i == 0) {
+    off[N] = tiles[ntiles];
+    choff[N] = tc[ntiles];
+  }
 }
 
 // chunk_table[choff[traj] + seq] = chunk (reserved-but-unused chunks carry traj = -1)
